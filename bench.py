@@ -1,0 +1,361 @@
+"""Benchmark of the gated local-global graph-attention forward on B200.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+                  [--workload arxiv] [--no-cpu-baseline]
+
+One step is one glga_forward (projection GEMM, global statistics, fused local branch +
+readout + gate) over the arxiv-shaped synthetic graph, with the graph already bound
+(glga_create, timed separately as create_ms) and inputs resident in HBM.  L2 is flushed
+(256 MiB write) between timed steps, outside the timed spans.  Metric: edge*heads/s =
+E * H / seconds per forward, E counting self-loops.
+
+Multi-GPU (torchrun, one rank per GPU): replicas only -- every rank runs the same forward
+on its own copy of the graph (weak scaling); value = sum of all ranks' edge*heads over
+the slowest rank's time.  `--impl reference` times the float64 CPU oracle on the host
+instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GLGA fwd edge·heads/s (1 B200, bf16 arxiv-shaped); local-branch HBM GB/s % of peak"
+UNIT = "edge*heads/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def local_bytes_model(N, E, D, H, r, s):
+    """Algorithmic bytes of the fused per-target kernel: CSR (row_ptr, col_idx), one k_j and
+    v_j row gather per edge, q_i and Y_i once per row, the gate logit, and S, z."""
+    return (4 * (N + 1) + 4 * E + 2 * D * s * E + D * s * N + D * s * N + 4 * N
+            + 4 * H * r * (r + 1))
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "sparse_graph_attention_tcgen05_b200", "csrc", "local.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """dram read+write bytes per launch of the local kernel from the committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"local_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None, None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("- ") and ":" in line:
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256_16") != kernel_source_hash():
+        return None, "stale"
+    try:
+        return float(vals["traffic_bytes_per_launch"]), vals.get("traffic_note")
+    except (KeyError, ValueError):
+        return None, None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1])); smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def cpu_baseline(w, csr, min_seconds=10.0, max_seconds=30.0):
+    import oracle
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
+                       csr[0], csr[1])
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el * (reps + 1) / reps > max_seconds:
+            break
+    return {"value": w.E * w.H * reps / el, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"the full {w.name} workload (N={w.N}, E={w.E}), {reps} float64 forward(s) "
+                      f"in {el:.1f} s on {oracle.num_threads()} OpenMP threads"}
+
+
+def run_reference(args, rank, world):
+    from sparse_graph_attention_tcgen05_b200.workloads import make_workload
+    import oracle
+    if rank != 0:
+        return
+    w = make_workload(args.workload)
+    csr = oracle.csr_from_coo(w.N, w.src, w.dst)
+    def step():
+        oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
+                       csr[0], csr[1])
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter(); step(); times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = w.E * w.H / sec
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "N": w.N, "E": w.E, "d": w.d, "H": w.H, "r": w.r,
+                       "io": w.io, "parallelism": "host oracle, rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"the full {w.name} workload per step (N={w.N}, E={w.E})"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default="arxiv")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from sparse_graph_attention_tcgen05_b200 import glga
+    from sparse_graph_attention_tcgen05_b200.workloads import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = make_workload(args.workload)
+    dt = glga.torch_dtype(w.io)
+    s_io = 4 if w.io == "f32" else 2
+
+    # ---- bind the graph (CSR build + create), timed separately ----
+    src = torch.from_numpy(w.src).to(dev)
+    dst = torch.from_numpy(w.dst).to(dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    row_ptr, col_idx = glga.csr_from_coo(w.N, src, dst)
+    t1 = time.perf_counter()
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+    torch.cuda.synchronize()
+    t2 = time.perf_counter()
+    create = {"csr_from_coo_ms": (t1 - t0) * 1e3, "glga_create_ms": (t2 - t1) * 1e3,
+              "buckets": layer.bucket_counts(), "workspace_bytes": layer.workspace_bytes()}
+
+    host = {k: torch.from_numpy(np.ascontiguousarray(a)).to(dt).pin_memory()
+            for k, a in (("X", w.X), ("W_Q", w.W_Q), ("W_K", w.W_K), ("W_V", w.W_V), ("w_g", w.w_g))}
+    X, WQ, WK, WV, wg = (host[k].to(dev) for k in ("X", "W_Q", "W_K", "W_V", "w_g"))
+    Y = torch.empty(w.N, w.D, dtype=dt, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        layer.forward(X, WQ, WK, WV, wg, b_g=w.b_g, eps=w.eps, Y=Y)
+
+    # ---- warm-up ----
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    assert layer.last_device_error() == 0
+
+    # ---- parity spot check of what is being timed (sampled rows vs the oracle) ----
+    parity = None
+    if rank == 0:
+        import oracle
+        csr = (row_ptr.cpu().numpy(), col_idx.cpu().numpy())
+        rng = np.random.default_rng(0)
+        rows = np.unique(np.concatenate([rng.choice(w.N, 256, replace=False),
+                                         np.argsort(np.diff(csr[0]))[-8:]]))
+        ref = oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
+                             csr[0], csr[1], rows=rows)
+        Yg = Y.float().cpu().numpy()[rows].astype(np.float64)
+        parity = float(np.abs(Yg - ref["Y"]).max() / np.abs(ref["Y"]).max())
+
+    # ---- timed region: K forwards, L2 flushed between them ----
+    layer.set_timing(True)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = layer.kernel_launches()
+    stage_sum = {k: 0.0 for k in glga.STAGES}
+    step_ms = []
+    barrier()
+    torch.cuda.synchronize()
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in visible.split(",") if v.strip()]
+    sampler = ClockSampler(ids[local_rank] if local_rank < len(ids) else local_rank)
+    wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        flush.zero_()
+        ev0.record(stream)
+        fwd()
+        ev1.record(stream)
+        ev1.synchronize()
+        step_ms.append(ev0.elapsed_time(ev1))
+        for k, v in layer.stage_times().items():
+            stage_sum[k] += v
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    barrier()
+    launches = layer.kernel_launches() - launches0
+    layer.set_timing(False)
+    assert layer.last_device_error() == 0
+
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / args.steps
+    value = world * w.E * w.H / (ms_per_step * 1e-3)
+    stages = {k: v / args.steps for k, v in stage_sum.items()}
+
+    # ---- end to end through the public API: pinned host -> device, forward, Y -> host ----
+    Yh = torch.empty(w.N, w.D, dtype=dt).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = Yh.numel() * Yh.element_size()
+    e2e_ms = []
+    for i in range(args.e2e_steps + 3):
+        ev0.record(stream)
+        X.copy_(host["X"], non_blocking=True)
+        WQ.copy_(host["W_Q"], non_blocking=True)
+        WK.copy_(host["W_K"], non_blocking=True)
+        WV.copy_(host["W_V"], non_blocking=True)
+        wg.copy_(host["w_g"], non_blocking=True)
+        fwd()
+        Yh.copy_(Y, non_blocking=True)
+        ev1.record(stream)
+        ev1.synchronize()
+        if i >= 3:
+            e2e_ms.append(ev0.elapsed_time(ev1))
+    e2e_step = max_over_ranks(sum(e2e_ms)) / len(e2e_ms)
+    e2e = {"value": world * w.E * w.H / (e2e_step * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
+
+    peaks, peak_kind = load_peaks()
+    B_loc = local_bytes_model(w.N, w.E, w.D, w.H, w.r, s_io)
+    t_local = stages["local"] * 1e-3
+    achieved = B_loc / t_local / 1e9
+    traffic, traffic_note = profiled_traffic(args.workload)
+    roofline = {"bound": "hbm", "kernel": "local_kernel (local branch + readout + gate)",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "algorithmic_bytes_per_launch": B_loc, "avg_launch_ms": stages["local"],
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s"}
+    if traffic_note:
+        roofline["traffic_note"] = traffic_note
+    gemm_flops = 2.0 * w.N * w.d * (3 * w.D + 1)
+    gemm_bytes = w.N * w.d * s_io + w.N * 3 * w.D * s_io + 4 * w.N
+    t_gemm = stages["gemm"] * 1e-3
+    tpeak = peaks["bf16_tflops"]
+    attainable = min(tpeak * 1e12, gemm_flops / gemm_bytes * peaks["hbm_gbs"] * 1e9)
+    projection = {"tflops": gemm_flops / t_gemm / 1e12, "frac_of_tensor_peak": gemm_flops / t_gemm / (tpeak * 1e12),
+                  "frac_of_attainable": gemm_flops / t_gemm / attainable,
+                  "arith_intensity_flop_per_byte": gemm_flops / gemm_bytes,
+                  "hbm_gbs": gemm_bytes / t_gemm / 1e9}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
+            "config": {"workload": args.workload, "N": w.N, "E": w.E, "d": w.d, "H": w.H,
+                       "r": w.r, "io": w.io, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between timed steps (256 MiB write, outside the timed spans)"},
+            "roofline": roofline, "projection": projection,
+            "stages_ms": stages, "create": create, "gpu_launches": launches,
+            "e2e": e2e, "clocks": clocks, "parity_max_rel_err": parity,
+            "wall_s_timed_region": wall}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, (row_ptr.cpu().numpy(), col_idx.cpu().numpy()))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+/*
+ * glga.h -- C ABI of libglga: the forward pass of a gated local-global graph-attention
+ * layer over a fixed sparse adjacency, on NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (method page "Gated Local-Global Graph Attention", section
+ * "Key formulas"; heads of width r as in the tinymesh page "Sparse attention
+ * experiment", section "Multiple heads are composition"):
+ *
+ *   per head h (columns h*r .. h*r+r-1):
+ *     q_i = x_i W_Q,  k_j = x_j W_K,  v_j = x_j W_V
+ *     L_i = sum over in-neighbours j of i of softmax_j(q_i . k_j / sqrt(r)) v_j
+ *     G_i = phi(q_i)^T S / (phi(q_i)^T z + eps),  S = sum_j phi(k_j) v_j^T,
+ *           z = sum_j phi(k_j),  phi(x) = elu(x) + 1,  j over all N nodes
+ *   g_i = sigmoid(x_i . w_g + b_g),  Y_i = g_i L_i + (1 - g_i) G_i   (heads concatenated)
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked (device) are CUDA device pointers on the current device; pointers
+ *    marked (host) are ordinary host memory.  All matrices are dense, row-major and
+ *    contiguous.  The caller owns every buffer it passes; the library never frees them.
+ *  - `io` is the element type of X, W_Q, W_K, W_V, w_g and Y: GLGA_F32 (float) or
+ *    GLGA_BF16 (bfloat16 bits).  Internal accumulation is float32.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - No entry point aborts, throws or prints; failures return a glga_status and leave a
+ *    one-line reason retrievable with glga_last_error_message() (per calling thread).
+ *  - The graph is a target-grouped CSR: row i lists the sources j of the edges j -> i
+ *    (A_ij = 1), so a row's entries are i's in-neighbours.  Self-loops are whatever the
+ *    CSR holds; the library never adds or removes edges.  A duplicated entry is one more
+ *    softmax term.  A row without entries has L_i = 0 (an empty weighted sum).
+ */
+#ifndef GLGA_H_
+#define GLGA_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GLGA_API __attribute__((visibility("default")))
+#else
+#define GLGA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct glga_ctx glga_ctx;
+
+typedef enum {
+    GLGA_OK = 0,
+    GLGA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned buffer       */
+    GLGA_ERR_BAD_GRAPH = 2,     /* CSR/COO violates its invariants (see glga_create)    */
+    GLGA_ERR_UNSUPPORTED = 3,   /* shape outside the supported set (see glga_create)    */
+    GLGA_ERR_OOM = 4,           /* a device allocation failed                           */
+    GLGA_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed                    */
+    GLGA_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (reported late)   */
+    GLGA_ERR_DEVICE = 7         /* a device-side check failed (reported late)           */
+} glga_status;
+
+typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
+
+/* Scheduling of target rows by in-degree (deg = row_ptr[i+1] - row_ptr[i]):
+ *   deg <= warp_max_degree                 -> bucket 0: one warp per row
+ *   warp_max_degree < deg <= chunk_edges   -> bucket 1: one thread block per row
+ *   deg > chunk_edges                      -> bucket 2: the row is cut into chunks of
+ *        chunk_edges edges, one thread block per chunk, chunks merged in order.
+ * Rows are kept in ascending order inside every bucket.  Requires
+ * 0 <= warp_max_degree <= chunk_edges and chunk_edges >= 1.                            */
+typedef struct {
+    int32_t warp_max_degree;
+    int32_t chunk_edges;
+} glga_options;
+
+/* Fills *opts with the defaults used when glga_create gets opts == NULL. */
+GLGA_API glga_status glga_default_options(glga_options *opts);
+
+/* glga_create -- bind a fixed graph and the layer shape; allocate all workspaces.
+ *   N        number of nodes (>= 0, < 2^31)
+ *   d        input width (>= 1)
+ *   H, r     heads and per-head width; r in {8, 16, 32, 64, 128}, H >= 1, and the row
+ *            width D = H*r must satisfy D*sizeof(io) <= 2048 bytes
+ *   row_ptr  (device) int32 [N+1], row_ptr[0] = 0, non-decreasing, row_ptr[N] = E
+ *   col_idx  (device) int32 [E], every entry in [0, N)
+ *   E        number of CSR entries (>= 0, < 2^31)
+ *   opts     (host, nullable) bucket thresholds; NULL selects the defaults
+ * The CSR is copied into the context and validated on the device (GLGA_ERR_BAD_GRAPH if
+ * it violates the invariants above), then bucketed by degree.  This call synchronises
+ * `stream` (validation result and bucket sizes are read back).  The caller may free its
+ * CSR afterwards.  Workspaces are O(N*(3*H*r + d) + E); nothing is O(N^2) or O(E*r).
+ * On success *out owns device memory until glga_destroy.                              */
+GLGA_API glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t r,
+                        glga_dtype io, const int32_t *row_ptr, const int32_t *col_idx,
+                        int64_t E, const glga_options *opts, void *stream);
+
+/* glga_forward -- Y = layer(X) for the graph bound at create.
+ *   X    (device) io [N, d]          W_Q, W_K, W_V (device) io [d, H*r]
+ *   w_g  (device) io [d]             b_g, eps (host) gate bias and readout epsilon
+ *   Y    (device) io [N, H*r], written entirely
+ * Enqueued on `stream` with no host synchronisation; the context's workspaces are
+ * reused, so calls on one context must be ordered (same stream, or synchronised).
+ * Device-side failures (bounded waits, debug checks) surface through
+ * glga_last_device_error().  eps must be > 0 and finite.                              */
+GLGA_API glga_status glga_forward(glga_ctx *ctx, const void *X, const void *W_Q, const void *W_K,
+                         const void *W_V, const void *w_g, float b_g, float eps, void *Y,
+                         void *stream);
+
+/* Frees every device buffer of the context (synchronises the device first).  NULL is a
+ * no-op.                                                                              */
+GLGA_API glga_status glga_destroy(glga_ctx *ctx);
+
+/* glga_csr_from_coo -- target-grouped CSR from an edge list (tinymesh page, "Target
+ * softmax": segment reductions traverse destination CSR).
+ *   src, dst  (device) int32 [E]: edge e is src[e] -> dst[e]
+ *   row_ptr   (device) int32 [N+1] out;  col_idx (device) int32 [E] out
+ * Rows are targets; inside a row the sources are sorted ascending; duplicates are kept.
+ * The result depends only on the multiset of edges, not on their order.  Returns
+ * GLGA_ERR_BAD_GRAPH if an endpoint is outside [0, N).  Allocates temporary device
+ * memory and synchronises `stream` once.                                              */
+GLGA_API glga_status glga_csr_from_coo(int64_t N, int64_t E, const int32_t *src, const int32_t *dst,
+                              int32_t *row_ptr, int32_t *col_idx, void *stream);
+
+/* Bucket sizes chosen at create: counts (host) int64 [4] = rows in buckets 0, 1, 2 and
+ * the number of bucket-2 chunks.                                                      */
+GLGA_API glga_status glga_bucket_counts(const glga_ctx *ctx, int64_t *counts);
+
+/* Copies the bucket lists (device -> device, on `stream`) into caller buffers sized by
+ * glga_bucket_counts: warp_rows [counts[0]], cta_rows [counts[1]], split_rows [counts[2]],
+ * chunk_row [counts[3]], chunk_begin [counts[3]] (the CSR offset of the chunk's first
+ * edge).  Any pointer may be NULL to skip that list.                                  */
+GLGA_API glga_status glga_get_buckets(const glga_ctx *ctx, int32_t *warp_rows, int32_t *cta_rows,
+                             int32_t *split_rows, int32_t *chunk_row, int32_t *chunk_begin,
+                             void *stream);
+
+/* Copies the intermediates of the last glga_forward (device -> device, on `stream`):
+ *   Q (io [N, H*r]), K and V (io [N, H*r] each), t (float [N], gate logit x_i . w_g),
+ *   S (float [H, r, r]), z (float [H, r]).  Any pointer may be NULL.                   */
+GLGA_API glga_status glga_get_intermediates(const glga_ctx *ctx, void *Q, void *K, void *V, float *t,
+                                   float *S, float *z, void *stream);
+
+/* Per-stage timing.  When enabled, glga_forward records CUDA events on its stream around
+ * every stage.  glga_stage_times synchronises on the last forward's final event and
+ * writes up to n_max durations in milliseconds (host) in this order:
+ *   0 weight packing and input preparation, 1 projection GEMM, 2 global statistics,
+ *   3 local branch + readout + gate (the fused per-target kernel), 4 whole forward.
+ * Returns the number of values written through *n_written.                            */
+GLGA_API glga_status glga_set_timing(glga_ctx *ctx, int enable);
+GLGA_API glga_status glga_stage_times(glga_ctx *ctx, float *ms, int32_t n_max, int32_t *n_written);
+
+/* Number of kernel launches glga_forward has issued on this context so far (host-side
+ * count, incremented at every launch).                                                */
+GLGA_API glga_status glga_kernel_launches(const glga_ctx *ctx, int64_t *n);
+
+/* Bytes of device memory the context holds (workspaces + CSR copy + buckets).         */
+GLGA_API glga_status glga_workspace_bytes(const glga_ctx *ctx, int64_t *bytes);
+
+/* Synchronises `stream` and reports (then clears) the device-side error flag of the
+ * context: GLGA_OK, GLGA_ERR_TIMEOUT or GLGA_ERR_DEVICE.                              */
+GLGA_API glga_status glga_last_device_error(glga_ctx *ctx, void *stream);
+
+/* Static strings; never NULL. */
+GLGA_API const char *glga_status_string(glga_status s);
+GLGA_API const char *glga_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLGA_H_ */

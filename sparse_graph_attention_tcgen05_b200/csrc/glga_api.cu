@@ -1,0 +1,382 @@
+// glga_api.cu -- the C ABI of libglga (declared in include/glga.h).
+//
+// Argument checking, context lifetime, workspace allocation, stage ordering on the
+// caller's stream and error reporting.  All arithmetic happens in the kernels of
+// projection.cu, global_stats.cu, local.cu and topology.cu.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "glga_internal.cuh"
+
+namespace glga {
+
+namespace {
+thread_local char g_msg[512] = "no error";
+}
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+}
+
+glga_status cuda_fail(cudaError_t e, const char *what) {
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    if (e == cudaErrorMemoryAllocation) return GLGA_ERR_OOM;
+    return GLGA_ERR_CUDA;
+}
+
+glga_status dev_alloc(Ctx *c, void **p, size_t bytes) {
+    if (bytes == 0) bytes = 16;
+    cudaError_t e = cudaMalloc(p, bytes);
+    if (e != cudaSuccess) {
+        *p = nullptr;
+        return cuda_fail(e, "cudaMalloc");
+    }
+    c->bytes += static_cast<int64_t>(bytes);
+    return GLGA_OK;
+}
+
+// Releases every device resource held by the context (the host object is freed by the
+// caller).
+static void release_ctx(Ctx *c) {
+    if (!c) return;
+    void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
+                    c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
+                    c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->dev_flag};
+    for (void *p : ptrs)
+        if (p) cudaFree(p);
+    for (auto &e : c->ev)
+        if (e) cudaEventDestroy(e);
+}
+
+}  // namespace glga
+
+using namespace glga;
+
+struct glga_ctx {
+    Ctx c;
+};
+
+extern "C" {
+
+const char *glga_status_string(glga_status s) {
+    switch (s) {
+        case GLGA_OK: return "ok";
+        case GLGA_ERR_INVALID_ARG: return "invalid argument";
+        case GLGA_ERR_BAD_GRAPH: return "invalid graph";
+        case GLGA_ERR_UNSUPPORTED: return "unsupported shape";
+        case GLGA_ERR_OOM: return "out of device memory";
+        case GLGA_ERR_CUDA: return "CUDA error";
+        case GLGA_ERR_TIMEOUT: return "device-side wait timed out";
+        case GLGA_ERR_DEVICE: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+const char *glga_last_error_message(void) { return g_msg; }
+
+glga_status glga_default_options(glga_options *opts) {
+    if (!opts) {
+        set_error("glga_default_options: null pointer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    opts->warp_max_degree = 128;
+    opts->chunk_edges = 1024;
+    return GLGA_OK;
+}
+
+glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t r,
+                        glga_dtype io, const int32_t *row_ptr, const int32_t *col_idx, int64_t E,
+                        const glga_options *opts, void *stream) {
+    if (!out) {
+        set_error("glga_create: out is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    *out = nullptr;
+    if (N < 0 || N > 2147483646LL || E < 0 || E > 2147483647LL || d < 1 || H < 1) {
+        set_error("glga_create: need 0 <= N < 2^31-1, 0 <= E < 2^31, d >= 1, H >= 1");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (io != GLGA_F32 && io != GLGA_BF16) {
+        set_error("glga_create: io must be GLGA_F32 or GLGA_BF16");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (!(r == 8 || r == 16 || r == 32 || r == 64 || r == 128)) {
+        set_error("glga_create: r must be one of 8, 16, 32, 64, 128 (got %d)", r);
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    const int elem = io == GLGA_F32 ? 4 : 2;
+    const int64_t D = static_cast<int64_t>(H) * r;
+    if (D * elem > 2048) {
+        set_error("glga_create: H*r*sizeof(io) = %lld bytes exceeds 2048",
+                  static_cast<long long>(D * elem));
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    if (!row_ptr || (E > 0 && !col_idx)) {
+        set_error("glga_create: null CSR pointer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    glga_options o;
+    glga_default_options(&o);
+    if (opts) o = *opts;
+    if (o.warp_max_degree < 0 || o.chunk_edges < 1 || o.warp_max_degree > o.chunk_edges) {
+        set_error("glga_create: need 0 <= warp_max_degree <= chunk_edges, chunk_edges >= 1");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    glga_ctx *h = new (std::nothrow) glga_ctx();
+    if (!h) {
+        set_error("glga_create: host allocation failed");
+        return GLGA_ERR_OOM;
+    }
+    Ctx *c = &h->c;
+    c->N = N;
+    c->E = E;
+    c->d = d;
+    c->H = H;
+    c->r = r;
+    c->D = static_cast<int32_t>(D);
+    c->io = io;
+    c->elem = elem;
+    c->opts = o;
+    glga_status st = GLGA_OK;
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+    int cc_major = 0, cc_minor = 0;
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, c->device);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&cc_minor, cudaDevAttrComputeCapabilityMinor, c->device);
+    if (e != cudaSuccess) st = cuda_fail(e, "device query");
+    if (st == GLGA_OK && !(cc_major == 10 && cc_minor == 0)) {
+        set_error("glga_create: needs an sm_100 device (B200); found sm_%d%d", cc_major, cc_minor);
+        st = GLGA_ERR_UNSUPPORTED;
+    }
+#define TRY(x) \
+    if (st == GLGA_OK) st = (x)
+    TRY(dev_alloc(c, reinterpret_cast<void **>(&c->dev_flag), 64));
+    TRY(dev_alloc(c, reinterpret_cast<void **>(&c->row_ptr), (N + 1) * sizeof(int32_t)));
+    TRY(dev_alloc(c, reinterpret_cast<void **>(&c->col_idx), (E > 0 ? E : 1) * sizeof(int32_t)));
+    if (st == GLGA_OK) {
+        e = cudaMemcpyAsync(c->row_ptr, row_ptr, (N + 1) * sizeof(int32_t),
+                            cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess && E > 0)
+            e = cudaMemcpyAsync(c->col_idx, col_idx, E * sizeof(int32_t),
+                                cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) st = cuda_fail(e, "CSR copy");
+    }
+    TRY(validate_csr(c, s));
+    TRY(build_buckets(c, s));
+    TRY(dev_alloc(c, &c->Q, static_cast<size_t>(N) * D * elem));
+    TRY(dev_alloc(c, &c->KV, static_cast<size_t>(N) * 2 * D * elem));
+    TRY(dev_alloc(c, reinterpret_cast<void **>(&c->t), static_cast<size_t>(N) * sizeof(float)));
+    TRY(projection_setup(c));
+    TRY(stats_setup(c));
+    TRY(local_setup(c));
+    if (st == GLGA_OK) {
+        e = cudaMemsetAsync(c->dev_flag, 0, 64, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) st = cuda_fail(e, "create sync");
+    }
+#undef TRY
+    if (st != GLGA_OK) {
+        cudaStreamSynchronize(s);
+        release_ctx(c);
+        delete h;
+        return st;
+    }
+    *out = h;
+    return GLGA_OK;
+}
+
+glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void *W_K,
+                         const void *W_V, const void *w_g, float b_g, float eps, void *Y,
+                         void *stream) {
+    if (!h) {
+        set_error("glga_forward: ctx is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    if (!W_Q || !W_K || !W_V || !w_g || (c->N > 0 && (!X || !Y))) {
+        set_error("glga_forward: null pointer argument");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (!(eps > 0.f) || !std::isfinite(eps) || !std::isfinite(b_g)) {
+        set_error("glga_forward: eps must be finite and > 0, b_g finite");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    const uintptr_t align_or = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Y);
+    if (align_or & 15u) {
+        set_error("glga_forward: X and Y must be 16-byte aligned");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (c->timing) {
+        for (auto &ev : c->ev)
+            if (!ev) GLGA_CUDA(cudaEventCreate(&ev));
+        GLGA_CUDA(cudaEventRecord(c->ev[kStagePrep], s));
+    }
+    glga_status st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, c->timing);
+    if (st != GLGA_OK) return st;
+    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageStats], s));
+    st = stats_run(c, s);
+    if (st != GLGA_OK) return st;
+    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageLocal], s));
+    st = local_run(c, b_g, eps, Y, s);
+    if (st != GLGA_OK) return st;
+    if (c->timing) {
+        GLGA_CUDA(cudaEventRecord(c->ev[kStageEnd], s));
+        c->ev_recorded = true;
+    }
+    return GLGA_OK;
+}
+
+glga_status glga_destroy(glga_ctx *h) {
+    if (!h) return GLGA_OK;
+    cudaDeviceSynchronize();
+    release_ctx(&h->c);
+    delete h;
+    return GLGA_OK;
+}
+
+glga_status glga_bucket_counts(const glga_ctx *h, int64_t *counts) {
+    if (!h || !counts) {
+        set_error("glga_bucket_counts: null pointer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    for (int k = 0; k < 4; ++k) counts[k] = h->c.nb[k];
+    return GLGA_OK;
+}
+
+glga_status glga_get_buckets(const glga_ctx *h, int32_t *warp_rows, int32_t *cta_rows,
+                             int32_t *split_rows, int32_t *chunk_row, int32_t *chunk_begin,
+                             void *stream) {
+    if (!h) {
+        set_error("glga_get_buckets: ctx is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    const Ctx *c = &h->c;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    struct {
+        int32_t *dst;
+        const int32_t *src;
+        int64_t n;
+    } items[] = {{warp_rows, c->warp_rows, c->nb[0]}, {cta_rows, c->cta_rows, c->nb[1]},
+                 {split_rows, c->split_rows, c->nb[2]}, {chunk_row, c->chunk_row, c->nb[3]},
+                 {chunk_begin, c->chunk_begin, c->nb[3]}};
+    for (auto &it : items)
+        if (it.dst && it.n > 0)
+            GLGA_CUDA(cudaMemcpyAsync(it.dst, it.src, it.n * sizeof(int32_t),
+                                      cudaMemcpyDeviceToDevice, s));
+    return GLGA_OK;
+}
+
+glga_status glga_get_intermediates(const glga_ctx *h, void *Q, void *K, void *V, float *t,
+                                   float *S, float *z, void *stream) {
+    if (!h) {
+        set_error("glga_get_intermediates: ctx is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    const Ctx *c = &h->c;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t row = static_cast<size_t>(c->D) * c->elem;
+    if (c->N > 0) {
+        if (Q) GLGA_CUDA(cudaMemcpyAsync(Q, c->Q, c->N * row, cudaMemcpyDeviceToDevice, s));
+        if (K)
+            GLGA_CUDA(cudaMemcpy2DAsync(K, row, c->KV, 2 * row, row, c->N,
+                                        cudaMemcpyDeviceToDevice, s));
+        if (V)
+            GLGA_CUDA(cudaMemcpy2DAsync(V, row, static_cast<const uint8_t *>(c->KV) + row, 2 * row,
+                                        row, c->N, cudaMemcpyDeviceToDevice, s));
+        if (t) GLGA_CUDA(cudaMemcpyAsync(t, c->t, c->N * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    }
+    const size_t sbytes = static_cast<size_t>(c->H) * c->r * c->r * sizeof(float);
+    if (S) GLGA_CUDA(cudaMemcpyAsync(S, c->Sz, sbytes, cudaMemcpyDeviceToDevice, s));
+    if (z)
+        GLGA_CUDA(cudaMemcpyAsync(z, c->Sz + static_cast<size_t>(c->H) * c->r * c->r,
+                                  static_cast<size_t>(c->H) * c->r * sizeof(float),
+                                  cudaMemcpyDeviceToDevice, s));
+    return GLGA_OK;
+}
+
+glga_status glga_set_timing(glga_ctx *h, int enable) {
+    if (!h) {
+        set_error("glga_set_timing: ctx is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    h->c.timing = enable != 0;
+    h->c.ev_recorded = false;
+    return GLGA_OK;
+}
+
+glga_status glga_stage_times(glga_ctx *h, float *ms, int32_t n_max, int32_t *n_written) {
+    if (!h || !ms || !n_written) {
+        set_error("glga_stage_times: null pointer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    *n_written = 0;
+    if (!c->timing || !c->ev_recorded) {
+        set_error("glga_stage_times: timing disabled or no forward recorded");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    GLGA_CUDA(cudaEventSynchronize(c->ev[kStageEnd]));
+    float v[5];
+    GLGA_CUDA(cudaEventElapsedTime(&v[0], c->ev[kStagePrep], c->ev[kStageGemm]));
+    GLGA_CUDA(cudaEventElapsedTime(&v[1], c->ev[kStageGemm], c->ev[kStageStats]));
+    GLGA_CUDA(cudaEventElapsedTime(&v[2], c->ev[kStageStats], c->ev[kStageLocal]));
+    GLGA_CUDA(cudaEventElapsedTime(&v[3], c->ev[kStageLocal], c->ev[kStageEnd]));
+    GLGA_CUDA(cudaEventElapsedTime(&v[4], c->ev[kStagePrep], c->ev[kStageEnd]));
+    const int n = n_max < 5 ? n_max : 5;
+    for (int i = 0; i < n; ++i) ms[i] = v[i];
+    *n_written = n;
+    return GLGA_OK;
+}
+
+glga_status glga_kernel_launches(const glga_ctx *h, int64_t *n) {
+    if (!h || !n) {
+        set_error("glga_kernel_launches: null pointer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    *n = h->c.launches;
+    return GLGA_OK;
+}
+
+glga_status glga_workspace_bytes(const glga_ctx *h, int64_t *bytes) {
+    if (!h || !bytes) {
+        set_error("glga_workspace_bytes: null pointer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    *bytes = h->c.bytes;
+    return GLGA_OK;
+}
+
+glga_status glga_last_device_error(glga_ctx *h, void *stream) {
+    if (!h) {
+        set_error("glga_last_device_error: ctx is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned f = 0;
+    GLGA_CUDA(cudaMemcpyAsync(&f, c->dev_flag, sizeof(unsigned), cudaMemcpyDeviceToHost, s));
+    GLGA_CUDA(cudaStreamSynchronize(s));
+    GLGA_CUDA(cudaMemsetAsync(c->dev_flag, 0, sizeof(unsigned), s));
+    if (f & kDevErrTimeout) {
+        set_error("a bounded device-side wait timed out");
+        return GLGA_ERR_TIMEOUT;
+    }
+    if (f) {
+        set_error("device-side check failed (flags 0x%x)", f);
+        return GLGA_ERR_DEVICE;
+    }
+    return GLGA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,293 @@
+// glga_internal.cuh -- shared declarations of libglga's CUDA sources (not installed).
+//
+// Device helpers wrap the sm_100a instructions the kernels use: mbarrier waits with an
+// upper bound, TMA 2-D tiled loads (no cluster multicast anywhere in this library),
+// tcgen05 TMEM allocation, MMA issue/commit and TMEM loads.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "glga.h"
+
+namespace glga {
+
+// ---------------------------------------------------------------------------------------
+// error reporting
+// ---------------------------------------------------------------------------------------
+void set_error(const char *fmt, ...);
+glga_status cuda_fail(cudaError_t e, const char *what);
+
+#define GLGA_CUDA(call)                                                    \
+    do {                                                                   \
+        cudaError_t _e = (call);                                           \
+        if (_e != cudaSuccess) return ::glga::cuda_fail(_e, #call);        \
+    } while (0)
+
+// Device-side error flag bits (ctx->dev_flag).
+enum : unsigned {
+    kDevErrTimeout = 1u,   // a bounded mbarrier wait gave up
+    kDevErrBounds = 2u,    // a device-side check found an out-of-range index
+};
+
+// Validation flag bits for topology checks.
+enum : unsigned {
+    kGraphBadRowPtr0 = 1u,
+    kGraphBadRowPtrEnd = 2u,
+    kGraphNotMonotone = 4u,
+    kGraphColOutOfRange = 8u,
+};
+
+// ---------------------------------------------------------------------------------------
+// context
+// ---------------------------------------------------------------------------------------
+struct TensorMap2D {
+    CUtensorMap map;
+    bool valid = false;
+};
+
+enum Stage { kStagePrep = 0, kStageGemm, kStageStats, kStageLocal, kStageEnd, kNumEvents };
+
+struct Ctx {
+    int device = 0;
+    int num_sms = 148;
+    int64_t N = 0, E = 0;
+    int32_t d = 0, H = 0, r = 0, D = 0;
+    glga_dtype io = GLGA_F32;
+    int elem = 4;                 // bytes per io element
+    glga_options opts{};
+
+    // topology (owned copies)
+    int32_t *row_ptr = nullptr, *col_idx = nullptr;
+    int64_t nb[4] = {0, 0, 0, 0};   // bucket sizes and chunk count
+    int32_t *warp_rows = nullptr, *cta_rows = nullptr, *split_rows = nullptr;
+    int32_t *chunk_row = nullptr, *chunk_begin = nullptr;
+    unsigned *chunk_ticket = nullptr;   // one counter per chunk slot (first chunk of a row)
+    float *chunk_part = nullptr;        // per chunk: m[H], l[H], acc[D]
+
+    // projection
+    int32_t dp = 0;               // padded input width (multiple of the K tile)
+    int32_t Dp = 0;               // padded GEMM width: 3*D + gate column + padding
+    int32_t BN = 0, n_tiles = 0, stages = 0, tmem_cols = 0;
+    int split = 1;                // 1: bf16 MMA; 3: 3-term tf32 split (fp32 io)
+    bool x_direct = false;        // A operand read straight from the caller's X
+    void *Wt = nullptr;           // [planes][Dp][dp]
+    void *Xp = nullptr;           // [planes][N][dp] (prepared A operand when !x_direct)
+    TensorMap2D tmB[2], tmA[2];
+
+    // intermediates
+    void *Q = nullptr;            // io [N, D]
+    void *KV = nullptr;           // io [N, 2D]  (k_j | v_j)
+    float *t = nullptr;           // [N] gate logits
+    float *Spart = nullptr;       // [P][H][r][r+1]
+    float *Sz = nullptr;          // [H][r][r+1]  S rows with z as the last column
+    int32_t stats_parts = 0, stats_rows_per_part = 0;
+
+    unsigned *dev_flag = nullptr;
+    int64_t bytes = 0;
+    int64_t launches = 0;         // kernels launched by glga_forward so far
+
+    bool timing = false;
+    cudaEvent_t ev[kNumEvents] = {};
+    bool ev_recorded = false;
+};
+
+// allocation helper that tracks bytes
+glga_status dev_alloc(Ctx *c, void **p, size_t bytes);
+
+// topology.cu
+glga_status validate_csr(Ctx *c, cudaStream_t s);
+glga_status build_buckets(Ctx *c, cudaStream_t s);
+glga_status exclusive_scan_i32(const int32_t *in, int32_t *out, int64_t n, int32_t *total_dev,
+                               cudaStream_t s, void *tmp, size_t tmp_bytes);
+size_t scan_tmp_bytes(int64_t n);
+
+// projection.cu
+glga_status projection_setup(Ctx *c);
+glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK,
+                           const void *WV, const void *wg, cudaStream_t s, bool time_prep);
+
+// global_stats.cu
+glga_status stats_setup(Ctx *c);
+glga_status stats_run(Ctx *c, cudaStream_t s);
+
+// local.cu
+glga_status local_setup(Ctx *c);
+glga_status local_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s);
+
+// tensor maps (driver entry point resolved at run time; no libcuda link dependency)
+glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
+                           uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                           uint32_t box_inner, uint32_t box_outer);
+
+// ---------------------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up after about
+// `limit_ns` nanoseconds of wall time (checked every 256 polls) or 2^26 polls, whichever
+// comes first, and returns false; the caller records the timeout and winds down.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint64_t limit_ns = 1000000000ull) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1; it < (1u << 26); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return false;
+}
+
+// 2-D tiled TMA load global -> shared, completing on an mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// --- tcgen05 ----------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 "matrix descriptor"): start address, leading
+// and stride byte offsets (16-byte units), version 1, swizzle mode in bits 61..63
+// (2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t swz) {
+    uint64_t dsc = 0;
+    dsc |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    dsc |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    dsc |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    dsc |= static_cast<uint64_t>(1u) << 46;
+    dsc |= static_cast<uint64_t>(swz & 7u) << 61;
+    return dsc;
+}
+
+// Instruction descriptor for kind::f16 / kind::tf32 with an f32 accumulator.
+// fmt: 1 = bf16, 2 = tf32.  a_mn / b_mn select MN-major operands.
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, uint32_t fmt, bool a_mn,
+                                                  bool b_mn) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((static_cast<uint32_t>(N) >> 3) << 17) |
+           ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// Arrives on `bar` once every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// TMEM -> registers: 32 lanes x 32 consecutive 32-bit columns (one row per thread).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Round-to-nearest (ties away) conversion of an f32 to tf32, kept in an f32 container.
+__device__ __forceinline__ float to_tf32(float x) {
+    uint32_t u;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(u) : "f"(x));
+    return __uint_as_float(u);
+}
+
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace glga

@@ -1,0 +1,496 @@
+// local.cu -- per-target kernel: local softmax branch + global readout + gate + blend.
+//
+// Method page "Gated Local-Global Graph Attention", Key formulas:
+//   L_i = sum_{j in N(i)} softmax_j(q_i . k_j / sqrt r) v_j
+//   G_i = phi(q_i)^T S / (phi(q_i)^T z + eps)
+//   Y_i = g_i L_i + (1 - g_i) G_i,  g_i = sigmoid(t_i + b_g)
+// evaluated per head and concatenated.  The softmax is the stable one of the tinymesh
+// page ("Target softmax"), computed in a single pass with a running maximum: the state
+// (m, l, acc) of a partial sum is rescaled by 2^(m_old - m_new) whenever the maximum
+// grows, and two partial states merge the same way, so edges may be split across lanes,
+// warps and thread blocks and merged in a fixed order.  No per-edge value is stored.
+//
+// Work is scheduled by the degree buckets built at create time:
+//   chunk blocks   bucket-2 rows cut into chunk_edges-edge chunks; each block merges its
+//                  8 warps, writes (m, l, acc) to scratch, and the last block of a row
+//                  (ticket counter) merges the row's chunks in chunk order and finishes
+//   row blocks     bucket-1 rows: 8 warps split the edges, merged in warp order
+//   warp blocks    bucket-0 rows: one warp per row, 8 rows per block
+// Heavy work comes first in block order so it starts early.
+//
+// Lane layout: a 16-byte vector holds VE = 16/sizeof(T) consecutive features; an edge's
+// k_j (or v_j) row is LPE lanes x VPL vectors; EPW = 32/LPE edges are in flight per warp
+// step (U steps unrolled), and the r features of a head live in LPH = r/VE adjacent
+// lanes, which reduce dot products with butterfly shuffles.
+#include <algorithm>
+#include <cmath>
+
+#include "glga_internal.cuh"
+
+namespace glga {
+namespace {
+
+constexpr int kLocalWarps = 8;
+constexpr int kLocalThreads = kLocalWarps * 32;
+
+template <typename T>
+struct Io;
+template <>
+struct Io<float> {
+    static constexpr int VE = 4;
+    __device__ __forceinline__ static void unpack(const uint4 &u, float (&f)[VE]) {
+        f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[VE]) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+};
+template <>
+struct Io<__nv_bfloat16> {
+    static constexpr int VE = 8;
+    __device__ __forceinline__ static void unpack(const uint4 &u, float (&f)[VE]) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[VE]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+__device__ __forceinline__ uint4 ld_gather(const void *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+struct LocalParams {
+    const int32_t *row_ptr;
+    const int32_t *col_idx;
+    const int32_t *warp_rows;
+    const int32_t *cta_rows;
+    const int32_t *chunk_row;
+    const int32_t *chunk_begin;
+    int64_t n_warp, n_cta, n_chunks;
+    int64_t warp_blocks;
+    int32_t chunk_edges;
+    const void *Q;
+    const void *KV;
+    const float *t;
+    const float *S;      // [H][r][r]
+    const float *z;      // [H][r]
+    float *part;         // per chunk: m[H] l[H] acc[D]
+    unsigned *ticket;
+    void *Y;
+    int32_t D, r, H, nvec, lpe, epw, lph;
+    float score_scale;   // log2(e) / sqrt(r)
+    float b_g, eps;
+};
+
+template <typename T, int VPL>
+struct State {
+    static constexpr int VE = Io<T>::VE;
+    float m[VPL], l[VPL], acc[VPL][VE];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            m[v] = -INFINITY;
+            l[v] = 0.f;
+#pragma unroll
+            for (int e = 0; e < VE; ++e) acc[v][e] = 0.f;
+        }
+    }
+    // merge another partial state into this one (per vector)
+    __device__ __forceinline__ void merge(int v, float m2, float l2, const float (&a2)[VE]) {
+        const float mn = fmaxf(m[v], m2);
+        if (mn == -INFINITY) return;
+        const float c1 = exp2f(m[v] - mn), c2 = exp2f(m2 - mn);
+        l[v] = l[v] * c1 + l2 * c2;
+#pragma unroll
+        for (int e = 0; e < VE; ++e) acc[v][e] = acc[v][e] * c1 + a2[e] * c2;
+        m[v] = mn;
+    }
+};
+
+struct Lane {
+    int lane, slot, li;
+};
+
+// Runs one warp over the CSR entries [e0, e1) of a row whose query vectors are in q.
+// On return every lane holds the merged state of its feature vectors over all slots.
+template <typename T, int VPL, int U>
+__device__ __forceinline__ void warp_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
+                                           int64_t e0, int64_t e1, const Lane &ln,
+                                           State<T, VPL> &st) {
+    constexpr int VE = Io<T>::VE;
+    st.init();
+    const int per_iter = p.epw * U;
+    const uint4 *KV = static_cast<const uint4 *>(p.KV);
+    const int64_t row_vecs = 2 * static_cast<int64_t>(p.nvec);
+    for (int64_t base = e0; base < e1; base += per_iter) {
+        int32_t myc = -1;
+        if (ln.lane < per_iter && base + ln.lane < e1) myc = __ldg(p.col_idx + base + ln.lane);
+        int32_t j[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) j[u] = __shfl_sync(0xffffffffu, myc, u * p.epw + ln.slot);
+        uint4 kr[U][VPL], vr[U][VPL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const int vid = v * 32 + ln.li;
+                if (j[u] >= 0 && vid < p.nvec) {
+                    const uint4 *rowp = KV + static_cast<int64_t>(j[u]) * row_vecs;
+                    kr[u][v] = ld_gather(rowp + vid);
+                    vr[u][v] = ld_gather(rowp + p.nvec + vid);
+                } else {
+                    kr[u][v] = make_uint4(0, 0, 0, 0);
+                    vr[u][v] = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+        float s[U][VPL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                float kf[VE];
+                Io<T>::unpack(kr[u][v], kf);
+                float dot = 0.f;
+#pragma unroll
+                for (int e = 0; e < VE; ++e) dot = fmaf(q[v][e], kf[e], dot);
+                for (int o = 1; o < p.lph; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                s[u][v] = (j[u] >= 0) ? dot * p.score_scale : -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            float mx = s[0][v];
+#pragma unroll
+            for (int u = 1; u < U; ++u) mx = fmaxf(mx, s[u][v]);
+            const float mn = fmaxf(st.m[v], mx);
+            if (mn == -INFINITY) continue;
+            const float corr = exp2f(st.m[v] - mn);
+            st.l[v] *= corr;
+#pragma unroll
+            for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float pr = exp2f(s[u][v] - mn);
+                float vf[VE];
+                Io<T>::unpack(vr[u][v], vf);
+                st.l[v] += pr;
+#pragma unroll
+                for (int e = 0; e < VE; ++e) st.acc[v][e] = fmaf(pr, vf[e], st.acc[v][e]);
+            }
+            st.m[v] = mn;
+        }
+    }
+    // merge the edge slots of the warp (lanes li, li + LPE, li + 2 LPE, ...)
+    for (int o = p.lpe; o < 32; o <<= 1) {
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, st.m[v], o);
+            const float l2 = __shfl_xor_sync(0xffffffffu, st.l[v], o);
+            float a2[VE];
+#pragma unroll
+            for (int e = 0; e < VE; ++e) a2[e] = __shfl_xor_sync(0xffffffffu, st.acc[v][e], o);
+            st.merge(v, m2, l2, a2);
+        }
+    }
+}
+
+template <typename T, int VPL>
+__device__ __forceinline__ void load_q(const LocalParams &p, int64_t row, const Lane &ln,
+                                       float (&q)[VPL][Io<T>::VE]) {
+    const uint4 *Q = static_cast<const uint4 *>(p.Q) + row * p.nvec;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const int vid = v * 32 + ln.li;
+        uint4 u = vid < p.nvec ? __ldg(Q + vid) : make_uint4(0, 0, 0, 0);
+        Io<T>::unpack(u, q[v]);
+    }
+}
+
+// L = acc / l, global readout, gate and blend; stores Y[row] (slot-0 lanes).
+template <typename T, int VPL>
+__device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row,
+                                           const float (&q)[VPL][Io<T>::VE],
+                                           const State<T, VPL> &st, const Lane &ln) {
+    constexpr int VE = Io<T>::VE;
+    const float tg = __ldg(p.t + row) + p.b_g;
+    const float g = 1.f / (1.f + expf(-tg));
+    uint4 *Y = static_cast<uint4 *>(p.Y) + row * p.nvec;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const int vid = v * 32 + ln.li;
+        const bool valid = vid < p.nvec;
+        const int e0 = vid * VE;                         // first feature of this vector
+        const int h = valid ? e0 / p.r : 0;
+        const int c0 = e0 - h * p.r;                     // column inside the head
+        float ph[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) ph[e] = q[v][e] > 0.f ? q[v][e] + 1.f : expf(q[v][e]);
+        // denominator phi(q)^T z + eps
+        const float *zh = p.z + h * p.r;
+        float den = 0.f;
+        if (valid) {
+#pragma unroll
+            for (int e = 0; e < VE; ++e) den = fmaf(ph[e], __ldg(zh + c0 + e), den);
+        }
+        for (int o = 1; o < p.lph; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        // numerator phi(q)^T S[:, c0 .. c0+VE)
+        float num[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) num[e] = 0.f;
+        const int gbase = ln.lane & ~(p.lph - 1);
+        const float *Sh = p.S + static_cast<int64_t>(h) * p.r * p.r + c0;
+        for (int jj = 0; jj < p.lph; ++jj) {
+#pragma unroll
+            for (int e2 = 0; e2 < VE; ++e2) {
+                const float pq = __shfl_sync(0xffffffffu, ph[e2], gbase + jj);
+                const float4 *srow = reinterpret_cast<const float4 *>(Sh + (jj * VE + e2) * p.r);
+                if (valid) {
+#pragma unroll
+                    for (int e4 = 0; e4 < VE / 4; ++e4) {
+                        const float4 sv = __ldg(srow + e4);
+                        num[4 * e4 + 0] = fmaf(pq, sv.x, num[4 * e4 + 0]);
+                        num[4 * e4 + 1] = fmaf(pq, sv.y, num[4 * e4 + 1]);
+                        num[4 * e4 + 2] = fmaf(pq, sv.z, num[4 * e4 + 2]);
+                        num[4 * e4 + 3] = fmaf(pq, sv.w, num[4 * e4 + 3]);
+                    }
+                }
+            }
+        }
+        const float inv_den = 1.f / (den + p.eps);
+        const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
+        float y[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+            const float L = st.acc[v][e] * inv_l;
+            const float G = num[e] * inv_den;
+            y[e] = g * L + (1.f - g) * G;
+        }
+        if (valid && ln.slot == 0) Y[vid] = Io<T>::pack(y);
+    }
+}
+
+template <typename T, int VPL>
+struct BlockScratch {
+    static constexpr int VE = Io<T>::VE;
+    float m[kLocalWarps][VPL][32];
+    float l[kLocalWarps][VPL][32];
+    float acc[kLocalWarps][VPL][VE][32];
+    int flag;
+};
+
+// 8 warps split [e0, e1); warp 0 returns the merge of all warps (warp order).
+template <typename T, int VPL, int U>
+__device__ __forceinline__ void block_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
+                                            int64_t e0, int64_t e1, const Lane &ln, int warp,
+                                            BlockScratch<T, VPL> &sh, State<T, VPL> &st) {
+    constexpr int VE = Io<T>::VE;
+    const int64_t len = e1 - e0;
+    const int64_t per = ceil_div(len, kLocalWarps);
+    const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
+    warp_edges<T, VPL, U>(p, q, a, b, ln, st);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        sh.m[warp][v][ln.lane] = st.m[v];
+        sh.l[warp][v][ln.lane] = st.l[v];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) sh.acc[warp][v][e][ln.lane] = st.acc[v][e];
+    }
+    __syncthreads();
+    if (warp == 0) {
+        for (int w = 1; w < kLocalWarps; ++w) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                float a2[VE];
+#pragma unroll
+                for (int e = 0; e < VE; ++e) a2[e] = sh.acc[w][v][e][ln.lane];
+                st.merge(v, sh.m[w][v][ln.lane], sh.l[w][v][ln.lane], a2);
+            }
+        }
+    }
+}
+
+template <typename T, int VPL, int U>
+__global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(const LocalParams p) {
+    constexpr int VE = Io<T>::VE;
+    __shared__ BlockScratch<T, VPL> sh;
+    const int warp = threadIdx.x >> 5;
+    Lane ln;
+    ln.lane = threadIdx.x & 31;
+    ln.slot = ln.lane / p.lpe;
+    ln.li = ln.lane % p.lpe;
+    int64_t bid = blockIdx.x;
+    float q[VPL][VE];
+    State<T, VPL> st;
+
+    if (bid < p.n_chunks) {
+        // ---------------- chunk of a bucket-2 row ----------------
+        const int64_t c = bid;
+        const int64_t row = p.chunk_row[c];
+        const int64_t rb = p.row_ptr[row], re = p.row_ptr[row + 1];
+        const int64_t e0 = p.chunk_begin[c];
+        const int64_t e1 = std::min<int64_t>(re, e0 + p.chunk_edges);
+        const int64_t nch = ceil_div(re - rb, p.chunk_edges);
+        const int64_t first = c - (e0 - rb) / p.chunk_edges;
+        load_q<T, VPL>(p, row, ln, q);
+        block_edges<T, VPL, U>(p, q, e0, e1, ln, warp, sh, st);
+        const int64_t stride = 2 * p.H + p.D;
+        if (warp == 0) {
+            float *dst = p.part + c * stride;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const int vid = v * 32 + ln.li;
+                if (vid < p.nvec && ln.slot == 0) {
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) dst[2 * p.H + vid * VE + e] = st.acc[v][e];
+                    if ((ln.li & (p.lph - 1)) == 0) {
+                        const int h = vid * VE / p.r;
+                        dst[h] = st.m[v];
+                        dst[p.H + h] = st.l[v];
+                    }
+                }
+            }
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (ln.lane == 0) {
+                const unsigned prev = atomicAdd(p.ticket + first, 1u);
+                last = (prev == static_cast<unsigned>(nch - 1));
+                if (last) p.ticket[first] = 0u;   // ready for the next forward
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                st.init();
+                for (int64_t k = 0; k < nch; ++k) {
+                    const float *src = p.part + (first + k) * stride;
+#pragma unroll
+                    for (int v = 0; v < VPL; ++v) {
+                        const int vid = v * 32 + ln.li;
+                        const int h = vid < p.nvec ? vid * VE / p.r : 0;
+                        float a2[VE];
+#pragma unroll
+                        for (int e = 0; e < VE; ++e)
+                            a2[e] = vid < p.nvec ? __ldcg(src + 2 * p.H + vid * VE + e) : 0.f;
+                        st.merge(v, __ldcg(src + h), __ldcg(src + p.H + h), a2);
+                    }
+                }
+                finish_row<T, VPL>(p, row, q, st, ln);
+            }
+        }
+        return;
+    }
+    bid -= p.n_chunks;
+    if (bid < p.n_cta) {
+        // ---------------- bucket-1 row: one block ----------------
+        const int64_t row = p.cta_rows[bid];
+        load_q<T, VPL>(p, row, ln, q);
+        block_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
+        if (warp == 0) finish_row<T, VPL>(p, row, q, st, ln);
+        return;
+    }
+    bid -= p.n_cta;
+    // ---------------- bucket-0 rows: one warp each ----------------
+    const int64_t idx = bid * kLocalWarps + warp;
+    if (idx >= p.n_warp) return;
+    const int64_t row = p.warp_rows[idx];
+    load_q<T, VPL>(p, row, ln, q);
+    warp_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, st);
+    finish_row<T, VPL>(p, row, q, st, ln);
+}
+
+template <typename T, int VPL, int U>
+glga_status launch_local(Ctx *c, const LocalParams &p, cudaStream_t s) {
+    const int64_t blocks = p.n_chunks + p.n_cta + p.warp_blocks;
+    if (blocks == 0) return GLGA_OK;
+    local_kernel<T, VPL, U><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
+    GLGA_CUDA(cudaGetLastError());
+    c->launches += 1;
+    return GLGA_OK;
+}
+
+}  // namespace
+
+glga_status local_setup(Ctx *c) {
+    const int64_t nc = c->nb[3];
+    glga_status st = GLGA_OK;
+    if (nc > 0) {
+        st = dev_alloc(c, reinterpret_cast<void **>(&c->chunk_part),
+                       static_cast<size_t>(nc) * (2 * c->H + c->D) * sizeof(float));
+        if (st == GLGA_OK)
+            st = dev_alloc(c, reinterpret_cast<void **>(&c->chunk_ticket), nc * sizeof(unsigned));
+        if (st == GLGA_OK) {
+            cudaError_t e = cudaMemset(c->chunk_ticket, 0, nc * sizeof(unsigned));
+            if (e != cudaSuccess) return cuda_fail(e, "ticket init");
+        }
+    }
+    return st;
+}
+
+glga_status local_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
+    LocalParams p;
+    p.row_ptr = c->row_ptr;
+    p.col_idx = c->col_idx;
+    p.warp_rows = c->warp_rows;
+    p.cta_rows = c->cta_rows;
+    p.chunk_row = c->chunk_row;
+    p.chunk_begin = c->chunk_begin;
+    p.n_warp = c->nb[0];
+    p.n_cta = c->nb[1];
+    p.n_chunks = c->nb[3];
+    p.warp_blocks = ceil_div(p.n_warp, kLocalWarps);
+    p.chunk_edges = c->opts.chunk_edges;
+    p.Q = c->Q;
+    p.KV = c->KV;
+    p.t = c->t;
+    p.S = c->Sz;
+    p.z = c->Sz + static_cast<int64_t>(c->H) * c->r * c->r;
+    p.part = c->chunk_part;
+    p.ticket = c->chunk_ticket;
+    p.Y = Y;
+    p.D = c->D;
+    p.r = c->r;
+    p.H = c->H;
+    const int VE = 16 / c->elem;
+    p.nvec = c->D / VE;
+    int lpe = 1;
+    while (lpe < p.nvec && lpe < 32) lpe <<= 1;
+    p.lpe = lpe;
+    p.epw = 32 / lpe;
+    p.lph = c->r / VE;
+    p.score_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->r)));
+    p.b_g = b_g;
+    p.eps = eps;
+    const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
+    if (c->io == GLGA_F32) {
+        if (vpl == 1) return launch_local<float, 1, 4>(c, p, s);
+        if (vpl == 2) return launch_local<float, 2, 2>(c, p, s);
+        if (vpl <= 4) return launch_local<float, 4, 1>(c, p, s);
+    } else {
+        if (vpl == 1) return launch_local<__nv_bfloat16, 1, 4>(c, p, s);
+        if (vpl == 2) return launch_local<__nv_bfloat16, 2, 2>(c, p, s);
+        if (vpl <= 4) return launch_local<__nv_bfloat16, 4, 1>(c, p, s);
+    }
+    set_error("row width too large for the local kernel");
+    return GLGA_ERR_UNSUPPORTED;
+}
+
+}  // namespace glga

@@ -1,0 +1,484 @@
+// projection.cu -- fused Q/K/V/gate projection on the tcgen05 tensor cores.
+//
+// One GEMM computes [Q | K | V | t] = X [W_Q | W_K | W_V | w_g] (method page "Gated
+// Local-Global Graph Attention", Key formulas: q = x W_Q, k = x W_K, v = x W_V and the
+// gate logit x w_g).  The weights are packed once per forward into one K-major operand
+// Wt [rows][dp] (row c = output column c; rows past 3D+1 are zero).  Output columns
+// [0, D) go to Q, [D, 3D) to KV (k_j | v_j per row, the layout the local kernel
+// gathers), column 3D to the float32 gate logit t.
+//
+// Kernel shape: 128 x BN tiles (BN <= 256, one MMA per 32-byte K step), K tiles of 128
+// bytes per row loaded by TMA with the 128-byte swizzle, an mbarrier ring of `stages`
+// buffers, one elected thread issuing tcgen05.mma into a TMEM accumulator, and all four
+// warps draining TMEM (tcgen05.ld 32x32b) into global memory.
+//
+// float32 I/O uses kind::tf32 with a 3-term split: every operand x is stored as
+// hi = tf32(x) and lo = tf32(x - hi) and the accumulator receives hi*hi + hi*lo + lo*hi,
+// which keeps ~2^-21 relative accuracy (plain tf32 would give ~2^-11).
+#include <algorithm>
+#include <cstdio>
+
+#include "glga_internal.cuh"
+
+namespace glga {
+
+namespace {
+constexpr int kBM = 128;
+constexpr int kRowBytes = 128;            // bytes of K per smem row (one swizzle span)
+constexpr int kMaxStages = 4;
+constexpr int kGemmThreads = 128;
+
+struct GemmParams {
+    int64_t M;
+    int32_t nk;          // K tiles
+    int32_t BN;          // columns per CTA (multiple of 16, <= 256)
+    int32_t stages;
+    int32_t tmem_cols;
+    int32_t D;
+    uint32_t a_bytes, b_bytes, stage_bytes;
+    void *Q;
+    void *KV;
+    float *t;
+    unsigned *flag;
+};
+
+template <typename T>
+__device__ __forceinline__ void store_vec32(T *dst, const uint32_t (&v)[32]);
+
+template <>
+__device__ __forceinline__ void store_vec32<float>(float *dst, const uint32_t (&v)[32]) {
+    float4 *o = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+template <>
+__device__ __forceinline__ void store_vec32<__nv_bfloat16>(__nv_bfloat16 *dst,
+                                                           const uint32_t (&v)[32]) {
+    uint4 *o = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 q;
+        q.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+        q.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+        q.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+        q.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+        o[i] = q;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Routes 32 consecutive accumulator columns [gc0, gc0+32) of one row to Q / KV / t.
+template <typename T>
+__device__ __forceinline__ void store_row_cols(const GemmParams &p, int64_t row, int gc0,
+                                               const uint32_t (&v)[32]) {
+    const int D = p.D;
+    T *Q = static_cast<T *>(p.Q);
+    T *KV = static_cast<T *>(p.KV);
+    if (gc0 + 32 <= D) {
+        store_vec32<T>(Q + row * D + gc0, v);
+    } else if (gc0 >= D && gc0 + 32 <= 3 * D) {
+        store_vec32<T>(KV + row * 2 * D + (gc0 - D), v);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int gc = gc0 + j;
+            const float x = __uint_as_float(v[j]);
+            if (gc < D)
+                Q[row * D + gc] = from_f32<T>(x);
+            else if (gc < 3 * D)
+                KV[row * 2 * D + (gc - D)] = from_f32<T>(x);
+            else if (gc == 3 * D)
+                p.t[row] = x;
+        }
+    }
+}
+
+// SPLIT = 1: bf16 operands, one MMA per K step.  SPLIT = 3: tf32 hi/lo planes.
+template <int SPLIT, typename T>
+__global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
+    const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+    GemmParams p) {
+    constexpr int kPlanes = SPLIT == 3 ? 2 : 1;
+    constexpr int kPairs = SPLIT == 3 ? 3 : 1;
+    constexpr uint32_t kFmt = SPLIT == 3 ? 2u : 1u;
+
+    extern __shared__ uint8_t dsmem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_base_sh;
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * p.BN;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&done_bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA0);
+        tma_prefetch_desc(&tmB0);
+        if (kPlanes == 2) {
+            tma_prefetch_desc(&tmA1);
+            tma_prefetch_desc(&tmB1);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, static_cast<uint32_t>(p.tmem_cols));
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer ----------------
+        int issued = 0;
+        bool ok = true;
+        for (int kb = 0; kb < p.nk; ++kb) {
+            const int s = kb % p.stages;
+            const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
+            if (kb >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+                ok = false;
+                break;
+            }
+            uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+            mbar_arrive_expect_tx(&full_bar[s], p.stage_bytes);
+            const int kx = kb * (kRowBytes / static_cast<int>(sizeof(T)));
+            tma_load_2d(st, &tmA0, &full_bar[s], kx, static_cast<int32_t>(m0));
+            if (kPlanes == 2) tma_load_2d(st + p.a_bytes, &tmA1, &full_bar[s], kx, static_cast<int32_t>(m0));
+            uint8_t *bst = st + kPlanes * p.a_bytes;
+            tma_load_2d(bst, &tmB0, &full_bar[s], kx, n0);
+            if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kx, n0);
+            ++issued;
+        }
+        if (!ok) {
+            atomicOr(p.flag, kDevErrTimeout);
+            // let the copies already in flight land before the block can exit
+            for (int kb = std::max(0, issued - p.stages); kb < issued; ++kb)
+                mbar_wait_bounded(&full_bar[kb % p.stages], static_cast<uint32_t>(kb / p.stages) & 1u);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- MMA issuer ----------------
+        const uint32_t idesc = instr_desc(kBM, p.BN, kFmt, false, false);
+        bool ok = true;
+        for (int kb = 0; kb < p.nk; ++kb) {
+            const int s = kb % p.stages;
+            const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
+            if (!mbar_wait_bounded(&full_bar[s], ph)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
+            const uint32_t b_addr = a_addr + kPlanes * p.a_bytes;
+#pragma unroll
+            for (int k = 0; k < kRowBytes / 32; ++k) {
+#pragma unroll
+                for (int pr = 0; pr < kPairs; ++pr) {
+                    const uint32_t ap = (pr == 2) ? 1u : 0u;   // (hi,hi) (hi,lo) (lo,hi)
+                    const uint32_t bp = (pr == 1) ? 1u : 0u;
+                    const uint64_t ad = smem_desc(a_addr + ap * p.a_bytes + k * 32, 16, 1024, 2);
+                    const uint64_t bd = smem_desc(b_addr + bp * p.b_bytes + k * 32, 16, 1024, 2);
+                    const uint32_t acc = (kb | k | pr) != 0;
+                    if (SPLIT == 3)
+                        umma_tf32(tmem, ad, bd, idesc, acc);
+                    else
+                        umma_bf16(tmem, ad, bd, idesc, acc);
+                }
+            }
+            umma_commit(&empty_bar[s]);
+        }
+        if (!ok) atomicOr(p.flag, kDevErrTimeout);
+        umma_commit(&done_bar);   // arrives once every MMA issued above has completed
+    }
+    __syncwarp();
+
+    // ---------------- epilogue: TMEM -> registers -> Q / KV / t ----------------
+    const bool done = mbar_wait_bounded(&done_bar, 0);
+    tc_fence_after();
+    if (!done) {
+        if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
+    } else {
+        const int64_t row = m0 + warp * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        for (int c0 = 0; c0 < p.BN; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
+            tmem_ld_wait();
+            if (row < p.M) store_row_cols<T>(p, row, n0 + c0, v);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// operand preparation
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float ld_f32(const T *p);
+template <>
+__device__ __forceinline__ float ld_f32<float>(const float *p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    return __bfloat162float(*p);
+}
+
+// Wt[c][k] (k < dp, c < rows): the packed K-major weight operand.
+template <int SPLIT, typename T>
+__global__ void pack_weights_kernel(const T *__restrict__ WQ, const T *__restrict__ WK,
+                                    const T *__restrict__ WV, const T *__restrict__ wg, int d,
+                                    int D, int dp, int rows, T *__restrict__ Wt) {
+    const int64_t total = static_cast<int64_t>(rows) * dp;
+    const int64_t plane = total;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(idx / dp);
+        const int k = static_cast<int>(idx % dp);
+        float v = 0.f;
+        if (k < d) {
+            if (c < D)
+                v = ld_f32<T>(WQ + static_cast<int64_t>(k) * D + c);
+            else if (c < 2 * D)
+                v = ld_f32<T>(WK + static_cast<int64_t>(k) * D + (c - D));
+            else if (c < 3 * D)
+                v = ld_f32<T>(WV + static_cast<int64_t>(k) * D + (c - 2 * D));
+            else if (c == 3 * D)
+                v = ld_f32<T>(wg + k);
+        }
+        if (SPLIT == 3) {
+            const float hi = to_tf32(v);
+            Wt[idx] = from_f32<T>(hi);
+            Wt[plane + idx] = from_f32<T>(to_tf32(v - hi));
+        } else {
+            Wt[idx] = from_f32<T>(v);
+        }
+    }
+}
+
+// Xp[i][k] (k < dp): zero-padded copy of X (and its tf32 hi/lo split for SPLIT = 3).
+template <int SPLIT, typename T>
+__global__ void prep_x_kernel(const T *__restrict__ X, int64_t N, int d, int dp,
+                              T *__restrict__ Xp) {
+    const int64_t total = N * dp;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t i = idx / dp;
+        const int k = static_cast<int>(idx % dp);
+        const float v = k < d ? ld_f32<T>(X + i * d + k) : 0.f;
+        if (SPLIT == 3) {
+            const float hi = to_tf32(v);
+            Xp[idx] = from_f32<T>(hi);
+            Xp[total + idx] = from_f32<T>(to_tf32(v - hi));
+        } else {
+            Xp[idx] = from_f32<T>(v);
+        }
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+template <int SPLIT, typename T>
+glga_status launch_gemm(Ctx *c, cudaStream_t s) {
+    GemmParams p;
+    p.M = c->N;
+    p.nk = c->dp / (kRowBytes / c->elem);
+    p.BN = c->BN;
+    p.stages = c->stages;
+    p.tmem_cols = c->tmem_cols;
+    p.D = c->D;
+    const int planes = SPLIT == 3 ? 2 : 1;
+    p.a_bytes = kBM * kRowBytes;
+    p.b_bytes = static_cast<uint32_t>(c->BN) * kRowBytes;
+    p.stage_bytes = planes * (p.a_bytes + p.b_bytes);
+    p.Q = c->Q;
+    p.KV = c->KV;
+    p.t = c->t;
+    p.flag = c->dev_flag;
+    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + 1024;
+    auto kern = proj_gemm_kernel<SPLIT, T>;
+    GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem)));
+    dim3 grid(static_cast<unsigned>(c->n_tiles), static_cast<unsigned>(ceil_div(c->N, kBM)));
+    const CUtensorMap &a1 = planes == 2 ? c->tmA[1].map : c->tmA[0].map;
+    const CUtensorMap &b1 = planes == 2 ? c->tmB[1].map : c->tmB[0].map;
+    kern<<<grid, kGemmThreads, smem, s>>>(c->tmA[0].map, a1, c->tmB[0].map, b1, p);
+    GLGA_CUDA(cudaGetLastError());
+    c->launches += 1;
+    return GLGA_OK;
+}
+
+}  // namespace
+
+glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
+                           uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                           uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        set_error("cuTensorMapEncodeTiled unavailable from the driver");
+        return GLGA_ERR_CUDA;
+    }
+    if ((reinterpret_cast<uintptr_t>(base) & 15u) || (row_bytes & 15u)) {
+        set_error("tensor map base/stride not 16-byte aligned");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) dims=%llu,%llu box=%u,%u", static_cast<int>(r),
+                  static_cast<unsigned long long>(inner), static_cast<unsigned long long>(outer),
+                  box_inner, box_outer);
+        return GLGA_ERR_CUDA;
+    }
+    return GLGA_OK;
+}
+
+glga_status projection_setup(Ctx *c) {
+    c->split = (c->io == GLGA_F32) ? 3 : 1;
+    const int kt = kRowBytes / c->elem;                  // K elements per tile row
+    c->dp = static_cast<int32_t>(ceil_div(c->d, kt) * kt);
+    const int Dp = 3 * c->D + 1;
+    c->n_tiles = static_cast<int32_t>(ceil_div(Dp, 256));
+    c->BN = static_cast<int32_t>(ceil_div(ceil_div(Dp, c->n_tiles), 16) * 16);
+    c->Dp = c->n_tiles * c->BN;
+    int tc = 32;
+    while (tc < c->BN) tc <<= 1;
+    c->tmem_cols = tc;
+    const int planes = c->split == 3 ? 2 : 1;
+    const uint32_t stage_bytes = planes * (kBM * kRowBytes + c->BN * kRowBytes);
+    const int nk = c->dp / kt;
+    // two CTAs per SM for bf16 (epilogue of one overlaps the loads of the other)
+    const uint32_t budget = (c->split == 3) ? 200u * 1024u : 110u * 1024u;
+    int st = static_cast<int>(budget / stage_bytes);
+    st = std::max(1, std::min(st, kMaxStages));
+    c->stages = std::min(st, std::max(nk, 1));
+
+    const size_t wt_bytes = static_cast<size_t>(planes) * c->Dp * c->dp * c->elem;
+    glga_status r = dev_alloc(c, &c->Wt, wt_bytes);
+    if (r != GLGA_OK) return r;
+    const CUtensorMapDataType dt =
+        c->io == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    for (int pl = 0; pl < planes; ++pl) {
+        const uint8_t *base = static_cast<const uint8_t *>(c->Wt) +
+                              static_cast<size_t>(pl) * c->Dp * c->dp * c->elem;
+        r = encode_tmap_2d(&c->tmB[pl].map, dt, base, c->dp, c->Dp,
+                           static_cast<uint64_t>(c->dp) * c->elem, kt, c->BN);
+        if (r != GLGA_OK) return r;
+        c->tmB[pl].valid = true;
+    }
+    // The A operand is read from the caller's X when it is bf16 with 16-byte rows;
+    // otherwise from a padded (and, for fp32, split) copy.
+    c->x_direct = (c->split == 1) && ((static_cast<int64_t>(c->d) * c->elem) % 16 == 0);
+    if (!c->x_direct && c->N > 0) {
+        const size_t xp_bytes = static_cast<size_t>(planes) * c->N * c->dp * c->elem;
+        r = dev_alloc(c, &c->Xp, xp_bytes);
+        if (r != GLGA_OK) return r;
+        for (int pl = 0; pl < planes; ++pl) {
+            const uint8_t *base = static_cast<const uint8_t *>(c->Xp) +
+                                  static_cast<size_t>(pl) * c->N * c->dp * c->elem;
+            r = encode_tmap_2d(&c->tmA[pl].map, dt, base, c->dp, c->N,
+                               static_cast<uint64_t>(c->dp) * c->elem, kt, kBM);
+            if (r != GLGA_OK) return r;
+            c->tmA[pl].valid = true;
+        }
+    }
+    return GLGA_OK;
+}
+
+glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV,
+                           const void *wg, cudaStream_t s, bool time_prep) {
+    (void)time_prep;
+    const int64_t wt_total = static_cast<int64_t>(c->Dp) * c->dp;
+    const unsigned wblocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(wt_total, 256), 2048));
+    if (c->io == GLGA_F32) {
+        pack_weights_kernel<3, float><<<wblocks, 256, 0, s>>>(
+            static_cast<const float *>(WQ), static_cast<const float *>(WK),
+            static_cast<const float *>(WV), static_cast<const float *>(wg), c->d, c->D, c->dp,
+            c->Dp, static_cast<float *>(c->Wt));
+    } else {
+        pack_weights_kernel<1, __nv_bfloat16><<<wblocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(WQ), static_cast<const __nv_bfloat16 *>(WK),
+            static_cast<const __nv_bfloat16 *>(WV), static_cast<const __nv_bfloat16 *>(wg), c->d,
+            c->D, c->dp, c->Dp, static_cast<__nv_bfloat16 *>(c->Wt));
+    }
+    GLGA_CUDA(cudaGetLastError());
+    c->launches += 1;
+    if (c->N == 0) return GLGA_OK;
+    const CUtensorMapDataType dt =
+        c->io == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (c->x_direct) {
+        glga_status r = encode_tmap_2d(&c->tmA[0].map, dt, X, c->d, c->N,
+                                       static_cast<uint64_t>(c->d) * c->elem,
+                                       kRowBytes / c->elem, kBM);
+        if (r != GLGA_OK) return r;
+        c->tmA[0].valid = true;
+    } else {
+        const int64_t total = c->N * c->dp;
+        const unsigned xblocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 8192));
+        if (c->io == GLGA_F32)
+            prep_x_kernel<3, float><<<xblocks, 256, 0, s>>>(static_cast<const float *>(X), c->N,
+                                                            c->d, c->dp, static_cast<float *>(c->Xp));
+        else
+            prep_x_kernel<1, __nv_bfloat16><<<xblocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16 *>(X), c->N, c->d, c->dp,
+                static_cast<__nv_bfloat16 *>(c->Xp));
+        GLGA_CUDA(cudaGetLastError());
+        c->launches += 1;
+    }
+    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageGemm], s));
+    if (c->io == GLGA_F32) return launch_gemm<3, float>(c, s);
+    return launch_gemm<1, __nv_bfloat16>(c, s);
+}
+
+}  // namespace glga

@@ -1,0 +1,222 @@
+"""Python binding of libglga (the C ABI in include/glga.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+PyTorch supplies device memory (tensor.data_ptr()) and streams
+(torch.cuda.current_stream().cuda_stream).  The binding raises if libglga.so is missing;
+there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libglga.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "glga.h")
+
+GLGA_F32, GLGA_BF16 = 0, 1
+STATUS = {0: "GLGA_OK", 1: "GLGA_ERR_INVALID_ARG", 2: "GLGA_ERR_BAD_GRAPH",
+          3: "GLGA_ERR_UNSUPPORTED", 4: "GLGA_ERR_OOM", 5: "GLGA_ERR_CUDA",
+          6: "GLGA_ERR_TIMEOUT", 7: "GLGA_ERR_DEVICE"}
+STAGES = ("prep", "gemm", "stats", "local", "forward")
+
+
+class GLGAError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("warp_max_degree", ctypes.c_int32), ("chunk_edges", ctypes.c_int32)]
+
+
+_lib = None
+_vp, _i64, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+
+
+def declared_symbols() -> list[str]:
+    """Names of the entry points declared in include/glga.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"GLGA_API\s+[\w\s\*]*?\b(glga_\w+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_graph_attention_tcgen05_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "glga_default_options": ([ctypes.POINTER(Options)], _i32),
+        "glga_create": ([ctypes.POINTER(_vp), _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
+                         ctypes.POINTER(Options), _vp], _i32),
+        "glga_forward": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _vp], _i32),
+        "glga_destroy": ([_vp], _i32),
+        "glga_csr_from_coo": ([_i64, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
+        "glga_bucket_counts": ([_vp, ctypes.POINTER(_i64)], _i32),
+        "glga_get_buckets": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+        "glga_get_intermediates": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+        "glga_set_timing": ([_vp, ctypes.c_int], _i32),
+        "glga_stage_times": ([_vp, ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)], _i32),
+        "glga_workspace_bytes": ([_vp, ctypes.POINTER(_i64)], _i32),
+        "glga_kernel_launches": ([_vp, ctypes.POINTER(_i64)], _i32),
+        "glga_last_device_error": ([_vp, _vp], _i32),
+        "glga_status_string": ([_i32], ctypes.c_char_p),
+        "glga_last_error_message": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        msg = lib().glga_last_error_message().decode(errors="replace")
+        raise GLGAError(status, where, msg)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def torch_dtype(io: str) -> torch.dtype:
+    return {"f32": torch.float32, "bf16": torch.bfloat16}[io]
+
+
+def default_options() -> Options:
+    o = Options()
+    _check(lib().glga_default_options(ctypes.byref(o)), "glga_default_options")
+    return o
+
+
+def csr_from_coo(N: int, src: torch.Tensor, dst: torch.Tensor, stream=None):
+    """Target-grouped CSR (rows = targets, ascending sources) built on the GPU."""
+    assert src.is_cuda and dst.is_cuda and src.dtype == torch.int32 and dst.dtype == torch.int32
+    src, dst = src.contiguous(), dst.contiguous()
+    E = src.numel()
+    row_ptr = torch.empty(N + 1, dtype=torch.int32, device=src.device)
+    col_idx = torch.empty(max(E, 1), dtype=torch.int32, device=src.device)
+    _check(lib().glga_csr_from_coo(N, E, _ptr(src), _ptr(dst), _ptr(row_ptr), _ptr(col_idx),
+                                   _stream(stream)), "glga_csr_from_coo")
+    return row_ptr, col_idx[:E]
+
+
+class Layer:
+    """One gated local-global graph-attention layer bound to a fixed graph.
+
+    `row_ptr`/`col_idx` are CUDA int32 tensors (target-grouped CSR).  `io` is "f32" or
+    "bf16": the element type of X, the weights and Y."""
+
+    def __init__(self, N, d, H, r, io, row_ptr, col_idx, options: Options | None = None,
+                 stream=None):
+        self.N, self.d, self.H, self.r, self.io = int(N), int(d), int(H), int(r), io
+        self.D = self.H * self.r
+        self.dtype = torch_dtype(io)
+        self.device = row_ptr.device
+        assert row_ptr.is_cuda and row_ptr.dtype == torch.int32 and row_ptr.numel() == N + 1
+        assert col_idx.dtype == torch.int32
+        self.E = int(col_idx.numel())
+        h = ctypes.c_void_p()
+        opt = ctypes.byref(options) if options is not None else None
+        _check(lib().glga_create(ctypes.byref(h), self.N, self.d, self.H, self.r,
+                                 GLGA_F32 if io == "f32" else GLGA_BF16,
+                                 _ptr(row_ptr.contiguous()),
+                                 _ptr(col_idx.contiguous()) if self.E else None, self.E, opt,
+                                 _stream(stream)), "glga_create")
+        self._h = h
+
+    # -- forward ---------------------------------------------------------------------
+    def forward(self, X, W_Q, W_K, W_V, w_g, b_g: float, eps: float, Y=None, stream=None):
+        for t in (X, W_Q, W_K, W_V, w_g):
+            assert t.dtype == self.dtype and t.is_cuda and t.is_contiguous()
+        assert X.shape == (self.N, self.d) and w_g.numel() == self.d
+        if Y is None:
+            Y = torch.empty(self.N, self.D, dtype=self.dtype, device=X.device)
+        _check(lib().glga_forward(self._h, _ptr(X), _ptr(W_Q), _ptr(W_K), _ptr(W_V), _ptr(w_g),
+                                  float(b_g), float(eps), _ptr(Y), _stream(stream)),
+               "glga_forward")
+        return Y
+
+    __call__ = forward
+
+    # -- introspection ---------------------------------------------------------------
+    def bucket_counts(self):
+        c = (_i64 * 4)()
+        _check(lib().glga_bucket_counts(self._h, c), "glga_bucket_counts")
+        return [int(x) for x in c]
+
+    def buckets(self, stream=None) -> dict:
+        n = self.bucket_counts()
+        out = {k: torch.empty(max(m, 1), dtype=torch.int32, device=self.device)
+               for k, m in zip(("warp_rows", "cta_rows", "split_rows", "chunk_row", "chunk_begin"),
+                               (n[0], n[1], n[2], n[3], n[3]))}
+        _check(lib().glga_get_buckets(self._h, *(_ptr(out[k]) for k in
+                                                 ("warp_rows", "cta_rows", "split_rows",
+                                                  "chunk_row", "chunk_begin")),
+                                      _stream(stream)), "glga_get_buckets")
+        sizes = {"warp_rows": n[0], "cta_rows": n[1], "split_rows": n[2], "chunk_row": n[3],
+                 "chunk_begin": n[3]}
+        return {k: v[: sizes[k]] for k, v in out.items()}
+
+    def intermediates(self, stream=None) -> dict:
+        dev = self.device
+        out = {"Q": torch.empty(self.N, self.D, dtype=self.dtype, device=dev),
+               "K": torch.empty(self.N, self.D, dtype=self.dtype, device=dev),
+               "V": torch.empty(self.N, self.D, dtype=self.dtype, device=dev),
+               "t": torch.empty(self.N, dtype=torch.float32, device=dev),
+               "S": torch.empty(self.H, self.r, self.r, dtype=torch.float32, device=dev),
+               "z": torch.empty(self.H, self.r, dtype=torch.float32, device=dev)}
+        _check(lib().glga_get_intermediates(self._h, *(_ptr(out[k]) for k in ("Q", "K", "V", "t", "S", "z")),
+                                            _stream(stream)), "glga_get_intermediates")
+        return out
+
+    def set_timing(self, enable: bool):
+        _check(lib().glga_set_timing(self._h, 1 if enable else 0), "glga_set_timing")
+
+    def stage_times(self) -> dict:
+        ms = (ctypes.c_float * 5)()
+        n = _i32()
+        _check(lib().glga_stage_times(self._h, ms, 5, ctypes.byref(n)), "glga_stage_times")
+        return {STAGES[i]: float(ms[i]) for i in range(n.value)}
+
+    def workspace_bytes(self) -> int:
+        b = _i64()
+        _check(lib().glga_workspace_bytes(self._h, ctypes.byref(b)), "glga_workspace_bytes")
+        return int(b.value)
+
+    def kernel_launches(self) -> int:
+        n = _i64()
+        _check(lib().glga_kernel_launches(self._h, ctypes.byref(n)), "glga_kernel_launches")
+        return int(n.value)
+
+    def last_device_error(self, stream=None) -> int:
+        return int(lib().glga_last_device_error(self._h, _stream(stream)))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().glga_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,66 @@
+"""CPU-side checks of the C ABI: the library loads, exports every entry point that
+include/glga.h declares, and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+
+import pytest
+
+from sparse_graph_attention_tcgen05_b200 import glga
+
+
+def test_library_exports_every_declared_symbol():
+    names = glga.declared_symbols()
+    assert "glga_create" in names and "glga_forward" in names and "glga_destroy" in names
+    L = glga.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert len(names) >= 15
+
+
+def test_status_strings_and_defaults():
+    L = glga.lib()
+    for s in range(8):
+        assert L.glga_status_string(s)
+    assert L.glga_status_string(99) == b"unknown status"
+    o = glga.default_options()
+    assert 0 <= o.warp_max_degree <= o.chunk_edges and o.chunk_edges >= 1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(r=24), 3),                 # r outside {8, 16, 32, 64, 128}
+    (dict(r=12), 3),
+    (dict(H=0), 1),
+    (dict(d=0), 1),
+    (dict(N=-1), 1),
+    (dict(H=17, r=128, io=1), 3),    # row width 4352 bytes > 2048
+    (dict(io=7), 1),
+])
+def test_create_rejects_bad_shapes_before_any_device_work(kw, status):
+    args = dict(N=4, d=8, H=1, r=8, io=0)
+    args.update(kw)
+    h = ctypes.c_void_p()
+    st = glga.lib().glga_create(ctypes.byref(h), args["N"], args["d"], args["H"], args["r"],
+                                args["io"], 16, 16, 0, None, None)
+    assert st == status
+    assert h.value is None
+    assert glga.lib().glga_last_error_message()
+
+
+def test_create_rejects_bad_options():
+    h = ctypes.c_void_p()
+    o = glga.Options(64, 32)             # warp_max_degree > chunk_edges
+    assert glga.lib().glga_create(ctypes.byref(h), 4, 8, 1, 8, 0, 16, 16, 0, ctypes.byref(o), None) == 1
+    o = glga.Options(0, 0)
+    assert glga.lib().glga_create(ctypes.byref(h), 4, 8, 1, 8, 0, 16, 16, 0, ctypes.byref(o), None) == 1
+
+
+def test_null_arguments():
+    L = glga.lib()
+    assert L.glga_create(None, 4, 8, 1, 8, 0, 16, 16, 0, None, None) == 1
+    assert L.glga_forward(None, 16, 16, 16, 16, 16, 0.0, 1e-6, 16, None) == 1
+    assert L.glga_destroy(None) == 0
+    assert L.glga_csr_from_coo(-1, 0, None, None, None, None, None) == 1
+    assert L.glga_csr_from_coo(4, 3, None, None, 16, 16, None) == 1
+    n = ctypes.c_int64()
+    assert L.glga_kernel_launches(None, ctypes.byref(n)) == 1
+    assert L.glga_workspace_bytes(None, ctypes.byref(n)) == 1
+    assert L.glga_default_options(None) == 1
