@@ -84,21 +84,26 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 }
 
 // Routes 32 consecutive accumulator columns [gc0, gc0+32) of one row to Q / KV / t.
+// Columns at or past n_end belong to the next column tile (or are padding) and are
+// skipped: TMEM past the tile's width holds no MMA result.
 template <typename T>
 __device__ __forceinline__ void store_row_cols(const GemmParams &p, int64_t row, int gc0,
-                                               const uint32_t (&v)[32]) {
+                                               int n_end, const uint32_t (&v)[32]) {
     const int D = p.D;
     T *Q = static_cast<T *>(p.Q);
     T *KV = static_cast<T *>(p.KV);
-    if (gc0 + 32 <= D) {
+    const bool whole = gc0 + 32 <= n_end;
+    if (whole && gc0 + 32 <= D) {
         store_vec32<T>(Q + row * D + gc0, v);
-    } else if (gc0 >= D && gc0 + 32 <= 3 * D) {
+    } else if (whole && gc0 >= D && gc0 + 32 <= 3 * D) {
         store_vec32<T>(KV + row * 2 * D + (gc0 - D), v);
     } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int gc = gc0 + j;
             const float x = __uint_as_float(v[j]);
+            if (gc >= n_end)
+                continue;
             if (gc < D)
                 Q[row * D + gc] = from_f32<T>(x);
             else if (gc < 3 * D)
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
             uint32_t v[32];
             tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
             tmem_ld_wait();
-            if (row < p.M) store_row_cols<T>(p, row, n0 + c0, v);
+            if (row < p.M) store_row_cols<T>(p, row, n0 + c0, n0 + p.BN, v);
         }
     }
     tc_fence_before();

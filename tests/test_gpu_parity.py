@@ -293,3 +293,23 @@ def test_workspace_is_linear_in_graph_size():
     assert b <= 2 * linear, (b, linear)
     assert b < w.E * w.D * s            # nothing proportional to E * r
     layer.close()
+
+
+@pytest.mark.parametrize("N,d,H,r,io", [(700, 128, 4, 32, "bf16"), (300, 512, 8, 64, "bf16"),
+                                        (517, 256, 8, 32, "bf16"), (260, 1433, 8, 8, "f32"),
+                                        (200, 13, 2, 16, "bf16"), (333, 40, 3, 16, "f32")])
+def test_projection_outputs_every_column(N, d, H, r, io):
+    """Q, K, V and the gate logit of the tcgen05 GEMM against the oracle's projections, all
+    rows and columns (several column tiles; tile widths not multiples of 32)."""
+    src = np.arange(N, dtype=np.int32)
+    w = make_custom(N, d, H, r, src, src, io=io, seed=N)
+    out = run_gpu(w, keep_layer=True)
+    inter = {k: v.float().cpu().numpy() for k, v in out["layer"].intermediates().items()}
+    torch.cuda.synchronize()
+    tol = 1e-5 if io == "f32" else 8e-3
+    for key, W in (("Q", w.W_Q), ("K", w.W_K), ("V", w.W_V)):
+        ref = oracle.project(w.X, W)
+        np.testing.assert_allclose(inter[key], ref, rtol=0, atol=tol * np.abs(ref).max(), err_msg=key)
+    ref_t = oracle.gate_logit(w.X, w.w_g)
+    np.testing.assert_allclose(inter["t"], ref_t, rtol=0, atol=1e-5 * np.abs(ref_t).max())
+    out["layer"].close()
