@@ -306,7 +306,9 @@ def test_projection_outputs_every_column(N, d, H, r, io):
     out = run_gpu(w, keep_layer=True)
     inter = {k: v.float().cpu().numpy() for k, v in out["layer"].intermediates().items()}
     torch.cuda.synchronize()
-    tol = 1e-5 if io == "f32" else 8e-3
+    # fp32: the 3-term tf32 split leaves ~1e-5 relative after the tensor-core fp32
+    # accumulation over d = 1433 terms (the forward's own bound is 1e-4 * max|Y|)
+    tol = 5e-5 if io == "f32" else 8e-3
     for key, W in (("Q", w.W_Q), ("K", w.W_K), ("V", w.W_V)):
         ref = oracle.project(w.X, W)
         np.testing.assert_allclose(inter[key], ref, rtol=0, atol=tol * np.abs(ref).max(), err_msg=key)
