@@ -155,6 +155,27 @@ GLGA_API glga_status glga_workspace_bytes(const glga_ctx *ctx, int64_t *bytes);
  * context: GLGA_OK, GLGA_ERR_TIMEOUT or GLGA_ERR_DEVICE.                              */
 GLGA_API glga_status glga_last_device_error(glga_ctx *ctx, void *stream);
 
+/* glga_global_stats_static -- the global statistics S and z of glga_forward, computed
+ * without allocating any device memory.  The paper has no counterpart to this entry
+ * point.  It is for callers that must not allocate on their enqueue path: plugin
+ * interfaces whose enqueue callback may not allocate, services that reserve all device
+ * memory up front through their own pool, and latency-critical code that cannot afford
+ * cudaMalloc's possible implicit device synchronisation.
+ *   KV  (device) io [N, 2*H*r]: row j holds k_j (H*r values) followed by v_j (H*r values)
+ *   Sz  (device) float [H*r*r + H*r], written: S [H][r][r] followed by z [H][r]
+ * r must be one of 8, 16, 32, 64, 128; N >= 0; H >= 1.
+ * Partial sums go to one fixed 2 MiB array inside the library's device image; every GPU
+ * that loads the library holds it until the process exits.  Limit: one row range needs
+ * H*r*(r+1)*4 bytes, which must fit in those 2 MiB; larger shapes return
+ * GLGA_ERR_UNSUPPORTED before any device work.  The first call on a device looks up the
+ * array's device address and caches it; make that first call before any stream capture.
+ * All calls share the array and it keeps the last call's contents: each call writes every
+ * partial sum it later reads, so nothing needs clearing, but calls that overlap on the
+ * GPU (other streams or threads) race on it; the caller must order them.  No cudaMalloc,
+ * cudaFree or allocating library routine is called.                                   */
+GLGA_API glga_status glga_global_stats_static(const void *KV, int64_t N, int32_t H, int32_t r,
+                                              glga_dtype io, float *Sz, void *stream);
+
 /* Static strings; never NULL. */
 GLGA_API const char *glga_status_string(glga_status s);
 GLGA_API const char *glga_last_error_message(void);

@@ -129,3 +129,114 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
 }
 
 }  // namespace glga
+
+// ---------------------------------------------------------------------------------------
+// glga_global_stats_static: the same global statistics for callers that cannot allocate
+// device memory.  The per-range partial sums live in a fixed 2 MiB array that is part of
+// this library's device image (every GPU that loads the library keeps it until the
+// process exits), so the call allocates nothing.
+// ---------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace glga {
+namespace {
+
+constexpr size_t kStaticScratchFloats = 512u * 1024u;   // 2 MiB of float partial sums
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) float g_static_stats_scratch[kStaticScratchFloats];
+
+std::mutex g_static_mu;
+float *g_static_scratch_addr[kMaxDevices] = {};
+int g_static_num_sms[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device.
+// The array's name in host code is only a host-side stand-in, never a device address.
+glga_status static_scratch(int dev, float **ptr, int *num_sms) {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_scratch_addr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_static_stats_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static stats scratch)");
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        g_static_scratch_addr[dev] = static_cast<float *>(p);
+        g_static_num_sms[dev] = sms;
+    }
+    *ptr = g_static_scratch_addr[dev];
+    *num_sms = g_static_num_sms[dev];
+    return GLGA_OK;
+}
+
+template <typename T>
+glga_status launch_static_parts(const T *kv, int64_t N, int H, int r, int64_t rows_per_part,
+                                      int parts, float *scratch, cudaStream_t s) {
+    dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(H));
+    const int D = H * r;
+    switch (r) {
+        case 8: stats_part_kernel<T, 8><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
+        case 16: stats_part_kernel<T, 16><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
+        case 32: stats_part_kernel<T, 32><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
+        case 64: stats_part_kernel<T, 64><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
+        case 128: stats_part_kernel<T, 128><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
+        default: set_error("unsupported r"); return GLGA_ERR_UNSUPPORTED;
+    }
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
+}
+
+}  // namespace
+
+}  // namespace glga
+
+extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32_t H, int32_t r,
+                                                glga_dtype io, float *Sz, void *stream) {
+    using namespace glga;
+    if (N < 0 || H < 1 || (N > 0 && !KV) || !Sz) {
+        set_error("glga_global_stats_static: need N >= 0, H >= 1, non-null KV (when N > 0) and Sz");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (io != GLGA_F32 && io != GLGA_BF16) {
+        set_error("glga_global_stats_static: io must be GLGA_F32 or GLGA_BF16");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (!(r == 8 || r == 16 || r == 32 || r == 64 || r == 128)) {
+        set_error("glga_global_stats_static: r must be one of 8, 16, 32, 64, 128 (got %d)", r);
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    const int64_t per_part = static_cast<int64_t>(H) * r * (r + 1);
+    if (per_part > static_cast<int64_t>(kStaticScratchFloats)) {
+        set_error("glga_global_stats_static: H*r*(r+1)*4 = %lld bytes of partial sums exceed the "
+                  "%zu-byte static scratch (use glga_forward, which sizes its own workspace)",
+                  static_cast<long long>(per_part * 4), kStaticScratchFloats * sizeof(float));
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    int dev = 0;
+    GLGA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_error("glga_global_stats_static: device ordinal %d not supported", dev);
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    float *scratch = nullptr;
+    int sms = 0;
+    glga_status st = static_scratch(dev, &scratch, &sms);
+    if (st != GLGA_OK) return st;
+    const int64_t fit = static_cast<int64_t>(kStaticScratchFloats) / per_part;
+    const int64_t want = std::max<int64_t>(1, ceil_div(2 * sms, H));
+    const int64_t parts = std::max<int64_t>(
+        1, std::min<int64_t>(std::min(want, fit), ceil_div(std::max<int64_t>(N, 1), kStatsRows)));
+    const int64_t rows_per_part = ceil_div(std::max<int64_t>(N, 1), parts);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = (io == GLGA_F32)
+             ? launch_static_parts<float>(static_cast<const float *>(KV), N, H, r, rows_per_part,
+                                          static_cast<int>(parts), scratch, s)
+             : launch_static_parts<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(KV), N, H, r,
+                                                  rows_per_part, static_cast<int>(parts), scratch, s);
+    if (st != GLGA_OK) return st;
+    const int total = static_cast<int>(per_part);
+    stats_reduce_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+        scratch, static_cast<int>(parts), H, r, Sz);
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
+}

@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
         "glga_stage_times": ([_vp, ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)], _i32),
         "glga_workspace_bytes": ([_vp, ctypes.POINTER(_i64)], _i32),
         "glga_kernel_launches": ([_vp, ctypes.POINTER(_i64)], _i32),
+        "glga_global_stats_static": ([_vp, _i64, _i32, _i32, _i32, _vp, _vp], _i32),
         "glga_last_device_error": ([_vp, _vp], _i32),
         "glga_status_string": ([_i32], ctypes.c_char_p),
         "glga_last_error_message": ([], ctypes.c_char_p),
@@ -117,6 +118,20 @@ def csr_from_coo(N: int, src: torch.Tensor, dst: torch.Tensor, stream=None):
     _check(lib().glga_csr_from_coo(N, E, _ptr(src), _ptr(dst), _ptr(row_ptr), _ptr(col_idx),
                                    _stream(stream)), "glga_csr_from_coo")
     return row_ptr, col_idx[:E]
+
+
+def global_stats_static(KV: torch.Tensor, H: int, r: int, io: str, Sz=None, stream=None):
+    """S [H, r, r] and z [H, r] from KV [N, 2*H*r] (row j = k_j | v_j) without any device
+    allocation inside the library (partial sums use its fixed static scratch).  Returns
+    the Sz buffer: S followed by z."""
+    assert KV.is_cuda and KV.is_contiguous() and KV.dtype == torch_dtype(io)
+    N = KV.shape[0]
+    if Sz is None:
+        Sz = torch.empty(H * r * r + H * r, dtype=torch.float32, device=KV.device)
+    _check(lib().glga_global_stats_static(_ptr(KV) if N else None, N, H, r,
+                                          GLGA_F32 if io == "f32" else GLGA_BF16, _ptr(Sz),
+                                          _stream(stream)), "glga_global_stats_static")
+    return Sz
 
 
 class Layer:
