@@ -180,6 +180,9 @@ def main():
     ap.add_argument("--workload", default="arxiv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="shrink the workload (small profiling captures only; reported lines use 1.0)")
+    ap.add_argument("--no-parity", action="store_true", help="skip the sampled-row oracle check")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -213,7 +216,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    w = make_workload(args.workload)
+    w = make_workload(args.workload, scale=args.scale)
     dt = glga.torch_dtype(w.io)
     s_io = 4 if w.io == "f32" else 2
 
@@ -247,7 +250,7 @@ def main():
 
     # ---- parity spot check of what is being timed (sampled rows vs the oracle) ----
     parity = None
-    if rank == 0:
+    if rank == 0 and not args.no_parity:
         import oracle
         csr = (row_ptr.cpu().numpy(), col_idx.cpu().numpy())
         rng = np.random.default_rng(0)
@@ -298,7 +301,7 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = Yh.numel() * Yh.element_size()
     e2e_ms = []
-    for i in range(args.e2e_steps + 3):
+    for i in range(max(args.e2e_steps, 1) + 3):
         ev0.record(stream)
         X.copy_(host["X"], non_blocking=True)
         WQ.copy_(host["W_Q"], non_blocking=True)
@@ -341,7 +344,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
-            "config": {"workload": args.workload, "N": w.N, "E": w.E, "d": w.d, "H": w.H,
+            "config": {"workload": args.workload if args.scale == 1.0 else f"{args.workload}@scale{args.scale}",
+                       "N": w.N, "E": w.E, "d": w.d, "H": w.H,
                        "r": w.r, "io": w.io, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between timed steps (256 MiB write, outside the timed spans)"},
             "roofline": roofline, "projection": projection,
