@@ -131,15 +131,17 @@ GLGA_API glga_status glga_get_buckets(const glga_ctx *ctx, int32_t *warp_rows, i
 
 /* Copies the intermediates of the last glga_forward (device -> device, on `stream`):
  *   Q (io [N, H*r]), K and V (io [N, H*r] each), t (float [N], gate logit x_i . w_g),
- *   S (float [H, r, r]), z (float [H, r]).  Any pointer may be NULL.                   */
+ *   S (float [H, r, r]), z (float [H, r]), L (io [N, H*r], the local branch).  Any
+ *   pointer may be NULL.                                                               */
 GLGA_API glga_status glga_get_intermediates(const glga_ctx *ctx, void *Q, void *K, void *V, float *t,
-                                   float *S, float *z, void *stream);
+                                   float *S, float *z, void *L, void *stream);
 
 /* Per-stage timing.  When enabled, glga_forward records CUDA events on its stream around
  * every stage.  glga_stage_times synchronises on the last forward's final event and
  * writes up to n_max durations in milliseconds (host) in this order:
- *   0 weight packing and input preparation, 1 projection GEMM, 2 global statistics,
- *   3 local branch + readout + gate (the fused per-target kernel), 4 whole forward.
+ *   0 weight packing and input preparation, 1 projection GEMM, 2 global statistics
+ *   (tensor-core partials + ordered reduction), 3 local branch (per-target softmax
+ *   kernel), 4 readout GEMM with the fused gate blend, 5 whole forward.
  * Returns the number of values written through *n_written.                            */
 GLGA_API glga_status glga_set_timing(glga_ctx *ctx, int enable);
 GLGA_API glga_status glga_stage_times(glga_ctx *ctx, float *ms, int32_t n_max, int32_t *n_written);

@@ -47,7 +47,7 @@ static void release_ctx(Ctx *c) {
     if (!c) return;
     void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
-                    c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->dev_flag};
+                    c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)
@@ -177,6 +177,7 @@ glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t
     TRY(dev_alloc(c, &c->KV, static_cast<size_t>(N) * 2 * D * elem));
     TRY(dev_alloc(c, reinterpret_cast<void **>(&c->t), static_cast<size_t>(N) * sizeof(float)));
     TRY(projection_setup(c));
+    TRY(readout_setup(c));
     TRY(stats_setup(c));
     TRY(local_setup(c));
     if (st == GLGA_OK) {
@@ -228,7 +229,10 @@ glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void
     st = stats_run(c, s);
     if (st != GLGA_OK) return st;
     if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageLocal], s));
-    st = local_run(c, b_g, eps, Y, s);
+    st = local_run(c, s);
+    if (st != GLGA_OK) return st;
+    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageReadout], s));
+    st = readout_run(c, b_g, eps, Y, s);
     if (st != GLGA_OK) return st;
     if (c->timing) {
         GLGA_CUDA(cudaEventRecord(c->ev[kStageEnd], s));
@@ -278,7 +282,7 @@ glga_status glga_get_buckets(const glga_ctx *h, int32_t *warp_rows, int32_t *cta
 }
 
 glga_status glga_get_intermediates(const glga_ctx *h, void *Q, void *K, void *V, float *t,
-                                   float *S, float *z, void *stream) {
+                                   float *S, float *z, void *L, void *stream) {
     if (!h) {
         set_error("glga_get_intermediates: ctx is NULL");
         return GLGA_ERR_INVALID_ARG;
@@ -295,6 +299,7 @@ glga_status glga_get_intermediates(const glga_ctx *h, void *Q, void *K, void *V,
             GLGA_CUDA(cudaMemcpy2DAsync(V, row, static_cast<const uint8_t *>(c->KV) + row, 2 * row,
                                         row, c->N, cudaMemcpyDeviceToDevice, s));
         if (t) GLGA_CUDA(cudaMemcpyAsync(t, c->t, c->N * sizeof(float), cudaMemcpyDeviceToDevice, s));
+        if (L) GLGA_CUDA(cudaMemcpyAsync(L, c->L, c->N * row, cudaMemcpyDeviceToDevice, s));
     }
     const size_t sbytes = static_cast<size_t>(c->H) * c->r * c->r * sizeof(float);
     if (S) GLGA_CUDA(cudaMemcpyAsync(S, c->Sz, sbytes, cudaMemcpyDeviceToDevice, s));
@@ -327,13 +332,14 @@ glga_status glga_stage_times(glga_ctx *h, float *ms, int32_t n_max, int32_t *n_w
         return GLGA_ERR_INVALID_ARG;
     }
     GLGA_CUDA(cudaEventSynchronize(c->ev[kStageEnd]));
-    float v[5];
+    float v[6];
     GLGA_CUDA(cudaEventElapsedTime(&v[0], c->ev[kStagePrep], c->ev[kStageGemm]));
     GLGA_CUDA(cudaEventElapsedTime(&v[1], c->ev[kStageGemm], c->ev[kStageStats]));
     GLGA_CUDA(cudaEventElapsedTime(&v[2], c->ev[kStageStats], c->ev[kStageLocal]));
-    GLGA_CUDA(cudaEventElapsedTime(&v[3], c->ev[kStageLocal], c->ev[kStageEnd]));
-    GLGA_CUDA(cudaEventElapsedTime(&v[4], c->ev[kStagePrep], c->ev[kStageEnd]));
-    const int n = n_max < 5 ? n_max : 5;
+    GLGA_CUDA(cudaEventElapsedTime(&v[3], c->ev[kStageLocal], c->ev[kStageReadout]));
+    GLGA_CUDA(cudaEventElapsedTime(&v[4], c->ev[kStageReadout], c->ev[kStageEnd]));
+    GLGA_CUDA(cudaEventElapsedTime(&v[5], c->ev[kStagePrep], c->ev[kStageEnd]));
+    const int n = n_max < 6 ? n_max : 6;
     for (int i = 0; i < n; ++i) ms[i] = v[i];
     *n_written = n;
     return GLGA_OK;

@@ -48,7 +48,7 @@ struct TensorMap2D {
     bool valid = false;
 };
 
-enum Stage { kStagePrep = 0, kStageGemm, kStageStats, kStageLocal, kStageEnd, kNumEvents };
+enum Stage { kStagePrep = 0, kStageGemm, kStageStats, kStageLocal, kStageReadout, kStageEnd, kNumEvents };
 
 struct Ctx {
     int device = 0;
@@ -81,9 +81,17 @@ struct Ctx {
     void *Q = nullptr;            // io [N, D]
     void *KV = nullptr;           // io [N, 2D]  (k_j | v_j)
     float *t = nullptr;           // [N] gate logits
-    float *Spart = nullptr;       // [P][H][r][r+1]
-    float *Sz = nullptr;          // [H][r][r+1]  S rows with z as the last column
-    int32_t stats_parts = 0, stats_rows_per_part = 0;
+    float *Spart = nullptr;       // [P][H][r][r+1] partial sums of the row ranges
+    float *Sz = nullptr;          // S [H][r][r] followed by z [H][r]
+    int32_t stats_parts = 0;
+    int64_t stats_rows_per_part = 0;
+    TensorMap2D tmK, tmV;         // K and V halves of KV for the statistics kernel
+
+    // readout GEMM (phi(Q) x [S | z] per head group, blended with L)
+    int32_t ro_groups = 0, ro_hg = 0, ro_kp = 0, ro_bn = 0;
+    void *Bro = nullptr;          // [planes][groups][ro_bn][ro_kp] K-major, io type
+    TensorMap2D tmBro[2], tmQ;
+    void *L = nullptr;            // io [N, D] local-branch output
 
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;
@@ -115,7 +123,11 @@ glga_status stats_run(Ctx *c, cudaStream_t s);
 
 // local.cu
 glga_status local_setup(Ctx *c);
-glga_status local_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s);
+glga_status local_run(Ctx *c, cudaStream_t s);
+
+// readout.cu
+glga_status readout_setup(Ctx *c);
+glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s);
 
 // tensor maps (driver entry point resolved at run time; no libcuda link dependency)
 glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,

@@ -1,134 +1,410 @@
-// global_stats.cu -- global statistics of the linear-attention branch.
+// global_stats.cu -- global statistics of the linear-attention branch on tensor cores.
 //
 // Method page "Gated Local-Global Graph Attention", Key formulas:
 //   S_h = sum_j phi(k_j^h) (v_j^h)^T,  z_h = sum_j phi(k_j^h),  phi = elu + 1,
-// summed over all N nodes.  Deterministic: the node range is cut into P fixed parts,
-// every part's sums are formed in node order by one thread per output, and the parts
-// are then added in part order.  Output layout: S [H][r][r] followed by z [H][r].
+// summed over all N nodes.  For a block of 128 features the kernel forms
+//   [S_blk | z_blk] = phi(K_blk)^T [V_blk | 1]
+// with tcgen05.mma: A = phi(K) and B = V are used in place as MN-major operands (the
+// node index is the contraction dimension), straight from the 128-byte-swizzled TMA
+// tiles after warps 0-3 apply phi (and, for fp32, the tf32 hi/lo split); z comes from a
+// second MMA against a constant "ones" column.  Only the diagonal r x r blocks (one per
+// head) are kept.
+//
+// Deterministic split-N tree: the nodes are cut into P fixed ranges, each CTA
+// accumulates its range in TMEM in node-tile order, writes its partial sums, and a
+// reduction adds the P partials in range order.  The reduction also writes S and z into
+// the block-diagonal operand of the readout GEMM.  Output layout: S [H][r][r], z [H][r].
 #include <algorithm>
+#include <mutex>
 
 #include "glga_internal.cuh"
 
 namespace glga {
 namespace {
 
-constexpr int kStatsThreads = 256;
-constexpr int kStatsRows = 32;      // node rows staged per shared-memory tile
+constexpr int kFB = 128;             // features per block: MMA M (phi(K)) and N (V)
+constexpr int kRowBytes = 128;
+constexpr int kMaxStages = 2;
+constexpr int kThreads = 192;
 
 template <typename T>
-__device__ __forceinline__ float to_f(T x);
-template <>
-__device__ __forceinline__ float to_f<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+struct StatsGeom {
+    static constexpr int kRows = sizeof(T) == 2 ? 128 : 32;          // node rows per stage
+    static constexpr int kUK = sizeof(T) == 2 ? 16 : 8;              // rows per MMA
+    static constexpr int kBoxes = kFB * static_cast<int>(sizeof(T)) / kRowBytes;
+    static constexpr uint32_t kBoxBytes = kRows * kRowBytes;
+    static constexpr uint32_t kOpBytes = kBoxes * kBoxBytes;           // one operand plane
+};
+
+struct StatsParams {
+    int64_t N;
+    int32_t D, H;
+    int64_t rows_per_part;   // multiple of the stage height
+    int32_t stages;
+    uint32_t stage_bytes;
+    float *part;             // [P][H][r][r+1]
+    unsigned *flag;
+};
 
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
-// grid: (P parts, H heads).  part[p][h][a][c] for c < r is S, c == r is z.
-template <typename T, int R>
-__global__ void __launch_bounds__(kStatsThreads) stats_part_kernel(const T *__restrict__ KV,
-                                                                   int64_t N, int D,
-                                                                   int64_t rows_per_part,
-                                                                   float *__restrict__ part) {
-    constexpr int kOut = R * (R + 1);
-    constexpr int kPer = (kOut + kStatsThreads - 1) / kStatsThreads;
-    __shared__ float sk[kStatsRows][R];
-    __shared__ float sv[kStatsRows][R + 1];
-    const int h = blockIdx.y;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_part;
-    const int64_t r1 = std::min<int64_t>(N, r0 + rows_per_part);
-    float acc[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
-    for (int64_t base = r0; base < r1; base += kStatsRows) {
-        const int nrow = static_cast<int>(std::min<int64_t>(kStatsRows, r1 - base));
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < kStatsRows * R; idx += kStatsThreads) {
-            const int rr = idx / R, a = idx % R;
-            float kx = 0.f, vx = 0.f;
-            if (rr < nrow) {
-                const T *row = KV + (base + rr) * 2 * static_cast<int64_t>(D);
-                kx = phi(to_f<T>(row[h * R + a]));
-                vx = to_f<T>(row[D + h * R + a]);
-            }
-            sk[rr][a] = kx;
-            sv[rr][a] = vx;
-            if (a == 0) sv[rr][R] = rr < nrow ? 1.f : 0.f;
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int SPLIT, typename T, int R>
+__global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                               const __grid_constant__ CUtensorMap tmV,
+                                                               StatsParams p) {
+    using G = StatsGeom<T>;
+    constexpr uint32_t kFmt = SPLIT == 3 ? 2u : 1u;
+    extern __shared__ uint8_t dsmem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t ready_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_base_sh;
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *ones = smem + static_cast<size_t>(p.stages) * p.stage_bytes;   // 16 x 128 B, K-major
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int part = blockIdx.x, fb = blockIdx.y;
+    const int64_t r0 = static_cast<int64_t>(part) * p.rows_per_part;
+    const int64_t r1 = std::min<int64_t>(p.N, r0 + p.rows_per_part);
+    const int ntiles = r1 > r0 ? static_cast<int>(ceil_div(r1 - r0, G::kRows)) : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&ready_bar[s], 128);
+            mbar_init(&empty_bar[s], 1);
         }
-        __syncthreads();
-        for (int rr = 0; rr < nrow; ++rr) {
-#pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                const int o = threadIdx.x + i * kStatsThreads;
-                if (o < kOut) acc[i] += sk[rr][o / (R + 1)] * sv[rr][o % (R + 1)];
-            }
-        }
+        mbar_init(&done_bar, 1);
+        fence_mbar_init();
     }
-    float *dst = part + (static_cast<int64_t>(blockIdx.x) * gridDim.y + h) * kOut;
+    if (warp < 4) {
+        // ones tile: row 0 = 1.0 everywhere, rows 1..15 = 0 (the swizzle only permutes
+        // 16-byte chunks inside a row, so row 0 reads as ones at any K offset)
+        uint32_t *o = reinterpret_cast<uint32_t *>(ones);
+        const uint32_t one = sizeof(T) == 2 ? 0x3F803F80u : 0x3F800000u;
+        for (int i = threadIdx.x; i < 16 * kRowBytes / 4; i += 128) o[i] = (i < kRowBytes / 4) ? one : 0u;
+        fence_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(&tmem_base_sh, 256u);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            int issued = 0;
+            bool ok = true;
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % p.stages;
+                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
+                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+                mbar_arrive_expect_tx(&full_bar[s], 2 * G::kOpBytes);
+                const int32_t y = static_cast<int32_t>(r0 + static_cast<int64_t>(it) * G::kRows);
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        const int o = threadIdx.x + i * kStatsThreads;
-        if (o < kOut) dst[o] = acc[i];
+                for (int b = 0; b < G::kBoxes; ++b) {
+                    const int32_t x = fb * kFB + b * (kRowBytes / static_cast<int>(sizeof(T)));
+                    tma_load_2d(st + b * G::kBoxBytes, &tmK, &full_bar[s], x, y);
+                    tma_load_2d(st + G::kOpBytes + b * G::kBoxBytes, &tmV, &full_bar[s], x, y);
+                }
+                ++issued;
+            }
+            if (!ok) {
+                atomicOr(p.flag, kDevErrTimeout);
+                for (int it = std::max(0, issued - p.stages); it < issued; ++it)
+                    mbar_wait_bounded(&full_bar[it % p.stages], static_cast<uint32_t>(it / p.stages) & 1u);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            const uint32_t idS = instr_desc(128, kFB, kFmt, true, true);
+            const uint32_t idZ = instr_desc(128, 16, kFmt, true, false);
+            const uint64_t dones = smem_desc(smem_u32(ones), 16, 1024, 2);
+            bool ok = true;
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % p.stages;
+                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
+                if (!mbar_wait_bounded(&ready_bar[s], ph)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t kb = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
+                const uint32_t vb = kb + G::kOpBytes;
+#pragma unroll
+                for (int ks = 0; ks < G::kRows / G::kUK; ++ks) {
+                    const uint32_t off = ks * G::kUK * kRowBytes;
+                    const uint32_t acc0 = (it | ks) != 0;
+                    if (SPLIT == 3) {
+                        const uint32_t klo = kb + 2 * G::kOpBytes, vlo = kb + 3 * G::kOpBytes;
+                        const uint64_t akh = smem_desc(kb + off, G::kBoxBytes, 1024, 2);
+                        const uint64_t akl = smem_desc(klo + off, G::kBoxBytes, 1024, 2);
+                        const uint64_t bvh = smem_desc(vb + off, G::kBoxBytes, 1024, 2);
+                        const uint64_t bvl = smem_desc(vlo + off, G::kBoxBytes, 1024, 2);
+                        umma_tf32(tmem, akh, bvh, idS, acc0);
+                        umma_tf32(tmem, akh, bvl, idS, 1u);
+                        umma_tf32(tmem, akl, bvh, idS, 1u);
+                        umma_tf32(tmem + kFB, akh, dones, idZ, acc0);
+                        umma_tf32(tmem + kFB, akl, dones, idZ, 1u);
+                    } else {
+                        const uint64_t ak = smem_desc(kb + off, G::kBoxBytes, 1024, 2);
+                        const uint64_t bv = smem_desc(vb + off, G::kBoxBytes, 1024, 2);
+                        umma_bf16(tmem, ak, bv, idS, acc0);
+                        umma_bf16(tmem + kFB, ak, dones, idZ, acc0);
+                    }
+                }
+                umma_commit(&empty_bar[s]);
+            }
+            if (!ok) atomicOr(p.flag, kDevErrTimeout);
+            umma_commit(&done_bar);
+        }
+    } else {
+        // ---------------- warps 0-3: phi(K) (zero past the range), tf32 split ----------
+        bool ok = true;
+        constexpr int kChunksPerBox = G::kBoxBytes / 16;
+        for (int it = 0; it < ntiles && ok; ++it) {
+            const int s = it % p.stages;
+            const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
+            if (!mbar_wait_bounded(&full_bar[s], ph)) {
+                ok = false;
+                break;
+            }
+            uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+            const int64_t y0 = r0 + static_cast<int64_t>(it) * G::kRows;
+            for (int c = threadIdx.x; c < G::kBoxes * kChunksPerBox; c += 128) {
+                const int row = (c % kChunksPerBox) / 8;
+                const bool valid = y0 + row < r1;
+                if (SPLIT == 3) {
+                    float4 *kh = reinterpret_cast<float4 *>(st) + c;
+                    float4 *vh = reinterpret_cast<float4 *>(st + G::kOpBytes) + c;
+                    float4 *kl = reinterpret_cast<float4 *>(st + 2 * G::kOpBytes) + c;
+                    float4 *vl = reinterpret_cast<float4 *>(st + 3 * G::kOpBytes) + c;
+                    const float4 k4 = *kh, v4 = *vh;
+                    const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, vv[4] = {v4.x, v4.y, v4.z, v4.w};
+                    float khi[4], klo[4], vhi[4], vlo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float f = valid ? phi(kv[e]) : 0.f;
+                        khi[e] = to_tf32(f);
+                        klo[e] = to_tf32(f - khi[e]);
+                        vhi[e] = to_tf32(vv[e]);
+                        vlo[e] = to_tf32(vv[e] - vhi[e]);
+                    }
+                    *kh = make_float4(khi[0], khi[1], khi[2], khi[3]);
+                    *kl = make_float4(klo[0], klo[1], klo[2], klo[3]);
+                    *vh = make_float4(vhi[0], vhi[1], vhi[2], vhi[3]);
+                    *vl = make_float4(vlo[0], vlo[1], vlo[2], vlo[3]);
+                } else {
+                    uint4 *kp = reinterpret_cast<uint4 *>(st) + c;
+                    uint4 u = *kp;
+                    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = valid ? phi(__uint_as_float(w[e] << 16)) : 0.f;
+                        const float b = valid ? phi(__uint_as_float(w[e] & 0xffff0000u)) : 0.f;
+                        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+                        w[e] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    *kp = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&ready_bar[s]);
+        }
+        if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+    }
+    __syncwarp();
+
+    if (warp < 4) {
+        // ---------------- epilogue: diagonal head blocks of S and z -> partial sums ---------
+        const bool done = ntiles == 0 ? true : mbar_wait_bounded(&done_bar, 0);
+        tc_fence_after();
+        if (!done && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+        const bool have = ntiles > 0 && done;
+        const int t = warp * 32 + lane;                  // TMEM lane = feature in the block
+        const int f = fb * kFB + t;
+        const bool live = f < p.D;
+        const int h = live ? f / R : 0, a = f % R;
+        const int hc0 = h * R - fb * kFB;                // head's first column in the block
+        float *dst = p.part + ((static_cast<int64_t>(part) * p.H + h) * R + a) * (R + 1);
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+        for (int q = 0; q < kFB / 32; ++q) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + q * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int col = q * 32 + j;
+                if (live && col >= hc0 && col < hc0 + R) dst[col - hc0] = have ? __uint_as_float(v[j]) : 0.f;
+            }
+        }
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + kFB, v);
+        tmem_ld_wait();
+        if (live) dst[R] = have ? __uint_as_float(v[0]) : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256u);
     }
 }
 
-// Sz: S [H][r][r] then z [H][r]; sums parts 0..P-1 in order.
+// Sums parts 0..P-1 in order.  Writes S [H][R][R] then z [H][R] to Sz and, when Bro is
+// given, the readout operand: group gi = h / hg holds, K-major, S_h at rows (n)
+// hl*R + c and columns (k) hl*R + a, and z_h at row hga*R + hl (hl = h - gi*hg, hga =
+// heads in group gi).  Every other entry of Bro stays zero from its initialisation.
+template <typename T>
 __global__ void stats_reduce_kernel(const float *__restrict__ part, int P, int H, int R,
-                                    float *__restrict__ Sz) {
+                                    float *__restrict__ Sz, T *__restrict__ Bro, int hg, int BNr,
+                                    int Kp, int64_t plane) {
     const int per_head = R * (R + 1);
     const int total = H * per_head;
     for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < total; o += gridDim.x * blockDim.x) {
         float s = 0.f;
-        for (int p = 0; p < P; ++p) s += part[static_cast<int64_t>(p) * total + o];
+        for (int q = 0; q < P; ++q) s += part[static_cast<int64_t>(q) * total + o];
         const int h = o / per_head, rem = o % per_head, a = rem / (R + 1), c = rem % (R + 1);
         if (c < R)
             Sz[(static_cast<int64_t>(h) * R + a) * R + c] = s;
         else
             Sz[static_cast<int64_t>(H) * R * R + h * R + a] = s;
+        if (Bro) {
+            const int gi = h / hg, hl = h - gi * hg, hga = min(hg, H - gi * hg);
+            const int n = c < R ? hl * R + c : hga * R + hl;
+            const int64_t idx = (static_cast<int64_t>(gi) * BNr + n) * Kp + hl * R + a;
+            if (sizeof(T) == 4) {
+                const float hi = to_tf32(s);
+                reinterpret_cast<float *>(Bro)[idx] = hi;
+                reinterpret_cast<float *>(Bro)[plane + idx] = to_tf32(s - hi);
+            } else {
+                Bro[idx] = __float2bfloat16_rn(s);
+            }
+        }
     }
 }
 
 template <typename T>
-glga_status launch_parts(Ctx *c, cudaStream_t s) {
-    dim3 grid(static_cast<unsigned>(c->stats_parts), static_cast<unsigned>(c->H));
-    const T *kv = static_cast<const T *>(c->KV);
-    switch (c->r) {
-        case 8: stats_part_kernel<T, 8><<<grid, kStatsThreads, 0, s>>>(kv, c->N, c->D, c->stats_rows_per_part, c->Spart); break;
-        case 16: stats_part_kernel<T, 16><<<grid, kStatsThreads, 0, s>>>(kv, c->N, c->D, c->stats_rows_per_part, c->Spart); break;
-        case 32: stats_part_kernel<T, 32><<<grid, kStatsThreads, 0, s>>>(kv, c->N, c->D, c->stats_rows_per_part, c->Spart); break;
-        case 64: stats_part_kernel<T, 64><<<grid, kStatsThreads, 0, s>>>(kv, c->N, c->D, c->stats_rows_per_part, c->Spart); break;
-        case 128: stats_part_kernel<T, 128><<<grid, kStatsThreads, 0, s>>>(kv, c->N, c->D, c->stats_rows_per_part, c->Spart); break;
+glga_status launch_stats(const CUtensorMap &mk, const CUtensorMap &mv, const StatsParams &p, int parts,
+                         int nblk, int r, cudaStream_t s) {
+    dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(nblk));
+    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + 2048 + 1024;
+    constexpr int SPLIT = sizeof(T) == 4 ? 3 : 1;
+#define GLGA_ST(RR)                                                                          \
+    case RR: {                                                                               \
+        auto kern = stats_tc_kernel<SPLIT, T, RR>;                                           \
+        GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                       static_cast<int>(smem)));                             \
+        kern<<<grid, kThreads, smem, s>>>(mk, mv, p);                                        \
+        break;                                                                               \
+    }
+    switch (r) {
+        GLGA_ST(8) GLGA_ST(16) GLGA_ST(32) GLGA_ST(64) GLGA_ST(128)
         default: set_error("unsupported r"); return GLGA_ERR_UNSUPPORTED;
     }
+#undef GLGA_ST
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;
+}
+
+// Row ranges: a multiple of the stage height, about two CTAs per SM in total.
+void plan_parts(int64_t N, int nblk, int num_sms, int rows, int64_t max_parts, int *parts,
+                int64_t *rows_per_part) {
+    const int64_t want = std::max<int64_t>(1, ceil_div(2 * num_sms, nblk));
+    const int64_t tiles = std::max<int64_t>(1, ceil_div(std::max<int64_t>(N, 1), rows));
+    int64_t P = std::max<int64_t>(1, std::min(std::min(want, tiles), max_parts));
+    const int64_t per = ceil_div(tiles, P) * rows;
+    P = std::max<int64_t>(1, ceil_div(std::max<int64_t>(N, 1), per));
+    *parts = static_cast<int>(P);
+    *rows_per_part = per;
+}
+
+glga_status encode_kv_maps(const void *KV, int64_t N, int D, int elem, CUtensorMap *mk, CUtensorMap *mv,
+                           int rows) {
+    const CUtensorMapDataType dt =
+        elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint64_t stride = static_cast<uint64_t>(2) * D * elem;
+    glga_status st = encode_tmap_2d(mk, dt, KV, D, N, stride, kRowBytes / elem, rows);
+    if (st != GLGA_OK) return st;
+    return encode_tmap_2d(mv, dt, static_cast<const uint8_t *>(KV) + static_cast<size_t>(D) * elem,
+                          D, N, stride, kRowBytes / elem, rows);
+}
+
+template <typename T>
+uint32_t stage_bytes() {
+    return (sizeof(T) == 4 ? 4 : 2) * StatsGeom<T>::kOpBytes;
 }
 
 }  // namespace
 
 glga_status stats_setup(Ctx *c) {
-    const int64_t want = std::max<int64_t>(1, ceil_div(2 * c->num_sms, c->H));
-    const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(want, ceil_div(std::max<int64_t>(c->N, 1), kStatsRows)));
-    c->stats_parts = static_cast<int32_t>(parts);
-    c->stats_rows_per_part = static_cast<int32_t>(ceil_div(std::max<int64_t>(c->N, 1), parts));
-    const size_t per = static_cast<size_t>(c->H) * c->r * (c->r + 1) * sizeof(float);
-    glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart), per * parts);
-    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->Sz), per);
+    const int nblk = static_cast<int>(ceil_div(c->D, kFB));
+    const int rows = c->io == GLGA_F32 ? StatsGeom<float>::kRows : StatsGeom<__nv_bfloat16>::kRows;
+    int parts = 1;
+    int64_t per = 0;
+    plan_parts(c->N, nblk, c->num_sms, rows, 1 << 20, &parts, &per);
+    c->stats_parts = parts;
+    c->stats_rows_per_part = per;
+    const size_t one = static_cast<size_t>(c->H) * c->r * (c->r + 1) * sizeof(float);
+    glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart), one * parts);
+    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->Sz), one);
+    if (st == GLGA_OK && c->N > 0)
+        st = encode_kv_maps(c->KV, c->N, c->D, c->elem, &c->tmK.map, &c->tmV.map, rows);
     return st;
 }
 
 glga_status stats_run(Ctx *c, cudaStream_t s) {
-    glga_status st = (c->io == GLGA_F32) ? launch_parts<float>(c, s) : launch_parts<__nv_bfloat16>(c, s);
-    if (st != GLGA_OK) return st;
+    if (c->N > 0) {
+        StatsParams p;
+        p.N = c->N;
+        p.D = c->D;
+        p.H = c->H;
+        p.rows_per_part = c->stats_rows_per_part;
+        p.stages = kMaxStages;
+        p.part = c->Spart;
+        p.flag = c->dev_flag;
+        const int nblk = static_cast<int>(ceil_div(c->D, kFB));
+        glga_status st;
+        if (c->io == GLGA_F32) {
+            p.stage_bytes = stage_bytes<float>();
+            st = launch_stats<float>(c->tmK.map, c->tmV.map, p, c->stats_parts, nblk, c->r, s);
+        } else {
+            p.stage_bytes = stage_bytes<__nv_bfloat16>();
+            st = launch_stats<__nv_bfloat16>(c->tmK.map, c->tmV.map, p, c->stats_parts, nblk, c->r, s);
+        }
+        if (st != GLGA_OK) return st;
+        c->launches += 1;
+    }
     const int total = c->H * c->r * (c->r + 1);
-    stats_reduce_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
-        c->Spart, c->stats_parts, c->H, c->r, c->Sz);
+    const int P = c->N > 0 ? c->stats_parts : 0;
+    const int64_t plane = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
+    if (c->io == GLGA_F32)
+        stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+            c->Spart, P, c->H, c->r, c->Sz, static_cast<float *>(c->Bro), c->ro_hg, c->ro_bn, c->ro_kp, plane);
+    else
+        stats_reduce_kernel<__nv_bfloat16><<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+            c->Spart, P, c->H, c->r, c->Sz, static_cast<__nv_bfloat16 *>(c->Bro), c->ro_hg, c->ro_bn,
+            c->ro_kp, plane);
     GLGA_CUDA(cudaGetLastError());
-    c->launches += 2;
+    c->launches += 1;
     return GLGA_OK;
 }
-
-}  // namespace glga
 
 // ---------------------------------------------------------------------------------------
 // glga_global_stats_static: the same global statistics for callers that cannot allocate
@@ -136,65 +412,51 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
 // this library's device image (every GPU that loads the library keeps it until the
 // process exits), so the call allocates nothing.
 // ---------------------------------------------------------------------------------------
-#include <mutex>
-
-namespace glga {
 namespace {
 
 constexpr size_t kStaticScratchFloats = 512u * 1024u;   // 2 MiB of float partial sums
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) float g_static_stats_scratch[kStaticScratchFloats];
+__device__ unsigned g_static_stats_flag;   // bounded-wait timeouts of these calls
 
 std::mutex g_static_mu;
 float *g_static_scratch_addr[kMaxDevices] = {};
+unsigned *g_static_flag_addr[kMaxDevices] = {};
 int g_static_num_sms[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once per device.
-// The array's name in host code is only a host-side stand-in, never a device address.
-glga_status static_scratch(int dev, float **ptr, int *num_sms) {
+// Device addresses of the scratch array and its flag on the current device, looked up
+// once per device.  Their names in host code are host-side stand-ins, never device
+// addresses.
+glga_status static_scratch(int dev, float **ptr, unsigned **flag, int *num_sms) {
     std::lock_guard<std::mutex> lock(g_static_mu);
     if (!g_static_scratch_addr[dev]) {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_static_stats_scratch);
+        void *q = nullptr, *f = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&q, g_static_stats_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static stats scratch)");
+        e = cudaGetSymbolAddress(&f, g_static_stats_flag);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static stats flag)");
         int sms = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-        g_static_scratch_addr[dev] = static_cast<float *>(p);
+        g_static_scratch_addr[dev] = static_cast<float *>(q);
+        g_static_flag_addr[dev] = static_cast<unsigned *>(f);
         g_static_num_sms[dev] = sms;
     }
     *ptr = g_static_scratch_addr[dev];
+    *flag = g_static_flag_addr[dev];
     *num_sms = g_static_num_sms[dev];
     return GLGA_OK;
 }
 
-template <typename T>
-glga_status launch_static_parts(const T *kv, int64_t N, int H, int r, int64_t rows_per_part,
-                                      int parts, float *scratch, cudaStream_t s) {
-    dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(H));
-    const int D = H * r;
-    switch (r) {
-        case 8: stats_part_kernel<T, 8><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
-        case 16: stats_part_kernel<T, 16><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
-        case 32: stats_part_kernel<T, 32><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
-        case 64: stats_part_kernel<T, 64><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
-        case 128: stats_part_kernel<T, 128><<<grid, kStatsThreads, 0, s>>>(kv, N, D, rows_per_part, scratch); break;
-        default: set_error("unsupported r"); return GLGA_ERR_UNSUPPORTED;
-    }
-    GLGA_CUDA(cudaGetLastError());
-    return GLGA_OK;
-}
-
 }  // namespace
-
 }  // namespace glga
 
 extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32_t H, int32_t r,
                                                 glga_dtype io, float *Sz, void *stream) {
     using namespace glga;
-    if (N < 0 || H < 1 || (N > 0 && !KV) || !Sz) {
-        set_error("glga_global_stats_static: need N >= 0, H >= 1, non-null KV (when N > 0) and Sz");
+    if (N < 0 || N > 2147483647LL || H < 1 || (N > 0 && !KV) || !Sz) {
+        set_error("glga_global_stats_static: need 0 <= N < 2^31, H >= 1, non-null KV (when N > 0) and Sz");
         return GLGA_ERR_INVALID_ARG;
     }
     if (io != GLGA_F32 && io != GLGA_BF16) {
@@ -212,6 +474,12 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
                   static_cast<long long>(per_part * 4), kStaticScratchFloats * sizeof(float));
         return GLGA_ERR_UNSUPPORTED;
     }
+    const int elem = io == GLGA_F32 ? 4 : 2;
+    const int64_t D = static_cast<int64_t>(H) * r;
+    if (N > 0 && (reinterpret_cast<uintptr_t>(KV) & 15u)) {
+        set_error("glga_global_stats_static: KV must be 16-byte aligned");
+        return GLGA_ERR_INVALID_ARG;
+    }
     int dev = 0;
     GLGA_CUDA(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kMaxDevices) {
@@ -219,24 +487,40 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         return GLGA_ERR_UNSUPPORTED;
     }
     float *scratch = nullptr;
+    unsigned *flag = nullptr;
     int sms = 0;
-    glga_status st = static_scratch(dev, &scratch, &sms);
+    glga_status st = static_scratch(dev, &scratch, &flag, &sms);
     if (st != GLGA_OK) return st;
-    const int64_t fit = static_cast<int64_t>(kStaticScratchFloats) / per_part;
-    const int64_t want = std::max<int64_t>(1, ceil_div(2 * sms, H));
-    const int64_t parts = std::max<int64_t>(
-        1, std::min<int64_t>(std::min(want, fit), ceil_div(std::max<int64_t>(N, 1), kStatsRows)));
-    const int64_t rows_per_part = ceil_div(std::max<int64_t>(N, 1), parts);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (io == GLGA_F32)
-             ? launch_static_parts<float>(static_cast<const float *>(KV), N, H, r, rows_per_part,
-                                          static_cast<int>(parts), scratch, s)
-             : launch_static_parts<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(KV), N, H, r,
-                                                  rows_per_part, static_cast<int>(parts), scratch, s);
-    if (st != GLGA_OK) return st;
+    int parts = 0;
+    if (N > 0) {
+        const int nblk = static_cast<int>(ceil_div(D, kFB));
+        const int rows = io == GLGA_F32 ? StatsGeom<float>::kRows : StatsGeom<__nv_bfloat16>::kRows;
+        int64_t per = 0;
+        plan_parts(N, nblk, sms, rows, static_cast<int64_t>(kStaticScratchFloats) / per_part, &parts, &per);
+        CUtensorMap mk, mv;
+        st = encode_kv_maps(KV, N, static_cast<int>(D), elem, &mk, &mv, rows);
+        if (st != GLGA_OK) return st;
+        StatsParams p;
+        p.N = N;
+        p.D = static_cast<int32_t>(D);
+        p.H = H;
+        p.rows_per_part = per;
+        p.stages = kMaxStages;
+        p.part = scratch;
+        p.flag = flag;
+        if (io == GLGA_F32) {
+            p.stage_bytes = stage_bytes<float>();
+            st = launch_stats<float>(mk, mv, p, parts, nblk, r, s);
+        } else {
+            p.stage_bytes = stage_bytes<__nv_bfloat16>();
+            st = launch_stats<__nv_bfloat16>(mk, mv, p, parts, nblk, r, s);
+        }
+        if (st != GLGA_OK) return st;
+    }
     const int total = static_cast<int>(per_part);
-    stats_reduce_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
-        scratch, static_cast<int>(parts), H, r, Sz);
+    stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+        scratch, parts, H, r, Sz, nullptr, 1, 0, 0, 0);
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;
 }

@@ -1,10 +1,9 @@
-// local.cu -- per-target kernel: local softmax branch + global readout + gate + blend.
+// local.cu -- per-target kernel: the local softmax branch.
 //
 // Method page "Gated Local-Global Graph Attention", Key formulas:
 //   L_i = sum_{j in N(i)} softmax_j(q_i . k_j / sqrt r) v_j
-//   G_i = phi(q_i)^T S / (phi(q_i)^T z + eps)
-//   Y_i = g_i L_i + (1 - g_i) G_i,  g_i = sigmoid(t_i + b_g)
-// evaluated per head and concatenated.  The softmax is the stable one of the tinymesh
+// evaluated per head for every target row and written to L [N, H*r]; the global readout
+// and the gate blend run afterwards in the readout GEMM's epilogue (readout.cu).  The softmax is the stable one of the tinymesh
 // page ("Target softmax"), computed in a single pass with a running maximum: the state
 // (m, l, acc) of a partial sum is rescaled by 2^(m_old - m_new) whenever the maximum
 // grows, and two partial states merge the same way, so edges may be split across lanes,
@@ -89,15 +88,11 @@ struct LocalParams {
     int32_t chunk_edges;
     const void *Q;
     const void *KV;
-    const float *t;
-    const float *S;      // [H][r][r]
-    const float *z;      // [H][r]
     float *part;         // per chunk: m[H] l[H] acc[D]
     unsigned *ticket;
-    void *Y;
+    void *L;             // io [N, D] local-branch output
     int32_t D, r, H, nvec, lpe, epw, lph;
     float score_scale;   // log2(e) / sqrt(r)
-    float b_g, eps;
 };
 
 template <typename T, int VPL>
@@ -173,7 +168,7 @@ __device__ __forceinline__ void warp_edges(const LocalParams &p, const float (&q
 #pragma unroll
                 for (int e = 0; e < VE; ++e) dot = fmaf(q[v][e], kf[e], dot);
                 for (int o = 1; o < p.lph; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                s[u][v] = (j[u] >= 0) ? dot * p.score_scale : -INFINITY;
+                s[u][v] = (j[u] >= 0) ? dot : -INFINITY;
             }
         }
 #pragma unroll
@@ -222,69 +217,25 @@ __device__ __forceinline__ void load_q(const LocalParams &p, int64_t row, const 
         const int vid = v * 32 + ln.li;
         uint4 u = vid < p.nvec ? __ldg(Q + vid) : make_uint4(0, 0, 0, 0);
         Io<T>::unpack(u, q[v]);
+#pragma unroll
+        for (int e = 0; e < Io<T>::VE; ++e) q[v][e] *= p.score_scale;   // log2(e)/sqrt(r) folded in
     }
 }
 
-// L = acc / l, global readout, gate and blend; stores Y[row] (slot-0 lanes).
+// L_i = acc / l per head (0 for a row without edges); stores L[row] (slot-0 lanes).
 template <typename T, int VPL>
 __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row,
-                                           const float (&q)[VPL][Io<T>::VE],
                                            const State<T, VPL> &st, const Lane &ln) {
     constexpr int VE = Io<T>::VE;
-    const float tg = __ldg(p.t + row) + p.b_g;
-    const float g = 1.f / (1.f + expf(-tg));
-    uint4 *Y = static_cast<uint4 *>(p.Y) + row * p.nvec;
+    uint4 *Lout = static_cast<uint4 *>(p.L) + row * p.nvec;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
         const int vid = v * 32 + ln.li;
-        const bool valid = vid < p.nvec;
-        const int e0 = vid * VE;                         // first feature of this vector
-        const int h = valid ? e0 / p.r : 0;
-        const int c0 = e0 - h * p.r;                     // column inside the head
-        float ph[VE];
-#pragma unroll
-        for (int e = 0; e < VE; ++e) ph[e] = q[v][e] > 0.f ? q[v][e] + 1.f : expf(q[v][e]);
-        // denominator phi(q)^T z + eps
-        const float *zh = p.z + h * p.r;
-        float den = 0.f;
-        if (valid) {
-#pragma unroll
-            for (int e = 0; e < VE; ++e) den = fmaf(ph[e], __ldg(zh + c0 + e), den);
-        }
-        for (int o = 1; o < p.lph; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        // numerator phi(q)^T S[:, c0 .. c0+VE)
-        float num[VE];
-#pragma unroll
-        for (int e = 0; e < VE; ++e) num[e] = 0.f;
-        const int gbase = ln.lane & ~(p.lph - 1);
-        const float *Sh = p.S + static_cast<int64_t>(h) * p.r * p.r + c0;
-        for (int jj = 0; jj < p.lph; ++jj) {
-#pragma unroll
-            for (int e2 = 0; e2 < VE; ++e2) {
-                const float pq = __shfl_sync(0xffffffffu, ph[e2], gbase + jj);
-                const float4 *srow = reinterpret_cast<const float4 *>(Sh + (jj * VE + e2) * p.r);
-                if (valid) {
-#pragma unroll
-                    for (int e4 = 0; e4 < VE / 4; ++e4) {
-                        const float4 sv = __ldg(srow + e4);
-                        num[4 * e4 + 0] = fmaf(pq, sv.x, num[4 * e4 + 0]);
-                        num[4 * e4 + 1] = fmaf(pq, sv.y, num[4 * e4 + 1]);
-                        num[4 * e4 + 2] = fmaf(pq, sv.z, num[4 * e4 + 2]);
-                        num[4 * e4 + 3] = fmaf(pq, sv.w, num[4 * e4 + 3]);
-                    }
-                }
-            }
-        }
-        const float inv_den = 1.f / (den + p.eps);
         const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
         float y[VE];
 #pragma unroll
-        for (int e = 0; e < VE; ++e) {
-            const float L = st.acc[v][e] * inv_l;
-            const float G = num[e] * inv_den;
-            y[e] = g * L + (1.f - g) * G;
-        }
-        if (valid && ln.slot == 0) Y[vid] = Io<T>::pack(y);
+        for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l;
+        if (vid < p.nvec && ln.slot == 0) Lout[vid] = Io<T>::pack(y);
     }
 }
 
@@ -393,7 +344,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                         st.merge(v, __ldcg(src + h), __ldcg(src + p.H + h), a2);
                     }
                 }
-                finish_row<T, VPL>(p, row, q, st, ln);
+                finish_row<T, VPL>(p, row, st, ln);
             }
         }
         return;
@@ -404,7 +355,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         const int64_t row = p.cta_rows[bid];
         load_q<T, VPL>(p, row, ln, q);
         block_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
-        if (warp == 0) finish_row<T, VPL>(p, row, q, st, ln);
+        if (warp == 0) finish_row<T, VPL>(p, row, st, ln);
         return;
     }
     bid -= p.n_cta;
@@ -414,7 +365,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     const int64_t row = p.warp_rows[idx];
     load_q<T, VPL>(p, row, ln, q);
     warp_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, st);
-    finish_row<T, VPL>(p, row, q, st, ln);
+    finish_row<T, VPL>(p, row, st, ln);
 }
 
 template <typename T, int VPL, int U>
@@ -445,7 +396,7 @@ glga_status local_setup(Ctx *c) {
     return st;
 }
 
-glga_status local_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
+glga_status local_run(Ctx *c, cudaStream_t s) {
     LocalParams p;
     p.row_ptr = c->row_ptr;
     p.col_idx = c->col_idx;
@@ -460,12 +411,9 @@ glga_status local_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     p.chunk_edges = c->opts.chunk_edges;
     p.Q = c->Q;
     p.KV = c->KV;
-    p.t = c->t;
-    p.S = c->Sz;
-    p.z = c->Sz + static_cast<int64_t>(c->H) * c->r * c->r;
     p.part = c->chunk_part;
     p.ticket = c->chunk_ticket;
-    p.Y = Y;
+    p.L = c->L;
     p.D = c->D;
     p.r = c->r;
     p.H = c->H;
@@ -477,8 +425,6 @@ glga_status local_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     p.epw = 32 / lpe;
     p.lph = c->r / VE;
     p.score_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->r)));
-    p.b_g = b_g;
-    p.eps = eps;
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
     if (c->io == GLGA_F32) {
         if (vpl == 1) return launch_local<float, 1, 4>(c, p, s);

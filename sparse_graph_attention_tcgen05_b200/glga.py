@@ -21,7 +21,7 @@ GLGA_F32, GLGA_BF16 = 0, 1
 STATUS = {0: "GLGA_OK", 1: "GLGA_ERR_INVALID_ARG", 2: "GLGA_ERR_BAD_GRAPH",
           3: "GLGA_ERR_UNSUPPORTED", 4: "GLGA_ERR_OOM", 5: "GLGA_ERR_CUDA",
           6: "GLGA_ERR_TIMEOUT", 7: "GLGA_ERR_DEVICE"}
-STAGES = ("prep", "gemm", "stats", "local", "forward")
+STAGES = ("prep", "gemm", "stats", "local", "readout", "forward")
 
 
 class GLGAError(RuntimeError):
@@ -62,7 +62,7 @@ def lib() -> ctypes.CDLL:
         "glga_csr_from_coo": ([_i64, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_bucket_counts": ([_vp, ctypes.POINTER(_i64)], _i32),
         "glga_get_buckets": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
-        "glga_get_intermediates": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+        "glga_get_intermediates": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_set_timing": ([_vp, ctypes.c_int], _i32),
         "glga_stage_times": ([_vp, ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)], _i32),
         "glga_workspace_bytes": ([_vp, ctypes.POINTER(_i64)], _i32),
@@ -198,8 +198,9 @@ class Layer:
                "V": torch.empty(self.N, self.D, dtype=self.dtype, device=dev),
                "t": torch.empty(self.N, dtype=torch.float32, device=dev),
                "S": torch.empty(self.H, self.r, self.r, dtype=torch.float32, device=dev),
-               "z": torch.empty(self.H, self.r, dtype=torch.float32, device=dev)}
-        _check(lib().glga_get_intermediates(self._h, *(_ptr(out[k]) for k in ("Q", "K", "V", "t", "S", "z")),
+               "z": torch.empty(self.H, self.r, dtype=torch.float32, device=dev),
+               "L": torch.empty(self.N, self.D, dtype=self.dtype, device=dev)}
+        _check(lib().glga_get_intermediates(self._h, *(_ptr(out[k]) for k in ("Q", "K", "V", "t", "S", "z", "L")),
                                             _stream(stream)), "glga_get_intermediates")
         return out
 
@@ -207,9 +208,9 @@ class Layer:
         _check(lib().glga_set_timing(self._h, 1 if enable else 0), "glga_set_timing")
 
     def stage_times(self) -> dict:
-        ms = (ctypes.c_float * 5)()
+        ms = (ctypes.c_float * 6)()
         n = _i32()
-        _check(lib().glga_stage_times(self._h, ms, 5, ctypes.byref(n)), "glga_stage_times")
+        _check(lib().glga_stage_times(self._h, ms, 6, ctypes.byref(n)), "glga_stage_times")
         return {STAGES[i]: float(ms[i]) for i in range(n.value)}
 
     def workspace_bytes(self) -> int:
