@@ -134,6 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
         if (lane == 0) {
             const uint32_t idS = instr_desc(128, kFB, kFmt, true, true);
             const uint32_t idZ = instr_desc(128, 16, kFmt, true, false);
+            const uint32_t idSk = instr_desc(128, kFB, kFmt, false, false);
+            const uint32_t idZk = instr_desc(128, 16, kFmt, false, false);
             const uint64_t dones = smem_desc(smem_u32(ones), 16, 1024, 2);
             bool ok = true;
             for (int it = 0; it < ntiles; ++it) {
@@ -151,16 +153,21 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                     const uint32_t off = ks * G::kUK * kRowBytes;
                     const uint32_t acc0 = (it | ks) != 0;
                     if (SPLIT == 3) {
-                        const uint32_t klo = kb + 2 * G::kOpBytes, vlo = kb + 3 * G::kOpBytes;
-                        const uint64_t akh = smem_desc(kb + off, G::kBoxBytes, 1024, 2);
-                        const uint64_t akl = smem_desc(klo + off, G::kBoxBytes, 1024, 2);
-                        const uint64_t bvh = smem_desc(vb + off, G::kBoxBytes, 1024, 2);
-                        const uint64_t bvl = smem_desc(vlo + off, G::kBoxBytes, 1024, 2);
-                        umma_tf32(tmem, akh, bvh, idS, acc0);
-                        umma_tf32(tmem, akh, bvl, idS, 1u);
-                        umma_tf32(tmem, akl, bvh, idS, 1u);
-                        umma_tf32(tmem + kFB, akh, dones, idZ, acc0);
-                        umma_tf32(tmem + kFB, akl, dones, idZ, 1u);
+                        // tf32 operands were transposed to K-major planes by warps 0-3
+                        // (MN-major tf32 would need the 32-byte-atom swizzle)
+                        const uint32_t kt = ks * 32;   // 8 node rows of tf32 = 32 bytes
+                        const uint32_t ah = kb + 2 * G::kOpBytes, al = kb + 3 * G::kOpBytes;
+                        const uint32_t bh = kb + 4 * G::kOpBytes, bl = kb + 5 * G::kOpBytes;
+                        const uint64_t akh = smem_desc(ah + kt, 16, 1024, 2);
+                        const uint64_t akl = smem_desc(al + kt, 16, 1024, 2);
+                        const uint64_t bvh = smem_desc(bh + kt, 16, 1024, 2);
+                        const uint64_t bvl = smem_desc(bl + kt, 16, 1024, 2);
+                        umma_tf32(tmem, akh, bvh, idSk, acc0);
+                        umma_tf32(tmem, akh, bvl, idSk, 1u);
+                        umma_tf32(tmem, akl, bvh, idSk, 1u);
+                        umma_tf32(tmem + kFB, akh, dones, idZk, acc0);
+                        umma_tf32(tmem + kFB, akl, dones, idZk, 1u);
+                        (void)off;
                     } else {
                         const uint64_t ak = smem_desc(kb + off, G::kBoxBytes, 1024, 2);
                         const uint64_t bv = smem_desc(vb + off, G::kBoxBytes, 1024, 2);
@@ -186,30 +193,38 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             }
             uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
             const int64_t y0 = r0 + static_cast<int64_t>(it) * G::kRows;
-            for (int c = threadIdx.x; c < G::kBoxes * kChunksPerBox; c += 128) {
+            if (SPLIT == 3) {
+                // Transpose the [node][feature] TMA tiles (128-byte swizzle) into K-major
+                // planes [feature][node] with the same swizzle, applying phi and the tf32
+                // split on the way: element (m, k) of a plane sits at
+                // (m/8)*1024 + (m%8)*128 + (((k/4) ^ (m%8)) * 16) + (k%4)*4.
+                const float *rk = reinterpret_cast<const float *>(st);
+                const float *rv = reinterpret_cast<const float *>(st + G::kOpBytes);
+                float *ah = reinterpret_cast<float *>(st + 2 * G::kOpBytes);
+                float *al = reinterpret_cast<float *>(st + 3 * G::kOpBytes);
+                float *bh = reinterpret_cast<float *>(st + 4 * G::kOpBytes);
+                float *bl = reinterpret_cast<float *>(st + 5 * G::kOpBytes);
+                for (int idx = threadIdx.x; idx < G::kRows * kFB; idx += 128) {
+                    const int k = idx / kFB, m = idx % kFB;
+                    const int e = m % 32;
+                    const int src = ((m / 32) * G::kBoxBytes + k * kRowBytes +
+                                     (((e / 4) ^ (k % 8)) * 16) + (e % 4) * 4) / 4;
+                    const int dst = ((m / 8) * 1024 + (m % 8) * kRowBytes +
+                                     (((k / 4) ^ (m % 8)) * 16) + (k % 4) * 4) / 4;
+                    const bool valid = y0 + k < r1;
+                    const float f = valid ? phi(rk[src]) : 0.f;
+                    const float v = rv[src];
+                    const float fh = to_tf32(f), vh = to_tf32(v);
+                    ah[dst] = fh;
+                    al[dst] = to_tf32(f - fh);
+                    bh[dst] = vh;
+                    bl[dst] = to_tf32(v - vh);
+                }
+            }
+            for (int c = threadIdx.x; SPLIT != 3 && c < G::kBoxes * kChunksPerBox; c += 128) {
                 const int row = (c % kChunksPerBox) / 8;
                 const bool valid = y0 + row < r1;
-                if (SPLIT == 3) {
-                    float4 *kh = reinterpret_cast<float4 *>(st) + c;
-                    float4 *vh = reinterpret_cast<float4 *>(st + G::kOpBytes) + c;
-                    float4 *kl = reinterpret_cast<float4 *>(st + 2 * G::kOpBytes) + c;
-                    float4 *vl = reinterpret_cast<float4 *>(st + 3 * G::kOpBytes) + c;
-                    const float4 k4 = *kh, v4 = *vh;
-                    const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, vv[4] = {v4.x, v4.y, v4.z, v4.w};
-                    float khi[4], klo[4], vhi[4], vlo[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float f = valid ? phi(kv[e]) : 0.f;
-                        khi[e] = to_tf32(f);
-                        klo[e] = to_tf32(f - khi[e]);
-                        vhi[e] = to_tf32(vv[e]);
-                        vlo[e] = to_tf32(vv[e] - vhi[e]);
-                    }
-                    *kh = make_float4(khi[0], khi[1], khi[2], khi[3]);
-                    *kl = make_float4(klo[0], klo[1], klo[2], klo[3]);
-                    *vh = make_float4(vhi[0], vhi[1], vhi[2], vhi[3]);
-                    *vl = make_float4(vlo[0], vlo[1], vlo[2], vlo[3]);
-                } else {
+                {
                     uint4 *kp = reinterpret_cast<uint4 *>(st) + c;
                     uint4 u = *kp;
                     uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -346,9 +361,11 @@ glga_status encode_kv_maps(const void *KV, int64_t N, int D, int elem, CUtensorM
                           D, N, stride, kRowBytes / elem, rows);
 }
 
+// bf16: K and V tiles (phi applied in place).  fp32: K and V tiles plus four K-major
+// tf32 planes (phi(K) hi/lo, V hi/lo).
 template <typename T>
 uint32_t stage_bytes() {
-    return (sizeof(T) == 4 ? 4 : 2) * StatsGeom<T>::kOpBytes;
+    return (sizeof(T) == 4 ? 6 : 2) * StatsGeom<T>::kOpBytes;
 }
 
 }  // namespace
