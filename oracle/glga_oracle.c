@@ -75,9 +75,18 @@ int oracle_csr_from_coo(int64_t N, int64_t E, const int32_t *src, const int32_t 
  *   bucket 1 if warp_max < deg <= chunk_edges,
  *   bucket 2 otherwise; a bucket-2 row is cut into ceil(deg / chunk_edges) chunks that
  *   start at row_ptr[i] + c * chunk_edges.
- * Rows are listed in ascending order inside each bucket; chunks follow their rows'
- * order, then c.  counts[0..2] = bucket sizes, counts[3] = number of chunks.
- * Passing NULL lists only counts.                                                        */
+ * Bucket 0 lists its rows by descending degree, ties by ascending row; buckets 1 and 2
+ * list rows in ascending order; chunks follow their rows' order, then c.
+ * counts[0..2] = bucket sizes, counts[3] = number of chunks.  Passing NULL lists only
+ * counts.                                                                               */
+static const int32_t *g_sort_row_ptr;
+static int cmp_deg_desc(const void *a, const void *b) {
+    const int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    const int32_t dx = g_sort_row_ptr[x + 1] - g_sort_row_ptr[x];
+    const int32_t dy = g_sort_row_ptr[y + 1] - g_sort_row_ptr[y];
+    if (dx != dy) return dx > dy ? -1 : 1;
+    return (x > y) - (x < y);
+}
 int oracle_degree_buckets(int64_t N, const int32_t *row_ptr, int32_t warp_max,
                           int32_t chunk_edges, int64_t *counts, int32_t *warp_rows,
                           int32_t *cta_rows, int32_t *split_rows, int32_t *chunk_row,
@@ -103,6 +112,10 @@ int oracle_degree_buckets(int64_t N, const int32_t *row_ptr, int32_t warp_max,
         }
     }
     counts[0] = n0; counts[1] = n1; counts[2] = n2; counts[3] = nc;
+    if (warp_rows && n0 > 1) {
+        g_sort_row_ptr = row_ptr;
+        qsort(warp_rows, (size_t)n0, sizeof(int32_t), cmp_deg_desc);
+    }
     return 0;
 }
 

@@ -47,7 +47,8 @@ static void release_ctx(Ctx *c) {
     if (!c) return;
     void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
-                    c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->dev_flag};
+                    c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
+                    c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)

@@ -64,6 +64,8 @@ struct Ctx {
     int64_t nb[4] = {0, 0, 0, 0};   // bucket sizes and chunk count
     int32_t *warp_rows = nullptr, *cta_rows = nullptr, *split_rows = nullptr;
     int32_t *chunk_row = nullptr, *chunk_begin = nullptr;
+    int32_t *task_start = nullptr;      // bucket-0 warp tasks: [n_tasks + 1] list positions
+    int64_t n_tasks = 0;
     unsigned *chunk_ticket = nullptr;   // one counter per chunk slot (first chunk of a row)
     float *chunk_part = nullptr;        // per chunk: m[H], l[H], acc[D]
 
@@ -89,8 +91,9 @@ struct Ctx {
 
     // readout GEMM (phi(Q) x [S | z] per head group, blended with L)
     int32_t ro_groups = 0, ro_hg = 0, ro_kp = 0, ro_bn = 0;
+    bool ro_tma_epi = false;      // L in / Y out through TMA boxes (group width fits boxes)
     void *Bro = nullptr;          // [planes][groups][ro_bn][ro_kp] K-major, io type
-    TensorMap2D tmBro[2], tmQ;
+    TensorMap2D tmBro[2], tmQ, tmL;
     void *L = nullptr;            // io [N, D] local-branch output
 
     unsigned *dev_flag = nullptr;
@@ -200,6 +203,32 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+// 2-D tiled TMA store shared -> global (bulk async group).  Elements outside the tensor
+// are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x,
+                                             int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until every committed bulk store has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy
+// (TMA, tcgen05) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {

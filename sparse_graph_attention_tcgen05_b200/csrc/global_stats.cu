@@ -24,12 +24,16 @@ namespace {
 
 constexpr int kFB = 128;             // features per block: MMA M (phi(K)) and N (V)
 constexpr int kRowBytes = 128;
-constexpr int kMaxStages = 2;
-constexpr int kThreads = 192;
+constexpr int kMaxStages = 3;
+constexpr int kWorkers = 256;        // warps 0-7: phi / split passes; warps 0-3: epilogue
+constexpr int kProdWarp = 8;         // TMA producer
+constexpr int kMmaWarp = 9;          // TMEM owner and MMA issuer
+constexpr int kThreads = 320;
 
 template <typename T>
 struct StatsGeom {
-    static constexpr int kRows = sizeof(T) == 2 ? 128 : 32;          // node rows per stage
+    static constexpr int kRows = sizeof(T) == 2 ? 64 : 32;           // node rows per stage
+    static constexpr int kStages = sizeof(T) == 2 ? 3 : 2;
     static constexpr int kUK = sizeof(T) == 2 ? 16 : 8;              // rows per MMA
     static constexpr int kBoxes = kFB * static_cast<int>(sizeof(T)) / kRowBytes;
     static constexpr uint32_t kBoxBytes = kRows * kRowBytes;
@@ -46,7 +50,7 @@ struct StatsParams {
     unsigned *flag;
 };
 
-__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
+__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -77,21 +81,21 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&ready_bar[s], 128);
+            mbar_init(&ready_bar[s], kWorkers);
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&done_bar, 1);
         fence_mbar_init();
     }
-    if (warp < 4) {
+    if (threadIdx.x < kWorkers) {
         // ones tile: row 0 = 1.0 everywhere, rows 1..15 = 0 (the swizzle only permutes
         // 16-byte chunks inside a row, so row 0 reads as ones at any K offset)
         uint32_t *o = reinterpret_cast<uint32_t *>(ones);
         const uint32_t one = sizeof(T) == 2 ? 0x3F803F80u : 0x3F800000u;
-        for (int i = threadIdx.x; i < 16 * kRowBytes / 4; i += 128) o[i] = (i < kRowBytes / 4) ? one : 0u;
+        for (int i = threadIdx.x; i < 16 * kRowBytes / 4; i += kWorkers) o[i] = (i < kRowBytes / 4) ? one : 0u;
         fence_async_smem();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&tmem_base_sh, 256u);
         tmem_relinquish();
     }
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 4) {
+    if (warp == kProdWarp) {
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                     mbar_wait_bounded(&full_bar[it % p.stages], static_cast<uint32_t>(it / p.stages) & 1u);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         if (lane == 0) {
             const uint32_t idS = instr_desc(128, kFB, kFmt, true, true);
             const uint32_t idZ = instr_desc(128, 16, kFmt, true, false);
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                 float *al = reinterpret_cast<float *>(st + 3 * G::kOpBytes);
                 float *bh = reinterpret_cast<float *>(st + 4 * G::kOpBytes);
                 float *bl = reinterpret_cast<float *>(st + 5 * G::kOpBytes);
-                for (int idx = threadIdx.x; idx < G::kRows * kFB; idx += 128) {
+                for (int idx = threadIdx.x; idx < G::kRows * kFB; idx += kWorkers) {
                     const int k = idx / kFB, m = idx % kFB;
                     const int e = m % 32;
                     const int src = ((m / 32) * G::kBoxBytes + k * kRowBytes +
@@ -221,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                     bl[dst] = to_tf32(v - vh);
                 }
             }
-            for (int c = threadIdx.x; SPLIT != 3 && c < G::kBoxes * kChunksPerBox; c += 128) {
+            for (int c = threadIdx.x; SPLIT != 3 && c < G::kBoxes * kChunksPerBox; c += kWorkers) {
                 const int row = (c % kChunksPerBox) / 8;
                 const bool valid = y0 + row < r1;
                 {
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 256u);
     }
@@ -286,15 +290,35 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
 // given, the readout operand: group gi = h / hg holds, K-major, S_h at rows (n)
 // hl*R + c and columns (k) hl*R + a, and z_h at row hga*R + hl (hl = h - gi*hg, hga =
 // heads in group gi).  Every other entry of Bro stays zero from its initialisation.
+// Block of 256 threads = 8 warps for 32 consecutive outputs: warp w adds parts
+// w, w+8, w+16, ... in order, then warp 0 adds the 8 warp sums in warp order.
 template <typename T>
-__global__ void stats_reduce_kernel(const float *__restrict__ part, int P, int H, int R,
+__global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restrict__ part, int P, int H, int R,
                                     float *__restrict__ Sz, T *__restrict__ Bro, int hg, int BNr,
                                     int Kp, int64_t plane) {
+    __shared__ float ws[8][32];
     const int per_head = R * (R + 1);
     const int total = H * per_head;
-    for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < total; o += gridDim.x * blockDim.x) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int o = blockIdx.x * 32 + lane;
+    float acc = 0.f;
+    if (o < total) {
+        int q = w;
+        for (; q + 24 < P; q += 32) {
+            const float a0 = part[static_cast<int64_t>(q) * total + o];
+            const float a1 = part[static_cast<int64_t>(q + 8) * total + o];
+            const float a2 = part[static_cast<int64_t>(q + 16) * total + o];
+            const float a3 = part[static_cast<int64_t>(q + 24) * total + o];
+            acc += a0; acc += a1; acc += a2; acc += a3;
+        }
+        for (; q < P; q += 8) acc += part[static_cast<int64_t>(q) * total + o];
+    }
+    ws[w][lane] = acc;
+    __syncthreads();
+    if (w == 0 && o < total) {
         float s = 0.f;
-        for (int q = 0; q < P; ++q) s += part[static_cast<int64_t>(q) * total + o];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s += ws[k][lane];
         const int h = o / per_head, rem = o % per_head, a = rem / (R + 1), c = rem % (R + 1);
         if (c < R)
             Sz[(static_cast<int64_t>(h) * R + a) * R + c] = s;
@@ -393,7 +417,7 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
         p.D = c->D;
         p.H = c->H;
         p.rows_per_part = c->stats_rows_per_part;
-        p.stages = kMaxStages;
+        p.stages = c->io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
         p.part = c->Spart;
         p.flag = c->dev_flag;
         const int nblk = static_cast<int>(ceil_div(c->D, kFB));
@@ -412,10 +436,10 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
     const int P = c->N > 0 ? c->stats_parts : 0;
     const int64_t plane = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
     if (c->io == GLGA_F32)
-        stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+        stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
             c->Spart, P, c->H, c->r, c->Sz, static_cast<float *>(c->Bro), c->ro_hg, c->ro_bn, c->ro_kp, plane);
     else
-        stats_reduce_kernel<__nv_bfloat16><<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+        stats_reduce_kernel<__nv_bfloat16><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
             c->Spart, P, c->H, c->r, c->Sz, static_cast<__nv_bfloat16 *>(c->Bro), c->ro_hg, c->ro_bn,
             c->ro_kp, plane);
     GLGA_CUDA(cudaGetLastError());
@@ -523,7 +547,7 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         p.D = static_cast<int32_t>(D);
         p.H = H;
         p.rows_per_part = per;
-        p.stages = kMaxStages;
+        p.stages = io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
         p.part = scratch;
         p.flag = flag;
         if (io == GLGA_F32) {
@@ -536,7 +560,7 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         if (st != GLGA_OK) return st;
     }
     const int total = static_cast<int>(per_part);
-    stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(
+    stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
         scratch, parts, H, r, Sz, nullptr, 1, 0, 0, 0);
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;

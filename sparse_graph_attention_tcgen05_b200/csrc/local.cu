@@ -3,26 +3,31 @@
 // Method page "Gated Local-Global Graph Attention", Key formulas:
 //   L_i = sum_{j in N(i)} softmax_j(q_i . k_j / sqrt r) v_j
 // evaluated per head for every target row and written to L [N, H*r]; the global readout
-// and the gate blend run afterwards in the readout GEMM's epilogue (readout.cu).  The softmax is the stable one of the tinymesh
-// page ("Target softmax"), computed in a single pass with a running maximum: the state
-// (m, l, acc) of a partial sum is rescaled by 2^(m_old - m_new) whenever the maximum
-// grows, and two partial states merge the same way, so edges may be split across lanes,
-// warps and thread blocks and merged in a fixed order.  No per-edge value is stored.
+// and the gate blend run afterwards in the readout GEMM's epilogue (readout.cu).  The
+// softmax is the stable one of the tinymesh page ("Target softmax"), computed in a
+// single pass with a running maximum: the state (m, l, acc) of a partial sum is rescaled
+// by 2^(m_old - m_new) whenever the maximum grows, and two partial states merge the same
+// way, so edges may be split across lanes, warps and thread blocks and merged in a fixed
+// order.  No per-edge value is stored.
 //
 // Work is scheduled by the degree buckets built at create time:
 //   chunk blocks   bucket-2 rows cut into chunk_edges-edge chunks; each block merges its
 //                  8 warps, writes (m, l, acc) to scratch, and the last block of a row
 //                  (ticket counter) merges the row's chunks in chunk order and finishes
 //   row blocks     bucket-1 rows: 8 warps split the edges, merged in warp order
-//   warp blocks    bucket-0 rows: one warp per row, 8 rows per block
+//   task warps     bucket-0 rows (descending degree) in tasks of <= 32 rows and about
+//                  kTaskEdges edges; each edge slot of the warp takes its own row
 // Heavy work comes first in block order so it starts early.
 //
 // Lane layout: a 16-byte vector holds VE = 16/sizeof(T) consecutive features; an edge's
-// k_j (or v_j) row is LPE lanes x VPL vectors; EPW = 32/LPE edges are in flight per warp
-// step (U steps unrolled), and the r features of a head live in LPH = r/VE adjacent
-// lanes, which reduce dot products with butterfly shuffles.
+// k_j (or v_j) row is LPE lanes x VPL vectors; EPW = 32/LPE edge slots per warp; the r
+// features of a head live in LPH = r/VE adjacent lanes, which reduce dot products with
+// butterfly shuffles.  Each slot walks a contiguous edge range U edges at a time; the
+// column indices of the next step (and, for task rows, the next row's q and first
+// columns) are loaded one step ahead so the k_j/v_j gathers do not wait behind them.
 #include <algorithm>
 #include <cmath>
+#include <vector>
 
 #include "glga_internal.cuh"
 
@@ -31,6 +36,8 @@ namespace {
 
 constexpr int kLocalWarps = 8;
 constexpr int kLocalThreads = kLocalWarps * 32;
+constexpr int kTaskRows = 32;
+constexpr int64_t kTaskEdges = 256;
 
 template <typename T>
 struct Io;
@@ -80,11 +87,12 @@ struct LocalParams {
     const int32_t *row_ptr;
     const int32_t *col_idx;
     const int32_t *warp_rows;
+    const int32_t *task_start;   // [n_tasks + 1] positions in warp_rows
     const int32_t *cta_rows;
     const int32_t *chunk_row;
     const int32_t *chunk_begin;
-    int64_t n_warp, n_cta, n_chunks;
-    int64_t warp_blocks;
+    int64_t n_tasks, n_cta, n_chunks;
+    int64_t task_blocks;
     int32_t chunk_edges;
     const void *Q;
     const void *KV;
@@ -124,23 +132,35 @@ struct Lane {
     int lane, slot, li;
 };
 
-// Runs one warp over the CSR entries [e0, e1) of a row whose query vectors are in q.
-// On return every lane holds the merged state of its feature vectors over all slots.
+// First column index of a slot's range as held by the lane that later broadcasts it:
+// lane li (< U) of the slot holds col_idx[e0 + li].
+template <int U>
+__device__ __forceinline__ int32_t first_cols(const LocalParams &p, int64_t e0, int64_t e1, const Lane &ln) {
+    return (ln.li < U && e0 + ln.li < e1) ? __ldg(p.col_idx + e0 + ln.li) : -1;
+}
+
+// One slot walks the CSR entries [e0, e1) U at a time (the trip count is the warp's
+// maximum over slots); `cols` holds the first step's column indices (first_cols).
+// On return each lane holds its slot's partial state for its feature vectors.
 template <typename T, int VPL, int U>
-__device__ __forceinline__ void warp_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
-                                           int64_t e0, int64_t e1, const Lane &ln,
+__device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
+                                           int64_t e0, int64_t e1, int32_t cols, const Lane &ln,
                                            State<T, VPL> &st) {
     constexpr int VE = Io<T>::VE;
     st.init();
-    const int per_iter = p.epw * U;
+    const int iters_mine = e1 > e0 ? static_cast<int>((e1 - e0 + U - 1) / U) : 0;
+    const int iters = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(iters_mine));
     const uint4 *KV = static_cast<const uint4 *>(p.KV);
     const int64_t row_vecs = 2 * static_cast<int64_t>(p.nvec);
-    for (int64_t base = e0; base < e1; base += per_iter) {
-        int32_t myc = -1;
-        if (ln.lane < per_iter && base + ln.lane < e1) myc = __ldg(p.col_idx + base + ln.lane);
+    const int src0 = ln.slot * p.lpe;
+    int32_t c_next = cols;
+    for (int it = 0; it < iters; ++it) {
+        const int32_t c_cur = c_next;
+        const int64_t nb = e0 + static_cast<int64_t>(it + 1) * U;
+        c_next = (ln.li < U && nb + ln.li < e1) ? __ldg(p.col_idx + nb + ln.li) : -1;
         int32_t j[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) j[u] = __shfl_sync(0xffffffffu, myc, u * p.epw + ln.slot);
+        for (int u = 0; u < U; ++u) j[u] = __shfl_sync(0xffffffffu, c_cur, src0 + u);
         uint4 kr[U][VPL], vr[U][VPL];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -194,7 +214,13 @@ __device__ __forceinline__ void warp_edges(const LocalParams &p, const float (&q
             st.m[v] = mn;
         }
     }
-    // merge the edge slots of the warp (lanes li, li + LPE, li + 2 LPE, ...)
+}
+
+// Merges the edge slots of the warp (lanes li, li + LPE, ...): afterwards every lane
+// holds the state over all slots.
+template <typename T, int VPL>
+__device__ __forceinline__ void merge_slots(const LocalParams &p, State<T, VPL> &st) {
+    constexpr int VE = Io<T>::VE;
     for (int o = p.lpe; o < 32; o <<= 1) {
 #pragma unroll
         for (int v = 0; v < VPL; ++v) {
@@ -209,23 +235,30 @@ __device__ __forceinline__ void warp_edges(const LocalParams &p, const float (&q
 }
 
 template <typename T, int VPL>
-__device__ __forceinline__ void load_q(const LocalParams &p, int64_t row, const Lane &ln,
-                                       float (&q)[VPL][Io<T>::VE]) {
+__device__ __forceinline__ void load_q_raw(const LocalParams &p, int64_t row, const Lane &ln, bool ok,
+                                           uint4 (&qr)[VPL]) {
     const uint4 *Q = static_cast<const uint4 *>(p.Q) + row * p.nvec;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
         const int vid = v * 32 + ln.li;
-        uint4 u = vid < p.nvec ? __ldg(Q + vid) : make_uint4(0, 0, 0, 0);
-        Io<T>::unpack(u, q[v]);
+        qr[v] = (ok && vid < p.nvec) ? __ldg(Q + vid) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+template <typename T, int VPL>
+__device__ __forceinline__ void scale_q(const LocalParams &p, const uint4 (&qr)[VPL], float (&q)[VPL][Io<T>::VE]) {
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        Io<T>::unpack(qr[v], q[v]);
 #pragma unroll
         for (int e = 0; e < Io<T>::VE; ++e) q[v][e] *= p.score_scale;   // log2(e)/sqrt(r) folded in
     }
 }
 
-// L_i = acc / l per head (0 for a row without edges); stores L[row] (slot-0 lanes).
+// L_i = acc / l per head (0 for a row without edges); stores L[row] from `slot`'s lanes.
 template <typename T, int VPL>
-__device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row,
-                                           const State<T, VPL> &st, const Lane &ln) {
+__device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, const State<T, VPL> &st,
+                                           const Lane &ln, int slot) {
     constexpr int VE = Io<T>::VE;
     uint4 *Lout = static_cast<uint4 *>(p.L) + row * p.nvec;
 #pragma unroll
@@ -235,7 +268,7 @@ __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row,
         float y[VE];
 #pragma unroll
         for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l;
-        if (vid < p.nvec && ln.slot == 0) Lout[vid] = Io<T>::pack(y);
+        if (vid < p.nvec && ln.slot == slot) Lout[vid] = Io<T>::pack(y);
     }
 }
 
@@ -245,19 +278,21 @@ struct BlockScratch {
     float m[kLocalWarps][VPL][32];
     float l[kLocalWarps][VPL][32];
     float acc[kLocalWarps][VPL][VE][32];
-    int flag;
 };
 
-// 8 warps split [e0, e1); warp 0 returns the merge of all warps (warp order).
+// 8 warps split [e0, e1) (each warp's share split again across its slots); warp 0
+// returns the merge of all warps in warp order.
 template <typename T, int VPL, int U>
 __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
                                             int64_t e0, int64_t e1, const Lane &ln, int warp,
                                             BlockScratch<T, VPL> &sh, State<T, VPL> &st) {
     constexpr int VE = Io<T>::VE;
-    const int64_t len = e1 - e0;
-    const int64_t per = ceil_div(len, kLocalWarps);
+    const int64_t per = ceil_div(e1 - e0, kLocalWarps);
     const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
-    warp_edges<T, VPL, U>(p, q, a, b, ln, st);
+    const int64_t per_s = ceil_div(b - a, p.epw);
+    const int64_t sa = std::min(b, a + ln.slot * per_s), sb = std::min(b, sa + per_s);
+    slot_edges<T, VPL, U>(p, q, sa, sb, first_cols<U>(p, sa, sb, ln), ln, st);
+    merge_slots<T, VPL>(p, st);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
         sh.m[warp][v][ln.lane] = st.m[v];
@@ -290,6 +325,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     ln.li = ln.lane % p.lpe;
     int64_t bid = blockIdx.x;
     float q[VPL][VE];
+    uint4 qr[VPL];
     State<T, VPL> st;
 
     if (bid < p.n_chunks) {
@@ -301,7 +337,8 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         const int64_t e1 = std::min<int64_t>(re, e0 + p.chunk_edges);
         const int64_t nch = ceil_div(re - rb, p.chunk_edges);
         const int64_t first = c - (e0 - rb) / p.chunk_edges;
-        load_q<T, VPL>(p, row, ln, q);
+        load_q_raw<T, VPL>(p, row, ln, true, qr);
+        scale_q<T, VPL>(p, qr, q);
         block_edges<T, VPL, U>(p, q, e0, e1, ln, warp, sh, st);
         const int64_t stride = 2 * p.H + p.D;
         if (warp == 0) {
@@ -344,7 +381,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                         st.merge(v, __ldcg(src + h), __ldcg(src + p.H + h), a2);
                     }
                 }
-                finish_row<T, VPL>(p, row, st, ln);
+                finish_row<T, VPL>(p, row, st, ln, 0);
             }
         }
         return;
@@ -353,24 +390,68 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     if (bid < p.n_cta) {
         // ---------------- bucket-1 row: one block ----------------
         const int64_t row = p.cta_rows[bid];
-        load_q<T, VPL>(p, row, ln, q);
+        load_q_raw<T, VPL>(p, row, ln, true, qr);
+        scale_q<T, VPL>(p, qr, q);
         block_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
-        if (warp == 0) finish_row<T, VPL>(p, row, st, ln);
+        if (warp == 0) finish_row<T, VPL>(p, row, st, ln, 0);
         return;
     }
     bid -= p.n_cta;
-    // ---------------- bucket-0 rows: one warp each ----------------
-    const int64_t idx = bid * kLocalWarps + warp;
-    if (idx >= p.n_warp) return;
-    const int64_t row = p.warp_rows[idx];
-    load_q<T, VPL>(p, row, ln, q);
-    warp_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, st);
-    finish_row<T, VPL>(p, row, st, ln);
+    // ---------------- bucket-0 task: up to 32 rows, one per slot per step ----------------
+    const int64_t task = bid * kLocalWarps + warp;
+    if (task >= p.n_tasks) return;
+    const int t0 = p.task_start[task];
+    const int n = p.task_start[task + 1] - t0;
+    int32_t myrow = 0, mybeg = 0, myend = 0;
+    if (ln.lane < n) {
+        myrow = __ldg(p.warp_rows + t0 + ln.lane);
+        mybeg = __ldg(p.row_ptr + myrow);
+        myend = __ldg(p.row_ptr + myrow + 1);
+    }
+    const int steps = (n + p.epw - 1) / p.epw;
+    // step 0 prefetch: this slot's first row
+    int k = ln.slot;
+    int32_t row = __shfl_sync(0xffffffffu, myrow, k & 31);
+    int32_t beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
+    int32_t end = __shfl_sync(0xffffffffu, myend, k & 31);
+    if (k >= n) beg = end = 0;
+    load_q_raw<T, VPL>(p, row, ln, k < n, qr);
+    int32_t cols = first_cols<U>(p, beg, end, ln);
+    for (int step = 0; step < steps; ++step) {
+        const bool valid = k < n;
+        const int32_t row_c = row;
+        const int64_t beg_c = beg, end_c = end;
+        const int32_t cols_c = cols;
+        scale_q<T, VPL>(p, qr, q);
+        // prefetch the next step's row while this one's gathers are in flight
+        k += p.epw;
+        row = __shfl_sync(0xffffffffu, myrow, k & 31);
+        beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
+        end = __shfl_sync(0xffffffffu, myend, k & 31);
+        if (k >= n) beg = end = 0;
+        load_q_raw<T, VPL>(p, row, ln, k < n, qr);
+        cols = first_cols<U>(p, beg, end, ln);
+        slot_edges<T, VPL, U>(p, q, beg_c, end_c, cols_c, ln, st);
+        if (valid) {
+            // every slot finishes its own row
+            constexpr int VEc = Io<T>::VE;
+            uint4 *Lout = static_cast<uint4 *>(p.L) + static_cast<int64_t>(row_c) * p.nvec;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const int vid = v * 32 + ln.li;
+                const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
+                float y[VEc];
+#pragma unroll
+                for (int e = 0; e < VEc; ++e) y[e] = st.acc[v][e] * inv_l;
+                if (vid < p.nvec) Lout[vid] = Io<T>::pack(y);
+            }
+        }
+    }
 }
 
 template <typename T, int VPL, int U>
 glga_status launch_local(Ctx *c, const LocalParams &p, cudaStream_t s) {
-    const int64_t blocks = p.n_chunks + p.n_cta + p.warp_blocks;
+    const int64_t blocks = p.n_chunks + p.n_cta + p.task_blocks;
     if (blocks == 0) return GLGA_OK;
     local_kernel<T, VPL, U><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
     GLGA_CUDA(cudaGetLastError());
@@ -393,7 +474,37 @@ glga_status local_setup(Ctx *c) {
             if (e != cudaSuccess) return cuda_fail(e, "ticket init");
         }
     }
-    return st;
+    if (st != GLGA_OK) return st;
+    // bucket-0 tasks: consecutive rows of the (descending-degree) list, at most kTaskRows
+    // rows and about kTaskEdges edges each
+    const int64_t n0 = c->nb[0];
+    std::vector<int32_t> ts(1, 0);
+    if (n0 > 0) {
+        std::vector<int32_t> rp(static_cast<size_t>(c->N) + 1), rows(static_cast<size_t>(n0));
+        cudaError_t e = cudaMemcpy(rp.data(), c->row_ptr, rp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess)
+            e = cudaMemcpy(rows.data(), c->warp_rows, rows.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "task build");
+        int cnt = 0;
+        int64_t edges = 0;
+        for (int64_t i = 0; i < n0; ++i) {
+            const int64_t deg = rp[rows[i] + 1] - rp[rows[i]];
+            if (cnt > 0 && (cnt == kTaskRows || edges + deg > kTaskEdges)) {
+                ts.push_back(static_cast<int32_t>(i));
+                cnt = 0;
+                edges = 0;
+            }
+            ++cnt;
+            edges += deg;
+        }
+        ts.push_back(static_cast<int32_t>(n0));
+    }
+    c->n_tasks = static_cast<int64_t>(ts.size()) - 1;
+    st = dev_alloc(c, reinterpret_cast<void **>(&c->task_start), ts.size() * sizeof(int32_t));
+    if (st != GLGA_OK) return st;
+    cudaError_t e = cudaMemcpy(c->task_start, ts.data(), ts.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "task upload");
+    return GLGA_OK;
 }
 
 glga_status local_run(Ctx *c, cudaStream_t s) {
@@ -401,13 +512,14 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.row_ptr = c->row_ptr;
     p.col_idx = c->col_idx;
     p.warp_rows = c->warp_rows;
+    p.task_start = c->task_start;
     p.cta_rows = c->cta_rows;
     p.chunk_row = c->chunk_row;
     p.chunk_begin = c->chunk_begin;
-    p.n_warp = c->nb[0];
+    p.n_tasks = c->n_tasks;
     p.n_cta = c->nb[1];
     p.n_chunks = c->nb[3];
-    p.warp_blocks = ceil_div(p.n_warp, kLocalWarps);
+    p.task_blocks = ceil_div(p.n_tasks, kLocalWarps);
     p.chunk_edges = c->opts.chunk_edges;
     p.Q = c->Q;
     p.KV = c->KV;
@@ -426,12 +538,17 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.lph = c->r / VE;
     p.score_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->r)));
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
+    // U edges per slot step; U <= LPE so the slot's lanes can hold its column indices
     if (c->io == GLGA_F32) {
-        if (vpl == 1) return launch_local<float, 1, 4>(c, p, s);
+        if (vpl == 1 && lpe >= 4) return launch_local<float, 1, 4>(c, p, s);
+        if (vpl == 1 && lpe == 2) return launch_local<float, 1, 2>(c, p, s);
+        if (vpl == 1) return launch_local<float, 1, 1>(c, p, s);
         if (vpl == 2) return launch_local<float, 2, 2>(c, p, s);
         if (vpl <= 4) return launch_local<float, 4, 1>(c, p, s);
     } else {
-        if (vpl == 1) return launch_local<__nv_bfloat16, 1, 4>(c, p, s);
+        if (vpl == 1 && lpe >= 4) return launch_local<__nv_bfloat16, 1, 4>(c, p, s);
+        if (vpl == 1 && lpe == 2) return launch_local<__nv_bfloat16, 1, 2>(c, p, s);
+        if (vpl == 1) return launch_local<__nv_bfloat16, 1, 1>(c, p, s);
         if (vpl == 2) return launch_local<__nv_bfloat16, 2, 2>(c, p, s);
         if (vpl <= 4) return launch_local<__nv_bfloat16, 4, 1>(c, p, s);
     }

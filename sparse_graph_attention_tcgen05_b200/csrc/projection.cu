@@ -26,7 +26,9 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kRowBytes = 128;            // bytes of K per smem row (one swizzle span)
 constexpr int kMaxStages = 4;
-constexpr int kGemmThreads = 128;
+constexpr int kProdWarp = 8;             // TMA producer
+constexpr int kMmaWarp = 9;              // TMEM owner and MMA issuer
+constexpr int kGemmThreads = 320;        // warps 0-7 drain TMEM in the epilogue
 
 struct GemmParams {
     int64_t M;
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
         mbar_init(&done_bar, 1);
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == kProdWarp && lane == 0) {
         tma_prefetch_desc(&tmA0);
         tma_prefetch_desc(&tmB0);
         if (kPlanes == 2) {
@@ -152,7 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
             tma_prefetch_desc(&tmB1);
         }
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&tmem_base_sh, static_cast<uint32_t>(p.tmem_cols));
         tmem_relinquish();
     }
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 0 && lane == 0) {
+    if (warp == kProdWarp && lane == 0) {
         // ---------------- TMA producer ----------------
         int issued = 0;
         bool ok = true;
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
             for (int kb = std::max(0, issued - p.stages); kb < issued; ++kb)
                 mbar_wait_bounded(&full_bar[kb % p.stages], static_cast<uint32_t>(kb / p.stages) & 1u);
         }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
         // ---------------- MMA issuer ----------------
         const uint32_t idesc = instr_desc(kBM, p.BN, kFmt, false, false);
         bool ok = true;
@@ -224,24 +226,29 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
     }
     __syncwarp();
 
-    // ---------------- epilogue: TMEM -> registers -> Q / KV / t ----------------
-    const bool done = mbar_wait_bounded(&done_bar, 0);
-    tc_fence_after();
-    if (!done) {
-        if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
-    } else {
-        const int64_t row = m0 + warp * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        for (int c0 = 0; c0 < p.BN; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
-            tmem_ld_wait();
-            if (row < p.M) store_row_cols<T>(p, row, n0 + c0, n0 + p.BN, v);
+    // ---------------- epilogue (warps 0-7): TMEM -> registers -> Q / KV / t ----------------
+    // warp w drains TMEM lanes 32*(w%4).. (its rows); warpgroup w/4 takes every other
+    // 32-column chunk
+    if (warp < 8) {
+        const bool done = mbar_wait_bounded(&done_bar, 0);
+        tc_fence_after();
+        if (!done) {
+            if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
+        } else {
+            const int quad = warp & 3, wg = warp >> 2;
+            const int64_t row = m0 + quad * 32 + lane;
+            const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+            for (int c0 = wg * 32; c0 < p.BN; c0 += 64) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
+                tmem_ld_wait();
+                if (row < p.M) store_row_cols<T>(p, row, n0 + c0, n0 + p.BN, v);
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
     }

@@ -8,12 +8,14 @@
 // where B_g (K = hg*r, N = hg*r + hg) holds S_h block-diagonally and z_h in column
 // hg*r + h.  B_g is written by the statistics reduction each forward.
 //
-// Kernel: 128-row tiles, 192 threads.  Warp 4 issues TMA loads of the q tile (128-byte
-// swizzle) and of B_g into an mbarrier ring; warps 0-3 apply phi to the landed q tile in
-// shared memory (for fp32 also splitting it into tf32 hi/lo planes), fence it for the
-// async proxy and arrive on a "ready" barrier; warp 5 issues tcgen05.mma into TMEM.  The
-// epilogue (warps 0-3, one row per thread) divides by the denominators, reads L and the
-// gate logit, blends and writes Y.
+// Kernel: 128-row tiles, 192 threads.  Warp 4 issues TMA loads (128-byte swizzle): the
+// group's L tile once, and the q tile and B_g through an mbarrier ring.  Warps 0-3
+// apply phi to each landed q tile in shared memory (for fp32 also splitting it into tf32
+// hi/lo planes), fence it for the async proxy and arrive on a "ready" barrier; warp 5
+// issues tcgen05.mma into TMEM.  Epilogue (warps 0-3, one row per thread): numerators
+// and denominators from TMEM, L and the blend in shared memory in place, then TMA bulk
+// stores of the Y tile.  Shapes whose head group is not a whole number of 128-byte
+// column boxes fall back to per-thread global loads and stores.
 #include <algorithm>
 
 #include "glga_internal.cuh"
@@ -24,7 +26,11 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kRowBytes = 128;
 constexpr int kMaxStages = 4;
-constexpr int kThreads = 192;
+constexpr int kWorkers = 256;        // warps 0-7: phi pass and epilogue
+constexpr int kProdWarp = 8;         // TMA producer
+constexpr int kMmaWarp = 9;          // TMEM owner and MMA issuer
+constexpr int kThreads = 320;
+constexpr uint32_t kBoxBytes = kBM * kRowBytes;   // one 128-row x 128-byte TMA box
 
 struct ReadoutParams {
     int64_t M;              // rows
@@ -32,6 +38,7 @@ struct ReadoutParams {
     int32_t nk;             // K tiles per group
     int32_t BNr;            // GEMM N per group (>= hg*r + hg, multiple of 16)
     int32_t stages, tmem_cols;
+    int32_t lboxes;         // 128-byte column boxes of the group's L/Y tile (0: no TMA path)
     uint32_t a_bytes, b_bytes, stage_bytes;
     const void *L;          // io [N, D]
     const float *t;         // [N]
@@ -44,19 +51,14 @@ template <typename T>
 struct IoT;
 template <>
 struct IoT<float> {
-    static constexpr int VE = 4;
-    __device__ __forceinline__ static void load32(const float *src, float (&v)[32]) {
-        const float4 *p = reinterpret_cast<const float4 *>(src);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 q = p[i];
-            v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
-        }
+    static constexpr int VE = 4;      // elements per 16 bytes
+    __device__ __forceinline__ static void unpack(const uint4 &u, float *v) {
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
     }
-    __device__ __forceinline__ static void store32(float *dst, const float (&v)[32]) {
-        float4 *p = reinterpret_cast<float4 *>(dst);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    __device__ __forceinline__ static uint4 pack(const float *v) {
+        return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                          __float_as_uint(v[3]));
     }
     __device__ __forceinline__ static float get(const float *p) { return *p; }
     __device__ __forceinline__ static void put(float *p, float x) { *p = x; }
@@ -64,41 +66,28 @@ struct IoT<float> {
 template <>
 struct IoT<__nv_bfloat16> {
     static constexpr int VE = 8;
-    __device__ __forceinline__ static void load32(const __nv_bfloat16 *src, float (&v)[32]) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(src);
+    __device__ __forceinline__ static void unpack(const uint4 &u, float *v) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 q = p[i];
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
-                v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-            }
+        for (int k = 0; k < 4; ++k) {
+            v[2 * k] = __uint_as_float(w[k] << 16);
+            v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
         }
     }
-    __device__ __forceinline__ static void store32(__nv_bfloat16 *dst, const float (&v)[32]) {
-        uint4 *p = reinterpret_cast<uint4 *>(dst);
+    __device__ __forceinline__ static uint4 pack(const float *v) {
+        uint32_t w[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
-                w[k] = *reinterpret_cast<uint32_t *>(&h);
-            }
-            p[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+            w[k] = *reinterpret_cast<uint32_t *>(&h);
         }
+        return make_uint4(w[0], w[1], w[2], w[3]);
     }
     __device__ __forceinline__ static float get(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
     __device__ __forceinline__ static void put(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 };
 
-__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : expf(x); }
-
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
+__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 // phi applied in place to one 16-byte chunk of the q tile (bf16: 8 values).
 __device__ __forceinline__ void phi_chunk_bf16(uint4 *p) {
@@ -132,39 +121,45 @@ template <int SPLIT, typename T, int R>
 __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                               const __grid_constant__ CUtensorMap tmB0,
                                                               const __grid_constant__ CUtensorMap tmB1,
+                                                              const __grid_constant__ CUtensorMap tmL,
+                                                              const __grid_constant__ CUtensorMap tmY,
                                                               ReadoutParams p) {
     constexpr int kPlanes = SPLIT == 3 ? 2 : 1;
     constexpr int kPairs = SPLIT == 3 ? 3 : 1;
     constexpr uint32_t kFmt = SPLIT == 3 ? 2u : 1u;
-    constexpr int KT = kRowBytes / static_cast<int>(sizeof(T));   // K elements per tile row
+    constexpr int KT = kRowBytes / static_cast<int>(sizeof(T));   // elements per tile row
+    constexpr int VE = IoT<T>::VE;
+    constexpr int kChunks32 = 32 / VE;                              // 16-byte chunks per 32 columns
 
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t ready_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
     __shared__ __align__(8) uint64_t done_bar;
+    __shared__ __align__(8) uint64_t l_bar;
     __shared__ uint32_t tmem_base_sh;
-    __shared__ float sinv[kBM][33];
 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *lbuf = smem + static_cast<size_t>(p.stages) * p.stage_bytes;   // L, then Y, tile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = blockIdx.x;                          // head group
     const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
     const int h0 = g * p.hg;
     const int hg = std::min(p.hg, p.D / R - h0);       // heads in this group
-    const int qx0 = h0 * R;                            // first q column of the group
+    const int qx0 = h0 * R;                            // first q / L / Y column of the group
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&ready_bar[s], 128);
+            mbar_init(&ready_bar[s], kWorkers);
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&done_bar, 1);
+        mbar_init(&l_bar, 1);
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&tmem_base_sh, static_cast<uint32_t>(p.tmem_cols));
         tmem_relinquish();
     }
@@ -173,9 +168,14 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 4) {
+    if (warp == kProdWarp) {
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
+            if (p.lboxes > 0) {
+                mbar_arrive_expect_tx(&l_bar, p.lboxes * kBoxBytes);
+                for (int b = 0; b < p.lboxes; ++b)
+                    tma_load_2d(lbuf + b * kBoxBytes, &tmL, &l_bar, qx0 + b * KT, static_cast<int32_t>(m0));
+            }
             int issued = 0;
             bool ok = true;
             for (int kb = 0; kb < p.nk; ++kb) {
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                     mbar_wait_bounded(&full_bar[kb % p.stages], static_cast<uint32_t>(kb / p.stages) & 1u);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         if (lane == 0) {
             const uint32_t idesc = instr_desc(kBM, p.BNr, kFmt, false, false);
             bool ok = true;
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
             umma_commit(&done_bar);
         }
     } else {
-        // ---------------- warps 0-3: phi on the landed q tiles ----------------
+        // ---------------- warps 0-7: phi on the landed q tiles ----------------
         bool ok = true;
         for (int kb = 0; kb < p.nk && ok; ++kb) {
             const int s = kb % p.stages;
@@ -245,10 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                 break;
             }
             uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
-            // thread t owns row t of the tile: 8 chunks of 16 bytes
-            uint4 *row = reinterpret_cast<uint4 *>(st + threadIdx.x * kRowBytes);
+            // threads 2t and 2t+1 own row t of the tile: 4 chunks of 16 bytes each
+            uint4 *row = reinterpret_cast<uint4 *>(st + (threadIdx.x >> 1) * kRowBytes) + (threadIdx.x & 1) * 4;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 if (SPLIT == 3) {
                     float4 *hi = reinterpret_cast<float4 *>(row + c);
                     float4 *lo = reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(row + c) + p.a_bytes);
@@ -257,63 +257,80 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                     phi_chunk_bf16(row + c);
                 }
             }
-            fence_async_smem();
+            fence_proxy_async_smem();
             mbar_arrive(&ready_bar[s]);
         }
         if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
     }
     __syncwarp();
 
-    if (warp < 4) {
+    if (warp < 8) {
         // ---------------- epilogue: G = num / (den + eps), blend with L, write Y ----------------
+        // warp w reads TMEM lanes 32*(w%4).. (its rows); warpgroup w/4 takes every other
+        // 32-column chunk
         const bool done = mbar_wait_bounded(&done_bar, 0);
+        const bool lok = p.lboxes == 0 || mbar_wait_bounded(&l_bar, 0);
         tc_fence_after();
-        if (!done) {
+        const int quad = warp & 3, wg = warp >> 2;
+        const int rt = quad * 32 + lane;
+        const int64_t row = m0 + rt;
+        const bool live = row < p.M;
+        if (!done || !lok) {
             if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
         } else {
-            const int rt = warp * 32 + lane;
-            const int64_t row = m0 + rt;
-            const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(hg * R), v);   // denominators
-            tmem_ld_wait();
-#pragma unroll
-            for (int h = 0; h < 32; ++h)
-                if (h < hg) sinv[rt][h] = 1.f / (__uint_as_float(v[h]) + p.eps);
-            const bool live = row < p.M;
+            const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
             const float gt = live ? __ldg(p.t + row) + p.b_g : 0.f;
-            const float gate = 1.f / (1.f + expf(-gt));
-            const T *L = static_cast<const T *>(p.L) + row * p.D + qx0;
-            T *Y = static_cast<T *>(p.Y) + row * p.D + qx0;
+            const float gate = 1.f / (1.f + __expf(-gt));
             const int ncol = hg * R;
-            for (int c0 = 0; c0 < ncol; c0 += 32) {
+            for (int c0 = wg * 32; c0 < ncol; c0 += 64) {
+                uint32_t v[32], dv[32];
                 tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
+                // denominators of the heads this chunk touches: column hg*R + head
+                tmem_ld32(tmem + lane_base + static_cast<uint32_t>(ncol + c0 / R), dv);
                 tmem_ld_wait();
-                if (!live) continue;
-                if (c0 + 32 <= ncol) {
-                    float lv[32], y[32];
-                    IoT<T>::load32(L + c0, lv);
+                float gv[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float Gv = __uint_as_float(v[j]) * sinv[rt][(c0 + j) / R];
-                        y[j] = gate * lv[j] + (1.f - gate) * Gv;
-                    }
-                    IoT<T>::store32(Y + c0, y);
-                } else {
+                for (int j = 0; j < 32; ++j)
+                    gv[j] = (1.f - gate) * __uint_as_float(v[j]) /
+                            (__uint_as_float(dv[R >= 32 ? 0 : j / R]) + p.eps);
+                if (p.lboxes > 0) {
+                    // L from the swizzled shared tile, Y written back in place
+                    const int b = c0 / KT, e0 = c0 % KT;
+                    uint8_t *base = lbuf + b * kBoxBytes + rt * kRowBytes;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (c0 + j < ncol) {
-                            const float Gv = __uint_as_float(v[j]) * sinv[rt][(c0 + j) / R];
-                            IoT<T>::put(Y + c0 + j, gate * IoT<T>::get(L + c0 + j) + (1.f - gate) * Gv);
-                        }
+                    for (int q = 0; q < kChunks32; ++q) {
+                        const int ch = (e0 / VE + q) ^ (rt & 7);
+                        uint4 *pch = reinterpret_cast<uint4 *>(base + ch * 16);
+                        float lv[VE], y[VE];
+                        IoT<T>::unpack(*pch, lv);
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) y[e] = gate * lv[e] + gv[q * VE + e];
+                        *pch = IoT<T>::pack(y);
                     }
+                } else if (live) {
+                    const T *L = static_cast<const T *>(p.L) + row * p.D + qx0;
+                    T *Y = static_cast<T *>(p.Y) + row * p.D + qx0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < ncol)
+                            IoT<T>::put(Y + c0 + j, gate * IoT<T>::get(L + c0 + j) + gv[j]);
                 }
+            }
+        }
+        if (p.lboxes > 0) {
+            fence_proxy_async_smem();
+            named_barrier_sync(1, kWorkers);
+            if (threadIdx.x == 0 && done && lok) {
+                for (int b = 0; b < p.lboxes; ++b)
+                    tma_store_2d(&tmY, lbuf + b * kBoxBytes, qx0 + b * KT, static_cast<int32_t>(m0));
+                bulk_commit_group();
+                bulk_wait_group_read0();
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
     }
@@ -321,14 +338,15 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
 
 template <int SPLIT, typename T>
 glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, size_t smem, const CUtensorMap &q,
-                             const CUtensorMap &b0, const CUtensorMap &b1, cudaStream_t s) {
+                             const CUtensorMap &b0, const CUtensorMap &b1, const CUtensorMap &ml,
+                             const CUtensorMap &my, cudaStream_t s) {
     dim3 grid(static_cast<unsigned>(p.n_groups), static_cast<unsigned>(ceil_div(p.M, kBM)));
 #define GLGA_RO(RR)                                                                              \
     case RR: {                                                                                   \
         auto kern = readout_kernel<SPLIT, T, RR>;                                                \
         GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
                                        static_cast<int>(smem)));                                 \
-        kern<<<grid, kThreads, smem, s>>>(q, b0, b1, p);                                         \
+        kern<<<grid, kThreads, smem, s>>>(q, b0, b1, ml, my, p);                                 \
         break;                                                                                   \
     }
     switch (p.r) {
@@ -345,11 +363,15 @@ glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, size_t smem, const 
 
 glga_status readout_setup(Ctx *c) {
     const int kt = kRowBytes / c->elem;
-    const int hg_max = std::max(1, 224 / c->r);
+    // hg*r + hg + 32 <= 256: numerators, denominators and the 32-column read past them
+    // fit one 256-column TMEM allocation
+    const int hg_max = std::max(1, 224 / (c->r + 1));
     c->ro_groups = static_cast<int32_t>(ceil_div(c->H, hg_max));
     c->ro_hg = static_cast<int32_t>(ceil_div(c->H, c->ro_groups));
     c->ro_kp = static_cast<int32_t>(ceil_div(static_cast<int64_t>(c->ro_hg) * c->r, kt) * kt);
     c->ro_bn = static_cast<int32_t>(ceil_div(c->ro_hg * c->r + c->ro_hg, 16) * 16);
+    const int last = c->H - (c->ro_groups - 1) * c->ro_hg;
+    c->ro_tma_epi = (c->ro_hg * c->r) % kt == 0 && (last * c->r) % kt == 0;
     const int planes = c->split == 3 ? 2 : 1;
     const size_t plane = static_cast<size_t>(c->ro_groups) * c->ro_bn * c->ro_kp * c->elem;
     glga_status st = dev_alloc(c, &c->Bro, planes * plane);
@@ -365,13 +387,16 @@ glga_status readout_setup(Ctx *c) {
         if (st != GLGA_OK) return st;
         c->tmBro[pl].valid = true;
     }
+    st = dev_alloc(c, &c->L, static_cast<size_t>(c->N) * c->D * c->elem);
+    if (st != GLGA_OK) return st;
     if (c->N > 0) {
-        st = encode_tmap_2d(&c->tmQ.map, dt, c->Q, c->D, c->N, static_cast<uint64_t>(c->D) * c->elem,
-                            kt, kBM);
+        const uint64_t rb = static_cast<uint64_t>(c->D) * c->elem;
+        st = encode_tmap_2d(&c->tmQ.map, dt, c->Q, c->D, c->N, rb, kt, kBM);
+        if (st == GLGA_OK) st = encode_tmap_2d(&c->tmL.map, dt, c->L, c->D, c->N, rb, kt, kBM);
         if (st != GLGA_OK) return st;
-        c->tmQ.valid = true;
+        c->tmQ.valid = c->tmL.valid = true;
     }
-    return dev_alloc(c, &c->L, static_cast<size_t>(c->N) * c->D * c->elem);
+    return GLGA_OK;
 }
 
 glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
@@ -385,25 +410,37 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     p.n_groups = c->ro_groups;
     p.nk = c->ro_kp / kt;
     p.BNr = c->ro_bn;
-    // the epilogue reads 32 columns starting at the first denominator column
+    // the epilogue reads 32 columns starting at a denominator column (<= hg*r + hg - 1)
     int tc = 32;
-    while (tc < p.BNr || tc < p.hg * p.r + 32) tc <<= 1;
+    while (tc < p.BNr || tc < p.hg * p.r + p.hg + 32) tc <<= 1;
     p.tmem_cols = tc;
     const int planes = c->split == 3 ? 2 : 1;
     p.a_bytes = kBM * kRowBytes;
     p.b_bytes = static_cast<uint32_t>(p.BNr) * kRowBytes;
     p.stage_bytes = planes * (p.a_bytes + p.b_bytes);
-    p.stages = std::max(1, std::min(std::min(p.nk, kMaxStages), static_cast<int>((200u * 1024u) / p.stage_bytes)));
+    p.lboxes = c->ro_tma_epi ? static_cast<int32_t>(ceil_div(static_cast<int64_t>(p.hg) * p.r, kt)) : 0;
+    const uint32_t lbytes = static_cast<uint32_t>(p.lboxes) * kBoxBytes;
+    p.stages = std::max(1, std::min(std::min(p.nk, kMaxStages),
+                                    static_cast<int>((200u * 1024u - lbytes) / p.stage_bytes)));
     p.L = c->L;
     p.t = c->t;
     p.Y = Y;
     p.b_g = b_g;
     p.eps = eps;
     p.flag = c->dev_flag;
-    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + 1024;
+    const CUtensorMapDataType dt =
+        c->io == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap my = c->tmL.map;   // placeholder when the TMA store path is off
+    if (p.lboxes > 0) {
+        glga_status st = encode_tmap_2d(&my, dt, Y, c->D, c->N, static_cast<uint64_t>(c->D) * c->elem,
+                                        kt, kBM);
+        if (st != GLGA_OK) return st;
+    }
+    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + lbytes + 1024;
     const CUtensorMap &b1 = planes == 2 ? c->tmBro[1].map : c->tmBro[0].map;
-    if (c->io == GLGA_F32) return launch_readout_r<3, float>(c, p, smem, c->tmQ.map, c->tmBro[0].map, b1, s);
-    return launch_readout_r<1, __nv_bfloat16>(c, p, smem, c->tmQ.map, c->tmBro[0].map, b1, s);
+    if (c->io == GLGA_F32)
+        return launch_readout_r<3, float>(c, p, smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
+    return launch_readout_r<1, __nv_bfloat16>(c, p, smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
 }
 
 }  // namespace glga

@@ -4,6 +4,7 @@
 // The target-grouped CSR is the form the tinymesh page ("Sparse attention experiment",
 // section "Target softmax") reduces over: one row per destination.  Everything here is
 // integer work and deterministic; its results are compared bit for bit with the oracle.
+#include <algorithm>
 #include <cstdio>
 #include <vector>
 
@@ -231,6 +232,21 @@ glga_status build_buckets(Ctx *c, cudaStream_t s) {
         if (e != cudaSuccess) st = cuda_fail(e, "bucket scatter");
     }
     cudaFree(scratch);
+    // Bucket 0 by descending degree, ties by ascending row: rows of similar degree share a
+    // warp task and the heaviest start first.
+    if (st == GLGA_OK && h[0] > 1) {
+        std::vector<int32_t> rp(static_cast<size_t>(N) + 1), rows(static_cast<size_t>(h[0]));
+        cudaError_t e = cudaMemcpy(rp.data(), c->row_ptr, rp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess)
+            e = cudaMemcpy(rows.data(), c->warp_rows, rows.size() * sizeof(int32_t), cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess) {
+            std::stable_sort(rows.begin(), rows.end(), [&rp](int32_t a, int32_t b) {
+                return rp[a + 1] - rp[a] > rp[b + 1] - rp[b];
+            });
+            e = cudaMemcpy(c->warp_rows, rows.data(), rows.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+        }
+        if (e != cudaSuccess) st = cuda_fail(e, "bucket-0 order");
+    }
     return st;
 }
 

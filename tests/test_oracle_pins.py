@@ -379,7 +379,9 @@ def test_buckets_partition_rows_and_edges(warp_max, chunk):
     rp, _ = oracle.csr_from_coo(w.N, w.src, w.dst)
     b = oracle.degree_buckets(rp, warp_max, chunk)
     deg = np.diff(rp)
-    np.testing.assert_array_equal(b["warp_rows"], np.nonzero(deg <= warp_max)[0])
+    small = np.nonzero(deg <= warp_max)[0]
+    # bucket 0: descending degree, ties by ascending row (numpy's stable lexsort)
+    np.testing.assert_array_equal(b["warp_rows"], small[np.lexsort((small, -deg[small]))])
     np.testing.assert_array_equal(b["cta_rows"], np.nonzero((deg > warp_max) & (deg <= chunk))[0])
     np.testing.assert_array_equal(b["split_rows"], np.nonzero(deg > chunk)[0])
     # chunks tile every split row's edges exactly once, in order
