@@ -72,7 +72,9 @@ struct Ctx {
     // projection
     int32_t dp = 0;               // padded input width (multiple of the K tile)
     int32_t Dp = 0;               // padded GEMM width: 3*D + gate column + padding
-    int32_t BN = 0, n_tiles = 0, stages = 0, tmem_cols = 0;
+    int32_t BN = 0, bn_last = 0, n_tiles = 0, stages = 0, tmem_cols = 0;
+    bool gemm_tma_epi = false;    // Q/K/V stored through shared memory + TMA
+    TensorMap2D tmKVs;            // KV store map (64-column boxes)
     int split = 1;                // 1: bf16 MMA; 3: 3-term tf32 split (fp32 io)
     bool x_direct = false;        // A operand read straight from the caller's X
     void *Wt = nullptr;           // [planes][Dp][dp]
@@ -222,6 +224,10 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_group_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Waits until at most the most recently committed bulk-store group is still reading.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 // Orders this thread's generic-proxy shared-memory writes before later async-proxy
 // (TMA, tcgen05) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -229,6 +235,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also returns the OR of `pred` over the participating threads.
+__device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "barrier.cta.red.or.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {

@@ -32,8 +32,13 @@ constexpr int kGemmThreads = 320;        // warps 0-7 drain TMEM in the epilogue
 
 struct GemmParams {
     int64_t M;
+    int64_t n_total_tiles;   // m-tiles x n-tiles
+    int32_t n_tiles;         // column tiles
     int32_t nk;          // K tiles
-    int32_t BN;          // columns per CTA (multiple of 16, <= 256)
+    int32_t BN;          // columns per tile (multiple of 16, <= 256)
+    int32_t bn_last;     // columns of the last column tile (BN, or BN + 16 with the gate)
+    int32_t tma_epi;     // 1: Q/K/V leave through smem + TMA stores (BN multiple of 64)
+    uint32_t stage_area; // bytes of the stage ring (staging buffers follow it)
     int32_t stages;
     int32_t tmem_cols;
     int32_t D;
@@ -116,11 +121,17 @@ __device__ __forceinline__ void store_row_cols(const GemmParams &p, int64_t row,
     }
 }
 
+// Persistent: CTA b walks tiles b, b + gridDim.x, ... (tile t = m-tile t / n_tiles,
+// n-tile t % n_tiles).  The producer streams every K block of every tile through the
+// stage ring; the MMA warp accumulates tile i into TMEM buffer i & 1 (256 columns each)
+// once the epilogue has drained that buffer's previous tile; warps 0-7 drain buffer
+// i & 1 while tile i + 1 accumulates in the other one.
 // SPLIT = 1: bf16 operands, one MMA per K step.  SPLIT = 3: tf32 hi/lo planes.
 template <int SPLIT, typename T>
-__global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
+__global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+    const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmKVs,
     GemmParams p) {
     constexpr int kPlanes = SPLIT == 3 ? 2 : 1;
     constexpr int kPairs = SPLIT == 3 ? 3 : 1;
@@ -129,21 +140,26 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
-    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ __align__(8) uint64_t accf_bar[2];    // MMA -> epilogue: buffer holds a tile
+    __shared__ __align__(8) uint64_t acce_bar[2];    // epilogue -> MMA: buffer drained
     __shared__ uint32_t tmem_base_sh;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * p.BN;
-    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+    const int64_t n_my = p.n_total_tiles > blockIdx.x
+                             ? (p.n_total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x
+                             : 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&done_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf_bar[b], 1);
+            mbar_init(&acce_bar[b], 8);
+        }
         fence_mbar_init();
     }
     if (warp == kProdWarp && lane == 0) {
@@ -164,65 +180,83 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
     const uint32_t tmem = tmem_base_sh;
 
     if (warp == kProdWarp && lane == 0) {
-        // ---------------- TMA producer ----------------
-        int issued = 0;
+        // ---------------- TMA producer: every K block of every tile of this CTA ----------
+        int64_t it = 0;       // global K-block counter (stage ring position)
         bool ok = true;
-        for (int kb = 0; kb < p.nk; ++kb) {
-            const int s = kb % p.stages;
-            const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
-            if (kb >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
-                ok = false;
-                break;
+        for (int64_t i = 0; i < n_my && ok; ++i) {
+            const int64_t tile = blockIdx.x + i * gridDim.x;
+            const int32_t m0 = static_cast<int32_t>((tile / p.n_tiles) * kBM);
+            const int32_t n0 = static_cast<int32_t>((tile % p.n_tiles) * p.BN);
+            for (int kb = 0; kb < p.nk; ++kb, ++it) {
+                const int s = static_cast<int>(it % p.stages);
+                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
+                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+                mbar_arrive_expect_tx(&full_bar[s], p.stage_bytes);
+                const int kx = kb * (kRowBytes / static_cast<int>(sizeof(T)));
+                tma_load_2d(st, &tmA0, &full_bar[s], kx, m0);
+                if (kPlanes == 2) tma_load_2d(st + p.a_bytes, &tmA1, &full_bar[s], kx, m0);
+                uint8_t *bst = st + kPlanes * p.a_bytes;
+                tma_load_2d(bst, &tmB0, &full_bar[s], kx, n0);
+                if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kx, n0);
             }
-            uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
-            mbar_arrive_expect_tx(&full_bar[s], p.stage_bytes);
-            const int kx = kb * (kRowBytes / static_cast<int>(sizeof(T)));
-            tma_load_2d(st, &tmA0, &full_bar[s], kx, static_cast<int32_t>(m0));
-            if (kPlanes == 2) tma_load_2d(st + p.a_bytes, &tmA1, &full_bar[s], kx, static_cast<int32_t>(m0));
-            uint8_t *bst = st + kPlanes * p.a_bytes;
-            tma_load_2d(bst, &tmB0, &full_bar[s], kx, n0);
-            if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kx, n0);
-            ++issued;
         }
         if (!ok) {
             atomicOr(p.flag, kDevErrTimeout);
             // let the copies already in flight land before the block can exit
-            for (int kb = std::max(0, issued - p.stages); kb < issued; ++kb)
-                mbar_wait_bounded(&full_bar[kb % p.stages], static_cast<uint32_t>(kb / p.stages) & 1u);
+            for (int64_t k = std::max<int64_t>(0, it - p.stages); k < it; ++k)
+                mbar_wait_bounded(&full_bar[k % p.stages], static_cast<uint32_t>(k / p.stages) & 1u);
         }
     } else if (warp == kMmaWarp && lane == 0) {
         // ---------------- MMA issuer ----------------
-        const uint32_t idesc = instr_desc(kBM, p.BN, kFmt, false, false);
+        const uint32_t idesc_main = instr_desc(kBM, p.BN, kFmt, false, false);
+        const uint32_t idesc_last = instr_desc(kBM, p.bn_last, kFmt, false, false);
         bool ok = true;
-        for (int kb = 0; kb < p.nk; ++kb) {
-            const int s = kb % p.stages;
-            const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
-            if (!mbar_wait_bounded(&full_bar[s], ph)) {
+        int64_t it = 0;
+        for (int64_t i = 0; i < n_my && ok; ++i) {
+            const int buf = static_cast<int>(i & 1);
+            const uint32_t acc_col = static_cast<uint32_t>(buf * 256);
+            const int64_t tile = blockIdx.x + i * gridDim.x;
+            const uint32_t idesc = (tile % p.n_tiles == p.n_tiles - 1) ? idesc_last : idesc_main;
+            // wait until the epilogue drained this buffer's previous tile (tile i - 2)
+            if (i >= 2 && !mbar_wait_bounded(&acce_bar[buf], static_cast<uint32_t>((i >> 1) - 1) & 1u)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
-            const uint32_t b_addr = a_addr + kPlanes * p.a_bytes;
-#pragma unroll
-            for (int k = 0; k < kRowBytes / 32; ++k) {
-#pragma unroll
-                for (int pr = 0; pr < kPairs; ++pr) {
-                    const uint32_t ap = (pr == 2) ? 1u : 0u;   // (hi,hi) (hi,lo) (lo,hi)
-                    const uint32_t bp = (pr == 1) ? 1u : 0u;
-                    const uint64_t ad = smem_desc(a_addr + ap * p.a_bytes + k * 32, 16, 1024, 2);
-                    const uint64_t bd = smem_desc(b_addr + bp * p.b_bytes + k * 32, 16, 1024, 2);
-                    const uint32_t acc = (kb | k | pr) != 0;
-                    if (SPLIT == 3)
-                        umma_tf32(tmem, ad, bd, idesc, acc);
-                    else
-                        umma_bf16(tmem, ad, bd, idesc, acc);
+            for (int kb = 0; kb < p.nk; ++kb, ++it) {
+                const int s = static_cast<int>(it % p.stages);
+                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
+                if (!mbar_wait_bounded(&full_bar[s], ph)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
+                const uint32_t b_addr = a_addr + kPlanes * p.a_bytes;
+#pragma unroll
+                for (int k = 0; k < kRowBytes / 32; ++k) {
+#pragma unroll
+                    for (int pr = 0; pr < kPairs; ++pr) {
+                        const uint32_t ap = (pr == 2) ? 1u : 0u;   // (hi,hi) (hi,lo) (lo,hi)
+                        const uint32_t bp = (pr == 1) ? 1u : 0u;
+                        const uint64_t ad = smem_desc(a_addr + ap * p.a_bytes + k * 32, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(b_addr + bp * p.b_bytes + k * 32, 16, 1024, 2);
+                        const uint32_t acc = (kb | k | pr) != 0;
+                        if (SPLIT == 3)
+                            umma_tf32(tmem + acc_col, ad, bd, idesc, acc);
+                        else
+                            umma_bf16(tmem + acc_col, ad, bd, idesc, acc);
+                    }
+                }
+                umma_commit(&empty_bar[s]);   // stage reusable once these MMAs finish
             }
-            umma_commit(&empty_bar[s]);
+            if (ok) umma_commit(&accf_bar[buf]);   // the tile's accumulator is complete
         }
         if (!ok) atomicOr(p.flag, kDevErrTimeout);
-        umma_commit(&done_bar);   // arrives once every MMA issued above has completed
     }
     __syncwarp();
 
@@ -230,21 +264,84 @@ __global__ void __launch_bounds__(kGemmThreads) proj_gemm_kernel(
     // warp w drains TMEM lanes 32*(w%4).. (its rows); warpgroup w/4 takes every other
     // 32-column chunk
     if (warp < 8) {
-        const bool done = mbar_wait_bounded(&done_bar, 0);
-        tc_fence_after();
-        if (!done) {
-            if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
-        } else {
-            const int quad = warp & 3, wg = warp >> 2;
-            const int64_t row = m0 + quad * 32 + lane;
-            const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-            for (int c0 = wg * 32; c0 < p.BN; c0 += 64) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
-                tmem_ld_wait();
-                if (row < p.M) store_row_cols<T>(p, row, n0 + c0, n0 + p.BN, v);
+        const int quad = warp & 3, wg = warp >> 2;
+        const int rt = quad * 32 + lane;                 // row inside the tile
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t box_bytes = kBM * kRowBytes;      // one 128-row x 64-column bf16 box
+        const int nbox = p.BN / 64;
+        bool ok = true;
+        for (int64_t i = 0; i < n_my; ++i) {
+            const int buf = static_cast<int>(i & 1);
+            const bool got = mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(i >> 1) & 1u);
+            // the 8 epilogue warps must agree before the named barriers below
+            const bool fail = p.tma_epi ? named_barrier_or(1, 256, !got) : !got;
+            if (fail) {
+                if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int64_t tile = blockIdx.x + i * gridDim.x;
+            const int64_t m0 = (tile / p.n_tiles) * kBM;
+            const int64_t row = m0 + rt;
+            const int ntile = static_cast<int>(tile % p.n_tiles);
+            const int n0 = ntile * p.BN;
+            const int bn = ntile == p.n_tiles - 1 ? p.bn_last : p.BN;
+            if (p.tma_epi) {
+                // Q/K/V columns go through staging buffer `buf`; its previous TMA store
+                // (tile i - 2) must have finished reading it first
+                uint8_t *sb = smem + p.stage_area + static_cast<size_t>(buf) * nbox * box_bytes;
+                if (threadIdx.x == 0) bulk_wait_group_read1();
+                named_barrier_sync(1, 256);
+                for (int c0 = wg * 32; c0 < bn; c0 += 64) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + c0), v);
+                    tmem_ld_wait();
+                    if (c0 < p.BN) {
+                        const int b = c0 / 64, e0 = (c0 % 64) / 8;
+                        uint8_t *rp = sb + b * box_bytes + rt * kRowBytes;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                            w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                            w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                            w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                            *reinterpret_cast<uint4 *>(rp + (((e0 + q) ^ (rt & 7)) * 16)) = w;
+                        }
+                    } else if (row < p.M) {
+                        p.t[row] = __uint_as_float(v[0]);   // gate logit column
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce_bar[buf]);
+                fence_proxy_async_smem();
+                named_barrier_sync(1, 256);
+                if (threadIdx.x == 0) {
+                    for (int b = 0; b < nbox; ++b) {
+                        const int gc = n0 + b * 64;
+                        if (gc < p.D)
+                            tma_store_2d(&tmQs, sb + b * box_bytes, gc, static_cast<int32_t>(m0));
+                        else
+                            tma_store_2d(&tmKVs, sb + b * box_bytes, gc - p.D, static_cast<int32_t>(m0));
+                    }
+                    bulk_commit_group();
+                }
+            } else {
+                for (int c0 = wg * 32; c0 < bn; c0 += 64) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + c0), v);
+                    tmem_ld_wait();
+                    if (row < p.M) store_row_cols<T>(p, row, n0 + c0, n0 + bn, v);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce_bar[buf]);
             }
         }
+        (void)ok;
+        if (p.tma_epi && threadIdx.x == 0) bulk_wait_group_read0();
     }
     tc_fence_before();
     __syncthreads();
@@ -340,27 +437,36 @@ template <int SPLIT, typename T>
 glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     GemmParams p;
     p.M = c->N;
+    p.n_tiles = c->n_tiles;
+    p.n_total_tiles = ceil_div(c->N, kBM) * c->n_tiles;
     p.nk = c->dp / (kRowBytes / c->elem);
     p.BN = c->BN;
+    p.bn_last = c->bn_last;
+    p.tma_epi = c->gemm_tma_epi ? 1 : 0;
     p.stages = c->stages;
-    p.tmem_cols = c->tmem_cols;
+    p.tmem_cols = c->tmem_cols;   // two 256-column accumulators
     p.D = c->D;
     const int planes = SPLIT == 3 ? 2 : 1;
     p.a_bytes = kBM * kRowBytes;
-    p.b_bytes = static_cast<uint32_t>(c->BN) * kRowBytes;
+    p.b_bytes = static_cast<uint32_t>(c->bn_last) * kRowBytes;
     p.stage_bytes = planes * (p.a_bytes + p.b_bytes);
+    p.stage_area = static_cast<uint32_t>(p.stages) * p.stage_bytes;
     p.Q = c->Q;
     p.KV = c->KV;
     p.t = c->t;
     p.flag = c->dev_flag;
-    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + 1024;
+    const uint32_t staging = p.tma_epi ? 2u * (c->BN / 64) * kBM * kRowBytes : 0u;
+    const size_t smem = static_cast<size_t>(p.stage_area) + staging + 1024;
     auto kern = proj_gemm_kernel<SPLIT, T>;
     GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(smem)));
-    dim3 grid(static_cast<unsigned>(c->n_tiles), static_cast<unsigned>(ceil_div(c->N, kBM)));
+    // persistent: one CTA per SM (it holds all 512 TMEM columns)
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(p.n_total_tiles, c->num_sms));
     const CUtensorMap &a1 = planes == 2 ? c->tmA[1].map : c->tmA[0].map;
     const CUtensorMap &b1 = planes == 2 ? c->tmB[1].map : c->tmB[0].map;
-    kern<<<grid, kGemmThreads, smem, s>>>(c->tmA[0].map, a1, c->tmB[0].map, b1, p);
+    const CUtensorMap &qs = c->gemm_tma_epi ? c->tmQ.map : c->tmB[0].map;      // unused otherwise
+    const CUtensorMap &kvs = c->gemm_tma_epi ? c->tmKVs.map : c->tmB[0].map;
+    kern<<<grid, kGemmThreads, smem, s>>>(c->tmA[0].map, a1, c->tmB[0].map, b1, qs, kvs, p);
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -400,21 +506,37 @@ glga_status projection_setup(Ctx *c) {
     c->split = (c->io == GLGA_F32) ? 3 : 1;
     const int kt = kRowBytes / c->elem;                  // K elements per tile row
     c->dp = static_cast<int32_t>(ceil_div(c->d, kt) * kt);
-    const int Dp = 3 * c->D + 1;
-    c->n_tiles = static_cast<int32_t>(ceil_div(Dp, 256));
-    c->BN = static_cast<int32_t>(ceil_div(ceil_div(Dp, c->n_tiles), 16) * 16);
-    c->Dp = c->n_tiles * c->BN;
-    int tc = 32;
-    while (tc < c->BN) tc <<= 1;
-    c->tmem_cols = tc;
+    const int D3 = 3 * c->D;
+    c->gemm_tma_epi = false;
+    if (c->split == 1 && c->D % 64 == 0) {
+        // Column tiles of BN (a multiple of the 64-column store box) over Q | K | V; the
+        // last tile also carries the gate column (+15 zero columns).  Q/K/V leave through
+        // shared memory and TMA stores.
+        c->BN = 64;
+        for (int bn = 192; bn >= 64; bn -= 64)
+            if (D3 % bn == 0) {
+                c->BN = bn;
+                break;
+            }
+        c->n_tiles = D3 / c->BN;
+        c->bn_last = c->BN + 16;
+        c->Dp = D3 + 16;
+        c->gemm_tma_epi = true;
+    } else {
+        const int Dp = D3 + 1;
+        c->n_tiles = static_cast<int32_t>(ceil_div(Dp, 256));
+        c->BN = static_cast<int32_t>(ceil_div(ceil_div(Dp, c->n_tiles), 16) * 16);
+        c->bn_last = c->BN;
+        c->Dp = c->n_tiles * c->BN;
+    }
+    c->tmem_cols = 512;
     const int planes = c->split == 3 ? 2 : 1;
-    const uint32_t stage_bytes = planes * (kBM * kRowBytes + c->BN * kRowBytes);
-    const int nk = c->dp / kt;
-    // two CTAs per SM for bf16 (epilogue of one overlaps the loads of the other)
-    const uint32_t budget = (c->split == 3) ? 200u * 1024u : 110u * 1024u;
+    const uint32_t stage_bytes = planes * (kBM * kRowBytes + c->bn_last * kRowBytes);
+    const uint32_t staging = c->gemm_tma_epi ? 2u * (c->BN / 64) * kBM * kRowBytes : 0u;
+    // one persistent CTA per SM: as many ring stages as fit (loads run ahead across tiles)
+    const uint32_t budget = 200u * 1024u - staging;
     int st = static_cast<int>(budget / stage_bytes);
-    st = std::max(1, std::min(st, kMaxStages));
-    c->stages = std::min(st, std::max(nk, 1));
+    c->stages = std::max(1, std::min(st, kMaxStages));
 
     const size_t wt_bytes = static_cast<size_t>(planes) * c->Dp * c->dp * c->elem;
     glga_status r = dev_alloc(c, &c->Wt, wt_bytes);
@@ -425,9 +547,15 @@ glga_status projection_setup(Ctx *c) {
         const uint8_t *base = static_cast<const uint8_t *>(c->Wt) +
                               static_cast<size_t>(pl) * c->Dp * c->dp * c->elem;
         r = encode_tmap_2d(&c->tmB[pl].map, dt, base, c->dp, c->Dp,
-                           static_cast<uint64_t>(c->dp) * c->elem, kt, c->BN);
+                           static_cast<uint64_t>(c->dp) * c->elem, kt, c->bn_last);
         if (r != GLGA_OK) return r;
         c->tmB[pl].valid = true;
+    }
+    if (c->gemm_tma_epi && c->N > 0) {
+        r = encode_tmap_2d(&c->tmKVs.map, dt, c->KV, 2 * static_cast<uint64_t>(c->D), c->N,
+                           2 * static_cast<uint64_t>(c->D) * c->elem, 64, kBM);
+        if (r != GLGA_OK) return r;
+        c->tmKVs.valid = true;
     }
     // The A operand is read from the caller's X when it is bf16 with 16-byte rows;
     // otherwise from a padded (and, for fp32, split) copy.
