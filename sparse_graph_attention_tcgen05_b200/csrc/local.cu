@@ -75,9 +75,10 @@ struct Io<__nv_bfloat16> {
     }
 };
 
+// volatile: the load must stay under its guard (it is never speculated)
 __device__ __forceinline__ uint4 ld_gather(const void *p) {
     uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
         : "l"(p));
     return r;
@@ -168,6 +169,7 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q
             for (int v = 0; v < VPL; ++v) {
                 const int vid = v * 32 + ln.li;
                 if (j[u] >= 0 && vid < p.nvec) {
+                    // (a masked-off slot never forms an address: j < 0 takes the else branch)
                     const uint4 *rowp = KV + static_cast<int64_t>(j[u]) * row_vecs;
                     kr[u][v] = ld_gather(rowp + vid);
                     vr[u][v] = ld_gather(rowp + p.nvec + vid);
