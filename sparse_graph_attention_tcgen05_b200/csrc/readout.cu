@@ -364,8 +364,9 @@ glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, size_t smem, const 
 glga_status readout_setup(Ctx *c) {
     const int kt = kRowBytes / c->elem;
     // hg*r + hg + 32 <= 256: numerators, denominators and the 32-column read past them
-    // fit one 256-column TMEM allocation
-    const int hg_max = std::max(1, 224 / (c->r + 1));
+    // fit one 256-column TMEM allocation.  Groups span at most 128 columns (one head for
+    // r >= 64): narrower groups let more CTAs share an SM and overlap their phases.
+    const int hg_max = std::max(1, std::min(224 / (c->r + 1), (c->r >= 64 ? 64 : 128) / c->r));
     c->ro_groups = static_cast<int32_t>(ceil_div(c->H, hg_max));
     c->ro_hg = static_cast<int32_t>(ceil_div(c->H, c->ro_groups));
     c->ro_kp = static_cast<int32_t>(ceil_div(static_cast<int64_t>(c->ro_hg) * c->r, kt) * kt);
