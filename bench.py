@@ -44,6 +44,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks_dist(x, world, device):
+    """The largest value of x over all ranks (every rank gets it); x itself at world 1."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world, units_per_rank, slowest_total_ms, steps):
+    """Whole-job units per second when every rank runs `steps` steps of `units_per_rank`
+    units and the slowest rank took `slowest_total_ms` for them."""
+    return world * units_per_rank * steps / (slowest_total_ms * 1e-3)
+
+
 def local_bytes_model(N, E, D, H, r, s):
     """Algorithmic bytes of the fused per-target kernel: CSR (row_ptr, col_idx), one k_j and
     v_j row gather per edge, q_i and Y_i once per row, the gate logit, and S, z."""
@@ -210,11 +227,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_dist(x, world, dev)
 
     w = make_workload(args.workload, scale=args.scale)
     dt = glga.torch_dtype(w.io)
@@ -293,7 +306,7 @@ def main():
 
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / args.steps
-    value = world * w.E * w.H / (ms_per_step * 1e-3)
+    value = replica_throughput(world, w.E * w.H, total_ms, args.steps)
     stages = {k: v / args.steps for k, v in stage_sum.items()}
 
     # ---- end to end through the public API: pinned host -> device, forward, Y -> host ----
@@ -314,8 +327,9 @@ def main():
         ev1.synchronize()
         if i >= 3:
             e2e_ms.append(ev0.elapsed_time(ev1))
-    e2e_step = max_over_ranks(sum(e2e_ms)) / len(e2e_ms)
-    e2e = {"value": world * w.E * w.H / (e2e_step * 1e-3), "unit": UNIT,
+    e2e_total = max_over_ranks(sum(e2e_ms))
+    e2e_step = e2e_total / len(e2e_ms)
+    e2e = {"value": replica_throughput(world, w.E * w.H, e2e_total, len(e2e_ms)), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
 
     peaks, peak_kind = load_peaks()
