@@ -183,19 +183,65 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after about
-// `limit_ns` nanoseconds of wall time (checked every 256 polls) or 2^26 polls, whichever
-// comes first, and returns false; the caller records the timeout and winds down.
+// As mbar_try_wait, but a thread whose phase is still open may be suspended for up to
+// `hint_ns` nanoseconds (or until the phase completes) instead of the hardware's
+// default window, so a waiting warp takes no issue slots while it waits.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Each poll may suspend the
+// thread for up to 1 ms; gives up after about `limit_ns` nanoseconds of wall time or
+// 2^26 polls, whichever comes first, and returns false; the caller records the timeout
+// and winds down.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns = 1000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1; it < (1u << 26); ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+        if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
 }
+
+// Position in a ring of n mbarrier-guarded slots: the slot and the parity of the
+// current pass over the ring, advanced without divisions.
+struct RingPos {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++slot == n) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+// Walks the tiles start, start + step, start + 2 step, ... of a row-major grid with
+// `cols` tiles per row, keeping (row, col) by increments instead of divisions.
+struct TileWalk {
+    int32_t row, col, step_row, step_col, cols;
+    __device__ __forceinline__ TileWalk(int32_t start, int32_t step, int32_t cols_)
+        : row(start / cols_), col(start % cols_), step_row(step / cols_), step_col(step % cols_),
+          cols(cols_) {}
+    __device__ __forceinline__ void next() {
+        col += step_col;
+        row += step_row;
+        if (col >= cols) {
+            col -= cols;
+            ++row;
+        }
+    }
+};
 
 // 2-D tiled TMA load global -> shared, completing on an mbarrier (no multicast).
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
@@ -334,6 +380,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
           "=r"(v[31])
         : "r"(taddr)
         : "memory");
+}
+// TMEM -> registers: 32 lanes x N (1, 2 or 4) consecutive 32-bit columns.
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&v)[N]) {
+    static_assert(N == 1 || N == 2 || N == 4, "tmem_ld_n: 1, 2 or 4 columns");
+    if constexpr (N == 1) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
+                     : "=r"(v[0]) : "r"(taddr) : "memory");
+    } else if constexpr (N == 2) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+                     : "=r"(v[0]), "=r"(v[1]) : "r"(taddr) : "memory");
+    } else {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(taddr) : "memory");
+    }
 }
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");

@@ -109,11 +109,11 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             int issued = 0;
+            RingPos rp;
             bool ok = true;
-            for (int it = 0; it < ntiles; ++it) {
-                const int s = it % p.stages;
-                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
-                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+            for (int it = 0; it < ntiles; ++it, rp.next(p.stages)) {
+                const int s = rp.slot;
+                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
                     ok = false;
                     break;
                 }
@@ -142,10 +142,10 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             const uint32_t idZk = instr_desc(128, 16, kFmt, false, false);
             const uint64_t dones = smem_desc(smem_u32(ones), 16, 1024, 2);
             bool ok = true;
-            for (int it = 0; it < ntiles; ++it) {
-                const int s = it % p.stages;
-                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
-                if (!mbar_wait_bounded(&ready_bar[s], ph)) {
+            RingPos rp;
+            for (int it = 0; it < ntiles; ++it, rp.next(p.stages)) {
+                const int s = rp.slot;
+                if (!mbar_wait_bounded(&ready_bar[s], rp.phase)) {
                     ok = false;
                     break;
                 }
@@ -188,10 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
         // ---------------- warps 0-3: phi(K) (zero past the range), tf32 split ----------
         bool ok = true;
         constexpr int kChunksPerBox = G::kBoxBytes / 16;
-        for (int it = 0; it < ntiles && ok; ++it) {
-            const int s = it % p.stages;
-            const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
-            if (!mbar_wait_bounded(&full_bar[s], ph)) {
+        RingPos rp;
+        for (int it = 0; it < ntiles && ok; ++it, rp.next(p.stages)) {
+            const int s = rp.slot;
+            if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
                 ok = false;
                 break;
             }

@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n_my = p.n_total_tiles > blockIdx.x
-                             ? (p.n_total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x
+    const int32_t n_my = p.n_total_tiles > blockIdx.x
+                             ? static_cast<int32_t>((p.n_total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x)
                              : 0;
 
     if (threadIdx.x == 0) {
@@ -181,16 +181,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
 
     if (warp == kProdWarp && lane == 0) {
         // ---------------- TMA producer: every K block of every tile of this CTA ----------
-        int64_t it = 0;       // global K-block counter (stage ring position)
+        int it = 0;           // K blocks issued so far
+        RingPos rp;           // stage ring position
+        TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
         bool ok = true;
-        for (int64_t i = 0; i < n_my && ok; ++i) {
-            const int64_t tile = blockIdx.x + i * gridDim.x;
-            const int32_t m0 = static_cast<int32_t>((tile / p.n_tiles) * kBM);
-            const int32_t n0 = static_cast<int32_t>((tile % p.n_tiles) * p.BN);
-            for (int kb = 0; kb < p.nk; ++kb, ++it) {
-                const int s = static_cast<int>(it % p.stages);
-                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
-                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+        for (int i = 0; i < n_my && ok; ++i, tw.next()) {
+            const int32_t m0 = tw.row * kBM;
+            const int32_t n0 = tw.col * p.BN;
+            for (int kb = 0; kb < p.nk; ++kb, ++it, rp.next(p.stages)) {
+                const int s = rp.slot;
+                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
                     ok = false;
                     break;
                 }
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         if (!ok) {
             atomicOr(p.flag, kDevErrTimeout);
             // let the copies already in flight land before the block can exit
-            for (int64_t k = std::max<int64_t>(0, it - p.stages); k < it; ++k)
+            for (int k = std::max(0, it - p.stages); k < it; ++k)
                 mbar_wait_bounded(&full_bar[k % p.stages], static_cast<uint32_t>(k / p.stages) & 1u);
         }
     } else if (warp == kMmaWarp && lane == 0) {
@@ -215,22 +215,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         const uint32_t idesc_main = instr_desc(kBM, p.BN, kFmt, false, false);
         const uint32_t idesc_last = instr_desc(kBM, p.bn_last, kFmt, false, false);
         bool ok = true;
-        int64_t it = 0;
-        for (int64_t i = 0; i < n_my && ok; ++i) {
-            const int buf = static_cast<int>(i & 1);
+        RingPos rp;
+        TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
+        for (int i = 0; i < n_my && ok; ++i, tw.next()) {
+            const int buf = i & 1;
             const uint32_t acc_col = static_cast<uint32_t>(buf * 256);
-            const int64_t tile = blockIdx.x + i * gridDim.x;
-            const uint32_t idesc = (tile % p.n_tiles == p.n_tiles - 1) ? idesc_last : idesc_main;
+            const uint32_t idesc = (tw.col == p.n_tiles - 1) ? idesc_last : idesc_main;
             // wait until the epilogue drained this buffer's previous tile (tile i - 2)
             if (i >= 2 && !mbar_wait_bounded(&acce_bar[buf], static_cast<uint32_t>((i >> 1) - 1) & 1u)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            for (int kb = 0; kb < p.nk; ++kb, ++it) {
-                const int s = static_cast<int>(it % p.stages);
-                const uint32_t ph = static_cast<uint32_t>(it / p.stages) & 1u;
-                if (!mbar_wait_bounded(&full_bar[s], ph)) {
+            for (int kb = 0; kb < p.nk; ++kb, rp.next(p.stages)) {
+                const int s = rp.slot;
+                if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
                     ok = false;
                     break;
                 }
@@ -270,8 +269,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         const uint32_t box_bytes = kBM * kRowBytes;      // one 128-row x 64-column bf16 box
         const int nbox = p.BN / 64;
         bool ok = true;
-        for (int64_t i = 0; i < n_my; ++i) {
-            const int buf = static_cast<int>(i & 1);
+        TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
+        for (int i = 0; i < n_my; ++i, tw.next()) {
+            const int buf = i & 1;
             const bool got = mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(i >> 1) & 1u);
             // the 8 epilogue warps must agree before the named barriers below
             const bool fail = p.tma_epi ? named_barrier_or(1, 256, !got) : !got;
@@ -281,10 +281,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 break;
             }
             tc_fence_after();
-            const int64_t tile = blockIdx.x + i * gridDim.x;
-            const int64_t m0 = (tile / p.n_tiles) * kBM;
+            const int64_t m0 = static_cast<int64_t>(tw.row) * kBM;
             const int64_t row = m0 + rt;
-            const int ntile = static_cast<int>(tile % p.n_tiles);
+            const int ntile = tw.col;
             const int n0 = ntile * p.BN;
             const int bn = ntile == p.n_tiles - 1 ? p.bn_last : p.BN;
             if (p.tma_epi) {

@@ -8,14 +8,21 @@
 // where B_g (K = hg*r, N = hg*r + hg) holds S_h block-diagonally and z_h in column
 // hg*r + h.  B_g is written by the statistics reduction each forward.
 //
-// Kernel: 128-row tiles, 192 threads.  Warp 4 issues TMA loads (128-byte swizzle): the
-// group's L tile once, and the q tile and B_g through an mbarrier ring.  Warps 0-3
-// apply phi to each landed q tile in shared memory (for fp32 also splitting it into tf32
-// hi/lo planes), fence it for the async proxy and arrive on a "ready" barrier; warp 5
-// issues tcgen05.mma into TMEM.  Epilogue (warps 0-3, one row per thread): numerators
-// and denominators from TMEM, L and the blend in shared memory in place, then TMA bulk
-// stores of the Y tile.  Shapes whose head group is not a whole number of 128-byte
-// column boxes fall back to per-thread global loads and stores.
+// Persistent kernel, one CTA per SM walking (row tile, head group) tiles round-robin;
+// W worker warps (a multiple of 4) and three single-thread roles:
+//   warp W     TMA producer: the q tile's K blocks through an mbarrier ring (and B_g's,
+//              unless B_g is resident)
+//   warp W+1   MMA issuer: accumulates tile i into TMEM buffer i & 1 (256 columns each)
+//   warp W+2   TMA producer: the group's L tile into one of 2-3 L/Y buffers
+//   warps 0..W-1  phi on each landed q block (fp32: also the tf32 hi/lo split), then the
+//              epilogue of the previous tile: numerators and denominators from TMEM, the
+//              blend with L and the gate in shared memory, TMA bulk stores of Y
+// so the loads and MMAs of tile i overlap the epilogue of tile i - 1.  When the grid is
+// a multiple of the number of head groups every CTA keeps one group, and B_g (a few tens
+// of KB) is loaded once and stays in shared memory.  The Y stores of a tile are waited
+// for one tile later, when their buffer is handed back to the L producer.  Shapes whose
+// head group is not a whole number of 128-byte column boxes use per-thread global loads
+// and stores in the epilogue instead of the L/Y buffers.
 #include <algorithm>
 
 #include "glga_internal.cuh"
@@ -25,21 +32,32 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kRowBytes = 128;
-constexpr int kMaxStages = 4;
-constexpr int kWorkers = 256;        // warps 0-7: phi pass and epilogue
-constexpr int kProdWarp = 8;         // TMA producer
-constexpr int kMmaWarp = 9;          // TMEM owner and MMA issuer
-constexpr int kThreads = 320;
+constexpr int kMaxStages = 8;
+constexpr int kWorkerWarps = 16;     // phi pass and epilogue
+constexpr int kWorkers = kWorkerWarps * 32;
+constexpr int kWG = kWorkerWarps / 4;         // worker warpgroups (TMEM lane quarters x kWG)
+constexpr int kTPR = kWorkers / 128;          // phi-pass threads per tile row
+constexpr int kProdWarp = kWorkerWarps;       // TMA producer (q, B_g)
+constexpr int kMmaWarp = kWorkerWarps + 1;    // TMEM owner and MMA issuer
+constexpr int kLWarp = kWorkerWarps + 2;      // L tile loader
+constexpr int kThreads = kWorkers + 96;
+constexpr int kMaxLBufs = 3;
+static_assert(kWorkerWarps % 4 == 0 && 8 % kTPR == 0, "worker warps: 4, 8 or 16");
 constexpr uint32_t kBoxBytes = kBM * kRowBytes;   // one 128-row x 128-byte TMA box
+constexpr uint32_t kAccCols = 256;                // TMEM columns per accumulator buffer
 
 struct ReadoutParams {
     int64_t M;              // rows
+    int64_t n_total;        // row tiles x head groups
     int32_t D, r, hg, n_groups;
     int32_t nk;             // K tiles per group
     int32_t BNr;            // GEMM N per group (>= hg*r + hg, multiple of 16)
-    int32_t stages, tmem_cols;
+    int32_t stages;
     int32_t lboxes;         // 128-byte column boxes of the group's L/Y tile (0: no TMA path)
+    int32_t lbufs;          // L/Y staging buffers (2 or 3)
+    int32_t b_resident;     // B_g loaded once per CTA (grid is a multiple of n_groups)
     uint32_t a_bytes, b_bytes, stage_bytes;
+    uint32_t bres_bytes;    // resident B_g: planes x nk x b_bytes (0 when streamed)
     const void *L;          // io [N, D]
     const float *t;         // [N]
     void *Y;                // io [N, D]
@@ -130,37 +148,53 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
     constexpr int KT = kRowBytes / static_cast<int>(sizeof(T));   // elements per tile row
     constexpr int VE = IoT<T>::VE;
     constexpr int kChunks32 = 32 / VE;                              // 16-byte chunks per 32 columns
+    constexpr int kHeads = R >= 32 ? 1 : 32 / R;                    // heads per 32 columns
+    constexpr int kCPT = 8 / kTPR;                                  // phi chunks per thread and row
 
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t ready_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
-    __shared__ __align__(8) uint64_t done_bar;
-    __shared__ __align__(8) uint64_t l_bar;
+    __shared__ __align__(8) uint64_t accf_bar[2];    // MMA -> epilogue: accumulator complete
+    __shared__ __align__(8) uint64_t acce_bar[2];    // epilogue -> MMA: accumulator drained
+    __shared__ __align__(8) uint64_t lfull_bar[kMaxLBufs];   // L tile landed in buffer b
+    __shared__ __align__(8) uint64_t lfree_bar[kMaxLBufs];   // Y stores finished reading b
+    __shared__ __align__(8) uint64_t bres_bar;       // resident B_g landed
+    __shared__ __align__(8) uint64_t drain_bar;      // error path: issued MMAs retired
     __shared__ uint32_t tmem_base_sh;
 
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
+    // shared memory: [resident B_g][K ring: stages x stage_bytes][L/Y: lbufs x lbytes]
+    uint8_t *bres = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t *lbuf = smem + static_cast<size_t>(p.stages) * p.stage_bytes;   // L, then Y, tile
+    uint8_t *smem = bres + p.bres_bytes;
+    const uint32_t lbytes = static_cast<uint32_t>(p.lboxes) * kBoxBytes;
+    uint8_t *lbase = smem + static_cast<size_t>(p.stages) * p.stage_bytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = blockIdx.x;                          // head group
-    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
-    const int h0 = g * p.hg;
-    const int hg = std::min(p.hg, p.D / R - h0);       // heads in this group
-    const int qx0 = h0 * R;                            // first q / L / Y column of the group
+    const int32_t n_my = p.n_total > blockIdx.x
+                             ? static_cast<int32_t>((p.n_total - blockIdx.x + gridDim.x - 1) / gridDim.x)
+                             : 0;
+    const uint32_t a_planes = kPlanes * p.a_bytes;   // q part of a ring stage
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&ready_bar[s], kWorkers);
+            mbar_init(&ready_bar[s], kWorkerWarps);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&done_bar, 1);
-        mbar_init(&l_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf_bar[b], 1);
+            mbar_init(&acce_bar[b], kWorkerWarps);
+        }
+        for (int b = 0; b < kMaxLBufs; ++b) {
+            mbar_init(&lfull_bar[b], 1);
+            mbar_init(&lfree_bar[b], 1);
+        }
+        mbar_init(&bres_bar, 1);
+        mbar_init(&drain_bar, 1);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(&tmem_base_sh, static_cast<uint32_t>(p.tmem_cols));
+        tmem_alloc(&tmem_base_sh, 2 * kAccCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -171,176 +205,277 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
     if (warp == kProdWarp) {
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
-            if (p.lboxes > 0) {
-                mbar_arrive_expect_tx(&l_bar, p.lboxes * kBoxBytes);
-                for (int b = 0; b < p.lboxes; ++b)
-                    tma_load_2d(lbuf + b * kBoxBytes, &tmL, &l_bar, qx0 + b * KT, static_cast<int32_t>(m0));
+            if (p.b_resident && n_my > 0) {
+                // every tile of this CTA belongs to head group blockIdx.x % n_groups
+                const int g = static_cast<int>(blockIdx.x % p.n_groups);
+                mbar_arrive_expect_tx(&bres_bar, p.bres_bytes);
+                for (int kb = 0; kb < p.nk; ++kb) {
+                    uint8_t *dst = bres + static_cast<size_t>(kb) * kPlanes * p.b_bytes;
+                    tma_load_2d(dst, &tmB0, &bres_bar, kb * KT, g * p.BNr);
+                    if (kPlanes == 2) tma_load_2d(dst + p.b_bytes, &tmB1, &bres_bar, kb * KT, g * p.BNr);
+                }
             }
-            int issued = 0;
+            int it = 0;
+            RingPos rp;
+            TileWalk tw(blockIdx.x, gridDim.x, p.n_groups);
             bool ok = true;
-            for (int kb = 0; kb < p.nk; ++kb) {
-                const int s = kb % p.stages;
-                const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
-                if (kb >= p.stages && !mbar_wait_bounded(&empty_bar[s], ph ^ 1u)) {
+            for (int i = 0; i < n_my && ok; ++i, tw.next()) {
+                const int g = tw.col;
+                const int32_t m0 = tw.row * kBM;
+                const int qx0 = g * p.hg * R;
+                for (int kb = 0; kb < p.nk; ++kb, ++it, rp.next(p.stages)) {
+                    const int s = rp.slot;
+                    if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+                    // TMA brings the raw q box (the fp32 lo plane is written by the
+                    // phi pass) and, when streamed, B_g's K block
+                    mbar_arrive_expect_tx(&full_bar[s], p.b_resident ? p.a_bytes
+                                                                     : p.a_bytes + kPlanes * p.b_bytes);
+                    tma_load_2d(st, &tmQ, &full_bar[s], qx0 + kb * KT, m0);
+                    if (!p.b_resident) {
+                        uint8_t *bst = st + a_planes;
+                        tma_load_2d(bst, &tmB0, &full_bar[s], kb * KT, g * p.BNr);
+                        if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kb * KT, g * p.BNr);
+                    }
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA can exit
+                atomicOr(p.flag, kDevErrTimeout);
+                for (int q = std::max(0, it - p.stages); q < it; ++q)
+                    mbar_wait_bounded(&full_bar[q % p.stages], static_cast<uint32_t>(q / p.stages) & 1u);
+                if (p.b_resident) mbar_wait_bounded(&bres_bar, 0);
+            }
+        }
+    } else if (warp == kLWarp) {
+        if (lane == 0 && p.lboxes > 0) {
+            // the L tile of tile i goes into buffer i % lbufs once the Y stores of tile
+            // i - lbufs have been read out of it
+            tma_prefetch_desc(&tmL);
+            int i = 0;
+            RingPos lp;
+            TileWalk tw(blockIdx.x, gridDim.x, p.n_groups);
+            bool ok = true;
+            for (; i < n_my; ++i, lp.next(p.lbufs), tw.next()) {
+                const int b = lp.slot;
+                if (i >= p.lbufs && !mbar_wait_bounded(&lfree_bar[b], lp.phase ^ 1u)) {
                     ok = false;
                     break;
                 }
-                uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
-                const uint32_t tx = p.a_bytes + kPlanes * p.b_bytes;
-                mbar_arrive_expect_tx(&full_bar[s], tx);
-                tma_load_2d(st, &tmQ, &full_bar[s], qx0 + kb * KT, static_cast<int32_t>(m0));
-                uint8_t *bst = st + kPlanes * p.a_bytes;
-                tma_load_2d(bst, &tmB0, &full_bar[s], kb * KT, g * p.BNr);
-                if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kb * KT, g * p.BNr);
-                ++issued;
+                const int g = tw.col;
+                const int32_t m0 = tw.row * kBM;
+                mbar_arrive_expect_tx(&lfull_bar[b], lbytes);
+                for (int bx = 0; bx < p.lboxes; ++bx)
+                    tma_load_2d(lbase + b * lbytes + bx * kBoxBytes, &tmL, &lfull_bar[b],
+                                g * p.hg * R + bx * KT, m0);
             }
             if (!ok) {
                 atomicOr(p.flag, kDevErrTimeout);
-                for (int kb = std::max(0, issued - p.stages); kb < issued; ++kb)
-                    mbar_wait_bounded(&full_bar[kb % p.stages], static_cast<uint32_t>(kb / p.stages) & 1u);
+                for (int q = std::max(0, i - p.lbufs); q < i; ++q)
+                    mbar_wait_bounded(&lfull_bar[q % p.lbufs], static_cast<uint32_t>(q / p.lbufs) & 1u);
             }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
             const uint32_t idesc = instr_desc(kBM, p.BNr, kFmt, false, false);
-            bool ok = true;
-            for (int kb = 0; kb < p.nk; ++kb) {
-                const int s = kb % p.stages;
-                const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
-                if (!mbar_wait_bounded(&ready_bar[s], ph)) {
+            RingPos rp;
+            bool ok = !p.b_resident || n_my == 0 || mbar_wait_bounded(&bres_bar, 0);
+            const uint32_t bres_addr = smem_u32(bres);
+            for (int i = 0; i < n_my && ok; ++i) {
+                const int buf = static_cast<int>(i & 1);
+                if (i >= 2 && !mbar_wait_bounded(&acce_bar[buf], static_cast<uint32_t>((i >> 1) - 1) & 1u)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
-                const uint32_t b_addr = a_addr + kPlanes * p.a_bytes;
-#pragma unroll
-                for (int k = 0; k < kRowBytes / 32; ++k) {
-#pragma unroll
-                    for (int pr = 0; pr < kPairs; ++pr) {
-                        const uint32_t ap = (pr == 2) ? 1u : 0u;
-                        const uint32_t bp = (pr == 1) ? 1u : 0u;
-                        const uint64_t ad = smem_desc(a_addr + ap * p.a_bytes + k * 32, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(b_addr + bp * p.b_bytes + k * 32, 16, 1024, 2);
-                        const uint32_t acc = (kb | k | pr) != 0;
-                        if (SPLIT == 3)
-                            umma_tf32(tmem, ad, bd, idesc, acc);
-                        else
-                            umma_bf16(tmem, ad, bd, idesc, acc);
+                const uint32_t dcol = tmem + static_cast<uint32_t>(buf) * kAccCols;
+                for (int kb = 0; kb < p.nk; ++kb, rp.next(p.stages)) {
+                    const int s = rp.slot;
+                    if (!mbar_wait_bounded(&ready_bar[s], rp.phase)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
+                    const uint32_t b_addr = p.b_resident
+                                                ? bres_addr + static_cast<uint32_t>(kb) * kPlanes * p.b_bytes
+                                                : a_addr + a_planes;
+#pragma unroll
+                    for (int k = 0; k < kRowBytes / 32; ++k) {
+#pragma unroll
+                        for (int pr = 0; pr < kPairs; ++pr) {
+                            const uint32_t ap = (pr == 2) ? 1u : 0u;
+                            const uint32_t bp = (pr == 1) ? 1u : 0u;
+                            const uint64_t ad = smem_desc(a_addr + ap * p.a_bytes + k * 32, 16, 1024, 2);
+                            const uint64_t bd = smem_desc(b_addr + bp * p.b_bytes + k * 32, 16, 1024, 2);
+                            const uint32_t acc = (kb | k | pr) != 0;
+                            if (SPLIT == 3)
+                                umma_tf32(dcol, ad, bd, idesc, acc);
+                            else
+                                umma_bf16(dcol, ad, bd, idesc, acc);
+                        }
+                    }
+                    umma_commit(&empty_bar[s]);
                 }
-                umma_commit(&empty_bar[s]);
+                if (ok) umma_commit(&accf_bar[buf]);
             }
-            if (!ok) atomicOr(p.flag, kDevErrTimeout);
-            umma_commit(&done_bar);
+            if (!ok) {
+                // drain the MMAs already issued before TMEM is released
+                atomicOr(p.flag, kDevErrTimeout);
+                umma_commit(&drain_bar);
+                mbar_wait_bounded(&drain_bar, 0);
+            }
         }
     } else {
-        // ---------------- warps 0-7: phi on the landed q tiles ----------------
+        // ------------ worker warps: phi of tile i, then the epilogue of tile i - 1 ------------
+        const int quad = warp & 3, wg = warp >> 2;
+        const int rt = quad * 32 + lane;                 // epilogue row inside the tile
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        const int trow = threadIdx.x / kTPR;             // phi-pass row
+        const int tpart = threadIdx.x % kTPR;
+        float t_prev = 0.f;                              // gate logit of tile i - 1's row
+        RingPos rp, lp;                                  // K ring; L/Y buffers (epilogue)
+        int lp_prev = 0;                                 // L/Y buffer of the previous epilogue
+        TileWalk tw(blockIdx.x, gridDim.x, p.n_groups);   // tile i (phi pass)
+        TileWalk te = tw;                                // tile i - 1 (epilogue)
         bool ok = true;
-        for (int kb = 0; kb < p.nk && ok; ++kb) {
-            const int s = kb % p.stages;
-            const uint32_t ph = static_cast<uint32_t>(kb / p.stages) & 1u;
-            if (!mbar_wait_bounded(&full_bar[s], ph)) {
-                ok = false;
-                break;
-            }
-            uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
-            // threads 2t and 2t+1 own row t of the tile: 4 chunks of 16 bytes each
-            uint4 *row = reinterpret_cast<uint4 *>(st + (threadIdx.x >> 1) * kRowBytes) + (threadIdx.x & 1) * 4;
+        for (int i = 0; i <= n_my && ok; ++i) {
+            float t_cur = 0.f;
+            if (i < n_my) {
+                // the gate logit of this tile's row, consumed one iteration later
+                const int64_t row = static_cast<int64_t>(tw.row) * kBM + rt;
+                if (row < p.M) t_cur = __ldg(p.t + row);
+                tw.next();
+                for (int kb = 0; kb < p.nk; ++kb, rp.next(p.stages)) {
+                    const int s = rp.slot;
+                    const bool got = mbar_wait_bounded(&full_bar[s], rp.phase);
+                    if (named_barrier_or(1, kWorkers, !got)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+                    // kTPR threads share a tile row, kCPT of its 8 16-byte chunks each; the
+                    // chunk order is rotated by the row so that the 8 threads of a
+                    // shared-memory phase touch 8 different bank groups
+                    uint4 *rowp = reinterpret_cast<uint4 *>(st + trow * kRowBytes);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (SPLIT == 3) {
-                    float4 *hi = reinterpret_cast<float4 *>(row + c);
-                    float4 *lo = reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(row + c) + p.a_bytes);
-                    phi_split_chunk_f32(hi, lo);
-                } else {
-                    phi_chunk_bf16(row + c);
+                    for (int c = 0; c < kCPT; ++c) {
+                        const int ch = (tpart * kCPT + c) ^ (trow & 7);
+                        if (SPLIT == 3) {
+                            float4 *hi = reinterpret_cast<float4 *>(rowp + ch);
+                            float4 *lo = reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(rowp + ch) + p.a_bytes);
+                            phi_split_chunk_f32(hi, lo);
+                        } else {
+                            phi_chunk_bf16(rowp + ch);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ready_bar[s]);
                 }
+                if (!ok) break;
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&ready_bar[s]);
+            if (i > 0) {
+                // ---- epilogue of tile k = i - 1 ----
+                const int k = i - 1;
+                const int buf = k & 1;
+                const int g = te.col;
+                const int64_t m0 = static_cast<int64_t>(te.row) * kBM;
+                te.next();
+                const int h0 = g * p.hg;
+                const int hg = std::min(p.hg, p.D / R - h0);
+                const int qx0 = h0 * R;
+                const int ncol = hg * R;
+                const int64_t row = m0 + rt;
+                const bool live = row < p.M;
+                const int lb_i = lp.slot;
+                bool got = mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(k >> 1) & 1u);
+                if (p.lboxes > 0) got = got && mbar_wait_bounded(&lfull_bar[lb_i], lp.phase);
+                if (named_barrier_or(1, kWorkers, !got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float gate = 1.f / (1.f + __expf(-(t_prev + p.b_g)));
+                const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(buf) * kAccCols;
+                uint8_t *lb = lbase + lb_i * lbytes;
+                for (int c0 = wg * 32; c0 < ncol; c0 += 32 * kWG) {
+                    uint32_t v[32], dv[kHeads];
+                    tmem_ld32(acc + static_cast<uint32_t>(c0), v);
+                    // denominators of the heads this chunk touches: column hg*R + head
+                    tmem_ld_n<kHeads>(acc + static_cast<uint32_t>(ncol + c0 / R), dv);
+                    tmem_ld_wait();
+                    float scale[kHeads];
+#pragma unroll
+                    for (int h = 0; h < kHeads; ++h)
+                        scale[h] = (1.f - gate) / (__uint_as_float(dv[h]) + p.eps);
+                    if (p.lboxes > 0) {
+                        // L from the swizzled shared tile, Y written back in place
+                        const int bx = c0 / KT, e0 = c0 % KT;
+                        uint8_t *base = lb + bx * kBoxBytes + rt * kRowBytes;
+#pragma unroll
+                        for (int q = 0; q < kChunks32; ++q) {
+                            const int ch = (e0 / VE + q) ^ (rt & 7);
+                            uint4 *pch = reinterpret_cast<uint4 *>(base + ch * 16);
+                            float lv[VE], y[VE];
+                            IoT<T>::unpack(*pch, lv);
+#pragma unroll
+                            for (int e = 0; e < VE; ++e) {
+                                const int j = q * VE + e;
+                                y[e] = gate * lv[e] + __uint_as_float(v[j]) * scale[j / R < kHeads ? j / R : 0];
+                            }
+                            *pch = IoT<T>::pack(y);
+                        }
+                    } else if (live) {
+                        const T *L = static_cast<const T *>(p.L) + row * p.D + qx0;
+                        T *Y = static_cast<T *>(p.Y) + row * p.D + qx0;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c0 + j < ncol)
+                                IoT<T>::put(Y + c0 + j, gate * IoT<T>::get(L + c0 + j) +
+                                                            __uint_as_float(v[j]) *
+                                                                scale[j / R < kHeads ? j / R : 0]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce_bar[buf]);   // accumulator buffer may be reused
+                if (p.lboxes > 0) {
+                    fence_proxy_async_smem();
+                    named_barrier_sync(2, kWorkers);
+                    if (threadIdx.x == 0) {
+                        for (int bx = 0; bx < p.lboxes; ++bx)
+                            tma_store_2d(&tmY, lb + bx * kBoxBytes, qx0 + bx * KT, static_cast<int32_t>(m0));
+                        bulk_commit_group();
+                        // the previous tile's stores have now been read out of their buffer,
+                        // which may take a new L tile
+                        bulk_wait_group_read1();
+                        if (k > 0) mbar_arrive(&lfree_bar[lp_prev]);
+                    }
+                }
+                lp_prev = lb_i;
+                lp.next(p.lbufs);
+            }
+            t_prev = t_cur;
         }
         if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
-    }
-    __syncwarp();
-
-    if (warp < 8) {
-        // ---------------- epilogue: G = num / (den + eps), blend with L, write Y ----------------
-        // warp w reads TMEM lanes 32*(w%4).. (its rows); warpgroup w/4 takes every other
-        // 32-column chunk
-        const bool done = mbar_wait_bounded(&done_bar, 0);
-        const bool lok = p.lboxes == 0 || mbar_wait_bounded(&l_bar, 0);
-        tc_fence_after();
-        const int quad = warp & 3, wg = warp >> 2;
-        const int rt = quad * 32 + lane;
-        const int64_t row = m0 + rt;
-        const bool live = row < p.M;
-        if (!done || !lok) {
-            if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
-        } else {
-            const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-            const float gt = live ? __ldg(p.t + row) + p.b_g : 0.f;
-            const float gate = 1.f / (1.f + __expf(-gt));
-            const int ncol = hg * R;
-            for (int c0 = wg * 32; c0 < ncol; c0 += 64) {
-                uint32_t v[32], dv[32];
-                tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), v);
-                // denominators of the heads this chunk touches: column hg*R + head
-                tmem_ld32(tmem + lane_base + static_cast<uint32_t>(ncol + c0 / R), dv);
-                tmem_ld_wait();
-                float gv[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    gv[j] = (1.f - gate) * __uint_as_float(v[j]) /
-                            (__uint_as_float(dv[R >= 32 ? 0 : j / R]) + p.eps);
-                if (p.lboxes > 0) {
-                    // L from the swizzled shared tile, Y written back in place
-                    const int b = c0 / KT, e0 = c0 % KT;
-                    uint8_t *base = lbuf + b * kBoxBytes + rt * kRowBytes;
-#pragma unroll
-                    for (int q = 0; q < kChunks32; ++q) {
-                        const int ch = (e0 / VE + q) ^ (rt & 7);
-                        uint4 *pch = reinterpret_cast<uint4 *>(base + ch * 16);
-                        float lv[VE], y[VE];
-                        IoT<T>::unpack(*pch, lv);
-#pragma unroll
-                        for (int e = 0; e < VE; ++e) y[e] = gate * lv[e] + gv[q * VE + e];
-                        *pch = IoT<T>::pack(y);
-                    }
-                } else if (live) {
-                    const T *L = static_cast<const T *>(p.L) + row * p.D + qx0;
-                    T *Y = static_cast<T *>(p.Y) + row * p.D + qx0;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < ncol)
-                            IoT<T>::put(Y + c0 + j, gate * IoT<T>::get(L + c0 + j) + gv[j]);
-                }
-            }
-        }
-        if (p.lboxes > 0) {
-            fence_proxy_async_smem();
-            named_barrier_sync(1, kWorkers);
-            if (threadIdx.x == 0 && done && lok) {
-                for (int b = 0; b < p.lboxes; ++b)
-                    tma_store_2d(&tmY, lbuf + b * kBoxBytes, qx0 + b * KT, static_cast<int32_t>(m0));
-                bulk_commit_group();
-                bulk_wait_group_read0();
-            }
-        }
+        if (threadIdx.x == 0) bulk_wait_group_read0();   // shared memory outlives the stores
     }
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, static_cast<uint32_t>(p.tmem_cols));
+        tmem_dealloc(tmem, 2 * kAccCols);
     }
 }
 
 template <int SPLIT, typename T>
-glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, size_t smem, const CUtensorMap &q,
-                             const CUtensorMap &b0, const CUtensorMap &b1, const CUtensorMap &ml,
-                             const CUtensorMap &my, cudaStream_t s) {
-    dim3 grid(static_cast<unsigned>(p.n_groups), static_cast<unsigned>(ceil_div(p.M, kBM)));
+glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, unsigned grid, size_t smem,
+                             const CUtensorMap &q, const CUtensorMap &b0, const CUtensorMap &b1,
+                             const CUtensorMap &ml, const CUtensorMap &my, cudaStream_t s) {
 #define GLGA_RO(RR)                                                                              \
     case RR: {                                                                                   \
         auto kern = readout_kernel<SPLIT, T, RR>;                                                \
@@ -364,8 +499,8 @@ glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, size_t smem, const 
 glga_status readout_setup(Ctx *c) {
     const int kt = kRowBytes / c->elem;
     // hg*r + hg + 32 <= 256: numerators, denominators and the 32-column read past them
-    // fit one 256-column TMEM allocation.  Groups span at most 128 columns (one head for
-    // r >= 64): narrower groups let more CTAs share an SM and overlap their phases.
+    // fit one 256-column TMEM buffer.  Groups span at most 128 columns (one head for
+    // r >= 64), which bounds the two L/Y staging buffers to 2 x 64 KB.
     const int hg_max = std::max(1, std::min(224 / (c->r + 1), (c->r >= 64 ? 64 : 128) / c->r));
     c->ro_groups = static_cast<int32_t>(ceil_div(c->H, hg_max));
     c->ro_hg = static_cast<int32_t>(ceil_div(c->H, c->ro_groups));
@@ -409,20 +544,57 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     p.r = c->r;
     p.hg = c->ro_hg;
     p.n_groups = c->ro_groups;
+    p.n_total = ceil_div(c->N, kBM) * c->ro_groups;
     p.nk = c->ro_kp / kt;
     p.BNr = c->ro_bn;
-    // the epilogue reads 32 columns starting at a denominator column (<= hg*r + hg - 1)
-    int tc = 32;
-    while (tc < p.BNr || tc < p.hg * p.r + p.hg + 32) tc <<= 1;
-    p.tmem_cols = tc;
     const int planes = c->split == 3 ? 2 : 1;
     p.a_bytes = kBM * kRowBytes;
     p.b_bytes = static_cast<uint32_t>(p.BNr) * kRowBytes;
-    p.stage_bytes = planes * (p.a_bytes + p.b_bytes);
     p.lboxes = c->ro_tma_epi ? static_cast<int32_t>(ceil_div(static_cast<int64_t>(p.hg) * p.r, kt)) : 0;
-    const uint32_t lbytes = static_cast<uint32_t>(p.lboxes) * kBoxBytes;
-    p.stages = std::max(1, std::min(std::min(p.nk, kMaxStages),
-                                    static_cast<int>((200u * 1024u - lbytes) / p.stage_bytes)));
+    // Dynamic shared memory: resident B_g (when it fits), the K ring, and 2-3 L/Y
+    // buffers (a third when two ring stages still fit beside it).
+    constexpr int64_t kBudget = 220 * 1024;
+    const int64_t lb1 = static_cast<int64_t>(p.lboxes) * kBoxBytes;
+    const int64_t bres = static_cast<int64_t>(planes) * p.nk * p.b_bytes;
+    p.b_resident = 0;
+    p.lbufs = 0;
+    for (int resident = 1; resident >= 0 && p.lbufs == 0; --resident) {
+        const int64_t stage = planes * (p.a_bytes + (resident ? 0 : p.b_bytes));
+        const int64_t fixed = resident ? bres : 0;
+        for (int nb = 3; nb >= 2 && p.lbufs == 0; --nb) {
+            const int64_t left = kBudget - fixed - nb * lb1;
+            if (left >= (nb == 3 ? 2 : 1) * stage) {
+                p.b_resident = resident;
+                p.lbufs = nb;
+                p.stage_bytes = static_cast<uint32_t>(stage);
+                p.stages = static_cast<int32_t>(std::min<int64_t>(kMaxStages, left / stage));
+            }
+        }
+    }
+    if (p.lbufs == 0) {
+        set_error("readout: shared memory plan does not fit");
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    p.bres_bytes = p.b_resident ? static_cast<uint32_t>(bres) : 0u;
+    const uint32_t lbytes = static_cast<uint32_t>(p.lbufs * lb1);
+    // persistent: one CTA per SM (it holds all 512 TMEM columns); with resident B_g the
+    // grid is a multiple of the group count so every CTA stays on one group
+    int64_t grid = std::min<int64_t>(p.n_total, c->num_sms);
+    if (p.b_resident) {
+        grid = grid / p.n_groups * p.n_groups;
+        if (grid == 0) {
+            p.b_resident = 0;
+            p.bres_bytes = 0;
+            grid = std::min<int64_t>(p.n_total, c->num_sms);
+            p.stage_bytes = planes * (p.a_bytes + p.b_bytes);
+            p.stages = static_cast<int32_t>(std::min<int64_t>(
+                kMaxStages, (kBudget - static_cast<int64_t>(lbytes)) / p.stage_bytes));
+            if (p.stages < 1) {
+                set_error("readout: shared memory plan does not fit");
+                return GLGA_ERR_UNSUPPORTED;
+            }
+        }
+    }
     p.L = c->L;
     p.t = c->t;
     p.Y = Y;
@@ -437,11 +609,12 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
                                         kt, kBM);
         if (st != GLGA_OK) return st;
     }
-    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + lbytes + 1024;
+    const size_t smem = static_cast<size_t>(p.bres_bytes) + static_cast<size_t>(p.stages) * p.stage_bytes +
+                        lbytes + 1024;
     const CUtensorMap &b1 = planes == 2 ? c->tmBro[1].map : c->tmBro[0].map;
     if (c->io == GLGA_F32)
-        return launch_readout_r<3, float>(c, p, smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
-    return launch_readout_r<1, __nv_bfloat16>(c, p, smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
+        return launch_readout_r<3, float>(c, p, static_cast<unsigned>(grid), smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
+    return launch_readout_r<1, __nv_bfloat16>(c, p, static_cast<unsigned>(grid), smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
 }
 
 }  // namespace glga
