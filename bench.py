@@ -61,11 +61,24 @@ def replica_throughput(world, units_per_rank, slowest_total_ms, steps):
     return world * units_per_rank * steps / (slowest_total_ms * 1e-3)
 
 
-def local_bytes_model(N, E, D, H, r, s):
-    """Algorithmic bytes of the fused per-target kernel: CSR (row_ptr, col_idx), one k_j and
-    v_j row gather per edge, q_i and Y_i once per row, the gate logit, and S, z."""
+def local_kernel_bytes(N, E, D, s):
+    """Algorithmic bytes of one launch of the local-branch kernel: CSR (row_ptr, col_idx),
+    one k_j and v_j row gather per edge, q_i read and L_i written once per row."""
+    return 4 * (N + 1) + 4 * E + 2 * D * s * E + D * s * N + D * s * N
+
+
+def branch_bytes_model(N, E, D, H, r, s):
+    """Algorithmic bytes of the local branch with the readout and gate (steps a3-a5 taken
+    together, as if fused): CSR, the k_j / v_j gathers, q_i and Y_i once per row, the gate
+    logit, and S, z."""
     return (4 * (N + 1) + 4 * E + 2 * D * s * E + D * s * N + D * s * N + 4 * N
             + 4 * H * r * (r + 1))
+
+
+def branch_compulsory_bytes(N, E, D, H, r, s):
+    """Lower bound on the DRAM traffic of steps a3-a5: every Q, K, V row read once, Y
+    written once, plus CSR, gate logits and S, z."""
+    return 4 * (N + 1) + 4 * E + 3 * D * s * N + D * s * N + 4 * N + 4 * H * r * (r + 1)
 
 
 def kernel_source_hash():
@@ -333,18 +346,24 @@ def main():
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
 
     peaks, peak_kind = load_peaks()
-    B_loc = local_bytes_model(w.N, w.E, w.D, w.H, w.r, s_io)
+    B_kern = local_kernel_bytes(w.N, w.E, w.D, s_io)
     t_local = stages["local"] * 1e-3
-    achieved = B_loc / t_local / 1e9
+    achieved = B_kern / t_local / 1e9
     traffic, traffic_note = profiled_traffic(args.workload)
-    roofline = {"bound": "hbm", "kernel": "local_kernel (local branch + readout + gate)",
+    roofline = {"bound": "hbm", "kernel": "local_kernel (local softmax branch; writes L)",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "algorithmic_bytes_per_launch": B_loc, "avg_launch_ms": stages["local"],
+                "algorithmic_bytes_per_launch": B_kern, "avg_launch_ms": stages["local"],
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6.65 TB/s"}
     if traffic_note:
         roofline["traffic_note"] = traffic_note
+    # steps a3-a5 (local branch, readout, gate) against the fused-branch byte model
+    B_loc = branch_bytes_model(w.N, w.E, w.D, w.H, w.r, s_io)
+    t_branch = (stages["local"] + stages["readout"]) * 1e-3
+    branch = {"bytes": B_loc, "ms": t_branch * 1e3, "gbs": B_loc / t_branch / 1e9,
+              "frac": B_loc / t_branch / 1e9 / peaks["hbm_gbs"],
+              "compulsory_bytes": branch_compulsory_bytes(w.N, w.E, w.D, w.H, w.r, s_io)}
     gemm_flops = 2.0 * w.N * w.d * (3 * w.D + 1)
     gemm_bytes = w.N * w.d * s_io + w.N * 3 * w.D * s_io + 4 * w.N
     t_gemm = stages["gemm"] * 1e-3
@@ -362,7 +381,7 @@ def main():
                        "N": w.N, "E": w.E, "d": w.d, "H": w.H,
                        "r": w.r, "io": w.io, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between timed steps (256 MiB write, outside the timed spans)"},
-            "roofline": roofline, "projection": projection,
+            "roofline": roofline, "local_branch_a3_a5": branch, "projection": projection,
             "stages_ms": stages, "create": create, "gpu_launches": launches,
             "e2e": e2e, "clocks": clocks, "parity_max_rel_err": parity,
             "wall_s_timed_region": wall}
