@@ -58,15 +58,26 @@ typedef enum {
 typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
 
 /* Scheduling of target rows by in-degree (deg = row_ptr[i+1] - row_ptr[i]):
- *   deg <= warp_max_degree                 -> bucket 0: one warp per row
+ *   deg <= warp_max_degree                 -> bucket 0: warp tasks; each edge slot of a
+ *        warp takes one row (rows ordered by descending degree, ties by ascending row,
+ *        and packed up to 32 rows / about 256 edges per task)
  *   warp_max_degree < deg <= chunk_edges   -> bucket 1: one thread block per row
  *   deg > chunk_edges                      -> bucket 2: the row is cut into chunks of
  *        chunk_edges edges, one thread block per chunk, chunks merged in order.
- * Rows are kept in ascending order inside every bucket.  Requires
- * 0 <= warp_max_degree <= chunk_edges and chunk_edges >= 1.                            */
+ * Buckets 1 and 2 keep rows in ascending order.  Requires
+ * 0 <= warp_max_degree <= chunk_edges and chunk_edges >= 1.
+ *
+ * debug_checks != 0 selects kernel builds that check every column index read from the
+ * CSR against [0, N) and every scheduled row; a failed check is skipped (the edge is
+ * masked) and reported as GLGA_ERR_DEVICE by glga_last_device_error.  Slower; for
+ * debugging only.
+ * debug_fail_alloc = n > 0 makes the n-th device allocation of glga_create fail with
+ * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.                    */
 typedef struct {
     int32_t warp_max_degree;
     int32_t chunk_edges;
+    int32_t debug_checks;
+    int32_t debug_fail_alloc;
 } glga_options;
 
 /* Fills *opts with the defaults used when glga_create gets opts == NULL. */
@@ -179,6 +190,21 @@ GLGA_API glga_status glga_global_stats_static(const void *KV, int64_t N, int32_t
                                               glga_dtype io, float *Sz, void *stream);
 
 /* Static strings; never NULL. */
+/* Test entry points of the failure paths (the pages have no counterpart).
+ *
+ * glga_debug_bounded_wait -- enqueues on `stream` one thread that waits on a
+ * shared-memory mbarrier nothing arrives on, with the same bounded wait the tensor-core
+ * kernels use, given up after `limit_ns` nanoseconds (1e3 <= limit_ns <= 1e10).  The
+ * thread then sets the context's device flag and returns, so the next
+ * glga_last_device_error reports GLGA_ERR_TIMEOUT and the context stays usable.
+ *
+ * glga_debug_set_col_idx -- overwrites entry e of the context's CSR copy with `value`,
+ * skipping glga_create's validation, so that the device-side checks of a context made
+ * with debug_checks != 0 can be exercised.  Refused (GLGA_ERR_INVALID_ARG) when the
+ * context was made without debug_checks or e is outside [0, E).  Stream-ordered.      */
+GLGA_API glga_status glga_debug_bounded_wait(glga_ctx *ctx, int64_t limit_ns, void *stream);
+GLGA_API glga_status glga_debug_set_col_idx(glga_ctx *ctx, int64_t e, int32_t value, void *stream);
+
 GLGA_API const char *glga_status_string(glga_status s);
 GLGA_API const char *glga_last_error_message(void);
 

@@ -9,13 +9,27 @@
 #include <cstring>
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "glga_internal.cuh"
 
 namespace glga {
 
 namespace {
 thread_local char g_msg[512] = "no error";
+
+// One thread waits on an mbarrier that nothing arrives on, with the bounded wait of the
+// tensor-core kernels; it gives up after limit_ns and raises the timeout flag.
+__global__ void bounded_wait_probe_kernel(unsigned *flag, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(flag, kDevErrTimeout);
 }
+}  // namespace
 
 void set_error(const char *fmt, ...) {
     va_list ap;
@@ -30,8 +44,21 @@ glga_status cuda_fail(cudaError_t e, const char *what) {
     return GLGA_ERR_CUDA;
 }
 
+glga_status debug_alloc_hook(Ctx *c) {
+    ++c->alloc_calls;
+    if (c->opts.debug_fail_alloc > 0 && c->alloc_calls == c->opts.debug_fail_alloc) {
+        set_error("simulated failure of device allocation %lld (debug_fail_alloc)",
+                  static_cast<long long>(c->alloc_calls));
+        return GLGA_ERR_OOM;
+    }
+    return GLGA_OK;
+}
+
 glga_status dev_alloc(Ctx *c, void **p, size_t bytes) {
     if (bytes == 0) bytes = 16;
+    *p = nullptr;
+    const glga_status hook = debug_alloc_hook(c);
+    if (hook != GLGA_OK) return hook;
     cudaError_t e = cudaMalloc(p, bytes);
     if (e != cudaSuccess) {
         *p = nullptr;
@@ -88,6 +115,8 @@ glga_status glga_default_options(glga_options *opts) {
     }
     opts->warp_max_degree = 128;
     opts->chunk_edges = 1024;
+    opts->debug_checks = 0;
+    opts->debug_fail_alloc = 0;
     return GLGA_OK;
 }
 
@@ -127,6 +156,10 @@ glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t
     if (opts) o = *opts;
     if (o.warp_max_degree < 0 || o.chunk_edges < 1 || o.warp_max_degree > o.chunk_edges) {
         set_error("glga_create: need 0 <= warp_max_degree <= chunk_edges, chunk_edges >= 1");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (o.debug_fail_alloc < 0) {
+        set_error("glga_create: debug_fail_alloc must be >= 0");
         return GLGA_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -224,16 +257,35 @@ glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void
             if (!ev) GLGA_CUDA(cudaEventCreate(&ev));
         GLGA_CUDA(cudaEventRecord(c->ev[kStagePrep], s));
     }
-    glga_status st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, c->timing);
+    // NVTX ranges mark the host-side enqueue of each stage (visible to profilers that
+    // attach an NVTX tool; no-ops otherwise)
+    struct Range {
+        explicit Range(const char *name) { nvtxRangePushA(name); }
+        ~Range() { nvtxRangePop(); }
+    } whole("glga_forward");
+    glga_status st;
+    {
+        Range r("glga.projection");
+        st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, c->timing);
+    }
     if (st != GLGA_OK) return st;
     if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageStats], s));
-    st = stats_run(c, s);
+    {
+        Range r("glga.global_stats");
+        st = stats_run(c, s);
+    }
     if (st != GLGA_OK) return st;
     if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageLocal], s));
-    st = local_run(c, s);
+    {
+        Range r("glga.local");
+        st = local_run(c, s);
+    }
     if (st != GLGA_OK) return st;
     if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageReadout], s));
-    st = readout_run(c, b_g, eps, Y, s);
+    {
+        Range r("glga.readout");
+        st = readout_run(c, b_g, eps, Y, s);
+    }
     if (st != GLGA_OK) return st;
     if (c->timing) {
         GLGA_CUDA(cudaEventRecord(c->ev[kStageEnd], s));
@@ -361,6 +413,29 @@ glga_status glga_workspace_bytes(const glga_ctx *h, int64_t *bytes) {
         return GLGA_ERR_INVALID_ARG;
     }
     *bytes = h->c.bytes;
+    return GLGA_OK;
+}
+
+glga_status glga_debug_bounded_wait(glga_ctx *h, int64_t limit_ns, void *stream) {
+    if (!h || limit_ns < 1000 || limit_ns > 10000000000LL) {
+        set_error("glga_debug_bounded_wait: need a context and 1e3 <= limit_ns <= 1e10");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bounded_wait_probe_kernel<<<1, 32, 0, s>>>(h->c.dev_flag, static_cast<uint64_t>(limit_ns));
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
+}
+
+glga_status glga_debug_set_col_idx(glga_ctx *h, int64_t e, int32_t value, void *stream) {
+    if (!h || !h->c.opts.debug_checks || e < 0 || e >= h->c.E) {
+        set_error("glga_debug_set_col_idx: needs a context made with debug_checks and 0 <= e < E");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the value is copied from this function's stack: wait for the copy before returning
+    GLGA_CUDA(cudaMemcpyAsync(h->c.col_idx + e, &value, sizeof(int32_t), cudaMemcpyHostToDevice, s));
+    GLGA_CUDA(cudaStreamSynchronize(s));
     return GLGA_OK;
 }
 

@@ -74,6 +74,7 @@ struct Ctx {
     int32_t Dp = 0;               // padded GEMM width: 3*D + gate column + padding
     int32_t BN = 0, bn_last = 0, n_tiles = 0, stages = 0, tmem_cols = 0;
     bool gemm_tma_epi = false;    // Q/K/V stored through shared memory + TMA
+    int32_t gemm_sbufs = 2;       // staging buffers of that epilogue (1 or 2)
     TensorMap2D tmKVs;            // KV store map (64-column boxes)
     int split = 1;                // 1: bf16 MMA; 3: 3-term tf32 split (fp32 io)
     bool x_direct = false;        // A operand read straight from the caller's X
@@ -100,6 +101,7 @@ struct Ctx {
 
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;
+    int64_t alloc_calls = 0;      // device allocations made by create (debug_fail_alloc)
     int64_t launches = 0;         // kernels launched by glga_forward so far
 
     bool timing = false;
@@ -109,6 +111,9 @@ struct Ctx {
 
 // allocation helper that tracks bytes
 glga_status dev_alloc(Ctx *c, void **p, size_t bytes);
+// Counts one device allocation of create; GLGA_ERR_OOM when it is the one
+// opts.debug_fail_alloc names (test hook of the clean-up path).
+glga_status debug_alloc_hook(Ctx *c);
 
 // topology.cu
 glga_status validate_csr(Ctx *c, cudaStream_t s);

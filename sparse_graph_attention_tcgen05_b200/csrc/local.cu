@@ -19,6 +19,11 @@
 //                  kTaskEdges edges; each edge slot of the warp takes its own row
 // Heavy work comes first in block order so it starts early.
 //
+// Debug instantiations (DBG, chosen by glga_options.debug_checks) check every column
+// index they read against [0, N) and every row taken from a schedule list; a bad one
+// raises kDevErrBounds on the context's flag and is skipped, so no access leaves its
+// buffer.  The default instantiations compile without the checks.
+//
 // Lane layout: a 16-byte vector holds VE = 16/sizeof(T) consecutive features; an edge's
 // k_j (or v_j) row is LPE lanes x VPL vectors; EPW = 32/LPE edge slots per warp; the r
 // features of a head live in LPH = r/VE adjacent lanes, which reduce dot products with
@@ -102,7 +107,41 @@ struct LocalParams {
     void *L;             // io [N, D] local-branch output
     int32_t D, r, H, nvec, lpe, epw, lph;
     float score_scale;   // log2(e) / sqrt(r)
+    int32_t N;           // rows (debug checks)
+    unsigned *flag;      // device error flag (debug checks)
 };
+
+// 2^x by the PTX ex2.approx.ftz instruction.  The arguments are differences from a
+// running maximum (<= 0); results below 2^-126 of the maximum flush to zero.
+__device__ __forceinline__ float exp2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// A column index read from the CSR; debug builds mask (and report) one outside [0, N).
+template <bool DBG>
+__device__ __forceinline__ int32_t checked_col(const LocalParams &p, int32_t j) {
+    if constexpr (DBG) {
+        if (j < 0 || j >= p.N) {
+            atomicOr(p.flag, kDevErrBounds);
+            return -1;
+        }
+    }
+    return j;
+}
+
+// A row taken from a schedule list; debug builds report one outside [0, N).
+template <bool DBG>
+__device__ __forceinline__ bool row_ok(const LocalParams &p, int64_t row) {
+    if constexpr (DBG) {
+        if (row < 0 || row >= p.N) {
+            atomicOr(p.flag, kDevErrBounds);
+            return false;
+        }
+    }
+    return true;
+}
 
 template <typename T, int VPL>
 struct State {
@@ -121,7 +160,7 @@ struct State {
     __device__ __forceinline__ void merge(int v, float m2, float l2, const float (&a2)[VE]) {
         const float mn = fmaxf(m[v], m2);
         if (mn == -INFINITY) return;
-        const float c1 = exp2f(m[v] - mn), c2 = exp2f(m2 - mn);
+        const float c1 = exp2_ftz(m[v] - mn), c2 = exp2_ftz(m2 - mn);
         l[v] = l[v] * c1 + l2 * c2;
 #pragma unroll
         for (int e = 0; e < VE; ++e) acc[v][e] = acc[v][e] * c1 + a2[e] * c2;
@@ -135,15 +174,15 @@ struct Lane {
 
 // First column index of a slot's range as held by the lane that later broadcasts it:
 // lane li (< U) of the slot holds col_idx[e0 + li].
-template <int U>
+template <int U, bool DBG>
 __device__ __forceinline__ int32_t first_cols(const LocalParams &p, int64_t e0, int64_t e1, const Lane &ln) {
-    return (ln.li < U && e0 + ln.li < e1) ? __ldg(p.col_idx + e0 + ln.li) : -1;
+    return (ln.li < U && e0 + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + e0 + ln.li)) : -1;
 }
 
 // One slot walks the CSR entries [e0, e1) U at a time (the trip count is the warp's
 // maximum over slots); `cols` holds the first step's column indices (first_cols).
 // On return each lane holds its slot's partial state for its feature vectors.
-template <typename T, int VPL, int U>
+template <typename T, int VPL, int U, bool DBG>
 __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
                                            int64_t e0, int64_t e1, int32_t cols, const Lane &ln,
                                            State<T, VPL> &st) {
@@ -158,7 +197,7 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q
     for (int it = 0; it < iters; ++it) {
         const int32_t c_cur = c_next;
         const int64_t nb = e0 + static_cast<int64_t>(it + 1) * U;
-        c_next = (ln.li < U && nb + ln.li < e1) ? __ldg(p.col_idx + nb + ln.li) : -1;
+        c_next = (ln.li < U && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
         int32_t j[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) j[u] = __shfl_sync(0xffffffffu, c_cur, src0 + u);
@@ -200,13 +239,13 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q
             for (int u = 1; u < U; ++u) mx = fmaxf(mx, s[u][v]);
             const float mn = fmaxf(st.m[v], mx);
             if (mn == -INFINITY) continue;
-            const float corr = exp2f(st.m[v] - mn);
+            const float corr = exp2_ftz(st.m[v] - mn);
             st.l[v] *= corr;
 #pragma unroll
             for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const float pr = exp2f(s[u][v] - mn);
+                const float pr = exp2_ftz(s[u][v] - mn);
                 float vf[VE];
                 Io<T>::unpack(vr[u][v], vf);
                 st.l[v] += pr;
@@ -284,7 +323,7 @@ struct BlockScratch {
 
 // 8 warps split [e0, e1) (each warp's share split again across its slots); warp 0
 // returns the merge of all warps in warp order.
-template <typename T, int VPL, int U>
+template <typename T, int VPL, int U, bool DBG>
 __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
                                             int64_t e0, int64_t e1, const Lane &ln, int warp,
                                             BlockScratch<T, VPL> &sh, State<T, VPL> &st) {
@@ -293,7 +332,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&
     const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
     const int64_t per_s = ceil_div(b - a, p.epw);
     const int64_t sa = std::min(b, a + ln.slot * per_s), sb = std::min(b, sa + per_s);
-    slot_edges<T, VPL, U>(p, q, sa, sb, first_cols<U>(p, sa, sb, ln), ln, st);
+    slot_edges<T, VPL, U, DBG>(p, q, sa, sb, first_cols<U, DBG>(p, sa, sb, ln), ln, st);
     merge_slots<T, VPL>(p, st);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
@@ -316,7 +355,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&
     }
 }
 
-template <typename T, int VPL, int U>
+template <typename T, int VPL, int U, bool DBG>
 __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(const LocalParams p) {
     constexpr int VE = Io<T>::VE;
     __shared__ BlockScratch<T, VPL> sh;
@@ -334,6 +373,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         // ---------------- chunk of a bucket-2 row ----------------
         const int64_t c = bid;
         const int64_t row = p.chunk_row[c];
+        if (!row_ok<DBG>(p, row)) return;
         const int64_t rb = p.row_ptr[row], re = p.row_ptr[row + 1];
         const int64_t e0 = p.chunk_begin[c];
         const int64_t e1 = std::min<int64_t>(re, e0 + p.chunk_edges);
@@ -341,7 +381,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         const int64_t first = c - (e0 - rb) / p.chunk_edges;
         load_q_raw<T, VPL>(p, row, ln, true, qr);
         scale_q<T, VPL>(p, qr, q);
-        block_edges<T, VPL, U>(p, q, e0, e1, ln, warp, sh, st);
+        block_edges<T, VPL, U, DBG>(p, q, e0, e1, ln, warp, sh, st);
         const int64_t stride = 2 * p.H + p.D;
         if (warp == 0) {
             float *dst = p.part + c * stride;
@@ -392,9 +432,10 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     if (bid < p.n_cta) {
         // ---------------- bucket-1 row: one block ----------------
         const int64_t row = p.cta_rows[bid];
+        if (!row_ok<DBG>(p, row)) return;
         load_q_raw<T, VPL>(p, row, ln, true, qr);
         scale_q<T, VPL>(p, qr, q);
-        block_edges<T, VPL, U>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
+        block_edges<T, VPL, U, DBG>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
         if (warp == 0) finish_row<T, VPL>(p, row, st, ln, 0);
         return;
     }
@@ -407,8 +448,12 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     int32_t myrow = 0, mybeg = 0, myend = 0;
     if (ln.lane < n) {
         myrow = __ldg(p.warp_rows + t0 + ln.lane);
-        mybeg = __ldg(p.row_ptr + myrow);
-        myend = __ldg(p.row_ptr + myrow + 1);
+        if (row_ok<DBG>(p, myrow)) {
+            mybeg = __ldg(p.row_ptr + myrow);
+            myend = __ldg(p.row_ptr + myrow + 1);
+        } else {
+            myrow = -1;   // (debug only) no edges, no output
+        }
     }
     const int steps = (n + p.epw - 1) / p.epw;
     // step 0 prefetch: this slot's first row
@@ -417,8 +462,8 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     int32_t beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
     int32_t end = __shfl_sync(0xffffffffu, myend, k & 31);
     if (k >= n) beg = end = 0;
-    load_q_raw<T, VPL>(p, row, ln, k < n, qr);
-    int32_t cols = first_cols<U>(p, beg, end, ln);
+    load_q_raw<T, VPL>(p, row, ln, k < n && (!DBG || row >= 0), qr);
+    int32_t cols = first_cols<U, DBG>(p, beg, end, ln);
     for (int step = 0; step < steps; ++step) {
         const bool valid = k < n;
         const int32_t row_c = row;
@@ -431,10 +476,10 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
         end = __shfl_sync(0xffffffffu, myend, k & 31);
         if (k >= n) beg = end = 0;
-        load_q_raw<T, VPL>(p, row, ln, k < n, qr);
-        cols = first_cols<U>(p, beg, end, ln);
-        slot_edges<T, VPL, U>(p, q, beg_c, end_c, cols_c, ln, st);
-        if (valid) {
+        load_q_raw<T, VPL>(p, row, ln, k < n && (!DBG || row >= 0), qr);
+        cols = first_cols<U, DBG>(p, beg, end, ln);
+        slot_edges<T, VPL, U, DBG>(p, q, beg_c, end_c, cols_c, ln, st);
+        if (valid && (!DBG || row_c >= 0)) {
             // every slot finishes its own row
             constexpr int VEc = Io<T>::VE;
             uint4 *Lout = static_cast<uint4 *>(p.L) + static_cast<int64_t>(row_c) * p.nvec;
@@ -455,7 +500,10 @@ template <typename T, int VPL, int U>
 glga_status launch_local(Ctx *c, const LocalParams &p, cudaStream_t s) {
     const int64_t blocks = p.n_chunks + p.n_cta + p.task_blocks;
     if (blocks == 0) return GLGA_OK;
-    local_kernel<T, VPL, U><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
+    if (c->opts.debug_checks)
+        local_kernel<T, VPL, U, true><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
+    else
+        local_kernel<T, VPL, U, false><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -539,6 +587,8 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.epw = 32 / lpe;
     p.lph = c->r / VE;
     p.score_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->r)));
+    p.N = static_cast<int32_t>(c->N);
+    p.flag = c->dev_flag;
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
     // U edges per slot step; U <= LPE so the slot's lanes can hold its column indices
     if (c->io == GLGA_F32) {

@@ -25,7 +25,7 @@ namespace glga {
 namespace {
 constexpr int kBM = 128;
 constexpr int kRowBytes = 128;            // bytes of K per smem row (one swizzle span)
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kProdWarp = 8;             // TMA producer
 constexpr int kMmaWarp = 9;              // TMEM owner and MMA issuer
 constexpr int kGemmThreads = 320;        // warps 0-7 drain TMEM in the epilogue
@@ -38,6 +38,7 @@ struct GemmParams {
     int32_t BN;          // columns per tile (multiple of 16, <= 256)
     int32_t bn_last;     // columns of the last column tile (BN, or BN + 16 with the gate)
     int32_t tma_epi;     // 1: Q/K/V leave through smem + TMA stores (BN multiple of 64)
+    int32_t sbufs;       // staging buffers of the TMA-store epilogue (1 or 2)
     uint32_t stage_area; // bytes of the stage ring (staging buffers follow it)
     int32_t stages;
     int32_t tmem_cols;
@@ -287,10 +288,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
             const int n0 = ntile * p.BN;
             const int bn = ntile == p.n_tiles - 1 ? p.bn_last : p.BN;
             if (p.tma_epi) {
-                // Q/K/V columns go through staging buffer `buf`; its previous TMA store
-                // (tile i - 2) must have finished reading it first
-                uint8_t *sb = smem + p.stage_area + static_cast<size_t>(buf) * nbox * box_bytes;
-                if (threadIdx.x == 0) bulk_wait_group_read1();
+                // Q/K/V columns go through a staging buffer (buffer i & 1 when there are
+                // two); the TMA store that last used it (tile i - sbufs) must have
+                // finished reading it first
+                const int sbuf = p.sbufs == 2 ? buf : 0;
+                uint8_t *sb = smem + p.stage_area + static_cast<size_t>(sbuf) * nbox * box_bytes;
+                if (threadIdx.x == 0) {
+                    if (p.sbufs == 2)
+                        bulk_wait_group_read1();
+                    else
+                        bulk_wait_group_read0();
+                }
                 named_barrier_sync(1, 256);
                 for (int c0 = wg * 32; c0 < bn; c0 += 64) {
                     uint32_t v[32];
@@ -442,6 +450,7 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     p.BN = c->BN;
     p.bn_last = c->bn_last;
     p.tma_epi = c->gemm_tma_epi ? 1 : 0;
+    p.sbufs = c->gemm_sbufs;
     p.stages = c->stages;
     p.tmem_cols = c->tmem_cols;   // two 256-column accumulators
     p.D = c->D;
@@ -454,7 +463,7 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     p.KV = c->KV;
     p.t = c->t;
     p.flag = c->dev_flag;
-    const uint32_t staging = p.tma_epi ? 2u * (c->BN / 64) * kBM * kRowBytes : 0u;
+    const uint32_t staging = p.tma_epi ? static_cast<uint32_t>(p.sbufs) * (c->BN / 64) * kBM * kRowBytes : 0u;
     const size_t smem = static_cast<size_t>(p.stage_area) + staging + 1024;
     auto kern = proj_gemm_kernel<SPLIT, T>;
     GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -531,9 +540,14 @@ glga_status projection_setup(Ctx *c) {
     c->tmem_cols = 512;
     const int planes = c->split == 3 ? 2 : 1;
     const uint32_t stage_bytes = planes * (kBM * kRowBytes + c->bn_last * kRowBytes);
-    const uint32_t staging = c->gemm_tma_epi ? 2u * (c->BN / 64) * kBM * kRowBytes : 0u;
-    // one persistent CTA per SM: as many ring stages as fit (loads run ahead across tiles)
-    const uint32_t budget = 200u * 1024u - staging;
+    // One persistent CTA per SM: as many ring stages as fit beside the epilogue's staging
+    // buffers (loads run ahead across tiles).  Two staging buffers let a tile's TMA store
+    // overlap the next tile's epilogue; one is used when two would leave fewer than four
+    // ring stages, since the operand loads in flight bound the MMA rate.
+    constexpr uint32_t kBudget = 220u * 1024u;
+    const uint32_t stg1 = c->gemm_tma_epi ? (c->BN / 64) * kBM * kRowBytes : 0u;
+    c->gemm_sbufs = (kBudget - 2u * stg1) / stage_bytes >= 4u ? 2 : 1;
+    const uint32_t budget = kBudget - static_cast<uint32_t>(c->gemm_sbufs) * stg1;
     int st = static_cast<int>(budget / stage_bytes);
     c->stages = std::max(1, std::min(st, kMaxStages));
 

@@ -198,6 +198,8 @@ glga_status build_buckets(Ctx *c, cudaStream_t s) {
     const size_t tmpb = scan_tmp_bytes(N);
     void *scratch = nullptr;
     const size_t nbytes = 8 * static_cast<size_t>(N) * sizeof(int32_t) + 4 * sizeof(int32_t) + tmpb;
+    const glga_status hook = debug_alloc_hook(c);
+    if (hook != GLGA_OK) return hook;
     GLGA_CUDA(cudaMalloc(&scratch, nbytes));
     int32_t *f = static_cast<int32_t *>(scratch);
     int32_t *o = f + 4 * N;

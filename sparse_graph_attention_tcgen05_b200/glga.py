@@ -31,7 +31,8 @@ class GLGAError(RuntimeError):
 
 
 class Options(ctypes.Structure):
-    _fields_ = [("warp_max_degree", ctypes.c_int32), ("chunk_edges", ctypes.c_int32)]
+    _fields_ = [("warp_max_degree", ctypes.c_int32), ("chunk_edges", ctypes.c_int32),
+                ("debug_checks", ctypes.c_int32), ("debug_fail_alloc", ctypes.c_int32)]
 
 
 _lib = None
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
         "glga_kernel_launches": ([_vp, ctypes.POINTER(_i64)], _i32),
         "glga_global_stats_static": ([_vp, _i64, _i32, _i32, _i32, _vp, _vp], _i32),
         "glga_last_device_error": ([_vp, _vp], _i32),
+        "glga_debug_bounded_wait": ([_vp, _i64, _vp], _i32),
+        "glga_debug_set_col_idx": ([_vp, _i64, _i32, _vp], _i32),
         "glga_status_string": ([_i32], ctypes.c_char_p),
         "glga_last_error_message": ([], ctypes.c_char_p),
     }
@@ -225,6 +228,16 @@ class Layer:
 
     def last_device_error(self, stream=None) -> int:
         return int(lib().glga_last_device_error(self._h, _stream(stream)))
+
+    def debug_bounded_wait(self, limit_ns: int, stream=None):
+        """Enqueue the bounded-wait probe (see glga_debug_bounded_wait)."""
+        _check(lib().glga_debug_bounded_wait(self._h, int(limit_ns), _stream(stream)),
+               "glga_debug_bounded_wait")
+
+    def debug_set_col_idx(self, e: int, value: int, stream=None):
+        """Overwrite one CSR entry of a debug_checks context (see glga_debug_set_col_idx)."""
+        _check(lib().glga_debug_set_col_idx(self._h, int(e), int(value), _stream(stream)),
+               "glga_debug_set_col_idx")
 
     def close(self):
         if getattr(self, "_h", None):

@@ -64,3 +64,17 @@ def test_null_arguments():
     assert L.glga_kernel_launches(None, ctypes.byref(n)) == 1
     assert L.glga_workspace_bytes(None, ctypes.byref(n)) == 1
     assert L.glga_default_options(None) == 1
+
+
+def test_debug_options_default_off_and_are_checked():
+    o = glga.default_options()
+    assert (o.debug_checks, o.debug_fail_alloc) == (0, 0)
+    h = ctypes.c_void_p()
+    o = glga.Options(8, 64, 0, -1)           # negative allocation index
+    assert glga.lib().glga_create(ctypes.byref(h), 4, 8, 1, 8, 0, 16, 16, 0, ctypes.byref(o), None) == 1
+
+
+def test_debug_entry_points_reject_a_null_context():
+    L = glga.lib()
+    assert L.glga_debug_bounded_wait(None, 1_000_000, None) == 1
+    assert L.glga_debug_set_col_idx(None, 0, 0, None) == 1
