@@ -161,10 +161,19 @@ def rows_output(rows, H, r, row_ptr, col_idx, Qrows, K, V, t_rows, S, z, b_g, ep
     return {"L": L, "G": G, "g": g, "Y": Y, "ops": ops}
 
 
-def forward(N, d, H, r, X, W_Q, W_K, W_V, w_g, b_g, eps, row_ptr, col_idx, rows=None):
+def forward(N, d, H, r, X, W_Q, W_K, W_V, w_g, b_g, eps, row_ptr, col_idx, rows=None,
+            seg_ptr=None):
     """Full layer forward in float64 for the target rows `rows` (all rows if None).
 
-    Returns a dict with Y, L, G, g for those rows, S, z, the row list, op counters and the
+    `seg_ptr` (optional, [n_seg + 1], 0 = seg_ptr[0] <= ... <= seg_ptr[n_seg] = N) splits
+    the nodes into contiguous segments, the elements of a batch: the global statistics S,
+    z are then summed over each segment's own nodes, and row i's readout uses the
+    statistics of its segment (method page, "Implementation notes": the layer takes
+    X [batch, N, d]; "Key formulas": the global sums run over the N nodes of one graph).
+    None means one segment holding every node.
+
+    Returns a dict with Y, L, G, g for those rows, S, z ([H, r, r] and [H, r]; with
+    segments [n_seg, H, r, r] and [n_seg, H, r]), the row list, op counters and the
     seconds spent per stage (projection, global statistics, per-target outputs)."""
     t0 = time.perf_counter()
     X = np.ascontiguousarray(X, dtype=np.float32)
@@ -175,18 +184,44 @@ def forward(N, d, H, r, X, W_Q, W_K, W_V, w_g, b_g, eps, row_ptr, col_idx, rows=
     Qr = project(Xr, W_Q)
     tr = gate_logit(Xr, w_g)
     t1 = time.perf_counter()
-    S, z = global_stats(K, V, H, r)
-    t2 = time.perf_counter()
-    out = rows_output(rows, H, r, row_ptr, col_idx, Qr, K, V, tr, S, z, b_g, eps)
+    if seg_ptr is None:
+        S, z = global_stats(K, V, H, r)
+        t2 = time.perf_counter()
+        out = rows_output(rows, H, r, row_ptr, col_idx, Qr, K, V, tr, S, z, b_g, eps)
+    else:
+        seg_ptr = np.asarray(seg_ptr, dtype=np.int64)
+        n_seg = seg_ptr.shape[0] - 1
+        if n_seg < 1 or seg_ptr[0] != 0 or seg_ptr[-1] != N or np.any(np.diff(seg_ptr) < 0):
+            raise ValueError("seg_ptr must run from 0 to N without decreasing")
+        S = np.zeros((n_seg, H, r, r))
+        z = np.zeros((n_seg, H, r))
+        for k in range(n_seg):
+            a, b = int(seg_ptr[k]), int(seg_ptr[k + 1])
+            if b > a:
+                S[k], z[k] = global_stats(K[a:b], V[a:b], H, r)
+        t2 = time.perf_counter()
+        # the segment of each listed row: the last segment starting at or before it
+        seg = np.searchsorted(seg_ptr, rows, side="right") - 1
+        D = H * r
+        out = {"L": np.empty((rows.shape[0], D)), "G": np.empty((rows.shape[0], D)),
+               "g": np.empty(rows.shape[0]), "Y": np.empty((rows.shape[0], D)),
+               "ops": np.zeros(3, dtype=np.int64)}
+        for k in np.unique(seg):
+            idx = np.nonzero(seg == k)[0]
+            part = rows_output(rows[idx], H, r, row_ptr, col_idx, Qr[idx], K, V, tr[idx],
+                               S[k], z[k], b_g, eps)
+            for key in ("L", "G", "g", "Y"):
+                out[key][idx] = part[key]
+            out["ops"] += part["ops"]
     t3 = time.perf_counter()
     out.update({"S": S, "z": z, "rows": rows, "t": tr, "Q": Qr,
                 "seconds": {"project": t1 - t0, "global_stats": t2 - t1, "rows": t3 - t2}})
     return out
 
 
-def forward_workload(w, rows=None, csr=None):
+def forward_workload(w, rows=None, csr=None, seg_ptr=None):
     """Oracle forward of a `Workload` (see the package's workloads module)."""
     if csr is None:
         csr = csr_from_coo(w.N, w.src, w.dst)
     return forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
-                   csr[0], csr[1], rows)
+                   csr[0], csr[1], rows, seg_ptr)

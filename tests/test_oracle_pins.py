@@ -393,3 +393,85 @@ def test_buckets_partition_rows_and_edges(warp_max, chunk):
     split_edges = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in b["split_rows"]] or [np.zeros(0, int)])
     assert np.all(cover[split_edges] == 1)
     assert cover.sum() == len(split_edges)
+
+
+# ---------------------------------------------------------------------------------------
+# Segments (the batch dimension of the method page's "Implementation notes"): each
+# contiguous node range has its own S and z.
+# ---------------------------------------------------------------------------------------
+def _batch(sizes, k, seed, d=12, H=2, r=8):
+    """Graphs of the given sizes (edges only inside each graph, self-loops included),
+    relabelled into one node range; shared weights."""
+    rng = np.random.default_rng(seed)
+    src, dst, offs = [], [], [0]
+    for n in sizes:
+        if n > 0:
+            s = rng.integers(0, n, n * k)
+            t = np.repeat(np.arange(n), k)
+            s = np.concatenate([s, np.arange(n)]) + offs[-1]
+            t = np.concatenate([t, np.arange(n)]) + offs[-1]
+            src.append(s); dst.append(t)
+        offs.append(offs[-1] + n)
+    N = offs[-1]
+    src = np.concatenate(src).astype(np.int32) if src else np.zeros(0, np.int32)
+    dst = np.concatenate(dst).astype(np.int32) if dst else np.zeros(0, np.int32)
+    w = make_custom(N, d, H, r, src, dst, io="f32", seed=seed + 1, b_g=0.3)
+    return w, np.array(offs, dtype=np.int64)
+
+
+def test_batch_of_graphs_equals_independent_layers():
+    """A batch of separate graphs with one segment per graph gives, row for row, what the
+    layer gives on each graph alone (statistics over that graph's nodes only)."""
+    sizes = [37, 0, 90, 1, 64, 5]
+    w, seg = _batch(sizes, 4, seed=21)
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    out = oracle.forward_workload(w, csr=(rp, ci), seg_ptr=seg)
+    assert out["S"].shape == (len(sizes), w.H, w.r, w.r)
+    for k, n in enumerate(sizes):
+        a, b = int(seg[k]), int(seg[k + 1])
+        if n == 0:
+            assert not out["S"][k].any() and not out["z"][k].any()
+            continue
+        m = (w.dst >= a) & (w.dst < b)
+        rp1, ci1 = oracle.csr_from_coo(n, w.src[m] - a, w.dst[m] - a)
+        alone = oracle.forward(n, w.d, w.H, w.r, w.X[a:b], w.W_Q, w.W_K, w.W_V, w.w_g,
+                               w.b_g, w.eps, rp1, ci1)
+        np.testing.assert_allclose(out["Y"][a:b], alone["Y"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(out["S"][k], alone["S"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(out["z"][k], alone["z"], rtol=1e-12)
+
+
+def test_one_segment_is_the_unsegmented_layer():
+    w = make_workload("tiny")
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    a = oracle.forward_workload(w, csr=(rp, ci))
+    b = oracle.forward_workload(w, csr=(rp, ci), seg_ptr=[0, w.N])
+    np.testing.assert_array_equal(a["Y"], b["Y"])
+    np.testing.assert_array_equal(a["S"], b["S"][0])
+
+
+def test_segment_statistics_against_einsum():
+    """S and z of each segment are the sums over exactly its nodes: a segment boundary
+    moved by one node moves exactly that node's contribution."""
+    w, seg = _batch([20, 30, 25], 3, seed=5)
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    X = w.X.astype(np.float64)
+    K = X @ w.W_K.astype(np.float64); V = X @ w.W_V.astype(np.float64)
+    pk = torch.nn.functional.elu(torch.tensor(K)).numpy() + 1.0
+    for cut in (seg, np.array([0, 21, 50, 75])):
+        out = oracle.forward_workload(w, csr=(rp, ci), seg_ptr=cut)
+        for k in range(3):
+            a, b = cut[k], cut[k + 1]
+            for h in range(w.H):
+                sl = slice(h * w.r, (h + 1) * w.r)
+                np.testing.assert_allclose(out["S"][k, h], np.einsum("ja,jc->ac", pk[a:b, sl], V[a:b, sl]),
+                                           rtol=1e-10, atol=1e-12)
+                np.testing.assert_allclose(out["z"][k, h], pk[a:b, sl].sum(0), rtol=1e-10)
+
+
+def test_bad_segments_are_rejected():
+    w = make_workload("tiny")
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    for seg in ([1, w.N], [0, w.N - 1], [0, 10, 5, w.N], [0]):
+        with pytest.raises(ValueError):
+            oracle.forward_workload(w, csr=(rp, ci), seg_ptr=seg)
