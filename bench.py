@@ -213,6 +213,9 @@ def main():
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink the workload (small profiling captures only; reported lines use 1.0)")
     ap.add_argument("--no-parity", action="store_true", help="skip the sampled-row oracle check")
+    ap.add_argument("--segment-len", type=int, default=0,
+                    help="segments of this many nodes, each with its own global statistics "
+                         "(a batch of graphs; 0 = one segment over all nodes)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -253,7 +256,10 @@ def main():
     t0 = time.perf_counter()
     row_ptr, col_idx = glga.csr_from_coo(w.N, src, dst)
     t1 = time.perf_counter()
-    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+    seg = None
+    if args.segment_len > 0:
+        seg = np.unique(np.concatenate([np.arange(0, w.N, args.segment_len), [w.N]])).astype(np.int64)
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx, segments=seg)
     torch.cuda.synchronize()
     t2 = time.perf_counter()
     create = {"csr_from_coo_ms": (t1 - t0) * 1e3, "glga_create_ms": (t2 - t1) * 1e3,
@@ -283,7 +289,7 @@ def main():
         rows = np.unique(np.concatenate([rng.choice(w.N, 256, replace=False),
                                          np.argsort(np.diff(csr[0]))[-8:]]))
         ref = oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
-                             csr[0], csr[1], rows=rows)
+                             csr[0], csr[1], rows=rows, seg_ptr=seg)
         Yg = Y.float().cpu().numpy()[rows].astype(np.float64)
         parity = float(np.abs(Yg - ref["Y"]).max() / np.abs(ref["Y"]).max())
 
@@ -380,7 +386,8 @@ def main():
             "config": {"workload": args.workload if args.scale == 1.0 else f"{args.workload}@scale{args.scale}",
                        "N": w.N, "E": w.E, "d": w.d, "H": w.H,
                        "r": w.r, "io": w.io, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed between timed steps (256 MiB write, outside the timed spans)"},
+                       "l2": "flushed between timed steps (256 MiB write, outside the timed spans)",
+                       "segments": 1 if seg is None else int(seg.shape[0] - 1)},
             "roofline": roofline, "local_branch_a3_a5": branch, "projection": projection,
             "stages_ms": stages, "create": create, "gpu_launches": launches,
             "e2e": e2e, "clocks": clocks, "parity_max_rel_err": parity,

@@ -101,6 +101,24 @@ GLGA_API glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H
                         glga_dtype io, const int32_t *row_ptr, const int32_t *col_idx,
                         int64_t E, const glga_options *opts, void *stream);
 
+/* glga_create_segmented -- as glga_create, for a batch of graphs laid out as contiguous
+ * node ranges (segments).  Method page "Gated Local-Global Graph Attention",
+ * "Implementation notes" (the layer takes X [batch, N, d]) and "Key formulas" (S and z
+ * sum over the nodes of one graph): the global statistics are summed per segment, and
+ * row i's readout uses the S, z of its own segment.  The local branch follows the CSR
+ * as always (edges may cross segments; a batch of separate graphs has none that do).
+ *   seg_ptr  (host) int64 [n_seg + 1]: segment k holds nodes [seg_ptr[k], seg_ptr[k+1]);
+ *            seg_ptr[0] = 0, non-decreasing, seg_ptr[n_seg] = N.  Empty segments are
+ *            allowed.  Copied; the caller keeps ownership.
+ *   n_seg    >= 1; n_seg = 1 with {0, N} is glga_create.
+ * GLGA_ERR_INVALID_ARG for a malformed seg_ptr.  The statistics workspace holds one
+ * H*r*(r+1)*4-byte partial per row range, and every non-empty segment takes at least
+ * one range; GLGA_ERR_UNSUPPORTED if that workspace would exceed 4 GiB.             */
+GLGA_API glga_status glga_create_segmented(glga_ctx **out, int64_t N, int32_t d, int32_t H,
+                        int32_t r, glga_dtype io, const int32_t *row_ptr,
+                        const int32_t *col_idx, int64_t E, const int64_t *seg_ptr,
+                        int64_t n_seg, const glga_options *opts, void *stream);
+
 /* glga_forward -- Y = layer(X) for the graph bound at create.
  *   X    (device) io [N, d]          W_Q, W_K, W_V (device) io [d, H*r]
  *   w_g  (device) io [d]             b_g, eps (host) gate bias and readout epsilon
@@ -142,8 +160,8 @@ GLGA_API glga_status glga_get_buckets(const glga_ctx *ctx, int32_t *warp_rows, i
 
 /* Copies the intermediates of the last glga_forward (device -> device, on `stream`):
  *   Q (io [N, H*r]), K and V (io [N, H*r] each), t (float [N], gate logit x_i . w_g),
- *   S (float [H, r, r]), z (float [H, r]), L (io [N, H*r], the local branch).  Any
- *   pointer may be NULL.                                                               */
+ *   S (float [n_seg, H, r, r]), z (float [n_seg, H, r]) with n_seg = 1 for glga_create,
+ *   L (io [N, H*r], the local branch).  Any pointer may be NULL.                        */
 GLGA_API glga_status glga_get_intermediates(const glga_ctx *ctx, void *Q, void *K, void *V, float *t,
                                    float *S, float *z, void *L, void *stream);
 

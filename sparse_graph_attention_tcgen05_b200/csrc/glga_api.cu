@@ -75,6 +75,7 @@ static void release_ctx(Ctx *c) {
     void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
                     c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
+                    c->part_ptr, c->seg_part_ptr, c->tile_seg, c->fix_row, c->fix_seg,
                     c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
@@ -123,6 +124,14 @@ glga_status glga_default_options(glga_options *opts) {
 glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t r,
                         glga_dtype io, const int32_t *row_ptr, const int32_t *col_idx, int64_t E,
                         const glga_options *opts, void *stream) {
+    const int64_t seg[2] = {0, N};
+    return glga_create_segmented(out, N, d, H, r, io, row_ptr, col_idx, E, seg, 1, opts, stream);
+}
+
+glga_status glga_create_segmented(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t r,
+                                  glga_dtype io, const int32_t *row_ptr, const int32_t *col_idx,
+                                  int64_t E, const int64_t *seg_ptr, int64_t n_seg,
+                                  const glga_options *opts, void *stream) {
     if (!out) {
         set_error("glga_create: out is NULL");
         return GLGA_ERR_INVALID_ARG;
@@ -162,6 +171,15 @@ glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t
         set_error("glga_create: debug_fail_alloc must be >= 0");
         return GLGA_ERR_INVALID_ARG;
     }
+    if (!seg_ptr || n_seg < 1 || n_seg > 2147483647LL || seg_ptr[0] != 0 || seg_ptr[n_seg] != N) {
+        set_error("glga_create: seg_ptr must hold n_seg + 1 >= 2 offsets from 0 to N");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    for (int64_t k = 0; k < n_seg; ++k)
+        if (seg_ptr[k + 1] < seg_ptr[k]) {
+            set_error("glga_create: seg_ptr decreases at segment %lld", static_cast<long long>(k));
+            return GLGA_ERR_INVALID_ARG;
+        }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     glga_ctx *h = new (std::nothrow) glga_ctx();
     if (!h) {
@@ -178,6 +196,8 @@ glga_status glga_create(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t
     c->io = io;
     c->elem = elem;
     c->opts = o;
+    c->n_seg = n_seg;
+    c->seg_ptr.assign(seg_ptr, seg_ptr + n_seg + 1);
     glga_status st = GLGA_OK;
     cudaError_t e = cudaGetDevice(&c->device);
     if (e == cudaSuccess)
@@ -354,11 +374,12 @@ glga_status glga_get_intermediates(const glga_ctx *h, void *Q, void *K, void *V,
         if (t) GLGA_CUDA(cudaMemcpyAsync(t, c->t, c->N * sizeof(float), cudaMemcpyDeviceToDevice, s));
         if (L) GLGA_CUDA(cudaMemcpyAsync(L, c->L, c->N * row, cudaMemcpyDeviceToDevice, s));
     }
-    const size_t sbytes = static_cast<size_t>(c->H) * c->r * c->r * sizeof(float);
-    if (S) GLGA_CUDA(cudaMemcpyAsync(S, c->Sz, sbytes, cudaMemcpyDeviceToDevice, s));
+    // Sz holds S [n_seg][H][r][r] followed by z [n_seg][H][r]
+    const size_t s_floats = static_cast<size_t>(c->n_seg) * c->H * c->r * c->r;
+    if (S) GLGA_CUDA(cudaMemcpyAsync(S, c->Sz, s_floats * sizeof(float), cudaMemcpyDeviceToDevice, s));
     if (z)
-        GLGA_CUDA(cudaMemcpyAsync(z, c->Sz + static_cast<size_t>(c->H) * c->r * c->r,
-                                  static_cast<size_t>(c->H) * c->r * sizeof(float),
+        GLGA_CUDA(cudaMemcpyAsync(z, c->Sz + s_floats,
+                                  static_cast<size_t>(c->n_seg) * c->H * c->r * sizeof(float),
                                   cudaMemcpyDeviceToDevice, s));
     return GLGA_OK;
 }

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "glga.h"
 
 namespace glga {
@@ -87,9 +89,10 @@ struct Ctx {
     void *KV = nullptr;           // io [N, 2D]  (k_j | v_j)
     float *t = nullptr;           // [N] gate logits
     float *Spart = nullptr;       // [P][H][r][r+1] partial sums of the row ranges
-    float *Sz = nullptr;          // S [H][r][r] followed by z [H][r]
+    float *Sz = nullptr;          // S [n_seg][H][r][r] followed by z [n_seg][H][r]
     int32_t stats_parts = 0;
     int64_t stats_rows_per_part = 0;
+    int32_t *part_ptr = nullptr;  // row ranges of the statistics kernel [stats_parts + 1]
     TensorMap2D tmK, tmV;         // K and V halves of KV for the statistics kernel
 
     // readout GEMM (phi(Q) x [S | z] per head group, blended with L)
@@ -98,6 +101,15 @@ struct Ctx {
     void *Bro = nullptr;          // [planes][groups][ro_bn][ro_kp] K-major, io type
     TensorMap2D tmBro[2], tmQ, tmL;
     void *L = nullptr;            // io [N, D] local-branch output
+
+    // segments (a batch of graphs as contiguous node ranges, each with its own S and z)
+    int64_t n_seg = 1;
+    std::vector<int64_t> seg_ptr;     // host copy [n_seg + 1]
+    int32_t *seg_part_ptr = nullptr;  // statistics ranges of each segment [n_seg + 1]
+    int32_t *tile_seg = nullptr;      // segment of each 128-row readout tile's first row
+    int32_t *fix_row = nullptr;       // rows whose segment differs from their tile's
+    int32_t *fix_seg = nullptr;       //   ... and that segment
+    int64_t n_fix = 0;
 
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;

@@ -16,6 +16,7 @@
 // the block-diagonal operand of the readout GEMM.  Output layout: S [H][r][r], z [H][r].
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "glga_internal.cuh"
 
@@ -43,7 +44,8 @@ struct StatsGeom {
 struct StatsParams {
     int64_t N;
     int32_t D, H;
-    int64_t rows_per_part;   // multiple of the stage height
+    int64_t rows_per_part;   // multiple of the stage height (when part_ptr is NULL)
+    const int32_t *part_ptr; // explicit row ranges [P + 1] (segments), or NULL
     int32_t stages;
     uint32_t stage_bytes;
     float *part;             // [P][H][r][r+1]
@@ -74,8 +76,9 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     uint8_t *ones = smem + static_cast<size_t>(p.stages) * p.stage_bytes;   // 16 x 128 B, K-major
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int part = blockIdx.x, fb = blockIdx.y;
-    const int64_t r0 = static_cast<int64_t>(part) * p.rows_per_part;
-    const int64_t r1 = std::min<int64_t>(p.N, r0 + p.rows_per_part);
+    // row range [r0, r1) of this part; rows of the last tile past r1 get phi(k) = 0
+    const int64_t r0 = p.part_ptr ? p.part_ptr[part] : static_cast<int64_t>(part) * p.rows_per_part;
+    const int64_t r1 = p.part_ptr ? p.part_ptr[part + 1] : std::min<int64_t>(p.N, r0 + p.rows_per_part);
     const int ntiles = r1 > r0 ? static_cast<int>(ceil_div(r1 - r0, G::kRows)) : 0;
 
     if (threadIdx.x == 0) {
@@ -286,32 +289,39 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     }
 }
 
-// Sums parts 0..P-1 in order.  Writes S [H][R][R] then z [H][R] to Sz and, when Bro is
-// given, the readout operand: group gi = h / hg holds, K-major, S_h at rows (n)
+// Segment k = blockIdx.y sums its parts (seg_part_ptr[k] .. seg_part_ptr[k+1] - 1, or
+// 0..P-1 when seg_part_ptr is NULL) in order.  Writes S_k [H][R][R] at Sz + k*H*R*R and
+// z_k [H][R] at Sz + n_seg*H*R*R + k*H*R and, when Bro is given, segment k's readout
+// operand at Bro + k*seg_stride: group gi = h / hg holds, K-major, S_h at rows (n)
 // hl*R + c and columns (k) hl*R + a, and z_h at row hga*R + hl (hl = h - gi*hg, hga =
 // heads in group gi).  Every other entry of Bro stays zero from its initialisation.
 // Block of 256 threads = 8 warps for 32 consecutive outputs: warp w adds parts
 // w, w+8, w+16, ... in order, then warp 0 adds the 8 warp sums in warp order.
 template <typename T>
-__global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restrict__ part, int P, int H, int R,
-                                    float *__restrict__ Sz, T *__restrict__ Bro, int hg, int BNr,
-                                    int Kp, int64_t plane) {
+__global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restrict__ part, int P,
+                                    const int32_t *__restrict__ seg_part_ptr, int64_t n_seg,
+                                    int H, int R, float *__restrict__ Sz, T *__restrict__ Bro,
+                                    int hg, int BNr, int Kp, int64_t seg_stride, int64_t plane) {
     __shared__ float ws[8][32];
     const int per_head = R * (R + 1);
     const int total = H * per_head;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int o = blockIdx.x * 32 + lane;
+    // segments blockIdx.y, blockIdx.y + gridDim.y, ... (the grid's y extent is capped)
+    for (int64_t seg = blockIdx.y; seg < n_seg; seg += gridDim.y) {
+    const int q0 = seg_part_ptr ? seg_part_ptr[seg] : 0;
+    const int q1 = seg_part_ptr ? seg_part_ptr[seg + 1] : P;
     float acc = 0.f;
     if (o < total) {
-        int q = w;
-        for (; q + 24 < P; q += 32) {
+        int q = q0 + w;
+        for (; q + 24 < q1; q += 32) {
             const float a0 = part[static_cast<int64_t>(q) * total + o];
             const float a1 = part[static_cast<int64_t>(q + 8) * total + o];
             const float a2 = part[static_cast<int64_t>(q + 16) * total + o];
             const float a3 = part[static_cast<int64_t>(q + 24) * total + o];
             acc += a0; acc += a1; acc += a2; acc += a3;
         }
-        for (; q < P; q += 8) acc += part[static_cast<int64_t>(q) * total + o];
+        for (; q < q1; q += 8) acc += part[static_cast<int64_t>(q) * total + o];
     }
     ws[w][lane] = acc;
     __syncthreads();
@@ -320,14 +330,15 @@ __global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restri
 #pragma unroll
         for (int k = 0; k < 8; ++k) s += ws[k][lane];
         const int h = o / per_head, rem = o % per_head, a = rem / (R + 1), c = rem % (R + 1);
+        const int64_t hrr = static_cast<int64_t>(H) * R * R;
         if (c < R)
-            Sz[(static_cast<int64_t>(h) * R + a) * R + c] = s;
+            Sz[seg * hrr + (static_cast<int64_t>(h) * R + a) * R + c] = s;
         else
-            Sz[static_cast<int64_t>(H) * R * R + h * R + a] = s;
+            Sz[n_seg * hrr + seg * H * R + h * R + a] = s;
         if (Bro) {
             const int gi = h / hg, hl = h - gi * hg, hga = min(hg, H - gi * hg);
             const int n = c < R ? hl * R + c : hga * R + hl;
-            const int64_t idx = (static_cast<int64_t>(gi) * BNr + n) * Kp + hl * R + a;
+            const int64_t idx = seg * seg_stride + (static_cast<int64_t>(gi) * BNr + n) * Kp + hl * R + a;
             if (sizeof(T) == 4) {
                 const float hi = to_tf32(s);
                 reinterpret_cast<float *>(Bro)[idx] = hi;
@@ -336,6 +347,73 @@ __global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restri
                 Bro[idx] = __float2bfloat16_rn(s);
             }
         }
+    }
+    __syncthreads();   // ws is rewritten by the next segment
+    }
+}
+
+// Segment-major reduction for batches of segments: block (h, y) reduces head h of
+// segments y, y + gridDim.y, ...: it adds each segment's ranges one after another in
+// range order (deterministic) into shared memory with coalesced reads of the partials,
+// then writes S_h and z_h of the segment to Sz and its block of the readout operand
+// (rows n of the K-major operand, R consecutive k each) with coalesced writes.  Layouts as
+// in stats_reduce_kernel.
+template <typename T>
+__global__ void __launch_bounds__(256) stats_reduce_segments_kernel(
+    const float *__restrict__ part, const int32_t *__restrict__ seg_part_ptr, int64_t n_seg, int H,
+    int R, float *__restrict__ Sz, T *__restrict__ Bro, int hg, int BNr, int Kp, int64_t seg_stride,
+    int64_t plane) {
+    extern __shared__ float red[];                  // [R][R + 1] of one head
+    const int h = blockIdx.x;
+    const int per_head = R * (R + 1);
+    const int total = H * per_head;
+    const int64_t hrr = static_cast<int64_t>(H) * R * R;
+    const int gi = h / hg, hl = h - gi * hg, hga = min(hg, H - gi * hg);
+    for (int64_t seg = blockIdx.y; seg < n_seg; seg += gridDim.y) {
+        const int q0 = seg_part_ptr[seg], q1 = seg_part_ptr[seg + 1];
+        // 8 outputs per thread at a time, so 8 independent loads are in flight
+        constexpr int kIlp = 8;
+        for (int i0 = threadIdx.x; i0 < per_head; i0 += kIlp * blockDim.x) {
+            float acc[kIlp];
+#pragma unroll
+            for (int k = 0; k < kIlp; ++k) acc[k] = 0.f;
+            for (int q = q0; q < q1; ++q) {
+                const float *src = part + static_cast<int64_t>(q) * total + h * per_head;
+#pragma unroll
+                for (int k = 0; k < kIlp; ++k) {
+                    const int i = i0 + k * blockDim.x;
+                    if (i < per_head) acc[k] += src[i];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kIlp; ++k) {
+                const int i = i0 + k * blockDim.x;
+                if (i < per_head) red[i] = acc[k];
+            }
+        }
+        __syncthreads();
+        float *S = Sz + seg * hrr + static_cast<int64_t>(h) * R * R;
+        for (int i = threadIdx.x; i < R * R; i += blockDim.x) S[i] = red[(i / R) * (R + 1) + i % R];
+        float *z = Sz + n_seg * hrr + seg * H * R + h * R;
+        for (int a = threadIdx.x; a < R; a += blockDim.x) z[a] = red[a * (R + 1) + R];
+        if (Bro) {
+            // operand rows n = hl*R + c (S_h column c) and n = hga*R + hl (z_h); k = hl*R + a
+            T *B = Bro + seg * seg_stride + static_cast<int64_t>(gi) * BNr * Kp;
+            for (int i = threadIdx.x; i < (R + 1) * R; i += blockDim.x) {
+                const int c = i / R, a = i % R;          // c == R: the z row
+                const float v = red[a * (R + 1) + c];
+                const int n = c < R ? hl * R + c : hga * R + hl;
+                const int64_t idx = static_cast<int64_t>(n) * Kp + hl * R + a;
+                if (sizeof(T) == 4) {
+                    const float hi = to_tf32(v);
+                    reinterpret_cast<float *>(B)[idx] = hi;
+                    reinterpret_cast<float *>(B)[plane + idx] = to_tf32(v - hi);
+                } else {
+                    B[idx] = __float2bfloat16_rn(v);
+                }
+            }
+        }
+        __syncthreads();                            // red is rewritten by the next segment
     }
 }
 
@@ -400,11 +478,33 @@ glga_status stats_setup(Ctx *c) {
     int parts = 1;
     int64_t per = 0;
     plan_parts(c->N, nblk, c->num_sms, rows, 1 << 20, &parts, &per);
+    // Row ranges of at most `per` rows that never cross a segment boundary: each
+    // non-empty segment is cut into ceil(len / per) ranges, summed by the reduction in
+    // order.  Without segments this is the plain cut into `per`-row ranges.
+    std::vector<int32_t> pp(1, 0), sp(1, 0);
+    for (int64_t k = 0; k < c->n_seg; ++k) {
+        const int64_t a = c->seg_ptr[k], b = c->seg_ptr[k + 1];
+        for (int64_t r0 = a; r0 < b; r0 += per) pp.push_back(static_cast<int32_t>(std::min(b, r0 + per)));
+        sp.push_back(static_cast<int32_t>(pp.size() - 1));
+    }
+    parts = static_cast<int>(pp.size() - 1);
     c->stats_parts = parts;
     c->stats_rows_per_part = per;
     const size_t one = static_cast<size_t>(c->H) * c->r * (c->r + 1) * sizeof(float);
-    glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart), one * parts);
-    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->Sz), one);
+    if (one * std::max(parts, 1) > (size_t{4} << 30)) {
+        set_error("glga_create: %d statistics ranges need more than 4 GiB of partial sums", parts);
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart), one * std::max(parts, 1));
+    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->Sz), one * c->n_seg);
+    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->part_ptr), pp.size() * sizeof(int32_t));
+    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->seg_part_ptr), sp.size() * sizeof(int32_t));
+    if (st == GLGA_OK) {
+        cudaError_t e = cudaMemcpy(c->part_ptr, pp.data(), pp.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess)
+            e = cudaMemcpy(c->seg_part_ptr, sp.data(), sp.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "statistics ranges");
+    }
     if (st == GLGA_OK && c->N > 0)
         st = encode_kv_maps(c->KV, c->N, c->D, c->elem, &c->tmK.map, &c->tmV.map, rows);
     return st;
@@ -417,6 +517,7 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
         p.D = c->D;
         p.H = c->H;
         p.rows_per_part = c->stats_rows_per_part;
+        p.part_ptr = c->part_ptr;
         p.stages = c->io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
         p.part = c->Spart;
         p.flag = c->dev_flag;
@@ -434,14 +535,43 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
     }
     const int total = c->H * c->r * (c->r + 1);
     const int P = c->N > 0 ? c->stats_parts : 0;
-    const int64_t plane = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
+    const int64_t seg_stride = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
+    const int64_t plane = c->n_seg * seg_stride;
+    const dim3 rgrid(static_cast<unsigned>(ceil_div(total, 32)),
+                     static_cast<unsigned>(std::min<int64_t>(c->n_seg, 65535)));
+    // with no rows every segment's sums are zero (no ranges to add)
+    const int32_t *spp = c->N > 0 ? c->seg_part_ptr : nullptr;
+    if (c->n_seg > 1 && spp) {
+        const dim3 sgrid(static_cast<unsigned>(c->H),
+                         static_cast<unsigned>(std::min<int64_t>(c->n_seg, 65535)));
+        const size_t red_bytes = static_cast<size_t>(c->r) * (c->r + 1) * sizeof(float);   // <= 66 KB
+        if (c->io == GLGA_F32) {
+            GLGA_CUDA(cudaFuncSetAttribute(stats_reduce_segments_kernel<float>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(red_bytes)));
+            stats_reduce_segments_kernel<float><<<sgrid, 256, red_bytes, s>>>(
+                c->Spart, spp, c->n_seg, c->H, c->r, c->Sz, static_cast<float *>(c->Bro), c->ro_hg,
+                c->ro_bn, c->ro_kp, seg_stride, plane);
+        } else {
+            GLGA_CUDA(cudaFuncSetAttribute(stats_reduce_segments_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(red_bytes)));
+            stats_reduce_segments_kernel<__nv_bfloat16><<<sgrid, 256, red_bytes, s>>>(
+                c->Spart, spp, c->n_seg, c->H, c->r, c->Sz, static_cast<__nv_bfloat16 *>(c->Bro),
+                c->ro_hg, c->ro_bn, c->ro_kp, seg_stride, plane);
+        }
+        GLGA_CUDA(cudaGetLastError());
+        c->launches += 1;
+        return GLGA_OK;
+    }
     if (c->io == GLGA_F32)
-        stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
-            c->Spart, P, c->H, c->r, c->Sz, static_cast<float *>(c->Bro), c->ro_hg, c->ro_bn, c->ro_kp, plane);
+        stats_reduce_kernel<float><<<rgrid, 256, 0, s>>>(
+            c->Spart, P, spp, c->n_seg, c->H, c->r, c->Sz, static_cast<float *>(c->Bro), c->ro_hg,
+            c->ro_bn, c->ro_kp, seg_stride, plane);
     else
-        stats_reduce_kernel<__nv_bfloat16><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
-            c->Spart, P, c->H, c->r, c->Sz, static_cast<__nv_bfloat16 *>(c->Bro), c->ro_hg, c->ro_bn,
-            c->ro_kp, plane);
+        stats_reduce_kernel<__nv_bfloat16><<<rgrid, 256, 0, s>>>(
+            c->Spart, P, spp, c->n_seg, c->H, c->r, c->Sz, static_cast<__nv_bfloat16 *>(c->Bro),
+            c->ro_hg, c->ro_bn, c->ro_kp, seg_stride, plane);
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -547,6 +677,7 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         p.D = static_cast<int32_t>(D);
         p.H = H;
         p.rows_per_part = per;
+        p.part_ptr = nullptr;
         p.stages = io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
         p.part = scratch;
         p.flag = flag;
@@ -561,7 +692,7 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
     }
     const int total = static_cast<int>(per_part);
     stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
-        scratch, parts, H, r, Sz, nullptr, 1, 0, 0, 0);
+        scratch, parts, nullptr, 1, H, r, static_cast<float *>(Sz), static_cast<float *>(nullptr), 1, 1, 1, 0, 0);
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;
 }

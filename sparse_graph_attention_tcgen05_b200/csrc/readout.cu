@@ -24,6 +24,7 @@
 // head group is not a whole number of 128-byte column boxes use per-thread global loads
 // and stores in the epilogue instead of the L/Y buffers.
 #include <algorithm>
+#include <vector>
 
 #include "glga_internal.cuh"
 
@@ -56,6 +57,7 @@ struct ReadoutParams {
     int32_t lboxes;         // 128-byte column boxes of the group's L/Y tile (0: no TMA path)
     int32_t lbufs;          // L/Y staging buffers (2 or 3)
     int32_t b_resident;     // B_g loaded once per CTA (grid is a multiple of n_groups)
+    const int32_t *tile_seg;  // segment of each row tile (NULL: one segment)
     uint32_t a_bytes, b_bytes, stage_bytes;
     uint32_t bres_bytes;    // resident B_g: planes x nk x b_bytes (0 when streamed)
     const void *L;          // io [N, D]
@@ -218,11 +220,21 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
             int it = 0;
             RingPos rp;
             TileWalk tw(blockIdx.x, gridDim.x, p.n_groups);
+            // with segments, B_g of the tile's segment: rows (seg * n_groups + g) * BNr of
+            // the operand; the segment id is loaded one tile ahead
+            int seg_next = (p.tile_seg && n_my > 0) ? __ldg(p.tile_seg + tw.row) : 0;
             bool ok = true;
             for (int i = 0; i < n_my && ok; ++i, tw.next()) {
                 const int g = tw.col;
                 const int32_t m0 = tw.row * kBM;
                 const int qx0 = g * p.hg * R;
+                const int seg = seg_next;
+                if (p.tile_seg && i + 1 < n_my) {
+                    TileWalk nx = tw;
+                    nx.next();
+                    seg_next = __ldg(p.tile_seg + nx.row);
+                }
+                const int32_t brow = (seg * p.n_groups + g) * p.BNr;
                 for (int kb = 0; kb < p.nk; ++kb, ++it, rp.next(p.stages)) {
                     const int s = rp.slot;
                     if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
@@ -237,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                     tma_load_2d(st, &tmQ, &full_bar[s], qx0 + kb * KT, m0);
                     if (!p.b_resident) {
                         uint8_t *bst = st + a_planes;
-                        tma_load_2d(bst, &tmB0, &full_bar[s], kb * KT, g * p.BNr);
-                        if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kb * KT, g * p.BNr);
+                        tma_load_2d(bst, &tmB0, &full_bar[s], kb * KT, brow);
+                        if (kPlanes == 2) tma_load_2d(bst + p.b_bytes, &tmB1, &full_bar[s], kb * KT, brow);
                     }
                 }
             }
@@ -494,6 +506,44 @@ glga_status launch_readout_r(Ctx *c, const ReadoutParams &p, unsigned grid, size
     return GLGA_OK;
 }
 
+// Rows whose segment differs from the segment of their 128-row tile's first row (tiles
+// that straddle a segment boundary): the tile GEMM used the first row's S, z for them,
+// so they are redone here on the CUDA cores, one warp per row, with their own segment's
+// fp32 statistics: G_i = phi(q_i)^T S / (phi(q_i)^T z + eps), then the same gate blend
+// with L_i as the tile epilogue.
+constexpr int kFixRowsPerBlock = 4;
+constexpr int kFixMaxD = 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(32 * kFixRowsPerBlock) readout_fixup_kernel(
+    const int32_t *__restrict__ rows, const int32_t *__restrict__ segs, int64_t n,
+    const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t,
+    const float *__restrict__ Sz, int64_t n_seg, int H, int R, float b_g, float eps, T *__restrict__ Y) {
+    __shared__ float ph[kFixRowsPerBlock][kFixMaxD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * kFixRowsPerBlock + warp;
+    if (m >= n) return;   // warp-uniform; no block-wide barrier follows
+    const int64_t row = rows[m], seg = segs[m];
+    const int D = H * R;
+    for (int c = lane; c < D; c += 32) ph[warp][c] = phi(IoT<T>::get(Q + row * D + c));
+    __syncwarp();
+    const float gate = 1.f / (1.f + __expf(-(t[row] + b_g)));
+    const int64_t hrr = static_cast<int64_t>(H) * R * R;
+    const float *S = Sz + seg * hrr;
+    const float *z = Sz + n_seg * hrr + seg * H * R;
+    for (int c = lane; c < D; c += 32) {
+        const int h = c / R, cc = c - h * R;
+        float num = 0.f, den = 0.f;
+        for (int a = 0; a < R; ++a) {
+            const float f = ph[warp][h * R + a];
+            num = fmaf(f, S[(static_cast<int64_t>(h) * R + a) * R + cc], num);
+            den = fmaf(f, z[h * R + a], den);
+        }
+        const float y = gate * IoT<T>::get(L + row * D + c) + (1.f - gate) * num / (den + eps);
+        IoT<T>::put(Y + row * D + c, y);
+    }
+}
+
 }  // namespace
 
 glga_status readout_setup(Ctx *c) {
@@ -509,7 +559,14 @@ glga_status readout_setup(Ctx *c) {
     const int last = c->H - (c->ro_groups - 1) * c->ro_hg;
     c->ro_tma_epi = (c->ro_hg * c->r) % kt == 0 && (last * c->r) % kt == 0;
     const int planes = c->split == 3 ? 2 : 1;
-    const size_t plane = static_cast<size_t>(c->ro_groups) * c->ro_bn * c->ro_kp * c->elem;
+    // one operand per segment and group: [planes][n_seg][groups][BNr][Kp]
+    const uint64_t b_rows = static_cast<uint64_t>(c->n_seg) * c->ro_groups * c->ro_bn;
+    const size_t plane = static_cast<size_t>(b_rows) * c->ro_kp * c->elem;
+    if (b_rows >= (uint64_t{1} << 31) || planes * plane > (size_t{4} << 30)) {
+        set_error("glga_create: %lld segments need more than 4 GiB of readout operands",
+                  static_cast<long long>(c->n_seg));
+        return GLGA_ERR_UNSUPPORTED;
+    }
     glga_status st = dev_alloc(c, &c->Bro, planes * plane);
     if (st != GLGA_OK) return st;
     cudaError_t e = cudaMemset(c->Bro, 0, planes * plane);   // off-diagonal blocks stay zero
@@ -518,8 +575,7 @@ glga_status readout_setup(Ctx *c) {
         c->io == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     for (int pl = 0; pl < planes; ++pl) {
         st = encode_tmap_2d(&c->tmBro[pl].map, dt, static_cast<uint8_t *>(c->Bro) + pl * plane,
-                            c->ro_kp, static_cast<uint64_t>(c->ro_groups) * c->ro_bn,
-                            static_cast<uint64_t>(c->ro_kp) * c->elem, kt, c->ro_bn);
+                            c->ro_kp, b_rows, static_cast<uint64_t>(c->ro_kp) * c->elem, kt, c->ro_bn);
         if (st != GLGA_OK) return st;
         c->tmBro[pl].valid = true;
     }
@@ -531,6 +587,31 @@ glga_status readout_setup(Ctx *c) {
         if (st == GLGA_OK) st = encode_tmap_2d(&c->tmL.map, dt, c->L, c->D, c->N, rb, kt, kBM);
         if (st != GLGA_OK) return st;
         c->tmQ.valid = c->tmL.valid = true;
+    }
+    if (c->n_seg > 1 && c->N > 0) {
+        // segment of every tile's first row, and the rows whose segment differs from it
+        const int64_t m_tiles = ceil_div(c->N, kBM);
+        std::vector<int32_t> ts(static_cast<size_t>(m_tiles)), fr, fs;
+        int64_t k = 0;
+        for (int64_t row = 0; row < c->N; ++row) {
+            while (c->seg_ptr[k + 1] <= row) ++k;   // skips empty segments
+            if (row % kBM == 0) ts[static_cast<size_t>(row / kBM)] = static_cast<int32_t>(k);
+            else if (k != ts[static_cast<size_t>(row / kBM)]) {
+                fr.push_back(static_cast<int32_t>(row));
+                fs.push_back(static_cast<int32_t>(k));
+            }
+        }
+        c->n_fix = static_cast<int64_t>(fr.size());
+        st = dev_alloc(c, reinterpret_cast<void **>(&c->tile_seg), ts.size() * sizeof(int32_t));
+        if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->fix_row), (fr.size() + 1) * sizeof(int32_t));
+        if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->fix_seg), (fs.size() + 1) * sizeof(int32_t));
+        if (st != GLGA_OK) return st;
+        e = cudaMemcpy(c->tile_seg, ts.data(), ts.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && !fr.empty())
+            e = cudaMemcpy(c->fix_row, fr.data(), fr.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess && !fs.empty())
+            e = cudaMemcpy(c->fix_seg, fs.data(), fs.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "segment tables");
     }
     return GLGA_OK;
 }
@@ -558,7 +639,8 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     const int64_t bres = static_cast<int64_t>(planes) * p.nk * p.b_bytes;
     p.b_resident = 0;
     p.lbufs = 0;
-    for (int resident = 1; resident >= 0 && p.lbufs == 0; --resident) {
+    // B_g stays resident only with one segment (otherwise it changes with the tile)
+    for (int resident = c->n_seg == 1 ? 1 : 0; resident >= 0 && p.lbufs == 0; --resident) {
         const int64_t stage = planes * (p.a_bytes + (resident ? 0 : p.b_bytes));
         const int64_t fixed = resident ? bres : 0;
         for (int nb = 3; nb >= 2 && p.lbufs == 0; --nb) {
@@ -601,6 +683,7 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     p.b_g = b_g;
     p.eps = eps;
     p.flag = c->dev_flag;
+    p.tile_seg = c->n_seg > 1 ? c->tile_seg : nullptr;
     const CUtensorMapDataType dt =
         c->io == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap my = c->tmL.map;   // placeholder when the TMA store path is off
@@ -612,9 +695,28 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s) {
     const size_t smem = static_cast<size_t>(p.bres_bytes) + static_cast<size_t>(p.stages) * p.stage_bytes +
                         lbytes + 1024;
     const CUtensorMap &b1 = planes == 2 ? c->tmBro[1].map : c->tmBro[0].map;
+    glga_status st =
+        c->io == GLGA_F32
+            ? launch_readout_r<3, float>(c, p, static_cast<unsigned>(grid), smem, c->tmQ.map,
+                                         c->tmBro[0].map, b1, c->tmL.map, my, s)
+            : launch_readout_r<1, __nv_bfloat16>(c, p, static_cast<unsigned>(grid), smem, c->tmQ.map,
+                                                 c->tmBro[0].map, b1, c->tmL.map, my, s);
+    if (st != GLGA_OK || c->n_fix == 0) return st;
+    // rows in a later segment than their tile's first row: redo them with their own S, z
+    const unsigned fgrid = static_cast<unsigned>(ceil_div(c->n_fix, kFixRowsPerBlock));
     if (c->io == GLGA_F32)
-        return launch_readout_r<3, float>(c, p, static_cast<unsigned>(grid), smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
-    return launch_readout_r<1, __nv_bfloat16>(c, p, static_cast<unsigned>(grid), smem, c->tmQ.map, c->tmBro[0].map, b1, c->tmL.map, my, s);
+        readout_fixup_kernel<float><<<fgrid, 32 * kFixRowsPerBlock, 0, s>>>(
+            c->fix_row, c->fix_seg, c->n_fix, static_cast<const float *>(c->Q),
+            static_cast<const float *>(c->L), c->t, c->Sz, c->n_seg, c->H, c->r, b_g, eps,
+            static_cast<float *>(Y));
+    else
+        readout_fixup_kernel<__nv_bfloat16><<<fgrid, 32 * kFixRowsPerBlock, 0, s>>>(
+            c->fix_row, c->fix_seg, c->n_fix, static_cast<const __nv_bfloat16 *>(c->Q),
+            static_cast<const __nv_bfloat16 *>(c->L), c->t, c->Sz, c->n_seg, c->H, c->r, b_g, eps,
+            static_cast<__nv_bfloat16 *>(Y));
+    GLGA_CUDA(cudaGetLastError());
+    c->launches += 1;
+    return GLGA_OK;
 }
 
 }  // namespace glga

@@ -11,6 +11,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
         "glga_create": ([ctypes.POINTER(_vp), _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
                          ctypes.POINTER(Options), _vp], _i32),
         "glga_forward": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _vp], _i32),
+        "glga_create_segmented": ([ctypes.POINTER(_vp), _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
+                                   _vp, _i64, ctypes.POINTER(Options), _vp], _i32),
         "glga_destroy": ([_vp], _i32),
         "glga_csr_from_coo": ([_i64, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_bucket_counts": ([_vp, ctypes.POINTER(_i64)], _i32),
@@ -141,10 +144,12 @@ class Layer:
     """One gated local-global graph-attention layer bound to a fixed graph.
 
     `row_ptr`/`col_idx` are CUDA int32 tensors (target-grouped CSR).  `io` is "f32" or
-    "bf16": the element type of X, the weights and Y."""
+    "bf16": the element type of X, the weights and Y.  `segments` (optional) are the
+    n_seg + 1 node offsets of a batch of graphs (glga_create_segmented): each segment gets
+    its own global statistics."""
 
     def __init__(self, N, d, H, r, io, row_ptr, col_idx, options: Options | None = None,
-                 stream=None):
+                 stream=None, segments=None):
         self.N, self.d, self.H, self.r, self.io = int(N), int(d), int(H), int(r), io
         self.D = self.H * self.r
         self.dtype = torch_dtype(io)
@@ -154,11 +159,20 @@ class Layer:
         self.E = int(col_idx.numel())
         h = ctypes.c_void_p()
         opt = ctypes.byref(options) if options is not None else None
-        _check(lib().glga_create(ctypes.byref(h), self.N, self.d, self.H, self.r,
-                                 GLGA_F32 if io == "f32" else GLGA_BF16,
-                                 _ptr(row_ptr.contiguous()),
-                                 _ptr(col_idx.contiguous()) if self.E else None, self.E, opt,
-                                 _stream(stream)), "glga_create")
+        io_code = GLGA_F32 if io == "f32" else GLGA_BF16
+        rpt, cit = row_ptr.contiguous(), col_idx.contiguous()   # alive through create
+        rp = _ptr(rpt)
+        ci = _ptr(cit) if self.E else None
+        if segments is None:
+            self.n_seg = None
+            _check(lib().glga_create(ctypes.byref(h), self.N, self.d, self.H, self.r, io_code, rp, ci,
+                                     self.E, opt, _stream(stream)), "glga_create")
+        else:
+            seg = np.ascontiguousarray(np.asarray(segments, dtype=np.int64))
+            self.n_seg = int(seg.shape[0]) - 1
+            _check(lib().glga_create_segmented(ctypes.byref(h), self.N, self.d, self.H, self.r, io_code,
+                                               rp, ci, self.E, seg.ctypes.data, self.n_seg, opt,
+                                               _stream(stream)), "glga_create_segmented")
         self._h = h
 
     # -- forward ---------------------------------------------------------------------
@@ -200,11 +214,13 @@ class Layer:
                "K": torch.empty(self.N, self.D, dtype=self.dtype, device=dev),
                "V": torch.empty(self.N, self.D, dtype=self.dtype, device=dev),
                "t": torch.empty(self.N, dtype=torch.float32, device=dev),
-               "S": torch.empty(self.H, self.r, self.r, dtype=torch.float32, device=dev),
-               "z": torch.empty(self.H, self.r, dtype=torch.float32, device=dev),
+               "S": torch.empty(self.n_seg or 1, self.H, self.r, self.r, dtype=torch.float32, device=dev),
+               "z": torch.empty(self.n_seg or 1, self.H, self.r, dtype=torch.float32, device=dev),
                "L": torch.empty(self.N, self.D, dtype=self.dtype, device=dev)}
         _check(lib().glga_get_intermediates(self._h, *(_ptr(out[k]) for k in ("Q", "K", "V", "t", "S", "z", "L")),
                                             _stream(stream)), "glga_get_intermediates")
+        if self.n_seg is None:           # one global segment: S [H, r, r], z [H, r]
+            out["S"], out["z"] = out["S"][0], out["z"][0]
         return out
 
     def set_timing(self, enable: bool):

@@ -2,6 +2,8 @@
 include/glga.h declares, and rejects bad arguments on the host before touching a GPU."""
 import ctypes
 
+import numpy as np
+
 import pytest
 
 from sparse_graph_attention_tcgen05_b200 import glga
@@ -78,3 +80,18 @@ def test_debug_entry_points_reject_a_null_context():
     L = glga.lib()
     assert L.glga_debug_bounded_wait(None, 1_000_000, None) == 1
     assert L.glga_debug_set_col_idx(None, 0, 0, None) == 1
+
+
+def test_segmented_create_rejects_malformed_segments():
+    """Host-side checks of glga_create_segmented (before any device call)."""
+    L = glga.lib()
+    h = ctypes.c_void_p()
+    N = 10
+    for seg in ([1, N], [0, N - 1], [0, 6, 4, N]):
+        arr = np.array(seg, dtype=np.int64)
+        assert L.glga_create_segmented(ctypes.byref(h), N, 8, 1, 8, 0, 16, 16, 0, arr.ctypes.data,
+                                       len(seg) - 1, None, None) == 1
+    arr = np.array([0, N], dtype=np.int64)
+    assert L.glga_create_segmented(ctypes.byref(h), N, 8, 1, 8, 0, 16, 16, 0, None, 1, None, None) == 1
+    assert L.glga_create_segmented(ctypes.byref(h), N, 8, 1, 8, 0, 16, 16, 0, arr.ctypes.data, 0,
+                                   None, None) == 1
