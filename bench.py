@@ -201,6 +201,61 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0):
+    """Forward time against N at fixed in-degree: the tiny config's shape (d=32, H=1,
+    r=16, fp32, k distinct uniform in-neighbours + self-loop; the method page's cost-proxy
+    setting |E|/N = 8, r = 16) at N = 2^e for each e.  Median of `steps` forwards, each
+    timed with CUDA events on the launching stream, L2 flushed between them.  Returns
+    [(N, E, ms)]."""
+    import torch
+    from sparse_graph_attention_tcgen05_b200 import glga
+    from sparse_graph_attention_tcgen05_b200.workloads import make_custom, uniform_in_neighbours
+    dev = torch.device("cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    out = []
+    for e in exponents:
+        N = 1 << e
+        src, dst = uniform_in_neighbours(N, k, seed)
+        w = make_custom(N, 32, 1, 16, src, dst, io="f32", seed=seed + 1)
+        row_ptr, col_idx = glga.csr_from_coo(N, torch.from_numpy(src).to(dev), torch.from_numpy(dst).to(dev))
+        layer = glga.Layer(N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+        args = [torch.from_numpy(a).to(dev) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+        Y = torch.empty(N, w.D, dtype=torch.float32, device=dev)
+        for _ in range(warmup):
+            layer.forward(*args, b_g=w.b_g, eps=w.eps, Y=Y)
+        times = []
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(steps):
+            flush.zero_()
+            ev0.record(stream)
+            layer.forward(*args, b_g=w.b_g, eps=w.eps, Y=Y)
+            ev1.record(stream)
+            ev1.synchronize()
+            times.append(ev0.elapsed_time(ev1))
+        assert layer.last_device_error() == 0
+        layer.close()
+        out.append((N, w.E, float(np.median(times))))
+    return out
+
+
+def loglog_slope(points):
+    """Least-squares slope of log(ms) against log(N)."""
+    x = np.log([p[0] for p in points])
+    y = np.log([p[2] for p in points])
+    return float(np.polyfit(x, y, 1)[0])
+
+
+def run_sweep():
+    pts = sweep_points(range(12, 22))
+    upper = [p for p in pts if p[0] >= (1 << 17)]
+    print(json.dumps({"sweep": "forward ms vs N at fixed in-degree 8 (+ self-loop), d=32, H=1, "
+                               "r=16, fp32; median of 30, L2 flushed",
+                      "points": [{"N": n, "E": e, "ms": ms} for n, e, ms in pts],
+                      "slope_loglog_all": loglog_slope(pts),
+                      "slope_loglog_N_ge_2^17": loglog_slope(upper)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -216,8 +271,13 @@ def main():
     ap.add_argument("--segment-len", type=int, default=0,
                     help="segments of this many nodes, each with its own global statistics "
                          "(a batch of graphs; 0 = one segment over all nodes)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the forward against N at fixed degree instead (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.sweep:
+        run_sweep()
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -22,7 +22,7 @@ import dataclasses
 import numpy as np
 
 __all__ = ["Workload", "CONFIGS", "make_workload", "round_to_bf16", "chung_lu_weights",
-           "make_custom"]
+           "make_custom", "uniform_in_neighbours"]
 
 
 @dataclasses.dataclass
@@ -280,6 +280,31 @@ def make_workload(name: str, seed: int = 0, scale: float = 1.0) -> Workload:
         raise KeyError(f"unknown workload {name!r}; known: {sorted(CONFIGS)}")
     eps = 1e-6
     return Workload(name, N, d, H, r, io, src, dst, X, WQ, WK, WV, wg, bg, eps, seed)
+
+
+def uniform_in_neighbours(N, k, seed):
+    """k distinct uniform in-neighbours != i for every node i, plus its self-loop, in O(N k)
+    (rows with a repeated draw are redrawn).  Used for size sweeps at fixed degree, where
+    the tiny config's exact sampler (quadratic in N) does not scale."""
+    rng = np.random.default_rng(np.random.PCG64(seed))
+    if N < 2 or k < 1:
+        loop = np.arange(N, dtype=np.int32)
+        return loop, loop.copy()
+    k = min(k, N - 1)
+    node = np.arange(N, dtype=np.int64)
+    src = np.empty((N, k), dtype=np.int64)
+    todo = node
+    while todo.size:
+        v = rng.integers(0, N - 1, (todo.size, k))
+        v = np.where(v >= todo[:, None], v + 1, v)        # skip the node itself
+        v.sort(axis=1)
+        dup = (v[:, 1:] == v[:, :-1]).any(axis=1) if k > 1 else np.zeros(todo.size, bool)
+        src[todo[~dup]] = v[~dup]
+        todo = todo[dup]
+    dst = np.repeat(node, k)
+    src = np.concatenate([src.reshape(-1), node]).astype(np.int32)
+    dst = np.concatenate([dst, node]).astype(np.int32)
+    return src, dst
 
 
 def make_custom(N, d, H, r, src, dst, io="f32", seed=0, b_g=0.0, eps=1e-6,
