@@ -256,6 +256,87 @@ def run_sweep():
                       "slope_loglog_N_ge_2^17": loglog_slope(upper)}), flush=True)
 
 
+def run_sharded(args, rank, world, local_rank):
+    """Row-sharded forward (sharded.ShardedForward): every rank owns a contiguous block of
+    target rows with about equal CSR entries, projects them, exchanges K/V rows and
+    partial statistics over NCCL and finishes its rows.  Total work is fixed as ranks are
+    added (strong scaling); value = E*H per step over the slowest rank's time."""
+    import torch
+    import torch.distributed as dist
+    from sparse_graph_attention_tcgen05_b200 import glga
+    from sparse_graph_attention_tcgen05_b200.sharded import (LibraryShard, ShardedForward,
+                                                             partition_rows, shard_csr)
+    from sparse_graph_attention_tcgen05_b200.workloads import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    elif world == 1 and not dist.is_initialized():
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    w = make_workload(args.workload, scale=args.scale)
+    dt = glga.torch_dtype(w.io)
+    row_ptr, col_idx = glga.csr_from_coo(w.N, torch.from_numpy(w.src).to(dev), torch.from_numpy(w.dst).to(dev))
+    rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
+    bounds = partition_rows(rp, world)
+    b0, b1 = int(bounds[rank]), int(bounds[rank + 1])
+    rpo, cio = shard_csr(rp, ci, b0, b1)
+    shard = LibraryShard(w.N, w.d, w.H, w.r, w.io, rpo, cio, b0, b1, device=dev)
+    fwd = ShardedForward(shard, bounds, rank, world)
+    X = torch.from_numpy(np.ascontiguousarray(w.X[b0:b1])).to(dt).to(dev)
+    W = [torch.from_numpy(a).to(dt).to(dev) for a in (w.W_Q, w.W_K, w.W_V, w.w_g)]
+    Y = torch.empty(b1 - b0, w.D, dtype=dt, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fwd(X, *W, w.b_g, w.eps, Y)
+    torch.cuda.synchronize()
+    assert shard.last_device_error() == 0
+    parity = None
+    if not args.no_parity and b1 > b0:
+        import oracle
+        rng = np.random.default_rng(rank)
+        rows = np.unique(rng.integers(b0, b1, min(256, b1 - b0)))
+        ref = oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
+                             rp, ci, rows=rows)
+        got = Y.float().cpu().numpy()[rows - b0].astype(np.float64)
+        parity = float(np.abs(got - ref["Y"]).max() / np.abs(ref["Y"]).max())
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        ev0.record(stream)
+        fwd(X, *W, w.b_g, w.eps, Y)
+        ev1.record(stream)
+        ev1.synchronize()
+        step_ms.append(ev0.elapsed_time(ev1))
+    torch.cuda.synchronize()
+    dist.barrier()
+    total = max_over_ranks_dist(sum(step_ms), world, dev)
+    assert shard.last_device_error() == 0
+    line = {"metric": METRIC, "value": w.E * w.H * args.steps / (total * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": w.io, "data": "synthetic",
+            "config": {"workload": args.workload if args.scale == 1.0 else f"{args.workload}@scale{args.scale}",
+                       "N": w.N, "E": w.E, "d": w.d, "H": w.H, "r": w.r, "io": w.io,
+                       "parallelism": f"row-sharded x{world} (NCCL: K/V broadcasts, partial S|z all-gather)",
+                       "rows_per_rank": [int(x) for x in np.diff(bounds)],
+                       "l2": "flushed between timed steps (256 MiB write, outside the timed spans)"},
+            "parity_max_rel_err": parity}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    shard.close()
+    dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -271,6 +352,8 @@ def main():
     ap.add_argument("--segment-len", type=int, default=0,
                     help="segments of this many nodes, each with its own global statistics "
                          "(a batch of graphs; 0 = one segment over all nodes)")
+    ap.add_argument("--sharded", action="store_true",
+                    help="row-sharded forward across the ranks (strong scaling) instead of replicas")
     ap.add_argument("--sweep", action="store_true",
                     help="time the forward against N at fixed degree instead (one JSON line)")
     args = ap.parse_args()
@@ -284,6 +367,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.sharded:
+        run_sharded(args, rank, world, local_rank)
         return
 
     import torch

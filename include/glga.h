@@ -150,6 +150,39 @@ GLGA_API glga_status glga_csr_from_coo(int64_t N, int64_t E, const int32_t *src,
  * the number of bucket-2 chunks.                                                      */
 GLGA_API glga_status glga_bucket_counts(const glga_ctx *ctx, int64_t *counts);
 
+/* Row-sharded forward (one context per rank; one process per GPU).  Target rows are cut
+ * into contiguous blocks; rank p owns rows [row_begin, row_end) of the n_nodes nodes.
+ * The one exchange step of the method, moved by the caller (NCCL over NVLink, e.g.
+ * torch.distributed): every rank's K/V rows to every rank, and the per-rank partial
+ * statistics (method page "Gated Local-Global Graph Attention", "Key formulas": S and z
+ * are sums over all nodes, so they split into per-rank partial sums).
+ *
+ * glga_create_sharded -- row_ptr (device) int32 [n_own + 1] and col_idx (device) int32
+ *   [E] are the CSR of the owned rows only (row_ptr[0] = 0, local row numbering), with
+ *   column indices in [0, n_nodes) (global node ids).  kv (device, caller-owned, 16-byte
+ *   aligned, io [n_nodes, 2*H*r], row j = k_j | v_j) is the K/V buffer the rank's
+ *   projection writes its rows into (rows row_begin .. row_end-1) and that the exchange
+ *   fills with the other ranks' rows; it must outlive the context.  Other arguments and
+ *   errors as glga_create.
+ * glga_forward_begin -- X (device) io [n_own, d]: the owned rows' inputs.  Projects them
+ *   (Q, t into the context; k, v into kv) and writes the rank's partial statistics to
+ *   own_partial (device) float [H][r][r+1] (per head, row a: S_h[a][0..r-1] then z_h[a]).
+ * glga_forward_end -- after the exchange: partials (device) float [P][H][r][r+1] holds the
+ *   P ranks' partials in rank order and kv holds every node's k/v.  Sums the partials in
+ *   a fixed order (the same on every rank), then computes the owned rows' Y (device, io
+ *   [n_own, H*r]).
+ * Both are stream-ordered with no host synchronisation.  glga_forward refuses a sharded
+ * context; glga_get_intermediates returns the owned rows.                             */
+GLGA_API glga_status glga_create_sharded(glga_ctx **out, int64_t n_nodes, int64_t row_begin,
+                        int64_t row_end, int32_t d, int32_t H, int32_t r, glga_dtype io,
+                        const int32_t *row_ptr, const int32_t *col_idx, int64_t E, void *kv,
+                        const glga_options *opts, void *stream);
+GLGA_API glga_status glga_forward_begin(glga_ctx *ctx, const void *X, const void *W_Q,
+                        const void *W_K, const void *W_V, const void *w_g, float *own_partial,
+                        void *stream);
+GLGA_API glga_status glga_forward_end(glga_ctx *ctx, const float *partials, int32_t P, float b_g,
+                        float eps, void *Y, void *stream);
+
 /* Copies the bucket lists (device -> device, on `stream`) into caller buffers sized by
  * glga_bucket_counts: warp_rows [counts[0]], cta_rows [counts[1]], split_rows [counts[2]],
  * chunk_row [counts[3]], chunk_begin [counts[3]] (the CSR offset of the chunk's first

@@ -72,6 +72,7 @@ glga_status dev_alloc(Ctx *c, void **p, size_t bytes) {
 // caller).
 static void release_ctx(Ctx *c) {
     if (!c) return;
+    if (c->kv_external) c->KV = nullptr;   // the caller's buffer
     void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
                     c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
@@ -90,6 +91,13 @@ using namespace glga;
 struct glga_ctx {
     Ctx c;
 };
+
+namespace {
+glga_status create_impl(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t r, glga_dtype io,
+                        const int32_t *row_ptr, const int32_t *col_idx, int64_t E,
+                        const int64_t *seg_ptr, int64_t n_seg, const glga_options *opts,
+                        void *stream, int64_t n_src, int64_t row0, void *kv_ext);
+}  // namespace
 
 extern "C" {
 
@@ -132,6 +140,33 @@ glga_status glga_create_segmented(glga_ctx **out, int64_t N, int32_t d, int32_t 
                                   glga_dtype io, const int32_t *row_ptr, const int32_t *col_idx,
                                   int64_t E, const int64_t *seg_ptr, int64_t n_seg,
                                   const glga_options *opts, void *stream) {
+    return create_impl(out, N, d, H, r, io, row_ptr, col_idx, E, seg_ptr, n_seg, opts, stream, N, 0,
+                       nullptr);
+}
+
+glga_status glga_create_sharded(glga_ctx **out, int64_t n_nodes, int64_t row_begin, int64_t row_end,
+                                int32_t d, int32_t H, int32_t r, glga_dtype io,
+                                const int32_t *row_ptr, const int32_t *col_idx, int64_t E,
+                                void *kv, const glga_options *opts, void *stream) {
+    if (n_nodes < 0 || n_nodes > 2147483646LL || row_begin < 0 || row_end < row_begin ||
+        row_end > n_nodes || !kv || (reinterpret_cast<uintptr_t>(kv) & 15u)) {
+        if (out) *out = nullptr;
+        set_error("glga_create_sharded: need 0 <= row_begin <= row_end <= n_nodes < 2^31-1 and a "
+                  "16-byte aligned K/V buffer");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    const int64_t n_own = row_end - row_begin;
+    const int64_t seg[2] = {0, n_own};
+    return create_impl(out, n_own, d, H, r, io, row_ptr, col_idx, E, seg, 1, opts, stream, n_nodes,
+                       row_begin, kv);
+}
+}  // extern "C"
+
+namespace {
+glga_status create_impl(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t r, glga_dtype io,
+                        const int32_t *row_ptr, const int32_t *col_idx, int64_t E,
+                        const int64_t *seg_ptr, int64_t n_seg, const glga_options *opts,
+                        void *stream, int64_t n_src, int64_t row0, void *kv_ext) {
     if (!out) {
         set_error("glga_create: out is NULL");
         return GLGA_ERR_INVALID_ARG;
@@ -198,6 +233,9 @@ glga_status glga_create_segmented(glga_ctx **out, int64_t N, int32_t d, int32_t 
     c->opts = o;
     c->n_seg = n_seg;
     c->seg_ptr.assign(seg_ptr, seg_ptr + n_seg + 1);
+    c->n_src = n_src;
+    c->row0 = row0;
+    c->sharded = kv_ext != nullptr;
     glga_status st = GLGA_OK;
     cudaError_t e = cudaGetDevice(&c->device);
     if (e == cudaSuccess)
@@ -228,7 +266,13 @@ glga_status glga_create_segmented(glga_ctx **out, int64_t N, int32_t d, int32_t 
     TRY(validate_csr(c, s));
     TRY(build_buckets(c, s));
     TRY(dev_alloc(c, &c->Q, static_cast<size_t>(N) * D * elem));
-    TRY(dev_alloc(c, &c->KV, static_cast<size_t>(N) * 2 * D * elem));
+    if (kv_ext) {
+        c->KV = kv_ext;
+        c->kv_external = true;
+    } else {
+        TRY(dev_alloc(c, &c->KV, static_cast<size_t>(n_src) * 2 * D * elem));
+    }
+    if (st == GLGA_OK) c->kv_own = static_cast<uint8_t *>(c->KV) + static_cast<size_t>(row0) * 2 * D * elem;
     TRY(dev_alloc(c, reinterpret_cast<void **>(&c->t), static_cast<size_t>(N) * sizeof(float)));
     TRY(projection_setup(c));
     TRY(readout_setup(c));
@@ -249,6 +293,9 @@ glga_status glga_create_segmented(glga_ctx **out, int64_t N, int32_t d, int32_t 
     *out = h;
     return GLGA_OK;
 }
+}  // namespace
+
+extern "C" {
 
 glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void *W_K,
                          const void *W_V, const void *w_g, float b_g, float eps, void *Y,
@@ -269,6 +316,10 @@ glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void
     const uintptr_t align_or = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Y);
     if (align_or & 15u) {
         set_error("glga_forward: X and Y must be 16-byte aligned");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (c->sharded) {
+        set_error("glga_forward: a row-sharded context runs glga_forward_begin / glga_forward_end");
         return GLGA_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -312,6 +363,50 @@ glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void
         c->ev_recorded = true;
     }
     return GLGA_OK;
+}
+
+glga_status glga_forward_begin(glga_ctx *h, const void *X, const void *W_Q, const void *W_K,
+                               const void *W_V, const void *w_g, float *own_partial, void *stream) {
+    if (!h || !h->c.sharded) {
+        set_error("glga_forward_begin: needs a context from glga_create_sharded");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    if (!W_Q || !W_K || !W_V || !w_g || !own_partial || (c->N > 0 && !X) ||
+        (reinterpret_cast<uintptr_t>(X) & 15u)) {
+        set_error("glga_forward_begin: null or misaligned pointer argument");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    nvtxRangePushA("glga_forward_begin");
+    glga_status st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, false);
+    if (st == GLGA_OK) st = stats_run_partial(c, own_partial, s);
+    nvtxRangePop();
+    return st;
+}
+
+glga_status glga_forward_end(glga_ctx *h, const float *partials, int32_t P, float b_g, float eps,
+                             void *Y, void *stream) {
+    if (!h || !h->c.sharded) {
+        set_error("glga_forward_end: needs a context from glga_create_sharded");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    if (!partials || P < 1 || (c->N > 0 && !Y) || (reinterpret_cast<uintptr_t>(Y) & 15u)) {
+        set_error("glga_forward_end: need partials of P >= 1 ranks and a 16-byte aligned Y");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (!(eps > 0.f) || !std::isfinite(eps) || !std::isfinite(b_g)) {
+        set_error("glga_forward_end: eps must be finite and > 0, b_g finite");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    nvtxRangePushA("glga_forward_end");
+    glga_status st = stats_finish(c, partials, P, s);
+    if (st == GLGA_OK) st = local_run(c, s);
+    if (st == GLGA_OK) st = readout_run(c, b_g, eps, Y, s);
+    nvtxRangePop();
+    return st;
 }
 
 glga_status glga_destroy(glga_ctx *h) {
@@ -366,10 +461,10 @@ glga_status glga_get_intermediates(const glga_ctx *h, void *Q, void *K, void *V,
     if (c->N > 0) {
         if (Q) GLGA_CUDA(cudaMemcpyAsync(Q, c->Q, c->N * row, cudaMemcpyDeviceToDevice, s));
         if (K)
-            GLGA_CUDA(cudaMemcpy2DAsync(K, row, c->KV, 2 * row, row, c->N,
+            GLGA_CUDA(cudaMemcpy2DAsync(K, row, c->kv_own, 2 * row, row, c->N,
                                         cudaMemcpyDeviceToDevice, s));
         if (V)
-            GLGA_CUDA(cudaMemcpy2DAsync(V, row, static_cast<const uint8_t *>(c->KV) + row, 2 * row,
+            GLGA_CUDA(cudaMemcpy2DAsync(V, row, static_cast<const uint8_t *>(c->kv_own) + row, 2 * row,
                                         row, c->N, cudaMemcpyDeviceToDevice, s));
         if (t) GLGA_CUDA(cudaMemcpyAsync(t, c->t, c->N * sizeof(float), cudaMemcpyDeviceToDevice, s));
         if (L) GLGA_CUDA(cudaMemcpyAsync(L, c->L, c->N * row, cudaMemcpyDeviceToDevice, s));

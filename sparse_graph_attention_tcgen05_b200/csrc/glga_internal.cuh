@@ -84,9 +84,17 @@ struct Ctx {
     void *Xp = nullptr;           // [planes][N][dp] (prepared A operand when !x_direct)
     TensorMap2D tmB[2], tmA[2];
 
+    // row sharding: the context's N target rows are rows row0 .. row0+N-1 of n_src nodes;
+    // its CSR columns and the K/V buffer index all n_src nodes (n_src = N, row0 = 0 when
+    // the context holds the whole graph)
+    int64_t n_src = 0, row0 = 0;
+    bool sharded = false;
+    bool kv_external = false;     // KV is the caller's buffer (not freed here)
+
     // intermediates
     void *Q = nullptr;            // io [N, D]
-    void *KV = nullptr;           // io [N, 2D]  (k_j | v_j)
+    void *KV = nullptr;           // io [n_src, 2D]  (k_j | v_j)
+    void *kv_own = nullptr;       // KV + row0 rows: the rows this context projects
     float *t = nullptr;           // [N] gate logits
     float *Spart = nullptr;       // [P][H][r][r+1] partial sums of the row ranges
     float *Sz = nullptr;          // S [n_seg][H][r][r] followed by z [n_seg][H][r]
@@ -142,6 +150,10 @@ glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK
 // global_stats.cu
 glga_status stats_setup(Ctx *c);
 glga_status stats_run(Ctx *c, cudaStream_t s);
+// row-sharded forward: this context's partial S | z (flat [H][r][r+1]) ...
+glga_status stats_run_partial(Ctx *c, float *own, cudaStream_t s);
+// ... and the final reduction of all ranks' partials ([P][H][r][r+1], in rank order)
+glga_status stats_finish(Ctx *c, const float *partials, int P, cudaStream_t s);
 
 // local.cu
 glga_status local_setup(Ctx *c);

@@ -301,7 +301,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restrict__ part, int P,
                                     const int32_t *__restrict__ seg_part_ptr, int64_t n_seg,
                                     int H, int R, float *__restrict__ Sz, T *__restrict__ Bro,
-                                    int hg, int BNr, int Kp, int64_t seg_stride, int64_t plane) {
+                                    int hg, int BNr, int Kp, int64_t seg_stride, int64_t plane,
+                                    float *__restrict__ flat) {
     __shared__ float ws[8][32];
     const int per_head = R * (R + 1);
     const int total = H * per_head;
@@ -325,10 +326,16 @@ __global__ void __launch_bounds__(256) stats_reduce_kernel(const float *__restri
     }
     ws[w][lane] = acc;
     __syncthreads();
+    float s = 0.f;
     if (w == 0 && o < total) {
-        float s = 0.f;
 #pragma unroll
         for (int k = 0; k < 8; ++k) s += ws[k][lane];
+    }
+    if (w == 0 && o < total && flat) {
+        // the sum of these ranges in the partial layout [H][R][R+1] (one row shard's
+        // contribution, exchanged between ranks before the final reduction)
+        flat[o] = s;
+    } else if (w == 0 && o < total) {
         const int h = o / per_head, rem = o % per_head, a = rem / (R + 1), c = rem % (R + 1);
         const int64_t hrr = static_cast<int64_t>(H) * R * R;
         if (c < R)
@@ -506,11 +513,13 @@ glga_status stats_setup(Ctx *c) {
         if (e != cudaSuccess) return cuda_fail(e, "statistics ranges");
     }
     if (st == GLGA_OK && c->N > 0)
-        st = encode_kv_maps(c->KV, c->N, c->D, c->elem, &c->tmK.map, &c->tmV.map, rows);
+        st = encode_kv_maps(c->kv_own, c->N, c->D, c->elem, &c->tmK.map, &c->tmV.map, rows);
     return st;
 }
 
-glga_status stats_run(Ctx *c, cudaStream_t s) {
+namespace {
+// Partial sums of S | z over the context's row ranges (Spart).
+glga_status stats_partials(Ctx *c, cudaStream_t s) {
     if (c->N > 0) {
         StatsParams p;
         p.N = c->N;
@@ -533,6 +542,40 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
         if (st != GLGA_OK) return st;
         c->launches += 1;
     }
+    return GLGA_OK;
+}
+
+// Final reduction of P partials (flat layout [P][H][r][r+1]) into S, z and the readout
+// operand; the order of the sums is fixed (the same on every rank).
+template <typename T>
+glga_status reduce_into_stats(Ctx *c, const float *part, int P, float *flat, cudaStream_t s) {
+    const int total = c->H * c->r * (c->r + 1);
+    const int64_t seg_stride = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
+    stats_reduce_kernel<T><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
+        part, P, nullptr, 1, c->H, c->r, c->Sz, static_cast<T *>(c->Bro), c->ro_hg, c->ro_bn, c->ro_kp,
+        seg_stride, seg_stride, flat);
+    GLGA_CUDA(cudaGetLastError());
+    c->launches += 1;
+    return GLGA_OK;
+}
+}  // namespace
+
+glga_status stats_run_partial(Ctx *c, float *own, cudaStream_t s) {
+    glga_status st = stats_partials(c, s);
+    if (st != GLGA_OK) return st;
+    const int P = c->N > 0 ? c->stats_parts : 0;
+    return c->io == GLGA_F32 ? reduce_into_stats<float>(c, c->Spart, P, own, s)
+                             : reduce_into_stats<__nv_bfloat16>(c, c->Spart, P, own, s);
+}
+
+glga_status stats_finish(Ctx *c, const float *partials, int P, cudaStream_t s) {
+    return c->io == GLGA_F32 ? reduce_into_stats<float>(c, partials, P, nullptr, s)
+                             : reduce_into_stats<__nv_bfloat16>(c, partials, P, nullptr, s);
+}
+
+glga_status stats_run(Ctx *c, cudaStream_t s) {
+    glga_status st0 = stats_partials(c, s);
+    if (st0 != GLGA_OK) return st0;
     const int total = c->H * c->r * (c->r + 1);
     const int P = c->N > 0 ? c->stats_parts : 0;
     const int64_t seg_stride = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
@@ -567,11 +610,11 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
     if (c->io == GLGA_F32)
         stats_reduce_kernel<float><<<rgrid, 256, 0, s>>>(
             c->Spart, P, spp, c->n_seg, c->H, c->r, c->Sz, static_cast<float *>(c->Bro), c->ro_hg,
-            c->ro_bn, c->ro_kp, seg_stride, plane);
+            c->ro_bn, c->ro_kp, seg_stride, plane, nullptr);
     else
         stats_reduce_kernel<__nv_bfloat16><<<rgrid, 256, 0, s>>>(
             c->Spart, P, spp, c->n_seg, c->H, c->r, c->Sz, static_cast<__nv_bfloat16 *>(c->Bro),
-            c->ro_hg, c->ro_bn, c->ro_kp, seg_stride, plane);
+            c->ro_hg, c->ro_bn, c->ro_kp, seg_stride, plane, nullptr);
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -692,7 +735,8 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
     }
     const int total = static_cast<int>(per_part);
     stats_reduce_kernel<float><<<static_cast<unsigned>(ceil_div(total, 32)), 256, 0, s>>>(
-        scratch, parts, nullptr, 1, H, r, static_cast<float *>(Sz), static_cast<float *>(nullptr), 1, 1, 1, 0, 0);
+        scratch, parts, nullptr, 1, H, r, static_cast<float *>(Sz), static_cast<float *>(nullptr), 1, 1, 1, 0, 0,
+        nullptr);
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;
 }

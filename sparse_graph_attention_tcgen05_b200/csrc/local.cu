@@ -107,7 +107,8 @@ struct LocalParams {
     void *L;             // io [N, D] local-branch output
     int32_t D, r, H, nvec, lpe, epw, lph;
     float score_scale;   // log2(e) / sqrt(r)
-    int32_t N;           // rows (debug checks)
+    int32_t N;           // source nodes: bound of column indices (debug checks)
+    int32_t n_rows;      // target rows of this context: bound of scheduled rows (debug checks)
     unsigned *flag;      // device error flag (debug checks)
 };
 
@@ -131,11 +132,11 @@ __device__ __forceinline__ int32_t checked_col(const LocalParams &p, int32_t j) 
     return j;
 }
 
-// A row taken from a schedule list; debug builds report one outside [0, N).
+// A row taken from a schedule list; debug builds report one outside [0, n_rows).
 template <bool DBG>
 __device__ __forceinline__ bool row_ok(const LocalParams &p, int64_t row) {
     if constexpr (DBG) {
-        if (row < 0 || row >= p.N) {
+        if (row < 0 || row >= p.n_rows) {
             atomicOr(p.flag, kDevErrBounds);
             return false;
         }
@@ -587,7 +588,8 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.epw = 32 / lpe;
     p.lph = c->r / VE;
     p.score_scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->r)));
-    p.N = static_cast<int32_t>(c->N);
+    p.N = static_cast<int32_t>(c->n_src);   // column indices range over all source nodes
+    p.n_rows = static_cast<int32_t>(c->N);
     p.flag = c->dev_flag;
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
     // U edges per slot step; U <= LPE so the slot's lanes can hold its column indices

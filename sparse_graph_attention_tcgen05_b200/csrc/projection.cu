@@ -460,7 +460,7 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     p.stage_bytes = planes * (p.a_bytes + p.b_bytes);
     p.stage_area = static_cast<uint32_t>(p.stages) * p.stage_bytes;
     p.Q = c->Q;
-    p.KV = c->KV;
+    p.KV = c->kv_own;
     p.t = c->t;
     p.flag = c->dev_flag;
     const uint32_t staging = p.tma_epi ? static_cast<uint32_t>(p.sbufs) * (c->BN / 64) * kBM * kRowBytes : 0u;
@@ -565,7 +565,7 @@ glga_status projection_setup(Ctx *c) {
         c->tmB[pl].valid = true;
     }
     if (c->gemm_tma_epi && c->N > 0) {
-        r = encode_tmap_2d(&c->tmKVs.map, dt, c->KV, 2 * static_cast<uint64_t>(c->D), c->N,
+        r = encode_tmap_2d(&c->tmKVs.map, dt, c->kv_own, 2 * static_cast<uint64_t>(c->D), c->N,
                            2 * static_cast<uint64_t>(c->D) * c->elem, 64, kBM);
         if (r != GLGA_OK) return r;
         c->tmKVs.valid = true;

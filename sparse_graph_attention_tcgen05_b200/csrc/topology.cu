@@ -115,7 +115,7 @@ glga_status exclusive_scan_i32(const int32_t *in, int32_t *out, int64_t n, int32
 // CSR validation
 // ---------------------------------------------------------------------------------------
 __global__ void validate_csr_kernel(const int32_t *__restrict__ rp, const int32_t *__restrict__ col,
-                                    int64_t N, int64_t E, unsigned *flag) {
+                                    int64_t N, int64_t E, int64_t n_cols, unsigned *flag) {
     unsigned bad = 0;
     const int64_t lim = (N + 1 > E) ? N + 1 : E;
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < lim;
@@ -123,7 +123,7 @@ __global__ void validate_csr_kernel(const int32_t *__restrict__ rp, const int32_
         if (i == 0 && rp[0] != 0) bad |= kGraphBadRowPtr0;
         if (i == N && static_cast<int64_t>(rp[N]) != E) bad |= kGraphBadRowPtrEnd;
         if (i < N && rp[i + 1] < rp[i]) bad |= kGraphNotMonotone;
-        if (i < E && (col[i] < 0 || static_cast<int64_t>(col[i]) >= N)) bad |= kGraphColOutOfRange;
+        if (i < E && (col[i] < 0 || static_cast<int64_t>(col[i]) >= n_cols)) bad |= kGraphColOutOfRange;
     }
     if (bad) atomicOr(flag, bad);
 }
@@ -132,7 +132,8 @@ glga_status validate_csr(Ctx *c, cudaStream_t s) {
     GLGA_CUDA(cudaMemsetAsync(c->dev_flag, 0, sizeof(unsigned), s));
     const int64_t lim = (c->N + 1 > c->E) ? c->N + 1 : c->E;
     const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(lim, 256), 4096));
-    validate_csr_kernel<<<blocks, 256, 0, s>>>(c->row_ptr, c->col_idx, c->N, c->E, c->dev_flag);
+    // rows are the context's targets; columns index all n_src nodes whose k/v it reads
+    validate_csr_kernel<<<blocks, 256, 0, s>>>(c->row_ptr, c->col_idx, c->N, c->E, c->n_src, c->dev_flag);
     GLGA_CUDA(cudaGetLastError());
     unsigned h = 0;
     GLGA_CUDA(cudaMemcpyAsync(&h, c->dev_flag, sizeof(unsigned), cudaMemcpyDeviceToHost, s));
@@ -141,7 +142,7 @@ glga_status validate_csr(Ctx *c, cudaStream_t s) {
         set_error("invalid CSR:%s%s%s%s", (h & kGraphBadRowPtr0) ? " row_ptr[0]!=0" : "",
                   (h & kGraphBadRowPtrEnd) ? " row_ptr[N]!=E" : "",
                   (h & kGraphNotMonotone) ? " row_ptr decreasing" : "",
-                  (h & kGraphColOutOfRange) ? " col_idx outside [0,N)" : "");
+                  (h & kGraphColOutOfRange) ? " col_idx outside [0, node count)" : "");
         return GLGA_ERR_BAD_GRAPH;
     }
     return GLGA_OK;

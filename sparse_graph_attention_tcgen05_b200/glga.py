@@ -62,6 +62,10 @@ def lib() -> ctypes.CDLL:
         "glga_forward": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _vp], _i32),
         "glga_create_segmented": ([ctypes.POINTER(_vp), _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
                                    _vp, _i64, ctypes.POINTER(Options), _vp], _i32),
+        "glga_create_sharded": ([ctypes.POINTER(_vp), _i64, _i64, _i64, _i32, _i32, _i32, _i32, _vp, _vp,
+                                 _i64, _vp, ctypes.POINTER(Options), _vp], _i32),
+        "glga_forward_begin": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
+        "glga_forward_end": ([_vp, _vp, _i32, ctypes.c_float, ctypes.c_float, _vp, _vp], _i32),
         "glga_destroy": ([_vp], _i32),
         "glga_csr_from_coo": ([_i64, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_bucket_counts": ([_vp, ctypes.POINTER(_i64)], _i32),

@@ -95,3 +95,10 @@ def test_segmented_create_rejects_malformed_segments():
     assert L.glga_create_segmented(ctypes.byref(h), N, 8, 1, 8, 0, 16, 16, 0, None, 1, None, None) == 1
     assert L.glga_create_segmented(ctypes.byref(h), N, 8, 1, 8, 0, 16, 16, 0, arr.ctypes.data, 0,
                                    None, None) == 1
+
+
+def test_every_declared_entry_point_has_a_binding_signature():
+    """ctypes would pass 64-bit integers as C ints without argtypes."""
+    L = glga.lib()
+    for name in glga.declared_symbols():
+        assert getattr(L, name).argtypes is not None, name
