@@ -25,16 +25,16 @@ namespace {
 
 constexpr int kFB = 128;             // features per block: MMA M (phi(K)) and N (V)
 constexpr int kRowBytes = 128;
-constexpr int kMaxStages = 3;
-constexpr int kWorkers = 256;        // warps 0-7: phi / split passes; warps 0-3: epilogue
-constexpr int kProdWarp = 8;         // TMA producer
-constexpr int kMmaWarp = 9;          // TMEM owner and MMA issuer
-constexpr int kThreads = 320;
+constexpr int kMaxStages = 6;
+constexpr int kWorkers = 512;        // warps 0-15: phi / split passes; warps 0-3: epilogue
+constexpr int kProdWarp = 16;        // TMA producer
+constexpr int kMmaWarp = 17;         // TMEM owner and MMA issuer
+constexpr int kThreads = 576;
 
 template <typename T>
 struct StatsGeom {
     static constexpr int kRows = sizeof(T) == 2 ? 64 : 32;           // node rows per stage
-    static constexpr int kStages = sizeof(T) == 2 ? 3 : 2;
+    static constexpr int kStages = sizeof(T) == 2 ? 6 : 2;
     static constexpr int kUK = sizeof(T) == 2 ? 16 : 8;              // rows per MMA
     static constexpr int kBoxes = kFB * static_cast<int>(sizeof(T)) / kRowBytes;
     static constexpr uint32_t kBoxBytes = kRows * kRowBytes;
@@ -447,10 +447,11 @@ glga_status launch_stats(const CUtensorMap &mk, const CUtensorMap &mv, const Sta
     return GLGA_OK;
 }
 
-// Row ranges: a multiple of the stage height, about two CTAs per SM in total.
+// Row ranges: a multiple of the stage height, about one CTA (range x feature block) per
+// SM in total.
 void plan_parts(int64_t N, int nblk, int num_sms, int rows, int64_t max_parts, int *parts,
                 int64_t *rows_per_part) {
-    const int64_t want = std::max<int64_t>(1, ceil_div(2 * num_sms, nblk));
+    const int64_t want = std::max<int64_t>(1, ceil_div(num_sms, nblk));
     const int64_t tiles = std::max<int64_t>(1, ceil_div(std::max<int64_t>(N, 1), rows));
     int64_t P = std::max<int64_t>(1, std::min(std::min(want, tiles), max_parts));
     const int64_t per = ceil_div(tiles, P) * rows;
