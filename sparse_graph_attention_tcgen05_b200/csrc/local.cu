@@ -173,6 +173,15 @@ struct Lane {
     int lane, slot, li;
 };
 
+// The 16-byte vector index (within a q / k / v / L row) of vector v of lane li.  J = false:
+// vectors v*32 + li (lanes interleave; a head spans r/VE lanes).  J = true ("joint"): the
+// lane's VPL vectors are consecutive, li*VPL + v, and all lie in one head (VPL*VE <= r),
+// so the lane computes one score per edge for all of them.
+template <bool J, int VPL>
+__device__ __forceinline__ int vid_of(int v, int li) {
+    return J ? li * VPL + v : v * 32 + li;
+}
+
 // First column index of a slot's range as held by the lane that later broadcasts it:
 // lane li (< U) of the slot holds col_idx[e0 + li].
 template <int U, bool DBG>
@@ -183,7 +192,7 @@ __device__ __forceinline__ int32_t first_cols(const LocalParams &p, int64_t e0, 
 // One slot walks the CSR entries [e0, e1) U at a time (the trip count is the warp's
 // maximum over slots); `cols` holds the first step's column indices (first_cols).
 // On return each lane holds its slot's partial state for its feature vectors.
-template <typename T, int VPL, int U, bool DBG>
+template <typename T, int VPL, int U, bool DBG, bool J>
 __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
                                            int64_t e0, int64_t e1, int32_t cols, const Lane &ln,
                                            State<T, VPL> &st) {
@@ -207,7 +216,7 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q
         for (int u = 0; u < U; ++u) {
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const int vid = v * 32 + ln.li;
+                const int vid = vid_of<J, VPL>(v, ln.li);
                 if (j[u] >= 0 && vid < p.nvec) {
                     // (a masked-off slot never forms an address: j < 0 takes the else branch)
                     const uint4 *rowp = KV + static_cast<int64_t>(j[u]) * row_vecs;
@@ -218,6 +227,50 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q
                     vr[u][v] = make_uint4(0, 0, 0, 0);
                 }
             }
+        }
+        if constexpr (J) {
+            // one score per edge for the lane's VPL vectors (one head): one exp, one max
+            // and one rescale per edge instead of VPL
+            float s1[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                float dot = 0.f;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    float kf[VE];
+                    Io<T>::unpack(kr[u][v], kf);
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) dot = fmaf(q[v][e], kf[e], dot);
+                }
+                for (int o = 1; o < p.lph; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                s1[u] = (j[u] >= 0) ? dot : -INFINITY;
+            }
+            float mx = s1[0];
+#pragma unroll
+            for (int u = 1; u < U; ++u) mx = fmaxf(mx, s1[u]);
+            const float mn = fmaxf(st.m[0], mx);
+            if (mn != -INFINITY) {
+                const float corr = exp2_ftz(st.m[0] - mn);
+                st.l[0] *= corr;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const float pr = exp2_ftz(s1[u] - mn);
+                    st.l[0] += pr;
+#pragma unroll
+                    for (int v = 0; v < VPL; ++v) {
+                        float vf[VE];
+                        Io<T>::unpack(vr[u][v], vf);
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) st.acc[v][e] = fmaf(pr, vf[e], st.acc[v][e]);
+                    }
+                }
+                st.m[0] = mn;
+            }
+            continue;
         }
         float s[U][VPL];
 #pragma unroll
@@ -256,6 +309,14 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q
             st.m[v] = mn;
         }
     }
+    if constexpr (J) {
+        // every vector of the lane carries the head's (m, l): the merges work per vector
+#pragma unroll
+        for (int v = 1; v < VPL; ++v) {
+            st.m[v] = st.m[0];
+            st.l[v] = st.l[0];
+        }
+    }
 }
 
 // Merges the edge slots of the warp (lanes li, li + LPE, ...): afterwards every lane
@@ -276,13 +337,13 @@ __device__ __forceinline__ void merge_slots(const LocalParams &p, State<T, VPL> 
     }
 }
 
-template <typename T, int VPL>
+template <typename T, int VPL, bool J>
 __device__ __forceinline__ void load_q_raw(const LocalParams &p, int64_t row, const Lane &ln, bool ok,
                                            uint4 (&qr)[VPL]) {
     const uint4 *Q = static_cast<const uint4 *>(p.Q) + row * p.nvec;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
-        const int vid = v * 32 + ln.li;
+        const int vid = vid_of<J, VPL>(v, ln.li);
         qr[v] = (ok && vid < p.nvec) ? __ldg(Q + vid) : make_uint4(0, 0, 0, 0);
     }
 }
@@ -298,14 +359,14 @@ __device__ __forceinline__ void scale_q(const LocalParams &p, const uint4 (&qr)[
 }
 
 // L_i = acc / l per head (0 for a row without edges); stores L[row] from `slot`'s lanes.
-template <typename T, int VPL>
+template <typename T, int VPL, bool J>
 __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, const State<T, VPL> &st,
                                            const Lane &ln, int slot) {
     constexpr int VE = Io<T>::VE;
     uint4 *Lout = static_cast<uint4 *>(p.L) + row * p.nvec;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
-        const int vid = v * 32 + ln.li;
+        const int vid = vid_of<J, VPL>(v, ln.li);
         const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
         float y[VE];
 #pragma unroll
@@ -324,7 +385,7 @@ struct BlockScratch {
 
 // 8 warps split [e0, e1) (each warp's share split again across its slots); warp 0
 // returns the merge of all warps in warp order.
-template <typename T, int VPL, int U, bool DBG>
+template <typename T, int VPL, int U, bool DBG, bool J>
 __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
                                             int64_t e0, int64_t e1, const Lane &ln, int warp,
                                             BlockScratch<T, VPL> &sh, State<T, VPL> &st) {
@@ -333,7 +394,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&
     const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
     const int64_t per_s = ceil_div(b - a, p.epw);
     const int64_t sa = std::min(b, a + ln.slot * per_s), sb = std::min(b, sa + per_s);
-    slot_edges<T, VPL, U, DBG>(p, q, sa, sb, first_cols<U, DBG>(p, sa, sb, ln), ln, st);
+    slot_edges<T, VPL, U, DBG, J>(p, q, sa, sb, first_cols<U, DBG>(p, sa, sb, ln), ln, st);
     merge_slots<T, VPL>(p, st);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
@@ -356,7 +417,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&
     }
 }
 
-template <typename T, int VPL, int U, bool DBG>
+template <typename T, int VPL, int U, bool DBG, bool J>
 __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(const LocalParams p) {
     constexpr int VE = Io<T>::VE;
     __shared__ BlockScratch<T, VPL> sh;
@@ -380,15 +441,15 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         const int64_t e1 = std::min<int64_t>(re, e0 + p.chunk_edges);
         const int64_t nch = ceil_div(re - rb, p.chunk_edges);
         const int64_t first = c - (e0 - rb) / p.chunk_edges;
-        load_q_raw<T, VPL>(p, row, ln, true, qr);
+        load_q_raw<T, VPL, J>(p, row, ln, true, qr);
         scale_q<T, VPL>(p, qr, q);
-        block_edges<T, VPL, U, DBG>(p, q, e0, e1, ln, warp, sh, st);
+        block_edges<T, VPL, U, DBG, J>(p, q, e0, e1, ln, warp, sh, st);
         const int64_t stride = 2 * p.H + p.D;
         if (warp == 0) {
             float *dst = p.part + c * stride;
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const int vid = v * 32 + ln.li;
+                const int vid = vid_of<J, VPL>(v, ln.li);
                 if (vid < p.nvec && ln.slot == 0) {
 #pragma unroll
                     for (int e = 0; e < VE; ++e) dst[2 * p.H + vid * VE + e] = st.acc[v][e];
@@ -415,7 +476,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                     const float *src = p.part + (first + k) * stride;
 #pragma unroll
                     for (int v = 0; v < VPL; ++v) {
-                        const int vid = v * 32 + ln.li;
+                        const int vid = vid_of<J, VPL>(v, ln.li);
                         const int h = vid < p.nvec ? vid * VE / p.r : 0;
                         float a2[VE];
 #pragma unroll
@@ -424,7 +485,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                         st.merge(v, __ldcg(src + h), __ldcg(src + p.H + h), a2);
                     }
                 }
-                finish_row<T, VPL>(p, row, st, ln, 0);
+                finish_row<T, VPL, J>(p, row, st, ln, 0);
             }
         }
         return;
@@ -434,10 +495,10 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         // ---------------- bucket-1 row: one block ----------------
         const int64_t row = p.cta_rows[bid];
         if (!row_ok<DBG>(p, row)) return;
-        load_q_raw<T, VPL>(p, row, ln, true, qr);
+        load_q_raw<T, VPL, J>(p, row, ln, true, qr);
         scale_q<T, VPL>(p, qr, q);
-        block_edges<T, VPL, U, DBG>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
-        if (warp == 0) finish_row<T, VPL>(p, row, st, ln, 0);
+        block_edges<T, VPL, U, DBG, J>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
+        if (warp == 0) finish_row<T, VPL, J>(p, row, st, ln, 0);
         return;
     }
     bid -= p.n_cta;
@@ -463,7 +524,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     int32_t beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
     int32_t end = __shfl_sync(0xffffffffu, myend, k & 31);
     if (k >= n) beg = end = 0;
-    load_q_raw<T, VPL>(p, row, ln, k < n && (!DBG || row >= 0), qr);
+    load_q_raw<T, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qr);
     int32_t cols = first_cols<U, DBG>(p, beg, end, ln);
     for (int step = 0; step < steps; ++step) {
         const bool valid = k < n;
@@ -477,16 +538,16 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
         end = __shfl_sync(0xffffffffu, myend, k & 31);
         if (k >= n) beg = end = 0;
-        load_q_raw<T, VPL>(p, row, ln, k < n && (!DBG || row >= 0), qr);
+        load_q_raw<T, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qr);
         cols = first_cols<U, DBG>(p, beg, end, ln);
-        slot_edges<T, VPL, U, DBG>(p, q, beg_c, end_c, cols_c, ln, st);
+        slot_edges<T, VPL, U, DBG, J>(p, q, beg_c, end_c, cols_c, ln, st);
         if (valid && (!DBG || row_c >= 0)) {
             // every slot finishes its own row
             constexpr int VEc = Io<T>::VE;
             uint4 *Lout = static_cast<uint4 *>(p.L) + static_cast<int64_t>(row_c) * p.nvec;
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const int vid = v * 32 + ln.li;
+                const int vid = vid_of<J, VPL>(v, ln.li);
                 const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
                 float y[VEc];
 #pragma unroll
@@ -497,14 +558,14 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     }
 }
 
-template <typename T, int VPL, int U>
+template <typename T, int VPL, int U, bool J = false>
 glga_status launch_local(Ctx *c, const LocalParams &p, cudaStream_t s) {
     const int64_t blocks = p.n_chunks + p.n_cta + p.task_blocks;
     if (blocks == 0) return GLGA_OK;
     if (c->opts.debug_checks)
-        local_kernel<T, VPL, U, true><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
+        local_kernel<T, VPL, U, true, J><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
     else
-        local_kernel<T, VPL, U, false><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
+        local_kernel<T, VPL, U, false, J><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -592,6 +653,16 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.n_rows = static_cast<int32_t>(c->N);
     p.flag = c->dev_flag;
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
+    // bf16 rows of 64 vectors (D = 512) with heads of >= 16 features: the joint layout,
+    // two consecutive vectors (16 features of one head) per lane.  (Measured: faster than
+    // the interleaved layout at D = 512, slower at D = 128, where its 118 registers leave
+    // 16 warps per SM instead of 24.)
+    if (c->io == GLGA_BF16 && c->r >= 16 && p.nvec == 64) {
+        p.lpe = p.nvec / 2;
+        p.epw = 32 / p.lpe;
+        p.lph = c->r / 16;
+        return launch_local<__nv_bfloat16, 2, 2, true>(c, p, s);
+    }
     // U edges per slot step; U <= LPE so the slot's lanes can hold its column indices
     if (c->io == GLGA_F32) {
         if (vpl == 1 && lpe >= 4) return launch_local<float, 1, 4>(c, p, s);
