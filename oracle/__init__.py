@@ -219,6 +219,20 @@ def forward(N, d, H, r, X, W_Q, W_K, W_V, w_g, b_g, eps, row_ptr, col_idx, rows=
     return out
 
 
+def block_output(X, Y, Wo, gamma, beta, ln_eps):
+    """The block around the layer, in float64: Z = LayerNorm(X + Y Wo) with
+    LayerNorm(u) = (u - mean(u)) / sqrt(var(u) + ln_eps) * gamma + beta over each row's d
+    features (population variance).  Method page "Gated Local-Global Graph Attention",
+    Implementation notes, item 2: "return LayerNorm(X + Wo(g*L+(1-g)*G))"; Wo is a plain
+    [H*r, d] matrix (no bias), as the key formulas write the other projections."""
+    X = np.asarray(X, dtype=np.float64)
+    U = X + np.asarray(Y, dtype=np.float64) @ np.asarray(Wo, dtype=np.float64)
+    mean = U.mean(axis=1, keepdims=True)
+    var = ((U - mean) ** 2).mean(axis=1, keepdims=True)
+    return (U - mean) / np.sqrt(var + ln_eps) * np.asarray(gamma, dtype=np.float64) + \
+        np.asarray(beta, dtype=np.float64)
+
+
 def forward_workload(w, rows=None, csr=None, seg_ptr=None):
     """Oracle forward of a `Workload` (see the package's workloads module)."""
     if csr is None:

@@ -475,3 +475,39 @@ def test_bad_segments_are_rejected():
     for seg in ([1, w.N], [0, w.N - 1], [0, 10, 5, w.N], [0]):
         with pytest.raises(ValueError):
             oracle.forward_workload(w, csr=(rp, ci), seg_ptr=seg)
+
+
+# ---------------------------------------------------------------------------------------
+# The block around the layer: Z = LayerNorm(X + Y Wo) (method page, Implementation notes)
+# ---------------------------------------------------------------------------------------
+def test_block_output_against_torch_layer_norm():
+    rng = np.random.default_rng(8)
+    N, D, d = 37, 24, 16
+    X, Y = rng.standard_normal((N, d)), rng.standard_normal((N, D))
+    Wo = rng.standard_normal((D, d)) / np.sqrt(D)
+    g, b = rng.standard_normal(d), rng.standard_normal(d)
+    Z = oracle.block_output(X, Y, Wo, g, b, 1e-5)
+    ln = torch.nn.functional.layer_norm(torch.tensor(X + Y @ Wo), (d,), torch.tensor(g),
+                                        torch.tensor(b), eps=1e-5)
+    np.testing.assert_allclose(Z, ln.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_block_output_closed_forms():
+    rng = np.random.default_rng(9)
+    N, D, d = 11, 8, 6
+    X, Y = rng.standard_normal((N, d)), rng.standard_normal((N, D))
+    ones, zeros = np.ones(d), np.zeros(d)
+    # unit gain, zero bias: every row has mean 0 and (nearly, by eps) variance 1
+    Z = oracle.block_output(X, Y, rng.standard_normal((D, d)), ones, zeros, 0.0)
+    np.testing.assert_allclose(Z.mean(1), 0, atol=1e-12)
+    np.testing.assert_allclose((Z ** 2).mean(1), 1, rtol=1e-12)
+    # Wo = 0: the layer's output drops out, Z = LayerNorm(X)
+    Z0 = oracle.block_output(X, Y, np.zeros((D, d)), ones, zeros, 0.0)
+    Xc = X - X.mean(1, keepdims=True)
+    np.testing.assert_allclose(Z0, Xc / np.sqrt((Xc ** 2).mean(1, keepdims=True)), rtol=1e-12)
+    # gain and bias act per feature after the normalisation
+    g, b = rng.standard_normal(d), rng.standard_normal(d)
+    np.testing.assert_allclose(oracle.block_output(X, Y, np.zeros((D, d)), g, b, 0.0), Z0 * g + b, rtol=1e-12)
+    # a constant row shift is removed by the normalisation
+    np.testing.assert_allclose(oracle.block_output(X + 3.0, Y, np.zeros((D, d)), ones, zeros, 0.0), Z0,
+                               rtol=1e-10, atol=1e-12)
