@@ -201,6 +201,37 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def time_block(layer, w, X, Y, dt, dev, flush, stream, steps, peaks):
+    """The block around the layer alone, Z = LayerNorm(X + Y Wo): CUDA events per call,
+    L2 flushed between calls; FLOPs 2*N*(H*r)*d, bytes Y + X + Z + Wo."""
+    import torch
+    rng = np.random.default_rng(3)
+    Wo = torch.from_numpy((rng.standard_normal((w.D, w.d)) / np.sqrt(w.D)).astype(np.float32)).to(dt).to(dev)
+    g = torch.ones(w.d, dtype=dt, device=dev)
+    b = torch.zeros(w.d, dtype=dt, device=dev)
+    Z = torch.empty(w.N, w.d, dtype=dt, device=dev)
+    for _ in range(3):
+        layer.block_output(Y, X, Wo, g, b, 1e-5, Z)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        ev0.record(stream)
+        layer.block_output(Y, X, Wo, g, b, 1e-5, Z)
+        ev1.record(stream)
+        ev1.synchronize()
+        ms.append(ev0.elapsed_time(ev1))
+    assert layer.last_device_error() == 0
+    t = float(np.mean(ms)) * 1e-3
+    s = 4 if w.io == "f32" else 2
+    flops = 2.0 * w.N * w.D * w.d
+    nbytes = s * (w.N * w.D + 2 * w.N * w.d + w.D * w.d)
+    return {"ms": t * 1e3, "tflops": flops / t / 1e12,
+            "frac_of_tensor_peak": flops / t / (peaks["bf16_tflops"] * 1e12),
+            "gbs": nbytes / t / 1e9, "frac_of_hbm": nbytes / t / 1e9 / peaks["hbm_gbs"],
+            "arith_intensity_flop_per_byte": flops / nbytes}
+
+
 def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0):
     """Forward time against N at fixed in-degree: the tiny config's shape (d=32, H=1,
     r=16, fp32, k distinct uniform in-neighbours + self-loop; the method page's cost-proxy
@@ -352,6 +383,8 @@ def main():
     ap.add_argument("--segment-len", type=int, default=0,
                     help="segments of this many nodes, each with its own global statistics "
                          "(a batch of graphs; 0 = one segment over all nodes)")
+    ap.add_argument("--block", action="store_true",
+                    help="also time the block around the layer, Z = LayerNorm(X + Y Wo)")
     ap.add_argument("--sharded", action="store_true",
                     help="row-sharded forward across the ranks (strong scaling) instead of replicas")
     ap.add_argument("--sweep", action="store_true",
@@ -538,6 +571,8 @@ def main():
             "stages_ms": stages, "create": create, "gpu_launches": launches,
             "e2e": e2e, "clocks": clocks, "parity_max_rel_err": parity,
             "wall_s_timed_region": wall}
+    if args.block:
+        line["block"] = time_block(layer, w, X, Y, dt, dev, flush, stream, args.steps, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, (row_ptr.cpu().numpy(), col_idx.cpu().numpy()))
     if rank == 0:

@@ -183,6 +183,22 @@ GLGA_API glga_status glga_forward_begin(glga_ctx *ctx, const void *X, const void
 GLGA_API glga_status glga_forward_end(glga_ctx *ctx, const float *partials, int32_t P, float b_g,
                         float eps, void *Y, void *stream);
 
+/* glga_block_output -- the block around the layer, Z = LayerNorm(X + Y Wo): the output
+ * projection, the residual and a LayerNorm over the d features.  Method page "Gated
+ * Local-Global Graph Attention", "Implementation notes", item 2 ("return
+ * LayerNorm(X + Wo(g*L+(1-g)*G))"); Wo has no bias, the LayerNorm uses the population
+ * variance and a per-feature gain and bias.
+ *   Y      (device) io [n, H*r]: a glga_forward output of this context (n = its rows)
+ *   X      (device) io [n, d]: the layer's input rows (the residual)
+ *   Wo     (device) io [H*r, d]      gamma, beta (device) io [d]
+ *   ln_eps (host) >= 0, added to the variance        Z (device) io [n, d], written
+ * Requires d to be a multiple of 32 and at most 512 (GLGA_ERR_UNSUPPORTED otherwise).
+ * Y, X and Z 16-byte aligned.  Stream-ordered, no host synchronisation; uses only
+ * workspaces allocated at create.                                                     */
+GLGA_API glga_status glga_block_output(glga_ctx *ctx, const void *Y, const void *X, const void *Wo,
+                        const void *gamma, const void *beta, float ln_eps, void *Z,
+                        void *stream);
+
 /* Copies the bucket lists (device -> device, on `stream`) into caller buffers sized by
  * glga_bucket_counts: warp_rows [counts[0]], cta_rows [counts[1]], split_rows [counts[2]],
  * chunk_row [counts[3]], chunk_begin [counts[3]] (the CSR offset of the chunk's first

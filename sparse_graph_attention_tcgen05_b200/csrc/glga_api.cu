@@ -77,7 +77,7 @@ static void release_ctx(Ctx *c) {
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
                     c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
                     c->part_ptr, c->seg_part_ptr, c->tile_seg, c->fix_row, c->fix_seg,
-                    c->dev_flag};
+                    c->Wo_t, c->Yp, c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)
@@ -278,6 +278,7 @@ glga_status create_impl(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t
     TRY(readout_setup(c));
     TRY(stats_setup(c));
     TRY(local_setup(c));
+    TRY(block_setup(c));
     if (st == GLGA_OK) {
         e = cudaMemsetAsync(c->dev_flag, 0, 64, s);
         if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -405,6 +406,30 @@ glga_status glga_forward_end(glga_ctx *h, const float *partials, int32_t P, floa
     glga_status st = stats_finish(c, partials, P, s);
     if (st == GLGA_OK) st = local_run(c, s);
     if (st == GLGA_OK) st = readout_run(c, b_g, eps, Y, s);
+    nvtxRangePop();
+    return st;
+}
+
+glga_status glga_block_output(glga_ctx *h, const void *Y, const void *X, const void *Wo,
+                              const void *gamma, const void *beta, float ln_eps, void *Z,
+                              void *stream) {
+    if (!h) {
+        set_error("glga_block_output: ctx is NULL");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    if (!Wo || !gamma || !beta || (c->N > 0 && (!Y || !X || !Z))) {
+        set_error("glga_block_output: null pointer argument");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    const uintptr_t a = reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(X) |
+                        reinterpret_cast<uintptr_t>(Z);
+    if ((a & 15u) || !(ln_eps >= 0.f) || !std::isfinite(ln_eps)) {
+        set_error("glga_block_output: Y, X, Z must be 16-byte aligned and ln_eps finite, >= 0");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    nvtxRangePushA("glga_block_output");
+    const glga_status st = block_run(c, Y, X, Wo, gamma, beta, ln_eps, Z, static_cast<cudaStream_t>(stream));
     nvtxRangePop();
     return st;
 }

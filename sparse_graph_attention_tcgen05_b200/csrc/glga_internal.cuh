@@ -119,6 +119,12 @@ struct Ctx {
     int32_t *fix_seg = nullptr;       //   ... and that segment
     int64_t n_fix = 0;
 
+    // block around the layer (Z = LayerNorm(X + Y Wo))
+    int32_t blk_kp = 0;           // K = H*r padded to the K tile
+    bool blk_y_direct = false;    // Y read in place as the A operand
+    void *Wo_t = nullptr;         // [planes][d][blk_kp] K-major Wo^T
+    void *Yp = nullptr;           // [planes][N][blk_kp] padded / split Y when not direct
+
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;
     int64_t alloc_calls = 0;      // device allocations made by create (debug_fail_alloc)
@@ -158,6 +164,12 @@ glga_status stats_finish(Ctx *c, const float *partials, int P, cudaStream_t s);
 // local.cu
 glga_status local_setup(Ctx *c);
 glga_status local_run(Ctx *c, cudaStream_t s);
+
+// block.cu
+bool block_supported(const Ctx *c);
+glga_status block_setup(Ctx *c);
+glga_status block_run(Ctx *c, const void *Y, const void *X, const void *Wo, const void *gamma,
+                      const void *beta, float ln_eps, void *Z, cudaStream_t s);
 
 // readout.cu
 glga_status readout_setup(Ctx *c);

@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
                                  _i64, _vp, ctypes.POINTER(Options), _vp], _i32),
         "glga_forward_begin": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_forward_end": ([_vp, _vp, _i32, ctypes.c_float, ctypes.c_float, _vp, _vp], _i32),
+        "glga_block_output": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp], _i32),
         "glga_destroy": ([_vp], _i32),
         "glga_csr_from_coo": ([_i64, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_bucket_counts": ([_vp, ctypes.POINTER(_i64)], _i32),
@@ -226,6 +227,16 @@ class Layer:
         if self.n_seg is None:           # one global segment: S [H, r, r], z [H, r]
             out["S"], out["z"] = out["S"][0], out["z"][0]
         return out
+
+    def block_output(self, Y, X, Wo, gamma, beta, ln_eps: float = 1e-5, Z=None, stream=None):
+        """Z = LayerNorm(X + Y Wo) (glga_block_output)."""
+        for t in (Y, X, Wo, gamma, beta):
+            assert t.dtype == self.dtype and t.is_cuda and t.is_contiguous()
+        if Z is None:
+            Z = torch.empty(X.shape[0], self.d, dtype=self.dtype, device=X.device)
+        _check(lib().glga_block_output(self._h, _ptr(Y), _ptr(X), _ptr(Wo), _ptr(gamma), _ptr(beta),
+                                       float(ln_eps), _ptr(Z), _stream(stream)), "glga_block_output")
+        return Z
 
     def set_timing(self, enable: bool):
         _check(lib().glga_set_timing(self._h, 1 if enable else 0), "glga_set_timing")
