@@ -232,6 +232,30 @@ def time_block(layer, w, X, Y, dt, dev, flush, stream, steps, peaks):
             "arith_intensity_flop_per_byte": flops / nbytes}
 
 
+def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
+    """glga_backward alone (after one forward with the same inputs): CUDA events per call,
+    L2 flushed between calls."""
+    import torch
+    rng = np.random.default_rng(4)
+    dY = torch.from_numpy(rng.standard_normal((w.N, w.D)).astype(np.float32)).to(dt).to(dev)
+    layer.forward(X, WQ, WK, WV, wg, b_g=w.b_g, eps=w.eps)
+    for _ in range(2):
+        layer.backward(X, WQ, WK, WV, wg, w.b_g, w.eps, dY)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        ev0.record(stream)
+        layer.backward(X, WQ, WK, WV, wg, w.b_g, w.eps, dY)
+        ev1.record(stream)
+        ev1.synchronize()
+        ms.append(ev0.elapsed_time(ev1))
+    assert layer.last_device_error() == 0
+    t = float(np.mean(ms))
+    return {"ms": t, "edge_heads_per_s": w.E * w.H / (t * 1e-3), "steps": steps,
+            "kernels": "CUDA-core (SIMT) kernels, fp32 arithmetic"}
+
+
 def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0):
     """Forward time against N at fixed in-degree: the tiny config's shape (d=32, H=1,
     r=16, fp32, k distinct uniform in-neighbours + self-loop; the method page's cost-proxy
@@ -383,6 +407,8 @@ def main():
     ap.add_argument("--segment-len", type=int, default=0,
                     help="segments of this many nodes, each with its own global statistics "
                          "(a batch of graphs; 0 = one segment over all nodes)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward pass (glga_backward) of the same forward")
     ap.add_argument("--block", action="store_true",
                     help="also time the block around the layer, Z = LayerNorm(X + Y Wo)")
     ap.add_argument("--sharded", action="store_true",
@@ -438,7 +464,9 @@ def main():
     seg = None
     if args.segment_len > 0:
         seg = np.unique(np.concatenate([np.arange(0, w.N, args.segment_len), [w.N]])).astype(np.int64)
-    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx, segments=seg)
+    opts = glga.default_options()
+    opts.backward = 1 if args.backward else 0
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx, opts, segments=seg)
     torch.cuda.synchronize()
     t2 = time.perf_counter()
     create = {"csr_from_coo_ms": (t1 - t0) * 1e3, "glga_create_ms": (t2 - t1) * 1e3,
@@ -573,6 +601,9 @@ def main():
             "wall_s_timed_region": wall}
     if args.block:
         line["block"] = time_block(layer, w, X, Y, dt, dev, flush, stream, args.steps, peaks)
+    if args.backward:
+        line["backward"] = time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream,
+                                         max(10, args.steps // 10))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, (row_ptr.cpu().numpy(), col_idx.cpu().numpy()))
     if rank == 0:

@@ -72,12 +72,16 @@ typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
  * masked) and reported as GLGA_ERR_DEVICE by glga_last_device_error.  Slower; for
  * debugging only.
  * debug_fail_alloc = n > 0 makes the n-th device allocation of glga_create fail with
- * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.                    */
+ * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.
+ * backward != 0 allocates the workspaces of glga_backward at create (a transposed CSR
+ * and fp32 buffers of about N*(6*H*r + 4*H + 1) floats); whole-graph, one-segment
+ * contexts only.                                                                     */
 typedef struct {
     int32_t warp_max_degree;
     int32_t chunk_edges;
     int32_t debug_checks;
     int32_t debug_fail_alloc;
+    int32_t backward;
 } glga_options;
 
 /* Fills *opts with the defaults used when glga_create gets opts == NULL. */
@@ -182,6 +186,22 @@ GLGA_API glga_status glga_forward_begin(glga_ctx *ctx, const void *X, const void
                         void *stream);
 GLGA_API glga_status glga_forward_end(glga_ctx *ctx, const float *partials, int32_t P, float b_g,
                         float eps, void *Y, void *stream);
+
+/* glga_backward -- gradients of sum(Y * dY) for the Y of the last glga_forward on this
+ * context, which must have been called with the same X, W_Q, W_K, W_V, w_g, b_g, eps
+ * (the forward's Q, K, V, gate logits, S, z and L are reused).  Method page "Gated
+ * Local-Global Graph Attention", "Key formulas", differentiated (the softmax maximum is
+ * held constant, tinymesh "Target softmax").
+ *   dY (device) io [N, H*r]
+ *   dX (device) float [N, d]; dW_Q, dW_K, dW_V (device) float [d, H*r]; dw_g (device)
+ *   float [d]; db_g (device) float [1] -- all written.
+ * Needs glga_options.backward at create.  Every sum runs in a fixed order (the source
+ * side walks a transposed CSR; no atomics), so repeated calls give identical bits.
+ * Stream-ordered, no host synchronisation.                                            */
+GLGA_API glga_status glga_backward(glga_ctx *ctx, const void *X, const void *W_Q, const void *W_K,
+                        const void *W_V, const void *w_g, float b_g, float eps, const void *dY,
+                        float *dX, float *dW_Q, float *dW_K, float *dW_V, float *dw_g, float *db_g,
+                        void *stream);
 
 /* glga_block_output -- the block around the layer, Z = LayerNorm(X + Y Wo): the output
  * projection, the residual and a LayerNorm over the d features.  Method page "Gated

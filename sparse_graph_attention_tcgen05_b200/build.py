@@ -18,7 +18,7 @@ LIB = os.path.join(PKG, "libglga.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["glga_api.cu", "topology.cu", "projection.cu", "global_stats.cu", "local.cu", "readout.cu",
-           "block.cu"]
+           "block.cu", "backward.cu"]
 HEADERS = [os.path.join(CSRC, "glga_internal.cuh"), os.path.join(INCLUDE, "glga.h")]
 
 NVCC_FLAGS = [

@@ -77,7 +77,9 @@ static void release_ctx(Ctx *c) {
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
                     c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
                     c->part_ptr, c->seg_part_ptr, c->tile_seg, c->fix_row, c->fix_seg,
-                    c->Wo_t, c->Yp, c->dev_flag};
+                    c->Wo_t, c->Yp, c->t_row_ptr, c->t_col, c->bw_dL, c->bw_dnum, c->bw_dden,
+                    c->bw_dg, c->bw_lse, c->bw_Dd, c->bw_dZ, c->bw_dsz_part, c->bw_dSz,
+                    c->bw_dw_part, c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)
@@ -126,6 +128,7 @@ glga_status glga_default_options(glga_options *opts) {
     opts->chunk_edges = 1024;
     opts->debug_checks = 0;
     opts->debug_fail_alloc = 0;
+    opts->backward = 0;
     return GLGA_OK;
 }
 
@@ -279,6 +282,7 @@ glga_status create_impl(glga_ctx **out, int64_t N, int32_t d, int32_t H, int32_t
     TRY(stats_setup(c));
     TRY(local_setup(c));
     TRY(block_setup(c));
+    TRY(backward_setup(c, s));
     if (st == GLGA_OK) {
         e = cudaMemsetAsync(c->dev_flag, 0, 64, s);
         if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -406,6 +410,31 @@ glga_status glga_forward_end(glga_ctx *h, const float *partials, int32_t P, floa
     glga_status st = stats_finish(c, partials, P, s);
     if (st == GLGA_OK) st = local_run(c, s);
     if (st == GLGA_OK) st = readout_run(c, b_g, eps, Y, s);
+    nvtxRangePop();
+    return st;
+}
+
+glga_status glga_backward(glga_ctx *h, const void *X, const void *W_Q, const void *W_K,
+                          const void *W_V, const void *w_g, float b_g, float eps, const void *dY,
+                          float *dX, float *dW_Q, float *dW_K, float *dW_V, float *dw_g, float *db_g,
+                          void *stream) {
+    if (!h || !h->c.opts.backward) {
+        set_error("glga_backward: needs a context created with glga_options.backward = 1");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    Ctx *c = &h->c;
+    if (!W_Q || !W_K || !W_V || !w_g || !dW_Q || !dW_K || !dW_V || !dw_g || !db_g ||
+        (c->N > 0 && (!X || !dY || !dX))) {
+        set_error("glga_backward: null pointer argument");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    if (!(eps > 0.f) || !std::isfinite(eps) || !std::isfinite(b_g)) {
+        set_error("glga_backward: eps must be finite and > 0, b_g finite");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    nvtxRangePushA("glga_backward");
+    const glga_status st = backward_run(c, X, W_Q, W_K, W_V, w_g, b_g, eps, dY, dX, dW_Q, dW_K, dW_V,
+                                        dw_g, db_g, static_cast<cudaStream_t>(stream));
     nvtxRangePop();
     return st;
 }

@@ -125,6 +125,16 @@ struct Ctx {
     void *Wo_t = nullptr;         // [planes][d][blk_kp] K-major Wo^T
     void *Yp = nullptr;           // [planes][N][blk_kp] padded / split Y when not direct
 
+    // backward pass workspaces (opts.backward)
+    int32_t *t_row_ptr = nullptr, *t_col = nullptr;   // transposed CSR: rows by source
+    float *bw_dL = nullptr, *bw_dnum = nullptr;       // [N, D]
+    float *bw_dden = nullptr, *bw_dg = nullptr, *bw_lse = nullptr, *bw_Dd = nullptr;   // [N, H]
+    float *bw_dZ = nullptr;                           // [N, 3D + 1]: dQ | dK | dV | dt
+    float *bw_dsz_part = nullptr, *bw_dSz = nullptr;  // dS | dz partials and sum
+    float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
+    int64_t bw_dz_ld = 0;
+    int32_t bw_parts = 0, bw_wparts = 0;
+
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;
     int64_t alloc_calls = 0;      // device allocations made by create (debug_fail_alloc)
@@ -170,6 +180,12 @@ bool block_supported(const Ctx *c);
 glga_status block_setup(Ctx *c);
 glga_status block_run(Ctx *c, const void *Y, const void *X, const void *Wo, const void *gamma,
                       const void *beta, float ln_eps, void *Z, cudaStream_t s);
+
+// backward.cu
+glga_status backward_setup(Ctx *c, cudaStream_t s);
+glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV,
+                         const void *wg, float b_g, float eps, const void *dY, float *dX, float *dWQ,
+                         float *dWK, float *dWV, float *dwg, float *db_g, cudaStream_t s);
 
 // readout.cu
 glga_status readout_setup(Ctx *c);

@@ -33,7 +33,8 @@ class GLGAError(RuntimeError):
 
 class Options(ctypes.Structure):
     _fields_ = [("warp_max_degree", ctypes.c_int32), ("chunk_edges", ctypes.c_int32),
-                ("debug_checks", ctypes.c_int32), ("debug_fail_alloc", ctypes.c_int32)]
+                ("debug_checks", ctypes.c_int32), ("debug_fail_alloc", ctypes.c_int32),
+                ("backward", ctypes.c_int32)]
 
 
 _lib = None
@@ -66,6 +67,8 @@ def lib() -> ctypes.CDLL:
                                  _i64, _vp, ctypes.POINTER(Options), _vp], _i32),
         "glga_forward_begin": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),
         "glga_forward_end": ([_vp, _vp, _i32, ctypes.c_float, ctypes.c_float, _vp, _vp], _i32),
+        "glga_backward": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _vp, _vp, _vp,
+                           _vp, _vp, _vp, _vp], _i32),
         "glga_block_output": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp], _i32),
         "glga_destroy": ([_vp], _i32),
         "glga_csr_from_coo": ([_i64, _i64, _vp, _vp, _vp, _vp, _vp], _i32),
@@ -226,6 +229,25 @@ class Layer:
                                             _stream(stream)), "glga_get_intermediates")
         if self.n_seg is None:           # one global segment: S [H, r, r], z [H, r]
             out["S"], out["z"] = out["S"][0], out["z"][0]
+        return out
+
+    def backward(self, X, W_Q, W_K, W_V, w_g, b_g: float, eps: float, dY, stream=None) -> dict:
+        """fp32 gradients of sum(Y * dY) (glga_backward); call after forward() with the
+        same inputs."""
+        for t in (X, W_Q, W_K, W_V, w_g, dY):
+            assert t.dtype == self.dtype and t.is_cuda and t.is_contiguous()
+        dev = X.device
+        f32 = torch.float32
+        out = {"dX": torch.empty(self.N, self.d, dtype=f32, device=dev),
+               "dW_Q": torch.empty(self.d, self.D, dtype=f32, device=dev),
+               "dW_K": torch.empty(self.d, self.D, dtype=f32, device=dev),
+               "dW_V": torch.empty(self.d, self.D, dtype=f32, device=dev),
+               "dw_g": torch.empty(self.d, dtype=f32, device=dev),
+               "db_g": torch.empty(1, dtype=f32, device=dev)}
+        _check(lib().glga_backward(self._h, _ptr(X), _ptr(W_Q), _ptr(W_K), _ptr(W_V), _ptr(w_g),
+                                   float(b_g), float(eps), _ptr(dY),
+                                   *(_ptr(out[k]) for k in ("dX", "dW_Q", "dW_K", "dW_V", "dw_g", "db_g")),
+                                   _stream(stream)), "glga_backward")
         return out
 
     def block_output(self, Y, X, Wo, gamma, beta, ln_eps: float = 1e-5, Z=None, stream=None):

@@ -1,0 +1,87 @@
+"""The backward pass on the GPU (glga_backward) against the float64 reference gradients
+of oracle/backward.py (pinned by finite differences of the C oracle).  Tolerances per
+gradient tensor, relative to its largest entry: fp32 io 2e-4 (fp32 arithmetic over sums of
+up to N terms); bf16 io 3e-2 (the forward's Q, K, V and L are stored in bf16, 2^-9
+relative, and every gradient term is a product of two or three of them)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.backward import backward as ref_backward
+from sparse_graph_attention_tcgen05_b200 import glga
+from sparse_graph_attention_tcgen05_b200.workloads import make_custom, make_workload, round_to_bf16
+from tests.gpu_helpers import to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOLB = {"f32": 2e-4, "bf16": 3e-2}
+NAMES = ("dX", "dW_Q", "dW_K", "dW_V", "dw_g", "db_g")
+
+
+def _run(w, dY, options=None):
+    row_ptr, col_idx = glga.csr_from_coo(w.N, to_dev(w.src), to_dev(w.dst))
+    o = options or glga.default_options()
+    o.backward = 1
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx, o)
+    dt = glga.torch_dtype(w.io)
+    args = [to_dev(a, dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+    layer.forward(*args, b_g=w.b_g, eps=w.eps)
+    g1 = layer.backward(*args, w.b_g, w.eps, to_dev(dY, dt))
+    g2 = layer.backward(*args, w.b_g, w.eps, to_dev(dY, dt))
+    torch.cuda.synchronize()
+    assert layer.last_device_error() == 0
+    for k in NAMES:                                   # fixed summation order
+        assert torch.equal(g1[k], g2[k]), k
+    layer.close()
+    return {k: v.cpu().numpy().astype(np.float64) for k, v in g1.items()}
+
+
+def _check(w, seed=0):
+    rng = np.random.default_rng(seed)
+    dY = rng.standard_normal((w.N, w.D)).astype(np.float32)
+    if w.io == "bf16":
+        dY = round_to_bf16(dY)
+    got = _run(w, dY)
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    ref = ref_backward(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY)
+    for k in NAMES:
+        r = np.asarray(ref[k], dtype=np.float64).reshape(got[k].shape)
+        scale = max(np.abs(r).max(), 1e-30)
+        err = np.abs(got[k] - r).max() / scale
+        assert np.all(np.isfinite(got[k])) and err <= TOLB[w.io], (k, err)
+
+
+def test_tiny_fp32():
+    _check(make_workload("tiny"))
+
+
+def test_citation_fp32():
+    _check(make_workload("citation"))
+
+
+def test_arxiv_shape_bf16():
+    _check(make_workload("arxiv", scale=0.02))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_skewed_degrees_and_isolated_rows(io):
+    rng = np.random.default_rng(11)
+    N = 300
+    deg = np.minimum(rng.zipf(1.6, N), 250)
+    deg[::7] = 0                                      # isolated targets
+    dst = np.repeat(np.arange(N), deg)
+    src = rng.integers(0, N, dst.shape[0])
+    w = make_custom(N, 24, 2, 32, src.astype(np.int32), dst.astype(np.int32), io=io, seed=3, b_g=0.1)
+    _check(w, seed=2)
+
+
+def test_backward_needs_the_option():
+    w = make_workload("tiny")
+    row_ptr, col_idx = glga.csr_from_coo(w.N, to_dev(w.src), to_dev(w.dst))
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+    args = [to_dev(a, torch.float32) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+    with pytest.raises(glga.GLGAError) as ei:
+        layer.backward(*args, w.b_g, w.eps, torch.zeros(w.N, w.D, device="cuda"))
+    assert ei.value.status == 1
+    layer.close()
