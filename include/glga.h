@@ -75,7 +75,7 @@ typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
  * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.
  * backward != 0 allocates the workspaces of glga_backward at create (a transposed CSR
  * and fp32 buffers of about N*(6*H*r + 4*H + 1) floats); whole-graph, one-segment
- * contexts only.                                                                     */
+ * contexts with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).                   */
 typedef struct {
     int32_t warp_max_degree;
     int32_t chunk_edges;

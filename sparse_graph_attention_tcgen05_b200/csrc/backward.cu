@@ -20,6 +20,7 @@
 // (one thread per row and head, tiled GEMMs for the projections); gradients are fp32.
 #include <algorithm>
 #include <cmath>
+#include <vector>
 
 #include "glga_internal.cuh"
 
@@ -36,76 +37,146 @@ __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p) { re
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 __device__ __forceinline__ float dphi(float x) { return x > 0.f ? 1.f : __expf(x); }
 
-constexpr int kMaxR = 128;
+// (ld_row / head_reduce: see the warp-cooperative row kernels below)
+template <typename T, int EPL>
+__device__ __forceinline__ void ld_row(const T *row, int lane, bool act, float (&x)[EPL]);
+__device__ __forceinline__ float head_reduce(float x, int lph);
 
-// One thread per (row i, head h): the gate, readout and blend backward.  Writes
-// dL [N, D], dnum [N, D], dden [N, H], the gate partial dg [N, H] and the global part of
-// dQ into dZ [:, 0:D].
-template <typename T>
-__global__ void bwd_readout_kernel(const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t,
-                                   const float *__restrict__ Sz, const T *__restrict__ dY, int64_t N, int H,
-                                   int R, float b_g, float eps, float *__restrict__ dL,
-                                   float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dg,
-                                   float *__restrict__ dZ, int64_t dz_ld) {
-    const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    if (idx >= N * H) return;
-    const int64_t i = idx / H;
-    const int h = static_cast<int>(idx % H);
+// One warp per row i (lanes over features, EPL each): the gate, readout and blend
+// backward.  Writes dL [N, D], dnum [N, D], dden [N, H], the global part of dQ into
+// dZ [:, 0:D] and dt into dZ [:, 3D] (dg summed over the whole row in lane order).
+template <typename T, int EPL>
+__global__ void __launch_bounds__(256) bwd_readout_kernel(
+    const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t, const float *__restrict__ Sz,
+    const float *__restrict__ ST, const T *__restrict__ dY, int64_t N, int H, int R, float b_g, float eps,
+    float *__restrict__ dL,
+    float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ, int64_t dz_ld) {
+    const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (i >= N) return;                                   // warp-uniform
     const int D = H * R;
+    const bool act = lane * EPL < D;
+    const int lph = R / EPL, h = act ? lane * EPL / R : 0;
     const float *S = Sz + static_cast<int64_t>(h) * R * R;
     const float *z = Sz + static_cast<int64_t>(H) * R * R + h * R;
-    const T *q = Q + i * D + h * R;
-    float phq[kMaxR];
-    float den = eps;
-    for (int a = 0; a < R; ++a) {
-        phq[a] = phi(ldf<T>(q + a));
-        den = fmaf(phq[a], z[a], den);
+    const T *qh = Q + i * D + h * R;                      // the lane's head
+    float q[EPL], dy[EPL], lv[EPL];
+    ld_row<T, EPL>(Q + i * D, lane, act, q);
+    ld_row<T, EPL>(dY + i * D, lane, act, dy);
+    ld_row<T, EPL>(L + i * D, lane, act, lv);
+    const int f0 = lane * EPL - h * R;                    // in-head index of the lane's first feature
+    float den = 0.f;
+    if (act) {
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) den = fmaf(phi(q[x]), z[f0 + x], den);
     }
+    den = head_reduce(den, lph) + eps;
+    // num_c = sum_a phi(q_a) S[a][c] for the lane's features c (phi(q_a) read back from
+    // the row, the same for the head's lanes)
+    float G[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) G[x] = 0.f;
+    if (act)
+        for (int a = 0; a < R; ++a) {
+            const float pa = phi(ldf<T>(qh + a));
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) G[x] = fmaf(pa, S[a * R + f0 + x], G[x]);
+        }
     const float g = 1.f / (1.f + __expf(-(t[i] + b_g)));
-    float dgp = 0.f, dG_dot_G = 0.f;
-    const int64_t o = i * D + h * R;
-    for (int c = 0; c < R; ++c) {
-        float num = 0.f;
-        for (int a = 0; a < R; ++a) num = fmaf(phq[a], S[a * R + c], num);
-        const float Gc = num / den;
-        const float dy = ldf<T>(dY + o + c);
-        dgp = fmaf(dy, ldf<T>(L + o + c) - Gc, dgp);
-        dL[o + c] = g * dy;
-        const float dGc = (1.f - g) * dy;
-        dnum[o + c] = dGc / den;
-        dG_dot_G = fmaf(dGc, Gc, dG_dot_G);
+    float dgp = 0.f, dGG = 0.f;
+    const int64_t o = i * D + lane * EPL;
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) {
+        G[x] /= den;
+        dgp = fmaf(dy[x], lv[x] - G[x], dgp);
+        const float dG = (1.f - g) * dy[x];
+        dGG = fmaf(dG, G[x], dGG);
+        if (act) {
+            dL[o + x] = g * dy[x];
+            dnum[o + x] = dG / den;
+        }
     }
-    const float dd = -dG_dot_G / den;
-    dden[idx] = dd;
-    dg[idx] = dgp;
-    for (int a = 0; a < R; ++a) {
-        float acc = z[a] * dd;
-        for (int c = 0; c < R; ++c) acc = fmaf(S[a * R + c], dnum[o + c], acc);
-        dZ[i * dz_ld + h * R + a] = acc * dphi(ldf<T>(q + a));
+    const float dd = -head_reduce(dGG, lph) / den;
+    if (act && (lane % lph) == 0) dden[i * H + h] = dd;
+    __syncwarp();                                         // dnum of the row is written
+    const float *dn = dnum + i * D + h * R;
+    const float *STh = ST + static_cast<int64_t>(h) * R * R;   // STh[c][a] = S[a][c]
+    if (act) {
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) {
+            float acc = z[f0 + x] * dd;
+            for (int c = 0; c < R; ++c) acc = fmaf(STh[c * R + f0 + x], dn[c], acc);
+            dZ[i * dz_ld + lane * EPL + x] = acc * dphi(q[x]);
+        }
     }
+    for (int w = 16; w > 0; w >>= 1) dgp += __shfl_xor_sync(0xffffffffu, dgp, w);
+    if (lane == 0) dZ[i * dz_ld + 3 * D] = g * (1.f - g) * dgp;
 }
 
-// Partial sums over the row range of part p of dS | dz in the layout [H][R][R+1]
-// (column R is dz): part[p][h][a][c] = sum_i phi(q_i[h R + a]) * (dnum_i[h R + c] or
-// dden_i[h]).
-template <typename T>
-__global__ void bwd_dsz_partial_kernel(const T *__restrict__ Q, const float *__restrict__ dnum,
-                                       const float *__restrict__ dden, int64_t N, int H, int R,
-                                       int64_t rows_per_part, float *__restrict__ part) {
-    const int total = H * R * (R + 1);
-    const int o = blockIdx.y * blockDim.x + threadIdx.x;
-    if (o >= total) return;
-    const int per_head = R * (R + 1);
-    const int h = o / per_head, rem = o % per_head, a = rem / (R + 1), c = rem % (R + 1);
+// Partial sums of dS | dz over the row range of block column p, per head h =
+// blockIdx.y, in the layout [H][R][R+1] (column R is dz):
+//   part[p][h][a][c] = sum_i phi(q_i[h R + a]) * (c < R ? dnum_i[h R + c] : dden_i[h]).
+// 32-row tiles of phi(Q_h) and [dnum_h | dden_h] are staged in shared memory; each thread
+// owns outputs o = tid, tid + 256, ... of the head's R (R + 1).
+template <typename T, int R>
+__global__ void __launch_bounds__(256) bwd_dsz_partial_kernel(const T *__restrict__ Q, const float *__restrict__ dnum,
+                                                              const float *__restrict__ dden, int64_t N, int H,
+                                                              int64_t rows_per_part, float *__restrict__ part) {
+    extern __shared__ float tile[];                      // [32][R] phi(q) then [32][R + 1] dnum | dden
+    constexpr int kRowsT = 32;
+    const int h = blockIdx.y;
     const int D = H * R;
+    const int per_head = R * (R + 1);
+    float *pq = tile, *pw = tile + kRowsT * R;
     const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_part;
     const int64_t r1 = std::min<int64_t>(N, r0 + rows_per_part);
-    float acc = 0.f;
-    for (int64_t i = r0; i < r1; ++i) {
-        const float w = c < R ? dnum[i * D + h * R + c] : dden[i * H + h];
-        acc = fmaf(phi(ldf<T>(Q + i * D + h * R + a)), w, acc);
+    constexpr int kMaxOut = (R * (R + 1) + 255) / 256;
+    float acc[kMaxOut];
+    const int n_out = (per_head - static_cast<int>(threadIdx.x) + 255) / 256;
+#pragma unroll
+    for (int u = 0; u < kMaxOut; ++u) acc[u] = 0.f;
+    for (int64_t i0 = r0; i0 < r1; i0 += kRowsT) {
+        for (int l = threadIdx.x; l < kRowsT * (R + 1); l += 256) {
+            const int rr = l / (R + 1), c = l % (R + 1);
+            const int64_t i = i0 + rr;
+            const bool in = i < r1;
+            if (c < R) {
+                pq[rr * R + c] = in ? phi(ldf<T>(Q + i * D + h * R + c)) : 0.f;
+                pw[rr * (R + 1) + c] = in ? dnum[i * D + h * R + c] : 0.f;
+            } else {
+                pw[rr * (R + 1) + R] = in ? dden[i * H + h] : 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kMaxOut; ++u) {
+            if (u < n_out) {
+                const int oo = threadIdx.x + u * 256;
+                const int a = oo / (R + 1), c = oo % (R + 1);
+                float sacc = acc[u];
+                for (int rr = 0; rr < kRowsT; ++rr) sacc = fmaf(pq[rr * R + a], pw[rr * (R + 1) + c], sacc);
+                acc[u] = sacc;
+            }
+        }
+        __syncthreads();
     }
-    part[static_cast<int64_t>(blockIdx.x) * total + o] = acc;
+    const int total = H * per_head;
+    float *out = part + static_cast<int64_t>(blockIdx.x) * total + h * per_head;
+#pragma unroll
+    for (int u = 0; u < kMaxOut; ++u)
+        if (u < n_out) out[threadIdx.x + u * 256] = acc[u];
+}
+
+// dst[h][c][a] = src[h][a][c] (a, c < R) for per-head R x R blocks with row stride ld.
+__global__ void bwd_transpose_heads_kernel(const float *__restrict__ src, int ld, int H, int R,
+                                           float *__restrict__ dst) {
+    const int64_t total = static_cast<int64_t>(H) * R * R;
+    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
+         o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int h = static_cast<int>(o / (static_cast<int64_t>(R) * R));
+        const int c = static_cast<int>((o / R) % R), a = static_cast<int>(o % R);
+        dst[o] = src[static_cast<int64_t>(h) * R * ld + static_cast<int64_t>(a) * ld + c];
+    }
 }
 
 // out[o] = sum over p = 0 .. P-1, in order, of part[p][o].
@@ -118,114 +189,289 @@ __global__ void bwd_sum_parts_kernel(const float *__restrict__ part, int P, int6
     }
 }
 
-// One thread per (target i, head h) over the forward CSR: the softmax's log-sum-exp,
-// D_i = dL_i . L_i, and the local part of dq_i added into dZ [:, 0:D].
-template <typename T>
-__global__ void bwd_local_q_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
-                                   const T *__restrict__ Q, const T *__restrict__ KV, const T *__restrict__ L,
-                                   const float *__restrict__ dL, int64_t N, int H, int R, float inv_sqrt_r,
-                                   float *__restrict__ lse, float *__restrict__ Dd, float *__restrict__ dZ,
-                                   int64_t dz_ld) {
-    const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    if (idx >= N * H) return;
-    const int64_t i = idx / H;
-    const int h = static_cast<int>(idx % H);
+// Warp-cooperative row kernels: one warp per row, lane l holds the EPL consecutive
+// features l*EPL .. l*EPL+EPL-1 of every row it reads (contiguous across the warp, so a
+// row is one coalesced read), and a head's r features lie in LPH = r/EPL adjacent lanes,
+// whose dot products meet in a butterfly of shuffles.
+
+template <typename T, int EPL>
+__device__ __forceinline__ void ld_row(const T *row, int lane, bool act, float (&x)[EPL]) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) x[e] = act ? ldf<T>(row + lane * EPL + e) : 0.f;
+}
+
+__device__ __forceinline__ float head_reduce(float x, int lph) {
+    for (int o = 1; o < lph; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+constexpr int kEU = 4;           // edges whose rows are loaded before any is used
+constexpr int kHeavyWarps = 32;  // warps per heavy row (one 1024-thread block)
+
+// Online (max, sum) of exp(s) over the edges [a, b) of target row q (this warp's lanes).
+template <typename T, int EPL>
+__device__ __forceinline__ void q_lse_range(const int32_t *col_idx, const T *KV, int D, int lane, bool act,
+                                            int lph, float inv_sqrt_r, const float (&q)[EPL], int32_t a,
+                                            int32_t b, float &m, float &l) {
+    for (int32_t e = a; e < b; e += kEU) {
+        float k[kEU][EPL];
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+            const bool live = e + u < b;
+            const int64_t jj = live ? col_idx[e + u] : 0;
+            ld_row<T, EPL>(KV + jj * 2 * D, lane, act && live, k[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+            float s = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) s = fmaf(q[x], k[u][x], s);
+            s = head_reduce(s, lph) * inv_sqrt_r;
+            if (e + u < b) {
+                const float mn = fmaxf(m, s);
+                l = l * __expf(m - mn) + __expf(s - mn);
+                m = mn;
+            }
+        }
+    }
+}
+
+// dq += sum over edges [a, b) of ds_ij k_j (ds already scaled by 1/sqrt(r)).
+template <typename T, int EPL>
+__device__ __forceinline__ void q_grad_range(const int32_t *col_idx, const T *KV, int D, int lane, bool act,
+                                             int lph, float inv_sqrt_r, const float (&q)[EPL],
+                                             const float (&dl)[EPL], float ls, float dd, int32_t a, int32_t b,
+                                             float (&dq)[EPL]) {
+    for (int32_t e = a; e < b; e += kEU) {
+        float k[kEU][EPL], v[kEU][EPL];
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+            const bool live = e + u < b;
+            const T *row = KV + (live ? static_cast<int64_t>(col_idx[e + u]) : 0) * 2 * D;
+            ld_row<T, EPL>(row, lane, act && live, k[u]);
+            ld_row<T, EPL>(row + D, lane, act && live, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+            float s = 0.f, dp = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) {
+                s = fmaf(q[x], k[u][x], s);
+                dp = fmaf(dl[x], v[u][x], dp);
+            }
+            s = head_reduce(s, lph);
+            dp = head_reduce(dp, lph);
+            const float ds = e + u < b ? __expf(s * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) dq[x] = fmaf(ds, k[u][x], dq[x]);
+        }
+    }
+}
+
+// Target rows of the forward CSR: per head the softmax's log-sum-exp and D_i = dL_i . L_i,
+// and the local part of dq_i added into dZ [:, 0:D].  Light rows (the `rows` list): one
+// warp each.  Heavy rows (HEAVY): one 1024-thread block each, its 32 warps taking
+// contiguous shares of the edges; their partial (max, sum) and dq are combined in warp
+// order through shared memory.
+template <typename T, int EPL, bool HEAVY>
+__global__ void __launch_bounds__(HEAVY ? 1024 : 256) bwd_local_q_kernel(
+    const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
+    const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
+    const T *__restrict__ L, const float *__restrict__ dL, int H, int R, float inv_sqrt_r,
+    float *__restrict__ lse, float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
+    __shared__ float sm_m[HEAVY ? kHeavyWarps : 1][32], sm_l[HEAVY ? kHeavyWarps : 1][32];
+    __shared__ float sm_dq[HEAVY ? 32 * 32 : 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t slot = HEAVY ? blockIdx.x : (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (slot >= n_rows) return;                           // uniform per warp (per block when HEAVY)
+    const int64_t i = rows[slot];
     const int D = H * R;
-    const T *q = Q + i * D + h * R;
-    const int32_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    const bool act = lane * EPL < D;
+    const int lph = R / EPL, h = act ? lane * EPL / R : 0;
+    float q[EPL], dl[EPL], lv[EPL];
+    ld_row<T, EPL>(Q + i * D, lane, act, q);
+    ld_row<float, EPL>(dL + i * D, lane, act, dl);
+    ld_row<T, EPL>(L + i * D, lane, act, lv);
+    const int32_t r0 = row_ptr[i], r1 = row_ptr[i + 1];
+    int32_t a = r0, b = r1;
+    if (HEAVY) {
+        const int32_t per = (r1 - r0 + kHeavyWarps - 1) / kHeavyWarps;
+        a = min(r1, r0 + warp * per);
+        b = min(r1, a + per);
+    }
     float m = -INFINITY, l = 0.f;
-    for (int32_t e = e0; e < e1; ++e) {
-        const T *k = KV + static_cast<int64_t>(col_idx[e]) * 2 * D + h * R;
-        float s = 0.f;
-        for (int a = 0; a < R; ++a) s = fmaf(ldf<T>(q + a), ldf<T>(k + a), s);
-        s *= inv_sqrt_r;
-        const float mn = fmaxf(m, s);
-        l = l * __expf(m - mn) + __expf(s - mn);
-        m = mn;
+    q_lse_range<T, EPL>(col_idx, KV, D, lane, act, lph, inv_sqrt_r, q, a, b, m, l);
+    if (HEAVY) {
+        sm_m[warp][lane] = m;
+        sm_l[warp][lane] = l;
+        __syncthreads();
+        m = -INFINITY;
+        l = 0.f;
+        for (int w = 0; w < kHeavyWarps; ++w) {          // warp order
+            const float m2 = sm_m[w][lane], l2 = sm_l[w][lane];
+            const float mn = fmaxf(m, m2);
+            if (mn != -INFINITY) {
+                l = l * __expf(m - mn) + l2 * __expf(m2 - mn);
+                m = mn;
+            }
+        }
     }
-    const float ls = e1 > e0 ? m + __logf(l) : 0.f;
+    const float ls = r1 > r0 ? m + __logf(l) : 0.f;
     float dd = 0.f;
-    const int64_t o = i * D + h * R;
-    for (int c = 0; c < R; ++c) dd = fmaf(dL[o + c], ldf<T>(L + o + c), dd);
-    lse[idx] = ls;
-    Dd[idx] = dd;
-    float dq[kMaxR];
-    for (int a = 0; a < R; ++a) dq[a] = 0.f;
-    for (int32_t e = e0; e < e1; ++e) {
-        const T *k = KV + static_cast<int64_t>(col_idx[e]) * 2 * D + h * R;
-        const T *v = k + D;
-        float s = 0.f, dp = 0.f;
-        for (int a = 0; a < R; ++a) {
-            s = fmaf(ldf<T>(q + a), ldf<T>(k + a), s);
-            dp = fmaf(dL[o + a], ldf<T>(v + a), dp);
-        }
-        const float p = __expf(s * inv_sqrt_r - ls);
-        const float ds = p * (dp - dd) * inv_sqrt_r;
-        for (int a = 0; a < R; ++a) dq[a] = fmaf(ds, ldf<T>(k + a), dq[a]);
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dd = fmaf(dl[x], lv[x], dd);
+    dd = head_reduce(dd, lph);
+    if (act && (lane % lph) == 0 && (!HEAVY || warp == 0)) {
+        lse[i * H + h] = ls;
+        Dd[i * H + h] = dd;
     }
-    for (int a = 0; a < R; ++a) dZ[i * dz_ld + h * R + a] += dq[a];
+    float dq[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+    q_grad_range<T, EPL>(col_idx, KV, D, lane, act, lph, inv_sqrt_r, q, dl, ls, dd, a, b, dq);
+    if (HEAVY) {
+        // add the warps' dq in warp order, one 32 * EPL-feature slice at a time
+        for (int w = 0; w < kHeavyWarps; ++w) {
+            if (warp == w) {
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) {
+                    const int f = lane * EPL + x;
+                    if (f < 32 * 32) sm_dq[f] = (w == 0 ? 0.f : sm_dq[f]) + dq[x];
+                }
+            }
+            __syncthreads();
+        }
+        if (warp == 0) {
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) dq[x] = sm_dq[lane * EPL + x];
+        } else {
+            return;
+        }
+    }
+    if (act) {
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) dZ[i * dz_ld + lane * EPL + x] += dq[x];
+    }
 }
 
-// One thread per (source j, head h) over the transposed CSR (the targets i of j): the
-// local terms of dk_j and dv_j, plus the global terms through phi(k_j), written to
-// dZ [:, D:2D] and [:, 2D:3D].  dSz holds dS | dz as [H][R][R+1].
-template <typename T>
-__global__ void bwd_local_kv_kernel(const int32_t *__restrict__ t_row_ptr, const int32_t *__restrict__ t_col,
-                                    const T *__restrict__ Q, const T *__restrict__ KV,
-                                    const float *__restrict__ dL, const float *__restrict__ lse,
-                                    const float *__restrict__ Dd, const float *__restrict__ dSz, int64_t N,
-                                    int H, int R, float inv_sqrt_r, float *__restrict__ dZ, int64_t dz_ld) {
-    const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    if (idx >= N * H) return;
-    const int64_t j = idx / H;
-    const int h = static_cast<int>(idx % H);
+// dk, dv += the terms of targets [a, b) of source row j (this warp's lanes).
+template <typename T, int EPL>
+__device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, const float *dL,
+                                              const float *lse, const float *Dd, int H, int D, int lane,
+                                              bool act, int lph, int h, float inv_sqrt_r, const float (&k)[EPL],
+                                              const float (&v)[EPL], int32_t a, int32_t b, float (&dk)[EPL],
+                                              float (&dv)[EPL]) {
+    for (int32_t e = a; e < b; e += kEU) {
+        float q[kEU][EPL], dl[kEU][EPL], ls[kEU], dd[kEU];
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+            const bool live = e + u < b;
+            const int64_t i = live ? t_col[e + u] : 0;
+            ld_row<T, EPL>(Q + i * D, lane, act && live, q[u]);
+            ld_row<float, EPL>(dL + i * D, lane, act && live, dl[u]);
+            ls[u] = live ? lse[i * H + h] : 0.f;
+            dd[u] = live ? Dd[i * H + h] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+            float s = 0.f, dp = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) {
+                s = fmaf(q[u][x], k[x], s);
+                dp = fmaf(dl[u][x], v[x], dp);
+            }
+            s = head_reduce(s, lph);
+            dp = head_reduce(dp, lph);
+            const bool live = e + u < b;
+            const float p = live ? __expf(s * inv_sqrt_r - ls[u]) : 0.f;
+            const float ds = p * (dp - dd[u]) * inv_sqrt_r;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) {
+                dv[x] = fmaf(p, dl[u][x], dv[x]);
+                dk[x] = fmaf(ds, q[u][x], dk[x]);
+            }
+        }
+    }
+}
+
+// Source rows of the transposed CSR (the targets i of j): the local terms of dk_j and
+// dv_j, plus the global terms through phi(k_j), written to dZ [:, D:2D] and [:, 2D:3D].
+// dSz holds dS | dz as [H][R][R+1].  Light rows one warp each, heavy rows one block each
+// (warp shares combined in warp order), as bwd_local_q_kernel.
+template <typename T, int EPL, bool HEAVY>
+__global__ void __launch_bounds__(HEAVY ? 1024 : 256) bwd_local_kv_kernel(
+    const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
+    const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
+    const float *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
+    const float *__restrict__ dSz, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
+    float *__restrict__ dZ, int64_t dz_ld) {
+    __shared__ float sm_dk[HEAVY ? 32 * 32 : 1], sm_dv[HEAVY ? 32 * 32 : 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t slot = HEAVY ? blockIdx.x : (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (slot >= n_rows) return;
+    const int64_t j = rows[slot];
     const int D = H * R;
-    const T *k = KV + j * 2 * D + h * R;
-    const T *v = k + D;
-    float dk[kMaxR], dv[kMaxR];
-    for (int a = 0; a < R; ++a) dk[a] = dv[a] = 0.f;
-    const int32_t e0 = t_row_ptr[j], e1 = t_row_ptr[j + 1];
-    for (int32_t e = e0; e < e1; ++e) {
-        const int64_t i = t_col[e];
-        const T *q = Q + i * D + h * R;
-        const float *dl = dL + i * D + h * R;
-        float s = 0.f, dp = 0.f;
-        for (int a = 0; a < R; ++a) {
-            s = fmaf(ldf<T>(q + a), ldf<T>(k + a), s);
-            dp = fmaf(dl[a], ldf<T>(v + a), dp);
+    const bool act = lane * EPL < D;
+    const int lph = R / EPL, h = act ? lane * EPL / R : 0;
+    const T *krow = KV + j * 2 * D;
+    float k[EPL], v[EPL], dk[EPL], dv[EPL];
+    ld_row<T, EPL>(krow, lane, act, k);
+    ld_row<T, EPL>(krow + D, lane, act, v);
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dk[x] = dv[x] = 0.f;
+    const int32_t r0 = t_row_ptr[j], r1 = t_row_ptr[j + 1];
+    int32_t a = r0, b = r1;
+    if (HEAVY) {
+        const int32_t per = (r1 - r0 + kHeavyWarps - 1) / kHeavyWarps;
+        a = min(r1, r0 + warp * per);
+        b = min(r1, a + per);
+    }
+    kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, act, lph, h, inv_sqrt_r, k, v, a, b, dk, dv);
+    if (HEAVY) {
+        for (int w = 0; w < kHeavyWarps; ++w) {
+            if (warp == w) {
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) {
+                    const int f = lane * EPL + x;
+                    if (f < 32 * 32) {
+                        sm_dk[f] = (w == 0 ? 0.f : sm_dk[f]) + dk[x];
+                        sm_dv[f] = (w == 0 ? 0.f : sm_dv[f]) + dv[x];
+                    }
+                }
+            }
+            __syncthreads();
         }
-        const float p = __expf(s * inv_sqrt_r - lse[i * H + h]);
-        const float ds = p * (dp - Dd[i * H + h]) * inv_sqrt_r;
-        for (int a = 0; a < R; ++a) {
-            dv[a] = fmaf(p, dl[a], dv[a]);
-            dk[a] = fmaf(ds, ldf<T>(q + a), dk[a]);
+        if (warp != 0) return;
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) {
+            dk[x] = sm_dk[lane * EPL + x];
+            dv[x] = sm_dv[lane * EPL + x];
         }
     }
-    // global branch: S = sum phi(k) v^T, z = sum phi(k)
-    const float *dS = dSz + static_cast<int64_t>(h) * R * (R + 1);
-    for (int a = 0; a < R; ++a) {
-        const float ka = ldf<T>(k + a);
-        float dphk = dS[a * (R + 1) + R];            // dz_a
-        for (int c = 0; c < R; ++c) dphk = fmaf(dS[a * (R + 1) + c], ldf<T>(v + c), dphk);
-        dk[a] = fmaf(dphk, dphi(ka), dk[a]);
-        const float pk = phi(ka);
-        for (int c = 0; c < R; ++c) dv[c] = fmaf(dS[a * (R + 1) + c], pk, dv[c]);
+    // global branch, S = sum phi(k) v^T and z = sum phi(k): for the lane's features
+    // (head h, in-head index f = lane*EPL + x - h*R)
+    if (act) {
+        const float *dS = dSz + static_cast<int64_t>(h) * R * (R + 1);
+        const float *dSTh = dST + static_cast<int64_t>(h) * R * R;   // dSTh[c][f] = dS[f][c]
+        const T *kh = krow + h * R, *vh = krow + D + h * R;
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) {
+            const int f = lane * EPL + x - h * R;
+            float dphk = dS[f * (R + 1) + R];             // dz_f
+            float dvg = 0.f;
+            for (int c = 0; c < R; ++c) {
+                dphk = fmaf(dSTh[c * R + f], ldf<T>(vh + c), dphk);
+                dvg = fmaf(dS[c * (R + 1) + f], phi(ldf<T>(kh + c)), dvg);
+            }
+            dk[x] = fmaf(dphk, dphi(k[x]), dk[x]);
+            dv[x] += dvg;
+        }
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) {
+            dZ[j * dz_ld + D + lane * EPL + x] = dk[x];
+            dZ[j * dz_ld + 2 * D + lane * EPL + x] = dv[x];
+        }
     }
-    for (int a = 0; a < R; ++a) {
-        dZ[j * dz_ld + D + h * R + a] = dk[a];
-        dZ[j * dz_ld + 2 * D + h * R + a] = dv[a];
-    }
-}
-
-// dt_i = g (1 - g) sum_h dg[i][h], the gate logit column of dZ.
-__global__ void bwd_dt_kernel(const float *__restrict__ t, const float *__restrict__ dg, int64_t N, int H,
-                              float b_g, float *__restrict__ dZ, int64_t dz_ld, int64_t col) {
-    const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    if (i >= N) return;
-    float s = 0.f;
-    for (int h = 0; h < H; ++h) s += dg[i * H + h];
-    const float g = 1.f / (1.f + __expf(-(t[i] + b_g)));
-    dZ[i * dz_ld + col] = g * (1.f - g) * s;
 }
 
 // db_g = sum_i dt_i in a fixed order: thread k sums i = k, k + 1024, ...; then a tree.
@@ -367,6 +613,91 @@ __global__ void bwd_expand_rows_kernel(const int32_t *__restrict__ row_ptr, int6
         for (int32_t e = row_ptr[i]; e < row_ptr[i + 1]; ++e) tgt[e] = static_cast<int32_t>(i);
 }
 
+// Features per lane of the warp-cooperative kernels: the smallest power of two with
+// 32 * EPL >= D (a lane must stay inside one head, so EPL <= r is required).
+int lane_features(int D) {
+    int e = 1;
+    while (32 * e < D) e <<= 1;
+    return e;
+}
+
+// Both local backward kernels with EPL = lane_features(D): light rows one warp each,
+// heavy rows (more than kHeavyDegree entries) one block each.
+template <typename T>
+void launch_local_bwd(Ctx *c, const T *Q, const T *KV, const T *L, float isr, int64_t Dz, cudaStream_t s) {
+    const int H = c->H, R = c->r;
+    const unsigned gq = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(c->bw_nq_light * 32, 256)));
+    const unsigned gk = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(c->bw_nk_light * 32, 256)));
+#define GLGA_LB(E)                                                                                        \
+    case E:                                                                                               \
+        if (c->bw_nq_light)                                                                               \
+            bwd_local_q_kernel<T, E, false><<<gq, 256, 0, s>>>(c->bw_q_rows, c->bw_nq_light, c->row_ptr,   \
+                c->col_idx, Q, KV, L, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);            \
+        if (c->bw_nq_heavy)                                                                               \
+            bwd_local_q_kernel<T, E, true><<<static_cast<unsigned>(c->bw_nq_heavy), 1024, 0, s>>>(        \
+                c->bw_q_rows + c->bw_nq_light, c->bw_nq_heavy, c->row_ptr, c->col_idx, Q, KV, L, c->bw_dL, \
+                H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);                                            \
+        if (c->bw_nk_light)                                                                               \
+            bwd_local_kv_kernel<T, E, false><<<gk, 256, 0, s>>>(c->bw_k_rows, c->bw_nk_light,             \
+                c->t_row_ptr, c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSz, c->bw_dST, H, R, isr, \
+                c->bw_dZ, Dz);                                                                            \
+        if (c->bw_nk_heavy)                                                                               \
+            bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(c->bw_nk_heavy), 1024, 0, s>>>(       \
+                c->bw_k_rows + c->bw_nk_light, c->bw_nk_heavy, c->t_row_ptr, c->t_col, Q, KV, c->bw_dL,    \
+                c->bw_lse, c->bw_Dd, c->bw_dSz, c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                 \
+        break;
+    switch (lane_features(c->D)) {
+        GLGA_LB(1) GLGA_LB(2) GLGA_LB(4) GLGA_LB(8) GLGA_LB(16) GLGA_LB(32)
+        default: break;
+    }
+#undef GLGA_LB
+}
+
+template <typename T>
+void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
+    const unsigned grid = static_cast<unsigned>(ceil_div(c->N * 32, 256));
+#define GLGA_RB(E)                                                                                       \
+    case E:                                                                                              \
+        bwd_readout_kernel<T, E><<<grid, 256, 0, s>>>(Q, static_cast<const T *>(c->L), c->t, c->Sz, c->bw_ST, dY, \
+                                                      c->N, c->H, c->r, b_g, eps, c->bw_dL, c->bw_dnum,  \
+                                                      c->bw_dden, c->bw_dZ, Dz);                         \
+        break;
+    switch (lane_features(c->D)) {
+        GLGA_RB(1) GLGA_RB(2) GLGA_RB(4) GLGA_RB(8) GLGA_RB(16) GLGA_RB(32)
+        default: break;
+    }
+#undef GLGA_RB
+}
+
+template <typename T>
+void launch_dsz_bwd(Ctx *c, const T *Q, int64_t rpp, cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>(c->bw_parts), static_cast<unsigned>(c->H));
+    const size_t smem = (32 * c->r + 32 * (c->r + 1)) * sizeof(float);
+#define GLGA_DZ(RR)                                                                                      \
+    case RR:                                                                                             \
+        bwd_dsz_partial_kernel<T, RR><<<grid, 256, smem, s>>>(Q, c->bw_dnum, c->bw_dden, c->N, c->H, rpp, \
+                                                              c->bw_dsz_part);                           \
+        break;
+    switch (c->r) {
+        GLGA_DZ(8) GLGA_DZ(16) GLGA_DZ(32) GLGA_DZ(64) GLGA_DZ(128)
+        default: break;
+    }
+#undef GLGA_DZ
+}
+
+// Light rows first, then heavy ones (more than kHeavyDegree entries), by a CSR's offsets.
+constexpr int64_t kHeavyDegree = 128;
+void split_rows(const std::vector<int32_t> &rp, std::vector<int32_t> &rows, int64_t &n_light, int64_t &n_heavy) {
+    const int64_t n = static_cast<int64_t>(rp.size()) - 1;
+    rows.clear();
+    for (int64_t i = 0; i < n; ++i)
+        if (rp[i + 1] - rp[i] <= kHeavyDegree) rows.push_back(static_cast<int32_t>(i));
+    n_light = static_cast<int64_t>(rows.size());
+    for (int64_t i = 0; i < n; ++i)
+        if (rp[i + 1] - rp[i] > kHeavyDegree) rows.push_back(static_cast<int32_t>(i));
+    n_heavy = static_cast<int64_t>(rows.size()) - n_light;
+}
+
 int64_t ceil_parts(int64_t N, int64_t want) { return std::max<int64_t>(1, std::min<int64_t>(want, N)); }
 
 }  // namespace
@@ -375,6 +706,10 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     if (!c->opts.backward) return GLGA_OK;
     if (c->sharded || c->n_seg != 1) {
         set_error("glga_create: the backward pass is for whole-graph, one-segment contexts");
+        return GLGA_ERR_UNSUPPORTED;
+    }
+    if (lane_features(c->D) > c->r) {
+        set_error("glga_create: the backward pass needs H*r <= 32*r (at most 32 heads)");
         return GLGA_ERR_UNSUPPORTED;
     }
     const int64_t N = c->N, E = c->E, D = c->D, H = c->H, R = c->r;
@@ -392,12 +727,13 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dL), nz * D * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dnum), nz * D * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dden), nz * H * f));
-    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dg), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_lse), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Dd), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dZ), nz * c->bw_dz_ld * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dsz_part), static_cast<size_t>(c->bw_parts) * H * R * (R + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dSz), static_cast<size_t>(H) * R * (R + 1) * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_ST), static_cast<size_t>(H) * R * R * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dST), static_cast<size_t>(H) * R * R * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dw_part),
                    static_cast<size_t>(c->bw_wparts) * c->d * c->bw_dz_ld * f));
 #undef BTRY
@@ -421,7 +757,19 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
         cudaStreamSynchronize(s);
         cudaFree(tgt);
     }
-    return st;
+    if (st != GLGA_OK) return st;
+    // row lists of the two local backward kernels: light rows first, then heavy rows
+    std::vector<int32_t> rp(static_cast<size_t>(N) + 1), trp(static_cast<size_t>(N) + 1), qr, kr;
+    GLGA_CUDA(cudaMemcpy(rp.data(), c->row_ptr, rp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
+    GLGA_CUDA(cudaMemcpy(trp.data(), c->t_row_ptr, trp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
+    split_rows(rp, qr, c->bw_nq_light, c->bw_nq_heavy);
+    split_rows(trp, kr, c->bw_nk_light, c->bw_nk_heavy);
+    st = dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_rows), (qr.size() + 1) * sizeof(int32_t));
+    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_rows), (kr.size() + 1) * sizeof(int32_t));
+    if (st != GLGA_OK) return st;
+    if (!qr.empty()) GLGA_CUDA(cudaMemcpy(c->bw_q_rows, qr.data(), qr.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+    if (!kr.empty()) GLGA_CUDA(cudaMemcpy(c->bw_k_rows, kr.data(), kr.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+    return GLGA_OK;
 }
 
 glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV,
@@ -431,8 +779,6 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
     const int H = c->H, R = c->r, D = c->D, d = c->d;
     const int Dz = static_cast<int>(c->bw_dz_ld);
     const float isr = 1.f / std::sqrt(static_cast<float>(R));
-    const int64_t nh = N * H;
-    const unsigned gnh = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(nh, 128)));
     const int total = H * R * (R + 1);
     const int64_t rpp = ceil_div(std::max<int64_t>(N, 1), c->bw_parts);
     const int64_t wrpp = ceil_div(std::max<int64_t>(N, 1), c->bw_wparts);
@@ -441,26 +787,17 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
     do {                                                                                                  \
         const T *Q = static_cast<const T *>(c->Q);                                                        \
         const T *KV = static_cast<const T *>(c->KV);                                                      \
+        const unsigned tgrid = static_cast<unsigned>(ceil_div(static_cast<int64_t>(H) * R * R, 256));    \
         if (N > 0) {                                                                                      \
-            bwd_readout_kernel<T><<<gnh, 128, 0, s>>>(Q, static_cast<const T *>(c->L), c->t, c->Sz,       \
-                                                      static_cast<const T *>(dY), N, H, R, b_g, eps,      \
-                                                      c->bw_dL, c->bw_dnum, c->bw_dden, c->bw_dg,         \
-                                                      c->bw_dZ, Dz);                                      \
-            bwd_dsz_partial_kernel<T><<<dim3(c->bw_parts, ceil_div(total, 256)), 256, 0, s>>>(           \
-                Q, c->bw_dnum, c->bw_dden, N, H, R, rpp, c->bw_dsz_part);                                 \
+            bwd_transpose_heads_kernel<<<tgrid, 256, 0, s>>>(c->Sz, R, H, R, c->bw_ST);                  \
+            launch_readout_bwd<T>(c, Q, static_cast<const T *>(dY), b_g, eps, Dz, s);                  \
+            launch_dsz_bwd<T>(c, Q, rpp, s);                                                              \
         }                                                                                                 \
         bwd_sum_parts_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(                 \
             c->bw_dsz_part, N > 0 ? c->bw_parts : 0, total, c->bw_dSz);                                   \
         if (N > 0) {                                                                                      \
-            bwd_local_q_kernel<T><<<gnh, 128, 0, s>>>(c->row_ptr, c->col_idx, Q, KV,                      \
-                                                      static_cast<const T *>(c->L), c->bw_dL, N, H, R,    \
-                                                      isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);            \
-            bwd_local_kv_kernel<T><<<gnh, 128, 0, s>>>(c->t_row_ptr, c->t_col, Q, KV, c->bw_dL,           \
-                                                       c->bw_lse, c->bw_Dd, c->bw_dSz, N, H, R, isr,      \
-                                                       c->bw_dZ, Dz);                                     \
-            bwd_dt_kernel<<<static_cast<unsigned>(ceil_div(N, 256)), 256, 0, s>>>(c->t, c->bw_dg, N, H,   \
-                                                                                  b_g, c->bw_dZ, Dz,      \
-                                                                                  3 * D);                 \
+            bwd_transpose_heads_kernel<<<tgrid, 256, 0, s>>>(c->bw_dSz, R + 1, H, R, c->bw_dST);         \
+            launch_local_bwd<T>(c, Q, KV, static_cast<const T *>(c->L), isr, Dz, s);                  \
             bwd_dw_kernel<T><<<dim3(ceil_div(d, kTile), ceil_div(Dz, kTile), c->bw_wparts), 256, 0, s>>>( \
                 static_cast<const T *>(X), c->bw_dZ, N, d, Dz, wrpp, c->bw_dw_part);                     \
             bwd_dx_kernel<T><<<dim3(ceil_div(N, kTile), ceil_div(d, kTile)), 256, 0, s>>>(                \
@@ -485,7 +822,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
         GLGA_CUDA(cudaMemsetAsync(db_g, 0, sizeof(float), s));
     }
     GLGA_CUDA(cudaGetLastError());
-    c->launches += N > 0 ? 10 : 1;
+    c->launches += N > 0 ? 12 : 1;
     return GLGA_OK;
 }
 

@@ -131,7 +131,10 @@ struct Ctx {
     float *bw_dden = nullptr, *bw_dg = nullptr, *bw_lse = nullptr, *bw_Dd = nullptr;   // [N, H]
     float *bw_dZ = nullptr;                           // [N, 3D + 1]: dQ | dK | dV | dt
     float *bw_dsz_part = nullptr, *bw_dSz = nullptr;  // dS | dz partials and sum
+    float *bw_ST = nullptr, *bw_dST = nullptr;        // per-head transposes of S and dS
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
+    int32_t *bw_q_rows = nullptr, *bw_k_rows = nullptr;   // light rows, then heavy rows
+    int64_t bw_nq_light = 0, bw_nq_heavy = 0, bw_nk_light = 0, bw_nk_heavy = 0;
     int64_t bw_dz_ld = 0;
     int32_t bw_parts = 0, bw_wparts = 0;
 
