@@ -20,6 +20,7 @@
 // (one thread per row and head, tiled GEMMs for the projections); gradients are fp32.
 #include <algorithm>
 #include <cmath>
+#include <type_traits>
 #include <vector>
 
 #include "glga_internal.cuh"
@@ -37,78 +38,193 @@ __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p) { re
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 __device__ __forceinline__ float dphi(float x) { return x > 0.f ? 1.f : __expf(x); }
 
-// (ld_row / head_reduce: see the warp-cooperative row kernels below)
-template <typename T, int EPL>
-__device__ __forceinline__ void ld_row(const T *row, int lane, bool act, float (&x)[EPL]);
-__device__ __forceinline__ float head_reduce(float x, int lph);
+// Warp-cooperative row kernels: one warp per row (or per chunk of a row's edges), lane l
+// holds the EPL consecutive features l*EPL .. l*EPL+EPL-1 of every row it reads
+// (contiguous across the warp, so a row is one coalesced read), and a head's r features
+// lie in LPH = r/EPL adjacent lanes, whose dot products meet in a butterfly of shuffles.
+// r is a power of two and EPL <= r, so LPH is a power of two, D is a multiple of EPL and
+// every lane's slice starts on an EPL-element boundary (the vector loads below rely on it).
 
-// One warp per row i (lanes over features, EPL each): the gate, readout and blend
-// backward.  Writes dL [N, D], dnum [N, D], dden [N, H], the global part of dQ into
-// dZ [:, 0:D] and dt into dZ [:, 3D] (dg summed over the whole row in lane order).
+template <int EPL>
+__device__ __forceinline__ void unpack_bf16(const uint32_t *w, float *x) {
+#pragma unroll
+    for (int e = 0; e < EPL / 2; ++e) {
+        const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
+        const float2 f = __bfloat1622float2(p);
+        x[2 * e] = f.x;
+        x[2 * e + 1] = f.y;
+    }
+}
+
+template <typename T, int EPL>
+__device__ __forceinline__ void ld_row(const T *row, int lane, bool act, float (&x)[EPL]) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+    if (!act) return;
+    const T *p = row + lane * EPL;
+    if constexpr (std::is_same<T, float>::value) {
+        if constexpr (EPL % 4 == 0) {
+#pragma unroll
+            for (int v = 0; v < EPL / 4; ++v) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(p) + v);
+                x[4 * v] = f.x; x[4 * v + 1] = f.y; x[4 * v + 2] = f.z; x[4 * v + 3] = f.w;
+            }
+        } else if constexpr (EPL == 2) {
+            const float2 f = __ldg(reinterpret_cast<const float2 *>(p));
+            x[0] = f.x; x[1] = f.y;
+        } else {
+            x[0] = __ldg(p);
+        }
+    } else {
+        if constexpr (EPL % 8 == 0) {
+#pragma unroll
+            for (int v = 0; v < EPL / 8; ++v) {
+                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p) + v);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                unpack_bf16<8>(ww, x + 8 * v);
+            }
+        } else if constexpr (EPL == 4) {
+            const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
+            const uint32_t ww[2] = {w.x, w.y};
+            unpack_bf16<4>(ww, x);
+        } else if constexpr (EPL == 2) {
+            const uint32_t w = __ldg(reinterpret_cast<const unsigned int *>(p));
+            unpack_bf16<2>(&w, x);
+        } else {
+            x[0] = __bfloat162float(*p);
+        }
+    }
+}
+
+// x = p[0 .. EPL-1] of an fp32 matrix row (p on an EPL-float boundary).  NC: through the
+// read-only path (data the kernel does not write); otherwise plain loads.
+template <int EPL, bool NC = true>
+__device__ __forceinline__ void ld_mrow(const float *p, float (&x)[EPL]) {
+    if constexpr (EPL % 4 == 0) {
+#pragma unroll
+        for (int v = 0; v < EPL / 4; ++v) {
+            const float4 *a = reinterpret_cast<const float4 *>(p) + v;
+            const float4 f = NC ? __ldg(a) : *a;
+            x[4 * v] = f.x; x[4 * v + 1] = f.y; x[4 * v + 2] = f.z; x[4 * v + 3] = f.w;
+        }
+    } else if constexpr (EPL == 2) {
+        const float2 *a = reinterpret_cast<const float2 *>(p);
+        const float2 f = NC ? __ldg(a) : *a;
+        x[0] = f.x; x[1] = f.y;
+    } else {
+        x[0] = NC ? __ldg(p) : *p;
+    }
+}
+
+// p[0 .. EPL-1] = x for an fp32 row slice on an EPL-float boundary.
+template <int EPL>
+__device__ __forceinline__ void st_mrow(float *p, const float (&x)[EPL]) {
+    if constexpr (EPL % 4 == 0) {
+#pragma unroll
+        for (int v = 0; v < EPL / 4; ++v)
+            reinterpret_cast<float4 *>(p)[v] = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+    } else if constexpr (EPL == 2) {
+        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    } else {
+        p[0] = x[0];
+    }
+}
+
+__device__ __forceinline__ float head_reduce(float x, int lph) {
+    for (int o = 1; o < lph; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// out[x] += sum over c < R of M[c * R + f0 + x] * u_c for one head: M is a row-major
+// R x R fp32 block, and u_c is held by the head's lanes (lane hb + c / EPL, element
+// c % EPL), so it travels by shuffle.  Every lane of the warp takes part (lanes outside
+// D pass f0 = 0 and hb = 0 and discard the result).
+template <int EPL>
+__device__ __forceinline__ void head_matvec(const float *M, int R, int f0, int hb, int lph, const float (&u)[EPL],
+                                            float (&out)[EPL]) {
+    for (int sl = 0; sl < lph; ++sl) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            const float uc = __shfl_sync(0xffffffffu, u[e], hb + sl);
+            float m[EPL];
+            ld_mrow<EPL>(M + static_cast<int64_t>(sl * EPL + e) * R + f0, m);
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) out[x] = fmaf(m[x], uc, out[x]);
+        }
+    }
+}
+
+// The lane's head h, in-head feature offset f0 and the head's first lane hb.
+struct LaneHead {
+    bool act;
+    int lph, h, f0, hb;
+    __device__ __forceinline__ LaneHead(int lane, int EPL, int D, int R) {
+        act = lane * EPL < D;
+        lph = R / EPL;
+        h = act ? lane * EPL / R : 0;
+        f0 = act ? lane * EPL - h * R : 0;
+        hb = act ? h * lph : 0;
+    }
+};
+
+// One warp per row i: the gate, readout and blend backward.  Writes dL [N, D],
+// dnum [N, D], dden [N, H], the global part of dQ into dZ [:, 0:D] and dt into dZ [:, 3D]
+// (dg summed over the whole row in lane order).  Sz holds S [H][R][R] then z [H][R];
+// ST [H][R][R] is S transposed per head.
 template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_readout_kernel(
     const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t, const float *__restrict__ Sz,
     const float *__restrict__ ST, const T *__restrict__ dY, int64_t N, int H, int R, float b_g, float eps,
-    float *__restrict__ dL,
-    float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ, int64_t dz_ld) {
+    float *__restrict__ dL, float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ,
+    int64_t dz_ld) {
     const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (i >= N) return;                                   // warp-uniform
     const int D = H * R;
-    const bool act = lane * EPL < D;
-    const int lph = R / EPL, h = act ? lane * EPL / R : 0;
-    const float *S = Sz + static_cast<int64_t>(h) * R * R;
-    const float *z = Sz + static_cast<int64_t>(H) * R * R + h * R;
-    const T *qh = Q + i * D + h * R;                      // the lane's head
-    float q[EPL], dy[EPL], lv[EPL];
-    ld_row<T, EPL>(Q + i * D, lane, act, q);
-    ld_row<T, EPL>(dY + i * D, lane, act, dy);
-    ld_row<T, EPL>(L + i * D, lane, act, lv);
-    const int f0 = lane * EPL - h * R;                    // in-head index of the lane's first feature
+    const LaneHead lh(lane, EPL, D, R);
+    const float *S = Sz + static_cast<int64_t>(lh.h) * R * R;
+    float q[EPL], dy[EPL], lv[EPL], ph[EPL], zz[EPL];
+    ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
+    ld_row<T, EPL>(dY + i * D, lane, lh.act, dy);
+    ld_row<T, EPL>(L + i * D, lane, lh.act, lv);
+    ld_mrow<EPL>(Sz + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, zz);
     float den = 0.f;
-    if (act) {
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) den = fmaf(phi(q[x]), z[f0 + x], den);
+    for (int x = 0; x < EPL; ++x) {
+        ph[x] = phi(q[x]);
+        den = fmaf(ph[x], zz[x], den);
     }
-    den = head_reduce(den, lph) + eps;
-    // num_c = sum_a phi(q_a) S[a][c] for the lane's features c (phi(q_a) read back from
-    // the row, the same for the head's lanes)
+    den = head_reduce(den, lh.lph) + eps;
     float G[EPL];
 #pragma unroll
     for (int x = 0; x < EPL; ++x) G[x] = 0.f;
-    if (act)
-        for (int a = 0; a < R; ++a) {
-            const float pa = phi(ldf<T>(qh + a));
-#pragma unroll
-            for (int x = 0; x < EPL; ++x) G[x] = fmaf(pa, S[a * R + f0 + x], G[x]);
-        }
+    head_matvec<EPL>(S, R, lh.f0, lh.hb, lh.lph, ph, G);  // num_f = sum_a phi(q_a) S[a][f]
     const float g = 1.f / (1.f + __expf(-(t[i] + b_g)));
-    float dgp = 0.f, dGG = 0.f;
-    const int64_t o = i * D + lane * EPL;
+    float dgp = 0.f, dGG = 0.f, gl[EPL], dn[EPL];
 #pragma unroll
     for (int x = 0; x < EPL; ++x) {
         G[x] /= den;
         dgp = fmaf(dy[x], lv[x] - G[x], dgp);
         const float dG = (1.f - g) * dy[x];
         dGG = fmaf(dG, G[x], dGG);
-        if (act) {
-            dL[o + x] = g * dy[x];
-            dnum[o + x] = dG / den;
-        }
+        gl[x] = g * dy[x];
+        dn[x] = dG / den;
     }
-    const float dd = -head_reduce(dGG, lph) / den;
-    if (act && (lane % lph) == 0) dden[i * H + h] = dd;
-    __syncwarp();                                         // dnum of the row is written
-    const float *dn = dnum + i * D + h * R;
-    const float *STh = ST + static_cast<int64_t>(h) * R * R;   // STh[c][a] = S[a][c]
-    if (act) {
+    const int64_t o = i * D + lane * EPL;
+    if (lh.act) {
+        st_mrow<EPL>(dL + o, gl);
+        st_mrow<EPL>(dnum + o, dn);
+    }
+    const float dd = -head_reduce(dGG, lh.lph) / den;
+    if (lh.act && (lane % lh.lph) == 0) dden[i * H + lh.h] = dd;
+    float acc[EPL];
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) {
-            float acc = z[f0 + x] * dd;
-            for (int c = 0; c < R; ++c) acc = fmaf(STh[c * R + f0 + x], dn[c], acc);
-            dZ[i * dz_ld + lane * EPL + x] = acc * dphi(q[x]);
-        }
-    }
+    for (int x = 0; x < EPL; ++x) acc[x] = zz[x] * dd;
+    // dphi(q)_f = sum_c S[f][c] dnum_c + z_f dden, through ST's rows c
+    head_matvec<EPL>(ST + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, dn, acc);
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) acc[x] *= dphi(q[x]);
+    if (lh.act) st_mrow<EPL>(dZ + i * dz_ld + lane * EPL, acc);
     for (int w = 16; w > 0; w >>= 1) dgp += __shfl_xor_sync(0xffffffffu, dgp, w);
     if (lane == 0) dZ[i * dz_ld + 3 * D] = g * (1.f - g) * dgp;
 }
@@ -116,66 +232,106 @@ __global__ void __launch_bounds__(256) bwd_readout_kernel(
 // Partial sums of dS | dz over the row range of block column p, per head h =
 // blockIdx.y, in the layout [H][R][R+1] (column R is dz):
 //   part[p][h][a][c] = sum_i phi(q_i[h R + a]) * (c < R ? dnum_i[h R + c] : dden_i[h]).
-// 32-row tiles of phi(Q_h) and [dnum_h | dden_h] are staged in shared memory; each thread
-// owns outputs o = tid, tid + 256, ... of the head's R (R + 1).
+// 32-row tiles of phi(Q_h), dnum_h and dden_h are staged in shared memory; each thread
+// owns 4 (a) x 4 (c) output tiles (NT of them when R >= 64) and, for the first column
+// tile, the dz entries of its 4 a's.  For R <= 32 the block's threads form G row groups
+// (group g takes rows g, g + G, ... of each staged tile), added in group order at the end.
 template <typename T, int R>
 __global__ void __launch_bounds__(256) bwd_dsz_partial_kernel(const T *__restrict__ Q, const float *__restrict__ dnum,
                                                               const float *__restrict__ dden, int64_t N, int H,
                                                               int64_t rows_per_part, float *__restrict__ part) {
-    extern __shared__ float tile[];                      // [32][R] phi(q) then [32][R + 1] dnum | dden
-    constexpr int kRowsT = 32;
-    const int h = blockIdx.y;
+    constexpr int kRowsT = 32, TR = R / 4, NTILE = TR * TR;
+    constexpr int G = NTILE >= 256 ? 1 : 256 / NTILE;
+    constexpr int NT = NTILE >= 256 ? NTILE / 256 : 1;
+    constexpr int PH = R * (R + 1);                      // outputs per head
+    extern __shared__ float4 dsm4[];
+    float *pq = reinterpret_cast<float *>(dsm4);          // [32][R] phi(q)
+    float *pw = pq + kRowsT * R;                          // [32][R] dnum
+    float *pd = pw + kRowsT * R;                          // [32] dden
+    float *red = pd + kRowsT;                             // [G][PH] when G > 1
+    const int h = blockIdx.y, t = threadIdx.x;
     const int D = H * R;
-    const int per_head = R * (R + 1);
-    float *pq = tile, *pw = tile + kRowsT * R;
+    const int g = G > 1 ? t / NTILE : 0;
     const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_part;
     const int64_t r1 = std::min<int64_t>(N, r0 + rows_per_part);
-    constexpr int kMaxOut = (R * (R + 1) + 255) / 256;
-    float acc[kMaxOut];
-    const int n_out = (per_head - static_cast<int>(threadIdx.x) + 255) / 256;
+    float acc[NT][4][4], accz[NT][4];
 #pragma unroll
-    for (int u = 0; u < kMaxOut; ++u) acc[u] = 0.f;
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            accz[n][u] = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[n][u][w] = 0.f;
+        }
     for (int64_t i0 = r0; i0 < r1; i0 += kRowsT) {
-        for (int l = threadIdx.x; l < kRowsT * (R + 1); l += 256) {
-            const int rr = l / (R + 1), c = l % (R + 1);
+        for (int l = t; l < kRowsT * R; l += 256) {
+            const int rr = l / R, c = l % R;
             const int64_t i = i0 + rr;
             const bool in = i < r1;
-            if (c < R) {
-                pq[rr * R + c] = in ? phi(ldf<T>(Q + i * D + h * R + c)) : 0.f;
-                pw[rr * (R + 1) + c] = in ? dnum[i * D + h * R + c] : 0.f;
-            } else {
-                pw[rr * (R + 1) + R] = in ? dden[i * H + h] : 0.f;
-            }
+            pq[l] = in ? phi(ldf<T>(Q + i * D + h * R + c)) : 0.f;
+            pw[l] = in ? dnum[i * D + h * R + c] : 0.f;
         }
+        if (t < kRowsT) pd[t] = i0 + t < r1 ? dden[(i0 + t) * H + h] : 0.f;
         __syncthreads();
 #pragma unroll
-        for (int u = 0; u < kMaxOut; ++u) {
-            if (u < n_out) {
-                const int oo = threadIdx.x + u * 256;
-                const int a = oo / (R + 1), c = oo % (R + 1);
-                float sacc = acc[u];
-                for (int rr = 0; rr < kRowsT; ++rr) sacc = fmaf(pq[rr * R + a], pw[rr * (R + 1) + c], sacc);
-                acc[u] = sacc;
+        for (int n = 0; n < NT; ++n) {
+            const int tile = G > 1 ? t % NTILE : t + n * 256;
+            const int a0 = (tile / TR) * 4, c0 = (tile % TR) * 4;
+            for (int rr = g; rr < kRowsT; rr += G) {
+                const float4 av = *reinterpret_cast<const float4 *>(pq + rr * R + a0);
+                const float4 bv = *reinterpret_cast<const float4 *>(pw + rr * R + c0);
+                const float a4[4] = {av.x, av.y, av.z, av.w}, b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) acc[n][u][w] = fmaf(a4[u], b4[w], acc[n][u][w]);
+                if (c0 == 0) {
+                    const float dd = pd[rr];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) accz[n][u] = fmaf(a4[u], dd, accz[n][u]);
+                }
             }
         }
         __syncthreads();
     }
-    const int total = H * per_head;
-    float *out = part + static_cast<int64_t>(blockIdx.x) * total + h * per_head;
+    float *out = part + static_cast<int64_t>(blockIdx.x) * H * PH + static_cast<int64_t>(h) * PH;
+    float *dst = G > 1 ? red + g * PH : out;
 #pragma unroll
-    for (int u = 0; u < kMaxOut; ++u)
-        if (u < n_out) out[threadIdx.x + u * 256] = acc[u];
+    for (int n = 0; n < NT; ++n) {
+        const int tile = G > 1 ? t % NTILE : t + n * 256;
+        const int a0 = (tile / TR) * 4, c0 = (tile % TR) * 4;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) dst[(a0 + u) * (R + 1) + c0 + w] = acc[n][u][w];
+            if (c0 == 0) dst[(a0 + u) * (R + 1) + R] = accz[n][u];
+        }
+    }
+    if constexpr (G > 1) {
+        __syncthreads();
+        for (int o = t; o < PH; o += 256) {
+            float v = 0.f;
+            for (int gg = 0; gg < G; ++gg) v += red[gg * PH + o];
+            out[o] = v;
+        }
+    }
 }
 
-// dst[h][c][a] = src[h][a][c] (a, c < R) for per-head R x R blocks with row stride ld.
-__global__ void bwd_transpose_heads_kernel(const float *__restrict__ src, int ld, int H, int R,
-                                           float *__restrict__ dst) {
-    const int64_t total = static_cast<int64_t>(H) * R * R;
+// Per-head R x R blocks of src (row stride ld, head stride R * ld): dstT[h][c][a] =
+// src[h][a][c] and, when dstC is given, the compact copy dstC[h][a][c] = src[h][a][c]
+// followed by column R of src as dstC[H R R + h R + a] (so dstC has the [S | z] layout).
+__global__ void bwd_heads_prep_kernel(const float *__restrict__ src, int ld, int H, int R, float *__restrict__ dstT,
+                                      float *__restrict__ dstC) {
+    const int64_t RR = static_cast<int64_t>(R) * R, total = static_cast<int64_t>(H) * RR;
     for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
          o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int h = static_cast<int>(o / (static_cast<int64_t>(R) * R));
-        const int c = static_cast<int>((o / R) % R), a = static_cast<int>(o % R);
-        dst[o] = src[static_cast<int64_t>(h) * R * ld + static_cast<int64_t>(a) * ld + c];
+        const int64_t h = o / RR;
+        const int u = static_cast<int>((o / R) % R), w = static_cast<int>(o % R);
+        dstT[o] = src[(h * R + w) * ld + u];
+        if (dstC) {
+            dstC[o] = src[(h * R + u) * ld + w];
+            if (w == 0) dstC[total + h * R + u] = src[(h * R + u) * ld + R];
+        }
     }
 }
 
@@ -189,24 +345,8 @@ __global__ void bwd_sum_parts_kernel(const float *__restrict__ part, int P, int6
     }
 }
 
-// Warp-cooperative row kernels: one warp per row, lane l holds the EPL consecutive
-// features l*EPL .. l*EPL+EPL-1 of every row it reads (contiguous across the warp, so a
-// row is one coalesced read), and a head's r features lie in LPH = r/EPL adjacent lanes,
-// whose dot products meet in a butterfly of shuffles.
-
-template <typename T, int EPL>
-__device__ __forceinline__ void ld_row(const T *row, int lane, bool act, float (&x)[EPL]) {
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) x[e] = act ? ldf<T>(row + lane * EPL + e) : 0.f;
-}
-
-__device__ __forceinline__ float head_reduce(float x, int lph) {
-    for (int o = 1; o < lph; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-constexpr int kEU = 4;           // edges whose rows are loaded before any is used
-constexpr int kHeavyWarps = 32;  // warps per heavy row (one 1024-thread block)
+constexpr int kEU = 4;            // edges whose rows are loaded before any is used
+constexpr int kChunk = 32;        // edges per chunk of a heavy row (one warp each)
 
 // Online (max, sum) of exp(s) over the edges [a, b) of target row q (this warp's lanes).
 template <typename T, int EPL>
@@ -268,89 +408,193 @@ __device__ __forceinline__ void q_grad_range(const int32_t *col_idx, const T *KV
     }
 }
 
-// Target rows of the forward CSR: per head the softmax's log-sum-exp and D_i = dL_i . L_i,
-// and the local part of dq_i added into dZ [:, 0:D].  Light rows (the `rows` list): one
-// warp each.  Heavy rows (HEAVY): one 1024-thread block each, its 32 warps taking
-// contiguous shares of the edges; their partial (max, sum) and dq are combined in warp
-// order through shared memory.
-template <typename T, int EPL, bool HEAVY>
-__global__ void __launch_bounds__(HEAVY ? 1024 : 256) bwd_local_q_kernel(
+// Light target rows of the forward CSR (one warp each, the `rows` list): per head the
+// softmax's log-sum-exp and D_i = dL_i . L_i, and the local part of dq_i added into
+// dZ [:, 0:D].
+template <typename T, int EPL>
+__global__ void __launch_bounds__(256) bwd_local_q_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ L, const float *__restrict__ dL, int H, int R, float inv_sqrt_r,
     float *__restrict__ lse, float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
-    __shared__ float sm_m[HEAVY ? kHeavyWarps : 1][32], sm_l[HEAVY ? kHeavyWarps : 1][32];
-    __shared__ float sm_dq[HEAVY ? 32 * 32 : 1];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t slot = HEAVY ? blockIdx.x : (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
-    if (slot >= n_rows) return;                           // uniform per warp (per block when HEAVY)
+    const int lane = threadIdx.x & 31;
+    const int64_t slot = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (slot >= n_rows) return;                           // warp-uniform
     const int64_t i = rows[slot];
     const int D = H * R;
-    const bool act = lane * EPL < D;
-    const int lph = R / EPL, h = act ? lane * EPL / R : 0;
+    const LaneHead lh(lane, EPL, D, R);
     float q[EPL], dl[EPL], lv[EPL];
-    ld_row<T, EPL>(Q + i * D, lane, act, q);
-    ld_row<float, EPL>(dL + i * D, lane, act, dl);
-    ld_row<T, EPL>(L + i * D, lane, act, lv);
+    ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
+    ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
+    ld_row<T, EPL>(L + i * D, lane, lh.act, lv);
     const int32_t r0 = row_ptr[i], r1 = row_ptr[i + 1];
-    int32_t a = r0, b = r1;
-    if (HEAVY) {
-        const int32_t per = (r1 - r0 + kHeavyWarps - 1) / kHeavyWarps;
-        a = min(r1, r0 + warp * per);
-        b = min(r1, a + per);
-    }
     float m = -INFINITY, l = 0.f;
-    q_lse_range<T, EPL>(col_idx, KV, D, lane, act, lph, inv_sqrt_r, q, a, b, m, l);
-    if (HEAVY) {
-        sm_m[warp][lane] = m;
-        sm_l[warp][lane] = l;
+    q_lse_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, r0, r1, m, l);
+    const float ls = r1 > r0 ? m + __logf(l) : 0.f;
+    float dd = 0.f;
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dd = fmaf(dl[x], lv[x], dd);
+    dd = head_reduce(dd, lh.lph);
+    if (lh.act && (lane % lh.lph) == 0) {
+        lse[i * H + lh.h] = ls;
+        Dd[i * H + lh.h] = dd;
+    }
+    float dq[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+    q_grad_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, dl, ls, dd, r0, r1, dq);
+    if (lh.act) {
+        float *o = dZ + i * dz_ld + lane * EPL;
+        float cur[EPL];
+        ld_mrow<EPL, false>(o, cur);
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) cur[x] += dq[x];
+        st_mrow<EPL>(o, cur);
+    }
+}
+
+// Chunks of heavy target rows, one warp each: chunk c covers the edges
+// [chunks[c].y, min(chunks[c].y + kChunk, row end)) of row chunks[c].x.
+//   PHASE 0: the chunk's per-lane online (max, sum) into ml[c][0:32] | ml[c][32:64].
+//   PHASE 1: the chunk's share of dq_i (the row's lse and D_i already final) into part[c][0:D].
+template <typename T, int EPL, int PHASE>
+__global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
+    const int2 *__restrict__ chunks, int64_t n_chunks, const int32_t *__restrict__ row_ptr,
+    const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
+    const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const float *__restrict__ Dd, float *__restrict__ ml, float *__restrict__ part) {
+    const int lane = threadIdx.x & 31;
+    const int64_t c = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (c >= n_chunks) return;                            // warp-uniform
+    const int2 ch = chunks[c];
+    const int64_t i = ch.x;
+    const int32_t a = ch.y, b = min(row_ptr[i + 1], ch.y + kChunk);
+    const int D = H * R;
+    const LaneHead lh(lane, EPL, D, R);
+    float q[EPL];
+    ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
+    if constexpr (PHASE == 0) {
+        float m = -INFINITY, l = 0.f;
+        q_lse_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, a, b, m, l);
+        ml[c * 64 + lane] = m;
+        ml[c * 64 + 32 + lane] = l;
+    } else {
+        float dl[EPL], dq[EPL];
+        ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+        const float ls = lse[i * H + lh.h], dd = Dd[i * H + lh.h];
+        q_grad_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, dl, ls, dd, a, b, dq);
+        if (lh.act) st_mrow<EPL>(part + c * D + lane * EPL, dq);
+    }
+}
+
+// Heavy rows are merged by one block of kMW warps each: warp w takes the row's chunks
+// c0 + w, c0 + w + kMW, ... (in order, kMU loads in flight), and warp 0 then combines the
+// warps' results in warp order through shared memory, so the order is fixed.
+constexpr int kMW = 8, kMU = 4;
+
+// Heavy target rows over their chunks [chunk_ptr[s], chunk_ptr[s + 1]):
+//   PHASE 0: merge the chunks' (max, sum) into lse_i, and D_i = dL_i . L_i.
+//   PHASE 1: dq_i = the chunks' shares summed, added into dZ [:, 0:D].
+// Dynamic shared memory: kMW * 64 floats (PHASE 0) or kMW * D floats (PHASE 1).
+template <typename T, int EPL, int PHASE>
+__global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
+    const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ chunk_ptr,
+    const float *__restrict__ ml, const float *__restrict__ part, const T *__restrict__ L,
+    const float *__restrict__ dL, int H, int R, float *__restrict__ lse, float *__restrict__ Dd,
+    float *__restrict__ dZ, int64_t dz_ld) {
+    extern __shared__ float msm[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t slot = blockIdx.x;
+    if (slot >= n_rows) return;                           // block-uniform
+    const int64_t i = rows[slot];
+    const int D = H * R;
+    const LaneHead lh(lane, EPL, D, R);
+    const int32_t c0 = chunk_ptr[slot], c1 = chunk_ptr[slot + 1];
+    if constexpr (PHASE == 0) {
+        float m = -INFINITY, l = 0.f;
+        for (int32_t c = c0 + warp; c < c1; c += kMU * kMW) {
+            float m2[kMU], l2[kMU];
+#pragma unroll
+            for (int u = 0; u < kMU; ++u) {
+                const int32_t cc = c + u * kMW;
+                m2[u] = cc < c1 ? ml[static_cast<int64_t>(cc) * 64 + lane] : -INFINITY;
+                l2[u] = cc < c1 ? ml[static_cast<int64_t>(cc) * 64 + 32 + lane] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kMU; ++u) {
+                const float mn = fmaxf(m, m2[u]);
+                if (mn != -INFINITY) {
+                    l = l * __expf(m - mn) + l2[u] * __expf(m2[u] - mn);
+                    m = mn;
+                }
+            }
+        }
+        msm[warp * 64 + lane] = m;
+        msm[warp * 64 + 32 + lane] = l;
         __syncthreads();
+        if (warp != 0) return;
         m = -INFINITY;
         l = 0.f;
-        for (int w = 0; w < kHeavyWarps; ++w) {          // warp order
-            const float m2 = sm_m[w][lane], l2 = sm_l[w][lane];
+        for (int w = 0; w < kMW; ++w) {
+            const float m2 = msm[w * 64 + lane], l2 = msm[w * 64 + 32 + lane];
             const float mn = fmaxf(m, m2);
             if (mn != -INFINITY) {
                 l = l * __expf(m - mn) + l2 * __expf(m2 - mn);
                 m = mn;
             }
         }
-    }
-    const float ls = r1 > r0 ? m + __logf(l) : 0.f;
-    float dd = 0.f;
+        float dl[EPL], lv[EPL];
+        ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
+        ld_row<T, EPL>(L + i * D, lane, lh.act, lv);
+        float dd = 0.f;
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) dd = fmaf(dl[x], lv[x], dd);
-    dd = head_reduce(dd, lph);
-    if (act && (lane % lph) == 0 && (!HEAVY || warp == 0)) {
-        lse[i * H + h] = ls;
-        Dd[i * H + h] = dd;
-    }
-    float dq[EPL];
+        for (int x = 0; x < EPL; ++x) dd = fmaf(dl[x], lv[x], dd);
+        dd = head_reduce(dd, lh.lph);
+        if (lh.act && (lane % lh.lph) == 0) {
+            lse[i * H + lh.h] = m + __logf(l);
+            Dd[i * H + lh.h] = dd;
+        }
+    } else {
+        float dq[EPL];
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
-    q_grad_range<T, EPL>(col_idx, KV, D, lane, act, lph, inv_sqrt_r, q, dl, ls, dd, a, b, dq);
-    if (HEAVY) {
-        // add the warps' dq in warp order, one 32 * EPL-feature slice at a time
-        for (int w = 0; w < kHeavyWarps; ++w) {
-            if (warp == w) {
+        for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+        if (lh.act) {
+            for (int32_t c = c0 + warp; c < c1; c += kMU * kMW) {
+                float pv[kMU][EPL];
 #pragma unroll
-                for (int x = 0; x < EPL; ++x) {
-                    const int f = lane * EPL + x;
-                    if (f < 32 * 32) sm_dq[f] = (w == 0 ? 0.f : sm_dq[f]) + dq[x];
+                for (int u = 0; u < kMU; ++u) {
+                    const int32_t cc = c + u * kMW;
+                    if (cc < c1) {
+                        ld_mrow<EPL>(part + static_cast<int64_t>(cc) * D + lane * EPL, pv[u]);
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < EPL; ++x) pv[u][x] = 0.f;
+                    }
                 }
+#pragma unroll
+                for (int u = 0; u < kMU; ++u)
+#pragma unroll
+                    for (int x = 0; x < EPL; ++x) dq[x] += pv[u][x];
             }
-            __syncthreads();
+            st_mrow<EPL>(msm + warp * D + lane * EPL, dq);
         }
-        if (warp == 0) {
+        __syncthreads();
+        if (warp != 0 || !lh.act) return;
+        float acc[EPL], pv[EPL];
+        float *o = dZ + i * dz_ld + lane * EPL;
+        ld_mrow<EPL, false>(o, acc);                       // the global part of dq_i
 #pragma unroll
-            for (int x = 0; x < EPL; ++x) dq[x] = sm_dq[lane * EPL + x];
-        } else {
-            return;
+        for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+        for (int w = 0; w < kMW; ++w) {
+            ld_mrow<EPL, false>(msm + w * D + lane * EPL, pv);
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) dq[x] += pv[x];
         }
-    }
-    if (act) {
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) dZ[i * dz_ld + lane * EPL + x] += dq[x];
+        for (int x = 0; x < EPL; ++x) acc[x] += dq[x];
+        st_mrow<EPL>(o, acc);
     }
 }
 
@@ -369,8 +613,8 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
             const int64_t i = live ? t_col[e + u] : 0;
             ld_row<T, EPL>(Q + i * D, lane, act && live, q[u]);
             ld_row<float, EPL>(dL + i * D, lane, act && live, dl[u]);
-            ls[u] = live ? lse[i * H + h] : 0.f;
-            dd[u] = live ? Dd[i * H + h] : 0.f;
+            ls[u] = live ? __ldg(lse + i * H + h) : 0.f;
+            dd[u] = live ? __ldg(Dd + i * H + h) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kEU; ++u) {
@@ -396,156 +640,290 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
 
 // Source rows of the transposed CSR (the targets i of j): the local terms of dk_j and
 // dv_j, plus the global terms through phi(k_j), written to dZ [:, D:2D] and [:, 2D:3D].
-// dSz holds dS | dz as [H][R][R+1].  Light rows one warp each, heavy rows one block each
-// (warp shares combined in warp order), as bwd_local_q_kernel.
-template <typename T, int EPL, bool HEAVY>
-__global__ void __launch_bounds__(HEAVY ? 1024 : 256) bwd_local_kv_kernel(
+// Light rows (PARTS false, one warp each) walk their edges; heavy rows (PARTS true, one
+// block of kMW warps each) sum their chunks' shares part[c][0:D] | part[c][D:2D], c in
+// [chunk_ptr[s], chunk_ptr[s + 1]), warp-strided and then in warp order.  dSc holds dS [H][R][R] then dz [H][R]; dST is dS transposed per head.
+template <typename T, int EPL, bool PARTS>
+__global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
-    const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
-    const float *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
-    const float *__restrict__ dSz, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
-    float *__restrict__ dZ, int64_t dz_ld) {
-    __shared__ float sm_dk[HEAVY ? 32 * 32 : 1], sm_dv[HEAVY ? 32 * 32 : 1];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t slot = HEAVY ? blockIdx.x : (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
-    if (slot >= n_rows) return;
+    const int32_t *__restrict__ t_col, const int32_t *__restrict__ chunk_ptr, const float *__restrict__ part,
+    const T *__restrict__ Q, const T *__restrict__ KV, const float *__restrict__ dL,
+    const float *__restrict__ lse, const float *__restrict__ Dd, const float *__restrict__ dSc,
+    const float *__restrict__ dST, int H, int R, float inv_sqrt_r, float *__restrict__ dZ, int64_t dz_ld) {
+    extern __shared__ float msm[];                       // PARTS: [kMW][2D]
+    const int lane = threadIdx.x & 31;
+    const int64_t slot = PARTS ? blockIdx.x : (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (slot >= n_rows) return;                           // warp-uniform (block-uniform with PARTS)
     const int64_t j = rows[slot];
     const int D = H * R;
-    const bool act = lane * EPL < D;
-    const int lph = R / EPL, h = act ? lane * EPL / R : 0;
+    const LaneHead lh(lane, EPL, D, R);
     const T *krow = KV + j * 2 * D;
     float k[EPL], v[EPL], dk[EPL], dv[EPL];
-    ld_row<T, EPL>(krow, lane, act, k);
-    ld_row<T, EPL>(krow + D, lane, act, v);
 #pragma unroll
     for (int x = 0; x < EPL; ++x) dk[x] = dv[x] = 0.f;
-    const int32_t r0 = t_row_ptr[j], r1 = t_row_ptr[j + 1];
-    int32_t a = r0, b = r1;
-    if (HEAVY) {
-        const int32_t per = (r1 - r0 + kHeavyWarps - 1) / kHeavyWarps;
-        a = min(r1, r0 + warp * per);
-        b = min(r1, a + per);
-    }
-    kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, act, lph, h, inv_sqrt_r, k, v, a, b, dk, dv);
-    if (HEAVY) {
-        for (int w = 0; w < kHeavyWarps; ++w) {
-            if (warp == w) {
+    if constexpr (PARTS) {
+        const int warp = threadIdx.x >> 5;
+        const int32_t c0 = chunk_ptr[slot], c1 = chunk_ptr[slot + 1];
+        if (lh.act) {
+            for (int32_t c = c0 + warp; c < c1; c += kMU * kMW) {
+                float pk[kMU][EPL], pv[kMU][EPL];
 #pragma unroll
-                for (int x = 0; x < EPL; ++x) {
-                    const int f = lane * EPL + x;
-                    if (f < 32 * 32) {
-                        sm_dk[f] = (w == 0 ? 0.f : sm_dk[f]) + dk[x];
-                        sm_dv[f] = (w == 0 ? 0.f : sm_dv[f]) + dv[x];
+                for (int u = 0; u < kMU; ++u) {
+                    const int32_t cc = c + u * kMW;
+                    if (cc < c1) {
+                        const float *pc = part + static_cast<int64_t>(cc) * 2 * D + lane * EPL;
+                        ld_mrow<EPL>(pc, pk[u]);
+                        ld_mrow<EPL>(pc + D, pv[u]);
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < EPL; ++x) pk[u][x] = pv[u][x] = 0.f;
                     }
                 }
+#pragma unroll
+                for (int u = 0; u < kMU; ++u)
+#pragma unroll
+                    for (int x = 0; x < EPL; ++x) {
+                        dk[x] += pk[u][x];
+                        dv[x] += pv[u][x];
+                    }
             }
-            __syncthreads();
+            st_mrow<EPL>(msm + warp * 2 * D + lane * EPL, dk);
+            st_mrow<EPL>(msm + warp * 2 * D + D + lane * EPL, dv);
         }
+        __syncthreads();
         if (warp != 0) return;
+        if (lh.act) {
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) {
-            dk[x] = sm_dk[lane * EPL + x];
-            dv[x] = sm_dv[lane * EPL + x];
-        }
-    }
-    // global branch, S = sum phi(k) v^T and z = sum phi(k): for the lane's features
-    // (head h, in-head index f = lane*EPL + x - h*R)
-    if (act) {
-        const float *dS = dSz + static_cast<int64_t>(h) * R * (R + 1);
-        const float *dSTh = dST + static_cast<int64_t>(h) * R * R;   // dSTh[c][f] = dS[f][c]
-        const T *kh = krow + h * R, *vh = krow + D + h * R;
+            for (int x = 0; x < EPL; ++x) dk[x] = dv[x] = 0.f;
+            for (int w = 0; w < kMW; ++w) {
+                float pk[EPL], pv[EPL];
+                ld_mrow<EPL, false>(msm + w * 2 * D + lane * EPL, pk);
+                ld_mrow<EPL, false>(msm + w * 2 * D + D + lane * EPL, pv);
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) {
-            const int f = lane * EPL + x - h * R;
-            float dphk = dS[f * (R + 1) + R];             // dz_f
-            float dvg = 0.f;
-            for (int c = 0; c < R; ++c) {
-                dphk = fmaf(dSTh[c * R + f], ldf<T>(vh + c), dphk);
-                dvg = fmaf(dS[c * (R + 1) + f], phi(ldf<T>(kh + c)), dvg);
+                for (int x = 0; x < EPL; ++x) {
+                    dk[x] += pk[x];
+                    dv[x] += pv[x];
+                }
             }
-            dk[x] = fmaf(dphk, dphi(k[x]), dk[x]);
-            dv[x] += dvg;
         }
+    }
+    ld_row<T, EPL>(krow, lane, lh.act, k);
+    ld_row<T, EPL>(krow + D, lane, lh.act, v);
+    if constexpr (!PARTS) {
+        kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, lh.act, lh.lph, lh.h, inv_sqrt_r, k, v,
+                              t_row_ptr[j], t_row_ptr[j + 1], dk, dv);
+    }
+    // global branch, S = sum phi(k) v^T and z = sum phi(k):
+    //   dphi(k_j)_f = sum_c dS[f][c] v_c + dz_f,  dv_j,f += sum_c dS[c][f] phi(k_c)
+    float dphk[EPL], dvg[EPL], pk[EPL];
+    ld_mrow<EPL>(dSc + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, dphk);
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) {
+        dvg[x] = 0.f;
+        pk[x] = phi(k[x]);
+    }
+    head_matvec<EPL>(dST + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, v, dphk);
+    head_matvec<EPL>(dSc + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, pk, dvg);
+    if (lh.act) {
 #pragma unroll
         for (int x = 0; x < EPL; ++x) {
-            dZ[j * dz_ld + D + lane * EPL + x] = dk[x];
-            dZ[j * dz_ld + 2 * D + lane * EPL + x] = dv[x];
+            dk[x] = fmaf(dphk[x], dphi(k[x]), dk[x]);
+            dv[x] += dvg[x];
         }
+        st_mrow<EPL>(dZ + j * dz_ld + D + lane * EPL, dk);
+        st_mrow<EPL>(dZ + j * dz_ld + 2 * D + lane * EPL, dv);
     }
 }
 
-// db_g = sum_i dt_i in a fixed order: thread k sums i = k, k + 1024, ...; then a tree.
-__global__ void __launch_bounds__(1024) bwd_dbg_kernel(const float *__restrict__ dZ, int64_t N, int64_t dz_ld,
-                                                       int64_t col, float *__restrict__ db_g) {
-    __shared__ float red[1024];
-    float s = 0.f;
-    for (int64_t i = threadIdx.x; i < N; i += 1024) s += dZ[i * dz_ld + col];
-    red[threadIdx.x] = s;
-    __syncthreads();
-    for (int w = 512; w > 0; w >>= 1) {
-        if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) *db_g = red[0];
-}
-
-constexpr int kTile = 64, kTk = 16;
-
-// part[p][a][k] = sum over rows i of range p of X[i][a] * dZ[i][k]  (a < d, k < Dz):
-// 64 x 64 output tiles, 16 rows per shared-memory step, 4 x 4 outputs per thread.
-template <typename T>
-__global__ void __launch_bounds__(256) bwd_dw_kernel(const T *__restrict__ X, const float *__restrict__ dZ,
-                                                     int64_t N, int d, int Dz, int64_t rows_per_part,
-                                                     float *__restrict__ part) {
-    __shared__ float As[kTk][kTile], Bs[kTk][kTile];
-    const int a0 = blockIdx.x * kTile, k0 = blockIdx.y * kTile;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.z) * rows_per_part;
-    const int64_t r1 = std::min<int64_t>(N, r0 + rows_per_part);
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    float acc[4][4] = {};
-    for (int64_t i0 = r0; i0 < r1; i0 += kTk) {
-        for (int l = threadIdx.x; l < kTk * kTile; l += 256) {
-            const int rr = l / kTile, cc = l % kTile;
-            const int64_t i = i0 + rr;
-            As[rr][cc] = (i < r1 && a0 + cc < d) ? ldf<T>(X + i * d + a0 + cc) : 0.f;
-            Bs[rr][cc] = (i < r1 && k0 + cc < Dz) ? dZ[i * Dz + k0 + cc] : 0.f;
-        }
-        __syncthreads();
+// Chunks of heavy source rows, one warp each (layout as bwd_q_chunk_kernel's, over the
+// transposed CSR): the chunk's shares of dk_j | dv_j into part[c][0:D] | part[c][D:2D].
+template <typename T, int EPL>
+__global__ void __launch_bounds__(256) bwd_kv_chunk_kernel(
+    const int2 *__restrict__ chunks, int64_t n_chunks, const int32_t *__restrict__ t_row_ptr,
+    const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
+    const float *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd, int H, int R,
+    float inv_sqrt_r, float *__restrict__ part) {
+    const int lane = threadIdx.x & 31;
+    const int64_t c = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (c >= n_chunks) return;
+    const int2 ch = chunks[c];
+    const int64_t j = ch.x;
+    const int32_t a = ch.y, b = min(t_row_ptr[j + 1], ch.y + kChunk);
+    const int D = H * R;
+    const LaneHead lh(lane, EPL, D, R);
+    float k[EPL], v[EPL], dk[EPL], dv[EPL];
+    ld_row<T, EPL>(KV + j * 2 * D, lane, lh.act, k);
+    ld_row<T, EPL>(KV + j * 2 * D + D, lane, lh.act, v);
 #pragma unroll
-        for (int rr = 0; rr < kTk; ++rr) {
-            float av[4], bv[4];
+    for (int x = 0; x < EPL; ++x) dk[x] = dv[x] = 0.f;
+    kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, lh.act, lh.lph, lh.h, inv_sqrt_r, k, v, a, b, dk, dv);
+    if (lh.act) {
+        float *pc = part + c * 2 * D + lane * EPL;
+        st_mrow<EPL>(pc, dk);
+        st_mrow<EPL>(pc + D, dv);
+    }
+}
+
+// dw_g and db_g over row range p = blockIdx.x (rows [p rpp, (p + 1) rpp)), dt = dZ[:, Kc]:
+// part[p][a][Kc] = sum_i X[i][a] dt_i for the 32 columns a of blockIdx.y, the block's
+// 8 warps taking rows i = r0 + w, r0 + w + 8, ... and their sums added in warp order;
+// blocks with blockIdx.y == 0 also sum dt_i over the range (thread-strided, then a
+// fixed tree) into dbg_part[p].
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_dwg_kernel(const T *__restrict__ X, const float *__restrict__ dZ,
+                                                      int64_t N, int d, int64_t dz_ld, int Kc, int Dc, int64_t rpp,
+                                                      float *__restrict__ part, float *__restrict__ dbg_part) {
+    __shared__ float red[256];
+    const int t = threadIdx.x, w = t >> 5, col = t & 31;
+    const int a = blockIdx.y * 32 + col;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rpp;
+    const int64_t r1 = std::min<int64_t>(N, r0 + rpp);
+    float acc = 0.f;
+    if (a < d) {
+        int64_t i = r0 + w;
+        for (; i + 24 < r1; i += 32) {
+            float xv[4], tv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                av[u] = As[rr][ty * 4 + u];
-                bv[u] = Bs[rr][tx * 4 + u];
+                xv[u] = ldf<T>(X + (i + 8 * u) * d + a);
+                tv[u] = __ldg(dZ + (i + 8 * u) * dz_ld + Kc);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+            for (int u = 0; u < 4; ++u) acc = fmaf(xv[u], tv[u], acc);
         }
+        for (; i < r1; i += 8) acc = fmaf(ldf<T>(X + i * d + a), __ldg(dZ + i * dz_ld + Kc), acc);
+    }
+    red[t] = acc;
+    __syncthreads();
+    if (w == 0 && a < d) {
+        float s = 0.f;
+        for (int ww = 0; ww < 8; ++ww) s += red[ww * 32 + col];
+        part[static_cast<int64_t>(blockIdx.x) * d * Dc + static_cast<int64_t>(a) * Dc + Kc] = s;
+    }
+    if (blockIdx.y != 0) return;                          // block-uniform
+    __syncthreads();
+    float sdt = 0.f;
+    for (int64_t i = r0 + t; i < r1; i += 256) sdt += __ldg(dZ + i * dz_ld + Kc);
+    red[t] = sdt;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (t < o) red[t] += red[t + o];
         __syncthreads();
     }
-    float *out = part + static_cast<int64_t>(blockIdx.z) * d * Dz;
+    if (t == 0) dbg_part[blockIdx.x] = red[0];
+}
+
+// db_g = the row-range sums in range order.
+__global__ void bwd_dbg_kernel(const float *__restrict__ dbg_part, int P, float *__restrict__ db_g) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        float s = 0.f;
+        for (int p = 0; p < P; ++p) s += dbg_part[p];
+        *db_g = s;
+    }
+}
+
+// Register-tiled fp32 GEMM tiles for the weight and input gradients: a 128 x 128 output
+// tile per 256-thread block, 8 reduction steps per shared-memory stage (two stages, the
+// next one loaded into registers while the current one is multiplied), and 8 x 8 outputs
+// per thread at rows {4ty.., 64 + 4ty..} and columns {4tx.., 64 + 4tx..} so that every
+// shared-memory read is a conflict-free float4.
+constexpr int kGT = 128, kGK = 8, kGPad = 4;
+
+__device__ __forceinline__ void gemm_stage(const float (&As)[kGK][kGT + kGPad], const float (&Bs)[kGK][kGT + kGPad],
+                                           int ty, int tx, float (&acc)[8][8]) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int kk = 0; kk < kGK; ++kk) {
+        float av[8], bv[8];
+        const float4 a0 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
+        const float4 a1 = *reinterpret_cast<const float4 *>(&As[kk][64 + ty * 4]);
+        const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
+        const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[kk][64 + tx * 4]);
+        av[0] = a0.x; av[1] = a0.y; av[2] = a0.z; av[3] = a0.w;
+        av[4] = a1.x; av[5] = a1.y; av[6] = a1.z; av[7] = a1.w;
+        bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
+        bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const int a = a0 + ty * 4 + u, k = k0 + tx * 4 + w;
-            if (a < d && k < Dz) out[static_cast<int64_t>(a) * Dz + k] = acc[u][w];
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+    }
+}
+
+
+// part[p][a][k] = sum over rows i of range p of X[i][a] * dZ[i][k]  (a < d, k < Kc = 3D;
+// column Kc is bwd_dwg_kernel's).  Stage: 8 rows of X (scalar loads, 128 columns) and
+// 8 rows of dZ (float4 loads, dz_ld % 4 == 0).
+template <typename T>
+__global__ void __launch_bounds__(256, 2) bwd_dw_kernel(const T *__restrict__ X, const float *__restrict__ dZ,
+                                                        int64_t N, int d, int64_t dz_ld, int Kc, int Dc,
+                                                        int64_t rows_per_part, float *__restrict__ part) {
+    __shared__ __align__(16) float As[2][kGK][kGT + kGPad];
+    __shared__ __align__(16) float Bs[2][kGK][kGT + kGPad];
+    const int a0 = blockIdx.x * kGT, k0 = blockIdx.y * kGT;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.z) * rows_per_part;
+    const int64_t r1 = std::min<int64_t>(N, r0 + rows_per_part);
+    const int t = threadIdx.x, tx = t % 16, ty = t / 16;
+    // loader roles: X column t % 128, rows t / 128 + 2j; dZ row t / 32, float4 (t % 32)
+    const int xa = t % kGT, xr = t / kGT;
+    const int zr = t / 32, zc = (t % 32) * 4;
+    float xa_reg[4];
+    float4 zb_reg;
+    auto load = [&](int64_t i0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t i = i0 + xr + 2 * j;
+            xa_reg[j] = (i < r1 && a0 + xa < d) ? ldf<T>(X + i * d + a0 + xa) : 0.f;
+        }
+        const int64_t i = i0 + zr;
+        const int k = k0 + zc;
+        zb_reg = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < r1 && k < Kc) {
+            zb_reg = *reinterpret_cast<const float4 *>(dZ + i * dz_ld + k);
+            if (k + 1 >= Kc) zb_reg.y = 0.f;
+            if (k + 2 >= Kc) zb_reg.z = 0.f;
+            if (k + 3 >= Kc) zb_reg.w = 0.f;
+        }
+    };
+    auto store = [&](int b) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) As[b][xr + 2 * j][xa] = xa_reg[j];
+        *reinterpret_cast<float4 *>(&Bs[b][zr][zc]) = zb_reg;
+    };
+    float acc[8][8] = {};
+    const int64_t steps = ceil_div(std::max<int64_t>(r1 - r0, 0), kGK);
+    if (steps > 0) {
+        load(r0);
+        store(0);
+        __syncthreads();
+        for (int64_t st = 0; st < steps; ++st) {
+            const bool more = st + 1 < steps;
+            if (more) load(r0 + (st + 1) * kGK);
+            gemm_stage(As[st & 1], Bs[st & 1], ty, tx, acc);
+            if (more) store((st + 1) & 1);
+            __syncthreads();
+        }
+    }
+    float *out = part + static_cast<int64_t>(blockIdx.z) * d * Dc;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const int a = a0 + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
+            const int k = k0 + (w < 4 ? tx * 4 + w : 64 + tx * 4 + w - 4);
+            if (a < d && k < Kc) out[static_cast<int64_t>(a) * Dc + k] = acc[u][w];
         }
 }
 
 // dW_Q | dW_K | dW_V | dw_g from the row-range parts, summed in range order.
-__global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, int d, int D, int Dz,
+__global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, int d, int D, int Dc,
                                      float *__restrict__ dWQ, float *__restrict__ dWK, float *__restrict__ dWV,
                                      float *__restrict__ dwg) {
-    const int64_t total = static_cast<int64_t>(d) * Dz;
+    const int64_t total = static_cast<int64_t>(d) * Dc;
     for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
          o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float acc = 0.f;
         for (int p = 0; p < P; ++p) acc += part[static_cast<int64_t>(p) * total + o];
-        const int a = static_cast<int>(o / Dz), k = static_cast<int>(o % Dz);
+        const int a = static_cast<int>(o / Dc), k = static_cast<int>(o % Dc);
         if (k < D) dWQ[static_cast<int64_t>(a) * D + k] = acc;
         else if (k < 2 * D) dWK[static_cast<int64_t>(a) * D + k - D] = acc;
         else if (k < 3 * D) dWV[static_cast<int64_t>(a) * D + k - 2 * D] = acc;
@@ -553,57 +931,75 @@ __global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, int 
     }
 }
 
-// Column k of [W_Q | W_K | W_V | w_g] at row a.
+// Wall[a][k] = column k of [W_Q | W_K | W_V | w_g] at row a, fp32, zero for Dc <= k < ld.
 template <typename T>
-__device__ __forceinline__ float w_all(const T *WQ, const T *WK, const T *WV, const T *wg, int D, int a, int k) {
-    if (k < D) return ldf<T>(WQ + static_cast<int64_t>(a) * D + k);
-    if (k < 2 * D) return ldf<T>(WK + static_cast<int64_t>(a) * D + k - D);
-    if (k < 3 * D) return ldf<T>(WV + static_cast<int64_t>(a) * D + k - 2 * D);
-    return ldf<T>(wg + a);
+__global__ void bwd_pack_w_kernel(const T *__restrict__ WQ, const T *__restrict__ WK, const T *__restrict__ WV,
+                                  const T *__restrict__ wg, int d, int D, int64_t ld, float *__restrict__ Wall) {
+    const int64_t total = static_cast<int64_t>(d) * ld;
+    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
+         o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t a = o / ld;
+        const int k = static_cast<int>(o % ld);
+        float v = 0.f;
+        if (k < D) v = ldf<T>(WQ + a * D + k);
+        else if (k < 2 * D) v = ldf<T>(WK + a * D + k - D);
+        else if (k < 3 * D) v = ldf<T>(WV + a * D + k - 2 * D);
+        else if (k == 3 * D) v = ldf<T>(wg + a);
+        Wall[o] = v;
+    }
 }
 
-// dX[i][a] = sum_k dZ[i][k] * W_all[a][k]: 64 x 64 tiles of (rows, a), 16 k per step.
-template <typename T>
-__global__ void __launch_bounds__(256) bwd_dx_kernel(const float *__restrict__ dZ, const T *__restrict__ WQ,
-                                                     const T *__restrict__ WK, const T *__restrict__ WV,
-                                                     const T *__restrict__ wg, int64_t N, int d, int D, int Dz,
-                                                     float *__restrict__ dX) {
-    __shared__ float As[kTk][kTile], Bs[kTk][kTile];
-    const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kTile;
-    const int a0 = blockIdx.y * kTile;
-    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < Dz; k0 += kTk) {
-        for (int l = threadIdx.x; l < kTk * kTile; l += 256) {
-            const int kk = l % kTk, rr = l / kTk;
-            const int64_t i = i0 + rr;
-            As[kk][rr] = (i < N && k0 + kk < Dz) ? dZ[i * Dz + k0 + kk] : 0.f;
-            Bs[kk][rr] = (a0 + rr < d && k0 + kk < Dz) ? w_all<T>(WQ, WK, WV, wg, D, a0 + rr, k0 + kk) : 0.f;
+// dX[i][a] = sum_{k < Dc} dZ[i][k] * Wall[a][k]: 128 x 128 tiles of (rows, a).  Stage:
+// 8 columns k of 128 rows of dZ and of Wall (a float4 per thread each, stored transposed).
+__global__ void __launch_bounds__(256, 2) bwd_dx_kernel(const float *__restrict__ dZ, const float *__restrict__ Wall,
+                                                        int64_t N, int d, int64_t ld, int Dc, float *__restrict__ dX) {
+    __shared__ __align__(16) float As[2][kGK][kGT + kGPad];
+    __shared__ __align__(16) float Bs[2][kGK][kGT + kGPad];
+    const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kGT;
+    const int a0 = blockIdx.y * kGT;
+    const int t = threadIdx.x, tx = t % 16, ty = t / 16;
+    const int lr = t / 2, lc = (t % 2) * 4;           // loader: row lr, columns lc .. lc + 3
+    float4 ar, br;
+    auto ld4 = [&](const float *base, int64_t row, int64_t rows, int k) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row < rows && k < Dc) {
+            v = *reinterpret_cast<const float4 *>(base + row * ld + k);
+            if (k + 1 >= Dc) v.y = 0.f;
+            if (k + 2 >= Dc) v.z = 0.f;
+            if (k + 3 >= Dc) v.w = 0.f;
         }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < kTk; ++kk) {
-            float av[4], bv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                av[u] = As[kk][ty * 4 + u];
-                bv[u] = Bs[kk][tx * 4 + u];
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
-        }
+        return v;
+    };
+    auto load = [&](int k0) {
+        ar = ld4(dZ, i0 + lr, N, k0 + lc);
+        br = ld4(Wall, a0 + lr, d, k0 + lc);
+    };
+    auto store = [&](int b) {
+        As[b][lc + 0][lr] = ar.x; As[b][lc + 1][lr] = ar.y; As[b][lc + 2][lr] = ar.z; As[b][lc + 3][lr] = ar.w;
+        Bs[b][lc + 0][lr] = br.x; Bs[b][lc + 1][lr] = br.y; Bs[b][lc + 2][lr] = br.z; Bs[b][lc + 3][lr] = br.w;
+    };
+    float acc[8][8] = {};
+    const int steps = (Dc + kGK - 1) / kGK;
+    load(0);
+    store(0);
+    __syncthreads();
+    for (int st = 0; st < steps; ++st) {
+        const bool more = st + 1 < steps;
+        if (more) load((st + 1) * kGK);
+        gemm_stage(As[st & 1], Bs[st & 1], ty, tx, acc);
+        if (more) store((st + 1) & 1);
         __syncthreads();
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
+        if (i >= N) continue;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const int64_t i = i0 + ty * 4 + u;
-            const int a = a0 + tx * 4 + w;
-            if (i < N && a < d) dX[i * d + a] = acc[u][w];
+        for (int w = 0; w < 8; ++w) {
+            const int a = a0 + (w < 4 ? tx * 4 + w : 64 + tx * 4 + w - 4);
+            if (a < d) dX[i * d + a] = acc[u][w];
         }
+    }
 }
 
 // expand the CSR's rows: tgt[e] = i for e in [row_ptr[i], row_ptr[i+1])
@@ -621,36 +1017,60 @@ int lane_features(int D) {
     return e;
 }
 
-// Both local backward kernels with EPL = lane_features(D): light rows one warp each,
-// heavy rows (more than kHeavyDegree entries) one block each.
+unsigned warp_grid(int64_t n) { return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256))); }
+
+// Both local backward kernels with EPL = lane_features(D): light rows one warp each;
+// heavy rows (more than kHeavyDegree entries) as kChunk-edge chunks, one warp each, whose
+// shares the per-row kernels merge in chunk order.
 template <typename T>
 void launch_local_bwd(Ctx *c, const T *Q, const T *KV, const T *L, float isr, int64_t Dz, cudaStream_t s) {
     const int H = c->H, R = c->r;
-    const unsigned gq = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(c->bw_nq_light * 32, 256)));
-    const unsigned gk = static_cast<unsigned>(std::max<int64_t>(1, ceil_div(c->bw_nk_light * 32, 256)));
+    const size_t D = static_cast<size_t>(c->D);
+    const int64_t nql = c->bw_nq_light, nqh = c->bw_nq_heavy, nkl = c->bw_nk_light, nkh = c->bw_nk_heavy;
+    const int64_t nqc = c->bw_nq_chunks, nkc = c->bw_nk_chunks;
+    const int32_t *qh = c->bw_q_rows + nql, *kh = c->bw_k_rows + nkl;
 #define GLGA_LB(E)                                                                                        \
     case E:                                                                                               \
-        if (c->bw_nq_light)                                                                               \
-            bwd_local_q_kernel<T, E, false><<<gq, 256, 0, s>>>(c->bw_q_rows, c->bw_nq_light, c->row_ptr,   \
+        if (nql)                                                                                          \
+            bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, s>>>(c->bw_q_rows, nql, c->row_ptr,         \
                 c->col_idx, Q, KV, L, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);            \
-        if (c->bw_nq_heavy)                                                                               \
-            bwd_local_q_kernel<T, E, true><<<static_cast<unsigned>(c->bw_nq_heavy), 1024, 0, s>>>(        \
-                c->bw_q_rows + c->bw_nq_light, c->bw_nq_heavy, c->row_ptr, c->col_idx, Q, KV, L, c->bw_dL, \
-                H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);                                            \
-        if (c->bw_nk_light)                                                                               \
-            bwd_local_kv_kernel<T, E, false><<<gk, 256, 0, s>>>(c->bw_k_rows, c->bw_nk_light,             \
-                c->t_row_ptr, c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSz, c->bw_dST, H, R, isr, \
-                c->bw_dZ, Dz);                                                                            \
-        if (c->bw_nk_heavy)                                                                               \
-            bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(c->bw_nk_heavy), 1024, 0, s>>>(       \
-                c->bw_k_rows + c->bw_nk_light, c->bw_nk_heavy, c->t_row_ptr, c->t_col, Q, KV, c->bw_dL,    \
-                c->bw_lse, c->bw_Dd, c->bw_dSz, c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                 \
+        if (nqh) {                                                                                        \
+            bwd_q_chunk_kernel<T, E, 0><<<warp_grid(nqc), 256, 0, s>>>(c->bw_q_chunks, nqc, c->row_ptr,    \
+                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_ml, c->bw_q_part);   \
+            bwd_q_heavy_kernel<T, E, 0><<<static_cast<unsigned>(nqh), kMW * 32, kMW * 64 * 4, s>>>(qh, nqh, \
+                c->bw_q_cptr, c->bw_q_ml,                                                                 \
+                c->bw_q_part, L, c->bw_dL, H, R, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);                      \
+            bwd_q_chunk_kernel<T, E, 1><<<warp_grid(nqc), 256, 0, s>>>(c->bw_q_chunks, nqc, c->row_ptr,    \
+                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_ml, c->bw_q_part);   \
+            bwd_q_heavy_kernel<T, E, 1><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, s>>>(qh, nqh, \
+                c->bw_q_cptr, c->bw_q_ml,                                                                 \
+                c->bw_q_part, L, c->bw_dL, H, R, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);                      \
+        }                                                                                                 \
+        if (nkl)                                                                                          \
+            bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, s>>>(c->bw_k_rows, nkl,             \
+                c->t_row_ptr, c->t_col, nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, \
+                c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                                      \
+        if (nkh) {                                                                                        \
+            bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, s>>>(c->bw_k_chunks, nkc, c->t_row_ptr,    \
+                c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
+            if (kMW * 2 * D * 4 > 48 * 1024)                                                             \
+                cudaFuncSetAttribute(bwd_local_kv_kernel<T, E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                     static_cast<int>(kMW * 2 * D * 4));                                     \
+            bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(nkh), kMW * 32, kMW * 2 * D * 4, s>>>( \
+                kh, nkh, c->t_row_ptr,                                                                    \
+                c->t_col, c->bw_k_cptr, c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc,   \
+                c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                                      \
+        }                                                                                                 \
         break;
     switch (lane_features(c->D)) {
         GLGA_LB(1) GLGA_LB(2) GLGA_LB(4) GLGA_LB(8) GLGA_LB(16) GLGA_LB(32)
         default: break;
     }
 #undef GLGA_LB
+}
+
+int local_bwd_launches(const Ctx *c) {
+    return (c->bw_nq_light > 0) + 4 * (c->bw_nq_heavy > 0) + (c->bw_nk_light > 0) + 2 * (c->bw_nk_heavy > 0);
 }
 
 template <typename T>
@@ -672,7 +1092,8 @@ void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, i
 template <typename T>
 void launch_dsz_bwd(Ctx *c, const T *Q, int64_t rpp, cudaStream_t s) {
     const dim3 grid(static_cast<unsigned>(c->bw_parts), static_cast<unsigned>(c->H));
-    const size_t smem = (32 * c->r + 32 * (c->r + 1)) * sizeof(float);
+    const int R = c->r, tiles = (R / 4) * (R / 4), G = tiles >= 256 ? 1 : 256 / tiles;
+    const size_t smem = (2 * 32 * R + 32 + (G > 1 ? static_cast<size_t>(G) * R * (R + 1) : 0)) * sizeof(float);
 #define GLGA_DZ(RR)                                                                                      \
     case RR:                                                                                             \
         bwd_dsz_partial_kernel<T, RR><<<grid, 256, smem, s>>>(Q, c->bw_dnum, c->bw_dden, c->N, c->H, rpp, \
@@ -685,17 +1106,33 @@ void launch_dsz_bwd(Ctx *c, const T *Q, int64_t rpp, cudaStream_t s) {
 #undef GLGA_DZ
 }
 
-// Light rows first, then heavy ones (more than kHeavyDegree entries), by a CSR's offsets.
-constexpr int64_t kHeavyDegree = 128;
-void split_rows(const std::vector<int32_t> &rp, std::vector<int32_t> &rows, int64_t &n_light, int64_t &n_heavy) {
+// Work lists over one CSR's offsets: light rows (at most kHeavyDegree entries) sorted by
+// degree, longest first (stable), so a block's warps carry similar loads; then heavy rows
+// in index order, each cut into chunks of kChunk entries (chunks[c] = {row, first entry})
+// with chunk_ptr[s] .. chunk_ptr[s + 1] the chunks of heavy row s.
+constexpr int64_t kHeavyDegree = 64;
+struct RowPlan {
+    std::vector<int32_t> rows, chunk_ptr;
+    std::vector<int2> chunks;
+    int64_t n_light = 0, n_heavy = 0;
+};
+void plan_rows(const std::vector<int32_t> &rp, RowPlan &p) {
     const int64_t n = static_cast<int64_t>(rp.size()) - 1;
-    rows.clear();
+    auto deg = [&](int32_t i) { return rp[i + 1] - rp[i]; };
+    p.rows.clear();
+    p.chunks.clear();
+    p.chunk_ptr.assign(1, 0);
     for (int64_t i = 0; i < n; ++i)
-        if (rp[i + 1] - rp[i] <= kHeavyDegree) rows.push_back(static_cast<int32_t>(i));
-    n_light = static_cast<int64_t>(rows.size());
-    for (int64_t i = 0; i < n; ++i)
-        if (rp[i + 1] - rp[i] > kHeavyDegree) rows.push_back(static_cast<int32_t>(i));
-    n_heavy = static_cast<int64_t>(rows.size()) - n_light;
+        if (deg(static_cast<int32_t>(i)) <= kHeavyDegree) p.rows.push_back(static_cast<int32_t>(i));
+    std::stable_sort(p.rows.begin(), p.rows.end(), [&](int32_t x, int32_t y) { return deg(x) > deg(y); });
+    p.n_light = static_cast<int64_t>(p.rows.size());
+    for (int64_t i = 0; i < n; ++i) {
+        if (deg(static_cast<int32_t>(i)) <= kHeavyDegree) continue;
+        p.rows.push_back(static_cast<int32_t>(i));
+        for (int32_t e = rp[i]; e < rp[i + 1]; e += kChunk) p.chunks.push_back(make_int2(static_cast<int>(i), e));
+        p.chunk_ptr.push_back(static_cast<int32_t>(p.chunks.size()));
+    }
+    p.n_heavy = static_cast<int64_t>(p.rows.size()) - p.n_light;
 }
 
 int64_t ceil_parts(int64_t N, int64_t want) { return std::max<int64_t>(1, std::min<int64_t>(want, N)); }
@@ -713,9 +1150,9 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
         return GLGA_ERR_UNSUPPORTED;
     }
     const int64_t N = c->N, E = c->E, D = c->D, H = c->H, R = c->r;
-    c->bw_dz_ld = 3 * D + 1;
+    c->bw_dz_ld = ceil_div(3 * D + 1, 4) * 4;        // rows start on 16 bytes (float4 GEMM loads)
     c->bw_parts = static_cast<int32_t>(ceil_parts(N, c->num_sms));
-    const int64_t tiles = ceil_div(c->d, kTile) * ceil_div(c->bw_dz_ld, kTile);
+    const int64_t tiles = ceil_div(c->d, kGT) * ceil_div(3 * D, kGT);
     c->bw_wparts = static_cast<int32_t>(ceil_parts(N, std::max<int64_t>(1, 2 * c->num_sms / tiles)));
     const size_t f = sizeof(float);
     const int64_t nz = std::max<int64_t>(N, 1);
@@ -734,8 +1171,11 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dSz), static_cast<size_t>(H) * R * (R + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_ST), static_cast<size_t>(H) * R * R * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dST), static_cast<size_t>(H) * R * R * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dSc), static_cast<size_t>(H) * R * (R + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dw_part),
-                   static_cast<size_t>(c->bw_wparts) * c->d * c->bw_dz_ld * f));
+                   static_cast<size_t>(c->bw_wparts) * c->d * (3 * D + 1) * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dbg_part), static_cast<size_t>(c->bw_wparts) * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Wall), static_cast<size_t>(c->d) * c->bw_dz_ld * f));
 #undef BTRY
     if (st != GLGA_OK) return st;
     // transposed CSR: rows by source j, listing the targets i of j's out-edges in order
@@ -759,16 +1199,41 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     }
     if (st != GLGA_OK) return st;
     // row lists of the two local backward kernels: light rows first, then heavy rows
-    std::vector<int32_t> rp(static_cast<size_t>(N) + 1), trp(static_cast<size_t>(N) + 1), qr, kr;
+    std::vector<int32_t> rp(static_cast<size_t>(N) + 1), trp(static_cast<size_t>(N) + 1);
     GLGA_CUDA(cudaMemcpy(rp.data(), c->row_ptr, rp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
     GLGA_CUDA(cudaMemcpy(trp.data(), c->t_row_ptr, trp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
-    split_rows(rp, qr, c->bw_nq_light, c->bw_nq_heavy);
-    split_rows(trp, kr, c->bw_nk_light, c->bw_nk_heavy);
-    st = dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_rows), (qr.size() + 1) * sizeof(int32_t));
-    if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_rows), (kr.size() + 1) * sizeof(int32_t));
+    RowPlan qp, kp;
+    plan_rows(rp, qp);
+    plan_rows(trp, kp);
+    c->bw_nq_light = qp.n_light;
+    c->bw_nq_heavy = qp.n_heavy;
+    c->bw_nk_light = kp.n_light;
+    c->bw_nk_heavy = kp.n_heavy;
+    c->bw_nq_chunks = static_cast<int64_t>(qp.chunks.size());
+    c->bw_nk_chunks = static_cast<int64_t>(kp.chunks.size());
+    const int64_t nqc = std::max<int64_t>(c->bw_nq_chunks, 1), nkc = std::max<int64_t>(c->bw_nk_chunks, 1);
+#define BTRY(x) \
+    if (st == GLGA_OK) st = (x)
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_rows), (qp.rows.size() + 1) * sizeof(int32_t)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_rows), (kp.rows.size() + 1) * sizeof(int32_t)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_cptr), qp.chunk_ptr.size() * sizeof(int32_t)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_cptr), kp.chunk_ptr.size() * sizeof(int32_t)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_chunks), nqc * sizeof(int2)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_chunks), nkc * sizeof(int2)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_ml), nqc * 64 * sizeof(float)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_part), nqc * D * sizeof(float)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_kv_part), nkc * 2 * D * sizeof(float)));
+#undef BTRY
     if (st != GLGA_OK) return st;
-    if (!qr.empty()) GLGA_CUDA(cudaMemcpy(c->bw_q_rows, qr.data(), qr.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
-    if (!kr.empty()) GLGA_CUDA(cudaMemcpy(c->bw_k_rows, kr.data(), kr.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+    auto up = [](void *dst, const void *src, size_t bytes) {
+        return bytes ? cudaMemcpy(dst, src, bytes, cudaMemcpyHostToDevice) : cudaSuccess;
+    };
+    GLGA_CUDA(up(c->bw_q_rows, qp.rows.data(), qp.rows.size() * sizeof(int32_t)));
+    GLGA_CUDA(up(c->bw_k_rows, kp.rows.data(), kp.rows.size() * sizeof(int32_t)));
+    GLGA_CUDA(up(c->bw_q_cptr, qp.chunk_ptr.data(), qp.chunk_ptr.size() * sizeof(int32_t)));
+    GLGA_CUDA(up(c->bw_k_cptr, kp.chunk_ptr.data(), kp.chunk_ptr.size() * sizeof(int32_t)));
+    GLGA_CUDA(up(c->bw_q_chunks, qp.chunks.data(), qp.chunks.size() * sizeof(int2)));
+    GLGA_CUDA(up(c->bw_k_chunks, kp.chunks.data(), kp.chunks.size() * sizeof(int2)));
     return GLGA_OK;
 }
 
@@ -782,27 +1247,34 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
     const int total = H * R * (R + 1);
     const int64_t rpp = ceil_div(std::max<int64_t>(N, 1), c->bw_parts);
     const int64_t wrpp = ceil_div(std::max<int64_t>(N, 1), c->bw_wparts);
-    const int64_t wtotal = static_cast<int64_t>(d) * Dz;
+    const int Dc = 3 * D + 1;                         // columns of dZ in use: dQ | dK | dV | dt
+    const int64_t wtotal = static_cast<int64_t>(d) * Dc;
 #define BWD_LAUNCHES(T)                                                                                   \
     do {                                                                                                  \
         const T *Q = static_cast<const T *>(c->Q);                                                        \
         const T *KV = static_cast<const T *>(c->KV);                                                      \
         const unsigned tgrid = static_cast<unsigned>(ceil_div(static_cast<int64_t>(H) * R * R, 256));    \
         if (N > 0) {                                                                                      \
-            bwd_transpose_heads_kernel<<<tgrid, 256, 0, s>>>(c->Sz, R, H, R, c->bw_ST);                  \
+            bwd_heads_prep_kernel<<<tgrid, 256, 0, s>>>(c->Sz, R, H, R, c->bw_ST, nullptr);              \
             launch_readout_bwd<T>(c, Q, static_cast<const T *>(dY), b_g, eps, Dz, s);                  \
             launch_dsz_bwd<T>(c, Q, rpp, s);                                                              \
         }                                                                                                 \
         bwd_sum_parts_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(                 \
             c->bw_dsz_part, N > 0 ? c->bw_parts : 0, total, c->bw_dSz);                                   \
         if (N > 0) {                                                                                      \
-            bwd_transpose_heads_kernel<<<tgrid, 256, 0, s>>>(c->bw_dSz, R + 1, H, R, c->bw_dST);         \
+            bwd_heads_prep_kernel<<<tgrid, 256, 0, s>>>(c->bw_dSz, R + 1, H, R, c->bw_dST, c->bw_dSc);   \
             launch_local_bwd<T>(c, Q, KV, static_cast<const T *>(c->L), isr, Dz, s);                  \
-            bwd_dw_kernel<T><<<dim3(ceil_div(d, kTile), ceil_div(Dz, kTile), c->bw_wparts), 256, 0, s>>>( \
-                static_cast<const T *>(X), c->bw_dZ, N, d, Dz, wrpp, c->bw_dw_part);                     \
-            bwd_dx_kernel<T><<<dim3(ceil_div(N, kTile), ceil_div(d, kTile)), 256, 0, s>>>(                \
-                c->bw_dZ, static_cast<const T *>(WQ), static_cast<const T *>(WK),                         \
-                static_cast<const T *>(WV), static_cast<const T *>(wg), N, d, D, Dz, dX);                \
+            bwd_pack_w_kernel<T><<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d * Dz, 256), 1024)),   \
+                                   256, 0, s>>>(static_cast<const T *>(WQ), static_cast<const T *>(WK),     \
+                                                static_cast<const T *>(WV), static_cast<const T *>(wg), d, \
+                                                D, Dz, c->bw_Wall);                                         \
+            bwd_dw_kernel<T><<<dim3(ceil_div(d, kGT), ceil_div(3 * D, kGT), c->bw_wparts), 256, 0, s>>>(   \
+                static_cast<const T *>(X), c->bw_dZ, N, d, Dz, 3 * D, Dc, wrpp, c->bw_dw_part);            \
+            bwd_dwg_kernel<T><<<dim3(static_cast<unsigned>(c->bw_wparts), ceil_div(d, 32)), 256, 0, s>>>(   \
+                static_cast<const T *>(X), c->bw_dZ, N, d, Dz, 3 * D, Dc, wrpp, c->bw_dw_part,             \
+                c->bw_dbg_part);                                                                           \
+            bwd_dx_kernel<<<dim3(static_cast<unsigned>(ceil_div(N, kGT)), ceil_div(d, kGT)), 256, 0, s>>>( \
+                c->bw_dZ, c->bw_Wall, N, d, Dz, Dc, dX);                                                   \
         }                                                                                                 \
     } while (0)
     if (c->io == GLGA_F32)
@@ -812,8 +1284,8 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
 #undef BWD_LAUNCHES
     if (N > 0) {
         bwd_dw_reduce_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(wtotal, 256), 4096)), 256, 0, s>>>(
-            c->bw_dw_part, c->bw_wparts, d, D, Dz, dWQ, dWK, dWV, dwg);
-        bwd_dbg_kernel<<<1, 1024, 0, s>>>(c->bw_dZ, N, Dz, 3 * D, db_g);
+            c->bw_dw_part, c->bw_wparts, d, D, Dc, dWQ, dWK, dWV, dwg);
+        bwd_dbg_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, c->bw_wparts, db_g);
     } else {
         GLGA_CUDA(cudaMemsetAsync(dWQ, 0, static_cast<size_t>(d) * D * sizeof(float), s));
         GLGA_CUDA(cudaMemsetAsync(dWK, 0, static_cast<size_t>(d) * D * sizeof(float), s));
@@ -822,7 +1294,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
         GLGA_CUDA(cudaMemsetAsync(db_g, 0, sizeof(float), s));
     }
     GLGA_CUDA(cudaGetLastError());
-    c->launches += N > 0 ? 12 : 1;
+    c->launches += N > 0 ? 11 + local_bwd_launches(c) : 1;
     return GLGA_OK;
 }
 

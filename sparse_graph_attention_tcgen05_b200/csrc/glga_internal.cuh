@@ -132,6 +132,13 @@ struct Ctx {
     float *bw_dZ = nullptr;                           // [N, 3D + 1]: dQ | dK | dV | dt
     float *bw_dsz_part = nullptr, *bw_dSz = nullptr;  // dS | dz partials and sum
     float *bw_ST = nullptr, *bw_dST = nullptr;        // per-head transposes of S and dS
+    float *bw_Wall = nullptr;                         // [d][dz_ld] fp32 [W_Q | W_K | W_V | w_g]
+    float *bw_dSc = nullptr;                          // dS [H][R][R] then dz [H][R]
+    int2 *bw_q_chunks = nullptr, *bw_k_chunks = nullptr;  // heavy rows' edge chunks {row, first}
+    int32_t *bw_q_cptr = nullptr, *bw_k_cptr = nullptr;   // chunk offsets per heavy row
+    int64_t bw_nq_chunks = 0, bw_nk_chunks = 0;
+    float *bw_q_ml = nullptr, *bw_q_part = nullptr, *bw_kv_part = nullptr;  // chunk shares
+    float *bw_dbg_part = nullptr;                     // [wparts] row-range sums of dt
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
     int32_t *bw_q_rows = nullptr, *bw_k_rows = nullptr;   // light rows, then heavy rows
     int64_t bw_nq_light = 0, bw_nq_heavy = 0, bw_nk_light = 0, bw_nk_heavy = 0;
