@@ -168,15 +168,15 @@ struct LaneHead {
 };
 
 // One warp per row i: the gate, readout and blend backward.  Writes dL [N, D],
-// dnum [N, D], dden [N, H], the global part of dQ into dZ [:, 0:D] and dt into dZ [:, 3D]
-// (dg summed over the whole row in lane order).  Sz holds S [H][R][R] then z [H][R];
+// D_i = dL_i . L_i per head into Dd [N, H], dnum [N, D], dden [N, H], the global part of
+// dQ into dZ [:, 0:D] and dt into dZ [:, 3D] (dg summed over the whole row in lane order).  Sz holds S [H][R][R] then z [H][R];
 // ST [H][R][R] is S transposed per head.
 template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_readout_kernel(
     const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t, const float *__restrict__ Sz,
     const float *__restrict__ ST, const T *__restrict__ dY, int64_t N, int H, int R, float b_g, float eps,
-    float *__restrict__ dL, float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ,
-    int64_t dz_ld) {
+    float *__restrict__ dL, float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden,
+    float *__restrict__ dZ, int64_t dz_ld) {
     const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (i >= N) return;                                   // warp-uniform
@@ -200,10 +200,11 @@ __global__ void __launch_bounds__(256) bwd_readout_kernel(
     for (int x = 0; x < EPL; ++x) G[x] = 0.f;
     head_matvec<EPL>(S, R, lh.f0, lh.hb, lh.lph, ph, G);  // num_f = sum_a phi(q_a) S[a][f]
     const float g = 1.f / (1.f + __expf(-(t[i] + b_g)));
-    float dgp = 0.f, dGG = 0.f, gl[EPL], dn[EPL];
+    float dgp = 0.f, dGG = 0.f, dLL = 0.f, gl[EPL], dn[EPL];
 #pragma unroll
     for (int x = 0; x < EPL; ++x) {
         G[x] /= den;
+        dLL = fmaf(g * dy[x], lv[x], dLL);
         dgp = fmaf(dy[x], lv[x] - G[x], dgp);
         const float dG = (1.f - g) * dy[x];
         dGG = fmaf(dG, G[x], dGG);
@@ -216,7 +217,11 @@ __global__ void __launch_bounds__(256) bwd_readout_kernel(
         st_mrow<EPL>(dnum + o, dn);
     }
     const float dd = -head_reduce(dGG, lh.lph) / den;
-    if (lh.act && (lane % lh.lph) == 0) dden[i * H + lh.h] = dd;
+    dLL = head_reduce(dLL, lh.lph);
+    if (lh.act && (lane % lh.lph) == 0) {
+        dden[i * H + lh.h] = dd;
+        Dd[i * H + lh.h] = dLL;
+    }
     float acc[EPL];
 #pragma unroll
     for (int x = 0; x < EPL; ++x) acc[x] = zz[x] * dd;
@@ -348,34 +353,6 @@ __global__ void bwd_sum_parts_kernel(const float *__restrict__ part, int P, int6
 constexpr int kEU = 4;            // edges whose rows are loaded before any is used
 constexpr int kChunk = 32;        // edges per chunk of a heavy row (one warp each)
 
-// Online (max, sum) of exp(s) over the edges [a, b) of target row q (this warp's lanes).
-template <typename T, int EPL>
-__device__ __forceinline__ void q_lse_range(const int32_t *col_idx, const T *KV, int D, int lane, bool act,
-                                            int lph, float inv_sqrt_r, const float (&q)[EPL], int32_t a,
-                                            int32_t b, float &m, float &l) {
-    for (int32_t e = a; e < b; e += kEU) {
-        float k[kEU][EPL];
-#pragma unroll
-        for (int u = 0; u < kEU; ++u) {
-            const bool live = e + u < b;
-            const int64_t jj = live ? col_idx[e + u] : 0;
-            ld_row<T, EPL>(KV + jj * 2 * D, lane, act && live, k[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kEU; ++u) {
-            float s = 0.f;
-#pragma unroll
-            for (int x = 0; x < EPL; ++x) s = fmaf(q[x], k[u][x], s);
-            s = head_reduce(s, lph) * inv_sqrt_r;
-            if (e + u < b) {
-                const float mn = fmaxf(m, s);
-                l = l * __expf(m - mn) + __expf(s - mn);
-                m = mn;
-            }
-        }
-    }
-}
-
 // dq += sum over edges [a, b) of ds_ij k_j (ds already scaled by 1/sqrt(r)).
 template <typename T, int EPL>
 __device__ __forceinline__ void q_grad_range(const int32_t *col_idx, const T *KV, int D, int lane, bool act,
@@ -408,37 +385,27 @@ __device__ __forceinline__ void q_grad_range(const int32_t *col_idx, const T *KV
     }
 }
 
-// Light target rows of the forward CSR (one warp each, the `rows` list): per head the
-// softmax's log-sum-exp and D_i = dL_i . L_i, and the local part of dq_i added into
-// dZ [:, 0:D].
+// Light target rows of the forward CSR (one warp each, the `rows` list): the local part
+// of dq_i added into dZ [:, 0:D].  lse holds the softmax's log-sum-exp per row and head
+// (written by the forward's local kernel), Dd holds D_i = dL_i . L_i (the readout's).
 template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_local_q_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
-    const T *__restrict__ L, const float *__restrict__ dL, int H, int R, float inv_sqrt_r,
-    float *__restrict__ lse, float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
+    const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
     const int lane = threadIdx.x & 31;
     const int64_t slot = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     if (slot >= n_rows) return;                           // warp-uniform
     const int64_t i = rows[slot];
     const int D = H * R;
     const LaneHead lh(lane, EPL, D, R);
-    float q[EPL], dl[EPL], lv[EPL];
+    const int32_t r0 = row_ptr[i], r1 = row_ptr[i + 1];
+    if (r0 == r1) return;                                 // no local term
+    float q[EPL], dl[EPL];
     ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
     ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
-    ld_row<T, EPL>(L + i * D, lane, lh.act, lv);
-    const int32_t r0 = row_ptr[i], r1 = row_ptr[i + 1];
-    float m = -INFINITY, l = 0.f;
-    q_lse_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, r0, r1, m, l);
-    const float ls = r1 > r0 ? m + __logf(l) : 0.f;
-    float dd = 0.f;
-#pragma unroll
-    for (int x = 0; x < EPL; ++x) dd = fmaf(dl[x], lv[x], dd);
-    dd = head_reduce(dd, lh.lph);
-    if (lh.act && (lane % lh.lph) == 0) {
-        lse[i * H + lh.h] = ls;
-        Dd[i * H + lh.h] = dd;
-    }
+    const float ls = __ldg(lse + i * H + lh.h), dd = __ldg(Dd + i * H + lh.h);
     float dq[EPL];
 #pragma unroll
     for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
@@ -454,15 +421,14 @@ __global__ void __launch_bounds__(256) bwd_local_q_kernel(
 }
 
 // Chunks of heavy target rows, one warp each: chunk c covers the edges
-// [chunks[c].y, min(chunks[c].y + kChunk, row end)) of row chunks[c].x.
-//   PHASE 0: the chunk's per-lane online (max, sum) into ml[c][0:32] | ml[c][32:64].
-//   PHASE 1: the chunk's share of dq_i (the row's lse and D_i already final) into part[c][0:D].
-template <typename T, int EPL, int PHASE>
+// [chunks[c].y, min(chunks[c].y + kChunk, row end)) of row chunks[c].x, and writes its
+// share of dq_i into part[c][0:D].
+template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
     const int2 *__restrict__ chunks, int64_t n_chunks, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
     const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
-    const float *__restrict__ Dd, float *__restrict__ ml, float *__restrict__ part) {
+    const float *__restrict__ Dd, float *__restrict__ part) {
     const int lane = threadIdx.x & 31;
     const int64_t c = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     if (c >= n_chunks) return;                            // warp-uniform
@@ -471,22 +437,14 @@ __global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
     const int32_t a = ch.y, b = min(row_ptr[i + 1], ch.y + kChunk);
     const int D = H * R;
     const LaneHead lh(lane, EPL, D, R);
-    float q[EPL];
+    float q[EPL], dl[EPL], dq[EPL];
     ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
-    if constexpr (PHASE == 0) {
-        float m = -INFINITY, l = 0.f;
-        q_lse_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, a, b, m, l);
-        ml[c * 64 + lane] = m;
-        ml[c * 64 + 32 + lane] = l;
-    } else {
-        float dl[EPL], dq[EPL];
-        ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
+    ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
-        const float ls = lse[i * H + lh.h], dd = Dd[i * H + lh.h];
-        q_grad_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, dl, ls, dd, a, b, dq);
-        if (lh.act) st_mrow<EPL>(part + c * D + lane * EPL, dq);
-    }
+    for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+    const float ls = __ldg(lse + i * H + lh.h), dd = __ldg(Dd + i * H + lh.h);
+    q_grad_range<T, EPL>(col_idx, KV, D, lane, lh.act, lh.lph, inv_sqrt_r, q, dl, ls, dd, a, b, dq);
+    if (lh.act) st_mrow<EPL>(part + c * D + lane * EPL, dq);
 }
 
 // Heavy rows are merged by one block of kMW warps each: warp w takes the row's chunks
@@ -494,16 +452,12 @@ __global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
 // warps' results in warp order through shared memory, so the order is fixed.
 constexpr int kMW = 8, kMU = 4;
 
-// Heavy target rows over their chunks [chunk_ptr[s], chunk_ptr[s + 1]):
-//   PHASE 0: merge the chunks' (max, sum) into lse_i, and D_i = dL_i . L_i.
-//   PHASE 1: dq_i = the chunks' shares summed, added into dZ [:, 0:D].
-// Dynamic shared memory: kMW * 64 floats (PHASE 0) or kMW * D floats (PHASE 1).
-template <typename T, int EPL, int PHASE>
+// Heavy target rows over their chunks [chunk_ptr[s], chunk_ptr[s + 1]): dq_i = the
+// chunks' shares summed, added into dZ [:, 0:D].  Dynamic shared memory: kMW * D floats.
+template <int EPL>
 __global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ chunk_ptr,
-    const float *__restrict__ ml, const float *__restrict__ part, const T *__restrict__ L,
-    const float *__restrict__ dL, int H, int R, float *__restrict__ lse, float *__restrict__ Dd,
-    float *__restrict__ dZ, int64_t dz_ld) {
+    const float *__restrict__ part, int H, int R, float *__restrict__ dZ, int64_t dz_ld) {
     extern __shared__ float msm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t slot = blockIdx.x;
@@ -512,90 +466,44 @@ __global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
     const int D = H * R;
     const LaneHead lh(lane, EPL, D, R);
     const int32_t c0 = chunk_ptr[slot], c1 = chunk_ptr[slot + 1];
-    if constexpr (PHASE == 0) {
-        float m = -INFINITY, l = 0.f;
+    float dq[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+    if (lh.act) {
         for (int32_t c = c0 + warp; c < c1; c += kMU * kMW) {
-            float m2[kMU], l2[kMU];
+            float pv[kMU][EPL];
 #pragma unroll
             for (int u = 0; u < kMU; ++u) {
                 const int32_t cc = c + u * kMW;
-                m2[u] = cc < c1 ? ml[static_cast<int64_t>(cc) * 64 + lane] : -INFINITY;
-                l2[u] = cc < c1 ? ml[static_cast<int64_t>(cc) * 64 + 32 + lane] : 0.f;
-            }
+                if (cc < c1) {
+                    ld_mrow<EPL>(part + static_cast<int64_t>(cc) * D + lane * EPL, pv[u]);
+                } else {
 #pragma unroll
-            for (int u = 0; u < kMU; ++u) {
-                const float mn = fmaxf(m, m2[u]);
-                if (mn != -INFINITY) {
-                    l = l * __expf(m - mn) + l2[u] * __expf(m2[u] - mn);
-                    m = mn;
+                    for (int x = 0; x < EPL; ++x) pv[u][x] = 0.f;
                 }
             }
+#pragma unroll
+            for (int u = 0; u < kMU; ++u)
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) dq[x] += pv[u][x];
         }
-        msm[warp * 64 + lane] = m;
-        msm[warp * 64 + 32 + lane] = l;
-        __syncthreads();
-        if (warp != 0) return;
-        m = -INFINITY;
-        l = 0.f;
-        for (int w = 0; w < kMW; ++w) {
-            const float m2 = msm[w * 64 + lane], l2 = msm[w * 64 + 32 + lane];
-            const float mn = fmaxf(m, m2);
-            if (mn != -INFINITY) {
-                l = l * __expf(m - mn) + l2 * __expf(m2 - mn);
-                m = mn;
-            }
-        }
-        float dl[EPL], lv[EPL];
-        ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
-        ld_row<T, EPL>(L + i * D, lane, lh.act, lv);
-        float dd = 0.f;
-#pragma unroll
-        for (int x = 0; x < EPL; ++x) dd = fmaf(dl[x], lv[x], dd);
-        dd = head_reduce(dd, lh.lph);
-        if (lh.act && (lane % lh.lph) == 0) {
-            lse[i * H + lh.h] = m + __logf(l);
-            Dd[i * H + lh.h] = dd;
-        }
-    } else {
-        float dq[EPL];
-#pragma unroll
-        for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
-        if (lh.act) {
-            for (int32_t c = c0 + warp; c < c1; c += kMU * kMW) {
-                float pv[kMU][EPL];
-#pragma unroll
-                for (int u = 0; u < kMU; ++u) {
-                    const int32_t cc = c + u * kMW;
-                    if (cc < c1) {
-                        ld_mrow<EPL>(part + static_cast<int64_t>(cc) * D + lane * EPL, pv[u]);
-                    } else {
-#pragma unroll
-                        for (int x = 0; x < EPL; ++x) pv[u][x] = 0.f;
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < kMU; ++u)
-#pragma unroll
-                    for (int x = 0; x < EPL; ++x) dq[x] += pv[u][x];
-            }
-            st_mrow<EPL>(msm + warp * D + lane * EPL, dq);
-        }
-        __syncthreads();
-        if (warp != 0 || !lh.act) return;
-        float acc[EPL], pv[EPL];
-        float *o = dZ + i * dz_ld + lane * EPL;
-        ld_mrow<EPL, false>(o, acc);                       // the global part of dq_i
-#pragma unroll
-        for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
-        for (int w = 0; w < kMW; ++w) {
-            ld_mrow<EPL, false>(msm + w * D + lane * EPL, pv);
-#pragma unroll
-            for (int x = 0; x < EPL; ++x) dq[x] += pv[x];
-        }
-#pragma unroll
-        for (int x = 0; x < EPL; ++x) acc[x] += dq[x];
-        st_mrow<EPL>(o, acc);
+        st_mrow<EPL>(msm + warp * D + lane * EPL, dq);
     }
+    __syncthreads();
+    if (warp != 0 || !lh.act) return;
+    float acc[EPL], pv[EPL];
+    float *o = dZ + i * dz_ld + lane * EPL;
+    ld_mrow<EPL, false>(o, acc);                           // the global part of dq_i
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
+    for (int w = 0; w < kMW; ++w) {
+        ld_mrow<EPL, false>(msm + w * D + lane * EPL, pv);
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) dq[x] += pv[x];
+    }
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) acc[x] += dq[x];
+    st_mrow<EPL>(o, acc);
 }
 
 // dk, dv += the terms of targets [a, b) of source row j (this warp's lanes).
@@ -1021,9 +929,11 @@ unsigned warp_grid(int64_t n) { return static_cast<unsigned>(std::max<int64_t>(1
 
 // Both local backward kernels with EPL = lane_features(D): light rows one warp each;
 // heavy rows (more than kHeavyDegree entries) as kChunk-edge chunks, one warp each, whose
-// shares the per-row kernels merge in chunk order.
+// shares the per-row kernels merge in chunk order.  The target-side (dq) kernels go to
+// stream sq and the source-side (dk, dv) kernels to sk: they read the same inputs and
+// write disjoint columns of dZ.
 template <typename T>
-void launch_local_bwd(Ctx *c, const T *Q, const T *KV, const T *L, float isr, int64_t Dz, cudaStream_t s) {
+void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cudaStream_t sq, cudaStream_t sk) {
     const int H = c->H, R = c->r;
     const size_t D = static_cast<size_t>(c->D);
     const int64_t nql = c->bw_nq_light, nqh = c->bw_nq_heavy, nkl = c->bw_nk_light, nkh = c->bw_nk_heavy;
@@ -1031,35 +941,28 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, const T *L, float isr, in
     const int32_t *qh = c->bw_q_rows + nql, *kh = c->bw_k_rows + nkl;
 #define GLGA_LB(E)                                                                                        \
     case E:                                                                                               \
-        if (nql)                                                                                          \
-            bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, s>>>(c->bw_q_rows, nql, c->row_ptr,         \
-                c->col_idx, Q, KV, L, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);            \
-        if (nqh) {                                                                                        \
-            bwd_q_chunk_kernel<T, E, 0><<<warp_grid(nqc), 256, 0, s>>>(c->bw_q_chunks, nqc, c->row_ptr,    \
-                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_ml, c->bw_q_part);   \
-            bwd_q_heavy_kernel<T, E, 0><<<static_cast<unsigned>(nqh), kMW * 32, kMW * 64 * 4, s>>>(qh, nqh, \
-                c->bw_q_cptr, c->bw_q_ml,                                                                 \
-                c->bw_q_part, L, c->bw_dL, H, R, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);                      \
-            bwd_q_chunk_kernel<T, E, 1><<<warp_grid(nqc), 256, 0, s>>>(c->bw_q_chunks, nqc, c->row_ptr,    \
-                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_ml, c->bw_q_part);   \
-            bwd_q_heavy_kernel<T, E, 1><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, s>>>(qh, nqh, \
-                c->bw_q_cptr, c->bw_q_ml,                                                                 \
-                c->bw_q_part, L, c->bw_dL, H, R, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);                      \
-        }                                                                                                 \
         if (nkl)                                                                                          \
-            bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, s>>>(c->bw_k_rows, nkl,             \
+            bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl,            \
                 c->t_row_ptr, c->t_col, nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, \
                 c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                                      \
         if (nkh) {                                                                                        \
-            bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, s>>>(c->bw_k_chunks, nkc, c->t_row_ptr,    \
+            bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, sk>>>(c->bw_k_chunks, nkc, c->t_row_ptr,   \
                 c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
             if (kMW * 2 * D * 4 > 48 * 1024)                                                             \
                 cudaFuncSetAttribute(bwd_local_kv_kernel<T, E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                      static_cast<int>(kMW * 2 * D * 4));                                     \
-            bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(nkh), kMW * 32, kMW * 2 * D * 4, s>>>( \
-                kh, nkh, c->t_row_ptr,                                                                    \
-                c->t_col, c->bw_k_cptr, c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc,   \
-                c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                                      \
+            bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(nkh), kMW * 32, kMW * 2 * D * 4, sk>>>( \
+                kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr, c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse,  \
+                c->bw_Dd, c->bw_dSc, c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                 \
+        }                                                                                                 \
+        if (nql)                                                                                          \
+            bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr,        \
+                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);               \
+        if (nqh) {                                                                                        \
+            bwd_q_chunk_kernel<T, E><<<warp_grid(nqc), 256, 0, sq>>>(c->bw_q_chunks, nqc, c->row_ptr,      \
+                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);               \
+            bwd_q_heavy_kernel<E><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, sq>>>(qh, nqh,      \
+                c->bw_q_cptr, c->bw_q_part, H, R, c->bw_dZ, Dz);                                          \
         }                                                                                                 \
         break;
     switch (lane_features(c->D)) {
@@ -1070,7 +973,7 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, const T *L, float isr, in
 }
 
 int local_bwd_launches(const Ctx *c) {
-    return (c->bw_nq_light > 0) + 4 * (c->bw_nq_heavy > 0) + (c->bw_nk_light > 0) + 2 * (c->bw_nk_heavy > 0);
+    return (c->bw_nq_light > 0) + 2 * (c->bw_nq_heavy > 0) + (c->bw_nk_light > 0) + 2 * (c->bw_nk_heavy > 0);
 }
 
 template <typename T>
@@ -1079,7 +982,8 @@ void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, i
 #define GLGA_RB(E)                                                                                       \
     case E:                                                                                              \
         bwd_readout_kernel<T, E><<<grid, 256, 0, s>>>(Q, static_cast<const T *>(c->L), c->t, c->Sz, c->bw_ST, dY, \
-                                                      c->N, c->H, c->r, b_g, eps, c->bw_dL, c->bw_dnum,  \
+                                                      c->N, c->H, c->r, b_g, eps, c->bw_dL, c->bw_Dd,    \
+                                                      c->bw_dnum,                                        \
                                                       c->bw_dden, c->bw_dZ, Dz);                         \
         break;
     switch (lane_features(c->D)) {
@@ -1160,6 +1064,12 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
 #define BTRY(x) \
     if (st == GLGA_OK) st = (x)
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->t_row_ptr), (N + 1) * sizeof(int32_t)));
+    if (st == GLGA_OK) {
+        cudaError_t e = cudaStreamCreateWithFlags(&c->bw_side, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->bw_ev_fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->bw_ev_join, cudaEventDisableTiming);
+        if (e != cudaSuccess) st = cuda_fail(e, "backward side stream");
+    }
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->t_col), std::max<int64_t>(E, 1) * sizeof(int32_t)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dL), nz * D * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dnum), nz * D * f));
@@ -1220,7 +1130,6 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_cptr), kp.chunk_ptr.size() * sizeof(int32_t)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_chunks), nqc * sizeof(int2)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_k_chunks), nkc * sizeof(int2)));
-    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_ml), nqc * 64 * sizeof(float)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_q_part), nqc * D * sizeof(float)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_kv_part), nkc * 2 * D * sizeof(float)));
 #undef BTRY
@@ -1257,13 +1166,17 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
         if (N > 0) {                                                                                      \
             bwd_heads_prep_kernel<<<tgrid, 256, 0, s>>>(c->Sz, R, H, R, c->bw_ST, nullptr);              \
             launch_readout_bwd<T>(c, Q, static_cast<const T *>(dY), b_g, eps, Dz, s);                  \
-            launch_dsz_bwd<T>(c, Q, rpp, s);                                                              \
-        }                                                                                                 \
-        bwd_sum_parts_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, s>>>(                 \
-            c->bw_dsz_part, N > 0 ? c->bw_parts : 0, total, c->bw_dSz);                                   \
-        if (N > 0) {                                                                                      \
-            bwd_heads_prep_kernel<<<tgrid, 256, 0, s>>>(c->bw_dSz, R + 1, H, R, c->bw_dST, c->bw_dSc);   \
-            launch_local_bwd<T>(c, Q, KV, static_cast<const T *>(c->L), isr, Dz, s);                  \
+            /* fork: the dS | dz chain and the source-side kernels on the side stream */                 \
+            GLGA_CUDA(cudaEventRecord(c->bw_ev_fork, s));                                                 \
+            GLGA_CUDA(cudaStreamWaitEvent(c->bw_side, c->bw_ev_fork, 0));                                 \
+            launch_dsz_bwd<T>(c, Q, rpp, c->bw_side);                                                     \
+            bwd_sum_parts_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, c->bw_side>>>(   \
+                c->bw_dsz_part, c->bw_parts, total, c->bw_dSz);                                           \
+            bwd_heads_prep_kernel<<<tgrid, 256, 0, c->bw_side>>>(c->bw_dSz, R + 1, H, R, c->bw_dST,      \
+                                                                c->bw_dSc);                               \
+            launch_local_bwd<T>(c, Q, KV, isr, Dz, s, c->bw_side);                                        \
+            GLGA_CUDA(cudaEventRecord(c->bw_ev_join, c->bw_side));                                        \
+            GLGA_CUDA(cudaStreamWaitEvent(s, c->bw_ev_join, 0));                                          \
             bwd_pack_w_kernel<T><<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d * Dz, 256), 1024)),   \
                                    256, 0, s>>>(static_cast<const T *>(WQ), static_cast<const T *>(WK),     \
                                                 static_cast<const T *>(WV), static_cast<const T *>(wg), d, \
@@ -1293,8 +1206,9 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
         GLGA_CUDA(cudaMemsetAsync(dwg, 0, static_cast<size_t>(d) * sizeof(float), s));
         GLGA_CUDA(cudaMemsetAsync(db_g, 0, sizeof(float), s));
     }
+    // (N == 0: no dS | dz to sum, and every gradient is zero)
     GLGA_CUDA(cudaGetLastError());
-    c->launches += N > 0 ? 11 + local_bwd_launches(c) : 1;
+    c->launches += N > 0 ? 11 + local_bwd_launches(c) : 0;
     return GLGA_OK;
 }
 

@@ -137,7 +137,9 @@ struct Ctx {
     int2 *bw_q_chunks = nullptr, *bw_k_chunks = nullptr;  // heavy rows' edge chunks {row, first}
     int32_t *bw_q_cptr = nullptr, *bw_k_cptr = nullptr;   // chunk offsets per heavy row
     int64_t bw_nq_chunks = 0, bw_nk_chunks = 0;
-    float *bw_q_ml = nullptr, *bw_q_part = nullptr, *bw_kv_part = nullptr;  // chunk shares
+    float *bw_q_part = nullptr, *bw_kv_part = nullptr;  // chunk shares
+    cudaStream_t bw_side = nullptr;                   // second stream of the backward (source side)
+    cudaEvent_t bw_ev_fork = nullptr, bw_ev_join = nullptr;
     float *bw_dbg_part = nullptr;                     // [wparts] row-range sums of dt
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
     int32_t *bw_q_rows = nullptr, *bw_k_rows = nullptr;   // light rows, then heavy rows

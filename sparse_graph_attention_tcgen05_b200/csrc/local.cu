@@ -105,6 +105,7 @@ struct LocalParams {
     float *part;         // per chunk: m[H] l[H] acc[D]
     unsigned *ticket;
     void *L;             // io [N, D] local-branch output
+    float *lse;          // [N, H] log-sum-exp of the row's scores for the backward pass, or null
     int32_t D, r, H, nvec, lpe, epw, lph;
     float score_scale;   // log2(e) / sqrt(r)
     int32_t N;           // source nodes: bound of column indices (debug checks)
@@ -358,8 +359,26 @@ __device__ __forceinline__ void scale_q(const LocalParams &p, const uint4 (&qr)[
     }
 }
 
+// lse_i = ln sum_j exp(s_ij) per head, ln 2 (m + log2 l) since the state keeps base-2
+// scores (0 for a row without edges), from the vector holding the head's first features.
+// Compiled in only for the LSE instantiations (contexts made for the backward pass), so
+// the plain forward's code is untouched.
+template <typename T, int VPL, bool J, bool LSE>
+__device__ __forceinline__ void store_lse(const LocalParams &p, int64_t row, const State<T, VPL> &st,
+                                          const Lane &ln, bool mine) {
+    if constexpr (!LSE) return;
+    constexpr int VE = Io<T>::VE;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const int vid = vid_of<J, VPL>(v, ln.li);
+        if (mine && vid < p.nvec && (vid * VE) % p.r == 0)
+            p.lse[row * p.H + vid * VE / p.r] =
+                st.l[v] > 0.f ? 0.69314718055994531f * (st.m[v] + __log2f(st.l[v])) : 0.f;
+    }
+}
+
 // L_i = acc / l per head (0 for a row without edges); stores L[row] from `slot`'s lanes.
-template <typename T, int VPL, bool J>
+template <typename T, int VPL, bool J, bool LSE>
 __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, const State<T, VPL> &st,
                                            const Lane &ln, int slot) {
     constexpr int VE = Io<T>::VE;
@@ -373,6 +392,7 @@ __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, co
         for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l;
         if (vid < p.nvec && ln.slot == slot) Lout[vid] = Io<T>::pack(y);
     }
+    store_lse<T, VPL, J, LSE>(p, row, st, ln, ln.slot == slot);
 }
 
 template <typename T, int VPL>
@@ -417,7 +437,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const float (&
     }
 }
 
-template <typename T, int VPL, int U, bool DBG, bool J>
+template <typename T, int VPL, int U, bool DBG, bool J, bool LSE>
 __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(const LocalParams p) {
     constexpr int VE = Io<T>::VE;
     __shared__ BlockScratch<T, VPL> sh;
@@ -485,7 +505,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                         st.merge(v, __ldcg(src + h), __ldcg(src + p.H + h), a2);
                     }
                 }
-                finish_row<T, VPL, J>(p, row, st, ln, 0);
+                finish_row<T, VPL, J, LSE>(p, row, st, ln, 0);
             }
         }
         return;
@@ -498,7 +518,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         load_q_raw<T, VPL, J>(p, row, ln, true, qr);
         scale_q<T, VPL>(p, qr, q);
         block_edges<T, VPL, U, DBG, J>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
-        if (warp == 0) finish_row<T, VPL, J>(p, row, st, ln, 0);
+        if (warp == 0) finish_row<T, VPL, J, LSE>(p, row, st, ln, 0);
         return;
     }
     bid -= p.n_cta;
@@ -554,6 +574,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                 for (int e = 0; e < VEc; ++e) y[e] = st.acc[v][e] * inv_l;
                 if (vid < p.nvec) Lout[vid] = Io<T>::pack(y);
             }
+            store_lse<T, VPL, J, LSE>(p, row_c, st, ln, true);
         }
     }
 }
@@ -562,10 +583,14 @@ template <typename T, int VPL, int U, bool J = false>
 glga_status launch_local(Ctx *c, const LocalParams &p, cudaStream_t s) {
     const int64_t blocks = p.n_chunks + p.n_cta + p.task_blocks;
     if (blocks == 0) return GLGA_OK;
-    if (c->opts.debug_checks)
-        local_kernel<T, VPL, U, true, J><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
-    else
-        local_kernel<T, VPL, U, false, J><<<static_cast<unsigned>(blocks), kLocalThreads, 0, s>>>(p);
+    const unsigned g = static_cast<unsigned>(blocks);
+    if (c->opts.debug_checks) {
+        if (p.lse) local_kernel<T, VPL, U, true, J, true><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, VPL, U, true, J, false><<<g, kLocalThreads, 0, s>>>(p);
+    } else {
+        if (p.lse) local_kernel<T, VPL, U, false, J, true><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, VPL, U, false, J, false><<<g, kLocalThreads, 0, s>>>(p);
+    }
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -638,6 +663,7 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.part = c->chunk_part;
     p.ticket = c->chunk_ticket;
     p.L = c->L;
+    p.lse = c->opts.backward ? c->bw_lse : nullptr;
     p.D = c->D;
     p.r = c->r;
     p.H = c->H;
