@@ -73,9 +73,11 @@ typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
  * debugging only.
  * debug_fail_alloc = n > 0 makes the n-th device allocation of glga_create fail with
  * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.
- * backward != 0 allocates the workspaces of glga_backward at create (a transposed CSR
- * and fp32 buffers of about N*(6*H*r + 4*H + 1) floats); whole-graph, one-segment
- * contexts with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).                   */
+ * backward != 0 allocates the workspaces of glga_backward at create (a transposed CSR,
+ * chunk lists of the rows with more than 64 entries, a second stream and fp32 buffers of
+ * about N*(6*H*r + 4*H + 1) floats); glga_forward on such a context also stores each
+ * row's softmax log-sum-exp per head for the backward.  Whole-graph, one-segment contexts
+ * with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).                             */
 typedef struct {
     int32_t warp_max_degree;
     int32_t chunk_edges;
@@ -196,8 +198,10 @@ GLGA_API glga_status glga_forward_end(glga_ctx *ctx, const float *partials, int3
  *   dX (device) float [N, d]; dW_Q, dW_K, dW_V (device) float [d, H*r]; dw_g (device)
  *   float [d]; db_g (device) float [1] -- all written.
  * Needs glga_options.backward at create.  Every sum runs in a fixed order (the source
- * side walks a transposed CSR; no atomics), so repeated calls give identical bits.
- * Stream-ordered, no host synchronisation.                                            */
+ * side walks a transposed CSR, rows with more than 64 entries are cut into 32-entry
+ * chunks summed in chunk order; no atomics), so repeated calls give identical bits.
+ * Stream-ordered, no host synchronisation: the source-side kernels run on a stream of the
+ * context forked from and joined back into `stream` by events (capture-safe).          */
 GLGA_API glga_status glga_backward(glga_ctx *ctx, const void *X, const void *W_Q, const void *W_K,
                         const void *W_V, const void *w_g, float b_g, float eps, const void *dY,
                         float *dX, float *dW_Q, float *dW_K, float *dW_V, float *dw_g, float *db_g,
