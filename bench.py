@@ -253,7 +253,8 @@ def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
     assert layer.last_device_error() == 0
     t = float(np.mean(ms))
     return {"ms": t, "edge_heads_per_s": w.E * w.H / (t * 1e-3), "steps": steps,
-            "kernels": "CUDA-core (SIMT) kernels, fp32 arithmetic"}
+            "kernels": ("CUDA-core (SIMT) kernels, fp32 arithmetic"
+                        + ("; dW and dX as cuBLAS GEMMs on the TF32 tensor cores" if w.io == "bf16" else ""))}
 
 
 def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0):

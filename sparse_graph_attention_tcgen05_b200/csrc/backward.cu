@@ -18,10 +18,14 @@
 // walk a transposed CSR built at create, so every sum has a fixed order and there are no
 // atomics (two runs give identical bits).  Plain CUDA-core kernels with fp32 arithmetic
 // (one thread per row and head, tiled GEMMs for the projections); gradients are fp32.
+#include <dlfcn.h>
+
 #include <algorithm>
 #include <cmath>
 #include <type_traits>
 #include <vector>
+
+#include <cublas_v2.h>   // types and enums only: the library is opened at run time
 
 #include "glga_internal.cuh"
 
@@ -822,16 +826,22 @@ __global__ void __launch_bounds__(256, 2) bwd_dw_kernel(const T *__restrict__ X,
         }
 }
 
-// dW_Q | dW_K | dW_V | dw_g from the row-range parts, summed in range order.
-__global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, int d, int D, int Dc,
-                                     float *__restrict__ dWQ, float *__restrict__ dWK, float *__restrict__ dWV,
-                                     float *__restrict__ dwg) {
+// dW_Q | dW_K | dW_V | dw_g from the row-range parts, summed in range order; when w3 is
+// given (one GEMM wrote the columns k < 3D whole, as w3[a][k] with row stride 3D) those
+// columns are copied from it and only column 3D comes from the parts.
+__global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, const float *__restrict__ w3, int d,
+                                     int D, int Dc, float *__restrict__ dWQ, float *__restrict__ dWK,
+                                     float *__restrict__ dWV, float *__restrict__ dwg) {
     const int64_t total = static_cast<int64_t>(d) * Dc;
     for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
          o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float acc = 0.f;
-        for (int p = 0; p < P; ++p) acc += part[static_cast<int64_t>(p) * total + o];
         const int a = static_cast<int>(o / Dc), k = static_cast<int>(o % Dc);
+        float acc = 0.f;
+        if (w3 && k < 3 * D) {
+            acc = w3[static_cast<int64_t>(a) * 3 * D + k];
+        } else {
+            for (int p = 0; p < P; ++p) acc += part[static_cast<int64_t>(p) * total + o];
+        }
         if (k < D) dWQ[static_cast<int64_t>(a) * D + k] = acc;
         else if (k < 2 * D) dWK[static_cast<int64_t>(a) * D + k - D] = acc;
         else if (k < 3 * D) dWV[static_cast<int64_t>(a) * D + k - 2 * D] = acc;
@@ -923,6 +933,47 @@ int lane_features(int D) {
     int e = 1;
     while (32 * e < D) e <<= 1;
     return e;
+}
+
+// cuBLAS, opened on first use by a context made for the backward pass (so the forward
+// never depends on it).  dW = X^T [dQ | dK | dV] and dX = dZ W^T are plain dense GEMMs;
+// for bf16 layers they run there on the TF32 tensor cores (fp32 operands rounded to
+// 10-bit mantissas, fp32 accumulation), for fp32 layers on the exact-fp32 SIMT kernels.
+struct CublasApi {
+    bool ok = false;
+    cublasStatus_t (*create)(cublasHandle_t *) = nullptr;
+    cublasStatus_t (*destroy)(cublasHandle_t) = nullptr;
+    cublasStatus_t (*set_stream)(cublasHandle_t, cudaStream_t) = nullptr;
+    cublasStatus_t (*set_workspace)(cublasHandle_t, void *, size_t) = nullptr;
+    cublasStatus_t (*gemm_ex)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int, const void *,
+                              const void *, cudaDataType, int, const void *, cudaDataType, int, const void *,
+                              void *, cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t) = nullptr;
+};
+
+const CublasApi &cublas_api() {
+    static const CublasApi api = [] {
+        CublasApi a;
+        void *lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
+        if (!lib) lib = dlopen("/usr/local/cuda/lib64/libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
+        if (!lib) return a;
+        a.create = reinterpret_cast<decltype(a.create)>(dlsym(lib, "cublasCreate_v2"));
+        a.destroy = reinterpret_cast<decltype(a.destroy)>(dlsym(lib, "cublasDestroy_v2"));
+        a.set_stream = reinterpret_cast<decltype(a.set_stream)>(dlsym(lib, "cublasSetStream_v2"));
+        a.set_workspace = reinterpret_cast<decltype(a.set_workspace)>(dlsym(lib, "cublasSetWorkspace_v2"));
+        a.gemm_ex = reinterpret_cast<decltype(a.gemm_ex)>(dlsym(lib, "cublasGemmEx"));
+        a.ok = a.create && a.destroy && a.set_stream && a.set_workspace && a.gemm_ex;
+        return a;
+    }();
+    return api;
+}
+
+constexpr size_t kCublasWorkspace = size_t(32) << 20;
+
+// Xf = X as fp32 (the TF32 GEMM takes both operands in fp32).
+__global__ void bwd_x_to_f32_kernel(const __nv_bfloat16 *__restrict__ X, int64_t n, float *__restrict__ Xf) {
+    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < n;
+         o += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        Xf[o] = __bfloat162float(X[o]);
 }
 
 unsigned warp_grid(int64_t n) { return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256))); }
@@ -1041,7 +1092,40 @@ void plan_rows(const std::vector<int32_t> &rp, RowPlan &p) {
 
 int64_t ceil_parts(int64_t N, int64_t want) { return std::max<int64_t>(1, std::min<int64_t>(want, N)); }
 
+// The two GEMMs on cuBLAS (column-major view of the row-major buffers; every leading
+// dimension a multiple of 4 floats):
+//   dW3[a][k] (k < 3D, row stride 3D) = sum_i dZ[i][k] Xf[i][a]:
+//     C [3D x d], ldc 3D = A [3D x N] (dZ^T, lda dz_ld) * B^T (B = Xf^T [d x N], ldb d)
+//   dX [N x d] = dZ Wall^T over all dz_ld columns (the padding columns of dZ and Wall are
+//     zero):  C [d x N], ldc d = A^T (A = Wall^T [dz_ld x d]) * B (B = dZ^T [dz_ld x N])
+glga_status cublas_gemms(Ctx *c, float *dX, cudaStream_t s) {
+    const CublasApi &api = cublas_api();
+    cublasHandle_t h = static_cast<cublasHandle_t>(c->bw_cublas);
+    const int N = static_cast<int>(c->N), d = c->d, D = c->D;
+    const int ld = static_cast<int>(c->bw_dz_ld);
+    const float one = 1.f, zero = 0.f;
+    cublasStatus_t e = api.set_stream(h, s);
+    if (e == CUBLAS_STATUS_SUCCESS)
+        e = api.gemm_ex(h, CUBLAS_OP_N, CUBLAS_OP_T, 3 * D, d, N, &one, c->bw_dZ, CUDA_R_32F, ld, c->bw_Xf,
+                        CUDA_R_32F, d, &zero, c->bw_dW3, CUDA_R_32F, 3 * D, CUBLAS_COMPUTE_32F_FAST_TF32,
+                        CUBLAS_GEMM_DEFAULT);
+    if (e == CUBLAS_STATUS_SUCCESS)
+        e = api.gemm_ex(h, CUBLAS_OP_T, CUBLAS_OP_N, d, N, ld, &one, c->bw_Wall, CUDA_R_32F, ld, c->bw_dZ,
+                        CUDA_R_32F, ld, &zero, dX, CUDA_R_32F, d, CUBLAS_COMPUTE_32F_FAST_TF32,
+                        CUBLAS_GEMM_DEFAULT);
+    if (e != CUBLAS_STATUS_SUCCESS) {
+        set_error("glga_backward: cuBLAS GEMM failed (status %d)", static_cast<int>(e));
+        return GLGA_ERR_CUDA;
+    }
+    return GLGA_OK;
+}
+
 }  // namespace
+
+void backward_release(Ctx *c) {
+    if (c->bw_cublas) cublas_api().destroy(static_cast<cublasHandle_t>(c->bw_cublas));
+    c->bw_cublas = nullptr;
+}
 
 glga_status backward_setup(Ctx *c, cudaStream_t s) {
     if (!c->opts.backward) return GLGA_OK;
@@ -1086,8 +1170,23 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
                    static_cast<size_t>(c->bw_wparts) * c->d * (3 * D + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dbg_part), static_cast<size_t>(c->bw_wparts) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Wall), static_cast<size_t>(c->d) * c->bw_dz_ld * f));
+    if (st == GLGA_OK && c->io == GLGA_BF16 && N > 0 && N <= INT32_MAX && cublas_api().ok) {
+        cublasHandle_t h = nullptr;
+        if (cublas_api().create(&h) == CUBLAS_STATUS_SUCCESS) {
+            c->bw_cublas = h;
+            BTRY(dev_alloc(c, &c->bw_cublas_ws, kCublasWorkspace));
+            BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Xf), static_cast<size_t>(N) * c->d * f));
+            BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dW3), static_cast<size_t>(c->d) * 3 * D * f));
+            if (st == GLGA_OK && cublas_api().set_workspace(h, c->bw_cublas_ws, kCublasWorkspace) != CUBLAS_STATUS_SUCCESS) {
+                set_error("glga_create: cuBLAS workspace");
+                st = GLGA_ERR_CUDA;
+            }
+        }
+    }
 #undef BTRY
     if (st != GLGA_OK) return st;
+    // dZ's padding columns (3D + 1 .. dz_ld - 1) are never written: zero them once
+    GLGA_CUDA(cudaMemset(c->bw_dZ, 0, static_cast<size_t>(nz) * c->bw_dz_ld * f));
     // transposed CSR: rows by source j, listing the targets i of j's out-edges in order
     int32_t *tgt = nullptr;
     if (E > 0) {
@@ -1177,6 +1276,20 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
             launch_local_bwd<T>(c, Q, KV, isr, Dz, s, c->bw_side);                                        \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_join, c->bw_side));                                        \
             GLGA_CUDA(cudaStreamWaitEvent(s, c->bw_ev_join, 0));                                          \
+            if (c->bw_cublas) {                                                                           \
+                bwd_pack_w_kernel<T><<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d * Dz, 256), 1024)), \
+                                       256, 0, s>>>(static_cast<const T *>(WQ), static_cast<const T *>(WK), \
+                                                    static_cast<const T *>(WV), static_cast<const T *>(wg), \
+                                                    d, D, Dz, c->bw_Wall);                                  \
+                bwd_x_to_f32_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(N * d, 256), 4096)),  \
+                                      256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), N * d, c->bw_Xf); \
+                const glga_status gs = cublas_gemms(c, dX, s);                                            \
+                if (gs != GLGA_OK) return gs;                                                             \
+                bwd_dwg_kernel<T><<<dim3(static_cast<unsigned>(c->bw_wparts), ceil_div(d, 32)), 256, 0, s>>>( \
+                    static_cast<const T *>(X), c->bw_dZ, N, d, Dz, 3 * D, Dc, wrpp, c->bw_dw_part,         \
+                    c->bw_dbg_part);                                                                       \
+                break;                                                                                    \
+            }                                                                                             \
             bwd_pack_w_kernel<T><<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d * Dz, 256), 1024)),   \
                                    256, 0, s>>>(static_cast<const T *>(WQ), static_cast<const T *>(WK),     \
                                                 static_cast<const T *>(WV), static_cast<const T *>(wg), d, \
@@ -1197,7 +1310,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
 #undef BWD_LAUNCHES
     if (N > 0) {
         bwd_dw_reduce_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(wtotal, 256), 4096)), 256, 0, s>>>(
-            c->bw_dw_part, c->bw_wparts, d, D, Dc, dWQ, dWK, dWV, dwg);
+            c->bw_dw_part, c->bw_wparts, c->bw_cublas ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
         bwd_dbg_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, c->bw_wparts, db_g);
     } else {
         GLGA_CUDA(cudaMemsetAsync(dWQ, 0, static_cast<size_t>(d) * D * sizeof(float), s));
@@ -1208,7 +1321,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
     }
     // (N == 0: no dS | dz to sum, and every gradient is zero)
     GLGA_CUDA(cudaGetLastError());
-    c->launches += N > 0 ? 11 + local_bwd_launches(c) : 0;
+    c->launches += N > 0 ? (c->bw_cublas ? 10 : 11) + local_bwd_launches(c) : 0;
     return GLGA_OK;
 }
 

@@ -73,6 +73,7 @@ glga_status dev_alloc(Ctx *c, void **p, size_t bytes) {
 static void release_ctx(Ctx *c) {
     if (!c) return;
     if (c->kv_external) c->KV = nullptr;   // the caller's buffer
+    backward_release(c);
     void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
                     c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
@@ -81,7 +82,7 @@ static void release_ctx(Ctx *c) {
                     c->bw_dg, c->bw_lse, c->bw_Dd, c->bw_dZ, c->bw_dsz_part, c->bw_dSz,
                     c->bw_dw_part, c->bw_q_rows, c->bw_k_rows, c->bw_ST, c->bw_dST, c->bw_Wall, c->bw_dbg_part,
                     c->bw_dSc, c->bw_q_chunks, c->bw_k_chunks, c->bw_q_cptr, c->bw_k_cptr,
-                    c->bw_q_part, c->bw_kv_part, c->dev_flag};
+                    c->bw_q_part, c->bw_kv_part, c->bw_cublas_ws, c->bw_Xf, c->bw_dW3, c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)

@@ -139,6 +139,10 @@ struct Ctx {
     int64_t bw_nq_chunks = 0, bw_nk_chunks = 0;
     float *bw_q_part = nullptr, *bw_kv_part = nullptr;  // chunk shares
     cudaStream_t bw_side = nullptr;                   // second stream of the backward (source side)
+    void *bw_cublas = nullptr;                        // cuBLAS handle (bf16 layers), or null
+    void *bw_cublas_ws = nullptr;                     // its workspace
+    float *bw_Xf = nullptr;                           // [N][d] fp32 copy of X for the dW GEMM
+    float *bw_dW3 = nullptr;                          // [d][3D] the dW GEMM's output
     cudaEvent_t bw_ev_fork = nullptr, bw_ev_join = nullptr;
     float *bw_dbg_part = nullptr;                     // [wparts] row-range sums of dt
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
@@ -194,6 +198,7 @@ glga_status block_run(Ctx *c, const void *Y, const void *X, const void *Wo, cons
                       const void *beta, float ln_eps, void *Z, cudaStream_t s);
 
 // backward.cu
+void backward_release(Ctx *c);
 glga_status backward_setup(Ctx *c, cudaStream_t s);
 glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV,
                          const void *wg, float b_g, float eps, const void *dY, float *dX, float *dWQ,
