@@ -241,7 +241,8 @@ __global__ void __launch_bounds__(256) bwd_readout_kernel(
 // Partial sums of dS | dz over the row range of block column p, per head h =
 // blockIdx.y, in the layout [H][R][R+1] (column R is dz):
 //   part[p][h][a][c] = sum_i phi(q_i[h R + a]) * (c < R ? dnum_i[h R + c] : dden_i[h]).
-// 32-row tiles of phi(Q_h), dnum_h and dden_h are staged in shared memory; each thread
+// Row tiles (32 rows; 8 at R = 128) of phi(Q_h), dnum_h and dden_h are staged in shared
+// memory, the next one prefetched into registers during the current one; each thread
 // owns 4 (a) x 4 (c) output tiles (NT of them when R >= 64) and, for the first column
 // tile, the dz entries of its 4 a's.  For R <= 32 the block's threads form G row groups
 // (group g takes rows g, g + G, ... of each staged tile), added in group order at the end.
@@ -249,7 +250,7 @@ template <typename T, int R>
 __global__ void __launch_bounds__(256) bwd_dsz_partial_kernel(const T *__restrict__ Q, const float *__restrict__ dnum,
                                                               const float *__restrict__ dden, int64_t N, int H,
                                                               int64_t rows_per_part, float *__restrict__ part) {
-    constexpr int kRowsT = 32, TR = R / 4, NTILE = TR * TR;
+    constexpr int kRowsT = R >= 128 ? 8 : 32, TR = R / 4, NTILE = TR * TR;   // rows per staged tile
     constexpr int G = NTILE >= 256 ? 1 : 256 / NTILE;
     constexpr int NT = NTILE >= 256 ? NTILE / 256 : 1;
     constexpr int PH = R * (R + 1);                      // outputs per head
@@ -272,16 +273,33 @@ __global__ void __launch_bounds__(256) bwd_dsz_partial_kernel(const T *__restric
 #pragma unroll
             for (int w = 0; w < 4; ++w) acc[n][u][w] = 0.f;
         }
-    for (int64_t i0 = r0; i0 < r1; i0 += kRowsT) {
-        for (int l = t; l < kRowsT * R; l += 256) {
-            const int rr = l / R, c = l % R;
-            const int64_t i = i0 + rr;
-            const bool in = i < r1;
-            pq[l] = in ? phi(ldf<T>(Q + i * D + h * R + c)) : 0.f;
-            pw[l] = in ? dnum[i * D + h * R + c] : 0.f;
+    // the next tile's inputs are loaded into registers while the current one is multiplied
+    constexpr int kPer = (kRowsT * R + 255) / 256;
+    float rq[kPer], rw[kPer], rd = 0.f;
+    auto fetch = [&](int64_t i0) {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int l = t + u * 256;
+            const int64_t i = i0 + l / R;
+            const bool in = l < kRowsT * R && i < r1;
+            rq[u] = in ? phi(ldf<T>(Q + i * D + h * R + l % R)) : 0.f;
+            rw[u] = in ? dnum[i * D + h * R + l % R] : 0.f;
         }
-        if (t < kRowsT) pd[t] = i0 + t < r1 ? dden[(i0 + t) * H + h] : 0.f;
+        if (t < kRowsT) rd = i0 + t < r1 ? dden[(i0 + t) * H + h] : 0.f;
+    };
+    if (r0 < r1) fetch(r0);
+    for (int64_t i0 = r0; i0 < r1; i0 += kRowsT) {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int l = t + u * 256;
+            if (l < kRowsT * R) {
+                pq[l] = rq[u];
+                pw[l] = rw[u];
+            }
+        }
+        if (t < kRowsT) pd[t] = rd;
         __syncthreads();
+        if (i0 + kRowsT < r1) fetch(i0 + kRowsT);
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const int tile = G > 1 ? t % NTILE : t + n * 256;

@@ -85,3 +85,23 @@ def test_backward_needs_the_option():
         layer.backward(*args, w.b_g, w.eps, torch.zeros(w.N, w.D, device="cuda"))
     assert ei.value.status == 1
     layer.close()
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_edgeless_graph(io):
+    # no local terms at all: only the global branch and the gate carry gradient
+    w = make_custom(70, 16, 2, 8, np.zeros(0, np.int32), np.zeros(0, np.int32), io=io, seed=4, b_g=0.3)
+    _check(w, seed=5)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_very_heavy_target_and_source(io):
+    # target 7 and source 11 each carry 5,000 entries (157 chunks of 32, the last one
+    # ragged), beside a light background of 3 entries per row; H*r = 32 puts one feature
+    # on each lane
+    rng = np.random.default_rng(8)
+    N = 600
+    dst = np.concatenate([np.full(5000, 7), rng.integers(0, N, 5000), np.repeat(np.arange(N), 3)])
+    src = np.concatenate([rng.integers(0, N, 5000), np.full(5000, 11), rng.integers(0, N, 3 * N)])
+    w = make_custom(N, 32, 2, 16, src.astype(np.int32), dst.astype(np.int32), io=io, seed=9, b_g=-0.2)
+    _check(w, seed=10)
