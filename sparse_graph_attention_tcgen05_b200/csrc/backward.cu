@@ -16,8 +16,10 @@
 //       dZ = [dQ | dK | dV | dt].
 // The target-grouped terms (dq) walk the forward CSR; the source-grouped terms (dk, dv)
 // walk a transposed CSR built at create, so every sum has a fixed order and there are no
-// atomics (two runs give identical bits).  Plain CUDA-core kernels with fp32 arithmetic
-// (one thread per row and head, tiled GEMMs for the projections); gradients are fp32.
+// atomics (two runs give identical bits).  CUDA-core kernels with fp32 arithmetic (one
+// warp per row or per 32-edge chunk of a heavy row, register-tiled GEMMs for the weight
+// and input gradients, which bf16 layers run on cuBLAS's TF32 tensor-core GEMMs instead);
+// gradients are fp32.  The log-sum-exp of each row's scores comes from the forward.
 #include <dlfcn.h>
 
 #include <algorithm>
