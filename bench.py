@@ -257,42 +257,104 @@ def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
                         + ("; dW and dX as cuBLAS GEMMs on the TF32 tensor cores" if w.io == "bf16" else ""))}
 
 
-def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0):
-    """Forward time against N at fixed in-degree: the tiny config's shape (d=32, H=1,
-    r=16, fp32, k distinct uniform in-neighbours + self-loop; the method page's cost-proxy
-    setting |E|/N = 8, r = 16) at N = 2^e for each e.  Median of `steps` forwards, each
-    timed with CUDA events on the launching stream, L2 flushed between them.  Returns
-    [(N, E, ms)]."""
+def median_event_ms(fn, steps, warmup, flush):
+    """Median over `steps` calls of fn, each timed with CUDA events on the current stream
+    with L2 flushed before it (outside the timed span), after `warmup` untimed calls."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    times = []
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(steps):
+        flush.zero_()
+        ev0.record(stream)
+        fn()
+        ev1.record(stream)
+        ev1.synchronize()
+        times.append(ev0.elapsed_time(ev1))
+    return float(np.median(times))
+
+
+def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0, d=32, H=1, r=16, io="f32", dense=None):
+    """Forward time against N at fixed in-degree: by default the tiny config's shape
+    (d=32, H=1, r=16, fp32, k distinct uniform in-neighbours + self-loop; the method page's
+    cost-proxy setting |E|/N = 8, r = 16) at N = 2^e for each e.  Median of `steps`
+    forwards, each timed with CUDA events on the launching stream, L2 flushed between
+    them.  Returns [(N, E, ms)], or [(N, E, ms, dense)] with dense(w, args, flush) called
+    on each point when given."""
     import torch
     from sparse_graph_attention_tcgen05_b200 import glga
     from sparse_graph_attention_tcgen05_b200.workloads import make_custom, uniform_in_neighbours
     dev = torch.device("cuda")
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
+    dt = glga.torch_dtype(io)
     out = []
     for e in exponents:
         N = 1 << e
         src, dst = uniform_in_neighbours(N, k, seed)
-        w = make_custom(N, 32, 1, 16, src, dst, io="f32", seed=seed + 1)
+        w = make_custom(N, d, H, r, src, dst, io=io, seed=seed + 1)
         row_ptr, col_idx = glga.csr_from_coo(N, torch.from_numpy(src).to(dev), torch.from_numpy(dst).to(dev))
         layer = glga.Layer(N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
-        args = [torch.from_numpy(a).to(dev) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
-        Y = torch.empty(N, w.D, dtype=torch.float32, device=dev)
-        for _ in range(warmup):
-            layer.forward(*args, b_g=w.b_g, eps=w.eps, Y=Y)
-        times = []
-        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for _ in range(steps):
-            flush.zero_()
-            ev0.record(stream)
-            layer.forward(*args, b_g=w.b_g, eps=w.eps, Y=Y)
-            ev1.record(stream)
-            ev1.synchronize()
-            times.append(ev0.elapsed_time(ev1))
+        args = [torch.from_numpy(a).to(dev).to(dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+        Y = torch.empty(N, w.D, dtype=dt, device=dev)
+        ms = median_event_ms(lambda: layer.forward(*args, b_g=w.b_g, eps=w.eps, Y=Y), steps, warmup, flush)
         assert layer.last_device_error() == 0
         layer.close()
-        out.append((N, w.E, float(np.median(times))))
+        if dense is None:
+            out.append((N, w.E, ms))
+        else:
+            out.append((N, w.E, ms, dense(w, args, flush)))
     return out
+
+
+def dense_attention_ms(w, args, flush, steps=20, warmup=3, masked_max_n=8192):
+    """The dense baseline of the method page's cost comparison at the layer's width: the
+    Q, K, V projections (torch matmul) and softmax attention of every node over all N nodes
+    (torch scaled_dot_product_attention, a library kernel), timed like the layer; also the
+    adjacency-masked form (each node over its CSR row only, as a boolean mask) up to
+    masked_max_n nodes.  Not the product path: a comparison only."""
+    import torch
+    import torch.nn.functional as F
+    X, WQ, WK, WV = args[:4]
+    N, H, r = w.N, w.H, w.r
+
+    def heads(t):
+        return t.view(1, N, H, r).transpose(1, 2)
+
+    def run(mask):
+        q, k, v = heads(X @ WQ), heads(X @ WK), heads(X @ WV)
+        return F.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+
+    res = {"dense_ms": median_event_ms(lambda: run(None), steps, warmup, flush), "masked_ms": None}
+    if N <= masked_max_n:
+        mask = torch.zeros(N, N, dtype=torch.bool, device=X.device)
+        mask[torch.from_numpy(w.dst.astype(np.int64)).to(X.device),
+             torch.from_numpy(w.src.astype(np.int64)).to(X.device)] = True
+        res["masked_ms"] = median_event_ms(lambda: run(mask), steps, warmup, flush)
+        del mask
+    return res
+
+
+def run_dense_sweep():
+    """Dense-vs-hybrid latency at matched width (the arxiv width: d=128, H=4, r=32, bf16):
+    N = 2^10 .. 2^16 at in-degree 8 (+ self-loop), then in-degree 4 .. 128 at N = 2^14."""
+    rows = []
+    for k, exps in ((8, range(10, 17)), (4, [14]), (16, [14]), (32, [14]), (64, [14]), (128, [14])):
+        for N, E, ms, dn in sweep_points(exps, k=k, steps=20, warmup=3, d=128, H=4, r=32, io="bf16",
+                                         dense=dense_attention_ms):
+            rows.append({"N": N, "in_degree": k, "E": E, "glga_ms": ms, **dn,
+                         "dense_over_glga": dn["dense_ms"] / ms,
+                         "masked_over_glga": None if dn["masked_ms"] is None else dn["masked_ms"] / ms})
+    n_pts = [p for p in rows if p["in_degree"] == 8]
+    print(json.dumps({"dense_sweep": "layer forward (glga) vs dense softmax attention (projections + "
+                                     "torch SDPA over all N; masked: over the CSR row) at d=128, H=4, "
+                                     "r=32, bf16; median of 20, L2 flushed",
+                      "points": rows,
+                      "glga_loglog_slope_N": loglog_slope([(p["N"], p["E"], p["glga_ms"]) for p in n_pts
+                                                           if p["N"] >= (1 << 13)]),
+                      "dense_loglog_slope_N": loglog_slope([(p["N"], p["E"], p["dense_ms"]) for p in n_pts
+                                                            if p["N"] >= (1 << 13)])}))
 
 
 def loglog_slope(points):
@@ -414,12 +476,17 @@ def main():
                     help="also time the block around the layer, Z = LayerNorm(X + Y Wo)")
     ap.add_argument("--sharded", action="store_true",
                     help="row-sharded forward across the ranks (strong scaling) instead of replicas")
+    ap.add_argument("--dense-sweep", action="store_true",
+                    help="layer forward against dense softmax attention over N and in-degree")
     ap.add_argument("--sweep", action="store_true",
                     help="time the forward against N at fixed degree instead (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.sweep:
         run_sweep()
+        return
+    if args.dense_sweep:
+        run_dense_sweep()
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
