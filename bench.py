@@ -5,9 +5,12 @@
 
 One step is one glga_forward (projection GEMM, global statistics, fused local branch +
 readout + gate) over the arxiv-shaped synthetic graph, with the graph already bound
-(glga_create, timed separately as create_ms) and inputs resident in HBM.  L2 is flushed
-(256 MiB write) between timed steps, outside the timed spans.  Metric: edge*heads/s =
-E * H / seconds per forward, E counting self-loops.
+(glga_create, timed separately as create_ms) and inputs resident in HBM.  The timed
+steps replay a CUDA graph of glga_forward captured once on the same buffers
+(Layer.capture: the same kernels, without host work between them); an eager loop with
+the library's stage events gives the per-stage times, the launch count and the `eager`
+figures.  L2 is flushed (256 MiB write) between timed steps, outside the timed spans.
+Metric: edge*heads/s = E * H / seconds per forward, E counting self-loops.
 
 Multi-GPU (torchrun, one rank per GPU): replicas only -- every rank runs the same forward
 on its own copy of the graph (weak scaling); value = sum of all ranks' edge*heads over
@@ -299,12 +302,16 @@ def sweep_points(exponents, k=8, steps=30, warmup=5, seed=0, d=32, H=1, r=16, io
         args = [torch.from_numpy(a).to(dev).to(dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
         Y = torch.empty(N, w.D, dtype=dt, device=dev)
         ms = median_event_ms(lambda: layer.forward(*args, b_g=w.b_g, eps=w.eps, Y=Y), steps, warmup, flush)
-        assert layer.last_device_error() == 0
-        layer.close()
         if dense is None:
             out.append((N, w.E, ms))
         else:
-            out.append((N, w.E, ms, dense(w, args, flush)))
+            extra = dense(w, args, flush)
+            graph, _ = layer.capture(*args, w.b_g, w.eps, Y=Y)
+            extra["glga_graph_ms"] = median_event_ms(graph.replay, steps, warmup, flush)
+            del graph
+            out.append((N, w.E, ms, extra))
+        assert layer.last_device_error() == 0
+        layer.close()
     return out
 
 
@@ -344,6 +351,7 @@ def run_dense_sweep():
         for N, E, ms, dn in sweep_points(exps, k=k, steps=20, warmup=3, d=128, H=4, r=32, io="bf16",
                                          dense=dense_attention_ms):
             rows.append({"N": N, "in_degree": k, "E": E, "glga_ms": ms, **dn,
+                         "dense_over_glga_graph": dn["dense_ms"] / dn["glga_graph_ms"],
                          "dense_over_glga": dn["dense_ms"] / ms,
                          "masked_over_glga": None if dn["masked_ms"] is None else dn["masked_ms"] / ms})
     n_pts = [p for p in rows if p["in_degree"] == 8]
@@ -568,12 +576,44 @@ def main():
         Yg = Y.float().cpu().numpy()[rows].astype(np.float64)
         parity = float(np.abs(Yg - ref["Y"]).max() / np.abs(ref["Y"]).max())
 
-    # ---- timed region: K forwards, L2 flushed between them ----
-    layer.set_timing(True)
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    # ---- eager forwards with the library's stage events: per-stage times, launch count ----
+    n_eager = min(args.steps, 500)
+    layer.set_timing(True)
     launches0 = layer.kernel_launches()
     stage_sum = {k: 0.0 for k in glga.STAGES}
+    eager_ms = []
+    for _ in range(n_eager):
+        flush.zero_()
+        ev0.record(stream)
+        fwd()
+        ev1.record(stream)
+        ev1.synchronize()
+        eager_ms.append(ev0.elapsed_time(ev1))
+        for k, v in layer.stage_times().items():
+            stage_sum[k] += v
+    launches_per_forward = (layer.kernel_launches() - launches0) / n_eager
+    layer.set_timing(False)
+    stages = {k: v / n_eager for k, v in stage_sum.items()}
+    eager_total = max_over_ranks(sum(eager_ms))
+    eager = {"value": replica_throughput(world, w.E * w.H, eager_total, n_eager), "unit": UNIT,
+             "ms_per_step": eager_total / n_eager, "steps": n_eager,
+             "note": "glga_forward called per step, stage events on"}
+
+    # ---- timed region: K forwards replayed from a CUDA graph of glga_forward
+    # (Layer.capture: the same six kernels on the same buffers, no host work between
+    # them), L2 flushed between steps; eager calls if the capture is refused ----
+    graph = None
+    try:
+        graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)
+        run_step = graph.replay
+    except RuntimeError as exc:
+        run_step = fwd
+        eager["capture_refused"] = str(exc).splitlines()[0][:200]
+    for _ in range(args.warmup):
+        run_step()
     step_ms = []
     barrier()
     torch.cuda.synchronize()
@@ -584,24 +624,22 @@ def main():
     for _ in range(args.steps):
         flush.zero_()
         ev0.record(stream)
-        fwd()
+        run_step()
         ev1.record(stream)
         ev1.synchronize()
         step_ms.append(ev0.elapsed_time(ev1))
-        for k, v in layer.stage_times().items():
-            stage_sum[k] += v
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     clocks = sampler.stop()
     barrier()
-    launches = layer.kernel_launches() - launches0
-    layer.set_timing(False)
+    graph_ok = graph is not None
+    del graph
     assert layer.last_device_error() == 0
+    launches = int(round(launches_per_forward * args.steps))
 
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / args.steps
     value = replica_throughput(world, w.E * w.H, total_ms, args.steps)
-    stages = {k: v / args.steps for k, v in stage_sum.items()}
 
     # ---- end to end through the public API: pinned host -> device, forward, Y -> host ----
     Yh = torch.empty(w.N, w.D, dtype=dt).pin_memory()
@@ -665,7 +703,8 @@ def main():
                        "segments": 1 if seg is None else int(seg.shape[0] - 1)},
             "roofline": roofline, "local_branch_a3_a5": branch, "projection": projection,
             "stages_ms": stages, "create": create, "gpu_launches": launches,
-            "e2e": e2e, "clocks": clocks, "parity_max_rel_err": parity,
+            "e2e": e2e, "eager": eager, "timed_region": "CUDA graph replay of glga_forward" if graph_ok
+            else "eager glga_forward", "clocks": clocks, "parity_max_rel_err": parity,
             "wall_s_timed_region": wall}
     if args.block:
         line["block"] = time_block(layer, w, X, Y, dt, dev, flush, stream, args.steps, peaks)

@@ -197,6 +197,25 @@ class Layer:
 
     __call__ = forward
 
+    def capture(self, X, W_Q, W_K, W_V, w_g, b_g: float, eps: float, Y=None):
+        """Records one glga_forward on these buffers into a CUDA graph and returns
+        (graph, Y): graph.replay() reruns the whole forward on the same X, weights and Y
+        (refill them in place between replays; b_g and eps are fixed at capture).  The
+        forward enqueues kernels only (no allocation, no host synchronisation, tensor maps
+        passed by value), so it records whole; one eager call first settles the lazy
+        per-kernel attributes outside the capture.  Stage timing must be off."""
+        if Y is None:
+            Y = torch.empty(self.N, self.D, dtype=self.dtype, device=X.device)
+        side = torch.cuda.Stream(device=X.device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(X, W_Q, W_K, W_V, w_g, b_g, eps, Y=Y)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            self.forward(X, W_Q, W_K, W_V, w_g, b_g, eps, Y=Y)
+        return graph, Y
+
     # -- introspection ---------------------------------------------------------------
     def bucket_counts(self):
         c = (_i64 * 4)()

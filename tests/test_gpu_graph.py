@@ -1,0 +1,38 @@
+"""glga_forward recorded into a CUDA graph (Layer.capture): a replay gives the same bits as
+an eager forward on the same buffers, also after the inputs are refilled in place."""
+import numpy as np
+import pytest
+import torch
+
+from sparse_graph_attention_tcgen05_b200 import glga
+from sparse_graph_attention_tcgen05_b200.workloads import make_workload
+from tests.gpu_helpers import to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name,scale", [("tiny", 1.0), ("citation", 1.0), ("arxiv", 0.05), ("packed", 0.02)])
+def test_graph_replay_matches_eager(name, scale):
+    w = make_workload(name, scale=scale)
+    row_ptr, col_idx = glga.csr_from_coo(w.N, to_dev(w.src), to_dev(w.dst))
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+    dt = glga.torch_dtype(w.io)
+    args = [to_dev(a, dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+    eager = layer.forward(*args, b_g=w.b_g, eps=w.eps).clone()
+    graph, Y = layer.capture(*args, w.b_g, w.eps)
+    Y.fill_(float("nan"))
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y, eager)
+    # new inputs, refilled in place: the replay follows them
+    rng = np.random.default_rng(12)
+    args[0].copy_(to_dev(rng.standard_normal(w.X.shape).astype(np.float32), dt))
+    args[3].mul_(0.5)
+    graph.replay()
+    torch.cuda.synchronize()
+    again = layer.forward(*args, b_g=w.b_g, eps=w.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, again) and not torch.equal(Y, eager)
+    assert layer.last_device_error() == 0
+    del graph
+    layer.close()
