@@ -255,7 +255,19 @@ def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
         ms.append(ev0.elapsed_time(ev1))
     assert layer.last_device_error() == 0
     t = float(np.mean(ms))
+    graph, _ = layer.capture_backward(X, WQ, WK, WV, wg, w.b_g, w.eps, dY)
+    gms = []
+    for _ in range(steps):
+        flush.zero_()
+        ev0.record(stream)
+        graph.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+        gms.append(ev0.elapsed_time(ev1))
+    del graph
+    tg = float(np.mean(gms))
     return {"ms": t, "edge_heads_per_s": w.E * w.H / (t * 1e-3), "steps": steps,
+            "graph_ms": tg, "graph_edge_heads_per_s": w.E * w.H / (tg * 1e-3),
             "kernels": ("CUDA-core (SIMT) kernels, fp32 arithmetic"
                         + ("; dW and dX as cuBLAS GEMMs on the TF32 tensor cores" if w.io == "bf16" else ""))}
 

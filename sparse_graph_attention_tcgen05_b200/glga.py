@@ -269,6 +269,23 @@ class Layer:
                                    _stream(stream)), "glga_backward")
         return out
 
+    def capture_backward(self, X, W_Q, W_K, W_V, w_g, b_g: float, eps: float, dY):
+        """Records one glga_backward on these buffers into a CUDA graph and returns
+        (graph, grads): graph.replay() recomputes the gradients into the same tensors from
+        the state of the last forward (run forward() or its graph first when the inputs
+        change).  The backward enqueues kernels, events between its two streams and, for
+        bf16 layers, cuBLAS GEMMs on a preset workspace, so it records whole; one eager call
+        first settles the lazily loaded kernels outside the capture."""
+        side = torch.cuda.Stream(device=X.device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.backward(X, W_Q, W_K, W_V, w_g, b_g, eps, dY)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            grads = self.backward(X, W_Q, W_K, W_V, w_g, b_g, eps, dY)
+        return graph, grads
+
     def block_output(self, Y, X, Wo, gamma, beta, ln_eps: float = 1e-5, Z=None, stream=None):
         """Z = LayerNorm(X + Y Wo) (glga_block_output)."""
         for t in (Y, X, Wo, gamma, beta):

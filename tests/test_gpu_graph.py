@@ -36,3 +36,35 @@ def test_graph_replay_matches_eager(name, scale):
     assert layer.last_device_error() == 0
     del graph
     layer.close()
+
+
+@pytest.mark.parametrize("name,scale", [("tiny", 1.0), ("arxiv", 0.05)])
+def test_backward_graph_replay_matches_eager(name, scale):
+    w = make_workload(name, scale=scale)
+    row_ptr, col_idx = glga.csr_from_coo(w.N, to_dev(w.src), to_dev(w.dst))
+    o = glga.default_options()
+    o.backward = 1
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx, o)
+    dt = glga.torch_dtype(w.io)
+    args = [to_dev(a, dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+    dY = to_dev(np.random.default_rng(3).standard_normal((w.N, w.D)).astype(np.float32), dt)
+    layer.forward(*args, b_g=w.b_g, eps=w.eps)
+    eager = {k: v.clone() for k, v in layer.backward(*args, w.b_g, w.eps, dY).items()}
+    graph, grads = layer.capture_backward(*args, w.b_g, w.eps, dY)
+    for v in grads.values():
+        v.fill_(float("nan"))
+    graph.replay()
+    torch.cuda.synchronize()
+    for k in eager:
+        assert torch.equal(grads[k], eager[k]), k
+    # a new upstream gradient, refilled in place
+    dY.mul_(-2.0)
+    graph.replay()
+    torch.cuda.synchronize()
+    again = layer.backward(*args, w.b_g, w.eps, dY)
+    torch.cuda.synchronize()
+    for k in eager:
+        assert torch.equal(grads[k], again[k]), k
+    assert layer.last_device_error() == 0
+    del graph
+    layer.close()
