@@ -570,6 +570,36 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
     }
 }
 
+// The global terms of source row j and the store, in the 32-lane layout (every lane of
+// the warp takes part in the shuffles):
+//   dphi(k_j)_f = sum_c dS[f][c] v_c + dz_f,  dv_j,f += sum_c dS[c][f] phi(k_c)
+// (S = sum phi(k) v^T, z = sum phi(k)); dk, dv hold the local terms on entry.
+template <int EPL>
+__device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t j, const float (&k)[EPL],
+                                          const float (&v)[EPL], float (&dk)[EPL], float (&dv)[EPL],
+                                          const float *dSc, const float *dST, int H, int R, float *dZ,
+                                          int64_t dz_ld) {
+    const int D = H * R;
+    float dphk[EPL], dvg[EPL], pk[EPL];
+    ld_mrow<EPL>(dSc + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, dphk);
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) {
+        dvg[x] = 0.f;
+        pk[x] = phi(k[x]);
+    }
+    head_matvec<EPL>(dST + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, v, dphk);
+    head_matvec<EPL>(dSc + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, pk, dvg);
+    if (lh.act) {
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) {
+            dk[x] = fmaf(dphk[x], dphi(k[x]), dk[x]);
+            dv[x] += dvg[x];
+        }
+        st_mrow<EPL>(dZ + j * dz_ld + D + lane * EPL, dk);
+        st_mrow<EPL>(dZ + j * dz_ld + 2 * D + lane * EPL, dv);
+    }
+}
+
 // Source rows of the transposed CSR (the targets i of j): the local terms of dk_j and
 // dv_j, plus the global terms through phi(k_j), written to dZ [:, D:2D] and [:, 2D:3D].
 // Light rows (PARTS false, one warp each) walk their edges; heavy rows (PARTS true, one
@@ -645,26 +675,89 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
         kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, lh.act, lh.lph, lh.h, inv_sqrt_r, k, v,
                               t_row_ptr[j], t_row_ptr[j + 1], dk, dv);
     }
-    // global branch, S = sum phi(k) v^T and z = sum phi(k):
-    //   dphi(k_j)_f = sum_c dS[f][c] v_c + dz_f,  dv_j,f += sum_c dS[c][f] phi(k_c)
-    float dphk[EPL], dvg[EPL], pk[EPL];
-    ld_mrow<EPL>(dSc + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, dphk);
+    kv_finish<EPL>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
+}
+
+// Light source rows with two edges per step: the warp's halves (slots) take alternate
+// edges of the row, lane hl = lane % 16 of a half holding the EPL2 = 2 EPL features
+// hl*EPL2 .. hl*EPL2+EPL2-1 (a head's r features in r/EPL2 lanes of the half), so the two
+// edges of a step share one shuffle butterfly and one exponential per lane.  The halves'
+// dk, dv are then added (lower + upper, the same sum in both) and moved to the 32-lane
+// layout for kv_finish.  Needs 2 EPL <= r.
+template <typename T, int EPL>
+__global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
+    const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
+    const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
+    const float *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
+    const float *__restrict__ dSc, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
+    float *__restrict__ dZ, int64_t dz_ld) {
+    constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
+    const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
+    const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (w >= n_rows) return;                              // warp-uniform
+    const int64_t j = rows[w];
+    const int D = H * R;
+    const bool act2 = hl * EPL2 < D;
+    const int lph2 = R / EPL2, h2 = act2 ? hl * EPL2 / R : 0;
+    const T *krow = KV + j * 2 * D;
+    float k2[EPL2], v2[EPL2], dk2[EPL2], dv2[EPL2];
+    ld_row<T, EPL2>(krow, hl, act2, k2);
+    ld_row<T, EPL2>(krow + D, hl, act2, v2);
+#pragma unroll
+    for (int x = 0; x < EPL2; ++x) dk2[x] = dv2[x] = 0.f;
+    const int32_t a = t_row_ptr[j], b = t_row_ptr[j + 1];
+    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {          // the same trip count in both halves
+        float q[kU][EPL2], dl[kU][EPL2], ls[kU], dd[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int32_t e = e0 + 2 * u + slot;
+            const bool live = e < b;
+            const int64_t i = live ? t_col[e] : 0;
+            ld_row<T, EPL2>(Q + i * D, hl, act2 && live, q[u]);
+            ld_row<float, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
+            ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
+            dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            float sc = 0.f, dp = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) {
+                sc = fmaf(q[u][x], k2[x], sc);
+                dp = fmaf(dl[u][x], v2[x], dp);
+            }
+            sc = head_reduce(sc, lph2);
+            dp = head_reduce(dp, lph2);
+            const bool live = e0 + 2 * u + slot < b;
+            const float p = live ? __expf(sc * inv_sqrt_r - ls[u]) : 0.f;
+            const float ds = p * (dp - dd[u]) * inv_sqrt_r;
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) {
+                dv2[x] = fmaf(p, dl[u][x], dv2[x]);
+                dk2[x] = fmaf(ds, q[u][x], dk2[x]);
+            }
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < EPL2; ++x) {
+        dk2[x] += __shfl_xor_sync(0xffffffffu, dk2[x], 16);
+        dv2[x] += __shfl_xor_sync(0xffffffffu, dv2[x], 16);
+    }
+    // to the 32-lane layout: lane l's features l*EPL .. are half-lane l/2's, part l % 2
+    const LaneHead lh(lane, EPL, D, R);
+    const int src = lane >> 1;
+    const bool hi = lane & 1;
+    float k[EPL], v[EPL], dk[EPL], dv[EPL];
 #pragma unroll
     for (int x = 0; x < EPL; ++x) {
-        dvg[x] = 0.f;
-        pk[x] = phi(k[x]);
+        const float k0 = __shfl_sync(0xffffffffu, dk2[x], src), k1 = __shfl_sync(0xffffffffu, dk2[EPL + x], src);
+        const float v0 = __shfl_sync(0xffffffffu, dv2[x], src), v1 = __shfl_sync(0xffffffffu, dv2[EPL + x], src);
+        dk[x] = hi ? k1 : k0;
+        dv[x] = hi ? v1 : v0;
     }
-    head_matvec<EPL>(dST + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, v, dphk);
-    head_matvec<EPL>(dSc + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, pk, dvg);
-    if (lh.act) {
-#pragma unroll
-        for (int x = 0; x < EPL; ++x) {
-            dk[x] = fmaf(dphk[x], dphi(k[x]), dk[x]);
-            dv[x] += dvg[x];
-        }
-        st_mrow<EPL>(dZ + j * dz_ld + D + lane * EPL, dk);
-        st_mrow<EPL>(dZ + j * dz_ld + 2 * D + lane * EPL, dv);
-    }
+    ld_row<T, EPL>(krow, lane, lh.act, k);
+    ld_row<T, EPL>(krow + D, lane, lh.act, v);
+    kv_finish<EPL>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
 }
 
 // Chunks of heavy source rows, one warp each (layout as bwd_q_chunk_kernel's, over the
@@ -996,7 +1089,25 @@ __global__ void bwd_x_to_f32_kernel(const __nv_bfloat16 *__restrict__ X, int64_t
         Xf[o] = __bfloat162float(X[o]);
 }
 
-unsigned warp_grid(int64_t n) { return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256))); }
+unsigned warp_grid(int64_t n) {
+    return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256)));
+}
+
+// Light source rows: two edges per warp step where a head spans at least two of the
+// 16-lane half's slices (2 EPL <= r, EPL <= 4), else one edge per step.
+template <typename T, int E>
+void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cudaStream_t sk) {
+    const int64_t nkl = c->bw_nk_light;
+    if constexpr (E <= 4) {
+        if (2 * E <= c->r) {
+            bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
+                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+            return;
+        }
+    }
+    bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
+        nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+}
 
 // Both local backward kernels with EPL = lane_features(D): light rows one warp each;
 // heavy rows (more than kHeavyDegree entries) as kChunk-edge chunks, one warp each, whose
@@ -1012,10 +1123,7 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
     const int32_t *qh = c->bw_q_rows + nql, *kh = c->bw_k_rows + nkl;
 #define GLGA_LB(E)                                                                                        \
     case E:                                                                                               \
-        if (nkl)                                                                                          \
-            bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl,            \
-                c->t_row_ptr, c->t_col, nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, \
-                c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                                      \
+        if (nkl) launch_kv_light<T, E>(c, Q, KV, isr, Dz, sk);                                           \
         if (nkh) {                                                                                        \
             bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, sk>>>(c->bw_k_chunks, nkc, c->t_row_ptr,   \
                 c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
