@@ -75,8 +75,10 @@ typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
  * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.
  * backward != 0 allocates the workspaces of glga_backward at create (a transposed CSR,
  * chunk lists of the rows with more than 64 entries, a second stream and fp32 buffers of
- * about N*(6*H*r + 4*H + 1) floats); glga_forward on such a context also stores each
- * row's softmax log-sum-exp per head for the backward.  Whole-graph, one-segment contexts
+ * about N*(6*H*r + 4*H + 1) floats; for bf16 layers also a cuBLAS handle, opened at run
+ * time, with a 32 MiB workspace and an fp32 copy of X for the weight-gradient GEMM);
+ * glga_forward on such a context also stores each row's softmax log-sum-exp per head for
+ * the backward.  Whole-graph, one-segment contexts
  * with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).                             */
 typedef struct {
     int32_t warp_max_degree;
