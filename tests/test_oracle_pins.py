@@ -570,3 +570,37 @@ def test_backward_matches_finite_differences_of_the_c_oracle():
             fd = (f(plus) - f(minus)) / (2 * h)
             an = float((np.asarray(g[gname]) * u).sum())
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+@pytest.mark.parametrize("max_edges,max_rows", [(7, 3), (20, 1000), (1 << 18, 1 << 16)])
+def test_backward_chunked_equals_backward(max_edges, max_rows):
+    """The bounded-memory reference gradients (row groups of at most max_edges entries and
+    max_rows rows; a row heavier than max_edges forms its own group) equal the whole-graph
+    ones, here with a 40-entry row, an isolated row and duplicated entries."""
+    from oracle.backward import NAMES, backward, backward_chunked
+    rng = np.random.default_rng(12)
+    N = 23
+    src = np.concatenate([rng.integers(0, N, 60), rng.integers(0, N, 40), [5, 5]])
+    dst = np.concatenate([rng.integers(0, N, 60), np.full(40, 9), [2, 2]])
+    keep = dst != 4                                   # row 4 isolated
+    w = make_custom(N, 6, 3, 4, src[keep].astype(np.int32), dst[keep].astype(np.int32), io="f32",
+                    seed=13, b_g=-0.4)
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    dY = rng.standard_normal((w.N, w.D))
+    ref = backward(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY)
+    got = backward_chunked(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY,
+                           max_edges=max_edges, max_rows=max_rows)
+    for k in NAMES:
+        np.testing.assert_allclose(got[k], np.reshape(ref[k], np.shape(got[k])), rtol=1e-11,
+                                   atol=1e-12 * max(1.0, np.abs(ref[k]).max()), err_msg=k)
+
+
+def test_backward_chunked_edgeless_graph():
+    from oracle.backward import NAMES, backward, backward_chunked
+    w = make_custom(9, 5, 2, 4, np.zeros(0, np.int32), np.zeros(0, np.int32), io="f32", seed=3, b_g=0.2)
+    rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
+    dY = np.random.default_rng(1).standard_normal((w.N, w.D))
+    ref = backward(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY)
+    got = backward_chunked(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY, max_edges=4)
+    for k in NAMES:
+        np.testing.assert_allclose(got[k], np.reshape(ref[k], np.shape(got[k])), rtol=1e-11, atol=1e-13, err_msg=k)
