@@ -1,20 +1,24 @@
 """Benchmark of the gated local-global graph-attention forward on B200.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
-                  [--workload arxiv] [--no-cpu-baseline]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--forwards-per-step R]
+                  [--impl mine|reference] [--workload arxiv] [--no-cpu-baseline]
 
-One step is one glga_forward (projection GEMM, global statistics, fused local branch +
-readout + gate) over the arxiv-shaped synthetic graph, with the graph already bound
-(glga_create, timed separately as create_ms) and inputs resident in HBM.  The timed
-steps replay a CUDA graph of glga_forward captured once on the same buffers
-(Layer.capture: the same kernels, without host work between them); an eager loop with
-the library's stage events gives the per-stage times, the launch count and the `eager`
-figures.  L2 is flushed (256 MiB write) between timed steps, outside the timed spans.
+One step is R forwards of the layer (projection GEMM, global statistics, local branch,
+readout with the gate blend) over the arxiv-shaped synthetic graph, with the graph already
+bound (glga_create, timed separately as create_ms) and inputs resident in HBM.  Every
+forward replays a CUDA graph of glga_forward captured once on the same buffers
+(Layer.capture: the same kernels, without host work between them) and is timed with its
+own pair of CUDA events on the launching stream; L2 is flushed (256 MiB write) before
+every forward, outside the timed spans, so the K steps' timed region lasts seconds and the
+clock sampler sees it.  The library's stage events, recorded inside the captured graph,
+give the local kernel's launch time over the timed region for the roofline.
 Metric: edge*heads/s = E * H / seconds per forward, E counting self-loops.
 
-Multi-GPU (torchrun, one rank per GPU): replicas only -- every rank runs the same forward
-on its own copy of the graph (weak scaling); value = sum of all ranks' edge*heads over
-the slowest rank's time.  `--impl reference` times the float64 CPU oracle on the host
+Multi-GPU (torchrun, one rank per GPU): the row-sharded forward (sharded.ShardedForward:
+each rank owns a block of target rows with about equal CSR entries; one NCCL all-gather of
+the K/V row blocks and one of the partial statistics per forward; strong scaling), or
+with --replicas every rank runs the whole forward on its own copy (weak scaling).  Time is
+the maximum over ranks.  `--impl reference` times the float64 CPU oracle on the host
 instead (rank 0 only).
 """
 from __future__ import annotations
@@ -36,6 +40,7 @@ sys.path.insert(0, ROOT)
 METRIC = "GLGA fwd edge·heads/s (1 B200, bf16 arxiv-shaped); local-branch HBM GB/s % of peak"
 UNIT = "edge*heads/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_NOTE = "flushed before every timed forward (256 MiB write, outside the timed spans)"
 
 
 def load_peaks():
@@ -91,24 +96,19 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """dram read+write bytes per launch of the local kernel from the committed ncu summary,
-    if it was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"local_kernel_{workload}.md")
+def profiled_counters(workload):
+    """ncu counters of the local kernel from the structured summary
+    profiles/local_kernel_<workload>.json, if it was taken on the current kernel source:
+    DRAM bytes per launch (scaled to the full workload) and warp instructions per edge."""
+    path = os.path.join(ROOT, "profiles", f"local_kernel_{workload}.json")
     if not os.path.exists(path):
-        return None, None
-    vals = {}
+        return None
     with open(path) as f:
-        for line in f:
-            if line.startswith("- ") and ":" in line:
-                k, v = line[2:].split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_sha256_16") != kernel_source_hash():
-        return None, "stale"
-    try:
-        return float(vals["traffic_bytes_per_launch"]), vals.get("traffic_note")
-    except (KeyError, ValueError):
-        return None, None
+        d = json.load(f)
+    if d.get("local_cu_sha256_16") != kernel_source_hash():
+        return {"stale": True, "file": os.path.relpath(path, ROOT)}
+    d["file"] = os.path.relpath(path, ROOT)
+    return d
 
 
 class ClockSampler:
@@ -174,13 +174,35 @@ def cpu_baseline(w, csr, min_seconds=10.0, max_seconds=30.0):
                       f"in {el:.1f} s on {oracle.num_threads()} OpenMP threads"}
 
 
+def run_mode(args, world):
+    """'sharded' (the default for more than one rank, or --sharded), 'replicas'
+    (--replicas with more than one rank) or 'single'."""
+    if args.sharded or (world > 1 and not args.replicas):
+        return "sharded"
+    return "replicas" if world > 1 else "single"
+
+
+def workload_config(args, w, world, mode, seg=None):
+    """The `config` of the JSON line: the workload and how it is split; both arms of the
+    bench (the library and the oracle) print the same one for the same command line."""
+    par = {"single": "single process",
+           "replicas": f"replicas x{world} (every rank the whole forward)",
+           "sharded": f"row-sharded x{world} (NCCL all-gathers of the K/V row blocks and the partial S|z)"}[mode]
+    return {"workload": args.workload if args.scale == 1.0 else f"{args.workload}@scale{args.scale}",
+            "N": w.N, "E": w.E, "d": w.d, "H": w.H, "r": w.r, "io": w.io,
+            "segments": 1 if seg is None else int(seg.shape[0] - 1), "parallelism": par, "l2": L2_NOTE}
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the float64 oracle as it stands, on the host cores, rank 0 only;
+    one step = one full oracle forward of the workload."""
     from sparse_graph_attention_tcgen05_b200.workloads import make_workload
     import oracle
     if rank != 0:
         return
-    w = make_workload(args.workload)
+    w = make_workload(args.workload, scale=args.scale)
     csr = oracle.csr_from_coo(w.N, w.src, w.dst)
+
     def step():
         oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
                        csr[0], csr[1])
@@ -195,13 +217,88 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": args.workload, "N": w.N, "E": w.E, "d": w.d, "H": w.H, "r": w.r,
-                       "io": w.io, "parallelism": "host oracle, rank 0 only"},
+            "config": workload_config(args, w, world, run_mode(args, world)),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle",
-                             "sample": f"the full {w.name} workload per step (N={w.N}, E={w.E})"},
+                             "sample": f"one full float64 oracle forward of the {w.name} workload per step "
+                                       f"(N={w.N}, E={w.E}) on {oracle.num_threads()} OpenMP threads, rank 0"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+class TimedRegion:
+    """K steps of R forwards: every forward is preceded by an L2 flush outside its span and
+    bracketed by its own CUDA events on `stream`; one host synchronisation per step.
+    `after_step` (optional) is called after each step's synchronisation."""
+
+    def __init__(self, stream, flush, R):
+        import torch
+        self.stream, self.flush, self.R = stream, flush, R
+        self.evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(R)]
+
+    def step(self, run_fwd):
+        for a, b in self.evs:
+            self.flush.zero_()
+            a.record(self.stream)
+            run_fwd()
+            b.record(self.stream)
+        self.evs[-1][1].synchronize()
+        self.last_ms = self.evs[-1][0].elapsed_time(self.evs[-1][1])   # the step's last forward
+        return sum(a.elapsed_time(b) for a, b in self.evs)
+
+    def run(self, run_fwd, K, gpu_index, barrier=None, after_step=None):
+        import torch
+        if barrier:
+            barrier()
+        torch.cuda.synchronize()
+        sampler = ClockSampler(gpu_index)
+        wall0 = time.perf_counter()
+        step_ms = []
+        for _ in range(K):
+            step_ms.append(self.step(run_fwd))
+            if after_step:
+                after_step()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        clocks = sampler.stop()
+        if barrier:
+            barrier()
+        return step_ms, clocks, wall
+
+
+def gpu_index_of(local_rank):
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in visible.split(",") if v.strip()]
+    return ids[local_rank] if local_rank < len(ids) else local_rank
+
+
+def roofline_local(w, t_local_ms, peaks, peak_kind, counters, source):
+    """Roofline object of the dominant kernel (the local softmax branch): algorithmic bytes
+    per launch over its average launch time, against the measured HBM copy rate; with the
+    ncu DRAM bytes per launch (when taken on the current source) the DRAM-level fraction."""
+    s_io = 4 if w.io == "f32" else 2
+    B_kern = local_kernel_bytes(w.N, w.E, w.D, s_io)
+    achieved = B_kern / (t_local_ms * 1e-3) / 1e9
+    ro = {"bound": "hbm", "kernel": "local_kernel (local softmax branch; writes L)",
+          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+          "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+          "algorithmic_bytes_per_launch": B_kern, "avg_launch_ms": t_local_ms, "launch_time_source": source,
+          "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+          else "fallback 6.65 TB/s (no MEASURED_PEAKS.json)",
+          "frac_note": "frac counts every k_j/v_j gather as HBM bytes; on this graph most gathers hit "
+                       "L2, so dram_frac (ncu DRAM bytes over the same launch time) is the HBM-level "
+                       "figure"}
+    if counters and not counters.get("stale"):
+        dram = float(counters["dram_bytes_per_launch"])
+        ro["traffic"] = dram
+        ro["dram_gbs"] = dram / (t_local_ms * 1e-3) / 1e9
+        ro["dram_frac"] = ro["dram_gbs"] / peaks["hbm_gbs"]
+        ro["warp_instructions_per_edge"] = counters.get("warp_instructions_per_edge")
+        ro["counters_from"] = counters["file"]
+    elif counters:
+        ro["counters_from"] = counters["file"] + " (stale: taken on another local.cu)"
+    return ro
 
 
 def time_block(layer, w, X, Y, dt, dev, flush, stream, steps, peaks):
@@ -269,7 +366,8 @@ def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
     return {"ms": t, "edge_heads_per_s": w.E * w.H / (t * 1e-3), "steps": steps,
             "graph_ms": tg, "graph_edge_heads_per_s": w.E * w.H / (tg * 1e-3),
             "kernels": ("CUDA-core (SIMT) kernels, fp32 arithmetic"
-                        + ("; dW and dX as cuBLAS GEMMs on the TF32 tensor cores" if w.io == "bf16" else ""))}
+                        + ("; dW and dX as tcgen05 GEMMs (bf16 dW operands, tf32 dX operands)" if w.io == "bf16"
+                           else "; dW and dX as CUDA-core fp32 GEMMs"))}
 
 
 def median_event_ms(fn, steps, warmup, flush):
@@ -394,131 +492,177 @@ def run_sweep():
                       "slope_loglog_N_ge_2^17": loglog_slope(upper)}), flush=True)
 
 
+def e2e_pipelined(layer, w, host, dt, dev, steps, warmup=3):
+    """End-to-end throughput through the public API (Layer.forward): every step copies its
+    inputs (X and the weights) from pinned host memory, runs the forward and copies Y back
+    to pinned host memory.  Copies run on their own streams with two buffer sets, so step
+    i's host->device copy and step i-1's device->host copy overlap step i's forward (PCIe
+    is full duplex); events order every buffer reuse.  Device time from the first copy's
+    start to the last copy's end."""
+    import torch
+    names = ("X", "W_Q", "W_K", "W_V", "w_g")
+    ins = [[torch.empty_like(host[k], device=dev) for k in names] for _ in range(2)]
+    Yd = [torch.empty(w.N, w.D, dtype=dt, device=dev) for _ in range(2)]
+    Yh = [torch.empty(w.N, w.D, dtype=dt).pin_memory() for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_fwd = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
+
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev_fwd[b])          # the forward that read buffer b is done
+            for t, k in zip(ins[b], names):
+                t.copy_(host[k], non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        if used[b]:
+            comp.wait_event(ev_out[b])              # Y buffer b has been copied out
+        layer.forward(*ins[b], b_g=w.b_g, eps=w.eps, Y=Yd[b], stream=comp)
+        ev_fwd[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_fwd[b])
+            Yh[b].copy_(Yd[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        used[b] = True
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for i in range(steps):
+        step(warmup + i)
+    t1.record(s_out)
+    t1.synchronize()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = Yh[0].numel() * Yh[0].element_size()
+    return ms, h2d, d2h
+
+
 def run_sharded(args, rank, world, local_rank):
     """Row-sharded forward (sharded.ShardedForward): every rank owns a contiguous block of
-    target rows with about equal CSR entries, projects them, exchanges K/V rows and
-    partial statistics over NCCL and finishes its rows.  Total work is fixed as ranks are
-    added (strong scaling); value = E*H per step over the slowest rank's time."""
+    target rows with about equal CSR entries, projects them, exchanges K/V row blocks and
+    partial statistics over NCCL (two all-gathers) and finishes its rows.  Total work is
+    fixed as ranks are added (strong scaling); value = E*H per forward over the slowest
+    rank's time."""
+    import datetime
+    import socket
     import torch
     import torch.distributed as dist
     from sparse_graph_attention_tcgen05_b200 import glga
-    from sparse_graph_attention_tcgen05_b200.sharded import (LibraryShard, ShardedForward,
-                                                             partition_rows, shard_csr)
+    from sparse_graph_attention_tcgen05_b200.sharded import LibraryShard, ShardedForward, ShardPlan
     from sparse_graph_attention_tcgen05_b200.workloads import make_workload
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    if world > 1 and not dist.is_initialized():
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    elif world == 1 and not dist.is_initialized():
-        import socket
-        with socket.socket() as sk:
-            sk.bind(("127.0.0.1", 0))
-            port = sk.getsockname()[1]
-        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    if not dist.is_initialized():
+        if world > 1:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        else:
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=300))
     w = make_workload(args.workload, scale=args.scale)
     dt = glga.torch_dtype(w.io)
     row_ptr, col_idx = glga.csr_from_coo(w.N, torch.from_numpy(w.src).to(dev), torch.from_numpy(w.dst).to(dev))
     rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
-    bounds = partition_rows(rp, world)
-    b0, b1 = int(bounds[rank]), int(bounds[rank + 1])
-    rpo, cio = shard_csr(rp, ci, b0, b1)
-    shard = LibraryShard(w.N, w.d, w.H, w.r, w.io, rpo, cio, b0, b1, device=dev)
-    fwd = ShardedForward(shard, bounds, rank, world)
-    X = torch.from_numpy(np.ascontiguousarray(w.X[b0:b1])).to(dt).to(dev)
-    W = [torch.from_numpy(a).to(dt).to(dev) for a in (w.W_Q, w.W_K, w.W_V, w.w_g)]
-    Y = torch.empty(b1 - b0, w.D, dtype=dt, device=dev)
+    plan = ShardPlan(rp, ci, world, rank)
+    shard = LibraryShard(plan.n_kv, w.d, w.H, w.r, w.io, plan.row_ptr, plan.col_idx, plan.kv0, plan.kv1,
+                         device=dev)
+    fwd = ShardedForward(shard, rank, world)
+    names = ("X", "W_Q", "W_K", "W_V", "w_g")
+    host = {"X": torch.from_numpy(np.ascontiguousarray(w.X[plan.b0:plan.b1])).to(dt).pin_memory()}
+    for k, a in zip(names[1:], (w.W_Q, w.W_K, w.W_V, w.w_g)):
+        host[k] = torch.from_numpy(a).to(dt).pin_memory()
+    X, WQ, WK, WV, wg = (host[k].to(dev) for k in names)
+    Y = torch.empty(plan.b1 - plan.b0, w.D, dtype=dt, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def run_fwd():
+        fwd(X, WQ, WK, WV, wg, w.b_g, w.eps, Y)
+
     for _ in range(args.warmup):
-        fwd(X, *W, w.b_g, w.eps, Y)
+        run_fwd()
     torch.cuda.synchronize()
     assert shard.last_device_error() == 0
     parity = None
-    if not args.no_parity and b1 > b0:
+    if not args.no_parity and plan.b1 > plan.b0:
         import oracle
         rng = np.random.default_rng(rank)
-        rows = np.unique(rng.integers(b0, b1, min(256, b1 - b0)))
+        rows = np.unique(rng.integers(plan.b0, plan.b1, min(256, plan.b1 - plan.b0)))
         ref = oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
                              rp, ci, rows=rows)
-        got = Y.float().cpu().numpy()[rows - b0].astype(np.float64)
+        got = Y.float().cpu().numpy()[rows - plan.b0].astype(np.float64)
         parity = float(np.abs(got - ref["Y"]).max() / np.abs(ref["Y"]).max())
     stream = torch.cuda.current_stream()
+    # the local kernel's launch time: stage events of the last forward of every step
+    shard.set_timing(True)
+    local_ms = []
+    launches0 = shard.kernel_launches()
+    tr = TimedRegion(stream, flush, args.forwards_per_step)
+    step_ms, clocks, wall = tr.run(run_fwd, args.steps, gpu_index_of(local_rank), barrier=dist.barrier,
+                                   after_step=lambda: local_ms.append(shard.stage_times()["local"]))
+    launches = shard.kernel_launches() - launches0
+    shard.set_timing(False)
+    assert shard.last_device_error() == 0
+    total = max_over_ranks_dist(sum(step_ms), world, dev)
+    n_fwd = args.steps * args.forwards_per_step
+    # end to end: the rank's X rows and the weights in, its Y rows out, per forward
+    Yh = torch.empty_like(Y, device="cpu").pin_memory()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    torch.cuda.synchronize()
-    step_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
+    e2e_ms = []
+    for i in range(args.e2e_steps + 3):
         ev0.record(stream)
-        fwd(X, *W, w.b_g, w.eps, Y)
+        for t, k in zip((X, WQ, WK, WV, wg), names):
+            t.copy_(host[k], non_blocking=True)
+        run_fwd()
+        Yh.copy_(Y, non_blocking=True)
         ev1.record(stream)
         ev1.synchronize()
-        step_ms.append(ev0.elapsed_time(ev1))
-    torch.cuda.synchronize()
-    dist.barrier()
-    total = max_over_ranks_dist(sum(step_ms), world, dev)
-    assert shard.last_device_error() == 0
-    line = {"metric": METRIC, "value": w.E * w.H * args.steps / (total * 1e-3), "unit": UNIT,
+        if i >= 3:
+            e2e_ms.append(ev0.elapsed_time(ev1))
+    e2e_total = max_over_ranks_dist(sum(e2e_ms), world, dev)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    peaks, peak_kind = load_peaks()
+    t_local = float(np.mean(local_ms)) if local_ms else float("nan")
+    line = {"metric": METRIC, "value": w.E * w.H * n_fwd / (total * 1e-3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "strong",
+            "ms_per_step": total / args.steps, "forwards_per_step": args.forwards_per_step,
+            "ms_per_forward": total / n_fwd, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": w.io, "data": "synthetic",
-            "config": {"workload": args.workload if args.scale == 1.0 else f"{args.workload}@scale{args.scale}",
-                       "N": w.N, "E": w.E, "d": w.d, "H": w.H, "r": w.r, "io": w.io,
-                       "parallelism": f"row-sharded x{world} (NCCL: K/V broadcasts, partial S|z all-gather)",
-                       "rows_per_rank": [int(x) for x in np.diff(bounds)],
-                       "l2": "flushed between timed steps (256 MiB write, outside the timed spans)"},
-            "parity_max_rel_err": parity}
+            "config": workload_config(args, w, world, "sharded"),
+            "rows_per_rank_0": plan.b1 - plan.b0, "kv_rows_padded": plan.n_kv,
+            "roofline": roofline_local(w, t_local, peaks, peak_kind, None,
+                                       "stage events of rank 0's local kernel (its own rows), timed region"),
+            "gpu_launches": int(launches),
+            "e2e": {"value": w.E * w.H * len(e2e_ms) / (e2e_total * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": Yh.numel() * Yh.element_size(),
+                    "ms_per_step": e2e_total / len(e2e_ms), "note": "per rank: its X rows and the weights "
+                    "in, its Y rows out, serial on one stream; bytes are rank 0's"},
+            "clocks": clocks, "wall_s_timed_region": wall, "parity_max_rel_err": parity}
+    # the roofline above uses rank 0's rows only: scale its algorithmic bytes to them
+    if plan.b1 > plan.b0:
+        frac_rows = (plan.b1 - plan.b0) / w.N
+        line["roofline"]["note"] = (f"algorithmic bytes of the whole graph; rank 0 holds {frac_rows:.3f} "
+                                    "of the rows and about 1/P of the entries")
     if rank == 0:
         print(json.dumps(line), flush=True)
     shard.close()
+    dist.barrier()
     dist.destroy_process_group()
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
-    ap.add_argument("--workload", default="arxiv")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--scale", type=float, default=1.0,
-                    help="shrink the workload (small profiling captures only; reported lines use 1.0)")
-    ap.add_argument("--no-parity", action="store_true", help="skip the sampled-row oracle check")
-    ap.add_argument("--segment-len", type=int, default=0,
-                    help="segments of this many nodes, each with its own global statistics "
-                         "(a batch of graphs; 0 = one segment over all nodes)")
-    ap.add_argument("--backward", action="store_true",
-                    help="also time the backward pass (glga_backward) of the same forward")
-    ap.add_argument("--block", action="store_true",
-                    help="also time the block around the layer, Z = LayerNorm(X + Y Wo)")
-    ap.add_argument("--sharded", action="store_true",
-                    help="row-sharded forward across the ranks (strong scaling) instead of replicas")
-    ap.add_argument("--dense-sweep", action="store_true",
-                    help="layer forward against dense softmax attention over N and in-degree")
-    ap.add_argument("--sweep", action="store_true",
-                    help="time the forward against N at fixed degree instead (one JSON line)")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.sweep:
-        run_sweep()
-        return
-    if args.dense_sweep:
-        run_dense_sweep()
-        return
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, rank, world)
-        return
-    if args.sharded:
-        run_sharded(args, rank, world, local_rank)
-        return
-
+def run_single(args, rank, world, local_rank, mode):
+    """One process per GPU, each running the whole forward (one GPU, or replicas)."""
     import torch
     import torch.distributed as dist
     from sparse_graph_attention_tcgen05_b200 import glga
@@ -528,8 +672,7 @@ def main():
     dev = torch.device("cuda", local_rank)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     def barrier():
         if world > 1:
@@ -581,7 +724,7 @@ def main():
         import oracle
         csr = (row_ptr.cpu().numpy(), col_idx.cpu().numpy())
         rng = np.random.default_rng(0)
-        rows = np.unique(np.concatenate([rng.choice(w.N, 256, replace=False),
+        rows = np.unique(np.concatenate([rng.choice(w.N, min(256, w.N), replace=False),
                                          np.argsort(np.diff(csr[0]))[-8:]]))
         ref = oracle.forward(w.N, w.d, w.H, w.r, w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps,
                              csr[0], csr[1], rows=rows, seg_ptr=seg)
@@ -592,7 +735,7 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     # ---- eager forwards with the library's stage events: per-stage times, launch count ----
-    n_eager = min(args.steps, 500)
+    n_eager = 100
     layer.set_timing(True)
     launches0 = layer.kernel_launches()
     stage_sum = {k: 0.0 for k in glga.STAGES}
@@ -607,88 +750,72 @@ def main():
         for k, v in layer.stage_times().items():
             stage_sum[k] += v
     launches_per_forward = (layer.kernel_launches() - launches0) / n_eager
-    layer.set_timing(False)
     stages = {k: v / n_eager for k, v in stage_sum.items()}
     eager_total = max_over_ranks(sum(eager_ms))
     eager = {"value": replica_throughput(world, w.E * w.H, eager_total, n_eager), "unit": UNIT,
              "ms_per_step": eager_total / n_eager, "steps": n_eager,
-             "note": "glga_forward called per step, stage events on"}
+             "note": "glga_forward called per forward, stage events on"}
 
-    # ---- timed region: K forwards replayed from a CUDA graph of glga_forward
-    # (Layer.capture: the same six kernels on the same buffers, no host work between
-    # them), L2 flushed between steps; eager calls if the capture is refused ----
-    graph = None
+    # ---- timed region: K steps of R forwards, each a replay of a CUDA graph of
+    # glga_forward (the same kernels on the same buffers, no host work between them) with
+    # the library's stage events inside the graph; eager calls if the capture is refused ----
+    graph, graph_timing = None, False
     try:
-        graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)
-        run_step = graph.replay
-    except RuntimeError as exc:
-        run_step = fwd
-        eager["capture_refused"] = str(exc).splitlines()[0][:200]
+        graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)   # timing still on
+        graph.replay()
+        torch.cuda.synchronize()
+        layer.stage_times()
+        graph_timing = True
+    except (RuntimeError, glga.GLGAError) as exc:
+        eager["capture_with_stage_events"] = str(exc).splitlines()[0][:200]
+        graph = None
+    if graph is None:
+        layer.set_timing(False)
+        try:
+            graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)
+        except RuntimeError as exc:
+            eager["capture_refused"] = str(exc).splitlines()[0][:200]
+            graph = None
+    run_step = graph.replay if graph is not None else fwd
     for _ in range(args.warmup):
         run_step()
-    step_ms = []
-    barrier()
-    torch.cuda.synchronize()
-    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    ids = [v.strip() for v in visible.split(",") if v.strip()]
-    sampler = ClockSampler(ids[local_rank] if local_rank < len(ids) else local_rank)
-    wall0 = time.perf_counter()
-    for _ in range(args.steps):
-        flush.zero_()
-        ev0.record(stream)
-        run_step()
-        ev1.record(stream)
-        ev1.synchronize()
-        step_ms.append(ev0.elapsed_time(ev1))
-    torch.cuda.synchronize()
-    wall = time.perf_counter() - wall0
-    clocks = sampler.stop()
-    barrier()
+    local_ms, fwd_check = [], []
+    tr = TimedRegion(stream, flush, args.forwards_per_step)
+
+    def after():
+        st = layer.stage_times()
+        local_ms.append(st["local"])
+        fwd_check.append(st["forward"] / tr.last_ms)
+    step_ms, clocks, wall = tr.run(run_step, args.steps, gpu_index_of(local_rank),
+                                   barrier=barrier if world > 1 else None,
+                                   after_step=after if graph_timing else None)
+    layer.set_timing(False)
+    # the graph's stage events must span the same forward as the outer events
+    if fwd_check and not 0.8 <= float(np.median(fwd_check)) <= 1.05:
+        eager["graph_stage_events"] = f"rejected (forward span / outer events = {float(np.median(fwd_check)):.3f})"
+        local_ms = []
     graph_ok = graph is not None
     del graph
     assert layer.last_device_error() == 0
-    launches = int(round(launches_per_forward * args.steps))
-
+    n_fwd = args.steps * args.forwards_per_step
+    launches = int(round(launches_per_forward * n_fwd))
     total_ms = max_over_ranks(sum(step_ms))
-    ms_per_step = total_ms / args.steps
-    value = replica_throughput(world, w.E * w.H, total_ms, args.steps)
+    value = replica_throughput(world, w.E * w.H, total_ms, n_fwd)
 
     # ---- end to end through the public API: pinned host -> device, forward, Y -> host ----
-    Yh = torch.empty(w.N, w.D, dtype=dt).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = Yh.numel() * Yh.element_size()
-    e2e_ms = []
-    for i in range(max(args.e2e_steps, 1) + 3):
-        ev0.record(stream)
-        X.copy_(host["X"], non_blocking=True)
-        WQ.copy_(host["W_Q"], non_blocking=True)
-        WK.copy_(host["W_K"], non_blocking=True)
-        WV.copy_(host["W_V"], non_blocking=True)
-        wg.copy_(host["w_g"], non_blocking=True)
-        fwd()
-        Yh.copy_(Y, non_blocking=True)
-        ev1.record(stream)
-        ev1.synchronize()
-        if i >= 3:
-            e2e_ms.append(ev0.elapsed_time(ev1))
-    e2e_total = max_over_ranks(sum(e2e_ms))
-    e2e_step = e2e_total / len(e2e_ms)
-    e2e = {"value": replica_throughput(world, w.E * w.H, e2e_total, len(e2e_ms)), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
+    e2e_ms, h2d, d2h = e2e_pipelined(layer, w, host, dt, dev, args.e2e_steps)
+    e2e_total = max_over_ranks(e2e_ms)
+    e2e = {"value": replica_throughput(world, w.E * w.H, e2e_total, args.e2e_steps), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_total / args.e2e_steps,
+           "note": "Layer.forward per step with its inputs copied in and Y copied out (pinned host "
+                   "buffers); copies on their own streams, double-buffered, overlapping the forwards"}
 
     peaks, peak_kind = load_peaks()
-    B_kern = local_kernel_bytes(w.N, w.E, w.D, s_io)
-    t_local = stages["local"] * 1e-3
-    achieved = B_kern / t_local / 1e9
-    traffic, traffic_note = profiled_traffic(args.workload)
-    roofline = {"bound": "hbm", "kernel": "local_kernel (local softmax branch; writes L)",
-                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "algorithmic_bytes_per_launch": B_kern, "avg_launch_ms": stages["local"],
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s"}
-    if traffic_note:
-        roofline["traffic_note"] = traffic_note
+    if local_ms:
+        t_local, src_t = float(np.mean(local_ms)), "stage events inside the replayed graph, one forward per timed step"
+    else:
+        t_local, src_t = stages["local"], "stage events of the eager forwards"
+    roofline = roofline_local(w, t_local, peaks, peak_kind, profiled_counters(args.workload), src_t)
     # steps a3-a5 (local branch, readout, gate) against the fused-branch byte model
     B_loc = branch_bytes_model(w.N, w.E, w.D, w.H, w.r, s_io)
     t_branch = (stages["local"] + stages["readout"]) * 1e-3
@@ -706,23 +833,19 @@ def main():
                   "hbm_gbs": gemm_bytes / t_gemm / 1e9}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": w.io, "data": "synthetic",
-            "config": {"workload": args.workload if args.scale == 1.0 else f"{args.workload}@scale{args.scale}",
-                       "N": w.N, "E": w.E, "d": w.d, "H": w.H,
-                       "r": w.r, "io": w.io, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed between timed steps (256 MiB write, outside the timed spans)",
-                       "segments": 1 if seg is None else int(seg.shape[0] - 1)},
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "forwards_per_step": args.forwards_per_step, "ms_per_forward": total_ms / n_fwd,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.io,
+            "data": "synthetic", "config": workload_config(args, w, world, mode, seg),
             "roofline": roofline, "local_branch_a3_a5": branch, "projection": projection,
             "stages_ms": stages, "create": create, "gpu_launches": launches,
-            "e2e": e2e, "eager": eager, "timed_region": "CUDA graph replay of glga_forward" if graph_ok
-            else "eager glga_forward", "clocks": clocks, "parity_max_rel_err": parity,
-            "wall_s_timed_region": wall}
+            "e2e": e2e, "eager": eager, "timed_region": ("CUDA graph replays of glga_forward" if graph_ok
+                                                         else "eager glga_forward"),
+            "clocks": clocks, "parity_max_rel_err": parity, "wall_s_timed_region": wall}
     if args.block:
-        line["block"] = time_block(layer, w, X, Y, dt, dev, flush, stream, args.steps, peaks)
+        line["block"] = time_block(layer, w, X, Y, dt, dev, flush, stream, 200, peaks)
     if args.backward:
-        line["backward"] = time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream,
-                                         max(10, args.steps // 10))
+        line["backward"] = time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, 50)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, (row_ptr.cpu().numpy(), col_idx.cpu().numpy()))
     if rank == 0:
@@ -730,6 +853,58 @@ def main():
     layer.close()
     if world > 1:
         dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--forwards-per-step", type=int, default=300,
+                    help="forwards per timed step (each with its own L2 flush and events)")
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default="arxiv")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="shrink the workload (small profiling captures only; reported lines use 1.0)")
+    ap.add_argument("--no-parity", action="store_true", help="skip the sampled-row oracle check")
+    ap.add_argument("--segment-len", type=int, default=0,
+                    help="segments of this many nodes, each with its own global statistics "
+                         "(a batch of graphs; 0 = one segment over all nodes)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward pass (glga_backward) of the same forward")
+    ap.add_argument("--block", action="store_true",
+                    help="also time the block around the layer, Z = LayerNorm(X + Y Wo)")
+    ap.add_argument("--sharded", action="store_true",
+                    help="the row-sharded forward also on one rank (the default for more than one)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with more than one rank, every rank runs the whole forward (weak scaling)")
+    ap.add_argument("--dense-sweep", action="store_true",
+                    help="layer forward against dense softmax attention over N and in-degree")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the forward against N at fixed degree instead (one JSON line)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    args.forwards_per_step = max(args.forwards_per_step, 1)
+    if args.sweep:
+        run_sweep()
+        return
+    if args.dense_sweep:
+        run_dense_sweep()
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    mode = run_mode(args, world)
+    if mode == "sharded":
+        run_sharded(args, rank, world, local_rank)
+    else:
+        run_single(args, rank, world, local_rank, mode)
 
 
 if __name__ == "__main__":

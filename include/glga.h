@@ -75,8 +75,8 @@ typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
  * GLGA_ERR_OOM (a test hook for the clean-up path); 0 disables it.
  * backward != 0 allocates the workspaces of glga_backward at create (a transposed CSR,
  * chunk lists of the rows with more than 64 entries, a second stream and fp32 buffers of
- * about N*(6*H*r + 4*H + 1) floats; for bf16 layers also a cuBLAS handle, opened at run
- * time, with a 32 MiB workspace and an fp32 copy of X for the weight-gradient GEMM);
+ * about N*(6*H*r + 4*H + 1) floats; for bf16 layers with d a multiple of 8 also the
+ * range partials of the tensor-core weight-gradient GEMM, about num_SMs*d*3*H*r floats);
  * glga_forward on such a context also stores each row's softmax log-sum-exp per head for
  * the backward.  Whole-graph, one-segment contexts
  * with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).                             */
@@ -245,7 +245,11 @@ GLGA_API glga_status glga_get_intermediates(const glga_ctx *ctx, void *Q, void *
  * writes up to n_max durations in milliseconds (host) in this order:
  *   0 weight packing and input preparation, 1 projection GEMM, 2 global statistics
  *   (tensor-core partials + ordered reduction), 3 local branch (per-target softmax
- *   kernel), 4 readout GEMM with the fused gate blend, 5 whole forward.
+ *   kernel), 4 readout GEMM with the fused gate blend, 5 whole forward.  Row-sharded
+ *   contexts record them in glga_forward_begin and glga_forward_end: stage 2 then also
+ *   spans the caller's exchange between the two calls.  A forward recorded into a CUDA
+ *   graph with timing on records the events as event record nodes: glga_stage_times
+ *   after a replay reports that replay's stages.
  * Returns the number of values written through *n_written.                            */
 GLGA_API glga_status glga_set_timing(glga_ctx *ctx, int enable);
 GLGA_API glga_status glga_stage_times(glga_ctx *ctx, float *ms, int32_t n_max, int32_t *n_written);
@@ -274,13 +278,24 @@ GLGA_API glga_status glga_last_device_error(glga_ctx *ctx, void *stream);
  * that loads the library holds it until the process exits.  Limit: one row range needs
  * H*r*(r+1)*4 bytes, which must fit in those 2 MiB; larger shapes return
  * GLGA_ERR_UNSUPPORTED before any device work.  The first call on a device looks up the
- * array's device address and caches it; make that first call before any stream capture.
+ * array's device address and caches it (again when the device's CUDA context has changed,
+ * e.g. after cudaDeviceReset); make that first call before any stream capture.
  * All calls share the array and it keeps the last call's contents: each call writes every
  * partial sum it later reads, so nothing needs clearing, but calls that overlap on the
  * GPU (other streams or threads) race on it; the caller must order them.  No cudaMalloc,
- * cudaFree or allocating library routine is called.                                   */
+ * cudaFree or allocating library routine is called.  The call is asynchronous: a bounded
+ * wait inside its kernel that gave up (the S and z of that call are then incomplete) is
+ * reported by glga_global_stats_static_error.                                           */
 GLGA_API glga_status glga_global_stats_static(const void *KV, int64_t N, int32_t H, int32_t r,
                                               glga_dtype io, float *Sz, void *stream);
+
+/* glga_global_stats_static_error -- synchronises `stream`, then reports and clears the
+ * device-side flag that the glga_global_stats_static calls on the current device raise:
+ * GLGA_OK, GLGA_ERR_TIMEOUT (a bounded wait of one of the calls since the last report gave
+ * up, so its S and z are incomplete) or GLGA_ERR_DEVICE.  One flag per device, shared by
+ * all those calls; it stays raised until this call clears it.  Allocates nothing.  The
+ * paper has no counterpart (it is the error path of the entry point above).           */
+GLGA_API glga_status glga_global_stats_static_error(void *stream);
 
 /* Static strings; never NULL. */
 /* Test entry points of the failure paths (the pages have no counterpart).
@@ -291,11 +306,16 @@ GLGA_API glga_status glga_global_stats_static(const void *KV, int64_t N, int32_t
  * thread then sets the context's device flag and returns, so the next
  * glga_last_device_error reports GLGA_ERR_TIMEOUT and the context stays usable.
  *
+ * glga_debug_static_bounded_wait -- the same probe for the flag of the
+ * glga_global_stats_static calls on the current device (reported by
+ * glga_global_stats_static_error).
+ *
  * glga_debug_set_col_idx -- overwrites entry e of the context's CSR copy with `value`,
  * skipping glga_create's validation, so that the device-side checks of a context made
  * with debug_checks != 0 can be exercised.  Refused (GLGA_ERR_INVALID_ARG) when the
  * context was made without debug_checks or e is outside [0, E).  Stream-ordered.      */
 GLGA_API glga_status glga_debug_bounded_wait(glga_ctx *ctx, int64_t limit_ns, void *stream);
+GLGA_API glga_status glga_debug_static_bounded_wait(int64_t limit_ns, void *stream);
 GLGA_API glga_status glga_debug_set_col_idx(glga_ctx *ctx, int64_t e, int32_t value, void *stream);
 
 GLGA_API const char *glga_status_string(glga_status s);

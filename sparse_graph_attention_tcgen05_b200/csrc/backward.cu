@@ -17,17 +17,15 @@
 // The target-grouped terms (dq) walk the forward CSR; the source-grouped terms (dk, dv)
 // walk a transposed CSR built at create, so every sum has a fixed order and there are no
 // atomics (two runs give identical bits).  CUDA-core kernels with fp32 arithmetic (one
-// warp per row or per 32-edge chunk of a heavy row, register-tiled GEMMs for the weight
-// and input gradients, which bf16 layers run on cuBLAS's TF32 tensor-core GEMMs instead);
-// gradients are fp32.  The log-sum-exp of each row's scores comes from the forward.
-#include <dlfcn.h>
-
+// warp per row or per 32-edge chunk of a heavy row); the two dense GEMMs dW = X^T dZ and
+// dX = dZ W^T run on the tcgen05 tensor cores for bf16 layers (bwd_dw_tc_kernel with bf16
+// operands, the persistent projection GEMM on kind::tf32) and as register-tiled fp32
+// CUDA-core GEMMs for fp32 layers; gradients are fp32.  The log-sum-exp of each row's
+// scores comes from the forward.
 #include <algorithm>
 #include <cmath>
 #include <type_traits>
 #include <vector>
-
-#include <cublas_v2.h>   // types and enums only: the library is opened at run time
 
 #include "glga_internal.cuh"
 
@@ -1048,47 +1046,6 @@ int lane_features(int D) {
     return e;
 }
 
-// cuBLAS, opened on first use by a context made for the backward pass (so the forward
-// never depends on it).  dW = X^T [dQ | dK | dV] and dX = dZ W^T are plain dense GEMMs;
-// for bf16 layers they run there on the TF32 tensor cores (fp32 operands rounded to
-// 10-bit mantissas, fp32 accumulation), for fp32 layers on the exact-fp32 SIMT kernels.
-struct CublasApi {
-    bool ok = false;
-    cublasStatus_t (*create)(cublasHandle_t *) = nullptr;
-    cublasStatus_t (*destroy)(cublasHandle_t) = nullptr;
-    cublasStatus_t (*set_stream)(cublasHandle_t, cudaStream_t) = nullptr;
-    cublasStatus_t (*set_workspace)(cublasHandle_t, void *, size_t) = nullptr;
-    cublasStatus_t (*gemm_ex)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int, const void *,
-                              const void *, cudaDataType, int, const void *, cudaDataType, int, const void *,
-                              void *, cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t) = nullptr;
-};
-
-const CublasApi &cublas_api() {
-    static const CublasApi api = [] {
-        CublasApi a;
-        void *lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-        if (!lib) lib = dlopen("/usr/local/cuda/lib64/libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-        if (!lib) return a;
-        a.create = reinterpret_cast<decltype(a.create)>(dlsym(lib, "cublasCreate_v2"));
-        a.destroy = reinterpret_cast<decltype(a.destroy)>(dlsym(lib, "cublasDestroy_v2"));
-        a.set_stream = reinterpret_cast<decltype(a.set_stream)>(dlsym(lib, "cublasSetStream_v2"));
-        a.set_workspace = reinterpret_cast<decltype(a.set_workspace)>(dlsym(lib, "cublasSetWorkspace_v2"));
-        a.gemm_ex = reinterpret_cast<decltype(a.gemm_ex)>(dlsym(lib, "cublasGemmEx"));
-        a.ok = a.create && a.destroy && a.set_stream && a.set_workspace && a.gemm_ex;
-        return a;
-    }();
-    return api;
-}
-
-constexpr size_t kCublasWorkspace = size_t(32) << 20;
-
-// Xf = X as fp32 (the TF32 GEMM takes both operands in fp32).
-__global__ void bwd_x_to_f32_kernel(const __nv_bfloat16 *__restrict__ X, int64_t n, float *__restrict__ Xf) {
-    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < n;
-         o += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        Xf[o] = __bfloat162float(X[o]);
-}
-
 unsigned warp_grid(int64_t n) {
     return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256)));
 }
@@ -1220,40 +1177,231 @@ void plan_rows(const std::vector<int32_t> &rp, RowPlan &p) {
 
 int64_t ceil_parts(int64_t N, int64_t want) { return std::max<int64_t>(1, std::min<int64_t>(want, N)); }
 
-// The two GEMMs on cuBLAS (column-major view of the row-major buffers; every leading
-// dimension a multiple of 4 floats):
-//   dW3[a][k] (k < 3D, row stride 3D) = sum_i dZ[i][k] Xf[i][a]:
-//     C [3D x d], ldc 3D = A [3D x N] (dZ^T, lda dz_ld) * B^T (B = Xf^T [d x N], ldb d)
-//   dX [N x d] = dZ Wall^T over all dz_ld columns (the padding columns of dZ and Wall are
-//     zero):  C [d x N], ldc d = A^T (A = Wall^T [dz_ld x d]) * B (B = dZ^T [dz_ld x N])
-glga_status cublas_gemms(Ctx *c, float *dX, cudaStream_t s) {
-    const CublasApi &api = cublas_api();
-    cublasHandle_t h = static_cast<cublasHandle_t>(c->bw_cublas);
-    const int N = static_cast<int>(c->N), d = c->d, D = c->D;
-    const int ld = static_cast<int>(c->bw_dz_ld);
-    const float one = 1.f, zero = 0.f;
-    cublasStatus_t e = api.set_stream(h, s);
-    if (e == CUBLAS_STATUS_SUCCESS)
-        e = api.gemm_ex(h, CUBLAS_OP_N, CUBLAS_OP_T, 3 * D, d, N, &one, c->bw_dZ, CUDA_R_32F, ld, c->bw_Xf,
-                        CUDA_R_32F, d, &zero, c->bw_dW3, CUDA_R_32F, 3 * D, CUBLAS_COMPUTE_32F_FAST_TF32,
-                        CUBLAS_GEMM_DEFAULT);
-    if (e == CUBLAS_STATUS_SUCCESS)
-        e = api.gemm_ex(h, CUBLAS_OP_T, CUBLAS_OP_N, d, N, ld, &one, c->bw_Wall, CUDA_R_32F, ld, c->bw_dZ,
-                        CUDA_R_32F, ld, &zero, dX, CUDA_R_32F, d, CUBLAS_COMPUTE_32F_FAST_TF32,
-                        CUBLAS_GEMM_DEFAULT);
-    if (e != CUBLAS_STATUS_SUCCESS) {
-        set_error("glga_backward: cuBLAS GEMM failed (status %d)", static_cast<int>(e));
-        return GLGA_ERR_CUDA;
+// ---------------------------------------------------------------------------------------
+// Weight gradient of bf16 layers on the tcgen05 tensor cores:
+//   part[p][a][k] = sum over the rows i of range p of X[i][a] dZ[i][k]   (a < d, k < 3D)
+// for 128 x 128 blocks (block fa of 128 input features, block fb of 128 dZ columns); the
+// node index is the contraction dimension.  Per 64-row stage a TMA producer loads the X
+// tile [64][128] (bf16, two 64-column boxes, 128-byte swizzle) and the dZ tile [64][128]
+// (float32, four 32-column boxes); warps 0-7 round dZ to bf16 into a third tile laid out
+// as TMA lays out bf16 (rows past the range are zeroed); one thread issues tcgen05.mma
+// with both operands MN-major (X^T as A, the bf16 dZ tile as B), accumulating the block
+// in TMEM over the range in row order.  Warps 0-3 write the block to the range's partial
+// sums, which bwd_sum_parts_kernel adds in range order (the result is the same on every
+// call).  Every mbarrier wait is bounded: on expiry the kernel raises the context's flag,
+// lets its copies land and returns.
+constexpr int kDwRows = 64;
+constexpr int kDwStages = 3;
+constexpr int kDwWorkers = 256;
+constexpr int kDwProd = 8, kDwMma = 9, kDwThreads = 320;
+constexpr uint32_t kDwBox = kDwRows * 128;                 // one 64-row box of 128-byte rows
+constexpr uint32_t kDwXBytes = 2 * kDwBox;                 // X tile (bf16)
+constexpr uint32_t kDwZBytes = 4 * kDwBox;                 // dZ tile (float32)
+constexpr uint32_t kDwStage = kDwXBytes + kDwZBytes + 2 * kDwBox;   // + dZ rounded to bf16
+
+struct DwParams {
+    int64_t N;
+    int32_t d, Kc;            // X columns; dZ columns in use (3D)
+    int64_t rows_per_part;
+    float *part;              // [P][d][Kc]
+    unsigned *flag;
+};
+
+__global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                                  const __grid_constant__ CUtensorMap tmZ,
+                                                                  DwParams p) {
+    extern __shared__ uint8_t dsmem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kDwStages];
+    __shared__ __align__(8) uint64_t ready_bar[kDwStages];
+    __shared__ __align__(8) uint64_t empty_bar[kDwStages];
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_base_sh;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int part = blockIdx.x, fa = blockIdx.y, fb = blockIdx.z;
+    const int64_t r0 = static_cast<int64_t>(part) * p.rows_per_part;
+    const int64_t r1 = std::min<int64_t>(p.N, r0 + p.rows_per_part);
+    const int ntiles = r1 > r0 ? static_cast<int>(ceil_div(r1 - r0, kDwRows)) : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDwStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&ready_bar[s], kDwWorkers);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&done_bar, 1);
+        fence_mbar_init();
     }
-    return GLGA_OK;
+    if (warp == kDwMma) {
+        tmem_alloc(&tmem_base_sh, 128u);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == kDwProd) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmX);
+            tma_prefetch_desc(&tmZ);
+            int issued = 0;
+            RingPos rp;
+            bool ok = true;
+            for (int it = 0; it < ntiles; ++it, rp.next(kDwStages)) {
+                const int s = rp.slot;
+                if (it >= kDwStages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = smem + static_cast<size_t>(s) * kDwStage;
+                mbar_arrive_expect_tx(&full_bar[s], kDwXBytes + kDwZBytes);
+                const int32_t y = static_cast<int32_t>(r0 + static_cast<int64_t>(it) * kDwRows);
+                for (int b = 0; b < 2; ++b) tma_load_2d(st + b * kDwBox, &tmX, &full_bar[s], fa * 128 + b * 64, y);
+                for (int b = 0; b < 4; ++b)
+                    tma_load_2d(st + kDwXBytes + b * kDwBox, &tmZ, &full_bar[s], fb * 128 + b * 32, y);
+                ++issued;
+            }
+            if (!ok) {
+                atomicOr(p.flag, kDevErrTimeout);
+                for (int it = std::max(0, issued - kDwStages); it < issued; ++it)
+                    mbar_wait_bounded(&full_bar[it % kDwStages], static_cast<uint32_t>(it / kDwStages) & 1u);
+            }
+        }
+    } else if (warp == kDwMma) {
+        if (lane == 0) {
+            const uint32_t idesc = instr_desc(128, 128, 1u, true, true);
+            bool ok = true;
+            RingPos rp;
+            for (int it = 0; it < ntiles; ++it, rp.next(kDwStages)) {
+                const int s = rp.slot;
+                if (!mbar_wait_bounded(&ready_bar[s], rp.phase)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xb = smem_u32(smem + static_cast<size_t>(s) * kDwStage);
+                const uint32_t bb = xb + kDwXBytes + kDwZBytes;
+#pragma unroll
+                for (int ks = 0; ks < kDwRows / 16; ++ks) {
+                    const uint32_t off = ks * 16 * 128;
+                    umma_bf16(tmem, smem_desc(xb + off, kDwBox, 1024, 2), smem_desc(bb + off, kDwBox, 1024, 2),
+                              idesc, (it | ks) != 0);
+                }
+                umma_commit(&empty_bar[s]);
+            }
+            if (!ok) atomicOr(p.flag, kDevErrTimeout);
+            umma_commit(&done_bar);
+        }
+    } else {
+        // ---------------- warps 0-7: dZ float32 -> bf16 (zero past the range) ----------
+        bool ok = true;
+        RingPos rp;
+        for (int it = 0; it < ntiles && ok; ++it, rp.next(kDwStages)) {
+            const int s = rp.slot;
+            if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
+                ok = false;
+                break;
+            }
+            const uint8_t *z = smem + static_cast<size_t>(s) * kDwStage + kDwXBytes;
+            uint8_t *bt = smem + static_cast<size_t>(s) * kDwStage + kDwXBytes + kDwZBytes;
+            const int64_t y0 = r0 + static_cast<int64_t>(it) * kDwRows;
+            // one 16-byte chunk of the bf16 tile (8 consecutive columns of one row) per step
+            for (int cidx = threadIdx.x; cidx < kDwRows * 16; cidx += kDwWorkers) {
+                const int k = cidx >> 4, ch = cidx & 15;
+                const int bo = ch >> 3, co = ch & 7;            // bf16 box, chunk in its row
+                const int g0 = bo * 64 + co * 8;                // first column in the tile
+                const int bi = g0 >> 5, j0 = (g0 & 31) >> 2;    // float32 box, its first chunk
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if (y0 + k < r1) {
+                    const uint8_t *zr = z + bi * kDwBox + k * 128;
+                    const float4 a = *reinterpret_cast<const float4 *>(zr + ((j0 ^ (k & 7)) * 16));
+                    const float4 b = *reinterpret_cast<const float4 *>(zr + (((j0 + 1) ^ (k & 7)) * 16));
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y), h1 = __floats2bfloat162_rn(a.z, a.w);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y), h3 = __floats2bfloat162_rn(b.z, b.w);
+                    w = make_uint4(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1),
+                                   *reinterpret_cast<uint32_t *>(&h2), *reinterpret_cast<uint32_t *>(&h3));
+                }
+                *reinterpret_cast<uint4 *>(bt + bo * kDwBox + k * 128 + ((co ^ (k & 7)) * 16)) = w;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&ready_bar[s]);
+        }
+        if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+    }
+    __syncwarp();
+
+    if (warp < 4) {
+        // ---------------- epilogue: the 128 x 128 block -> the range's partial sums ---------
+        const bool done = ntiles == 0 ? true : mbar_wait_bounded(&done_bar, 0);
+        tc_fence_after();
+        if (!done && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+        const bool have = ntiles > 0 && done;
+        const int a = fa * 128 + warp * 32 + lane;         // TMEM lane = input feature
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        float *dst = p.part + (static_cast<int64_t>(part) * p.d + a) * p.Kc;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + q * 32, v);
+            tmem_ld_wait();
+            const int k0 = fb * 128 + q * 32;
+            if (a < p.d) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (k0 + j < p.Kc) dst[k0 + j] = have ? __uint_as_float(v[j]) : 0.f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kDwMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128u);
+    }
+}
+
+// Whether the bf16 tensor-core GEMMs serve this context's backward: bf16 layers whose X
+// rows are 16-byte multiples (TMA).  Other layers keep the CUDA-core GEMM kernels.
+bool bwd_tc_gemms(const Ctx *c) { return c->io == GLGA_BF16 && c->d % 8 == 0 && c->N > 0; }
+
+// dW (columns < 3D) and dX of a bf16 layer on the tensor cores:
+//   dW3 [d][3D] = sum of the range partials of bwd_dw_tc_kernel, in range order;
+//   dX [N][d] = dZ [N][3D + 1] Wall^T, the persistent GEMM on kind::tf32 (fp32 dZ and
+//   Wall read as tf32).
+glga_status tc_gemms(Ctx *c, const void *X, float *dX, cudaStream_t s) {
+    const int64_t N = c->N;
+    const int d = c->d, D = c->D, Kc = 3 * D;
+    CUtensorMap mx, mz;
+    glga_status st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(d),
+                                    static_cast<uint64_t>(N), static_cast<uint64_t>(d) * 2, 64, kDwRows);
+    if (st == GLGA_OK)
+        st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dZ, static_cast<uint64_t>(Kc),
+                            static_cast<uint64_t>(N), static_cast<uint64_t>(c->bw_dz_ld) * 4, 32, kDwRows);
+    if (st != GLGA_OK) return st;
+    DwParams p;
+    p.N = N;
+    p.d = d;
+    p.Kc = Kc;
+    p.rows_per_part = c->bw_dwtc_rpp;
+    p.part = c->bw_dwtc_part;
+    p.flag = c->dev_flag;
+    const size_t smem = static_cast<size_t>(kDwStages) * kDwStage + 1024;
+    GLGA_CUDA(cudaFuncSetAttribute(bwd_dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem)));
+    const dim3 grid(static_cast<unsigned>(c->bw_dwtc_parts), static_cast<unsigned>(ceil_div(d, 128)),
+                    static_cast<unsigned>(ceil_div(Kc, 128)));
+    bwd_dw_tc_kernel<<<grid, kDwThreads, smem, s>>>(mx, mz, p);
+    GLGA_CUDA(cudaGetLastError());
+    const int64_t total = static_cast<int64_t>(d) * Kc;
+    bwd_sum_parts_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 4096)), 256, 0, s>>>(
+        c->bw_dwtc_part, c->bw_dwtc_parts, total, c->bw_dW3);
+    GLGA_CUDA(cudaGetLastError());
+    return gemm_nt_f32out(c, GLGA_F32, c->bw_dZ, N, c->bw_dz_ld, c->bw_Wall, d, c->bw_dz_ld, Kc + 1, dX, d, s);
 }
 
 }  // namespace
-
-void backward_release(Ctx *c) {
-    if (c->bw_cublas) cublas_api().destroy(static_cast<cublasHandle_t>(c->bw_cublas));
-    c->bw_cublas = nullptr;
-}
 
 glga_status backward_setup(Ctx *c, cudaStream_t s) {
     if (!c->opts.backward) return GLGA_OK;
@@ -1298,18 +1446,17 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
                    static_cast<size_t>(c->bw_wparts) * c->d * (3 * D + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dbg_part), static_cast<size_t>(c->bw_wparts) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Wall), static_cast<size_t>(c->d) * c->bw_dz_ld * f));
-    if (st == GLGA_OK && c->io == GLGA_BF16 && N > 0 && N <= INT32_MAX && cublas_api().ok) {
-        cublasHandle_t h = nullptr;
-        if (cublas_api().create(&h) == CUBLAS_STATUS_SUCCESS) {
-            c->bw_cublas = h;
-            BTRY(dev_alloc(c, &c->bw_cublas_ws, kCublasWorkspace));
-            BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Xf), static_cast<size_t>(N) * c->d * f));
-            BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dW3), static_cast<size_t>(c->d) * 3 * D * f));
-            if (st == GLGA_OK && cublas_api().set_workspace(h, c->bw_cublas_ws, kCublasWorkspace) != CUBLAS_STATUS_SUCCESS) {
-                set_error("glga_create: cuBLAS workspace");
-                st = GLGA_ERR_CUDA;
-            }
-        }
+    if (bwd_tc_gemms(c)) {
+        // weight-gradient partials of the tensor-core GEMM: 64-row-aligned ranges, about
+        // one thread block per SM over the (feature block, column block) grid
+        const int64_t blocks = ceil_div(c->d, 128) * ceil_div(3 * D, 128);
+        const int64_t want = std::max<int64_t>(1, c->num_sms / blocks);
+        const int64_t rpp = ceil_div(ceil_div(N, want), kDwRows) * kDwRows;
+        c->bw_dwtc_rpp = rpp;
+        c->bw_dwtc_parts = static_cast<int32_t>(ceil_div(N, rpp));
+        BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dwtc_part),
+                       static_cast<size_t>(c->bw_dwtc_parts) * c->d * 3 * D * f));
+        BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dW3), static_cast<size_t>(c->d) * 3 * D * f));
     }
 #undef BTRY
     if (st != GLGA_OK) return st;
@@ -1404,14 +1551,12 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
             launch_local_bwd<T>(c, Q, KV, isr, Dz, s, c->bw_side);                                        \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_join, c->bw_side));                                        \
             GLGA_CUDA(cudaStreamWaitEvent(s, c->bw_ev_join, 0));                                          \
-            if (c->bw_cublas) {                                                                           \
+            if (bwd_tc_gemms(c)) {                                                                        \
                 bwd_pack_w_kernel<T><<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d * Dz, 256), 1024)), \
                                        256, 0, s>>>(static_cast<const T *>(WQ), static_cast<const T *>(WK), \
                                                     static_cast<const T *>(WV), static_cast<const T *>(wg), \
                                                     d, D, Dz, c->bw_Wall);                                  \
-                bwd_x_to_f32_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(N * d, 256), 4096)),  \
-                                      256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), N * d, c->bw_Xf); \
-                const glga_status gs = cublas_gemms(c, dX, s);                                            \
+                const glga_status gs = tc_gemms(c, X, dX, s);                                             \
                 if (gs != GLGA_OK) return gs;                                                             \
                 bwd_dwg_kernel<T><<<dim3(static_cast<unsigned>(c->bw_wparts), ceil_div(d, 32)), 256, 0, s>>>( \
                     static_cast<const T *>(X), c->bw_dZ, N, d, Dz, 3 * D, Dc, wrpp, c->bw_dw_part,         \
@@ -1438,7 +1583,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
 #undef BWD_LAUNCHES
     if (N > 0) {
         bwd_dw_reduce_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(wtotal, 256), 4096)), 256, 0, s>>>(
-            c->bw_dw_part, c->bw_wparts, c->bw_cublas ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
+            c->bw_dw_part, c->bw_wparts, bwd_tc_gemms(c) ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
         bwd_dbg_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, c->bw_wparts, db_g);
     } else {
         GLGA_CUDA(cudaMemsetAsync(dWQ, 0, static_cast<size_t>(d) * D * sizeof(float), s));
@@ -1449,7 +1594,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
     }
     // (N == 0: no dS | dz to sum, and every gradient is zero)
     GLGA_CUDA(cudaGetLastError());
-    c->launches += N > 0 ? (c->bw_cublas ? 10 : 11) + local_bwd_launches(c) : 0;
+    c->launches += N > 0 ? (bwd_tc_gemms(c) ? 12 : 11) + local_bwd_launches(c) : 0;
     return GLGA_OK;
 }
 

@@ -31,11 +31,29 @@ __global__ void bounded_wait_probe_kernel(unsigned *flag, uint64_t limit_ns) {
 }
 }  // namespace
 
+glga_status launch_bounded_wait_probe(unsigned *flag, uint64_t limit_ns, cudaStream_t s) {
+    bounded_wait_probe_kernel<<<1, 32, 0, s>>>(flag, limit_ns);
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
+}
+
 void set_error(const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
     vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
     va_end(ap);
+}
+
+glga_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? GLGA_OK : cuda_fail(e, "CUDA call"); }
+
+cudaError_t record_stage(Ctx *c, int stage, cudaStream_t s) {
+    // while the stream is being captured into a CUDA graph the event becomes an event
+    // record node, so every replay of the graph records it
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return e;
+    if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(c->ev[stage], s, cudaEventRecordExternal);
+    return cudaEventRecord(c->ev[stage], s);
 }
 
 glga_status cuda_fail(cudaError_t e, const char *what) {
@@ -73,7 +91,6 @@ glga_status dev_alloc(Ctx *c, void **p, size_t bytes) {
 static void release_ctx(Ctx *c) {
     if (!c) return;
     if (c->kv_external) c->KV = nullptr;   // the caller's buffer
-    backward_release(c);
     void *ptrs[] = {c->row_ptr, c->col_idx, c->warp_rows, c->cta_rows, c->split_rows,
                     c->chunk_row, c->chunk_begin, c->chunk_ticket, c->chunk_part, c->Wt,
                     c->Xp, c->Q, c->KV, c->t, c->Spart, c->Sz, c->Bro, c->L, c->task_start,
@@ -82,7 +99,7 @@ static void release_ctx(Ctx *c) {
                     c->bw_dg, c->bw_lse, c->bw_Dd, c->bw_dZ, c->bw_dsz_part, c->bw_dSz,
                     c->bw_dw_part, c->bw_q_rows, c->bw_k_rows, c->bw_ST, c->bw_dST, c->bw_Wall, c->bw_dbg_part,
                     c->bw_dSc, c->bw_q_chunks, c->bw_k_chunks, c->bw_q_cptr, c->bw_k_cptr,
-                    c->bw_q_part, c->bw_kv_part, c->bw_cublas_ws, c->bw_Xf, c->bw_dW3, c->dev_flag};
+                    c->bw_q_part, c->bw_kv_part, c->bw_dwtc_part, c->bw_dW3, c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)
@@ -337,7 +354,7 @@ glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void
     if (c->timing) {
         for (auto &ev : c->ev)
             if (!ev) GLGA_CUDA(cudaEventCreate(&ev));
-        GLGA_CUDA(cudaEventRecord(c->ev[kStagePrep], s));
+        GLGA_CUDA(record_stage(c, kStagePrep, s));
     }
     // NVTX ranges mark the host-side enqueue of each stage (visible to profilers that
     // attach an NVTX tool; no-ops otherwise)
@@ -351,26 +368,26 @@ glga_status glga_forward(glga_ctx *h, const void *X, const void *W_Q, const void
         st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, c->timing);
     }
     if (st != GLGA_OK) return st;
-    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageStats], s));
+    if (c->timing) GLGA_CUDA(record_stage(c, kStageStats, s));
     {
         Range r("glga.global_stats");
         st = stats_run(c, s);
     }
     if (st != GLGA_OK) return st;
-    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageLocal], s));
+    if (c->timing) GLGA_CUDA(record_stage(c, kStageLocal, s));
     {
         Range r("glga.local");
         st = local_run(c, s);
     }
     if (st != GLGA_OK) return st;
-    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageReadout], s));
+    if (c->timing) GLGA_CUDA(record_stage(c, kStageReadout, s));
     {
         Range r("glga.readout");
         st = readout_run(c, b_g, eps, Y, s);
     }
     if (st != GLGA_OK) return st;
     if (c->timing) {
-        GLGA_CUDA(cudaEventRecord(c->ev[kStageEnd], s));
+        GLGA_CUDA(record_stage(c, kStageEnd, s));
         c->ev_recorded = true;
     }
     return GLGA_OK;
@@ -389,8 +406,14 @@ glga_status glga_forward_begin(glga_ctx *h, const void *X, const void *W_Q, cons
         return GLGA_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (c->timing) {
+        for (auto &ev : c->ev)
+            if (!ev) GLGA_CUDA(cudaEventCreate(&ev));
+        GLGA_CUDA(record_stage(c, kStagePrep, s));
+    }
     nvtxRangePushA("glga_forward_begin");
-    glga_status st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, false);
+    glga_status st = projection_run(c, X, W_Q, W_K, W_V, w_g, s, c->timing);
+    if (st == GLGA_OK && c->timing) st = cuda_ok(record_stage(c, kStageStats, s));
     if (st == GLGA_OK) st = stats_run_partial(c, own_partial, s);
     nvtxRangePop();
     return st;
@@ -412,10 +435,20 @@ glga_status glga_forward_end(glga_ctx *h, const float *partials, int32_t P, floa
         return GLGA_ERR_INVALID_ARG;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (c->timing && !c->ev[kStagePrep]) {
+        set_error("glga_forward_end: timing is on but glga_forward_begin ran without it");
+        return GLGA_ERR_INVALID_ARG;
+    }
     nvtxRangePushA("glga_forward_end");
     glga_status st = stats_finish(c, partials, P, s);
+    if (st == GLGA_OK && c->timing) st = cuda_ok(record_stage(c, kStageLocal, s));
     if (st == GLGA_OK) st = local_run(c, s);
+    if (st == GLGA_OK && c->timing) st = cuda_ok(record_stage(c, kStageReadout, s));
     if (st == GLGA_OK) st = readout_run(c, b_g, eps, Y, s);
+    if (st == GLGA_OK && c->timing) {
+        st = cuda_ok(record_stage(c, kStageEnd, s));
+        c->ev_recorded = st == GLGA_OK;
+    }
     nvtxRangePop();
     return st;
 }
@@ -597,10 +630,8 @@ glga_status glga_debug_bounded_wait(glga_ctx *h, int64_t limit_ns, void *stream)
         set_error("glga_debug_bounded_wait: need a context and 1e3 <= limit_ns <= 1e10");
         return GLGA_ERR_INVALID_ARG;
     }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    bounded_wait_probe_kernel<<<1, 32, 0, s>>>(h->c.dev_flag, static_cast<uint64_t>(limit_ns));
-    GLGA_CUDA(cudaGetLastError());
-    return GLGA_OK;
+    return launch_bounded_wait_probe(h->c.dev_flag, static_cast<uint64_t>(limit_ns),
+                                     static_cast<cudaStream_t>(stream));
 }
 
 glga_status glga_debug_set_col_idx(glga_ctx *h, int64_t e, int32_t value, void *stream) {

@@ -21,6 +21,7 @@ namespace glga {
 // ---------------------------------------------------------------------------------------
 void set_error(const char *fmt, ...);
 glga_status cuda_fail(cudaError_t e, const char *what);
+glga_status cuda_ok(cudaError_t e);   // GLGA_OK, or cuda_fail's status for an error
 
 #define GLGA_CUDA(call)                                                    \
     do {                                                                   \
@@ -139,10 +140,10 @@ struct Ctx {
     int64_t bw_nq_chunks = 0, bw_nk_chunks = 0;
     float *bw_q_part = nullptr, *bw_kv_part = nullptr;  // chunk shares
     cudaStream_t bw_side = nullptr;                   // second stream of the backward (source side)
-    void *bw_cublas = nullptr;                        // cuBLAS handle (bf16 layers), or null
-    void *bw_cublas_ws = nullptr;                     // its workspace
-    float *bw_Xf = nullptr;                           // [N][d] fp32 copy of X for the dW GEMM
-    float *bw_dW3 = nullptr;                          // [d][3D] the dW GEMM's output
+    float *bw_dwtc_part = nullptr;                    // [P][d][3D] tensor-core dW range partials
+    int64_t bw_dwtc_rpp = 0;                          // ... rows per range (multiple of 64)
+    int32_t bw_dwtc_parts = 0;                        // ... ranges
+    float *bw_dW3 = nullptr;                          // [d][3D] their sum
     cudaEvent_t bw_ev_fork = nullptr, bw_ev_join = nullptr;
     float *bw_dbg_part = nullptr;                     // [wparts] row-range sums of dt
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
@@ -161,6 +162,15 @@ struct Ctx {
     bool ev_recorded = false;
 };
 
+// One thread waits on an mbarrier nothing arrives on, with the bounded wait of the
+// tensor-core kernels, and sets kDevErrTimeout in *flag after limit_ns (test entry points).
+glga_status launch_bounded_wait_probe(unsigned *flag, uint64_t limit_ns, cudaStream_t s);
+
+struct Ctx;
+// Records stage event `stage` of the context on s (an event record node of the graph when
+// s is being captured, so graph replays record it too).
+cudaError_t record_stage(Ctx *c, int stage, cudaStream_t s);
+
 // allocation helper that tracks bytes
 glga_status dev_alloc(Ctx *c, void **p, size_t bytes);
 // Counts one device allocation of create; GLGA_ERR_OOM when it is the one
@@ -178,6 +188,12 @@ size_t scan_tmp_bytes(int64_t n);
 glga_status projection_setup(Ctx *c);
 glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK,
                            const void *WV, const void *wg, cudaStream_t s, bool time_prep);
+// C [M][ldc] (float32, columns < ncols written) = A [M][K] * B [ncols][K]^T on the tcgen05
+// tensor cores: A and B row-major with leading dimensions lda, ldb (elements, 16-byte
+// multiples), element type t (GLGA_BF16: kind::f16; GLGA_F32: kind::tf32, one term).
+// Stream-ordered; the persistent projection kernel with a float32 epilogue.
+glga_status gemm_nt_f32out(Ctx *c, glga_dtype t, const void *A, int64_t M, int64_t lda, const void *B,
+                           int64_t ncols, int64_t ldb, int64_t K, float *C, int64_t ldc, cudaStream_t s);
 
 // global_stats.cu
 glga_status stats_setup(Ctx *c);
@@ -198,7 +214,6 @@ glga_status block_run(Ctx *c, const void *Y, const void *X, const void *Wo, cons
                       const void *beta, float ln_eps, void *Z, cudaStream_t s);
 
 // backward.cu
-void backward_release(Ctx *c);
 glga_status backward_setup(Ctx *c, cudaStream_t s);
 glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV,
                          const void *wg, float b_g, float eps, const void *dY, float *dX, float *dWQ,

@@ -636,31 +636,73 @@ __device__ __align__(256) float g_static_stats_scratch[kStaticScratchFloats];
 __device__ unsigned g_static_stats_flag;   // bounded-wait timeouts of these calls
 
 std::mutex g_static_mu;
-float *g_static_scratch_addr[kMaxDevices] = {};
-unsigned *g_static_flag_addr[kMaxDevices] = {};
-int g_static_num_sms[kMaxDevices] = {};
+struct StaticSlot {
+    void *ctx = nullptr;          // the CUDA context the addresses belong to
+    float *scratch = nullptr;
+    unsigned *flag = nullptr;
+    int num_sms = 0;
+};
+StaticSlot g_static_slot[kMaxDevices];
 
-// Device addresses of the scratch array and its flag on the current device, looked up
-// once per device.  Their names in host code are host-side stand-ins, never device
-// addresses.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+// The current CUDA context (driver entry point resolved at run time), or null.
+void *current_context() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    }
+    CUcontext cx = nullptr;
+    if (!fn || fn(&cx) != CUDA_SUCCESS) return nullptr;
+    return cx;
+}
+
+// Device addresses of the scratch array and its flag on the current device.  Their names
+// in host code are host-side stand-ins, never device addresses.  The lookup runs once per
+// device and again whenever the device's context is not the one the cached addresses
+// belong to (after cudaDeviceReset, the module is loaded anew at other addresses).
 glga_status static_scratch(int dev, float **ptr, unsigned **flag, int *num_sms) {
+    void *cx = current_context();
+    cudaError_t e = cudaSuccess;
+    if (!cx) {
+        // no context current yet: cudaSetDevice initialises the device's primary context
+        e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+        cx = current_context();
+    }
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_scratch_addr[dev]) {
+    StaticSlot &sl = g_static_slot[dev];
+    if (!sl.scratch || cx != sl.ctx) {
         void *q = nullptr, *f = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&q, g_static_stats_scratch);
+        e = cudaGetSymbolAddress(&q, g_static_stats_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static stats scratch)");
         e = cudaGetSymbolAddress(&f, g_static_stats_flag);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static stats flag)");
         int sms = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-        g_static_scratch_addr[dev] = static_cast<float *>(q);
-        g_static_flag_addr[dev] = static_cast<unsigned *>(f);
-        g_static_num_sms[dev] = sms;
+        sl.ctx = cx;
+        sl.scratch = static_cast<float *>(q);
+        sl.flag = static_cast<unsigned *>(f);
+        sl.num_sms = sms;
     }
-    *ptr = g_static_scratch_addr[dev];
-    *flag = g_static_flag_addr[dev];
-    *num_sms = g_static_num_sms[dev];
+    *ptr = sl.scratch;
+    *flag = sl.flag;
+    *num_sms = sl.num_sms;
+    return GLGA_OK;
+}
+
+glga_status static_device(int *dev) {
+    GLGA_CUDA(cudaGetDevice(dev));
+    if (*dev < 0 || *dev >= kMaxDevices) {
+        set_error("static statistics scratch: device ordinal %d not supported", *dev);
+        return GLGA_ERR_UNSUPPORTED;
+    }
     return GLGA_OK;
 }
 
@@ -696,15 +738,12 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         return GLGA_ERR_INVALID_ARG;
     }
     int dev = 0;
-    GLGA_CUDA(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= kMaxDevices) {
-        set_error("glga_global_stats_static: device ordinal %d not supported", dev);
-        return GLGA_ERR_UNSUPPORTED;
-    }
+    glga_status st = static_device(&dev);
+    if (st != GLGA_OK) return st;
     float *scratch = nullptr;
     unsigned *flag = nullptr;
     int sms = 0;
-    glga_status st = static_scratch(dev, &scratch, &flag, &sms);
+    st = static_scratch(dev, &scratch, &flag, &sms);
     if (st != GLGA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int parts = 0;
@@ -740,4 +779,51 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         nullptr);
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;
+}
+
+extern "C" glga_status glga_global_stats_static_error(void *stream) {
+    using namespace glga;
+    int dev = 0;
+    glga_status st = static_device(&dev);
+    if (st != GLGA_OK) return st;
+    float *scratch = nullptr;
+    unsigned *flag = nullptr;
+    int sms = 0;
+    st = static_scratch(dev, &scratch, &flag, &sms);
+    if (st != GLGA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned f = 0;
+    GLGA_CUDA(cudaMemcpyAsync(&f, flag, sizeof(unsigned), cudaMemcpyDeviceToHost, s));
+    GLGA_CUDA(cudaStreamSynchronize(s));
+    if (f) {
+        GLGA_CUDA(cudaMemsetAsync(flag, 0, sizeof(unsigned), s));
+        GLGA_CUDA(cudaStreamSynchronize(s));
+    }
+    if (f & kDevErrTimeout) {
+        set_error("glga_global_stats_static: a bounded device-side wait timed out; the S and z of "
+                  "that call are incomplete");
+        return GLGA_ERR_TIMEOUT;
+    }
+    if (f) {
+        set_error("glga_global_stats_static: device-side check failed (flags 0x%x)", f);
+        return GLGA_ERR_DEVICE;
+    }
+    return GLGA_OK;
+}
+
+extern "C" glga_status glga_debug_static_bounded_wait(int64_t limit_ns, void *stream) {
+    using namespace glga;
+    if (limit_ns < 1000 || limit_ns > 10000000000LL) {
+        set_error("glga_debug_static_bounded_wait: need 1e3 <= limit_ns <= 1e10");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    glga_status st = static_device(&dev);
+    if (st != GLGA_OK) return st;
+    float *scratch = nullptr;
+    unsigned *flag = nullptr;
+    int sms = 0;
+    st = static_scratch(dev, &scratch, &flag, &sms);
+    if (st != GLGA_OK) return st;
+    return launch_bounded_wait_probe(flag, static_cast<uint64_t>(limit_ns), static_cast<cudaStream_t>(stream));
 }

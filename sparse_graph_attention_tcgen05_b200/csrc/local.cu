@@ -5,10 +5,13 @@
 // evaluated per head for every target row and written to L [N, H*r]; the global readout
 // and the gate blend run afterwards in the readout GEMM's epilogue (readout.cu).  The
 // softmax is the stable one of the tinymesh page ("Target softmax"), computed in a
-// single pass with a running maximum: the state (m, l, acc) of a partial sum is rescaled
-// by 2^(m_old - m_new) whenever the maximum grows, and two partial states merge the same
-// way, so edges may be split across lanes, warps and thread blocks and merged in a fixed
-// order.  No per-edge value is stored.
+// single pass: the state (m, l, acc) of a partial sum holds l = sum 2^(x_j - m) and
+// acc = sum 2^(x_j - m) v_j for base-2 scores x_j = s_ij log2(e) and a reference m.  Any
+// reference gives the same acc / l; m is raised (and l, acc rescaled by 2^(m_old - m_new))
+// only when a score exceeds it by more than 2^kTau, so most edge steps skip the rescale
+// and every weight stays below 2^kTau.  Two partial states merge the same way, so edges
+// may be split across lanes, warps and thread blocks and merged in a fixed order.  No
+// per-edge value is stored.
 //
 // Work is scheduled by the degree buckets built at create time:
 //   chunk blocks   bucket-2 rows cut into chunk_edges-edge chunks; each block merges its
@@ -26,10 +29,18 @@
 //
 // Lane layout: a 16-byte vector holds VE = 16/sizeof(T) consecutive features; an edge's
 // k_j (or v_j) row is LPE lanes x VPL vectors; EPW = 32/LPE edge slots per warp; the r
-// features of a head live in LPH = r/VE adjacent lanes, which reduce dot products with
-// butterfly shuffles.  Each slot walks a contiguous edge range U edges at a time; the
-// column indices of the next step (and, for task rows, the next row's q and first
-// columns) are loaded one step ahead so the k_j/v_j gathers do not wait behind them.
+// features of a head live in LPH adjacent lanes, which reduce dot products with butterfly
+// shuffles.  In the joint layout (J) a lane's VPL vectors are consecutive features of one
+// head, so the lane keeps one softmax state for all of them.  Each slot walks a
+// contiguous edge range U edges at a time; the column indices of the next step (and, for
+// task rows, the next row's q and first columns) are loaded one step ahead so the
+// k_j/v_j gathers do not wait behind them.
+//
+// Arithmetic: q_i and k_j stay in the io type; for bf16 the dot product runs on the
+// mixed-precision fma.rn.f32.bf16 (bf16 operands, exact products, f32 accumulation), so
+// the gathered rows are never unpacked.  The score scale log2(e)/sqrt(r) is applied to
+// the f32 dot product inside the exponent.  The v_j side accumulates in f32 with f32
+// weights (bf16 v_j widened exactly).
 #include <algorithm>
 #include <cmath>
 #include <vector>
@@ -43,12 +54,50 @@ constexpr int kLocalWarps = 8;
 constexpr int kLocalThreads = kLocalWarps * 32;
 constexpr int kTaskRows = 32;
 constexpr int64_t kTaskEdges = 256;
+// Start of the running reference: a finite stand-in for -infinity, so that an empty state
+// merges without inf - inf.
+constexpr float kMInit = -3.0e38f;
+// The reference is raised only when a base-2 score exceeds it by more than this.
+constexpr float kTau = 8.f;
+
+// d = a * b + c with a and b the bf16 halves (AH / BH: high half) of 32-bit words:
+// exact product, one f32 rounding.
+template <int AH, int BH>
+__device__ __forceinline__ float mfma(uint32_t a, uint32_t b, float c) {
+    float d;
+    if constexpr (AH == 0 && BH == 0)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a0, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if constexpr (AH == 1 && BH == 1)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a1, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if constexpr (AH == 0 && BH == 1)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a0, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a1, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+// Two f32 values rounded to bf16 (nearest even) in one word: lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t w;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
+    return w;
+}
 
 template <typename T>
 struct Io;
 template <>
 struct Io<float> {
     static constexpr int VE = 4;
+    __device__ __forceinline__ static float dot(const uint4 &q, const uint4 &k, float acc) {
+        acc = fmaf(__uint_as_float(q.x), __uint_as_float(k.x), acc);
+        acc = fmaf(__uint_as_float(q.y), __uint_as_float(k.y), acc);
+        acc = fmaf(__uint_as_float(q.z), __uint_as_float(k.z), acc);
+        return fmaf(__uint_as_float(q.w), __uint_as_float(k.w), acc);
+    }
     __device__ __forceinline__ static void unpack(const uint4 &u, float (&f)[VE]) {
         f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
         f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
@@ -61,6 +110,18 @@ struct Io<float> {
 template <>
 struct Io<__nv_bfloat16> {
     static constexpr int VE = 8;
+    __device__ __forceinline__ static float dot(const uint4 &q, const uint4 &k, float acc) {
+        // two chains, so consecutive FMAs do not wait on each other
+        float a2 = mfma<1, 1>(q.x, k.x, 0.f);
+        acc = mfma<0, 0>(q.x, k.x, acc);
+        acc = mfma<0, 0>(q.y, k.y, acc);
+        a2 = mfma<1, 1>(q.y, k.y, a2);
+        acc = mfma<0, 0>(q.z, k.z, acc);
+        a2 = mfma<1, 1>(q.z, k.z, a2);
+        acc = mfma<0, 0>(q.w, k.w, acc);
+        a2 = mfma<1, 1>(q.w, k.w, a2);
+        return acc + a2;
+    }
     __device__ __forceinline__ static void unpack(const uint4 &u, float (&f)[VE]) {
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -70,13 +131,8 @@ struct Io<__nv_bfloat16> {
         }
     }
     __device__ __forceinline__ static uint4 pack(const float (&f)[VE]) {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t *>(&h);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
+        return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                          pack_bf16x2(f[6], f[7]));
     }
 };
 
@@ -113,8 +169,8 @@ struct LocalParams {
     unsigned *flag;      // device error flag (debug checks)
 };
 
-// 2^x by the PTX ex2.approx.ftz instruction.  The arguments are differences from a
-// running maximum (<= 0); results below 2^-126 of the maximum flush to zero.
+// 2^x by the PTX ex2.approx.ftz instruction.  The arguments are scores minus a reference
+// (<= kTau); results below 2^-126 flush to zero.
 __device__ __forceinline__ float exp2_ftz(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -145,28 +201,73 @@ __device__ __forceinline__ bool row_ok(const LocalParams &p, int64_t row) {
     return true;
 }
 
-template <typename T, int VPL>
+constexpr int pow2_at_least(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+// Compile-time shape of one instantiation.  NV (16-byte vectors per q/k/v row) and LPH
+// (lanes per head) are fixed for the hot shapes and 0 for the generic build, which reads
+// them from the parameters.
+template <typename T, int NV, int LPH, int VPL, bool J>
+struct Shape {
+    static constexpr int VE = Io<T>::VE;
+    static constexpr int NH = J ? 1 : VPL;   // heads (softmax states) per lane
+    __device__ __forceinline__ static int nvec(const LocalParams &p) { return NV ? NV : p.nvec; }
+    __device__ __forceinline__ static int lph(const LocalParams &p) { return LPH ? LPH : p.lph; }
+    __device__ __forceinline__ static int lpe(const LocalParams &p) {
+        if constexpr (NV != 0) return J ? NV / VPL : (NV >= 32 ? 32 : pow2_at_least(NV));
+        return p.lpe;
+    }
+    __device__ __forceinline__ static int epw(const LocalParams &p) { return 32 / lpe(p); }
+    // vector index (within a row) of the lane's vector v; its head is vid * VE / r
+    __device__ __forceinline__ static int vid(int v, int li) { return J ? li * VPL + v : v * 32 + li; }
+    // lanes per edge of a compile-time layout (0: read from the parameters)
+    static constexpr int kLpe = NV == 0 ? 0 : (J ? NV / VPL : (NV >= 32 ? 32 : pow2_at_least(NV)));
+    // every vector of a compile-time layout that fills its lanes is in range
+    static constexpr bool kFull =
+        NV != 0 && (J || NV == 32 * VPL || (VPL == 1 && NV < 32 && (NV & (NV - 1)) == 0));
+    __device__ __forceinline__ static bool lane_ok(const LocalParams &p, int v, int li) {
+        if constexpr (kFull) return true;
+        return vid(v, li) < nvec(p);
+    }
+    // byte offset of the lane's vector v inside a k (or v, q, L) row
+    __device__ __forceinline__ static int voff(int v) { return J ? v * 16 : v * 512; }
+};
+
+template <typename T, int VPL, bool J>
 struct State {
     static constexpr int VE = Io<T>::VE;
-    float m[VPL], l[VPL], acc[VPL][VE];
+    static constexpr int NH = J ? 1 : VPL;
+    float m[NH], l[NH], acc[VPL][VE];
     __device__ __forceinline__ void init() {
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            m[v] = -INFINITY;
-            l[v] = 0.f;
+        for (int h = 0; h < NH; ++h) {
+            m[h] = kMInit;
+            l[h] = 0.f;
+        }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
 #pragma unroll
             for (int e = 0; e < VE; ++e) acc[v][e] = 0.f;
-        }
     }
-    // merge another partial state into this one (per vector)
-    __device__ __forceinline__ void merge(int v, float m2, float l2, const float (&a2)[VE]) {
-        const float mn = fmaxf(m[v], m2);
-        if (mn == -INFINITY) return;
-        const float c1 = exp2_ftz(m[v] - mn), c2 = exp2_ftz(m2 - mn);
-        l[v] = l[v] * c1 + l2 * c2;
+    __device__ __forceinline__ static constexpr int head_of(int v) { return J ? 0 : v; }
+    // merge another partial state (m2, l2, a2) into this one
+    __device__ __forceinline__ void merge(const float (&m2)[NH], const float (&l2)[NH], const float (&a2)[VPL][VE]) {
+        float c1[NH], c2[NH];
 #pragma unroll
-        for (int e = 0; e < VE; ++e) acc[v][e] = acc[v][e] * c1 + a2[e] * c2;
-        m[v] = mn;
+        for (int h = 0; h < NH; ++h) {
+            const float mn = fmaxf(m[h], m2[h]);
+            c1[h] = exp2_ftz(m[h] - mn);
+            c2[h] = exp2_ftz(m2[h] - mn);
+            l[h] = l[h] * c1[h] + l2[h] * c2[h];
+            m[h] = mn;
+        }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+#pragma unroll
+            for (int e = 0; e < VE; ++e) acc[v][e] = acc[v][e] * c1[head_of(v)] + a2[v][e] * c2[head_of(v)];
     }
 };
 
@@ -174,282 +275,328 @@ struct Lane {
     int lane, slot, li;
 };
 
-// The 16-byte vector index (within a q / k / v / L row) of vector v of lane li.  J = false:
-// vectors v*32 + li (lanes interleave; a head spans r/VE lanes).  J = true ("joint"): the
-// lane's VPL vectors are consecutive, li*VPL + v, and all lie in one head (VPL*VE <= r),
-// so the lane computes one score per edge for all of them.
-template <bool J, int VPL>
-__device__ __forceinline__ int vid_of(int v, int li) {
-    return J ? li * VPL + v : v * 32 + li;
+// Column indices of a slot's range as held by the lanes that later broadcast them: lane
+// li (< CB) of the slot holds col_idx[e0 + li].  CB = U (one step's edges) for runtime
+// layouts, the slot's lane count for compile-time ones (a batch of several steps).
+template <int CB, bool DBG>
+__device__ __forceinline__ int32_t first_cols(const LocalParams &p, int64_t e0, int64_t e1, const Lane &ln) {
+    return (ln.li < CB && e0 + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + e0 + ln.li)) : -1;
 }
 
-// First column index of a slot's range as held by the lane that later broadcasts it:
-// lane li (< U) of the slot holds col_idx[e0 + li].
-template <int U, bool DBG>
-__device__ __forceinline__ int32_t first_cols(const LocalParams &p, int64_t e0, int64_t e1, const Lane &ln) {
-    return (ln.li < U && e0 + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + e0 + ln.li)) : -1;
+template <typename T, int NV, int LPH, int VPL, int U, bool J>
+constexpr int col_batch() {
+    return Shape<T, NV, LPH, VPL, J>::kLpe != 0 ? Shape<T, NV, LPH, VPL, J>::kLpe : U;
 }
 
 // One slot walks the CSR entries [e0, e1) U at a time (the trip count is the warp's
-// maximum over slots); `cols` holds the first step's column indices (first_cols).
+// maximum over slots); `cols` holds the first column batch (first_cols).  With PIPE the
+// k_j / v_j gathers of step i + 1 are issued before step i is consumed (two register
+// buffers), so a warp keeps a step's loads in flight while it computes the previous one.
 // On return each lane holds its slot's partial state for its feature vectors.
-template <typename T, int VPL, int U, bool DBG, bool J>
-__device__ __forceinline__ void slot_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
-                                           int64_t e0, int64_t e1, int32_t cols, const Lane &ln,
-                                           State<T, VPL> &st) {
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE>
+__device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q)[VPL], int64_t e0,
+                                           int64_t e1, int32_t cols, const Lane &ln,
+                                           State<T, VPL, J> &st) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
+    using St = State<T, VPL, J>;
     constexpr int VE = Io<T>::VE;
+    constexpr int NH = Sh::NH;
     st.init();
     const int iters_mine = e1 > e0 ? static_cast<int>((e1 - e0 + U - 1) / U) : 0;
     const int iters = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(iters_mine));
-    const uint4 *KV = static_cast<const uint4 *>(p.KV);
-    const int64_t row_vecs = 2 * static_cast<int64_t>(p.nvec);
-    const int src0 = ln.slot * p.lpe;
-    int32_t c_next = cols;
-    for (int it = 0; it < iters; ++it) {
-        const int32_t c_cur = c_next;
-        const int64_t nb = e0 + static_cast<int64_t>(it + 1) * U;
-        c_next = (ln.li < U && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
-        int32_t j[U];
+    const int nvec = Sh::nvec(p);
+    const uint32_t row_bytes = 32u * static_cast<uint32_t>(nvec);   // k_j | v_j
+    const char *kvl = static_cast<const char *>(p.KV) + 16 * Sh::vid(0, ln.li);
+    const int src0 = ln.slot * Sh::lpe(p);
+    const int lph = Sh::lph(p);
+    const float scale = p.score_scale;
+    bool ok[VPL];
 #pragma unroll
-        for (int u = 0; u < U; ++u) j[u] = __shfl_sync(0xffffffffu, c_cur, src0 + u);
-        uint4 kr[U][VPL], vr[U][VPL];
+    for (int v = 0; v < VPL; ++v) ok[v] = Sh::lane_ok(p, v, ln.li);
+    // column indices arrive in batches of CB edges (CB / U steps each); the next batch is
+    // loaded while the current one is used.  The batches follow the load stream.
+    constexpr int CB = col_batch<T, NV, LPH, VPL, U, J>();
+    constexpr int PER = CB / U;
+    static_assert(CB % U == 0, "a batch holds whole steps");
+    int32_t c_cur = cols;
+    int32_t c_next = -1;
+    if (PER > 1 && iters > PER) {
+        const int64_t nb = e0 + CB;
+        c_next = (ln.li < CB && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
+    }
+    // issues the gathers of step `step` into (kb, vb); jb gets its column indices (-1:
+    // no edge; such a slot keeps its previous, finite contents and gets weight 0)
+    auto load = [&](int step, uint4 (&kb)[U][VPL], uint4 (&vb)[U][VPL], int32_t (&jb)[U]) {
+        const int sub = PER > 1 ? step % PER : 0;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-#pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                const int vid = vid_of<J, VPL>(v, ln.li);
-                if (j[u] >= 0 && vid < p.nvec) {
-                    // (a masked-off slot never forms an address: j < 0 takes the else branch)
-                    const uint4 *rowp = KV + static_cast<int64_t>(j[u]) * row_vecs;
-                    kr[u][v] = ld_gather(rowp + vid);
-                    vr[u][v] = ld_gather(rowp + p.nvec + vid);
-                } else {
-                    kr[u][v] = make_uint4(0, 0, 0, 0);
-                    vr[u][v] = make_uint4(0, 0, 0, 0);
-                }
+        for (int u = 0; u < U; ++u) jb[u] = __shfl_sync(0xffffffffu, c_cur, src0 + sub * U + u);
+        if (sub == PER - 1) {
+            if (PER > 1) {
+                c_cur = c_next;
+                const int64_t nb = e0 + static_cast<int64_t>(step / PER + 2) * CB;
+                c_next = (ln.li < CB && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
+            } else {
+                const int64_t nb = e0 + static_cast<int64_t>(step + 1) * U;
+                c_cur = (ln.li < U && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
             }
         }
-        if constexpr (J) {
-            // one score per edge for the lane's VPL vectors (one head): one exp, one max
-            // and one rescale per edge instead of VPL
-            float s1[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                float dot = 0.f;
+        for (int u = 0; u < U; ++u) {
+            if (jb[u] >= 0) {
+                const char *rowp = kvl + static_cast<size_t>(static_cast<uint32_t>(jb[u])) * row_bytes;
 #pragma unroll
                 for (int v = 0; v < VPL; ++v) {
-                    float kf[VE];
-                    Io<T>::unpack(kr[u][v], kf);
-#pragma unroll
-                    for (int e = 0; e < VE; ++e) dot = fmaf(q[v][e], kf[e], dot);
-                }
-                for (int o = 1; o < p.lph; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                s1[u] = (j[u] >= 0) ? dot : -INFINITY;
-            }
-            float mx = s1[0];
-#pragma unroll
-            for (int u = 1; u < U; ++u) mx = fmaxf(mx, s1[u]);
-            const float mn = fmaxf(st.m[0], mx);
-            if (mn != -INFINITY) {
-                const float corr = exp2_ftz(st.m[0] - mn);
-                st.l[0] *= corr;
-#pragma unroll
-                for (int v = 0; v < VPL; ++v)
-#pragma unroll
-                    for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const float pr = exp2_ftz(s1[u] - mn);
-                    st.l[0] += pr;
-#pragma unroll
-                    for (int v = 0; v < VPL; ++v) {
-                        float vf[VE];
-                        Io<T>::unpack(vr[u][v], vf);
-#pragma unroll
-                        for (int e = 0; e < VE; ++e) st.acc[v][e] = fmaf(pr, vf[e], st.acc[v][e]);
+                    if (ok[v]) {
+                        kb[u][v] = ld_gather(rowp + Sh::voff(v));
+                        vb[u][v] = ld_gather(rowp + 16 * nvec + Sh::voff(v));
                     }
                 }
-                st.m[0] = mn;
             }
-            continue;
         }
-        float s[U][VPL];
+    };
+    // folds one step's edges into the state
+    auto consume = [&](const uint4 (&kb)[U][VPL], const uint4 (&vb)[U][VPL], const int32_t (&jb)[U]) {
+        // scores (f32 dot products, unscaled), reduced over the head's lanes
+        float sc[U][NH];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                float kf[VE];
-                Io<T>::unpack(kr[u][v], kf);
+            for (int h = 0; h < NH; ++h) {
                 float dot = 0.f;
 #pragma unroll
-                for (int e = 0; e < VE; ++e) dot = fmaf(q[v][e], kf[e], dot);
-                for (int o = 1; o < p.lph; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                s[u][v] = (j[u] >= 0) ? dot : -INFINITY;
+                for (int v = 0; v < VPL; ++v)
+                    if (St::head_of(v) == h) dot = Io<T>::dot(q[v], kb[u][v], dot);
+                if constexpr (LPH != 0) {
+#pragma unroll
+                    for (int o = 1; o < LPH; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                } else {
+                    for (int o = 1; o < lph; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                }
+                sc[u][h] = (jb[u] >= 0) ? dot : -INFINITY;
+            }
+        }
+        // raise the reference only when a score exceeds it by more than kTau
+        float mx[NH];
+        bool need = false;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+            mx[h] = sc[0][h];
+#pragma unroll
+            for (int u = 1; u < U; ++u) mx[h] = fmaxf(mx[h], sc[u][h]);
+            mx[h] *= scale;
+            need |= mx[h] > st.m[h] + kTau;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const float mn = fmaxf(st.m[h], mx[h]);
+                const float corr = exp2_ftz(st.m[h] - mn);
+                st.l[h] *= corr;
+                st.m[h] = mn;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+                    if (St::head_of(v) == h)
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
             }
         }
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            float mx = s[0][v];
+        for (int u = 0; u < U; ++u) {
+            float pr[NH];
 #pragma unroll
-            for (int u = 1; u < U; ++u) mx = fmaxf(mx, s[u][v]);
-            const float mn = fmaxf(st.m[v], mx);
-            if (mn == -INFINITY) continue;
-            const float corr = exp2_ftz(st.m[v] - mn);
-            st.l[v] *= corr;
+            for (int h = 0; h < NH; ++h) {
+                pr[h] = exp2_ftz(fmaf(sc[u][h], scale, -st.m[h]));
+                st.l[h] += pr[h];
+            }
 #pragma unroll
-            for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const float pr = exp2_ftz(s[u][v] - mn);
+            for (int v = 0; v < VPL; ++v) {
                 float vf[VE];
-                Io<T>::unpack(vr[u][v], vf);
-                st.l[v] += pr;
+                Io<T>::unpack(vb[u][v], vf);
+                const float w = pr[St::head_of(v)];
 #pragma unroll
-                for (int e = 0; e < VE; ++e) st.acc[v][e] = fmaf(pr, vf[e], st.acc[v][e]);
+                for (int e = 0; e < VE; ++e) st.acc[v][e] = fmaf(w, vf[e], st.acc[v][e]);
             }
-            st.m[v] = mn;
         }
-    }
-    if constexpr (J) {
-        // every vector of the lane carries the head's (m, l): the merges work per vector
+    };
+    uint4 kA[U][VPL], vA[U][VPL];
+    int32_t jA[U];
 #pragma unroll
-        for (int v = 1; v < VPL; ++v) {
-            st.m[v] = st.m[0];
-            st.l[v] = st.l[0];
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) kA[u][v] = vA[u][v] = make_uint4(0, 0, 0, 0);
+    if constexpr (!PIPE) {
+        for (int it = 0; it < iters; ++it) {
+            load(it, kA, vA, jA);
+            consume(kA, vA, jA);
+        }
+    } else {
+        uint4 kB[U][VPL], vB[U][VPL];
+        int32_t jB[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) kB[u][v] = vB[u][v] = make_uint4(0, 0, 0, 0);
+        if (iters > 0) load(0, kA, vA, jA);
+        for (int it = 0; it < iters; it += 2) {
+            if (it + 1 < iters) load(it + 1, kB, vB, jB);
+            consume(kA, vA, jA);
+            if (it + 1 < iters) {
+                if (it + 2 < iters) load(it + 2, kA, vA, jA);
+                consume(kB, vB, jB);
+            }
         }
     }
 }
 
 // Merges the edge slots of the warp (lanes li, li + LPE, ...): afterwards every lane
 // holds the state over all slots.
-template <typename T, int VPL>
-__device__ __forceinline__ void merge_slots(const LocalParams &p, State<T, VPL> &st) {
+template <typename T, int NV, int LPH, int VPL, bool J>
+__device__ __forceinline__ void merge_slots(const LocalParams &p, State<T, VPL, J> &st) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
     constexpr int VE = Io<T>::VE;
-    for (int o = p.lpe; o < 32; o <<= 1) {
+    constexpr int NH = Sh::NH;
+    for (int o = Sh::lpe(p); o < 32; o <<= 1) {
+        float m2[NH], l2[NH], a2[VPL][VE];
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, st.m[v], o);
-            const float l2 = __shfl_xor_sync(0xffffffffu, st.l[v], o);
-            float a2[VE];
-#pragma unroll
-            for (int e = 0; e < VE; ++e) a2[e] = __shfl_xor_sync(0xffffffffu, st.acc[v][e], o);
-            st.merge(v, m2, l2, a2);
+        for (int h = 0; h < NH; ++h) {
+            m2[h] = __shfl_xor_sync(0xffffffffu, st.m[h], o);
+            l2[h] = __shfl_xor_sync(0xffffffffu, st.l[h], o);
         }
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+#pragma unroll
+            for (int e = 0; e < VE; ++e) a2[v][e] = __shfl_xor_sync(0xffffffffu, st.acc[v][e], o);
+        st.merge(m2, l2, a2);
     }
 }
 
-template <typename T, int VPL, bool J>
-__device__ __forceinline__ void load_q_raw(const LocalParams &p, int64_t row, const Lane &ln, bool ok,
-                                           uint4 (&qr)[VPL]) {
-    const uint4 *Q = static_cast<const uint4 *>(p.Q) + row * p.nvec;
+template <typename T, int NV, int LPH, int VPL, bool J>
+__device__ __forceinline__ void load_q(const LocalParams &p, int64_t row, const Lane &ln, bool valid,
+                                       uint4 (&qr)[VPL]) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
+    const char *Q = static_cast<const char *>(p.Q) + row * 16 * Sh::nvec(p) + 16 * Sh::vid(0, ln.li);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-        const int vid = vid_of<J, VPL>(v, ln.li);
-        qr[v] = (ok && vid < p.nvec) ? __ldg(Q + vid) : make_uint4(0, 0, 0, 0);
-    }
-}
-
-template <typename T, int VPL>
-__device__ __forceinline__ void scale_q(const LocalParams &p, const uint4 (&qr)[VPL], float (&q)[VPL][Io<T>::VE]) {
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-        Io<T>::unpack(qr[v], q[v]);
-#pragma unroll
-        for (int e = 0; e < Io<T>::VE; ++e) q[v][e] *= p.score_scale;   // log2(e)/sqrt(r) folded in
-    }
+    for (int v = 0; v < VPL; ++v)
+        qr[v] = (valid && Sh::lane_ok(p, v, ln.li)) ? __ldg(reinterpret_cast<const uint4 *>(Q + Sh::voff(v)))
+                                                    : make_uint4(0, 0, 0, 0);
 }
 
 // lse_i = ln sum_j exp(s_ij) per head, ln 2 (m + log2 l) since the state keeps base-2
 // scores (0 for a row without edges), from the vector holding the head's first features.
 // Compiled in only for the LSE instantiations (contexts made for the backward pass), so
 // the plain forward's code is untouched.
-template <typename T, int VPL, bool J, bool LSE>
-__device__ __forceinline__ void store_lse(const LocalParams &p, int64_t row, const State<T, VPL> &st,
+template <typename T, int NV, int LPH, int VPL, bool J, bool LSE>
+__device__ __forceinline__ void store_lse(const LocalParams &p, int64_t row, const State<T, VPL, J> &st,
                                           const Lane &ln, bool mine) {
     if constexpr (!LSE) return;
+    using Sh = Shape<T, NV, LPH, VPL, J>;
     constexpr int VE = Io<T>::VE;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
-        const int vid = vid_of<J, VPL>(v, ln.li);
-        if (mine && vid < p.nvec && (vid * VE) % p.r == 0)
+        const int vid = Sh::vid(v, ln.li);
+        const int h = State<T, VPL, J>::head_of(v);
+        if (mine && Sh::lane_ok(p, v, ln.li) && (vid * VE) % p.r == 0)
             p.lse[row * p.H + vid * VE / p.r] =
-                st.l[v] > 0.f ? 0.69314718055994531f * (st.m[v] + __log2f(st.l[v])) : 0.f;
+                st.l[h] > 0.f ? 0.69314718055994531f * (st.m[h] + __log2f(st.l[h])) : 0.f;
     }
 }
 
-// L_i = acc / l per head (0 for a row without edges); stores L[row] from `slot`'s lanes.
-template <typename T, int VPL, bool J, bool LSE>
-__device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, const State<T, VPL> &st,
-                                           const Lane &ln, int slot) {
+// L_i = acc / l per head (0 for a row without edges), stored from lanes with `mine`.
+template <typename T, int NV, int LPH, int VPL, bool J, bool LSE>
+__device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, const State<T, VPL, J> &st,
+                                           const Lane &ln, bool mine) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
     constexpr int VE = Io<T>::VE;
-    uint4 *Lout = static_cast<uint4 *>(p.L) + row * p.nvec;
+    constexpr int NH = Sh::NH;
+    float inv_l[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) inv_l[h] = st.l[h] > 0.f ? 1.f / st.l[h] : 0.f;
+    char *Lout = static_cast<char *>(p.L) + row * 16 * Sh::nvec(p) + 16 * Sh::vid(0, ln.li);
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
-        const int vid = vid_of<J, VPL>(v, ln.li);
-        const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
         float y[VE];
 #pragma unroll
-        for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l;
-        if (vid < p.nvec && ln.slot == slot) Lout[vid] = Io<T>::pack(y);
+        for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l[State<T, VPL, J>::head_of(v)];
+        if (mine && Sh::lane_ok(p, v, ln.li)) *reinterpret_cast<uint4 *>(Lout + Sh::voff(v)) = Io<T>::pack(y);
     }
-    store_lse<T, VPL, J, LSE>(p, row, st, ln, ln.slot == slot);
+    store_lse<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, mine);
 }
 
-template <typename T, int VPL>
+template <typename T, int VPL, bool J>
 struct BlockScratch {
     static constexpr int VE = Io<T>::VE;
-    float m[kLocalWarps][VPL][32];
-    float l[kLocalWarps][VPL][32];
+    static constexpr int NH = J ? 1 : VPL;
+    float m[kLocalWarps][NH][32];
+    float l[kLocalWarps][NH][32];
     float acc[kLocalWarps][VPL][VE][32];
 };
 
 // 8 warps split [e0, e1) (each warp's share split again across its slots); warp 0
 // returns the merge of all warps in warp order.
-template <typename T, int VPL, int U, bool DBG, bool J>
-__device__ __forceinline__ void block_edges(const LocalParams &p, const float (&q)[VPL][Io<T>::VE],
-                                            int64_t e0, int64_t e1, const Lane &ln, int warp,
-                                            BlockScratch<T, VPL> &sh, State<T, VPL> &st) {
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE>
+__device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&q)[VPL], int64_t e0,
+                                            int64_t e1, const Lane &ln, int warp,
+                                            BlockScratch<T, VPL, J> &sh, State<T, VPL, J> &st) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
     constexpr int VE = Io<T>::VE;
+    constexpr int NH = Sh::NH;
     const int64_t per = ceil_div(e1 - e0, kLocalWarps);
     const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
-    const int64_t per_s = ceil_div(b - a, p.epw);
+    const int64_t per_s = ceil_div(b - a, Sh::epw(p));
     const int64_t sa = std::min(b, a + ln.slot * per_s), sb = std::min(b, sa + per_s);
-    slot_edges<T, VPL, U, DBG, J>(p, q, sa, sb, first_cols<U, DBG>(p, sa, sb, ln), ln, st);
-    merge_slots<T, VPL>(p, st);
+    slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, sa, sb,
+                                               first_cols<col_batch<T, NV, LPH, VPL, U, J>(), DBG>(p, sa, sb, ln),
+                                               ln, st);
+    merge_slots<T, NV, LPH, VPL, J>(p, st);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-        sh.m[warp][v][ln.lane] = st.m[v];
-        sh.l[warp][v][ln.lane] = st.l[v];
+    for (int h = 0; h < NH; ++h) {
+        sh.m[warp][h][ln.lane] = st.m[h];
+        sh.l[warp][h][ln.lane] = st.l[h];
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
 #pragma unroll
         for (int e = 0; e < VE; ++e) sh.acc[warp][v][e][ln.lane] = st.acc[v][e];
-    }
     __syncthreads();
     if (warp == 0) {
         for (int w = 1; w < kLocalWarps; ++w) {
+            float m2[NH], l2[NH], a2[VPL][VE];
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                float a2[VE];
-#pragma unroll
-                for (int e = 0; e < VE; ++e) a2[e] = sh.acc[w][v][e][ln.lane];
-                st.merge(v, sh.m[w][v][ln.lane], sh.l[w][v][ln.lane], a2);
+            for (int h = 0; h < NH; ++h) {
+                m2[h] = sh.m[w][h][ln.lane];
+                l2[h] = sh.l[w][h][ln.lane];
             }
+#pragma unroll
+            for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                for (int e = 0; e < VE; ++e) a2[v][e] = sh.acc[w][v][e][ln.lane];
+            st.merge(m2, l2, a2);
         }
     }
 }
 
-template <typename T, int VPL, int U, bool DBG, bool J, bool LSE>
-__global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(const LocalParams p) {
+// Blocks per SM the register budget aims at: 3 (at most 85 registers) while the gather
+// buffers take at most 32 registers (8 per edge step and vector, doubled when pipelined),
+// else 2.
+constexpr int local_min_blocks(int VPL, int U, bool PIPE) {
+    return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? 3 : 2;
+}
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE>
+__global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
+    local_kernel(const LocalParams p) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
+    using St = State<T, VPL, J>;
     constexpr int VE = Io<T>::VE;
-    __shared__ BlockScratch<T, VPL> sh;
+    constexpr int NH = Sh::NH;
+    __shared__ BlockScratch<T, VPL, J> sh;
     const int warp = threadIdx.x >> 5;
     Lane ln;
     ln.lane = threadIdx.x & 31;
-    ln.slot = ln.lane / p.lpe;
-    ln.li = ln.lane % p.lpe;
+    ln.slot = ln.lane / Sh::lpe(p);
+    ln.li = ln.lane % Sh::lpe(p);
     int64_t bid = blockIdx.x;
-    float q[VPL][VE];
-    uint4 qr[VPL];
-    State<T, VPL> st;
+    uint4 q[VPL];
+    St st;
 
     if (bid < p.n_chunks) {
         // ---------------- chunk of a bucket-2 row ----------------
@@ -461,22 +608,21 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         const int64_t e1 = std::min<int64_t>(re, e0 + p.chunk_edges);
         const int64_t nch = ceil_div(re - rb, p.chunk_edges);
         const int64_t first = c - (e0 - rb) / p.chunk_edges;
-        load_q_raw<T, VPL, J>(p, row, ln, true, qr);
-        scale_q<T, VPL>(p, qr, q);
-        block_edges<T, VPL, U, DBG, J>(p, q, e0, e1, ln, warp, sh, st);
+        load_q<T, NV, LPH, VPL, J>(p, row, ln, true, q);
+        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, e0, e1, ln, warp, sh, st);
         const int64_t stride = 2 * p.H + p.D;
         if (warp == 0) {
             float *dst = p.part + c * stride;
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const int vid = vid_of<J, VPL>(v, ln.li);
-                if (vid < p.nvec && ln.slot == 0) {
+                const int vid = Sh::vid(v, ln.li);
+                if (Sh::lane_ok(p, v, ln.li) && ln.slot == 0) {
 #pragma unroll
                     for (int e = 0; e < VE; ++e) dst[2 * p.H + vid * VE + e] = st.acc[v][e];
-                    if ((ln.li & (p.lph - 1)) == 0) {
+                    if ((vid * VE) % p.r == 0) {
                         const int h = vid * VE / p.r;
-                        dst[h] = st.m[v];
-                        dst[p.H + h] = st.l[v];
+                        dst[h] = st.m[St::head_of(v)];
+                        dst[p.H + h] = st.l[St::head_of(v)];
                     }
                 }
             }
@@ -494,18 +640,22 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
                 st.init();
                 for (int64_t k = 0; k < nch; ++k) {
                     const float *src = p.part + (first + k) * stride;
+                    float m2[NH], l2[NH], a2[VPL][VE];
 #pragma unroll
                     for (int v = 0; v < VPL; ++v) {
-                        const int vid = vid_of<J, VPL>(v, ln.li);
-                        const int h = vid < p.nvec ? vid * VE / p.r : 0;
-                        float a2[VE];
+                        const int vid = Sh::vid(v, ln.li);
+                        const bool okv = Sh::lane_ok(p, v, ln.li);
+                        const int h = okv ? vid * VE / p.r : 0;
 #pragma unroll
-                        for (int e = 0; e < VE; ++e)
-                            a2[e] = vid < p.nvec ? __ldcg(src + 2 * p.H + vid * VE + e) : 0.f;
-                        st.merge(v, __ldcg(src + h), __ldcg(src + p.H + h), a2);
+                        for (int e = 0; e < VE; ++e) a2[v][e] = okv ? __ldcg(src + 2 * p.H + vid * VE + e) : 0.f;
+                        if (St::head_of(v) == v || v == 0) {
+                            m2[St::head_of(v)] = okv ? __ldcg(src + h) : kMInit;
+                            l2[St::head_of(v)] = okv ? __ldcg(src + p.H + h) : 0.f;
+                        }
                     }
+                    st.merge(m2, l2, a2);
                 }
-                finish_row<T, VPL, J, LSE>(p, row, st, ln, 0);
+                finish_row<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, ln.slot == 0);
             }
         }
         return;
@@ -515,10 +665,9 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
         // ---------------- bucket-1 row: one block ----------------
         const int64_t row = p.cta_rows[bid];
         if (!row_ok<DBG>(p, row)) return;
-        load_q_raw<T, VPL, J>(p, row, ln, true, qr);
-        scale_q<T, VPL>(p, qr, q);
-        block_edges<T, VPL, U, DBG, J>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
-        if (warp == 0) finish_row<T, VPL, J, LSE>(p, row, st, ln, 0);
+        load_q<T, NV, LPH, VPL, J>(p, row, ln, true, q);
+        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
+        if (warp == 0) finish_row<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, ln.slot == 0);
         return;
     }
     bid -= p.n_cta;
@@ -527,6 +676,7 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
     if (task >= p.n_tasks) return;
     const int t0 = p.task_start[task];
     const int n = p.task_start[task + 1] - t0;
+    const int epw = Sh::epw(p);
     int32_t myrow = 0, mybeg = 0, myend = 0;
     if (ln.lane < n) {
         myrow = __ldg(p.warp_rows + t0 + ln.lane);
@@ -537,59 +687,55 @@ __global__ void __launch_bounds__(kLocalThreads, VPL == 1 ? 3 : 2) local_kernel(
             myrow = -1;   // (debug only) no edges, no output
         }
     }
-    const int steps = (n + p.epw - 1) / p.epw;
+    const int steps = (n + epw - 1) / epw;
     // step 0 prefetch: this slot's first row
     int k = ln.slot;
     int32_t row = __shfl_sync(0xffffffffu, myrow, k & 31);
     int32_t beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
     int32_t end = __shfl_sync(0xffffffffu, myend, k & 31);
     if (k >= n) beg = end = 0;
-    load_q_raw<T, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qr);
-    int32_t cols = first_cols<U, DBG>(p, beg, end, ln);
+    uint4 qn[VPL];
+    load_q<T, NV, LPH, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qn);
+    int32_t cols = first_cols<col_batch<T, NV, LPH, VPL, U, J>(), DBG>(p, beg, end, ln);
     for (int step = 0; step < steps; ++step) {
         const bool valid = k < n;
         const int32_t row_c = row;
         const int64_t beg_c = beg, end_c = end;
         const int32_t cols_c = cols;
-        scale_q<T, VPL>(p, qr, q);
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) q[v] = qn[v];
         // prefetch the next step's row while this one's gathers are in flight
-        k += p.epw;
+        k += epw;
         row = __shfl_sync(0xffffffffu, myrow, k & 31);
         beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
         end = __shfl_sync(0xffffffffu, myend, k & 31);
         if (k >= n) beg = end = 0;
-        load_q_raw<T, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qr);
-        cols = first_cols<U, DBG>(p, beg, end, ln);
-        slot_edges<T, VPL, U, DBG, J>(p, q, beg_c, end_c, cols_c, ln, st);
-        if (valid && (!DBG || row_c >= 0)) {
-            // every slot finishes its own row
-            constexpr int VEc = Io<T>::VE;
-            uint4 *Lout = static_cast<uint4 *>(p.L) + static_cast<int64_t>(row_c) * p.nvec;
-#pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                const int vid = vid_of<J, VPL>(v, ln.li);
-                const float inv_l = st.l[v] > 0.f ? 1.f / st.l[v] : 0.f;
-                float y[VEc];
-#pragma unroll
-                for (int e = 0; e < VEc; ++e) y[e] = st.acc[v][e] * inv_l;
-                if (vid < p.nvec) Lout[vid] = Io<T>::pack(y);
-            }
-            store_lse<T, VPL, J, LSE>(p, row_c, st, ln, true);
-        }
+        load_q<T, NV, LPH, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qn);
+        cols = first_cols<col_batch<T, NV, LPH, VPL, U, J>(), DBG>(p, beg, end, ln);
+        slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, beg_c, end_c, cols_c, ln, st);
+        // every slot finishes its own row
+        if (valid && (!DBG || row_c >= 0)) finish_row<T, NV, LPH, VPL, J, LSE>(p, row_c, st, ln, true);
     }
 }
 
-template <typename T, int VPL, int U, bool J = false>
-glga_status launch_local(Ctx *c, const LocalParams &p, cudaStream_t s) {
+template <typename T, int NV, int LPH, int VPL, int U, bool J, bool PIPE>
+glga_status launch_local(Ctx *c, LocalParams p, cudaStream_t s) {
+    using Sh = Shape<T, NV, LPH, VPL, J>;
+    if constexpr (NV != 0) {
+        // compile-time layout: its lane geometry replaces the generic one
+        p.lpe = Sh::kLpe;
+        p.epw = 32 / Sh::kLpe;
+        p.lph = LPH != 0 ? LPH : p.r / (Io<T>::VE * (J ? VPL : 1));
+    }
     const int64_t blocks = p.n_chunks + p.n_cta + p.task_blocks;
     if (blocks == 0) return GLGA_OK;
     const unsigned g = static_cast<unsigned>(blocks);
     if (c->opts.debug_checks) {
-        if (p.lse) local_kernel<T, VPL, U, true, J, true><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, VPL, U, true, J, false><<<g, kLocalThreads, 0, s>>>(p);
+        if (p.lse) local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE><<<g, kLocalThreads, 0, s>>>(p);
     } else {
-        if (p.lse) local_kernel<T, VPL, U, false, J, true><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, VPL, U, false, J, false><<<g, kLocalThreads, 0, s>>>(p);
+        if (p.lse) local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE><<<g, kLocalThreads, 0, s>>>(p);
     }
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
@@ -644,6 +790,16 @@ glga_status local_setup(Ctx *c) {
     return GLGA_OK;
 }
 
+#ifndef GLGA_LOCAL_V128
+#define GLGA_LOCAL_V128 0
+#endif
+#ifndef GLGA_LOCAL_V256
+#define GLGA_LOCAL_V256 0
+#endif
+#ifndef GLGA_LOCAL_V512
+#define GLGA_LOCAL_V512 0
+#endif
+
 glga_status local_run(Ctx *c, cudaStream_t s) {
     LocalParams p;
     p.row_ptr = c->row_ptr;
@@ -679,29 +835,48 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     p.n_rows = static_cast<int32_t>(c->N);
     p.flag = c->dev_flag;
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
-    // bf16 rows of 64 vectors (D = 512) with heads of >= 16 features: the joint layout,
-    // two consecutive vectors (16 features of one head) per lane.  (Measured: faster than
-    // the interleaved layout at D = 512, slower at D = 128, where its 118 registers leave
-    // 16 warps per SM instead of 24.)
-    if (c->io == GLGA_BF16 && c->r >= 16 && p.nvec == 64) {
-        p.lpe = p.nvec / 2;
-        p.epw = 32 / p.lpe;
-        p.lph = c->r / 16;
-        return launch_local<__nv_bfloat16, 2, 2, true>(c, p, s);
-    }
-    // U edges per slot step; U <= LPE so the slot's lanes can hold its column indices
-    if (c->io == GLGA_F32) {
-        if (vpl == 1 && lpe >= 4) return launch_local<float, 1, 4>(c, p, s);
-        if (vpl == 1 && lpe == 2) return launch_local<float, 1, 2>(c, p, s);
-        if (vpl == 1) return launch_local<float, 1, 1>(c, p, s);
-        if (vpl == 2) return launch_local<float, 2, 2>(c, p, s);
-        if (vpl <= 4) return launch_local<float, 4, 1>(c, p, s);
+    if (c->io == GLGA_BF16) {
+        using B = __nv_bfloat16;
+        // hot shapes with compile-time layouts (v: a lane's vectors interleave across the
+        // row; j: a lane's VPL vectors are consecutive features of one head)
+        if (p.nvec == 16 && c->r == 32) {   // D = 128, 4 heads of 32
+            switch (GLGA_LOCAL_V128) {
+                case 1: return launch_local<B, 16, 4, 1, 4, false, false>(c, p, s);
+                case 2: return launch_local<B, 16, 4, 1, 2, false, true>(c, p, s);
+                case 3: return launch_local<B, 16, 2, 2, 2, true, true>(c, p, s);
+                case 4: return launch_local<B, 16, 2, 2, 2, true, false>(c, p, s);
+                case 5: return launch_local<B, 16, 2, 2, 1, true, true>(c, p, s);
+                default: return launch_local<B, 16, 4, 1, 4, false, true>(c, p, s);
+            }
+        }
+        if (p.nvec == 32 && c->r == 32) {   // D = 256, 8 heads of 32
+            switch (GLGA_LOCAL_V256) {
+                case 1: return launch_local<B, 32, 2, 2, 2, true, false>(c, p, s);
+                case 2: return launch_local<B, 32, 2, 2, 2, true, true>(c, p, s);
+                case 3: return launch_local<B, 32, 4, 1, 4, false, false>(c, p, s);
+                default: return launch_local<B, 32, 4, 1, 4, false, true>(c, p, s);
+            }
+        }
+        if (p.nvec == 64 && c->r == 64) {   // D = 512, 8 heads of 64
+            switch (GLGA_LOCAL_V512) {
+                case 1: return launch_local<B, 64, 4, 2, 2, true, false>(c, p, s);
+                case 2: return launch_local<B, 64, 2, 4, 1, true, true>(c, p, s);
+                default: return launch_local<B, 64, 4, 2, 2, true, true>(c, p, s);
+            }
+        }
+        if (p.nvec == 64 && c->r >= 16) return launch_local<B, 64, 0, 2, 2, true, false>(c, p, s);
+        if (vpl == 1 && lpe >= 4) return launch_local<B, 0, 0, 1, 4, false, false>(c, p, s);
+        if (vpl == 1 && lpe == 2) return launch_local<B, 0, 0, 1, 2, false, false>(c, p, s);
+        if (vpl == 1) return launch_local<B, 0, 0, 1, 1, false, false>(c, p, s);
+        if (vpl == 2) return launch_local<B, 0, 0, 2, 2, false, false>(c, p, s);
+        if (vpl <= 4) return launch_local<B, 0, 0, 4, 1, false, false>(c, p, s);
     } else {
-        if (vpl == 1 && lpe >= 4) return launch_local<__nv_bfloat16, 1, 4>(c, p, s);
-        if (vpl == 1 && lpe == 2) return launch_local<__nv_bfloat16, 1, 2>(c, p, s);
-        if (vpl == 1) return launch_local<__nv_bfloat16, 1, 1>(c, p, s);
-        if (vpl == 2) return launch_local<__nv_bfloat16, 2, 2>(c, p, s);
-        if (vpl <= 4) return launch_local<__nv_bfloat16, 4, 1>(c, p, s);
+        // U edges per slot step; U <= LPE so the slot's lanes can hold its column indices
+        if (vpl == 1 && lpe >= 4) return launch_local<float, 0, 0, 1, 4, false, false>(c, p, s);
+        if (vpl == 1 && lpe == 2) return launch_local<float, 0, 0, 1, 2, false, false>(c, p, s);
+        if (vpl == 1) return launch_local<float, 0, 0, 1, 1, false, false>(c, p, s);
+        if (vpl == 2) return launch_local<float, 0, 0, 2, 2, false, false>(c, p, s);
+        if (vpl <= 4) return launch_local<float, 0, 0, 4, 1, false, false>(c, p, s);
     }
     set_error("row width too large for the local kernel");
     return GLGA_ERR_UNSUPPORTED;

@@ -15,6 +15,10 @@
 // float32 I/O uses kind::tf32 with a 3-term split: every operand x is stored as
 // hi = tf32(x) and lo = tf32(x - hi) and the accumulator receives hi*hi + hi*lo + lo*hi,
 // which keeps ~2^-21 relative accuracy (plain tf32 would give ~2^-11).
+//
+// The same kernel also serves as a plain GEMM with a float32 output (gemm_nt_f32out):
+// C [M][ncols] = A [M][K] B [ncols][K]^T, both operands K-major, bf16 on kind::f16 or
+// float32 on kind::tf32 with one term (the backward pass's input gradient).
 #include <algorithm>
 #include <cstdio>
 
@@ -47,6 +51,9 @@ struct GemmParams {
     void *Q;
     void *KV;
     float *t;
+    float *C;            // plain GEMM: float32 output [M][ldc] (first ncols columns), else null
+    int64_t ldc;
+    int32_t ncols;
     unsigned *flag;
 };
 
@@ -136,7 +143,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
     GemmParams p) {
     constexpr int kPlanes = SPLIT == 3 ? 2 : 1;
     constexpr int kPairs = SPLIT == 3 ? 3 : 1;
-    constexpr uint32_t kFmt = SPLIT == 3 ? 2u : 1u;
+    constexpr uint32_t kFmt = sizeof(T) == 4 ? 2u : 1u;   // tf32 or bf16 operands
 
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
@@ -287,7 +294,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
             const int ntile = tw.col;
             const int n0 = ntile * p.BN;
             const int bn = ntile == p.n_tiles - 1 ? p.bn_last : p.BN;
-            if (p.tma_epi) {
+            if (p.C) {
+                // plain GEMM: float32 rows of C, columns below ncols
+                for (int c0 = wg * 32; c0 < bn; c0 += 64) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + c0), v);
+                    tmem_ld_wait();
+                    const int gc0 = n0 + c0;
+                    if (row < p.M) {
+                        float *crow = p.C + row * p.ldc + gc0;
+                        if (gc0 + 32 <= p.ncols && (p.ldc & 3) == 0) {
+                            store_vec32<float>(crow, v);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (gc0 + j < p.ncols) crow[j] = __uint_as_float(v[j]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce_bar[buf]);
+            } else if (p.tma_epi) {
                 // Q/K/V columns go through a staging buffer (buffer i & 1 when there are
                 // two); the TMA store that last used it (tile i - sbufs) must have
                 // finished reading it first
@@ -462,6 +490,9 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     p.Q = c->Q;
     p.KV = c->kv_own;
     p.t = c->t;
+    p.C = nullptr;
+    p.ldc = 0;
+    p.ncols = 0;
     p.flag = c->dev_flag;
     const uint32_t staging = p.tma_epi ? static_cast<uint32_t>(p.sbufs) * (c->BN / 64) * kBM * kRowBytes : 0u;
     const size_t smem = static_cast<size_t>(p.stage_area) + staging + 1024;
@@ -481,6 +512,60 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
 }
 
 }  // namespace
+
+glga_status gemm_nt_f32out(Ctx *c, glga_dtype t, const void *A, int64_t M, int64_t lda, const void *B,
+                           int64_t ncols, int64_t ldb, int64_t K, float *C, int64_t ldc, cudaStream_t s) {
+    if (M <= 0 || ncols <= 0) return GLGA_OK;
+    const int elem = t == GLGA_F32 ? 4 : 2;
+    const int kt = kRowBytes / elem;                      // K elements per tile row
+    if ((lda * elem) % 16 || (ldb * elem) % 16 || K < 1 || K > lda || K > ldb || ncols > 1 << 20) {
+        set_error("gemm_nt_f32out: operand rows must be 16-byte multiples and hold K elements");
+        return GLGA_ERR_INVALID_ARG;
+    }
+    GemmParams p;
+    p.M = M;
+    p.BN = static_cast<int32_t>(std::min<int64_t>(256, ceil_div(ncols, 16) * 16));
+    p.n_tiles = static_cast<int32_t>(ceil_div(ncols, p.BN));
+    p.bn_last = static_cast<int32_t>(ceil_div(ncols - static_cast<int64_t>(p.n_tiles - 1) * p.BN, 16) * 16);
+    p.n_total_tiles = ceil_div(M, kBM) * p.n_tiles;
+    p.nk = static_cast<int32_t>(ceil_div(K, kt));
+    p.tma_epi = 0;
+    p.sbufs = 1;
+    p.tmem_cols = 512;
+    p.D = 0;
+    p.a_bytes = kBM * kRowBytes;
+    p.b_bytes = static_cast<uint32_t>(p.BN) * kRowBytes;
+    p.stage_bytes = p.a_bytes + p.b_bytes;
+    p.stages = std::max(1, std::min(kMaxStages, static_cast<int>((220u * 1024u) / p.stage_bytes)));
+    p.stage_area = static_cast<uint32_t>(p.stages) * p.stage_bytes;
+    p.Q = p.KV = nullptr;
+    p.t = nullptr;
+    p.C = C;
+    p.ldc = ldc;
+    p.ncols = static_cast<int32_t>(ncols);
+    p.flag = c->dev_flag;
+    const CUtensorMapDataType dt = t == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap ma, mb;
+    glga_status r = encode_tmap_2d(&ma, dt, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                                   static_cast<uint64_t>(lda) * elem, kt, kBM);
+    if (r == GLGA_OK)
+        r = encode_tmap_2d(&mb, dt, B, static_cast<uint64_t>(K), static_cast<uint64_t>(ncols),
+                           static_cast<uint64_t>(ldb) * elem, kt, static_cast<uint32_t>(p.BN));
+    if (r != GLGA_OK) return r;
+    const size_t smem = static_cast<size_t>(p.stage_area) + 1024;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(p.n_total_tiles, c->num_sms));
+    if (t == GLGA_F32) {
+        auto kern = proj_gemm_kernel<1, float>;
+        GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+        kern<<<grid, kGemmThreads, smem, s>>>(ma, ma, mb, mb, mb, mb, p);
+    } else {
+        auto kern = proj_gemm_kernel<1, __nv_bfloat16>;
+        GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+        kern<<<grid, kGemmThreads, smem, s>>>(ma, ma, mb, mb, mb, mb, p);
+    }
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
+}
 
 glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
                            uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
@@ -607,7 +692,10 @@ glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK
     }
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
-    if (c->N == 0) return GLGA_OK;
+    if (c->N == 0) {
+        if (c->timing) GLGA_CUDA(record_stage(c, kStageGemm, s));
+        return GLGA_OK;
+    }
     const CUtensorMapDataType dt =
         c->io == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (c->x_direct) {
@@ -629,7 +717,7 @@ glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK
         GLGA_CUDA(cudaGetLastError());
         c->launches += 1;
     }
-    if (c->timing) GLGA_CUDA(cudaEventRecord(c->ev[kStageGemm], s));
+    if (c->timing) GLGA_CUDA(record_stage(c, kStageGemm, s));
     if (c->io == GLGA_F32) return launch_gemm<3, float>(c, s);
     return launch_gemm<1, __nv_bfloat16>(c, s);
 }

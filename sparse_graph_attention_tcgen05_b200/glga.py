@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         "glga_workspace_bytes": ([_vp, ctypes.POINTER(_i64)], _i32),
         "glga_kernel_launches": ([_vp, ctypes.POINTER(_i64)], _i32),
         "glga_global_stats_static": ([_vp, _i64, _i32, _i32, _i32, _vp, _vp], _i32),
+        "glga_global_stats_static_error": ([_vp], _i32),
+        "glga_debug_static_bounded_wait": ([_i64, _vp], _i32),
         "glga_last_device_error": ([_vp, _vp], _i32),
         "glga_debug_bounded_wait": ([_vp, _i64, _vp], _i32),
         "glga_debug_set_col_idx": ([_vp, _i64, _i32, _vp], _i32),
@@ -148,6 +150,12 @@ def global_stats_static(KV: torch.Tensor, H: int, r: int, io: str, Sz=None, stre
     return Sz
 
 
+def global_stats_static_error(stream=None) -> int:
+    """Status of the global_stats_static calls on the current device since the last report
+    (glga_global_stats_static_error; synchronises the stream and clears the flag)."""
+    return int(lib().glga_global_stats_static_error(_stream(stream)))
+
+
 class Layer:
     """One gated local-global graph-attention layer bound to a fixed graph.
 
@@ -203,7 +211,9 @@ class Layer:
         (refill them in place between replays; b_g and eps are fixed at capture).  The
         forward enqueues kernels only (no allocation, no host synchronisation, tensor maps
         passed by value), so it records whole; one eager call first settles the lazy
-        per-kernel attributes outside the capture.  Stage timing must be off."""
+        per-kernel attributes outside the capture.  With stage timing on, the stage events
+        are captured as event record nodes, so stage_times() after a replay reports that
+        replay's stages."""
         if Y is None:
             Y = torch.empty(self.N, self.D, dtype=self.dtype, device=X.device)
         side = torch.cuda.Stream(device=X.device)
@@ -273,8 +283,8 @@ class Layer:
         """Records one glga_backward on these buffers into a CUDA graph and returns
         (graph, grads): graph.replay() recomputes the gradients into the same tensors from
         the state of the last forward (run forward() or its graph first when the inputs
-        change).  The backward enqueues kernels, events between its two streams and, for
-        bf16 layers, cuBLAS GEMMs on a preset workspace, so it records whole; one eager call
+        change).  The backward enqueues kernels and events between its two streams (the
+        tensor maps of its GEMMs passed by value), so it records whole; one eager call
         first settles the lazily loaded kernels outside the capture."""
         side = torch.cuda.Stream(device=X.device)
         side.wait_stream(torch.cuda.current_stream())

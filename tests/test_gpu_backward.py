@@ -9,6 +9,7 @@ import torch
 
 import oracle
 from oracle.backward import backward as ref_backward
+from oracle.backward import backward_chunked
 from sparse_graph_attention_tcgen05_b200 import glga
 from sparse_graph_attention_tcgen05_b200.workloads import make_custom, make_workload, round_to_bf16
 from tests.gpu_helpers import to_dev
@@ -37,14 +38,15 @@ def _run(w, dY, options=None):
     return {k: v.cpu().numpy().astype(np.float64) for k, v in g1.items()}
 
 
-def _check(w, seed=0):
+def _check(w, seed=0, chunked=False):
     rng = np.random.default_rng(seed)
     dY = rng.standard_normal((w.N, w.D)).astype(np.float32)
     if w.io == "bf16":
         dY = round_to_bf16(dY)
     got = _run(w, dY)
     rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
-    ref = ref_backward(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY)
+    ref_fn = backward_chunked if chunked else ref_backward
+    ref = ref_fn(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY)
     for k in NAMES:
         r = np.asarray(ref[k], dtype=np.float64).reshape(got[k].shape)
         scale = max(np.abs(r).max(), 1e-30)
@@ -62,6 +64,14 @@ def test_citation_fp32():
 
 def test_arxiv_shape_bf16():
     _check(make_workload("arxiv", scale=0.02))
+
+
+def test_arxiv_full_size_bf16():
+    """The configuration `bench.py --backward` times: the whole arxiv-shaped graph (N =
+    169,343, E = 2,474,639; rows of up to 22,812 entries cut into 32-entry chunks; target
+    and source sides on two streams), every gradient tensor compared in full with the
+    float64 reference taken one group of target rows at a time."""
+    _check(make_workload("arxiv"), chunked=True)
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
@@ -105,3 +115,14 @@ def test_very_heavy_target_and_source(io):
     src = np.concatenate([rng.integers(0, N, 5000), np.full(5000, 11), rng.integers(0, N, 3 * N)])
     w = make_custom(N, 32, 2, 16, src.astype(np.int32), dst.astype(np.int32), io=io, seed=9, b_g=-0.2)
     _check(w, seed=10)
+
+
+def test_bf16_rows_not_16_byte_multiples():
+    # d = 13: X rows of 26 bytes cannot be loaded by TMA, so this bf16 layer's dW and dX run
+    # on the CUDA-core GEMM kernels instead of the tensor-core ones
+    rng = np.random.default_rng(21)
+    N = 257
+    dst = np.concatenate([np.repeat(np.arange(N), 3), np.full(90, 5)])
+    src = rng.integers(0, N, dst.shape[0])
+    w = make_custom(N, 13, 2, 16, src.astype(np.int32), dst.astype(np.int32), io="bf16", seed=23, b_g=0.4)
+    _check(w, seed=24)

@@ -1,9 +1,10 @@
 """Row-sharded forward on the GPU (glga_create_sharded, glga_forward_begin/end).
 
 With one GPU the ranks are emulated one after another in this process: every shard runs
-its begin phase, the test copies each owner's K/V rows into every other shard's buffer and
-stacks the partial statistics in rank order (what the NCCL broadcasts and all-gather do
-between processes), then every shard runs its end phase.  No kernel waits on another
+its begin phase, the test copies each owner's block of K/V rows (the padded layout of
+sharded.ShardPlan) into every other shard's buffer and stacks the partial statistics in
+rank order (what the two NCCL all-gathers do between processes), then every shard runs
+its end phase.  No kernel waits on another
 rank.  A one-rank NCCL process group runs sharded.ShardedForward's real collectives."""
 import socket
 
@@ -14,7 +15,7 @@ import torch.distributed as dist
 
 import oracle
 from sparse_graph_attention_tcgen05_b200 import glga
-from sparse_graph_attention_tcgen05_b200.sharded import LibraryShard, ShardedForward, partition_rows, shard_csr
+from sparse_graph_attention_tcgen05_b200.sharded import LibraryShard, ShardedForward, ShardPlan, partition_rows
 from sparse_graph_attention_tcgen05_b200.workloads import make_workload
 from tests.gpu_helpers import assert_close_to_oracle, run_gpu, to_dev
 
@@ -26,16 +27,17 @@ def _emulate(w, bounds, csr):
     P = len(bounds) - 1
     dt = glga.torch_dtype(w.io)
     W = [to_dev(a, dt) for a in (w.W_Q, w.W_K, w.W_V, w.w_g)]
-    shards = []
+    shards, plans = [], []
     for p in range(P):
-        b0, b1 = int(bounds[p]), int(bounds[p + 1])
-        rpo, cio = shard_csr(rp, ci, b0, b1)
-        sh = LibraryShard(w.N, w.d, w.H, w.r, w.io, rpo, cio, b0, b1)
-        sh.begin(to_dev(w.X[b0:b1], dt), *W)
+        plan = ShardPlan(rp, ci, P, p, bounds=bounds)
+        sh = LibraryShard(plan.n_kv, w.d, w.H, w.r, w.io, plan.row_ptr, plan.col_idx, plan.kv0, plan.kv1)
+        sh.kv.fill_(float("nan"))                            # padding rows are never read
+        sh.begin(to_dev(w.X[plan.b0:plan.b1], dt), *W)
         shards.append(sh)
+        plans.append(plan)
     torch.cuda.synchronize()
-    for p, owner in enumerate(shards):                       # the K/V exchange
-        a, b = int(bounds[p]), int(bounds[p + 1])
+    for plan, owner in zip(plans, shards):                   # the K/V exchange
+        a, b = plan.kv0, plan.kv1
         for other in shards:
             if other is not owner and b > a:
                 other.kv[a:b].copy_(owner.kv[a:b])
@@ -93,10 +95,10 @@ def test_one_rank_nccl_group_equals_the_plain_layer(io_name):
     csr = oracle.csr_from_coo(w.N, w.src, w.dst)
     dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
     try:
-        bounds = partition_rows(csr[0], 1)
-        sh = LibraryShard(w.N, w.d, w.H, w.r, w.io, csr[0], csr[1], 0, w.N)
+        plan = ShardPlan(csr[0], csr[1], 1, 0)
+        sh = LibraryShard(plan.n_kv, w.d, w.H, w.r, w.io, plan.row_ptr, plan.col_idx, plan.kv0, plan.kv1)
         dt = glga.torch_dtype(w.io)
-        fwd = ShardedForward(sh, bounds, 0, 1)
+        fwd = ShardedForward(sh, 0, 1)
         Y = fwd(*(to_dev(a, dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)), w.b_g, w.eps)
         torch.cuda.synchronize()
         assert sh.last_device_error() == 0

@@ -2,8 +2,8 @@
 begin -> exchange -> end protocol of sharded.ShardedForward on two and three gloo ranks
 (one process each).  The ranks' arithmetic is done by a float64 stand-in built from the
 oracle (test infrastructure; the product's shards run libglga), so the test checks that
-the partition, the K/V broadcasts and the rank-ordered sum of the partial statistics
-reproduce the unsharded layer."""
+the partition, the padded K/V layout and its all-gather, and the rank-ordered sum of the
+partial statistics reproduce the unsharded layer."""
 import os
 import socket
 
@@ -14,7 +14,8 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
-from sparse_graph_attention_tcgen05_b200.sharded import ShardedForward, partition_rows, shard_csr
+from sparse_graph_attention_tcgen05_b200.sharded import (ShardedForward, ShardPlan, block_rows, padded_positions,
+                                                         partition_rows, shard_csr)
 from sparse_graph_attention_tcgen05_b200.workloads import make_workload
 
 
@@ -34,13 +35,30 @@ def test_partition_is_contiguous_and_balances_entries():
     np.testing.assert_array_equal(partition_rows(np.zeros(11, np.int64), 5), [0, 2, 4, 6, 8, 10])
 
 
-class OracleShard:
-    """float64 CPU stand-in for sharded.LibraryShard (same interface)."""
+def test_padded_positions_are_block_offsets():
+    bounds = np.array([0, 3, 3, 10, 12])                 # block 1 is empty, B = 7
+    assert block_rows(bounds) == 7
+    np.testing.assert_array_equal(padded_positions(bounds, np.arange(12)),
+                                  [0, 1, 2, 14, 15, 16, 17, 18, 19, 20, 21, 22])
+    rp = np.array([0, 2, 2, 5, 6, 6, 6, 7, 9, 9, 10, 11, 12])
+    ci = np.array([0, 11, 3, 4, 9, 2, 10, 1, 7, 5, 6, 8])
+    rpo, cio = shard_csr(rp, ci, 3, 10, bounds)
+    np.testing.assert_array_equal(rpo, [0, 1, 1, 1, 2, 4, 4, 5])
+    np.testing.assert_array_equal(cio, padded_positions(bounds, ci[5:10]))
+    plan = ShardPlan(rp, ci, 4, 2)
+    assert plan.B == block_rows(plan.bounds) and plan.n_kv == 4 * plan.B
+    assert plan.kv0 == 2 * plan.B and plan.kv1 - plan.kv0 == plan.b1 - plan.b0
 
-    def __init__(self, w, rp_own, ci_own, b0, b1):
+
+class OracleShard:
+    """float64 CPU stand-in for sharded.LibraryShard (same interface; K/V buffer in the
+    padded layout of ShardPlan)."""
+
+    def __init__(self, w, plan):
+        rp_own, ci_own, b0, b1 = plan.row_ptr, plan.col_idx, plan.kv0, plan.kv1
         self.w, self.b0, self.b1 = w, b0, b1
         self.D = w.H * w.r
-        self.kv = torch.zeros(w.N, 2 * self.D, dtype=torch.float64)
+        self.kv = torch.full((plan.n_kv, 2 * self.D), float("nan"), dtype=torch.float64)
         self.n_part = w.H * w.r * (w.r + 1)
         self.own = torch.zeros(self.n_part, dtype=torch.float64)
         self.rp, self.ci = rp_own, ci_own
@@ -79,12 +97,10 @@ def _rank_main(rank, world, port, name, results):
     try:
         w = make_workload(name)
         rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
-        b = partition_rows(rp, world)
-        b0, b1 = int(b[rank]), int(b[rank + 1])
-        rpo, cio = shard_csr(rp, ci, b0, b1)
-        fwd = ShardedForward(OracleShard(w, rpo, cio, b0, b1), b, rank, world)
-        Y = fwd(w.X[b0:b1], w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps)
-        results[rank] = (b0, b1, Y.numpy())
+        plan = ShardPlan(rp, ci, world, rank)
+        fwd = ShardedForward(OracleShard(w, plan), rank, world)
+        Y = fwd(w.X[plan.b0:plan.b1], w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps)
+        results[rank] = (plan.b0, plan.b1, Y.numpy())
     finally:
         dist.destroy_process_group()
 
