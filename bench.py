@@ -237,17 +237,17 @@ class TimedRegion:
         self.evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     for _ in range(R)]
 
-    def step(self, run_fwd):
-        for a, b in self.evs:
+    def step(self, run_fwd, run_last=None):
+        for i, (a, b) in enumerate(self.evs):
             self.flush.zero_()
             a.record(self.stream)
-            run_fwd()
+            (run_last if run_last is not None and i == self.R - 1 else run_fwd)()
             b.record(self.stream)
         self.evs[-1][1].synchronize()
         self.last_ms = self.evs[-1][0].elapsed_time(self.evs[-1][1])   # the step's last forward
         return sum(a.elapsed_time(b) for a, b in self.evs)
 
-    def run(self, run_fwd, K, gpu_index, barrier=None, after_step=None):
+    def run(self, run_fwd, K, gpu_index, barrier=None, after_step=None, run_last=None):
         import torch
         if barrier:
             barrier()
@@ -256,7 +256,7 @@ class TimedRegion:
         wall0 = time.perf_counter()
         step_ms = []
         for _ in range(K):
-            step_ms.append(self.step(run_fwd))
+            step_ms.append(self.step(run_fwd, run_last))
             if after_step:
                 after_step()
         torch.cuda.synchronize()
@@ -757,25 +757,27 @@ def run_single(args, rank, world, local_rank, mode):
              "note": "glga_forward called per forward, stage events on"}
 
     # ---- timed region: K steps of R forwards, each a replay of a CUDA graph of
-    # glga_forward (the same kernels on the same buffers, no host work between them) with
-    # the library's stage events inside the graph; eager calls if the capture is refused ----
-    graph, graph_timing = None, False
+    # glga_forward (the same kernels on the same buffers, no host work between them); the
+    # last forward of every step replays a second graph that also records the library's
+    # stage events (event record nodes), for the local kernel's launch time; eager calls
+    # if the capture is refused ----
+    graph, graph_t = None, None
+    layer.set_timing(False)
     try:
-        graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)   # timing still on
-        graph.replay()
-        torch.cuda.synchronize()
-        layer.stage_times()
-        graph_timing = True
-    except (RuntimeError, glga.GLGAError) as exc:
-        eager["capture_with_stage_events"] = str(exc).splitlines()[0][:200]
-        graph = None
-    if graph is None:
-        layer.set_timing(False)
+        graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)
+    except RuntimeError as exc:
+        eager["capture_refused"] = str(exc).splitlines()[0][:200]
+    if graph is not None:
+        layer.set_timing(True)
         try:
-            graph, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)
-        except RuntimeError as exc:
-            eager["capture_refused"] = str(exc).splitlines()[0][:200]
-            graph = None
+            graph_t, _ = layer.capture(X, WQ, WK, WV, wg, w.b_g, w.eps, Y=Y)
+            graph_t.replay()
+            torch.cuda.synchronize()
+            layer.stage_times()
+        except (RuntimeError, glga.GLGAError) as exc:
+            eager["capture_with_stage_events"] = str(exc).splitlines()[0][:200]
+            graph_t = None
+            layer.set_timing(False)
     run_step = graph.replay if graph is not None else fwd
     for _ in range(args.warmup):
         run_step()
@@ -788,14 +790,15 @@ def run_single(args, rank, world, local_rank, mode):
         fwd_check.append(st["forward"] / tr.last_ms)
     step_ms, clocks, wall = tr.run(run_step, args.steps, gpu_index_of(local_rank),
                                    barrier=barrier if world > 1 else None,
-                                   after_step=after if graph_timing else None)
+                                   after_step=after if graph_t is not None else None,
+                                   run_last=graph_t.replay if graph_t is not None else None)
     layer.set_timing(False)
     # the graph's stage events must span the same forward as the outer events
     if fwd_check and not 0.8 <= float(np.median(fwd_check)) <= 1.05:
         eager["graph_stage_events"] = f"rejected (forward span / outer events = {float(np.median(fwd_check)):.3f})"
         local_ms = []
     graph_ok = graph is not None
-    del graph
+    del graph, graph_t
     assert layer.last_device_error() == 0
     n_fwd = args.steps * args.forwards_per_step
     launches = int(round(launches_per_forward * n_fwd))
@@ -812,7 +815,8 @@ def run_single(args, rank, world, local_rank, mode):
 
     peaks, peak_kind = load_peaks()
     if local_ms:
-        t_local, src_t = float(np.mean(local_ms)), "stage events inside the replayed graph, one forward per timed step"
+        t_local, src_t = float(np.mean(local_ms)), ("stage events recorded inside the replayed graph of the "
+                                                    "last forward of every timed step")
     else:
         t_local, src_t = stages["local"], "stage events of the eager forwards"
     roofline = roofline_local(w, t_local, peaks, peak_kind, profiled_counters(args.workload), src_t)

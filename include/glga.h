@@ -88,7 +88,8 @@ typedef struct {
     int32_t backward;
 } glga_options;
 
-/* Fills *opts with the defaults used when glga_create gets opts == NULL. */
+/* Fills *opts with the defaults used when glga_create gets opts == NULL:
+ * warp_max_degree 256, chunk_edges 2048, no debug checks, no backward workspaces.     */
 GLGA_API glga_status glga_default_options(glga_options *opts);
 
 /* glga_create -- bind a fixed graph and the layer shape; allocate all workspaces.

@@ -147,8 +147,8 @@ glga_status glga_default_options(glga_options *opts) {
         set_error("glga_default_options: null pointer");
         return GLGA_ERR_INVALID_ARG;
     }
-    opts->warp_max_degree = 128;
-    opts->chunk_edges = 1024;
+    opts->warp_max_degree = 256;
+    opts->chunk_edges = 2048;
     opts->debug_checks = 0;
     opts->debug_fail_alloc = 0;
     opts->backward = 0;

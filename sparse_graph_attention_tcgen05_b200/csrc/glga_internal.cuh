@@ -78,7 +78,7 @@ struct Ctx {
     int32_t BN = 0, bn_last = 0, n_tiles = 0, stages = 0, tmem_cols = 0;
     bool gemm_tma_epi = false;    // Q/K/V stored through shared memory + TMA
     int32_t gemm_sbufs = 2;       // staging buffers of that epilogue (1 or 2)
-    TensorMap2D tmKVs;            // KV store map (64-column boxes)
+    TensorMap2D tmKVs, tmQs;      // K|V and Q store maps (64-column x 32-row boxes)
     int split = 1;                // 1: bf16 MMA; 3: 3-term tf32 split (fp32 io)
     bool x_direct = false;        // A operand read straight from the caller's X
     void *Wt = nullptr;           // [planes][Dp][dp]

@@ -10,10 +10,13 @@
 // second MMA against a constant "ones" column.  Only the diagonal r x r blocks (one per
 // head) are kept.
 //
-// Deterministic split-N tree: the nodes are cut into P fixed ranges, each CTA
-// accumulates its range in TMEM in node-tile order, writes its partial sums, and a
-// reduction adds the P partials in range order.  The reduction also writes S and z into
-// the block-diagonal operand of the readout GEMM.  Output layout: S [H][r][r], z [H][r].
+// Deterministic split-N tree: the nodes are cut into P fixed ranges; the CTAs of a
+// feature block walk the ranges g, g + G, g + 2G, ... (persistent when ranges are many,
+// as with per-segment statistics), accumulating each range in TMEM in node-tile order
+// (two accumulators, so a range's epilogue overlaps the next range's MMAs) and writing
+// its partial sums; a reduction adds the P partials in range order.  The reduction also
+// writes S and z into the block-diagonal operand of the readout GEMM.  Output layout:
+// S [H][r][r], z [H][r].
 #include <algorithm>
 #include <mutex>
 #include <vector>
@@ -26,10 +29,13 @@ namespace {
 constexpr int kFB = 128;             // features per block: MMA M (phi(K)) and N (V)
 constexpr int kRowBytes = 128;
 constexpr int kMaxStages = 6;
-constexpr int kWorkers = 512;        // warps 0-15: phi / split passes; warps 0-3: epilogue
+constexpr int kWorkers = 512;        // warps 0-15: phi / split passes
+constexpr int kWorkerWarps = kWorkers / 32;
 constexpr int kProdWarp = 16;        // TMA producer
 constexpr int kMmaWarp = 17;         // TMEM owner and MMA issuer
-constexpr int kThreads = 576;
+constexpr int kEpiWarp0 = 18;        // warps 18-21: epilogue (partial sums of each range)
+constexpr int kThreads = 704;
+constexpr uint32_t kAccStride = 256; // TMEM columns between the two accumulators
 
 template <typename T>
 struct StatsGeom {
@@ -44,10 +50,12 @@ struct StatsGeom {
 struct StatsParams {
     int64_t N;
     int32_t D, H;
+    int32_t n_parts;         // P row ranges, walked by gridDim.x CTAs per feature block
     int64_t rows_per_part;   // multiple of the stage height (when part_ptr is NULL)
     const int32_t *part_ptr; // explicit row ranges [P + 1] (segments), or NULL
     int32_t stages;
     uint32_t stage_bytes;
+    uint32_t scratch_off;    // epilogue staging in dynamic shared memory (0: direct stores)
     float *part;             // [P][H][r][r+1]
     unsigned *flag;
 };
@@ -68,18 +76,27 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t ready_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
-    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ __align__(8) uint64_t accf_bar[2];   // MMA -> epilogue: a range is accumulated
+    __shared__ __align__(8) uint64_t acce_bar[2];   // epilogue -> MMA: the accumulator is drained
     __shared__ uint32_t tmem_base_sh;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *ones = smem + static_cast<size_t>(p.stages) * p.stage_bytes;   // 16 x 128 B, K-major
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int part = blockIdx.x, fb = blockIdx.y;
-    // row range [r0, r1) of this part; rows of the last tile past r1 get phi(k) = 0
-    const int64_t r0 = p.part_ptr ? p.part_ptr[part] : static_cast<int64_t>(part) * p.rows_per_part;
-    const int64_t r1 = p.part_ptr ? p.part_ptr[part + 1] : std::min<int64_t>(p.N, r0 + p.rows_per_part);
-    const int ntiles = r1 > r0 ? static_cast<int>(ceil_div(r1 - r0, G::kRows)) : 0;
+    const int fb = blockIdx.y;
+    // this CTA's ranges: blockIdx.x, blockIdx.x + gridDim.x, ...
+    const int n_my = p.n_parts > static_cast<int>(blockIdx.x)
+                         ? (p.n_parts - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x
+                         : 0;
+    // row range [r0, r1) of range `part`; rows of its last tile past r1 get phi(k) = 0
+    auto range_of = [&](int part, int64_t &r0, int64_t &r1) {
+        r0 = p.part_ptr ? p.part_ptr[part] : static_cast<int64_t>(part) * p.rows_per_part;
+        r1 = p.part_ptr ? p.part_ptr[part + 1] : std::min<int64_t>(p.N, r0 + p.rows_per_part);
+    };
+    auto tiles_of = [&](int64_t r0, int64_t r1) {
+        return r1 > r0 ? static_cast<int>(ceil_div(r1 - r0, G::kRows)) : 0;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -87,7 +104,10 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             mbar_init(&ready_bar[s], kWorkers);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&done_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf_bar[b], 1);
+            mbar_init(&acce_bar[b], 4);
+        }
         fence_mbar_init();
     }
     if (threadIdx.x < kWorkers) {
@@ -99,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
         fence_async_smem();
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(&tmem_base_sh, 256u);
+        tmem_alloc(&tmem_base_sh, 512u);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -114,22 +134,27 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             int issued = 0;
             RingPos rp;
             bool ok = true;
-            for (int it = 0; it < ntiles; ++it, rp.next(p.stages)) {
-                const int s = rp.slot;
-                if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
-                mbar_arrive_expect_tx(&full_bar[s], 2 * G::kOpBytes);
-                const int32_t y = static_cast<int32_t>(r0 + static_cast<int64_t>(it) * G::kRows);
+            for (int k = 0; k < n_my && ok; ++k) {
+                int64_t r0, r1;
+                range_of(static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), r0, r1);
+                const int ntiles = tiles_of(r0, r1);
+                for (int it = 0; it < ntiles; ++it, rp.next(p.stages)) {
+                    const int s = rp.slot;
+                    if (issued >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+                    mbar_arrive_expect_tx(&full_bar[s], 2 * G::kOpBytes);
+                    const int32_t y = static_cast<int32_t>(r0 + static_cast<int64_t>(it) * G::kRows);
 #pragma unroll
-                for (int b = 0; b < G::kBoxes; ++b) {
-                    const int32_t x = fb * kFB + b * (kRowBytes / static_cast<int>(sizeof(T)));
-                    tma_load_2d(st + b * G::kBoxBytes, &tmK, &full_bar[s], x, y);
-                    tma_load_2d(st + G::kOpBytes + b * G::kBoxBytes, &tmV, &full_bar[s], x, y);
+                    for (int b = 0; b < G::kBoxes; ++b) {
+                        const int32_t x = fb * kFB + b * (kRowBytes / static_cast<int>(sizeof(T)));
+                        tma_load_2d(st + b * G::kBoxBytes, &tmK, &full_bar[s], x, y);
+                        tma_load_2d(st + G::kOpBytes + b * G::kBoxBytes, &tmV, &full_bar[s], x, y);
+                    }
+                    ++issued;
                 }
-                ++issued;
             }
             if (!ok) {
                 atomicOr(p.flag, kDevErrTimeout);
@@ -146,92 +171,109 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             const uint64_t dones = smem_desc(smem_u32(ones), 16, 1024, 2);
             bool ok = true;
             RingPos rp;
-            for (int it = 0; it < ntiles; ++it, rp.next(p.stages)) {
-                const int s = rp.slot;
-                if (!mbar_wait_bounded(&ready_bar[s], rp.phase)) {
+            for (int k = 0; k < n_my && ok; ++k) {
+                const int buf = k & 1;
+                const uint32_t acc_base = tmem + static_cast<uint32_t>(buf) * kAccStride;
+                // the epilogue must have drained this accumulator's previous range (k - 2)
+                if (k >= 2 && !mbar_wait_bounded(&acce_bar[buf], static_cast<uint32_t>((k >> 1) - 1) & 1u)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t kb = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
-                const uint32_t vb = kb + G::kOpBytes;
-#pragma unroll
-                for (int ks = 0; ks < G::kRows / G::kUK; ++ks) {
-                    const uint32_t off = ks * G::kUK * kRowBytes;
-                    const uint32_t acc0 = (it | ks) != 0;
-                    if (SPLIT == 3) {
-                        // tf32 operands were transposed to K-major planes by warps 0-3
-                        // (MN-major tf32 would need the 32-byte-atom swizzle)
-                        const uint32_t kt = ks * 32;   // 8 node rows of tf32 = 32 bytes
-                        const uint32_t ah = kb + 2 * G::kOpBytes, al = kb + 3 * G::kOpBytes;
-                        const uint32_t bh = kb + 4 * G::kOpBytes, bl = kb + 5 * G::kOpBytes;
-                        const uint64_t akh = smem_desc(ah + kt, 16, 1024, 2);
-                        const uint64_t akl = smem_desc(al + kt, 16, 1024, 2);
-                        const uint64_t bvh = smem_desc(bh + kt, 16, 1024, 2);
-                        const uint64_t bvl = smem_desc(bl + kt, 16, 1024, 2);
-                        umma_tf32(tmem, akh, bvh, idSk, acc0);
-                        umma_tf32(tmem, akh, bvl, idSk, 1u);
-                        umma_tf32(tmem, akl, bvh, idSk, 1u);
-                        umma_tf32(tmem + kFB, akh, dones, idZk, acc0);
-                        umma_tf32(tmem + kFB, akl, dones, idZk, 1u);
-                        (void)off;
-                    } else {
-                        const uint64_t ak = smem_desc(kb + off, G::kBoxBytes, 1024, 2);
-                        const uint64_t bv = smem_desc(vb + off, G::kBoxBytes, 1024, 2);
-                        umma_bf16(tmem, ak, bv, idS, acc0);
-                        umma_bf16(tmem + kFB, ak, dones, idZ, acc0);
+                int64_t r0, r1;
+                range_of(static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), r0, r1);
+                const int ntiles = tiles_of(r0, r1);
+                for (int it = 0; it < ntiles; ++it, rp.next(p.stages)) {
+                    const int s = rp.slot;
+                    if (!mbar_wait_bounded(&ready_bar[s], rp.phase)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+                    const uint32_t kb = smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes);
+                    const uint32_t vb = kb + G::kOpBytes;
+#pragma unroll
+                    for (int ks = 0; ks < G::kRows / G::kUK; ++ks) {
+                        const uint32_t off = ks * G::kUK * kRowBytes;
+                        const uint32_t acc0 = (it | ks) != 0;
+                        if (SPLIT == 3) {
+                            // tf32 operands were transposed to K-major planes by the workers
+                            // (MN-major tf32 would need the 32-byte-atom swizzle)
+                            const uint32_t kt = ks * 32;   // 8 node rows of tf32 = 32 bytes
+                            const uint32_t ah = kb + 2 * G::kOpBytes, al = kb + 3 * G::kOpBytes;
+                            const uint32_t bh = kb + 4 * G::kOpBytes, bl = kb + 5 * G::kOpBytes;
+                            const uint64_t akh = smem_desc(ah + kt, 16, 1024, 2);
+                            const uint64_t akl = smem_desc(al + kt, 16, 1024, 2);
+                            const uint64_t bvh = smem_desc(bh + kt, 16, 1024, 2);
+                            const uint64_t bvl = smem_desc(bl + kt, 16, 1024, 2);
+                            umma_tf32(acc_base, akh, bvh, idSk, acc0);
+                            umma_tf32(acc_base, akh, bvl, idSk, 1u);
+                            umma_tf32(acc_base, akl, bvh, idSk, 1u);
+                            umma_tf32(acc_base + kFB, akh, dones, idZk, acc0);
+                            umma_tf32(acc_base + kFB, akl, dones, idZk, 1u);
+                            (void)off;
+                        } else {
+                            const uint64_t ak = smem_desc(kb + off, G::kBoxBytes, 1024, 2);
+                            const uint64_t bv = smem_desc(vb + off, G::kBoxBytes, 1024, 2);
+                            umma_bf16(acc_base, ak, bv, idS, acc0);
+                            umma_bf16(acc_base + kFB, ak, dones, idZ, acc0);
+                        }
+                    }
+                    umma_commit(&empty_bar[s]);
                 }
-                umma_commit(&empty_bar[s]);
+                // (a range without rows commits at once; its epilogue writes zeros)
+                if (ok) umma_commit(&accf_bar[buf]);
             }
             if (!ok) atomicOr(p.flag, kDevErrTimeout);
-            umma_commit(&done_bar);
         }
-    } else {
-        // ---------------- warps 0-3: phi(K) (zero past the range), tf32 split ----------
+    } else if (warp < kWorkerWarps) {
+        // ---------------- warps 0-15: phi(K) (zero past the range), tf32 split ----------
         bool ok = true;
         constexpr int kChunksPerBox = G::kBoxBytes / 16;
         RingPos rp;
-        for (int it = 0; it < ntiles && ok; ++it, rp.next(p.stages)) {
-            const int s = rp.slot;
-            if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
-                ok = false;
-                break;
-            }
-            uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
-            const int64_t y0 = r0 + static_cast<int64_t>(it) * G::kRows;
-            if (SPLIT == 3) {
-                // Transpose the [node][feature] TMA tiles (128-byte swizzle) into K-major
-                // planes [feature][node] with the same swizzle, applying phi and the tf32
-                // split on the way: element (m, k) of a plane sits at
-                // (m/8)*1024 + (m%8)*128 + (((k/4) ^ (m%8)) * 16) + (k%4)*4.
-                const float *rk = reinterpret_cast<const float *>(st);
-                const float *rv = reinterpret_cast<const float *>(st + G::kOpBytes);
-                float *ah = reinterpret_cast<float *>(st + 2 * G::kOpBytes);
-                float *al = reinterpret_cast<float *>(st + 3 * G::kOpBytes);
-                float *bh = reinterpret_cast<float *>(st + 4 * G::kOpBytes);
-                float *bl = reinterpret_cast<float *>(st + 5 * G::kOpBytes);
-                for (int idx = threadIdx.x; idx < G::kRows * kFB; idx += kWorkers) {
-                    const int k = idx / kFB, m = idx % kFB;
-                    const int e = m % 32;
-                    const int src = ((m / 32) * G::kBoxBytes + k * kRowBytes +
-                                     (((e / 4) ^ (k % 8)) * 16) + (e % 4) * 4) / 4;
-                    const int dst = ((m / 8) * 1024 + (m % 8) * kRowBytes +
-                                     (((k / 4) ^ (m % 8)) * 16) + (k % 4) * 4) / 4;
-                    const bool valid = y0 + k < r1;
-                    const float f = valid ? phi(rk[src]) : 0.f;
-                    const float v = rv[src];
-                    const float fh = to_tf32(f), vh = to_tf32(v);
-                    ah[dst] = fh;
-                    al[dst] = to_tf32(f - fh);
-                    bh[dst] = vh;
-                    bl[dst] = to_tf32(v - vh);
+        for (int k = 0; k < n_my && ok; ++k) {
+            int64_t r0, r1;
+            range_of(static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), r0, r1);
+            const int ntiles = tiles_of(r0, r1);
+            for (int it = 0; it < ntiles && ok; ++it, rp.next(p.stages)) {
+                const int s = rp.slot;
+                if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
+                    ok = false;
+                    break;
                 }
-            }
-            for (int c = threadIdx.x; SPLIT != 3 && c < G::kBoxes * kChunksPerBox; c += kWorkers) {
-                const int row = (c % kChunksPerBox) / 8;
-                const bool valid = y0 + row < r1;
-                {
+                uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
+                const int64_t y0 = r0 + static_cast<int64_t>(it) * G::kRows;
+                if (SPLIT == 3) {
+                    // Transpose the [node][feature] TMA tiles (128-byte swizzle) into K-major
+                    // planes [feature][node] with the same swizzle, applying phi and the tf32
+                    // split on the way: element (m, k) of a plane sits at
+                    // (m/8)*1024 + (m%8)*128 + (((k/4) ^ (m%8)) * 16) + (k%4)*4.
+                    const float *rk = reinterpret_cast<const float *>(st);
+                    const float *rv = reinterpret_cast<const float *>(st + G::kOpBytes);
+                    float *ah = reinterpret_cast<float *>(st + 2 * G::kOpBytes);
+                    float *al = reinterpret_cast<float *>(st + 3 * G::kOpBytes);
+                    float *bh = reinterpret_cast<float *>(st + 4 * G::kOpBytes);
+                    float *bl = reinterpret_cast<float *>(st + 5 * G::kOpBytes);
+                    for (int idx = threadIdx.x; idx < G::kRows * kFB; idx += kWorkers) {
+                        const int kr = idx / kFB, m = idx % kFB;
+                        const int e = m % 32;
+                        const int src = ((m / 32) * G::kBoxBytes + kr * kRowBytes +
+                                         (((e / 4) ^ (kr % 8)) * 16) + (e % 4) * 4) / 4;
+                        const int dst = ((m / 8) * 1024 + (m % 8) * kRowBytes +
+                                         (((kr / 4) ^ (m % 8)) * 16) + (kr % 4) * 4) / 4;
+                        const bool valid = y0 + kr < r1;
+                        const float f = valid ? phi(rk[src]) : 0.f;
+                        const float v = rv[src];
+                        const float fh = to_tf32(f), vh = to_tf32(v);
+                        ah[dst] = fh;
+                        al[dst] = to_tf32(f - fh);
+                        bh[dst] = vh;
+                        bl[dst] = to_tf32(v - vh);
+                    }
+                }
+                for (int c = threadIdx.x; SPLIT != 3 && c < G::kBoxes * kChunksPerBox; c += kWorkers) {
+                    const int row = (c % kChunksPerBox) / 8;
+                    const bool valid = y0 + row < r1;
                     uint4 *kp = reinterpret_cast<uint4 *>(st) + c;
                     uint4 u = *kp;
                     uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -244,48 +286,75 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                     }
                     *kp = make_uint4(w[0], w[1], w[2], w[3]);
                 }
+                fence_async_smem();
+                mbar_arrive(&ready_bar[s]);
             }
-            fence_async_smem();
-            mbar_arrive(&ready_bar[s]);
         }
         if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
-    }
-    __syncwarp();
-
-    if (warp < 4) {
-        // ---------------- epilogue: diagonal head blocks of S and z -> partial sums ---------
-        const bool done = ntiles == 0 ? true : mbar_wait_bounded(&done_bar, 0);
-        tc_fence_after();
-        if (!done && lane == 0) atomicOr(p.flag, kDevErrTimeout);
-        const bool have = ntiles > 0 && done;
-        const int t = warp * 32 + lane;                  // TMEM lane = feature in the block
+    } else {
+        // ---------------- warps 18-21: diagonal head blocks of S and z -> partials ----------
+        const int quad = warp & 3;                        // TMEM lanes this warp may read
+        const int t = quad * 32 + lane;                   // TMEM lane = feature in the block
         const int f = fb * kFB + t;
         const bool live = f < p.D;
         const int h = live ? f / R : 0, a = f % R;
-        const int hc0 = h * R - fb * kFB;                // head's first column in the block
-        float *dst = p.part + ((static_cast<int64_t>(part) * p.H + h) * R + a) * (R + 1);
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const int hc0 = h * R - fb * kFB;                 // head's first column in the block
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        bool ok = true;
+        for (int k = 0; k < n_my; ++k) {
+            const int buf = k & 1;
+            const int part = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+            int64_t r0, r1;
+            range_of(part, r0, r1);
+            const bool have = ok && tiles_of(r0, r1) > 0;
+            if (ok && !mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(k >> 1) & 1u)) {
+                ok = false;
+                if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
+            }
+            tc_fence_after();
+            // this feature's row of the range's partial sums ([H][R][R+1] layout: the row
+            // of feature f = h*R + a starts at f*(R+1)); with staging, the warp's 32 rows
+            // (one contiguous block of 32*(R+1) floats) go through shared memory and leave
+            // as coalesced stores
+            float *sw = p.scratch_off ? reinterpret_cast<float *>(dsmem_raw + p.scratch_off) +
+                                            (warp - kEpiWarp0) * 32 * (R + 1)
+                                      : nullptr;
+            float *dst = sw ? sw + lane * (R + 1)
+                            : p.part + ((static_cast<int64_t>(part) * p.H + h) * R + a) * (R + 1);
+            const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(buf) * kAccStride;
 #pragma unroll
-        for (int q = 0; q < kFB / 32; ++q) {
+            for (int q = 0; q < kFB / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(acc + q * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int col = q * 32 + j;
+                    if (live && col >= hc0 && col < hc0 + R) dst[col - hc0] = have ? __uint_as_float(v[j]) : 0.f;
+                }
+            }
             uint32_t v[32];
-            tmem_ld32(tmem + lane_base + q * 32, v);
+            tmem_ld32(acc + kFB, v);
             tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int col = q * 32 + j;
-                if (live && col >= hc0 && col < hc0 + R) dst[col - hc0] = have ? __uint_as_float(v[j]) : 0.f;
+            if (live) dst[R] = have ? __uint_as_float(v[0]) : 0.f;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce_bar[buf]);
+            if (sw) {
+                // rows fb*128 + quad*32 .. (those below D) of the range's block
+                const int f0 = fb * kFB + quad * 32;
+                const int rows = max(0, min(32, p.D - f0));
+                float *g = p.part + (static_cast<int64_t>(part) * p.H * R + f0) * (R + 1);
+                for (int i = lane; i < rows * (R + 1); i += 32) g[i] = sw[i];
+                __syncwarp();
             }
         }
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + kFB, v);
-        tmem_ld_wait();
-        if (live) dst[R] = have ? __uint_as_float(v[0]) : 0.f;
     }
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256u);
+        tmem_dealloc(tmem, 512u);
     }
 }
 
@@ -424,18 +493,34 @@ __global__ void __launch_bounds__(256) stats_reduce_segments_kernel(
     }
 }
 
+// P = p.n_parts row ranges per feature block, walked by min(P, num_sms / nblk) CTAs each
+// (one range per CTA when the ranges are about one per SM).
 template <typename T>
-glga_status launch_stats(const CUtensorMap &mk, const CUtensorMap &mv, const StatsParams &p, int parts,
+glga_status launch_stats(const CUtensorMap &mk, const CUtensorMap &mv, const StatsParams &p, int num_sms,
                          int nblk, int r, cudaStream_t s) {
-    dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(nblk));
-    const size_t smem = static_cast<size_t>(p.stages) * p.stage_bytes + 2048 + 1024;
+    const int g = std::max(1, std::min(p.n_parts, std::max(1, num_sms / nblk)));
+    dim3 grid(static_cast<unsigned>(g), static_cast<unsigned>(nblk));
+    // several ranges per CTA: stage the epilogue's partial sums in shared memory (4 warps x
+    // 32 rows x (r + 1) floats) when two or more ring stages still fit beside it
+    StatsParams q = p;
+    q.scratch_off = 0;
+    const size_t scratch = static_cast<size_t>(4) * 32 * (r + 1) * sizeof(float);
+    constexpr size_t kSmemMax = 226 * 1024;   // dynamic shared memory, leaving room for the static part
+    if (g < p.n_parts) {
+        const int st = static_cast<int>(std::min<size_t>(p.stages, (kSmemMax - 2048 - 1024 - scratch) / p.stage_bytes));
+        if (st >= 2) {
+            q.stages = st;
+            q.scratch_off = static_cast<uint32_t>(1024 + static_cast<size_t>(st) * p.stage_bytes + 2048);
+        }
+    }
+    const size_t smem = static_cast<size_t>(q.stages) * q.stage_bytes + 2048 + 1024 + (q.scratch_off ? scratch : 0);
     constexpr int SPLIT = sizeof(T) == 4 ? 3 : 1;
 #define GLGA_ST(RR)                                                                          \
     case RR: {                                                                               \
         auto kern = stats_tc_kernel<SPLIT, T, RR>;                                           \
         GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                                        static_cast<int>(smem)));                             \
-        kern<<<grid, kThreads, smem, s>>>(mk, mv, p);                                        \
+        kern<<<grid, kThreads, smem, s>>>(mk, mv, q);                                        \
         break;                                                                               \
     }
     switch (r) {
@@ -526,6 +611,7 @@ glga_status stats_partials(Ctx *c, cudaStream_t s) {
         p.N = c->N;
         p.D = c->D;
         p.H = c->H;
+        p.n_parts = c->stats_parts;
         p.rows_per_part = c->stats_rows_per_part;
         p.part_ptr = c->part_ptr;
         p.stages = c->io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
@@ -535,10 +621,10 @@ glga_status stats_partials(Ctx *c, cudaStream_t s) {
         glga_status st;
         if (c->io == GLGA_F32) {
             p.stage_bytes = stage_bytes<float>();
-            st = launch_stats<float>(c->tmK.map, c->tmV.map, p, c->stats_parts, nblk, c->r, s);
+            st = launch_stats<float>(c->tmK.map, c->tmV.map, p, c->num_sms, nblk, c->r, s);
         } else {
             p.stage_bytes = stage_bytes<__nv_bfloat16>();
-            st = launch_stats<__nv_bfloat16>(c->tmK.map, c->tmV.map, p, c->stats_parts, nblk, c->r, s);
+            st = launch_stats<__nv_bfloat16>(c->tmK.map, c->tmV.map, p, c->num_sms, nblk, c->r, s);
         }
         if (st != GLGA_OK) return st;
         c->launches += 1;
@@ -759,6 +845,7 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         p.N = N;
         p.D = static_cast<int32_t>(D);
         p.H = H;
+        p.n_parts = parts;
         p.rows_per_part = per;
         p.part_ptr = nullptr;
         p.stages = io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
@@ -766,10 +853,10 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         p.flag = flag;
         if (io == GLGA_F32) {
             p.stage_bytes = stage_bytes<float>();
-            st = launch_stats<float>(mk, mv, p, parts, nblk, r, s);
+            st = launch_stats<float>(mk, mv, p, sms, nblk, r, s);
         } else {
             p.stage_bytes = stage_bytes<__nv_bfloat16>();
-            st = launch_stats<__nv_bfloat16>(mk, mv, p, parts, nblk, r, s);
+            st = launch_stats<__nv_bfloat16>(mk, mv, p, sms, nblk, r, s);
         }
         if (st != GLGA_OK) return st;
     }

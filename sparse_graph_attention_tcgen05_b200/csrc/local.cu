@@ -34,7 +34,9 @@
 // head, so the lane keeps one softmax state for all of them.  Each slot walks a
 // contiguous edge range U edges at a time; the column indices of the next step (and, for
 // task rows, the next row's q and first columns) are loaded one step ahead so the
-// k_j/v_j gathers do not wait behind them.
+// k_j/v_j gathers do not wait behind them.  Options of the compile-time layouts, chosen per
+// shape by measurement: PIPE issues the next step's gathers before the current step is
+// consumed (two register buffers), CB loads the column indices of several steps at once.
 //
 // Arithmetic: q_i and k_j stay in the io type; for bf16 the dot product runs on the
 // mixed-precision fma.rn.f32.bf16 (bf16 operands, exact products, f32 accumulation), so
@@ -283,9 +285,11 @@ __device__ __forceinline__ int32_t first_cols(const LocalParams &p, int64_t e0, 
     return (ln.li < CB && e0 + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + e0 + ln.li)) : -1;
 }
 
-template <typename T, int NV, int LPH, int VPL, int U, bool J>
+// Column indices per load: a batch of the slot's LPE lanes (CB, compile-time layouts
+// only) or one step's U.
+template <typename T, int NV, int LPH, int VPL, int U, bool J, bool CB>
 constexpr int col_batch() {
-    return Shape<T, NV, LPH, VPL, J>::kLpe != 0 ? Shape<T, NV, LPH, VPL, J>::kLpe : U;
+    return (CB && Shape<T, NV, LPH, VPL, J>::kLpe != 0) ? Shape<T, NV, LPH, VPL, J>::kLpe : U;
 }
 
 // One slot walks the CSR entries [e0, e1) U at a time (the trip count is the warp's
@@ -293,7 +297,7 @@ constexpr int col_batch() {
 // k_j / v_j gathers of step i + 1 are issued before step i is consumed (two register
 // buffers), so a warp keeps a step's loads in flight while it computes the previous one.
 // On return each lane holds its slot's partial state for its feature vectors.
-template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE>
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE, bool CB>
 __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q)[VPL], int64_t e0,
                                            int64_t e1, int32_t cols, const Lane &ln,
                                            State<T, VPL, J> &st) {
@@ -313,16 +317,17 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
     bool ok[VPL];
 #pragma unroll
     for (int v = 0; v < VPL; ++v) ok[v] = Sh::lane_ok(p, v, ln.li);
-    // column indices arrive in batches of CB edges (CB / U steps each); the next batch is
-    // loaded while the current one is used.  The batches follow the load stream.
-    constexpr int CB = col_batch<T, NV, LPH, VPL, U, J>();
-    constexpr int PER = CB / U;
-    static_assert(CB % U == 0, "a batch holds whole steps");
+    // column indices arrive in batches of NB edges (NB / U steps each; NB = U without
+    // batching); the next batch is loaded while the current one is used.  The batches
+    // follow the load stream.
+    constexpr int NB = col_batch<T, NV, LPH, VPL, U, J, CB>();
+    constexpr int PER = NB / U;
+    static_assert(NB % U == 0, "a batch holds whole steps");
     int32_t c_cur = cols;
     int32_t c_next = -1;
     if (PER > 1 && iters > PER) {
-        const int64_t nb = e0 + CB;
-        c_next = (ln.li < CB && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
+        const int64_t nb = e0 + NB;
+        c_next = (ln.li < NB && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
     }
     // issues the gathers of step `step` into (kb, vb); jb gets its column indices (-1:
     // no edge; such a slot keeps its previous, finite contents and gets weight 0)
@@ -333,8 +338,8 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
         if (sub == PER - 1) {
             if (PER > 1) {
                 c_cur = c_next;
-                const int64_t nb = e0 + static_cast<int64_t>(step / PER + 2) * CB;
-                c_next = (ln.li < CB && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
+                const int64_t nb = e0 + static_cast<int64_t>(step / PER + 2) * NB;
+                c_next = (ln.li < NB && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
             } else {
                 const int64_t nb = e0 + static_cast<int64_t>(step + 1) * U;
                 c_cur = (ln.li < U && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
@@ -533,7 +538,7 @@ struct BlockScratch {
 
 // 8 warps split [e0, e1) (each warp's share split again across its slots); warp 0
 // returns the merge of all warps in warp order.
-template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE>
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE, bool CB>
 __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&q)[VPL], int64_t e0,
                                             int64_t e1, const Lane &ln, int warp,
                                             BlockScratch<T, VPL, J> &sh, State<T, VPL, J> &st) {
@@ -544,8 +549,8 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&
     const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
     const int64_t per_s = ceil_div(b - a, Sh::epw(p));
     const int64_t sa = std::min(b, a + ln.slot * per_s), sb = std::min(b, sa + per_s);
-    slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, sa, sb,
-                                               first_cols<col_batch<T, NV, LPH, VPL, U, J>(), DBG>(p, sa, sb, ln),
+    slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, sa, sb,
+                                               first_cols<col_batch<T, NV, LPH, VPL, U, J, CB>(), DBG>(p, sa, sb, ln),
                                                ln, st);
     merge_slots<T, NV, LPH, VPL, J>(p, st);
 #pragma unroll
@@ -581,7 +586,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&
 constexpr int local_min_blocks(int VPL, int U, bool PIPE) {
     return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? 3 : 2;
 }
-template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE>
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE, bool CB>
 __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
     local_kernel(const LocalParams p) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
@@ -609,7 +614,7 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
         const int64_t nch = ceil_div(re - rb, p.chunk_edges);
         const int64_t first = c - (e0 - rb) / p.chunk_edges;
         load_q<T, NV, LPH, VPL, J>(p, row, ln, true, q);
-        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, e0, e1, ln, warp, sh, st);
+        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, e0, e1, ln, warp, sh, st);
         const int64_t stride = 2 * p.H + p.D;
         if (warp == 0) {
             float *dst = p.part + c * stride;
@@ -666,7 +671,7 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
         const int64_t row = p.cta_rows[bid];
         if (!row_ok<DBG>(p, row)) return;
         load_q<T, NV, LPH, VPL, J>(p, row, ln, true, q);
-        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
+        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
         if (warp == 0) finish_row<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, ln.slot == 0);
         return;
     }
@@ -696,7 +701,7 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
     if (k >= n) beg = end = 0;
     uint4 qn[VPL];
     load_q<T, NV, LPH, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qn);
-    int32_t cols = first_cols<col_batch<T, NV, LPH, VPL, U, J>(), DBG>(p, beg, end, ln);
+    int32_t cols = first_cols<col_batch<T, NV, LPH, VPL, U, J, CB>(), DBG>(p, beg, end, ln);
     for (int step = 0; step < steps; ++step) {
         const bool valid = k < n;
         const int32_t row_c = row;
@@ -711,14 +716,14 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
         end = __shfl_sync(0xffffffffu, myend, k & 31);
         if (k >= n) beg = end = 0;
         load_q<T, NV, LPH, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qn);
-        cols = first_cols<col_batch<T, NV, LPH, VPL, U, J>(), DBG>(p, beg, end, ln);
-        slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE>(p, q, beg_c, end_c, cols_c, ln, st);
+        cols = first_cols<col_batch<T, NV, LPH, VPL, U, J, CB>(), DBG>(p, beg, end, ln);
+        slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, beg_c, end_c, cols_c, ln, st);
         // every slot finishes its own row
         if (valid && (!DBG || row_c >= 0)) finish_row<T, NV, LPH, VPL, J, LSE>(p, row_c, st, ln, true);
     }
 }
 
-template <typename T, int NV, int LPH, int VPL, int U, bool J, bool PIPE>
+template <typename T, int NV, int LPH, int VPL, int U, bool J, bool PIPE = false, bool CB = false>
 glga_status launch_local(Ctx *c, LocalParams p, cudaStream_t s) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
     if constexpr (NV != 0) {
@@ -731,11 +736,11 @@ glga_status launch_local(Ctx *c, LocalParams p, cudaStream_t s) {
     if (blocks == 0) return GLGA_OK;
     const unsigned g = static_cast<unsigned>(blocks);
     if (c->opts.debug_checks) {
-        if (p.lse) local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE><<<g, kLocalThreads, 0, s>>>(p);
+        if (p.lse) local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
     } else {
-        if (p.lse) local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE><<<g, kLocalThreads, 0, s>>>(p);
+        if (p.lse) local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
     }
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
@@ -790,16 +795,6 @@ glga_status local_setup(Ctx *c) {
     return GLGA_OK;
 }
 
-#ifndef GLGA_LOCAL_V128
-#define GLGA_LOCAL_V128 0
-#endif
-#ifndef GLGA_LOCAL_V256
-#define GLGA_LOCAL_V256 0
-#endif
-#ifndef GLGA_LOCAL_V512
-#define GLGA_LOCAL_V512 0
-#endif
-
 glga_status local_run(Ctx *c, cudaStream_t s) {
     LocalParams p;
     p.row_ptr = c->row_ptr;
@@ -837,33 +832,14 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     const int vpl = static_cast<int>(ceil_div(p.nvec, 32));
     if (c->io == GLGA_BF16) {
         using B = __nv_bfloat16;
-        // hot shapes with compile-time layouts (v: a lane's vectors interleave across the
-        // row; j: a lane's VPL vectors are consecutive features of one head)
-        if (p.nvec == 16 && c->r == 32) {   // D = 128, 4 heads of 32
-            switch (GLGA_LOCAL_V128) {
-                case 1: return launch_local<B, 16, 4, 1, 4, false, false>(c, p, s);
-                case 2: return launch_local<B, 16, 4, 1, 2, false, true>(c, p, s);
-                case 3: return launch_local<B, 16, 2, 2, 2, true, true>(c, p, s);
-                case 4: return launch_local<B, 16, 2, 2, 2, true, false>(c, p, s);
-                case 5: return launch_local<B, 16, 2, 2, 1, true, true>(c, p, s);
-                default: return launch_local<B, 16, 4, 1, 4, false, true>(c, p, s);
-            }
-        }
-        if (p.nvec == 32 && c->r == 32) {   // D = 256, 8 heads of 32
-            switch (GLGA_LOCAL_V256) {
-                case 1: return launch_local<B, 32, 2, 2, 2, true, false>(c, p, s);
-                case 2: return launch_local<B, 32, 2, 2, 2, true, true>(c, p, s);
-                case 3: return launch_local<B, 32, 4, 1, 4, false, false>(c, p, s);
-                default: return launch_local<B, 32, 4, 1, 4, false, true>(c, p, s);
-            }
-        }
-        if (p.nvec == 64 && c->r == 64) {   // D = 512, 8 heads of 64
-            switch (GLGA_LOCAL_V512) {
-                case 1: return launch_local<B, 64, 4, 2, 2, true, false>(c, p, s);
-                case 2: return launch_local<B, 64, 2, 4, 1, true, true>(c, p, s);
-                default: return launch_local<B, 64, 4, 2, 2, true, true>(c, p, s);
-            }
-        }
+        // hot shapes with compile-time layouts, chosen by measurement: a lane's vector
+        // interleaved across the row (D = 128 and 256: one vector per lane, 4 edges per
+        // step, 3 blocks per SM); at D = 512 two consecutive vectors of one head per lane,
+        // the next step's gathers issued before the current one is consumed, column
+        // indices in batches
+        if (p.nvec == 16 && c->r == 32) return launch_local<B, 16, 4, 1, 4, false>(c, p, s);
+        if (p.nvec == 32 && c->r == 32) return launch_local<B, 32, 4, 1, 4, false>(c, p, s);
+        if (p.nvec == 64 && c->r == 64) return launch_local<B, 64, 4, 2, 2, true, true, true>(c, p, s);
         if (p.nvec == 64 && c->r >= 16) return launch_local<B, 64, 0, 2, 2, true, false>(c, p, s);
         if (vpl == 1 && lpe >= 4) return launch_local<B, 0, 0, 1, 4, false, false>(c, p, s);
         if (vpl == 1 && lpe == 2) return launch_local<B, 0, 0, 1, 2, false, false>(c, p, s);

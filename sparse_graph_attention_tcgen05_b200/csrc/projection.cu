@@ -281,9 +281,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         for (int i = 0; i < n_my; ++i, tw.next()) {
             const int buf = i & 1;
             const bool got = mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(i >> 1) & 1u);
-            // the 8 epilogue warps must agree before the named barriers below
-            const bool fail = p.tma_epi ? named_barrier_or(1, 256, !got) : !got;
-            if (fail) {
+            // (no barrier spans the epilogue warps: each gives up on its own wait)
+            if (!got) {
                 if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
                 ok = false;
                 break;
@@ -316,24 +315,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acce_bar[buf]);
             } else if (p.tma_epi) {
-                // Q/K/V columns go through a staging buffer (buffer i & 1 when there are
-                // two); the TMA store that last used it (tile i - sbufs) must have
-                // finished reading it first
+                // Each warp owns whole 64-column boxes of its 32 rows (boxes wg, wg + 2, ...;
+                // in the last column tile warpgroup 1 also takes the gate column past them):
+                // it stages them in shared memory (buffer i & 1 when there are two) and
+                // stores them with its own TMA bulk stores, waiting only for its own
+                // earlier stores out of that buffer, so no barrier spans the warps.
                 const int sbuf = p.sbufs == 2 ? buf : 0;
                 uint8_t *sb = smem + p.stage_area + static_cast<size_t>(sbuf) * nbox * box_bytes;
-                if (threadIdx.x == 0) {
+                if (lane == 0) {
                     if (p.sbufs == 2)
                         bulk_wait_group_read1();
                     else
                         bulk_wait_group_read0();
                 }
-                named_barrier_sync(1, 256);
-                for (int c0 = wg * 32; c0 < bn; c0 += 64) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + c0), v);
-                    tmem_ld_wait();
-                    if (c0 < p.BN) {
-                        const int b = c0 / 64, e0 = (c0 % 64) / 8;
+                __syncwarp();
+                for (int b = wg; b < nbox; b += 2) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + b * 64 + half * 32), v);
+                        tmem_ld_wait();
                         uint8_t *rp = sb + b * box_bytes + rt * kRowBytes;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -342,24 +343,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                             w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
                             w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
                             w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                            *reinterpret_cast<uint4 *>(rp + (((e0 + q) ^ (rt & 7)) * 16)) = w;
+                            *reinterpret_cast<uint4 *>(rp + (((half * 4 + q) ^ (rt & 7)) * 16)) = w;
                         }
-                    } else if (row < p.M) {
-                        p.t[row] = __uint_as_float(v[0]);   // gate logit column
                     }
+                }
+                if (bn > p.BN && wg == 1) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + p.BN), v);
+                    tmem_ld_wait();
+                    if (row < p.M) p.t[row] = __uint_as_float(v[0]);   // gate logit column
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acce_bar[buf]);
                 fence_proxy_async_smem();
-                named_barrier_sync(1, 256);
-                if (threadIdx.x == 0) {
-                    for (int b = 0; b < nbox; ++b) {
+                __syncwarp();
+                if (lane == 0) {
+                    const int64_t y = m0 + quad * 32;
+                    for (int b = wg; b < nbox && y < p.M; b += 2) {
                         const int gc = n0 + b * 64;
+                        const uint8_t *src = sb + b * box_bytes + quad * 32 * kRowBytes;
                         if (gc < p.D)
-                            tma_store_2d(&tmQs, sb + b * box_bytes, gc, static_cast<int32_t>(m0));
+                            tma_store_2d(&tmQs, src, gc, static_cast<int32_t>(y));
                         else
-                            tma_store_2d(&tmKVs, sb + b * box_bytes, gc - p.D, static_cast<int32_t>(m0));
+                            tma_store_2d(&tmKVs, src, gc - p.D, static_cast<int32_t>(y));
                     }
                     bulk_commit_group();
                 }
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
             }
         }
         (void)ok;
-        if (p.tma_epi && threadIdx.x == 0) bulk_wait_group_read0();
+        if (p.tma_epi && lane == 0) bulk_wait_group_read0();   // shared memory outlives the stores
     }
     tc_fence_before();
     __syncthreads();
@@ -503,7 +510,7 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(p.n_total_tiles, c->num_sms));
     const CUtensorMap &a1 = planes == 2 ? c->tmA[1].map : c->tmA[0].map;
     const CUtensorMap &b1 = planes == 2 ? c->tmB[1].map : c->tmB[0].map;
-    const CUtensorMap &qs = c->gemm_tma_epi ? c->tmQ.map : c->tmB[0].map;      // unused otherwise
+    const CUtensorMap &qs = c->gemm_tma_epi ? c->tmQs.map : c->tmB[0].map;     // unused otherwise
     const CUtensorMap &kvs = c->gemm_tma_epi ? c->tmKVs.map : c->tmB[0].map;
     kern<<<grid, kGemmThreads, smem, s>>>(c->tmA[0].map, a1, c->tmB[0].map, b1, qs, kvs, p);
     GLGA_CUDA(cudaGetLastError());
@@ -650,10 +657,15 @@ glga_status projection_setup(Ctx *c) {
         c->tmB[pl].valid = true;
     }
     if (c->gemm_tma_epi && c->N > 0) {
+        // store maps: 64-column x 32-row boxes, one per epilogue warp and box
         r = encode_tmap_2d(&c->tmKVs.map, dt, c->kv_own, 2 * static_cast<uint64_t>(c->D), c->N,
-                           2 * static_cast<uint64_t>(c->D) * c->elem, 64, kBM);
+                           2 * static_cast<uint64_t>(c->D) * c->elem, 64, 32);
         if (r != GLGA_OK) return r;
         c->tmKVs.valid = true;
+        r = encode_tmap_2d(&c->tmQs.map, dt, c->Q, static_cast<uint64_t>(c->D), c->N,
+                           static_cast<uint64_t>(c->D) * c->elem, 64, 32);
+        if (r != GLGA_OK) return r;
+        c->tmQs.valid = true;
     }
     // The A operand is read from the caller's X when it is bf16 with 16-byte rows;
     // otherwise from a padded (and, for fp32, split) copy.

@@ -354,6 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
         TileWalk tw(blockIdx.x, gridDim.x, p.n_groups);   // tile i (phi pass)
         TileWalk te = tw;                                // tile i - 1 (epilogue)
         bool ok = true;
+        // a bounded wait of a phi pass that gave up: the workers agree on it at the next
+        // epilogue's barrier (one per tile), so all of them leave the loop together
+        bool bad = false;
         for (int i = 0; i <= n_my && ok; ++i) {
             float t_cur = 0.f;
             if (i < n_my) {
@@ -363,10 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                 tw.next();
                 for (int kb = 0; kb < p.nk; ++kb, rp.next(p.stages)) {
                     const int s = rp.slot;
-                    const bool got = mbar_wait_bounded(&full_bar[s], rp.phase);
-                    if (named_barrier_or(1, kWorkers, !got)) {
-                        ok = false;
-                        break;
+                    if (bad || !mbar_wait_bounded(&full_bar[s], rp.phase)) {
+                        bad = true;        // (the MMA warp's own bounded wait then gives up too)
+                        continue;
                     }
                     uint8_t *st = smem + static_cast<size_t>(s) * p.stage_bytes;
                     // kTPR threads share a tile row, kCPT of its 8 16-byte chunks each; the
@@ -388,7 +390,6 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ready_bar[s]);
                 }
-                if (!ok) break;
             }
             if (i > 0) {
                 // ---- epilogue of tile k = i - 1 ----
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                 const int64_t row = m0 + rt;
                 const bool live = row < p.M;
                 const int lb_i = lp.slot;
-                bool got = mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(k >> 1) & 1u);
+                bool got = !bad && mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(k >> 1) & 1u);
                 if (p.lboxes > 0) got = got && mbar_wait_bounded(&lfull_bar[lb_i], lp.phase);
                 if (named_barrier_or(1, kWorkers, !got)) {
                     ok = false;
