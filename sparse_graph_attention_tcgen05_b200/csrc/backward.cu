@@ -1227,7 +1227,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDwStages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&ready_bar[s], kDwWorkers);
+            mbar_init(&ready_bar[s], kDwWorkers / 32);   // one arrival per worker warp
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&done_bar, 1);
@@ -1300,7 +1300,8 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
         RingPos rp;
         for (int it = 0; it < ntiles && ok; ++it, rp.next(kDwStages)) {
             const int s = rp.slot;
-            if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
+            // the warp agrees on the outcome, so it stays converged for its arrival
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], rp.phase))) {
                 ok = false;
                 break;
             }
@@ -1326,7 +1327,8 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
                 *reinterpret_cast<uint4 *>(bt + bo * kDwBox + k * 128 + ((co ^ (k & 7)) * 16)) = w;
             }
             fence_proxy_async_smem();
-            mbar_arrive(&ready_bar[s]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ready_bar[s]);
         }
         if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
     }

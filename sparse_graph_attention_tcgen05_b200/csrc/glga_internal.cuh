@@ -115,6 +115,8 @@ struct Ctx {
     int64_t n_seg = 1;
     std::vector<int64_t> seg_ptr;     // host copy [n_seg + 1]
     int32_t *seg_part_ptr = nullptr;  // statistics ranges of each segment [n_seg + 1]
+    bool stats_direct = false;        // every non-empty segment one range: no reduction pass
+    int32_t *part_seg = nullptr;      // ... and the segment of each range
     int32_t *tile_seg = nullptr;      // segment of each 128-row readout tile's first row
     int32_t *fix_row = nullptr;       // rows whose segment differs from their tile's
     int32_t *fix_seg = nullptr;       //   ... and that segment

@@ -58,6 +58,15 @@ struct StatsParams {
     uint32_t scratch_off;    // epilogue staging in dynamic shared memory (0: direct stores)
     float *part;             // [P][H][r][r+1]
     unsigned *flag;
+    // final statistics written by the epilogue (every non-empty segment is one range, so
+    // a range's sums are its segment's S and z): range -> segment, S | z and the readout
+    // operand (layouts of stats_reduce_kernel); null part_seg: partial sums only
+    const int32_t *part_seg;
+    int64_t n_seg;
+    float *Sz;
+    void *Bro;
+    int32_t hg, BNr, Kp;
+    int64_t seg_stride, plane;
 };
 
 __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
@@ -101,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&ready_bar[s], kWorkers);
+            mbar_init(&ready_bar[s], kWorkerWarps);   // one arrival per worker warp
             mbar_init(&empty_bar[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -237,7 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             const int ntiles = tiles_of(r0, r1);
             for (int it = 0; it < ntiles && ok; ++it, rp.next(p.stages)) {
                 const int s = rp.slot;
-                if (!mbar_wait_bounded(&full_bar[s], rp.phase)) {
+                // the warp agrees on the outcome, so it stays converged for its arrival
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], rp.phase))) {
                     ok = false;
                     break;
                 }
@@ -287,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                     *kp = make_uint4(w[0], w[1], w[2], w[3]);
                 }
                 fence_async_smem();
-                mbar_arrive(&ready_bar[s]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ready_bar[s]);
             }
         }
         if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
@@ -307,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             int64_t r0, r1;
             range_of(part, r0, r1);
             const bool have = ok && tiles_of(r0, r1) > 0;
-            if (ok && !mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(k >> 1) & 1u)) {
+            if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(k >> 1) & 1u))) {
                 ok = false;
                 if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
             }
@@ -340,7 +351,36 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce_bar[buf]);
-            if (sw) {
+            if (sw && p.part_seg) {
+                // the range is its segment: S rows (coalesced, from the staging), z, and the
+                // segment's readout operand block (transposed S_h and z_h; consecutive
+                // features write consecutive K positions)
+                __syncwarp();
+                const int64_t seg = p.part_seg[part];
+                const int f0 = fb * kFB + quad * 32;
+                const int rows = max(0, min(32, p.D - f0));
+                const int64_t hrr = static_cast<int64_t>(p.H) * R * R;
+                float *gS = p.Sz + seg * hrr + static_cast<int64_t>(f0) * R;
+                for (int i = lane; i < rows * R; i += 32) gS[i] = sw[(i / R) * (R + 1) + i % R];
+                if (live) {
+                    p.Sz[p.n_seg * hrr + seg * p.H * R + f] = sw[lane * (R + 1) + R];
+                    const int gi = h / p.hg, hl = h - gi * p.hg, hga = min(p.hg, p.H - gi * p.hg);
+                    const int64_t base = seg * p.seg_stride + static_cast<int64_t>(gi) * p.BNr * p.Kp + hl * R + a;
+                    for (int cc = 0; cc <= R; ++cc) {
+                        const float x = sw[lane * (R + 1) + cc];
+                        const int n = cc < R ? hl * R + cc : hga * R + hl;
+                        const int64_t idx = base + static_cast<int64_t>(n) * p.Kp;
+                        if (sizeof(T) == 4) {
+                            const float hi = to_tf32(x);
+                            reinterpret_cast<float *>(p.Bro)[idx] = hi;
+                            reinterpret_cast<float *>(p.Bro)[p.plane + idx] = to_tf32(x - hi);
+                        } else {
+                            reinterpret_cast<__nv_bfloat16 *>(p.Bro)[idx] = __float2bfloat16_rn(x);
+                        }
+                    }
+                }
+                __syncwarp();
+            } else if (sw) {
                 // rows fb*128 + quad*32 .. (those below D) of the range's block
                 const int f0 = fb * kFB + quad * 32;
                 const int rows = max(0, min(32, p.D - f0));
@@ -493,6 +533,16 @@ __global__ void __launch_bounds__(256) stats_reduce_segments_kernel(
     }
 }
 
+// Ring stages that fit beside the epilogue's staging buffer (4 warps x 32 rows x (r + 1)
+// floats), or 0 when fewer than two do.
+size_t stats_scratch_bytes(int r) { return static_cast<size_t>(4) * 32 * (r + 1) * sizeof(float); }
+int stats_stages_with_scratch(uint32_t stage_bytes, int stages, int r) {
+    constexpr size_t kSmemMax = 226 * 1024;   // dynamic shared memory, leaving room for the static part
+    const int st = static_cast<int>(
+        std::min<size_t>(stages, (kSmemMax - 2048 - 1024 - stats_scratch_bytes(r)) / stage_bytes));
+    return st >= 2 ? st : 0;
+}
+
 // P = p.n_parts row ranges per feature block, walked by min(P, num_sms / nblk) CTAs each
 // (one range per CTA when the ranges are about one per SM).
 template <typename T>
@@ -500,17 +550,20 @@ glga_status launch_stats(const CUtensorMap &mk, const CUtensorMap &mv, const Sta
                          int nblk, int r, cudaStream_t s) {
     const int g = std::max(1, std::min(p.n_parts, std::max(1, num_sms / nblk)));
     dim3 grid(static_cast<unsigned>(g), static_cast<unsigned>(nblk));
-    // several ranges per CTA: stage the epilogue's partial sums in shared memory (4 warps x
-    // 32 rows x (r + 1) floats) when two or more ring stages still fit beside it
+    // several ranges per CTA, or final statistics written by the epilogue: the epilogue
+    // stages each range's sums in shared memory (coalesced stores) when two or more ring
+    // stages still fit beside the staging buffer
     StatsParams q = p;
     q.scratch_off = 0;
-    const size_t scratch = static_cast<size_t>(4) * 32 * (r + 1) * sizeof(float);
-    constexpr size_t kSmemMax = 226 * 1024;   // dynamic shared memory, leaving room for the static part
-    if (g < p.n_parts) {
-        const int st = static_cast<int>(std::min<size_t>(p.stages, (kSmemMax - 2048 - 1024 - scratch) / p.stage_bytes));
+    const size_t scratch = stats_scratch_bytes(r);
+    if (g < p.n_parts || p.part_seg) {
+        const int st = stats_stages_with_scratch(p.stage_bytes, p.stages, r);
         if (st >= 2) {
             q.stages = st;
             q.scratch_off = static_cast<uint32_t>(1024 + static_cast<size_t>(st) * p.stage_bytes + 2048);
+        } else if (p.part_seg) {
+            set_error("statistics: the epilogue staging does not fit beside the ring");
+            return GLGA_ERR_UNSUPPORTED;
         }
     }
     const size_t smem = static_cast<size_t>(q.stages) * q.stage_bytes + 2048 + 1024 + (q.scratch_off ? scratch : 0);
@@ -583,6 +636,18 @@ glga_status stats_setup(Ctx *c) {
     parts = static_cast<int>(pp.size() - 1);
     c->stats_parts = parts;
     c->stats_rows_per_part = per;
+    // every non-empty segment one range: the statistics kernel's epilogue writes the final
+    // S, z and readout operand of each segment, and no reduction runs
+    std::vector<int32_t> pseg;
+    bool one_each = c->n_seg > 1 && c->N > 0;
+    for (int64_t k = 0; k < c->n_seg && one_each; ++k) {
+        const int32_t cnt = sp[k + 1] - sp[k];
+        if (cnt > 1) one_each = false;
+        if (cnt == 1) pseg.push_back(static_cast<int32_t>(k));
+    }
+    const uint32_t sb = c->io == GLGA_F32 ? stage_bytes<float>() : stage_bytes<__nv_bfloat16>();
+    const int kst = c->io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
+    c->stats_direct = one_each && stats_stages_with_scratch(sb, kst, c->r) >= 2;
     const size_t one = static_cast<size_t>(c->H) * c->r * (c->r + 1) * sizeof(float);
     if (one * std::max(parts, 1) > (size_t{4} << 30)) {
         set_error("glga_create: %d statistics ranges need more than 4 GiB of partial sums", parts);
@@ -590,6 +655,18 @@ glga_status stats_setup(Ctx *c) {
     }
     glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart), one * std::max(parts, 1));
     if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->Sz), one * c->n_seg);
+    if (st == GLGA_OK) {
+        // empty segments keep zero statistics (the direct epilogue never writes them)
+        cudaError_t e = cudaMemset(c->Sz, 0, one * c->n_seg);
+        if (e != cudaSuccess) return cuda_fail(e, "statistics init");
+    }
+    if (st == GLGA_OK && c->stats_direct) {
+        st = dev_alloc(c, reinterpret_cast<void **>(&c->part_seg), pseg.size() * sizeof(int32_t));
+        if (st == GLGA_OK) {
+            cudaError_t e = cudaMemcpy(c->part_seg, pseg.data(), pseg.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+            if (e != cudaSuccess) return cuda_fail(e, "statistics segments");
+        }
+    }
     if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->part_ptr), pp.size() * sizeof(int32_t));
     if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->seg_part_ptr), sp.size() * sizeof(int32_t));
     if (st == GLGA_OK) {
@@ -614,6 +691,15 @@ glga_status stats_partials(Ctx *c, cudaStream_t s) {
         p.n_parts = c->stats_parts;
         p.rows_per_part = c->stats_rows_per_part;
         p.part_ptr = c->part_ptr;
+        p.part_seg = c->stats_direct ? c->part_seg : nullptr;
+        p.n_seg = c->n_seg;
+        p.Sz = c->Sz;
+        p.Bro = c->Bro;
+        p.hg = c->ro_hg;
+        p.BNr = c->ro_bn;
+        p.Kp = c->ro_kp;
+        p.seg_stride = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
+        p.plane = c->n_seg * p.seg_stride;
         p.stages = c->io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
         p.part = c->Spart;
         p.flag = c->dev_flag;
@@ -663,6 +749,7 @@ glga_status stats_finish(Ctx *c, const float *partials, int P, cudaStream_t s) {
 glga_status stats_run(Ctx *c, cudaStream_t s) {
     glga_status st0 = stats_partials(c, s);
     if (st0 != GLGA_OK) return st0;
+    if (c->stats_direct) return GLGA_OK;   // the epilogue wrote S, z and the readout operand
     const int total = c->H * c->r * (c->r + 1);
     const int P = c->N > 0 ? c->stats_parts : 0;
     const int64_t seg_stride = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
@@ -848,6 +935,7 @@ extern "C" glga_status glga_global_stats_static(const void *KV, int64_t N, int32
         p.n_parts = parts;
         p.rows_per_part = per;
         p.part_ptr = nullptr;
+        p.part_seg = nullptr;
         p.stages = io == GLGA_F32 ? StatsGeom<float>::kStages : StatsGeom<__nv_bfloat16>::kStages;
         p.part = scratch;
         p.flag = flag;

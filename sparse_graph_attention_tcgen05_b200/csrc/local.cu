@@ -138,6 +138,23 @@ struct Io<__nv_bfloat16> {
     }
 };
 
+// a[0..7] += w * (the 8 bf16 values of u, widened exactly), on the packed f32x2 FMA: four
+// instructions for the eight products.
+__device__ __forceinline__ void acc_bf16x8_f32x2(float (&a)[8], float w, const uint4 &u) {
+    asm("{\n\t.reg .b64 wv, v, c;\n\t.reg .b32 lo, hi;\n\t"
+        "mov.b64 wv, {%8, %8};\n\t"
+        "shl.b32 lo, %9, 16;\n\tand.b32 hi, %9, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
+        "mov.b64 c, {%0, %1};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%0, %1}, c;\n\t"
+        "shl.b32 lo, %10, 16;\n\tand.b32 hi, %10, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
+        "mov.b64 c, {%2, %3};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%2, %3}, c;\n\t"
+        "shl.b32 lo, %11, 16;\n\tand.b32 hi, %11, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
+        "mov.b64 c, {%4, %5};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%4, %5}, c;\n\t"
+        "shl.b32 lo, %12, 16;\n\tand.b32 hi, %12, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
+        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%6, %7}, c;\n\t}"
+        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]), "+f"(a[7])
+        : "f"(w), "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w));
+}
+
 // volatile: the load must stay under its guard (it is never speculated)
 __device__ __forceinline__ uint4 ld_gather(const void *p) {
     uint4 r;
@@ -415,9 +432,15 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
             }
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
+                const float w = pr[St::head_of(v)];
+#ifdef GLGA_LOCAL_FMA2
+                if constexpr (sizeof(T) == 2) {
+                    acc_bf16x8_f32x2(st.acc[v], w, vb[u][v]);
+                    continue;
+                }
+#endif
                 float vf[VE];
                 Io<T>::unpack(vb[u][v], vf);
-                const float w = pr[St::head_of(v)];
 #pragma unroll
                 for (int e = 0; e < VE; ++e) st.acc[v][e] = fmaf(w, vf[e], st.acc[v][e]);
             }
@@ -583,8 +606,11 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&
 // Blocks per SM the register budget aims at: 3 (at most 85 registers) while the gather
 // buffers take at most 32 registers (8 per edge step and vector, doubled when pipelined),
 // else 2.
+#ifndef GLGA_LOCAL_MINB3
+#define GLGA_LOCAL_MINB3 3
+#endif
 constexpr int local_min_blocks(int VPL, int U, bool PIPE) {
-    return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? 3 : 2;
+    return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? GLGA_LOCAL_MINB3 : 2;
 }
 template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE, bool CB>
 __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
@@ -837,6 +863,13 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
         // step, 3 blocks per SM); at D = 512 two consecutive vectors of one head per lane,
         // the next step's gathers issued before the current one is consumed, column
         // indices in batches
+#if defined(GLGA_LOCAL_X128)
+        if (p.nvec == 16 && c->r == 32) {
+            if (GLGA_LOCAL_X128 == 1) return launch_local<B, 16, 4, 1, 2, false>(c, p, s);
+            if (GLGA_LOCAL_X128 == 2) return launch_local<B, 16, 4, 1, 8, false>(c, p, s);
+            return launch_local<B, 16, 4, 1, 4, false>(c, p, s);
+        }
+#endif
         if (p.nvec == 16 && c->r == 32) return launch_local<B, 16, 4, 1, 4, false>(c, p, s);
         if (p.nvec == 32 && c->r == 32) return launch_local<B, 32, 4, 1, 4, false>(c, p, s);
         if (p.nvec == 64 && c->r == 64) return launch_local<B, 64, 4, 2, 2, true, true, true>(c, p, s);

@@ -280,8 +280,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
         for (int i = 0; i < n_my; ++i, tw.next()) {
             const int buf = i & 1;
-            const bool got = mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(i >> 1) & 1u);
-            // (no barrier spans the epilogue warps: each gives up on its own wait)
+            // no barrier spans the epilogue warps: each warp agrees on its own wait (the
+            // TMEM loads below are warp-collective)
+            const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(i >> 1) & 1u));
             if (!got) {
                 if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
                 ok = false;

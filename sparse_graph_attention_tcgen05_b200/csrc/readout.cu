@@ -366,7 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1) readout_kernel(const __grid_const
                 tw.next();
                 for (int kb = 0; kb < p.nk; ++kb, rp.next(p.stages)) {
                     const int s = rp.slot;
-                    if (bad || !mbar_wait_bounded(&full_bar[s], rp.phase)) {
+                    // the warp agrees on the outcome (it stays converged for its arrival)
+                    if (!__all_sync(0xffffffffu, !bad && mbar_wait_bounded(&full_bar[s], rp.phase))) {
                         bad = true;        // (the MMA warp's own bounded wait then gives up too)
                         continue;
                     }

@@ -90,10 +90,13 @@ def test_segments_inside_tiles(io, H, r):
     _check_stats(w, inter, ref)
 
 
-def test_many_tiny_segments():
+@pytest.mark.parametrize("io,H,r", [("bf16", 2, 32), ("f32", 8, 8), ("bf16", 4, 64)])
+def test_many_tiny_segments(io, H, r):
+    # every non-empty segment fits one statistics range: the statistics kernel writes each
+    # segment's S, z and readout operand itself (no reduction pass); empty segments too
     rng = np.random.default_rng(3)
     sizes = rng.integers(0, 8, 400)
-    w, seg = _unaligned("bf16", 2, 32, seed=9, sizes=sizes)
+    w, seg = _unaligned(io, H, r, seed=9, sizes=sizes)
     Y, inter = _run(w, seg)
     ref = _oracle(w, seg)
     assert_close_to_oracle(w, Y, ref)
