@@ -79,13 +79,21 @@ typedef enum { GLGA_F32 = 0, GLGA_BF16 = 1 } glga_dtype;
  * range partials of the tensor-core weight-gradient GEMM, about num_SMs*d*3*H*r floats);
  * glga_forward on such a context also stores each row's softmax log-sum-exp per head for
  * the backward.  Whole-graph, one-segment contexts
- * with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).                             */
+ * with at most 32 heads (GLGA_ERR_UNSUPPORTED otherwise).
+ * fuse_stats != 0 asks for the global statistics inside the projection GEMM: a
+ * one-segment bf16 context with H*r = 128 and r dividing 64 then accumulates
+ * phi(K)^T [V | 1] in the GEMM's epilogue (per-CTA partial sums, then the same
+ * fixed-order reduction) instead of launching the statistics kernel; other contexts
+ * ignore it.  Off by default: on the arxiv-shaped graph the fused GEMM plus reduction
+ * take longer than the GEMM and the statistics kernel, and the statistics kernel's pass
+ * over K and V also leaves them in L2 for the local kernel that follows.               */
 typedef struct {
     int32_t warp_max_degree;
     int32_t chunk_edges;
     int32_t debug_checks;
     int32_t debug_fail_alloc;
     int32_t backward;
+    int32_t fuse_stats;
 } glga_options;
 
 /* Fills *opts with the defaults used when glga_create gets opts == NULL:

@@ -152,6 +152,7 @@ glga_status glga_default_options(glga_options *opts) {
     opts->debug_checks = 0;
     opts->debug_fail_alloc = 0;
     opts->backward = 0;
+    opts->fuse_stats = 0;
     return GLGA_OK;
 }
 

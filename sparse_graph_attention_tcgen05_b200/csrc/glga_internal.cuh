@@ -116,6 +116,8 @@ struct Ctx {
     std::vector<int64_t> seg_ptr;     // host copy [n_seg + 1]
     int32_t *seg_part_ptr = nullptr;  // statistics ranges of each segment [n_seg + 1]
     bool stats_direct = false;        // every non-empty segment one range: no reduction pass
+    bool stats_fused = false;         // S | z partials from the projection epilogue (one per CTA)
+    int32_t stats_fused_parts = 0;    // ... the projection's grid size
     int32_t *part_seg = nullptr;      // ... and the segment of each range
     int32_t *tile_seg = nullptr;      // segment of each 128-row readout tile's first row
     int32_t *fix_row = nullptr;       // rows whose segment differs from their tile's

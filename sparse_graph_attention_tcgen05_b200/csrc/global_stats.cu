@@ -653,7 +653,9 @@ glga_status stats_setup(Ctx *c) {
         set_error("glga_create: %d statistics ranges need more than 4 GiB of partial sums", parts);
         return GLGA_ERR_UNSUPPORTED;
     }
-    glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart), one * std::max(parts, 1));
+    // (the projection epilogue writes one partial per CTA when the statistics are fused)
+    glga_status st = dev_alloc(c, reinterpret_cast<void **>(&c->Spart),
+                               one * std::max(std::max(parts, c->stats_fused_parts), 1));
     if (st == GLGA_OK) st = dev_alloc(c, reinterpret_cast<void **>(&c->Sz), one * c->n_seg);
     if (st == GLGA_OK) {
         // empty segments keep zero statistics (the direct epilogue never writes them)
@@ -683,7 +685,7 @@ glga_status stats_setup(Ctx *c) {
 namespace {
 // Partial sums of S | z over the context's row ranges (Spart).
 glga_status stats_partials(Ctx *c, cudaStream_t s) {
-    if (c->N > 0) {
+    if (c->N > 0 && !c->stats_fused) {
         StatsParams p;
         p.N = c->N;
         p.D = c->D;
@@ -736,7 +738,7 @@ glga_status reduce_into_stats(Ctx *c, const float *part, int P, float *flat, cud
 glga_status stats_run_partial(Ctx *c, float *own, cudaStream_t s) {
     glga_status st = stats_partials(c, s);
     if (st != GLGA_OK) return st;
-    const int P = c->N > 0 ? c->stats_parts : 0;
+    const int P = c->N == 0 ? 0 : c->stats_fused ? c->stats_fused_parts : c->stats_parts;
     return c->io == GLGA_F32 ? reduce_into_stats<float>(c, c->Spart, P, own, s)
                              : reduce_into_stats<__nv_bfloat16>(c, c->Spart, P, own, s);
 }
@@ -751,13 +753,14 @@ glga_status stats_run(Ctx *c, cudaStream_t s) {
     if (st0 != GLGA_OK) return st0;
     if (c->stats_direct) return GLGA_OK;   // the epilogue wrote S, z and the readout operand
     const int total = c->H * c->r * (c->r + 1);
-    const int P = c->N > 0 ? c->stats_parts : 0;
+    const int P = c->N == 0 ? 0 : c->stats_fused ? c->stats_fused_parts : c->stats_parts;
     const int64_t seg_stride = static_cast<int64_t>(c->ro_groups) * c->ro_bn * c->ro_kp;
     const int64_t plane = c->n_seg * seg_stride;
     const dim3 rgrid(static_cast<unsigned>(ceil_div(total, 32)),
                      static_cast<unsigned>(std::min<int64_t>(c->n_seg, 65535)));
-    // with no rows every segment's sums are zero (no ranges to add)
-    const int32_t *spp = c->N > 0 ? c->seg_part_ptr : nullptr;
+    // with no rows every segment's sums are zero (no ranges to add); the fused partials
+    // (one segment) are parts 0 .. P-1
+    const int32_t *spp = c->N > 0 && !c->stats_fused ? c->seg_part_ptr : nullptr;
     if (c->n_seg > 1 && spp) {
         const dim3 sgrid(static_cast<unsigned>(c->H),
                          static_cast<unsigned>(std::min<int64_t>(c->n_seg, 65535)));

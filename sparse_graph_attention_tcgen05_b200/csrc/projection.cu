@@ -55,7 +55,35 @@ struct GemmParams {
     int64_t ldc;
     int32_t ncols;
     unsigned *flag;
+    // statistics in the epilogue (bf16, D = 128, heads inside 64-feature groups): column
+    // tiles are [K_g | V_g] for the feature groups g, then [Q | gate]; each CTA walks whole
+    // row blocks and accumulates phi(K_g)^T [V_g | 1] in TMEM across them
+    int32_t fuse;
+    int32_t groups;          // feature groups of 64 (KV column tiles)
+    int32_t R;               // head width r
+    uint32_t acc_stride;     // TMEM columns between the two projection accumulators
+    uint32_t stats_col0;     // first TMEM column of the statistics accumulators
+    float *part;             // [gridDim.x][H][r][r + 1] per-CTA partial sums
 };
+
+constexpr uint32_t kStatsCols = 96;      // TMEM columns per feature group: S (64) | z (16)
+constexpr uint32_t kFusedAccStride = 160; // projection accumulators (<= 144 columns) when fused
+
+// Tile i of this CTA: tiles blockIdx.x + i * gridDim.x of the row-major tile grid, or, when
+// the statistics are fused, column tile i % n_tiles of row block blockIdx.x + (i / n_tiles)
+// * gridDim.x (a CTA owns whole row blocks, so K_g and V_g of a row meet in one CTA).
+__device__ __forceinline__ void tile_at(const GemmParams &p, int32_t i, int32_t &row, int32_t &col) {
+    if (p.fuse) {
+        row = static_cast<int32_t>(blockIdx.x) + (i / p.n_tiles) * static_cast<int32_t>(gridDim.x);
+        col = i % p.n_tiles;
+    } else {
+        const int64_t t = static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(i) * gridDim.x;
+        row = static_cast<int32_t>(t / p.n_tiles);
+        col = static_cast<int32_t>(t % p.n_tiles);
+    }
+}
+
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 template <typename T>
 __device__ __forceinline__ void store_vec32(T *dst, const uint32_t (&v)[32]);
@@ -150,14 +178,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
     __shared__ __align__(8) uint64_t accf_bar[2];    // MMA -> epilogue: buffer holds a tile
     __shared__ __align__(8) uint64_t acce_bar[2];    // epilogue -> MMA: buffer drained
+    __shared__ __align__(8) uint64_t staged_bar[2];  // epilogue -> MMA: staging b written (fused)
+    __shared__ __align__(8) uint64_t sdone_bar[2];   // MMA -> epilogue: staging b read (fused)
     __shared__ uint32_t tmem_base_sh;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t n_my = p.n_total_tiles > blockIdx.x
-                             ? static_cast<int32_t>((p.n_total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x)
-                             : 0;
+    int32_t n_my;
+    if (p.fuse) {
+        const int64_t nrb = p.n_total_tiles / p.n_tiles;   // row blocks
+        n_my = nrb > blockIdx.x ? static_cast<int32_t>((nrb - blockIdx.x + gridDim.x - 1) / gridDim.x) * p.n_tiles
+                                : 0;
+    } else {
+        n_my = p.n_total_tiles > blockIdx.x
+                   ? static_cast<int32_t>((p.n_total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x)
+                   : 0;
+    }
+    const uint32_t box_bytes = kBM * kRowBytes;          // one 128-row x 64-column bf16 box
+    // fused statistics: two staging buffers of three boxes each (K_g | phi(K_g) | V_g, or
+    // the two Q boxes; tile i uses buffer i & 1), then the "ones" operand of the z MMA
+    uint8_t *ones = smem + p.stage_area + 6 * box_bytes;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -168,7 +209,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
             mbar_init(&accf_bar[b], 1);
             mbar_init(&acce_bar[b], 8);
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&staged_bar[b], 8);
+            mbar_init(&sdone_bar[b], 1);
+        }
         fence_mbar_init();
+    }
+    if (p.fuse && threadIdx.x < 256) {
+        // ones tile (16 rows of 128 bytes, K-major): row 0 = 1.0, rows 1..15 = 0; the
+        // swizzle permutes 16-byte chunks inside a row only, so row 0 reads as ones at
+        // every K offset
+        uint32_t *o = reinterpret_cast<uint32_t *>(ones);
+        for (int k = threadIdx.x; k < 16 * kRowBytes / 4; k += 256) o[k] = k < kRowBytes / 4 ? 0x3F803F80u : 0u;
+        fence_proxy_async_smem();
     }
     if (warp == kProdWarp && lane == 0) {
         tma_prefetch_desc(&tmA0);
@@ -191,11 +244,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         // ---------------- TMA producer: every K block of every tile of this CTA ----------
         int it = 0;           // K blocks issued so far
         RingPos rp;           // stage ring position
-        TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
         bool ok = true;
-        for (int i = 0; i < n_my && ok; ++i, tw.next()) {
-            const int32_t m0 = tw.row * kBM;
-            const int32_t n0 = tw.col * p.BN;
+        for (int i = 0; i < n_my && ok; ++i) {
+            int32_t trow, tcol;
+            tile_at(p, i, trow, tcol);
+            const int32_t m0 = trow * kBM;
+            const int32_t n0 = tcol * p.BN;
             for (int kb = 0; kb < p.nk; ++kb, ++it, rp.next(p.stages)) {
                 const int s = rp.slot;
                 if (it >= p.stages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
@@ -222,13 +276,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         // ---------------- MMA issuer ----------------
         const uint32_t idesc_main = instr_desc(kBM, p.BN, kFmt, false, false);
         const uint32_t idesc_last = instr_desc(kBM, p.bn_last, kFmt, false, false);
+        // fused statistics of tile j (its staging buffer is written): for a [K_g | V_g]
+        // tile, S_g += phi(K_g)^T V_g and z_g += phi(K_g)^T 1 with the node rows as the
+        // contraction; A = [phi(K_g) | V_g] (M = 128, MN-major, the upper 64 rows of the
+        // product are not used), B = V_g (N = 64, MN-major) and the ones tile (N = 16)
+        const uint32_t idS = instr_desc(128, 64, 1u, true, true);
+        const uint32_t idZ = instr_desc(128, 16, 1u, true, false);
+        auto stats_step = [&](int32_t j) -> bool {
+            // staging buffer j & 1 is written for the (j >> 1)-th time
+            if (!mbar_wait_bounded(&staged_bar[j & 1], static_cast<uint32_t>(j >> 1) & 1u)) return false;
+            tc_fence_after();
+            const int32_t col = j % p.n_tiles;
+            if (col < p.groups) {
+                const uint32_t sbase = smem_u32(smem + p.stage_area + (j & 1) * 3 * box_bytes);
+                const uint32_t acc_s = tmem + p.stats_col0 + static_cast<uint32_t>(col) * kStatsCols;
+                const uint64_t dones = smem_desc(smem_u32(ones), 16, 1024, 2);
+#pragma unroll
+                for (int ks = 0; ks < kBM / 16; ++ks) {
+                    const uint64_t ad = smem_desc(sbase + box_bytes + ks * 16 * kRowBytes, box_bytes, 1024, 2);
+                    const uint64_t bd = smem_desc(sbase + 2 * box_bytes + ks * 16 * kRowBytes, box_bytes, 1024, 2);
+                    const uint32_t acc = (j >= p.n_tiles || ks > 0) ? 1u : 0u;
+                    umma_bf16(acc_s, ad, bd, idS, acc);
+                    umma_bf16(acc_s + 64, ad, dones, idZ, acc);
+                }
+            }
+            umma_commit(&sdone_bar[j & 1]);   // the staging buffer may be rewritten
+            return true;
+        };
         bool ok = true;
         RingPos rp;
-        TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
-        for (int i = 0; i < n_my && ok; ++i, tw.next()) {
+        for (int i = 0; i < n_my && ok; ++i) {
+            int32_t trow, tcol;
+            tile_at(p, i, trow, tcol);
+            (void)trow;
             const int buf = i & 1;
-            const uint32_t acc_col = static_cast<uint32_t>(buf * 256);
-            const uint32_t idesc = (tw.col == p.n_tiles - 1) ? idesc_last : idesc_main;
+            const uint32_t acc_col = static_cast<uint32_t>(buf) * p.acc_stride;
+            const uint32_t idesc = (tcol == p.n_tiles - 1) ? idesc_last : idesc_main;
             // wait until the epilogue drained this buffer's previous tile (tile i - 2)
             if (i >= 2 && !mbar_wait_bounded(&acce_bar[buf], static_cast<uint32_t>((i >> 1) - 1) & 1u)) {
                 ok = false;
@@ -262,7 +345,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 umma_commit(&empty_bar[s]);   // stage reusable once these MMAs finish
             }
             if (ok) umma_commit(&accf_bar[buf]);   // the tile's accumulator is complete
+            // the previous tile's statistics, while this tile's MMAs run
+            if (ok && p.fuse && i >= 1 && !stats_step(i - 1)) ok = false;
         }
+        if (ok && p.fuse && n_my > 0 && !stats_step(n_my - 1)) ok = false;
         if (!ok) atomicOr(p.flag, kDevErrTimeout);
     }
     __syncwarp();
@@ -274,12 +360,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
         const int quad = warp & 3, wg = warp >> 2;
         const int rt = quad * 32 + lane;                 // row inside the tile
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t box_bytes = kBM * kRowBytes;      // one 128-row x 64-column bf16 box
         const int nbox = p.BN / 64;
         bool ok = true;
-        TileWalk tw(blockIdx.x, gridDim.x, p.n_tiles);
-        for (int i = 0; i < n_my; ++i, tw.next()) {
+        for (int i = 0; i < n_my; ++i) {
+            int32_t trow, tcol;
+            tile_at(p, i, trow, tcol);
             const int buf = i & 1;
+            const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(buf) * p.acc_stride;
             // no barrier spans the epilogue warps: each warp agrees on its own wait (the
             // TMEM loads below are warp-collective)
             const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&accf_bar[buf], static_cast<uint32_t>(i >> 1) & 1u));
@@ -289,16 +376,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 break;
             }
             tc_fence_after();
-            const int64_t m0 = static_cast<int64_t>(tw.row) * kBM;
+            const int64_t m0 = static_cast<int64_t>(trow) * kBM;
             const int64_t row = m0 + rt;
-            const int ntile = tw.col;
+            const int ntile = tcol;
             const int n0 = ntile * p.BN;
             const int bn = ntile == p.n_tiles - 1 ? p.bn_last : p.BN;
             if (p.C) {
                 // plain GEMM: float32 rows of C, columns below ncols
                 for (int c0 = wg * 32; c0 < bn; c0 += 64) {
                     uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + c0), v);
+                    tmem_ld32(acc + static_cast<uint32_t>(c0), v);
                     tmem_ld_wait();
                     const int gc0 = n0 + c0;
                     if (row < p.M) {
@@ -315,6 +402,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acce_bar[buf]);
+            } else if (p.fuse) {
+                // Staging buffer i & 1 of three boxes.  [K_g | V_g] tile: warpgroup g & 1
+                // stages K_g (box 0) and phi(K_g) (box 1, zero past row M), the other V_g
+                // (box 2); [Q | gate] tile: warpgroup w stages Q box w, warpgroup 1 the gate
+                // column.  A buffer is rewritten only after the statistics MMAs of its
+                // previous tile (i - 2) and this warp's TMA stores out of it have read it.
+                uint8_t *sb = smem + p.stage_area + buf * 3 * box_bytes;
+                if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait_bounded(&sdone_bar[buf], static_cast<uint32_t>((i >> 1) - 1) & 1u))) {
+                    if (lane == 0) atomicOr(p.flag, kDevErrTimeout);
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) bulk_wait_group_read1();   // (the other buffer's stores may still run)
+                __syncwarp();
+                const bool kv = ntile < p.groups;
+                const bool kwarp = kv && wg == (ntile & 1);
+                const int box = kv ? (kwarp ? 0 : 2) : wg;
+                const uint32_t c_src = kv ? (kwarp ? 0u : 64u) : static_cast<uint32_t>(wg * 64);
+                const bool valid = row < p.M;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t v[32];
+                    tmem_ld32(acc + c_src + static_cast<uint32_t>(half * 32), v);
+                    tmem_ld_wait();
+                    uint8_t *rp = sb + box * box_bytes + rt * kRowBytes;
+                    uint8_t *fp = sb + box_bytes + rt * kRowBytes;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = pack_bf16x2(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
+                        const int chunk = ((half * 4 + q) ^ (rt & 7)) * 16;
+                        *reinterpret_cast<uint4 *>(rp + chunk) = make_uint4(w[0], w[1], w[2], w[3]);
+                        if (kwarp) {
+                            // phi of the stored (bf16) k; rows past M contribute nothing to z
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float a = valid ? phi_elu1(__uint_as_float(w[e] << 16)) : 0.f;
+                                const float b2 = valid ? phi_elu1(__uint_as_float(w[e] & 0xffff0000u)) : 0.f;
+                                w[e] = pack_bf16x2(a, b2);
+                            }
+                            *reinterpret_cast<uint4 *>(fp + chunk) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                if (!kv && wg == 1) {
+                    uint32_t v[32];
+                    tmem_ld32(acc + static_cast<uint32_t>(p.BN), v);
+                    tmem_ld_wait();
+                    if (valid) p.t[row] = __uint_as_float(v[0]);   // gate logit column
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce_bar[buf]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int64_t y = m0 + quad * 32;
+                    if (y < p.M) {
+                        const uint8_t *src = sb + box * box_bytes + quad * 32 * kRowBytes;
+                        if (kv)
+                            tma_store_2d(&tmKVs, src, (kwarp ? 0 : p.D) + ntile * 64, static_cast<int32_t>(y));
+                        else
+                            tma_store_2d(&tmQs, src, wg * 64, static_cast<int32_t>(y));
+                    }
+                    bulk_commit_group();
+                    mbar_arrive(&staged_bar[buf]);   // phi(K_g) and V_g are in place for the MMA
+                }
             } else if (p.tma_epi) {
                 // Each warp owns whole 64-column boxes of its 32 rows (boxes wg, wg + 2, ...;
                 // in the last column tile warpgroup 1 also takes the gate column past them):
@@ -334,7 +490,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         uint32_t v[32];
-                        tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + b * 64 + half * 32), v);
+                        tmem_ld32(acc + static_cast<uint32_t>(b * 64 + half * 32), v);
                         tmem_ld_wait();
                         uint8_t *rp = sb + b * box_bytes + rt * kRowBytes;
 #pragma unroll
@@ -350,7 +506,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 }
                 if (bn > p.BN && wg == 1) {
                     uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + p.BN), v);
+                    tmem_ld32(acc + static_cast<uint32_t>(p.BN), v);
                     tmem_ld_wait();
                     if (row < p.M) p.t[row] = __uint_as_float(v[0]);   // gate logit column
                 }
@@ -374,7 +530,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
             } else {
                 for (int c0 = wg * 32; c0 < bn; c0 += 64) {
                     uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * 256 + c0), v);
+                    tmem_ld32(acc + static_cast<uint32_t>(c0), v);
                     tmem_ld_wait();
                     if (row < p.M) store_row_cols<T>(p, row, n0 + c0, n0 + bn, v);
                 }
@@ -383,8 +539,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                 if (lane == 0) mbar_arrive(&acce_bar[buf]);
             }
         }
-        (void)ok;
-        if (p.tma_epi && lane == 0) bulk_wait_group_read0();   // shared memory outlives the stores
+        if (p.fuse && quad < 2 && wg < p.groups) {
+            // this CTA's statistics: warps of quads 0-1 in warpgroup g read feature group g
+            // (TMEM lanes = its 64 features) and write the rows of their heads' blocks
+            const int g = wg;
+            const int f = g * 64 + quad * 32 + lane;            // feature
+            const int h = f / p.R, a = f - h * p.R;
+            const int hc0 = h * p.R - g * 64;                   // the head's first V column
+            uint32_t s0[32], s1[32], zv[32];
+            // the last tile's commit follows every statistics MMA of the CTA
+            const int32_t jl = n_my - 1;
+            const bool got = ok && n_my > 0 &&
+                             __all_sync(0xffffffffu, mbar_wait_bounded(&sdone_bar[jl & 1], static_cast<uint32_t>(jl >> 1) & 1u));
+            if (ok && n_my > 0 && !got && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+            tc_fence_after();
+            const uint32_t acc_s = tmem + lane_base + p.stats_col0 + static_cast<uint32_t>(g) * kStatsCols;
+            tmem_ld32(acc_s, s0);
+            tmem_ld32(acc_s + 32, s1);
+            tmem_ld32(acc_s + 64, zv);
+            tmem_ld_wait();
+            float *dst = p.part + (static_cast<int64_t>(blockIdx.x) * p.D + f) * (p.R + 1);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (j >= hc0 && j < hc0 + p.R) dst[j - hc0] = got ? __uint_as_float(s0[j]) : 0.f;
+                if (j + 32 >= hc0 && j + 32 < hc0 + p.R) dst[j + 32 - hc0] = got ? __uint_as_float(s1[j]) : 0.f;
+            }
+            dst[p.R] = got ? __uint_as_float(zv[0]) : 0.f;
+        }
+        if ((p.tma_epi || p.fuse) && lane == 0) bulk_wait_group_read0();   // shared memory outlives the stores
     }
     tc_fence_before();
     __syncthreads();
@@ -410,7 +592,7 @@ __device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16 *p) {
 template <int SPLIT, typename T>
 __global__ void pack_weights_kernel(const T *__restrict__ WQ, const T *__restrict__ WK,
                                     const T *__restrict__ WV, const T *__restrict__ wg, int d,
-                                    int D, int dp, int rows, T *__restrict__ Wt) {
+                                    int D, int dp, int rows, int fused, T *__restrict__ Wt) {
     const int64_t total = static_cast<int64_t>(rows) * dp;
     const int64_t plane = total;
     for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
@@ -418,7 +600,17 @@ __global__ void pack_weights_kernel(const T *__restrict__ WQ, const T *__restric
         const int c = static_cast<int>(idx / dp);
         const int k = static_cast<int>(idx % dp);
         float v = 0.f;
-        if (k < d) {
+        if (k < d && fused && c < 2 * D) {
+            // [K_g | V_g] for the 64-feature groups g, then Q and the gate
+            const int g = c / 128, w = c % 128;
+            const T *src = w < 64 ? WK : WV;
+            v = ld_f32<T>(src + static_cast<int64_t>(k) * D + g * 64 + (w & 63));
+        } else if (k < d && fused) {
+            if (c < 3 * D)
+                v = ld_f32<T>(WQ + static_cast<int64_t>(k) * D + (c - 2 * D));
+            else if (c == 3 * D)
+                v = ld_f32<T>(wg + k);
+        } else if (k < d) {
             if (c < D)
                 v = ld_f32<T>(WQ + static_cast<int64_t>(k) * D + c);
             else if (c < 2 * D)
@@ -502,13 +694,23 @@ glga_status launch_gemm(Ctx *c, cudaStream_t s) {
     p.ldc = 0;
     p.ncols = 0;
     p.flag = c->dev_flag;
-    const uint32_t staging = p.tma_epi ? static_cast<uint32_t>(p.sbufs) * (c->BN / 64) * kBM * kRowBytes : 0u;
+    p.fuse = c->stats_fused ? 1 : 0;
+    p.groups = c->stats_fused ? c->D / 64 : 0;
+    p.R = c->r;
+    p.acc_stride = c->stats_fused ? kFusedAccStride : 256u;
+    p.stats_col0 = 2 * kFusedAccStride;
+    p.part = c->Spart;
+    // fused: two staging buffers of three boxes and the 2 KB ones tile
+    const uint32_t staging = c->stats_fused ? 6u * kBM * kRowBytes + 2048u
+                             : p.tma_epi ? static_cast<uint32_t>(p.sbufs) * (c->BN / 64) * kBM * kRowBytes : 0u;
     const size_t smem = static_cast<size_t>(p.stage_area) + staging + 1024;
     auto kern = proj_gemm_kernel<SPLIT, T>;
     GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(smem)));
-    // persistent: one CTA per SM (it holds all 512 TMEM columns)
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(p.n_total_tiles, c->num_sms));
+    // persistent: one CTA per SM (it holds all 512 TMEM columns); fused statistics give
+    // each CTA whole row blocks
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(
+        c->stats_fused ? p.n_total_tiles / p.n_tiles : p.n_total_tiles, c->num_sms));
     const CUtensorMap &a1 = planes == 2 ? c->tmA[1].map : c->tmA[0].map;
     const CUtensorMap &b1 = planes == 2 ? c->tmB[1].map : c->tmB[0].map;
     const CUtensorMap &qs = c->gemm_tma_epi ? c->tmQs.map : c->tmB[0].map;     // unused otherwise
@@ -552,6 +754,12 @@ glga_status gemm_nt_f32out(Ctx *c, glga_dtype t, const void *A, int64_t M, int64
     p.ldc = ldc;
     p.ncols = static_cast<int32_t>(ncols);
     p.flag = c->dev_flag;
+    p.fuse = 0;
+    p.groups = 0;
+    p.R = 0;
+    p.acc_stride = 256;
+    p.stats_col0 = 0;
+    p.part = nullptr;
     const CUtensorMapDataType dt = t == GLGA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap ma, mb;
     glga_status r = encode_tmap_2d(&ma, dt, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
@@ -609,7 +817,19 @@ glga_status projection_setup(Ctx *c) {
     c->dp = static_cast<int32_t>(ceil_div(c->d, kt) * kt);
     const int D3 = 3 * c->D;
     c->gemm_tma_epi = false;
-    if (c->split == 1 && c->D % 64 == 0) {
+    // global statistics in the epilogue (on request): bf16, D = 128 (two 64-feature
+    // groups), heads inside a group, one segment
+    c->stats_fused = c->opts.fuse_stats && c->split == 1 && c->D == 128 && 64 % c->r == 0 &&
+                     c->n_seg == 1 && c->N > 0;
+    c->stats_fused_parts = c->stats_fused ? static_cast<int32_t>(std::min<int64_t>(ceil_div(c->N, kBM), c->num_sms)) : 0;
+    if (c->stats_fused) {
+        // column tiles [K_0 | V_0], [K_1 | V_1], [Q | gate + 15 zero columns]
+        c->BN = 128;
+        c->n_tiles = 3;
+        c->bn_last = c->BN + 16;
+        c->Dp = D3 + 16;
+        c->gemm_tma_epi = true;
+    } else if (c->split == 1 && c->D % 64 == 0) {
         // Column tiles of BN (a multiple of the 64-column store box) over Q | K | V; the
         // last tile also carries the gate column (+15 zero columns).  Q/K/V leave through
         // shared memory and TMA stores.
@@ -638,9 +858,11 @@ glga_status projection_setup(Ctx *c) {
     // overlap the next tile's epilogue; one is used when two would leave fewer than four
     // ring stages, since the operand loads in flight bound the MMA rate.
     constexpr uint32_t kBudget = 220u * 1024u;
-    const uint32_t stg1 = c->gemm_tma_epi ? (c->BN / 64) * kBM * kRowBytes : 0u;
-    c->gemm_sbufs = (kBudget - 2u * stg1) / stage_bytes >= 4u ? 2 : 1;
-    const uint32_t budget = kBudget - static_cast<uint32_t>(c->gemm_sbufs) * stg1;
+    // (fused statistics: always two buffers of three boxes, plus the 2 KB ones tile)
+    const uint32_t stg1 = c->stats_fused ? 3u * kBM * kRowBytes
+                          : c->gemm_tma_epi ? (c->BN / 64) * kBM * kRowBytes : 0u;
+    c->gemm_sbufs = c->stats_fused || (kBudget - 2u * stg1) / stage_bytes >= 4u ? 2 : 1;
+    const uint32_t budget = kBudget - static_cast<uint32_t>(c->gemm_sbufs) * stg1 - (c->stats_fused ? 2048u : 0u);
     int st = static_cast<int>(budget / stage_bytes);
     c->stages = std::max(1, std::min(st, kMaxStages));
 
@@ -696,12 +918,12 @@ glga_status projection_run(Ctx *c, const void *X, const void *WQ, const void *WK
         pack_weights_kernel<3, float><<<wblocks, 256, 0, s>>>(
             static_cast<const float *>(WQ), static_cast<const float *>(WK),
             static_cast<const float *>(WV), static_cast<const float *>(wg), c->d, c->D, c->dp,
-            c->Dp, static_cast<float *>(c->Wt));
+            c->Dp, 0, static_cast<float *>(c->Wt));
     } else {
         pack_weights_kernel<1, __nv_bfloat16><<<wblocks, 256, 0, s>>>(
             static_cast<const __nv_bfloat16 *>(WQ), static_cast<const __nv_bfloat16 *>(WK),
             static_cast<const __nv_bfloat16 *>(WV), static_cast<const __nv_bfloat16 *>(wg), c->d,
-            c->D, c->dp, c->Dp, static_cast<__nv_bfloat16 *>(c->Wt));
+            c->D, c->dp, c->Dp, c->stats_fused ? 1 : 0, static_cast<__nv_bfloat16 *>(c->Wt));
     }
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;

@@ -34,7 +34,7 @@ class GLGAError(RuntimeError):
 class Options(ctypes.Structure):
     _fields_ = [("warp_max_degree", ctypes.c_int32), ("chunk_edges", ctypes.c_int32),
                 ("debug_checks", ctypes.c_int32), ("debug_fail_alloc", ctypes.c_int32),
-                ("backward", ctypes.c_int32)]
+                ("backward", ctypes.c_int32), ("fuse_stats", ctypes.c_int32)]
 
 
 _lib = None
