@@ -139,23 +139,42 @@ __device__ __forceinline__ float head_reduce(float x, int lph) {
     return x;
 }
 
-// out[x] += sum over c < R of M[c * R + f0 + x] * u_c for one head: M is a row-major
-// R x R fp32 block, and u_c is held by the head's lanes (lane hb + c / EPL, element
-// c % EPL), so it travels by shuffle.  Every lane of the warp takes part (lanes outside
-// D pass f0 = 0 and hb = 0 and discard the result).
-template <int EPL>
-__device__ __forceinline__ void head_matvec(const float *M, int R, int f0, int hb, int lph, const float (&u)[EPL],
-                                            float (&out)[EPL]) {
-    for (int sl = 0; sl < lph; ++sl) {
+// out[k][x] += sum over c < R of M[c * R + f0 + x] * u[k]_c for one head and each of the
+// warp's RPW rows k: M is a row-major R x R fp32 block, and u[k]_c is held by the head's
+// lanes (lane hb + c / EPL, element c % EPL), so it travels by shuffle; each row of M is
+// loaded once for all RPW rows.  LPH = R / EPL when known at compile time (the loop is
+// then unrolled), else 0 and lph gives it.  Every lane of the warp takes part (lanes
+// outside D pass f0 = 0 and hb = 0 and discard the result).
+template <int EPL, int LPH, int RPW>
+__device__ __forceinline__ void head_matvec(const float *M, int R, int f0, int hb, int lph,
+                                            const float (&u)[RPW][EPL], float (&out)[RPW][EPL]) {
+    auto step = [&](int sl) {
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
-            const float uc = __shfl_sync(0xffffffffu, u[e], hb + sl);
             float m[EPL];
             ld_mrow<EPL>(M + static_cast<int64_t>(sl * EPL + e) * R + f0, m);
 #pragma unroll
-            for (int x = 0; x < EPL; ++x) out[x] = fmaf(m[x], uc, out[x]);
+            for (int k = 0; k < RPW; ++k) {
+                const float uc = __shfl_sync(0xffffffffu, u[k][e], hb + sl);
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) out[k][x] = fmaf(m[x], uc, out[k][x]);
+            }
         }
+    };
+    if constexpr (LPH > 0) {
+#pragma unroll 4
+        for (int sl = 0; sl < LPH; ++sl) step(sl);
+    } else {
+        for (int sl = 0; sl < lph; ++sl) step(sl);
     }
+}
+
+// One row (the source side's global terms).
+template <int EPL>
+__device__ __forceinline__ void head_matvec(const float *M, int R, int f0, int hb, int lph, const float (&u)[EPL],
+                                            float (&out)[EPL]) {
+    head_matvec<EPL, 0, 1>(M, R, f0, hb, lph, reinterpret_cast<const float (&)[1][EPL]>(u),
+                           reinterpret_cast<float (&)[1][EPL]>(out));
 }
 
 // The lane's head h, in-head feature offset f0 and the head's first lane hb.
@@ -171,71 +190,91 @@ struct LaneHead {
     }
 };
 
-// One warp per row i: the gate, readout and blend backward.  Writes dL [N, D],
-// D_i = dL_i . L_i per head into Dd [N, H], dnum [N, D], dden [N, H], the global part of
-// dQ into dZ [:, 0:D] and dt into dZ [:, 3D] (dg summed over the whole row in lane order).  Sz holds S [H][R][R] then z [H][R];
-// ST [H][R][R] is S transposed per head.
-template <typename T, int EPL>
-__global__ void __launch_bounds__(256) bwd_readout_kernel(
+// One warp per RPW consecutive rows i: the gate, readout and blend backward.  Writes dL
+// [N, D], D_i = dL_i . L_i per head into Dd [N, H], dnum [N, D], dden [N, H], the global
+// part of dQ into dZ [:, 0:D] and dt into dZ [:, 3D] (dg summed over the whole row in lane
+// order).  Sz holds S [H][R][R] then z [H][R]; ST [H][R][R] is S transposed per head.
+// Rows past N (in the last warp) compute on zeros and store nothing.
+template <typename T, int EPL, int LPH, int RPW>
+__global__ void __launch_bounds__(256, EPL <= 8 ? 2 : 1) bwd_readout_kernel(
     const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t, const float *__restrict__ Sz,
     const float *__restrict__ ST, const T *__restrict__ dY, int64_t N, int H, int R, float b_g, float eps,
     float *__restrict__ dL, float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden,
     float *__restrict__ dZ, int64_t dz_ld) {
-    const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    const int64_t i0 = ((blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5) * RPW;
     const int lane = threadIdx.x & 31;
-    if (i >= N) return;                                   // warp-uniform
+    if (i0 >= N) return;                                  // warp-uniform
     const int D = H * R;
     const LaneHead lh(lane, EPL, D, R);
     const float *S = Sz + static_cast<int64_t>(lh.h) * R * R;
-    float q[EPL], dy[EPL], lv[EPL], ph[EPL], zz[EPL];
-    ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
-    ld_row<T, EPL>(dY + i * D, lane, lh.act, dy);
-    ld_row<T, EPL>(L + i * D, lane, lh.act, lv);
+    float q[RPW][EPL], dy[RPW][EPL], lv[RPW][EPL], ph[RPW][EPL], zz[EPL];
+    bool live[RPW];
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+        const int64_t i = i0 + k;
+        live[k] = i < N;
+        ld_row<T, EPL>(Q + i * D, lane, lh.act && live[k], q[k]);
+        ld_row<T, EPL>(dY + i * D, lane, lh.act && live[k], dy[k]);
+        ld_row<T, EPL>(L + i * D, lane, lh.act && live[k], lv[k]);
+    }
     ld_mrow<EPL>(Sz + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, zz);
-    float den = 0.f;
+    float den[RPW], G[RPW][EPL];
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) {
-        ph[x] = phi(q[x]);
-        den = fmaf(ph[x], zz[x], den);
-    }
-    den = head_reduce(den, lh.lph) + eps;
-    float G[EPL];
+    for (int k = 0; k < RPW; ++k) {
+        den[k] = 0.f;
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) G[x] = 0.f;
-    head_matvec<EPL>(S, R, lh.f0, lh.hb, lh.lph, ph, G);  // num_f = sum_a phi(q_a) S[a][f]
-    const float g = 1.f / (1.f + __expf(-(t[i] + b_g)));
-    float dgp = 0.f, dGG = 0.f, dLL = 0.f, gl[EPL], dn[EPL];
+        for (int x = 0; x < EPL; ++x) {
+            ph[k][x] = phi(q[k][x]);
+            den[k] = fmaf(ph[k][x], zz[x], den[k]);
+            G[k][x] = 0.f;
+        }
+        den[k] = head_reduce(den[k], lh.lph) + eps;
+    }
+    head_matvec<EPL, LPH, RPW>(S, R, lh.f0, lh.hb, lh.lph, ph, G);  // num_f = sum_a phi(q_a) S[a][f]
+    float dn[RPW][EPL], acc[RPW][EPL], dgp[RPW], gk[RPW];
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) {
-        G[x] /= den;
-        dLL = fmaf(g * dy[x], lv[x], dLL);
-        dgp = fmaf(dy[x], lv[x] - G[x], dgp);
-        const float dG = (1.f - g) * dy[x];
-        dGG = fmaf(dG, G[x], dGG);
-        gl[x] = g * dy[x];
-        dn[x] = dG / den;
-    }
-    const int64_t o = i * D + lane * EPL;
-    if (lh.act) {
-        st_mrow<EPL>(dL + o, gl);
-        st_mrow<EPL>(dnum + o, dn);
-    }
-    const float dd = -head_reduce(dGG, lh.lph) / den;
-    dLL = head_reduce(dLL, lh.lph);
-    if (lh.act && (lane % lh.lph) == 0) {
-        dden[i * H + lh.h] = dd;
-        Dd[i * H + lh.h] = dLL;
-    }
-    float acc[EPL];
+    for (int k = 0; k < RPW; ++k) {
+        const int64_t i = i0 + k;
+        const float g = live[k] ? 1.f / (1.f + __expf(-(t[i] + b_g))) : 0.f;
+        gk[k] = g;
+        float dGG = 0.f, dLL = 0.f, gl[EPL];
+        dgp[k] = 0.f;
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) acc[x] = zz[x] * dd;
+        for (int x = 0; x < EPL; ++x) {
+            G[k][x] /= den[k];
+            dLL = fmaf(g * dy[k][x], lv[k][x], dLL);
+            dgp[k] = fmaf(dy[k][x], lv[k][x] - G[k][x], dgp[k]);
+            const float dG = (1.f - g) * dy[k][x];
+            dGG = fmaf(dG, G[k][x], dGG);
+            gl[x] = g * dy[k][x];
+            dn[k][x] = dG / den[k];
+        }
+        const int64_t o = i * D + lane * EPL;
+        if (lh.act && live[k]) {
+            st_mrow<EPL>(dL + o, gl);
+            st_mrow<EPL>(dnum + o, dn[k]);
+        }
+        const float dd = -head_reduce(dGG, lh.lph) / den[k];
+        dLL = head_reduce(dLL, lh.lph);
+        if (lh.act && live[k] && (lane % lh.lph) == 0) {
+            dden[i * H + lh.h] = dd;
+            Dd[i * H + lh.h] = dLL;
+        }
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) acc[k][x] = zz[x] * dd;
+    }
     // dphi(q)_f = sum_c S[f][c] dnum_c + z_f dden, through ST's rows c
-    head_matvec<EPL>(ST + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, dn, acc);
+    head_matvec<EPL, LPH, RPW>(ST + static_cast<int64_t>(lh.h) * R * R, R, lh.f0, lh.hb, lh.lph, dn, acc);
 #pragma unroll
-    for (int x = 0; x < EPL; ++x) acc[x] *= dphi(q[x]);
-    if (lh.act) st_mrow<EPL>(dZ + i * dz_ld + lane * EPL, acc);
-    for (int w = 16; w > 0; w >>= 1) dgp += __shfl_xor_sync(0xffffffffu, dgp, w);
-    if (lane == 0) dZ[i * dz_ld + 3 * D] = g * (1.f - g) * dgp;
+    for (int k = 0; k < RPW; ++k) {
+        const int64_t i = i0 + k;
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) acc[k][x] *= dphi(q[k][x]);
+        if (lh.act && live[k]) st_mrow<EPL>(dZ + i * dz_ld + lane * EPL, acc[k]);
+        float d = dgp[k];
+        for (int w = 16; w > 0; w >>= 1) d += __shfl_xor_sync(0xffffffffu, d, w);
+        if (lane == 0 && live[k]) dZ[i * dz_ld + 3 * D] = gk[k] * (1.f - gk[k]) * d;
+    }
 }
 
 // Partial sums of dS | dz over the row range of block column p, per head h =
@@ -1112,21 +1151,30 @@ int local_bwd_launches(const Ctx *c) {
     return (c->bw_nq_light > 0) + 2 * (c->bw_nq_heavy > 0) + (c->bw_nk_light > 0) + 2 * (c->bw_nk_heavy > 0);
 }
 
+// Two rows per warp for up to 4 features per lane (one above that); the head loop
+// unrolled for the lane layout of H*r = 128 with r = 32.
+template <typename T, int EPL, int LPH>
+void launch_readout_bwd_e(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
+    constexpr int kRpw = EPL <= 4 ? 2 : 1;
+    const unsigned grid = static_cast<unsigned>(ceil_div(ceil_div(c->N, kRpw) * 32, 256));
+    bwd_readout_kernel<T, EPL, LPH, kRpw><<<grid, 256, 0, s>>>(Q, static_cast<const T *>(c->L), c->t, c->Sz,
+                                                               c->bw_ST, dY, c->N, c->H, c->r, b_g, eps, c->bw_dL,
+                                                               c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz);
+}
+
 template <typename T>
 void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
-    const unsigned grid = static_cast<unsigned>(ceil_div(c->N * 32, 256));
-#define GLGA_RB(E)                                                                                       \
-    case E:                                                                                              \
-        bwd_readout_kernel<T, E><<<grid, 256, 0, s>>>(Q, static_cast<const T *>(c->L), c->t, c->Sz, c->bw_ST, dY, \
-                                                      c->N, c->H, c->r, b_g, eps, c->bw_dL, c->bw_Dd,    \
-                                                      c->bw_dnum,                                        \
-                                                      c->bw_dden, c->bw_dZ, Dz);                         \
-        break;
-    switch (lane_features(c->D)) {
-        GLGA_RB(1) GLGA_RB(2) GLGA_RB(4) GLGA_RB(8) GLGA_RB(16) GLGA_RB(32)
+    const int E = lane_features(c->D), lph = c->r / E;
+    if (E == 4 && lph == 8) return launch_readout_bwd_e<T, 4, 8>(c, Q, dY, b_g, eps, Dz, s);
+    switch (E) {
+        case 1: return launch_readout_bwd_e<T, 1, 0>(c, Q, dY, b_g, eps, Dz, s);
+        case 2: return launch_readout_bwd_e<T, 2, 0>(c, Q, dY, b_g, eps, Dz, s);
+        case 4: return launch_readout_bwd_e<T, 4, 0>(c, Q, dY, b_g, eps, Dz, s);
+        case 8: return launch_readout_bwd_e<T, 8, 0>(c, Q, dY, b_g, eps, Dz, s);
+        case 16: return launch_readout_bwd_e<T, 16, 0>(c, Q, dY, b_g, eps, Dz, s);
+        case 32: return launch_readout_bwd_e<T, 32, 0>(c, Q, dY, b_g, eps, Dz, s);
         default: break;
     }
-#undef GLGA_RB
 }
 
 template <typename T>

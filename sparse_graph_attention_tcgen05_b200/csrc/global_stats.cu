@@ -285,16 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1) stats_tc_kernel(const __grid_cons
                     const int row = (c % kChunksPerBox) / 8;
                     const bool valid = y0 + row < r1;
                     uint4 *kp = reinterpret_cast<uint4 *>(st) + c;
-                    uint4 u = *kp;
-                    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float a = valid ? phi(__uint_as_float(w[e] << 16)) : 0.f;
-                        const float b = valid ? phi(__uint_as_float(w[e] & 0xffff0000u)) : 0.f;
-                        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-                        w[e] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-                    *kp = make_uint4(w[0], w[1], w[2], w[3]);
+                    const uint4 u = *kp;
+                    *kp = valid ? make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w))
+                                : make_uint4(0u, 0u, 0u, 0u);
                 }
                 fence_async_smem();
                 __syncwarp();

@@ -138,29 +138,41 @@ struct Io<__nv_bfloat16> {
     }
 };
 
-// a[0..7] += w * (the 8 bf16 values of u, widened exactly), on the packed f32x2 FMA: four
-// instructions for the eight products.
-__device__ __forceinline__ void acc_bf16x8_f32x2(float (&a)[8], float w, const uint4 &u) {
-    asm("{\n\t.reg .b64 wv, v, c;\n\t.reg .b32 lo, hi;\n\t"
-        "mov.b64 wv, {%8, %8};\n\t"
-        "shl.b32 lo, %9, 16;\n\tand.b32 hi, %9, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
-        "mov.b64 c, {%0, %1};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%0, %1}, c;\n\t"
-        "shl.b32 lo, %10, 16;\n\tand.b32 hi, %10, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
-        "mov.b64 c, {%2, %3};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%2, %3}, c;\n\t"
-        "shl.b32 lo, %11, 16;\n\tand.b32 hi, %11, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
-        "mov.b64 c, {%4, %5};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%4, %5}, c;\n\t"
-        "shl.b32 lo, %12, 16;\n\tand.b32 hi, %12, 0xffff0000;\n\tmov.b64 v, {lo, hi};\n\t"
-        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 c, wv, v, c;\n\tmov.b64 {%6, %7}, c;\n\t}"
-        : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]), "+f"(a[7])
-        : "f"(w), "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w));
+// Per-shape kernel options (bit flags of the OPT template parameter), chosen by
+// measurement for each hot shape:
+constexpr int kOptWB = 1;   // bf16 softmax weights, two edges per mixed-precision FMA word
+constexpr int kOptL1 = 2;   // gathers allocate in L1 (hub rows are re-read by nearby rows)
+constexpr int kOptEF = 4;   // q rows and L rows (each touched once) marked evict-first in L2,
+                            // so the gathered k_j | v_j rows keep more of it
+
+// a 16-byte load / store whose L2 lines are the first to go
+__device__ __forceinline__ uint4 ld_evict_first(const void *p) {
+    uint4 r;
+    asm volatile("{\n\t.reg .b64 pol;\n\t"
+                 "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+                 "ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], pol;\n\t}"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st_evict_first(void *p, const uint4 &v) {
+    asm volatile("{\n\t.reg .b64 pol;\n\t"
+                 "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+                 "st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, pol;\n\t}"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // volatile: the load must stay under its guard (it is never speculated)
+template <bool L1>
 __device__ __forceinline__ uint4 ld_gather(const void *p) {
     uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
+    if constexpr (L1)
+        asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+            : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+            : "l"(p));
+    else
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+            : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+            : "l"(p));
     return r;
 }
 
@@ -314,7 +326,7 @@ constexpr int col_batch() {
 // k_j / v_j gathers of step i + 1 are issued before step i is consumed (two register
 // buffers), so a warp keeps a step's loads in flight while it computes the previous one.
 // On return each lane holds its slot's partial state for its feature vectors.
-template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE, bool CB>
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE, bool CB, int OPT>
 __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q)[VPL], int64_t e0,
                                            int64_t e1, int32_t cols, const Lane &ln,
                                            State<T, VPL, J> &st) {
@@ -369,8 +381,8 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
 #pragma unroll
                 for (int v = 0; v < VPL; ++v) {
                     if (ok[v]) {
-                        kb[u][v] = ld_gather(rowp + Sh::voff(v));
-                        vb[u][v] = ld_gather(rowp + 16 * nvec + Sh::voff(v));
+                        kb[u][v] = ld_gather<(OPT & kOptL1) != 0>(rowp + Sh::voff(v));
+                        vb[u][v] = ld_gather<(OPT & kOptL1) != 0>(rowp + 16 * nvec + Sh::voff(v));
                     }
                 }
             }
@@ -422,6 +434,42 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
                         for (int e = 0; e < VE; ++e) st.acc[v][e] *= corr;
             }
         }
+        if constexpr (sizeof(T) == 2 && (OPT & kOptWB) != 0) {
+            // weights rounded to bf16 (as attention kernels round P before the P V
+            // product), two edges per 32-bit word on the mixed-precision FMA; l sums
+            // exactly the rounded weights, so each row's weights still sum to one
+            constexpr uint32_t kOne = 0x3f803f80u;
+#pragma unroll
+            for (int u = 0; u < U; u += 2) {
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const float p0 = exp2_ftz(fmaf(sc[u][h], scale, -st.m[h]));
+                    const float p1 = u + 1 < U ? exp2_ftz(fmaf(sc[u + 1][h], scale, -st.m[h])) : 0.f;
+                    const uint32_t w = pack_bf16x2(p0, p1);
+                    st.l[h] = mfma<0, 0>(w, kOne, st.l[h]);
+                    if (u + 1 < U) st.l[h] = mfma<1, 0>(w, kOne, st.l[h]);
+#pragma unroll
+                    for (int v = 0; v < VPL; ++v) {
+                        if (St::head_of(v) != h) continue;
+                        const uint32_t a[4] = {vb[u][v].x, vb[u][v].y, vb[u][v].z, vb[u][v].w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            st.acc[v][2 * i] = mfma<0, 0>(w, a[i], st.acc[v][2 * i]);
+                            st.acc[v][2 * i + 1] = mfma<0, 1>(w, a[i], st.acc[v][2 * i + 1]);
+                        }
+                        if (u + 1 < U) {
+                            const uint32_t b[4] = {vb[u + 1][v].x, vb[u + 1][v].y, vb[u + 1][v].z, vb[u + 1][v].w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                st.acc[v][2 * i] = mfma<1, 0>(w, b[i], st.acc[v][2 * i]);
+                                st.acc[v][2 * i + 1] = mfma<1, 1>(w, b[i], st.acc[v][2 * i + 1]);
+                            }
+                        }
+                    }
+                }
+            }
+            return;
+        }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             float pr[NH];
@@ -433,12 +481,6 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
                 const float w = pr[St::head_of(v)];
-#ifdef GLGA_LOCAL_FMA2
-                if constexpr (sizeof(T) == 2) {
-                    acc_bf16x8_f32x2(st.acc[v], w, vb[u][v]);
-                    continue;
-                }
-#endif
                 float vf[VE];
                 Io<T>::unpack(vb[u][v], vf);
 #pragma unroll
@@ -498,15 +540,19 @@ __device__ __forceinline__ void merge_slots(const LocalParams &p, State<T, VPL, 
     }
 }
 
-template <typename T, int NV, int LPH, int VPL, bool J>
+template <typename T, int NV, int LPH, int VPL, bool J, int OPT>
 __device__ __forceinline__ void load_q(const LocalParams &p, int64_t row, const Lane &ln, bool valid,
                                        uint4 (&qr)[VPL]) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
     const char *Q = static_cast<const char *>(p.Q) + row * 16 * Sh::nvec(p) + 16 * Sh::vid(0, ln.li);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v)
-        qr[v] = (valid && Sh::lane_ok(p, v, ln.li)) ? __ldg(reinterpret_cast<const uint4 *>(Q + Sh::voff(v)))
-                                                    : make_uint4(0, 0, 0, 0);
+    for (int v = 0; v < VPL; ++v) {
+        const bool on = valid && Sh::lane_ok(p, v, ln.li);
+        if constexpr ((OPT & kOptEF) != 0)
+            qr[v] = on ? ld_evict_first(Q + Sh::voff(v)) : make_uint4(0, 0, 0, 0);
+        else
+            qr[v] = on ? __ldg(reinterpret_cast<const uint4 *>(Q + Sh::voff(v))) : make_uint4(0, 0, 0, 0);
+    }
 }
 
 // lse_i = ln sum_j exp(s_ij) per head, ln 2 (m + log2 l) since the state keeps base-2
@@ -530,7 +576,7 @@ __device__ __forceinline__ void store_lse(const LocalParams &p, int64_t row, con
 }
 
 // L_i = acc / l per head (0 for a row without edges), stored from lanes with `mine`.
-template <typename T, int NV, int LPH, int VPL, bool J, bool LSE>
+template <typename T, int NV, int LPH, int VPL, bool J, bool LSE, int OPT>
 __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, const State<T, VPL, J> &st,
                                            const Lane &ln, bool mine) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
@@ -545,7 +591,12 @@ __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, co
         float y[VE];
 #pragma unroll
         for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l[State<T, VPL, J>::head_of(v)];
-        if (mine && Sh::lane_ok(p, v, ln.li)) *reinterpret_cast<uint4 *>(Lout + Sh::voff(v)) = Io<T>::pack(y);
+        if (mine && Sh::lane_ok(p, v, ln.li)) {
+            if constexpr ((OPT & kOptEF) != 0)
+                st_evict_first(Lout + Sh::voff(v), Io<T>::pack(y));
+            else
+                *reinterpret_cast<uint4 *>(Lout + Sh::voff(v)) = Io<T>::pack(y);
+        }
     }
     store_lse<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, mine);
 }
@@ -561,7 +612,7 @@ struct BlockScratch {
 
 // 8 warps split [e0, e1) (each warp's share split again across its slots); warp 0
 // returns the merge of all warps in warp order.
-template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE, bool CB>
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool PIPE, bool CB, int OPT>
 __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&q)[VPL], int64_t e0,
                                             int64_t e1, const Lane &ln, int warp,
                                             BlockScratch<T, VPL, J> &sh, State<T, VPL, J> &st) {
@@ -572,7 +623,7 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&
     const int64_t a = std::min(e1, e0 + warp * per), b = std::min(e1, a + per);
     const int64_t per_s = ceil_div(b - a, Sh::epw(p));
     const int64_t sa = std::min(b, a + ln.slot * per_s), sb = std::min(b, sa + per_s);
-    slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, sa, sb,
+    slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB, OPT>(p, q, sa, sb,
                                                first_cols<col_batch<T, NV, LPH, VPL, U, J, CB>(), DBG>(p, sa, sb, ln),
                                                ln, st);
     merge_slots<T, NV, LPH, VPL, J>(p, st);
@@ -606,13 +657,10 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&
 // Blocks per SM the register budget aims at: 3 (at most 85 registers) while the gather
 // buffers take at most 32 registers (8 per edge step and vector, doubled when pipelined),
 // else 2.
-#ifndef GLGA_LOCAL_MINB3
-#define GLGA_LOCAL_MINB3 3
-#endif
 constexpr int local_min_blocks(int VPL, int U, bool PIPE) {
-    return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? GLGA_LOCAL_MINB3 : 2;
+    return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? 3 : 2;
 }
-template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE, bool CB>
+template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE, bool CB, int OPT>
 __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
     local_kernel(const LocalParams p) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
@@ -639,8 +687,8 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
         const int64_t e1 = std::min<int64_t>(re, e0 + p.chunk_edges);
         const int64_t nch = ceil_div(re - rb, p.chunk_edges);
         const int64_t first = c - (e0 - rb) / p.chunk_edges;
-        load_q<T, NV, LPH, VPL, J>(p, row, ln, true, q);
-        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, e0, e1, ln, warp, sh, st);
+        load_q<T, NV, LPH, VPL, J, OPT>(p, row, ln, true, q);
+        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB, OPT>(p, q, e0, e1, ln, warp, sh, st);
         const int64_t stride = 2 * p.H + p.D;
         if (warp == 0) {
             float *dst = p.part + c * stride;
@@ -686,7 +734,7 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
                     }
                     st.merge(m2, l2, a2);
                 }
-                finish_row<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, ln.slot == 0);
+                finish_row<T, NV, LPH, VPL, J, LSE, OPT>(p, row, st, ln, ln.slot == 0);
             }
         }
         return;
@@ -696,9 +744,9 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
         // ---------------- bucket-1 row: one block ----------------
         const int64_t row = p.cta_rows[bid];
         if (!row_ok<DBG>(p, row)) return;
-        load_q<T, NV, LPH, VPL, J>(p, row, ln, true, q);
-        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
-        if (warp == 0) finish_row<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, ln.slot == 0);
+        load_q<T, NV, LPH, VPL, J, OPT>(p, row, ln, true, q);
+        block_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB, OPT>(p, q, p.row_ptr[row], p.row_ptr[row + 1], ln, warp, sh, st);
+        if (warp == 0) finish_row<T, NV, LPH, VPL, J, LSE, OPT>(p, row, st, ln, ln.slot == 0);
         return;
     }
     bid -= p.n_cta;
@@ -726,7 +774,7 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
     int32_t end = __shfl_sync(0xffffffffu, myend, k & 31);
     if (k >= n) beg = end = 0;
     uint4 qn[VPL];
-    load_q<T, NV, LPH, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qn);
+    load_q<T, NV, LPH, VPL, J, OPT>(p, row, ln, k < n && (!DBG || row >= 0), qn);
     int32_t cols = first_cols<col_batch<T, NV, LPH, VPL, U, J, CB>(), DBG>(p, beg, end, ln);
     for (int step = 0; step < steps; ++step) {
         const bool valid = k < n;
@@ -741,15 +789,15 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
         beg = __shfl_sync(0xffffffffu, mybeg, k & 31);
         end = __shfl_sync(0xffffffffu, myend, k & 31);
         if (k >= n) beg = end = 0;
-        load_q<T, NV, LPH, VPL, J>(p, row, ln, k < n && (!DBG || row >= 0), qn);
+        load_q<T, NV, LPH, VPL, J, OPT>(p, row, ln, k < n && (!DBG || row >= 0), qn);
         cols = first_cols<col_batch<T, NV, LPH, VPL, U, J, CB>(), DBG>(p, beg, end, ln);
-        slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB>(p, q, beg_c, end_c, cols_c, ln, st);
+        slot_edges<T, NV, LPH, VPL, U, DBG, J, PIPE, CB, OPT>(p, q, beg_c, end_c, cols_c, ln, st);
         // every slot finishes its own row
-        if (valid && (!DBG || row_c >= 0)) finish_row<T, NV, LPH, VPL, J, LSE>(p, row_c, st, ln, true);
+        if (valid && (!DBG || row_c >= 0)) finish_row<T, NV, LPH, VPL, J, LSE, OPT>(p, row_c, st, ln, true);
     }
 }
 
-template <typename T, int NV, int LPH, int VPL, int U, bool J, bool PIPE = false, bool CB = false>
+template <typename T, int NV, int LPH, int VPL, int U, bool J, bool PIPE = false, bool CB = false, int OPT = 0>
 glga_status launch_local(Ctx *c, LocalParams p, cudaStream_t s) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
     if constexpr (NV != 0) {
@@ -762,11 +810,11 @@ glga_status launch_local(Ctx *c, LocalParams p, cudaStream_t s) {
     if (blocks == 0) return GLGA_OK;
     const unsigned g = static_cast<unsigned>(blocks);
     if (c->opts.debug_checks) {
-        if (p.lse) local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
+        if (p.lse) local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
     } else {
-        if (p.lse) local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE, CB><<<g, kLocalThreads, 0, s>>>(p);
+        if (p.lse) local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
+        else local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
     }
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
@@ -863,15 +911,9 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
         // step, 3 blocks per SM); at D = 512 two consecutive vectors of one head per lane,
         // the next step's gathers issued before the current one is consumed, column
         // indices in batches
-#if defined(GLGA_LOCAL_X128)
-        if (p.nvec == 16 && c->r == 32) {
-            if (GLGA_LOCAL_X128 == 1) return launch_local<B, 16, 4, 1, 2, false>(c, p, s);
-            if (GLGA_LOCAL_X128 == 2) return launch_local<B, 16, 4, 1, 8, false>(c, p, s);
-            return launch_local<B, 16, 4, 1, 4, false>(c, p, s);
-        }
-#endif
-        if (p.nvec == 16 && c->r == 32) return launch_local<B, 16, 4, 1, 4, false>(c, p, s);
-        if (p.nvec == 32 && c->r == 32) return launch_local<B, 32, 4, 1, 4, false>(c, p, s);
+        // (D = 128: bf16 weights; D = 256: L1-allocating gathers)
+        if (p.nvec == 16 && c->r == 32) return launch_local<B, 16, 4, 1, 4, false, false, false, kOptWB>(c, p, s);
+        if (p.nvec == 32 && c->r == 32) return launch_local<B, 32, 4, 1, 4, false, false, false, kOptL1>(c, p, s);
         if (p.nvec == 64 && c->r == 64) return launch_local<B, 64, 4, 2, 2, true, true, true>(c, p, s);
         if (p.nvec == 64 && c->r >= 16) return launch_local<B, 64, 0, 2, 2, true, false>(c, p, s);
         if (vpl == 1 && lpe >= 4) return launch_local<B, 0, 0, 1, 4, false, false>(c, p, s);

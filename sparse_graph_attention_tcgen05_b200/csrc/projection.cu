@@ -83,7 +83,6 @@ __device__ __forceinline__ void tile_at(const GemmParams &p, int32_t i, int32_t 
     }
 }
 
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 template <typename T>
 __device__ __forceinline__ void store_vec32(T *dst, const uint32_t (&v)[32]);
@@ -437,13 +436,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
                         const int chunk = ((half * 4 + q) ^ (rt & 7)) * 16;
                         *reinterpret_cast<uint4 *>(rp + chunk) = make_uint4(w[0], w[1], w[2], w[3]);
                         if (kwarp) {
-                            // phi of the stored (bf16) k; rows past M contribute nothing to z
+                            // phi of the stored (bf16) k, as the statistics kernel forms it;
+                            // rows past M contribute nothing to z
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float a = valid ? phi_elu1(__uint_as_float(w[e] << 16)) : 0.f;
-                                const float b2 = valid ? phi_elu1(__uint_as_float(w[e] & 0xffff0000u)) : 0.f;
-                                w[e] = pack_bf16x2(a, b2);
-                            }
+                            for (int e = 0; e < 4; ++e) w[e] = valid ? phi_bf16x2(w[e]) : 0u;
                             *reinterpret_cast<uint4 *>(fp + chunk) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }

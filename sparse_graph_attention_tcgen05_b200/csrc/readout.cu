@@ -111,16 +111,8 @@ __device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __exp
 
 // phi applied in place to one 16-byte chunk of the q tile (bf16: 8 values).
 __device__ __forceinline__ void phi_chunk_bf16(uint4 *p) {
-    uint4 u = *p;
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float a = phi(__uint_as_float(w[k] << 16));
-        const float b = phi(__uint_as_float(w[k] & 0xffff0000u));
-        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-        w[k] = *reinterpret_cast<uint32_t *>(&h);
-    }
-    *p = make_uint4(w[0], w[1], w[2], w[3]);
+    const uint4 u = *p;
+    *p = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
 }
 
 // fp32: phi, then split into tf32 hi (in place) and lo (same offset in the lo plane).
