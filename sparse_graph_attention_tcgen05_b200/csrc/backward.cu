@@ -481,6 +481,82 @@ __global__ void __launch_bounds__(256) bwd_local_q_kernel(
     }
 }
 
+// Light target rows with two edges per step (the layout of bwd_local_kv2_kernel): the
+// warp's 16-lane halves take alternate edges of the row, lane hl of a half holding the
+// EPL2 = 2 EPL features hl*EPL2 .. hl*EPL2+EPL2-1 of q_i, dL_i and of the gathered k_j,
+// v_j, so a step's two edges share one shuffle butterfly and one exponential per lane.
+// The halves' dq are added (the same sum in both), moved to the 32-lane layout and added
+// into dZ [:, 0:D].  Needs 2 EPL <= r.
+template <typename T, int EPL>
+__global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
+    const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
+    const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
+    const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
+    constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
+    const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
+    const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (w >= n_rows) return;                              // warp-uniform
+    const int64_t i = rows[w];
+    const int32_t a = row_ptr[i], b = row_ptr[i + 1];
+    if (a == b) return;                                   // no local term
+    const int D = H * R;
+    const bool act2 = hl * EPL2 < D;
+    const int lph2 = R / EPL2, h2 = act2 ? hl * EPL2 / R : 0;
+    float q2[EPL2], dl2[EPL2], dq2[EPL2];
+    ld_row<T, EPL2>(Q + i * D, hl, act2, q2);
+    ld_row<float, EPL2>(dL + i * D, hl, act2, dl2);
+    const float ls = __ldg(lse + i * H + h2), dd = __ldg(Dd + i * H + h2);
+#pragma unroll
+    for (int x = 0; x < EPL2; ++x) dq2[x] = 0.f;
+    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {          // the same trip count in both halves
+        float k[kU][EPL2], v[kU][EPL2];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int32_t e = e0 + 2 * u + slot;
+            const bool live = e < b;
+            const T *row = KV + (live ? static_cast<int64_t>(col_idx[e]) : 0) * 2 * D;
+            ld_row<T, EPL2>(row, hl, act2 && live, k[u]);
+            ld_row<T, EPL2>(row + D, hl, act2 && live, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            float sc = 0.f, dp = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) {
+                sc = fmaf(q2[x], k[u][x], sc);
+                dp = fmaf(dl2[x], v[u][x], dp);
+            }
+            sc = head_reduce(sc, lph2);
+            dp = head_reduce(dp, lph2);
+            const bool live = e0 + 2 * u + slot < b;
+            const float ds = live ? __expf(sc * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) dq2[x] = fmaf(ds, k[u][x], dq2[x]);
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < EPL2; ++x) dq2[x] += __shfl_xor_sync(0xffffffffu, dq2[x], 16);
+    // to the 32-lane layout: lane l's features l*EPL .. are half-lane l/2's, part l % 2
+    const LaneHead lh(lane, EPL, D, R);
+    const int src = lane >> 1;
+    const bool hi = lane & 1;
+    float dq[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; ++x) {
+        const float q0 = __shfl_sync(0xffffffffu, dq2[x], src), q1 = __shfl_sync(0xffffffffu, dq2[EPL + x], src);
+        dq[x] = hi ? q1 : q0;
+    }
+    if (lh.act) {
+        float *o = dZ + i * dz_ld + lane * EPL;
+        float cur[EPL];
+        ld_mrow<EPL, false>(o, cur);
+#pragma unroll
+        for (int x = 0; x < EPL; ++x) cur[x] += dq[x];
+        st_mrow<EPL>(o, cur);
+    }
+}
+
 // Chunks of heavy target rows, one warp each: chunk c covers the edges
 // [chunks[c].y, min(chunks[c].y + kChunk, row end)) of row chunks[c].x, and writes its
 // share of dq_i into part[c][0:D].
@@ -1105,6 +1181,21 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
         nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
 }
 
+// Light target rows: two edges per warp step under the same condition as the source side.
+template <typename T, int E>
+void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cudaStream_t sq) {
+    const int64_t nql = c->bw_nq_light;
+    if constexpr (E <= 4) {
+        if (2 * E <= c->r) {
+            bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
+                Q, KV, c->bw_dL, c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
+            return;
+        }
+    }
+    bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx, Q, KV,
+        c->bw_dL, c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
+}
+
 // Both local backward kernels with EPL = lane_features(D): light rows one warp each;
 // heavy rows (more than kHeavyDegree entries) as kChunk-edge chunks, one warp each, whose
 // shares the per-row kernels merge in chunk order.  The target-side (dq) kernels go to
@@ -1130,9 +1221,7 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
                 kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr, c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse,  \
                 c->bw_Dd, c->bw_dSc, c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                 \
         }                                                                                                 \
-        if (nql)                                                                                          \
-            bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr,        \
-                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);               \
+        if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                            \
         if (nqh) {                                                                                        \
             bwd_q_chunk_kernel<T, E><<<warp_grid(nqc), 256, 0, sq>>>(c->bw_q_chunks, nqc, c->row_ptr,      \
                 c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);               \

@@ -291,16 +291,22 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
     return ok != 0;
 }
 
+// Suspend-time hint of one poll (ns): the thread may sleep up to this long unless the
+// phase completes first.
+#ifndef GLGA_MBAR_SUSPEND_NS
+#define GLGA_MBAR_SUSPEND_NS 1000000u
+#endif
+
 // Waits for the phase with the given parity to complete.  Each poll may suspend the
-// thread for up to 1 ms; gives up after about `limit_ns` nanoseconds of wall time or
-// 2^26 polls, whichever comes first, and returns false; the caller records the timeout
-// and winds down.
+// thread for up to GLGA_MBAR_SUSPEND_NS (1 ms); gives up after about `limit_ns`
+// nanoseconds of wall time or 2^26 polls, whichever comes first, and returns false; the
+// caller records the timeout and winds down.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns = 1000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1; it < (1u << 26); ++it) {
-        if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
+        if (mbar_try_wait_suspend(bar, parity, GLGA_MBAR_SUSPEND_NS)) return true;
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;

@@ -141,38 +141,29 @@ struct Io<__nv_bfloat16> {
 // Per-shape kernel options (bit flags of the OPT template parameter), chosen by
 // measurement for each hot shape:
 constexpr int kOptWB = 1;   // bf16 softmax weights, two edges per mixed-precision FMA word
-constexpr int kOptL1 = 2;   // gathers allocate in L1 (hub rows are re-read by nearby rows)
-constexpr int kOptEF = 4;   // q rows and L rows (each touched once) marked evict-first in L2,
-                            // so the gathered k_j | v_j rows keep more of it
+constexpr int kOptAsync = 2;   // gathers by cp.async into a two-step shared-memory ring per
+                               // warp: the next step's loads wait in shared memory, not in
+                               // registers, while the current step is computed
 
-// a 16-byte load / store whose L2 lines are the first to go
-__device__ __forceinline__ uint4 ld_evict_first(const void *p) {
-    uint4 r;
-    asm volatile("{\n\t.reg .b64 pol;\n\t"
-                 "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
-                 "ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], pol;\n\t}"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-    return r;
+constexpr int kRingSteps = 2;
+// Dynamic shared memory of the cp.async ring: [warp][step % 2][U][VPL][k | v][lane] x 16 B.
+constexpr size_t async_ring_bytes(int U, int VPL) {
+    return static_cast<size_t>(kLocalWarps) * kRingSteps * U * VPL * 2 * 32 * 16;
 }
-__device__ __forceinline__ void st_evict_first(void *p, const uint4 &v) {
-    asm volatile("{\n\t.reg .b64 pol;\n\t"
-                 "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
-                 "st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, pol;\n\t}"
-                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // volatile: the load must stay under its guard (it is never speculated)
-template <bool L1>
 __device__ __forceinline__ uint4 ld_gather(const void *p) {
     uint4 r;
-    if constexpr (L1)
-        asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-            : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-            : "l"(p));
-    else
-        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-            : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-            : "l"(p));
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
     return r;
 }
 
@@ -360,7 +351,8 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
     }
     // issues the gathers of step `step` into (kb, vb); jb gets its column indices (-1:
     // no edge; such a slot keeps its previous, finite contents and gets weight 0)
-    auto load = [&](int step, uint4 (&kb)[U][VPL], uint4 (&vb)[U][VPL], int32_t (&jb)[U]) {
+    // the column indices of step `step` (taken in step order)
+    auto cols_of = [&](int step, int32_t (&jb)[U]) {
         const int sub = PER > 1 ? step % PER : 0;
 #pragma unroll
         for (int u = 0; u < U; ++u) jb[u] = __shfl_sync(0xffffffffu, c_cur, src0 + sub * U + u);
@@ -374,6 +366,9 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
                 c_cur = (ln.li < U && nb + ln.li < e1) ? checked_col<DBG>(p, __ldg(p.col_idx + nb + ln.li)) : -1;
             }
         }
+    };
+    auto load = [&](int step, uint4 (&kb)[U][VPL], uint4 (&vb)[U][VPL], int32_t (&jb)[U]) {
+        cols_of(step, jb);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (jb[u] >= 0) {
@@ -381,8 +376,8 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
 #pragma unroll
                 for (int v = 0; v < VPL; ++v) {
                     if (ok[v]) {
-                        kb[u][v] = ld_gather<(OPT & kOptL1) != 0>(rowp + Sh::voff(v));
-                        vb[u][v] = ld_gather<(OPT & kOptL1) != 0>(rowp + 16 * nvec + Sh::voff(v));
+                        kb[u][v] = ld_gather(rowp + Sh::voff(v));
+                        vb[u][v] = ld_gather(rowp + 16 * nvec + Sh::voff(v));
                     }
                 }
             }
@@ -494,7 +489,57 @@ __device__ __forceinline__ void slot_edges(const LocalParams &p, const uint4 (&q
     for (int u = 0; u < U; ++u)
 #pragma unroll
         for (int v = 0; v < VPL; ++v) kA[u][v] = vA[u][v] = make_uint4(0, 0, 0, 0);
-    if constexpr (!PIPE) {
+    if constexpr ((OPT & kOptAsync) != 0 && !PIPE) {
+        // this lane's slots of the warp's ring (written and read by the lane alone, so the
+        // lane's own cp.async.wait_group makes them visible; never-written slots hold
+        // zeros or an earlier edge's finite values and get weight 0)
+        constexpr int S = kRingSteps;
+        extern __shared__ uint4 local_ring[];
+        uint4 *ring = local_ring + (threadIdx.x >> 5) * (S * U * VPL * 2 * 32) + ln.lane;
+        auto slot = [&](int stage, int u, int v, int kv) { return ring + (((stage * U + u) * VPL + v) * 2 + kv) * 32; };
+        auto issue = [&](int step, int32_t (&jb)[U]) {
+            cols_of(step, jb);
+            const int stage = step % S;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (jb[u] >= 0) {
+                    const char *rowp = kvl + static_cast<size_t>(static_cast<uint32_t>(jb[u])) * row_bytes;
+#pragma unroll
+                    for (int v = 0; v < VPL; ++v) {
+                        if (ok[v]) {
+                            cp_async16(slot(stage, u, v, 0), rowp + Sh::voff(v));
+                            cp_async16(slot(stage, u, v, 1), rowp + 16 * nvec + Sh::voff(v));
+                        }
+                    }
+                }
+            }
+            cp_async_commit();
+        };
+        // step it + 1's gathers are issued before step it is waited for and consumed
+        int32_t jN[U];
+        if (iters > 0) issue(0, jA);
+        for (int it = 0; it < iters; ++it) {
+            if (it + 1 < iters) {
+                issue(it + 1, jN);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            const int stage = it % S;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    kA[u][v] = *slot(stage, u, v, 0);
+                    vA[u][v] = *slot(stage, u, v, 1);
+                }
+            consume(kA, vA, jA);
+            if (it + 1 < iters) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) jA[u] = jN[u];
+            }
+        }
+    } else if constexpr (!PIPE) {
         for (int it = 0; it < iters; ++it) {
             load(it, kA, vA, jA);
             consume(kA, vA, jA);
@@ -546,13 +591,9 @@ __device__ __forceinline__ void load_q(const LocalParams &p, int64_t row, const 
     using Sh = Shape<T, NV, LPH, VPL, J>;
     const char *Q = static_cast<const char *>(p.Q) + row * 16 * Sh::nvec(p) + 16 * Sh::vid(0, ln.li);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-        const bool on = valid && Sh::lane_ok(p, v, ln.li);
-        if constexpr ((OPT & kOptEF) != 0)
-            qr[v] = on ? ld_evict_first(Q + Sh::voff(v)) : make_uint4(0, 0, 0, 0);
-        else
-            qr[v] = on ? __ldg(reinterpret_cast<const uint4 *>(Q + Sh::voff(v))) : make_uint4(0, 0, 0, 0);
-    }
+    for (int v = 0; v < VPL; ++v)
+        qr[v] = (valid && Sh::lane_ok(p, v, ln.li)) ? __ldg(reinterpret_cast<const uint4 *>(Q + Sh::voff(v)))
+                                                    : make_uint4(0, 0, 0, 0);
 }
 
 // lse_i = ln sum_j exp(s_ij) per head, ln 2 (m + log2 l) since the state keeps base-2
@@ -591,12 +632,7 @@ __device__ __forceinline__ void finish_row(const LocalParams &p, int64_t row, co
         float y[VE];
 #pragma unroll
         for (int e = 0; e < VE; ++e) y[e] = st.acc[v][e] * inv_l[State<T, VPL, J>::head_of(v)];
-        if (mine && Sh::lane_ok(p, v, ln.li)) {
-            if constexpr ((OPT & kOptEF) != 0)
-                st_evict_first(Lout + Sh::voff(v), Io<T>::pack(y));
-            else
-                *reinterpret_cast<uint4 *>(Lout + Sh::voff(v)) = Io<T>::pack(y);
-        }
+        if (mine && Sh::lane_ok(p, v, ln.li)) *reinterpret_cast<uint4 *>(Lout + Sh::voff(v)) = Io<T>::pack(y);
     }
     store_lse<T, NV, LPH, VPL, J, LSE>(p, row, st, ln, mine);
 }
@@ -673,6 +709,14 @@ __global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
     ln.lane = threadIdx.x & 31;
     ln.slot = ln.lane / Sh::lpe(p);
     ln.li = ln.lane % Sh::lpe(p);
+    if constexpr ((OPT & kOptAsync) != 0) {
+        // the gather ring starts at zero (slots of masked edges are read with weight 0)
+        extern __shared__ uint4 local_ring[];
+        constexpr int S = kRingSteps;
+        uint4 *ring = local_ring + warp * (S * U * VPL * 2 * 32) + ln.lane;
+#pragma unroll
+        for (int k = 0; k < S * U * VPL * 2; ++k) ring[k * 32] = make_uint4(0u, 0u, 0u, 0u);
+    }
     int64_t bid = blockIdx.x;
     uint4 q[VPL];
     St st;
@@ -809,13 +853,21 @@ glga_status launch_local(Ctx *c, LocalParams p, cudaStream_t s) {
     const int64_t blocks = p.n_chunks + p.n_cta + p.task_blocks;
     if (blocks == 0) return GLGA_OK;
     const unsigned g = static_cast<unsigned>(blocks);
+    const size_t dyn = (OPT & kOptAsync) != 0 ? async_ring_bytes(U, VPL) : 0;
+    auto go = [&](auto kern) -> glga_status {
+        if (dyn > 0) GLGA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn)));
+        kern<<<g, kLocalThreads, dyn, s>>>(p);
+        return GLGA_OK;
+    };
+    glga_status st;
     if (c->opts.debug_checks) {
-        if (p.lse) local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
+        st = p.lse ? go(local_kernel<T, NV, LPH, VPL, U, true, J, true, PIPE, CB, OPT>)
+                   : go(local_kernel<T, NV, LPH, VPL, U, true, J, false, PIPE, CB, OPT>);
     } else {
-        if (p.lse) local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
-        else local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE, CB, OPT><<<g, kLocalThreads, 0, s>>>(p);
+        st = p.lse ? go(local_kernel<T, NV, LPH, VPL, U, false, J, true, PIPE, CB, OPT>)
+                   : go(local_kernel<T, NV, LPH, VPL, U, false, J, false, PIPE, CB, OPT>);
     }
+    if (st != GLGA_OK) return st;
     GLGA_CUDA(cudaGetLastError());
     c->launches += 1;
     return GLGA_OK;
@@ -907,13 +959,14 @@ glga_status local_run(Ctx *c, cudaStream_t s) {
     if (c->io == GLGA_BF16) {
         using B = __nv_bfloat16;
         // hot shapes with compile-time layouts, chosen by measurement: a lane's vector
-        // interleaved across the row (D = 128 and 256: one vector per lane, 4 edges per
-        // step, 3 blocks per SM); at D = 512 two consecutive vectors of one head per lane,
+        // interleaved across the row (D = 128 and 256: one vector per lane, 2 edges per
+        // step, 64 registers); at D = 512 two consecutive vectors of one head per lane,
         // the next step's gathers issued before the current one is consumed, column
         // indices in batches
-        // (D = 128: bf16 weights; D = 256: L1-allocating gathers)
-        if (p.nvec == 16 && c->r == 32) return launch_local<B, 16, 4, 1, 4, false, false, false, kOptWB>(c, p, s);
-        if (p.nvec == 32 && c->r == 32) return launch_local<B, 32, 4, 1, 4, false, false, false, kOptL1>(c, p, s);
+        // (D = 128 and 256: gathers through the cp.async ring, 2 edges per slot step;
+        // D = 128 also with bf16 weights)
+        if (p.nvec == 16 && c->r == 32) return launch_local<B, 16, 4, 1, 2, false, false, false, kOptWB | kOptAsync>(c, p, s);
+        if (p.nvec == 32 && c->r == 32) return launch_local<B, 32, 4, 1, 2, false, false, false, kOptAsync>(c, p, s);
         if (p.nvec == 64 && c->r == 64) return launch_local<B, 64, 4, 2, 2, true, true, true>(c, p, s);
         if (p.nvec == 64 && c->r >= 16) return launch_local<B, 64, 0, 2, 2, true, false>(c, p, s);
         if (vpl == 1 && lpe >= 4) return launch_local<B, 0, 0, 1, 4, false, false>(c, p, s);
