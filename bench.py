@@ -849,7 +849,7 @@ def run_single(args, rank, world, local_rank, mode):
     if args.block:
         line["block"] = time_block(layer, w, X, Y, dt, dev, flush, stream, 200, peaks)
     if args.backward:
-        line["backward"] = time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, 50)
+        line["backward"] = time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, args.backward_steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, (row_ptr.cpu().numpy(), col_idx.cpu().numpy()))
     if rank == 0:
@@ -876,6 +876,8 @@ def main():
     ap.add_argument("--segment-len", type=int, default=0,
                     help="segments of this many nodes, each with its own global statistics "
                          "(a batch of graphs; 0 = one segment over all nodes)")
+    ap.add_argument("--backward-steps", type=int, default=50,
+                    help="timed glga_backward calls (and as many graph replays) with --backward")
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward pass (glga_backward) of the same forward")
     ap.add_argument("--block", action="store_true",
