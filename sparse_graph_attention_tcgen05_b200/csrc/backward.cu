@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(256, EPL <= 8 ? 2 : 1) bwd_readout_kernel(
     if (i0 >= N) return;                                  // warp-uniform
     const int D = H * R;
     const LaneHead lh(lane, EPL, D, R);
+    const int lph = LPH > 0 ? LPH : lh.lph;              // lanes per head (a constant when known)
     const float *S = Sz + static_cast<int64_t>(lh.h) * R * R;
     float q[RPW][EPL], dy[RPW][EPL], lv[RPW][EPL], ph[RPW][EPL], zz[EPL];
     bool live[RPW];
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(256, EPL <= 8 ? 2 : 1) bwd_readout_kernel(
             den[k] = fmaf(ph[k][x], zz[x], den[k]);
             G[k][x] = 0.f;
         }
-        den[k] = head_reduce(den[k], lh.lph) + eps;
+        den[k] = head_reduce(den[k], lph) + eps;
     }
     head_matvec<EPL, LPH, RPW>(S, R, lh.f0, lh.hb, lh.lph, ph, G);  // num_f = sum_a phi(q_a) S[a][f]
     float dn[RPW][EPL], acc[RPW][EPL], dgp[RPW], gk[RPW];
@@ -238,25 +239,26 @@ __global__ void __launch_bounds__(256, EPL <= 8 ? 2 : 1) bwd_readout_kernel(
         const float g = live[k] ? 1.f / (1.f + __expf(-(t[i] + b_g))) : 0.f;
         gk[k] = g;
         float dGG = 0.f, dLL = 0.f, gl[EPL];
+        const float inv_den = 1.f / den[k];              // one division per row and head
         dgp[k] = 0.f;
 #pragma unroll
         for (int x = 0; x < EPL; ++x) {
-            G[k][x] /= den[k];
+            G[k][x] *= inv_den;
             dLL = fmaf(g * dy[k][x], lv[k][x], dLL);
             dgp[k] = fmaf(dy[k][x], lv[k][x] - G[k][x], dgp[k]);
             const float dG = (1.f - g) * dy[k][x];
             dGG = fmaf(dG, G[k][x], dGG);
             gl[x] = g * dy[k][x];
-            dn[k][x] = dG / den[k];
+            dn[k][x] = dG * inv_den;
         }
         const int64_t o = i * D + lane * EPL;
         if (lh.act && live[k]) {
             st_mrow<EPL>(dL + o, gl);
             st_mrow<EPL>(dnum + o, dn[k]);
         }
-        const float dd = -head_reduce(dGG, lh.lph) / den[k];
-        dLL = head_reduce(dLL, lh.lph);
-        if (lh.act && live[k] && (lane % lh.lph) == 0) {
+        const float dd = -head_reduce(dGG, lph) * inv_den;
+        dLL = head_reduce(dLL, lph);
+        if (lh.act && live[k] && (lane % lph) == 0) {
             dden[i * H + lh.h] = dd;
             Dd[i * H + lh.h] = dLL;
         }
@@ -481,6 +483,12 @@ __global__ void __launch_bounds__(256) bwd_local_q_kernel(
     }
 }
 
+// bf16 rows with 4 features per lane (8 per half-lane: one 16-byte slice) go through a
+// shared-memory ring of cp.async gathers in bwd_local_q2_kernel.
+template <typename T, int EPL>
+constexpr bool kQRing = sizeof(T) == 2 && EPL == 4;
+constexpr size_t kQRingBytes = 8 * 2 * 2 * 2 * 32 * 16;   // 8 warps x 2 steps x kU x (k, v) x 32 lanes
+
 // Light target rows with two edges per step (the layout of bwd_local_kv2_kernel): the
 // warp's 16-lane halves take alternate edges of the row, lane hl of a half holding the
 // EPL2 = 2 EPL features hl*EPL2 .. hl*EPL2+EPL2-1 of q_i, dL_i and of the gathered k_j,
@@ -509,16 +517,16 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     const float ls = __ldg(lse + i * H + h2), dd = __ldg(Dd + i * H + h2);
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dq2[x] = 0.f;
-    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {          // the same trip count in both halves
-        float k[kU][EPL2], v[kU][EPL2];
+    if constexpr (kQRing<T, EPL>) {
+        // never-written cells (edges past the row's end) are read with ds = 0: keep them finite
+        extern __shared__ uint4 q_ring[];
+        uint4 *ring = q_ring + (threadIdx.x >> 5) * (2 * kU * 2 * 32) + lane;
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int32_t e = e0 + 2 * u + slot;
-            const bool live = e < b;
-            const T *row = KV + (live ? static_cast<int64_t>(col_idx[e]) : 0) * 2 * D;
-            ld_row<T, EPL2>(row, hl, act2 && live, k[u]);
-            ld_row<T, EPL2>(row + D, hl, act2 && live, v[u]);
-        }
+        for (int c = 0; c < 2 * kU * 2; ++c) ring[c * 32] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // the edges of step it (kU per half); the gathers of step it + 1 wait in this warp's
+    // two-step shared-memory ring (bf16 rows of 8 features per lane) while step it is used
+    auto use_step = [&](int32_t e0, const float (&k)[kU][EPL2], const float (&v)[kU][EPL2]) {
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             float sc = 0.f, dp = 0.f;
@@ -533,6 +541,56 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
             const float ds = live ? __expf(sc * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
 #pragma unroll
             for (int x = 0; x < EPL2; ++x) dq2[x] = fmaf(ds, k[u][x], dq2[x]);
+        }
+    };
+    if constexpr (kQRing<T, EPL>) {
+        extern __shared__ uint4 q_ring[];
+        uint4 *ring = q_ring + (threadIdx.x >> 5) * (2 * kU * 2 * 32) + lane;
+        auto cell = [&](int st, int u, int kv) { return ring + ((st * kU + u) * 2 + kv) * 32; };
+        auto issue = [&](int32_t e0, int st) {
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int32_t e = e0 + 2 * u + slot;
+                if (e < b && act2) {
+                    const T *row = KV + static_cast<int64_t>(col_idx[e]) * 2 * D + hl * EPL2;
+                    cp_async16(cell(st, u, 0), row);
+                    cp_async16(cell(st, u, 1), row + D);
+                }
+            }
+            cp_async_commit();
+        };
+        const int n_steps = (b - a + 2 * kU - 1) / (2 * kU);
+        issue(a, 0);
+        for (int it = 0; it < n_steps; ++it) {
+            const int32_t e0 = a + it * 2 * kU;
+            if (it + 1 < n_steps) {
+                issue(e0 + 2 * kU, (it + 1) & 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            float k[kU][EPL2], v[kU][EPL2];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const uint4 kw = *cell(it & 1, u, 0), vw = *cell(it & 1, u, 1);
+                const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, vv[4] = {vw.x, vw.y, vw.z, vw.w};
+                unpack_bf16<EPL2>(kk, k[u]);
+                unpack_bf16<EPL2>(vv, v[u]);
+            }
+            use_step(e0, k, v);
+        }
+    } else {
+        for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {      // the same trip count in both halves
+            float k[kU][EPL2], v[kU][EPL2];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int32_t e = e0 + 2 * u + slot;
+                const bool live = e < b;
+                const T *row = KV + (live ? static_cast<int64_t>(col_idx[e]) : 0) * 2 * D;
+                ld_row<T, EPL2>(row, hl, act2 && live, k[u]);
+                ld_row<T, EPL2>(row + D, hl, act2 && live, v[u]);
+            }
+            use_step(e0, k, v);
         }
     }
 #pragma unroll
@@ -1187,7 +1245,10 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
     const int64_t nql = c->bw_nq_light;
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
-            bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
+            if (kQRing<T, E> && kQRingBytes > 48 * 1024)
+                cudaFuncSetAttribute(bwd_local_q2_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kQRingBytes));
+            bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
                 Q, KV, c->bw_dL, c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
             return;
         }

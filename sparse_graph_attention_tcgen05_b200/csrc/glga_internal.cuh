@@ -520,6 +520,15 @@ __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
     return y;
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), its group commit and the wait for
+// all but the N most recent groups of this thread.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Round-to-nearest (ties away) conversion of an f32 to tf32, kept in an f32 container.
 __device__ __forceinline__ float to_tf32(float x) {
     uint32_t u;

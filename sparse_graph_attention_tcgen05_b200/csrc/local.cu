@@ -151,12 +151,6 @@ constexpr size_t async_ring_bytes(int U, int VPL) {
     return static_cast<size_t>(kLocalWarps) * kRingSteps * U * VPL * 2 * 32 * 16;
 }
 
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // volatile: the load must stay under its guard (it is never speculated)
 __device__ __forceinline__ uint4 ld_gather(const void *p) {
