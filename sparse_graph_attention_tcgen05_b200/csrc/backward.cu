@@ -877,18 +877,8 @@ __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dk2[x] = dv2[x] = 0.f;
     const int32_t a = t_row_ptr[j], b = t_row_ptr[j + 1];
-    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {          // the same trip count in both halves
-        float q[kU][EPL2], dl[kU][EPL2], ls[kU], dd[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int32_t e = e0 + 2 * u + slot;
-            const bool live = e < b;
-            const int64_t i = live ? t_col[e] : 0;
-            ld_row<T, EPL2>(Q + i * D, hl, act2 && live, q[u]);
-            ld_row<float, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
-            ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
-            dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
-        }
+    auto use_step = [&](int32_t e0, const float (&q)[kU][EPL2], const float (&dl)[kU][EPL2], const float (&ls)[kU],
+                        const float (&dd)[kU]) {
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             float sc = 0.f, dp = 0.f;
@@ -908,6 +898,20 @@ __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
                 dk2[x] = fmaf(ds, q[u][x], dk2[x]);
             }
         }
+    };
+    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {      // the same trip count in both halves
+        float q[kU][EPL2], dl[kU][EPL2], ls[kU], dd[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int32_t e = e0 + 2 * u + slot;
+            const bool live = e < b;
+            const int64_t i = live ? t_col[e] : 0;
+            ld_row<T, EPL2>(Q + i * D, hl, act2 && live, q[u]);
+            ld_row<float, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
+            ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
+            dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
+        }
+        use_step(e0, q, dl, ls, dd);
     }
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) {
@@ -1301,6 +1305,247 @@ int local_bwd_launches(const Ctx *c) {
     return (c->bw_nq_light > 0) + 2 * (c->bw_nq_heavy > 0) + (c->bw_nk_light > 0) + 2 * (c->bw_nk_heavy > 0);
 }
 
+// ---------------------------------------------------------------------------------------
+// Readout backward on the tensor cores (bf16 layers, H*r = 128, r <= 64, one head group):
+// per 128-row tile,
+//   [num | den] = phi(Q) B_g            (tcgen05, B_g = the forward's readout operand)
+//   epilogue:  G, dL = g dY, dnum = (1-g) dY / den, dden = -(dG . G)/den, D_i, dt
+//   dphi = dnum blockdiag(S_h)          (tcgen05, A = dnum rounded to bf16)
+//   dq_global = (dphi + z dden) phi'(q)
+// One thread per tile row and column half (8 warps: warp w reads TMEM lanes 32 (w % 4)
+// and columns 64 (w / 4) ..): per-head sums stay in the thread.  Operands are written
+// to shared memory in the 128-byte-swizzled K-major layout the MMA reads.
+constexpr int kBroTcD = 128;
+constexpr int kBroTcBN = kBroTcD + 16;            // num | den (H <= 8) | zero columns
+constexpr uint32_t kBroTcAtom = 128 * 128;        // one 64-column atom of a 128-row operand
+constexpr uint32_t kBroTcB1Atom = kBroTcBN * 128; // one 64-column atom of B_g (144 rows)
+constexpr size_t kBroTcSmem = 1024 + 2 * kBroTcAtom + 2 * kBroTcB1Atom + 2 * kBroTcAtom + kBroTcD * 4 + 2 * 128 * 4;
+
+// byte offset of element (row, k) of a K-major operand with 64-element atoms of `rows` rows
+__device__ __forceinline__ uint32_t swz_off(int row, int k, uint32_t atom_bytes) {
+    return static_cast<uint32_t>(k >> 6) * atom_bytes + static_cast<uint32_t>(row) * 128u +
+           ((static_cast<uint32_t>((k & 63) >> 3) ^ static_cast<uint32_t>(row & 7)) << 4) +
+           static_cast<uint32_t>(k & 7) * 2u;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+template <int R>
+__global__ void __launch_bounds__(256, 2) bwd_readout_tc_kernel(
+    const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ L, const float *__restrict__ t,
+    const __nv_bfloat16 *__restrict__ Bg, int ro_kp, const float *__restrict__ Sz,
+    const __nv_bfloat16 *__restrict__ dY, int64_t N, int H, float b_g, float eps, float *__restrict__ dL,
+    float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ,
+    int64_t dz_ld, unsigned *flag) {
+    constexpr int D = kBroTcD;
+    constexpr int kHH = 64 / R;                   // heads in a 64-column half
+    extern __shared__ uint8_t bro_raw[];
+    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ uint32_t tmem_sh;
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(bro_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sA = sm;                              // phi(Q), then dnum: 2 atoms
+    uint8_t *sB1 = sA + 2 * kBroTcAtom;            // B_g: 2 atoms of 144 rows
+    uint8_t *sB2 = sB1 + 2 * kBroTcB1Atom;         // blockdiag(S_h): 2 atoms
+    float *zf = reinterpret_cast<float *>(sB2 + 2 * kBroTcAtom);
+    float *dtx = zf + D;                           // [2][128] dt partials of the two halves
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int rt = quad * 32 + lane;               // row in the tile
+    const float *S = Sz;
+    const float *z = Sz + static_cast<int64_t>(H) * R * R;
+
+    // operands that stay for the whole launch: B_g, blockdiag(S_h), z
+    for (int ch = tid; ch < kBroTcBN * (D / 8); ch += blockDim.x) {
+        const int n = ch / (D / 8), k8 = (ch % (D / 8)) * 8;
+        const uint4 v = *reinterpret_cast<const uint4 *>(Bg + static_cast<int64_t>(n) * ro_kp + k8);
+        *reinterpret_cast<uint4 *>(sB1 + swz_off(n, k8, kBroTcB1Atom)) = v;
+    }
+    for (int ch = tid; ch < D * (D / 8); ch += blockDim.x) {
+        const int f = ch / (D / 8), c8 = (ch % (D / 8)) * 8;
+        const int h = f / R;
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int c = c8 + e;
+            v[e] = (c / R == h) ? S[(static_cast<int64_t>(h) * R + (f - h * R)) * R + (c - h * R)] : 0.f;
+        }
+        *reinterpret_cast<uint4 *>(sB2 + swz_off(f, c8, kBroTcAtom)) =
+            make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]), bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
+    }
+    for (int f = tid; f < D; f += blockDim.x) zf[f] = z[f];
+    if (tid == 0) {
+        mbar_init(&mma_bar, 1);
+        fence_mbar_init();
+    }
+    fence_proxy_async_smem();
+    if (warp == 0) {
+        tmem_alloc(&tmem_sh, 256u);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_sh;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t idesc1 = instr_desc(128, kBroTcBN, 1u, false, false);
+    const uint32_t idesc2 = instr_desc(128, D, 1u, false, false);
+    const int64_t n_tiles = ceil_div(N, 128);
+    uint32_t phase = 0;
+    // the tile's MMAs: 8 K steps of 16 over the two atoms of A and B, one thread
+    auto mma = [&](const uint8_t *sb, uint32_t b_atom, uint32_t idesc) {
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sb);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t ko = static_cast<uint32_t>(ks >> 2), kb = static_cast<uint32_t>(ks & 3) * 32u;
+                umma_bf16(tmem, smem_desc(a0 + ko * kBroTcAtom + kb, 16, 1024, 2),
+                          smem_desc(b0 + ko * b_atom + kb, 16, 1024, 2), idesc, ks != 0);
+            }
+            umma_commit(&mma_bar);
+        }
+    };
+    // every thread waits; the block leaves together if any wait gave up
+    auto wait_mma = [&]() -> bool {
+        const bool got = mbar_wait_bounded(&mma_bar, phase);
+        phase ^= 1u;
+        const bool bad = __syncthreads_or(!got) != 0;
+        if (bad && tid == 0) atomicOr(flag, kDevErrTimeout);
+        tc_fence_after();
+        return !bad;
+    };
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int64_t row = tile * 128 + rt;
+        const bool valid = row < N;
+        const __nv_bfloat16 *qrow = Q + row * D + half * 64;
+        // ---- A = phi(q) for this thread's 64 columns (zero past N) ----
+#pragma unroll
+        for (int k8 = 0; k8 < 64; k8 += 8) {
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (valid) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(qrow + k8);
+                w = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
+            }
+            *reinterpret_cast<uint4 *>(sA + swz_off(rt, half * 64 + k8, kBroTcAtom)) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        mma(sB1, kBroTcB1Atom, idesc1);
+        if (!wait_mma()) break;
+        // ---- epilogue 1 ----
+        uint32_t dv[8];
+        tmem_ld_n<4>(tmem + lane_base + D, *reinterpret_cast<uint32_t (*)[4]>(&dv[0]));
+        tmem_ld_n<4>(tmem + lane_base + D + 4, *reinterpret_cast<uint32_t (*)[4]>(&dv[4]));
+        tmem_ld_wait();
+        const float g = valid ? 1.f / (1.f + __expf(-(t[row] + b_g))) : 0.f;
+        float inv[kHH], dda[kHH], Dda[kHH];
+#pragma unroll
+        for (int hh = 0; hh < kHH; ++hh) {
+            const int h = half * kHH + hh;
+            inv[hh] = 1.f / (__uint_as_float(dv[h < 8 ? h : 0]) + eps);
+            dda[hh] = 0.f;
+            Dda[hh] = 0.f;
+        }
+        float dtp = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c0 = half * 64 + cc * 32;
+            uint32_t nv[32];
+            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), nv);
+            tmem_ld_wait();
+            uint4 yw[4], lw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                yw[i] = valid ? *reinterpret_cast<const uint4 *>(dY + row * D + c0 + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
+                lw[i] = valid ? *reinterpret_cast<const uint4 *>(L + row * D + c0 + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float dlv[32], dnv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const uint32_t yword = (&yw[j / 8].x)[(j % 8) / 2], lword = (&lw[j / 8].x)[(j % 8) / 2];
+                const float y = __uint_as_float((j & 1) ? (yword & 0xffff0000u) : (yword << 16));
+                const float lv = __uint_as_float((j & 1) ? (lword & 0xffff0000u) : (lword << 16));
+                const int hh = (cc * 32 + j) / R;
+                const float G = __uint_as_float(nv[j]) * inv[hh];
+                const float dG = (1.f - g) * y;
+                dlv[j] = g * y;
+                dnv[j] = dG * inv[hh];
+                dda[hh] = fmaf(dG, G, dda[hh]);
+                Dda[hh] = fmaf(dlv[j], lv, Dda[hh]);
+                dtp = fmaf(y, lv - G, dtp);
+            }
+            if (valid) {
+                float4 *o1 = reinterpret_cast<float4 *>(dL + row * D + c0);
+                float4 *o2 = reinterpret_cast<float4 *>(dnum + row * D + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    o1[i] = make_float4(dlv[4 * i], dlv[4 * i + 1], dlv[4 * i + 2], dlv[4 * i + 3]);
+                    o2[i] = make_float4(dnv[4 * i], dnv[4 * i + 1], dnv[4 * i + 2], dnv[4 * i + 3]);
+                }
+            }
+            // A = dnum in bf16 (phi(q) has been read by the first MMA)
+#pragma unroll
+            for (int k8 = 0; k8 < 32; k8 += 8)
+                *reinterpret_cast<uint4 *>(sA + swz_off(rt, c0 + k8, kBroTcAtom)) =
+                    make_uint4(bf16x2_bits(dnv[k8], dnv[k8 + 1]), bf16x2_bits(dnv[k8 + 2], dnv[k8 + 3]),
+                               bf16x2_bits(dnv[k8 + 4], dnv[k8 + 5]), bf16x2_bits(dnv[k8 + 6], dnv[k8 + 7]));
+        }
+        float ddh[kHH];
+#pragma unroll
+        for (int hh = 0; hh < kHH; ++hh) {
+            const int h = half * kHH + hh;
+            ddh[hh] = -dda[hh] * inv[hh];
+            if (valid) {
+                dden[row * H + h] = ddh[hh];
+                Dd[row * H + h] = Dda[hh];
+            }
+        }
+        dtx[half * 128 + rt] = dtp;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        mma(sB2, kBroTcAtom, idesc2);
+        if (half == 0 && valid) dZ[row * dz_ld + 3 * D] = g * (1.f - g) * (dtx[rt] + dtx[128 + rt]);
+        if (!wait_mma()) break;
+        // ---- epilogue 2: dq_global = (dphi + z dden) phi'(q) ----
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c0 = half * 64 + cc * 32;
+            uint32_t av[32];
+            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), av);
+            tmem_ld_wait();
+            if (valid) {
+                uint4 qw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) qw[i] = *reinterpret_cast<const uint4 *>(Q + row * D + c0 + 8 * i);
+                float out[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t qword = (&qw[j / 8].x)[(j % 8) / 2];
+                    const float q = __uint_as_float((j & 1) ? (qword & 0xffff0000u) : (qword << 16));
+                    const int hh = (cc * 32 + j) / R;
+                    out[j] = fmaf(zf[c0 + j], ddh[hh], __uint_as_float(av[j])) * dphi(q);
+                }
+                float4 *o = reinterpret_cast<float4 *>(dZ + row * dz_ld + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();   // TMEM and the A operand are rewritten by the next tile
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256u);
+    }
+}
+
 // Two rows per warp for up to 4 features per lane (one above that); the head loop
 // unrolled for the lane layout of H*r = 128 with r = 32.
 template <typename T, int EPL, int LPH>
@@ -1312,8 +1557,30 @@ void launch_readout_bwd_e(Ctx *c, const T *Q, const T *dY, float b_g, float eps,
                                                                c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz);
 }
 
+template <int R>
+void launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *dY, float b_g, float eps, int64_t Dz,
+                           cudaStream_t s) {
+    const int64_t tiles = ceil_div(c->N, 128);
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * c->num_sms));
+    cudaFuncSetAttribute(bwd_readout_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kBroTcSmem));
+    bwd_readout_tc_kernel<R><<<grid, 256, kBroTcSmem, s>>>(
+        Q, static_cast<const __nv_bfloat16 *>(c->L), c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz,
+        dY, c->N, c->H, b_g, eps, c->bw_dL, c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz, c->dev_flag);
+}
+
+// The readout backward runs on the tensor cores for bf16 layers with H*r = 128, r in
+// {16, 32, 64} and one head group (the forward's readout operand then holds every head);
+// elsewhere on the CUDA cores.
 template <typename T>
 void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
+    if constexpr (sizeof(T) == 2) {
+        if (c->D == kBroTcD && c->ro_groups == 1 && c->ro_kp == kBroTcD && c->ro_bn == kBroTcBN && c->n_seg == 1) {
+            if (c->r == 32) return launch_readout_bwd_tc<32>(c, Q, dY, b_g, eps, Dz, s);
+            if (c->r == 16) return launch_readout_bwd_tc<16>(c, Q, dY, b_g, eps, Dz, s);
+            if (c->r == 64) return launch_readout_bwd_tc<64>(c, Q, dY, b_g, eps, Dz, s);
+        }
+    }
     const int E = lane_features(c->D), lph = c->r / E;
     if (E == 4 && lph == 8) return launch_readout_bwd_e<T, 4, 8>(c, Q, dY, b_g, eps, Dz, s);
     switch (E) {

@@ -126,3 +126,16 @@ def test_bf16_rows_not_16_byte_multiples():
     src = rng.integers(0, N, dst.shape[0])
     w = make_custom(N, 13, 2, 16, src.astype(np.int32), dst.astype(np.int32), io="bf16", seed=23, b_g=0.4)
     _check(w, seed=24)
+
+
+@pytest.mark.parametrize("H,r,N", [(8, 16, 1000), (4, 32, 1000), (2, 64, 1000), (4, 32, 40000)])
+def test_tensor_core_readout_backward(H, r, N):
+    # bf16 layers with H*r = 128 run the readout backward on the tensor cores (one thread
+    # per tile row and column half, phi(Q) B_g and dnum blockdiag(S) as tcgen05 MMAs): every
+    # head width it takes, a ragged last 128-row tile, and at N = 40,000 more tiles than
+    # CTAs (the persistent loop)
+    rng = np.random.default_rng(N + r)
+    src = np.concatenate([rng.integers(0, N, 4 * N), np.arange(N)]).astype(np.int32)
+    dst = np.concatenate([np.repeat(np.arange(N), 4), np.arange(N)]).astype(np.int32)
+    w = make_custom(N, 64, H, r, src, dst, io="bf16", seed=N * 3 + H, b_g=0.2)
+    _check(w, seed=H, chunked=N > 5000)
