@@ -1312,14 +1312,20 @@ int local_bwd_launches(const Ctx *c) {
 //   epilogue:  G, dL = g dY, dnum = (1-g) dY / den, dden = -(dG . G)/den, D_i, dt
 //   dphi = dnum blockdiag(S_h)          (tcgen05, A = dnum rounded to bf16)
 //   dq_global = (dphi + z dden) phi'(q)
-// One thread per tile row and column half (8 warps: warp w reads TMEM lanes 32 (w % 4)
-// and columns 64 (w / 4) ..): per-head sums stay in the thread.  Operands are written
-// to shared memory in the 128-byte-swizzled K-major layout the MMA reads.
+// 16 warps, one CTA per SM: warp w reads TMEM lanes 32 (w % 4) (its 32 tile rows) and
+// owns columns 32 (w / 4) .. +31, one thread per row.  Row data moves between global
+// memory and the threads through a 4 KB staging area per warp with coalesced warp-wide
+// copies (bf16 inputs: 8 rows x 64 B per instruction; float32 outputs: 4 rows x 128 B),
+// swizzled so the threads' 16-byte row accesses are free of bank conflicts.  Per-head
+// and per-row sums that span column quarters meet in shared memory.
 constexpr int kBroTcD = 128;
 constexpr int kBroTcBN = kBroTcD + 16;            // num | den (H <= 8) | zero columns
+constexpr int kBroTcWarps = 16;
 constexpr uint32_t kBroTcAtom = 128 * 128;        // one 64-column atom of a 128-row operand
 constexpr uint32_t kBroTcB1Atom = kBroTcBN * 128; // one 64-column atom of B_g (144 rows)
-constexpr size_t kBroTcSmem = 1024 + 2 * kBroTcAtom + 2 * kBroTcB1Atom + 2 * kBroTcAtom + kBroTcD * 4 + 2 * 128 * 4;
+constexpr uint32_t kBroTcStage = 4096;            // staging bytes per warp
+constexpr size_t kBroTcSmem = 1024 + 2 * kBroTcAtom + 2 * kBroTcB1Atom + 2 * kBroTcAtom +
+                              kBroTcWarps * kBroTcStage + (kBroTcD + 3 * 4 * 128) * 4;
 
 // byte offset of element (row, k) of a K-major operand with 64-element atoms of `rows` rows
 __device__ __forceinline__ uint32_t swz_off(int row, int k, uint32_t atom_bytes) {
@@ -1333,15 +1339,56 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// The warp's 32 rows x 32 bf16 columns (64 B per row) of a row-major [N][ld] bf16 matrix,
+// starting at global row r0 and column c0, into the lane's registers (lane = row): four
+// coalesced loads of 8 rows x 64 B through the staging area (row r at byte r * 64, its
+// 16-byte piece p at slot p ^ ((r >> 1) & 3)).  Rows at or past N read as zero.
+__device__ __forceinline__ void warp_rows_bf16(const __nv_bfloat16 *src, int64_t ld, int64_t r0, int64_t N, int c0,
+                                               uint8_t *stage, int lane, uint4 (&out)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 8 * i + (lane >> 2), p = lane & 3;
+        const int64_t gr = r0 + r;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (gr < N) v = __ldg(reinterpret_cast<const uint4 *>(src + gr * ld + c0) + p);
+        *reinterpret_cast<uint4 *>(stage + r * 64 + ((p ^ ((r >> 1) & 3)) << 4)) = v;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        out[p] = *reinterpret_cast<const uint4 *>(stage + lane * 64 + ((p ^ ((lane >> 1) & 3)) << 4));
+    __syncwarp();
+}
+
+// The lane's 32 floats (its row, columns c0 .. c0 + 31) to a row-major float32 matrix:
+// each 4-float piece p into the staging area (row r at byte r * 128, piece p at slot
+// p ^ (r & 7)) as it is computed, then eight coalesced stores of 4 rows x 128 B.  Rows at
+// or past N are not written.
+__device__ __forceinline__ void stage_f32_piece(uint8_t *stage, int lane, int p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4 *>(stage + lane * 128 + ((p ^ (lane & 7)) << 4)) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void warp_rows_f32_flush(float *dst, int64_t ld, int64_t r0, int64_t N, int c0,
+                                                    uint8_t *stage, int lane) {
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + (lane >> 3), p = lane & 7;
+        const int64_t gr = r0 + r;
+        const float4 x = *reinterpret_cast<const float4 *>(stage + r * 128 + ((p ^ (r & 7)) << 4));
+        if (gr < N) reinterpret_cast<float4 *>(dst + gr * ld + c0)[p] = x;
+    }
+    __syncwarp();
+}
+
 template <int R>
-__global__ void __launch_bounds__(256, 2) bwd_readout_tc_kernel(
+__global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
     const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ L, const float *__restrict__ t,
     const __nv_bfloat16 *__restrict__ Bg, int ro_kp, const float *__restrict__ Sz,
     const __nv_bfloat16 *__restrict__ dY, int64_t N, int H, float b_g, float eps, float *__restrict__ dL,
     float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ,
     int64_t dz_ld, unsigned *flag) {
     constexpr int D = kBroTcD;
-    constexpr int kHH = 64 / R;                   // heads in a 64-column half
+    constexpr int kHQ = R >= 32 ? 1 : 32 / R;     // heads in a 32-column quarter
     extern __shared__ uint8_t bro_raw[];
     __shared__ __align__(8) uint64_t mma_bar;
     __shared__ uint32_t tmem_sh;
@@ -1349,12 +1396,16 @@ __global__ void __launch_bounds__(256, 2) bwd_readout_tc_kernel(
     uint8_t *sA = sm;                              // phi(Q), then dnum: 2 atoms
     uint8_t *sB1 = sA + 2 * kBroTcAtom;            // B_g: 2 atoms of 144 rows
     uint8_t *sB2 = sB1 + 2 * kBroTcB1Atom;         // blockdiag(S_h): 2 atoms
-    float *zf = reinterpret_cast<float *>(sB2 + 2 * kBroTcAtom);
-    float *dtx = zf + D;                           // [2][128] dt partials of the two halves
+    uint8_t *stg_all = sB2 + 2 * kBroTcAtom;       // staging, kBroTcStage per warp
+    float *zf = reinterpret_cast<float *>(stg_all + kBroTcWarps * kBroTcStage);
+    float *xdt = zf + D;                           // [4 quarters][128 rows] dt partials
+    float *xdd = xdt + 4 * 128;                    // ... (dG . G) partials (r = 64: a head spans 2)
+    float *xDd = xdd + 4 * 128;                    // ... (dL . L) partials
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, cq = warp >> 2;     // TMEM lane quarter, column quarter
     const int rt = quad * 32 + lane;               // row in the tile
-    const float *S = Sz;
+    const int c0 = cq * 32;                        // first column of this warp
+    uint8_t *stg = stg_all + warp * kBroTcStage;
     const float *z = Sz + static_cast<int64_t>(H) * R * R;
 
     // operands that stay for the whole launch: B_g, blockdiag(S_h), z
@@ -1370,7 +1421,7 @@ __global__ void __launch_bounds__(256, 2) bwd_readout_tc_kernel(
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int c = c8 + e;
-            v[e] = (c / R == h) ? S[(static_cast<int64_t>(h) * R + (f - h * R)) * R + (c - h * R)] : 0.f;
+            v[e] = (c / R == h) ? Sz[(static_cast<int64_t>(h) * R + (f - h * R)) * R + (c - h * R)] : 0.f;
         }
         *reinterpret_cast<uint4 *>(sB2 + swz_off(f, c8, kBroTcAtom)) =
             make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]), bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
@@ -1417,19 +1468,22 @@ __global__ void __launch_bounds__(256, 2) bwd_readout_tc_kernel(
         tc_fence_after();
         return !bad;
     };
+    auto bf = [](const uint4 (&w)[4], int j) {
+        const uint32_t word = (&w[j / 8].x)[(j % 8) / 2];
+        return __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16));
+    };
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t row = tile * 128 + rt;
+        const int64_t m0 = tile * 128, r0 = m0 + quad * 32;
+        const int64_t row = m0 + rt;
         const bool valid = row < N;
-        const __nv_bfloat16 *qrow = Q + row * D + half * 64;
-        // ---- A = phi(q) for this thread's 64 columns (zero past N) ----
+        // ---- A = phi(q) for this warp's rows and 32 columns (zero past N) ----
+        {
+            uint4 qw[4];
+            warp_rows_bf16(Q, D, r0, N, c0, stg, lane, qw);
 #pragma unroll
-        for (int k8 = 0; k8 < 64; k8 += 8) {
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (valid) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(qrow + k8);
-                w = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
-            }
-            *reinterpret_cast<uint4 *>(sA + swz_off(rt, half * 64 + k8, kBroTcAtom)) = w;
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4 *>(sA + swz_off(rt, c0 + 8 * i, kBroTcAtom)) =
+                    make_uint4(phi_bf16x2(qw[i].x), phi_bf16x2(qw[i].y), phi_bf16x2(qw[i].z), phi_bf16x2(qw[i].w));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1441,102 +1495,112 @@ __global__ void __launch_bounds__(256, 2) bwd_readout_tc_kernel(
         tmem_ld_n<4>(tmem + lane_base + D, *reinterpret_cast<uint32_t (*)[4]>(&dv[0]));
         tmem_ld_n<4>(tmem + lane_base + D + 4, *reinterpret_cast<uint32_t (*)[4]>(&dv[4]));
         tmem_ld_wait();
-        const float g = valid ? 1.f / (1.f + __expf(-(t[row] + b_g))) : 0.f;
-        float inv[kHH], dda[kHH], Dda[kHH];
+        const float g = valid ? 1.f / (1.f + __expf(-(__ldg(t + row) + b_g))) : 0.f;
+        float inv[kHQ], dda[kHQ], Dda[kHQ];
 #pragma unroll
-        for (int hh = 0; hh < kHH; ++hh) {
-            const int h = half * kHH + hh;
-            inv[hh] = 1.f / (__uint_as_float(dv[h < 8 ? h : 0]) + eps);
-            dda[hh] = 0.f;
-            Dda[hh] = 0.f;
+        for (int hq = 0; hq < kHQ; ++hq) {
+            const int h = c0 / R + hq;
+            inv[hq] = 1.f / (__uint_as_float(dv[h < 8 ? h : 0]) + eps);
+            dda[hq] = 0.f;
+            Dda[hq] = 0.f;
         }
+        uint4 yw[4], lw[4];
+        warp_rows_bf16(dY, D, r0, N, c0, stg, lane, yw);
+        warp_rows_bf16(L, D, r0, N, c0, stg, lane, lw);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 4 * p + e, hq = j / R < kHQ ? j / R : 0;
+                v[e] = g * bf(yw, j);
+                Dda[hq] = fmaf(v[e], bf(lw, j), Dda[hq]);
+            }
+            stage_f32_piece(stg, lane, p, v[0], v[1], v[2], v[3]);
+        }
+        warp_rows_f32_flush(dL, D, r0, N, c0, stg, lane);
         float dtp = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c0 = half * 64 + cc * 32;
-            uint32_t nv[32];
-            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), nv);
+        for (int hb = 0; hb < 2; ++hb) {           // 16 columns at a time
+            uint32_t nv[16];
+            tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), nv);
             tmem_ld_wait();
-            uint4 yw[4], lw[4];
+            float dn[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                yw[i] = valid ? *reinterpret_cast<const uint4 *>(dY + row * D + c0 + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
-                lw[i] = valid ? *reinterpret_cast<const uint4 *>(L + row * D + c0 + 8 * i) : make_uint4(0u, 0u, 0u, 0u);
-            }
-            float dlv[32], dnv[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const uint32_t yword = (&yw[j / 8].x)[(j % 8) / 2], lword = (&lw[j / 8].x)[(j % 8) / 2];
-                const float y = __uint_as_float((j & 1) ? (yword & 0xffff0000u) : (yword << 16));
-                const float lv = __uint_as_float((j & 1) ? (lword & 0xffff0000u) : (lword << 16));
-                const int hh = (cc * 32 + j) / R;
-                const float G = __uint_as_float(nv[j]) * inv[hh];
+            for (int e = 0; e < 16; ++e) {
+                const int j = 16 * hb + e, hq = j / R < kHQ ? j / R : 0;
+                const float y = bf(yw, j);
+                const float G = __uint_as_float(nv[e]) * inv[hq];
                 const float dG = (1.f - g) * y;
-                dlv[j] = g * y;
-                dnv[j] = dG * inv[hh];
-                dda[hh] = fmaf(dG, G, dda[hh]);
-                Dda[hh] = fmaf(dlv[j], lv, Dda[hh]);
-                dtp = fmaf(y, lv - G, dtp);
+                dn[e] = dG * inv[hq];
+                dda[hq] = fmaf(dG, G, dda[hq]);
+                dtp = fmaf(y, bf(lw, j) - G, dtp);
             }
-            if (valid) {
-                float4 *o1 = reinterpret_cast<float4 *>(dL + row * D + c0);
-                float4 *o2 = reinterpret_cast<float4 *>(dnum + row * D + c0);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    o1[i] = make_float4(dlv[4 * i], dlv[4 * i + 1], dlv[4 * i + 2], dlv[4 * i + 3]);
-                    o2[i] = make_float4(dnv[4 * i], dnv[4 * i + 1], dnv[4 * i + 2], dnv[4 * i + 3]);
-                }
-            }
+            for (int p = 0; p < 4; ++p) stage_f32_piece(stg, lane, 4 * hb + p, dn[4 * p], dn[4 * p + 1], dn[4 * p + 2], dn[4 * p + 3]);
             // A = dnum in bf16 (phi(q) has been read by the first MMA)
 #pragma unroll
-            for (int k8 = 0; k8 < 32; k8 += 8)
-                *reinterpret_cast<uint4 *>(sA + swz_off(rt, c0 + k8, kBroTcAtom)) =
-                    make_uint4(bf16x2_bits(dnv[k8], dnv[k8 + 1]), bf16x2_bits(dnv[k8 + 2], dnv[k8 + 3]),
-                               bf16x2_bits(dnv[k8 + 4], dnv[k8 + 5]), bf16x2_bits(dnv[k8 + 6], dnv[k8 + 7]));
+            for (int i = 0; i < 2; ++i)
+                *reinterpret_cast<uint4 *>(sA + swz_off(rt, c0 + 16 * hb + 8 * i, kBroTcAtom)) =
+                    make_uint4(bf16x2_bits(dn[8 * i], dn[8 * i + 1]), bf16x2_bits(dn[8 * i + 2], dn[8 * i + 3]),
+                               bf16x2_bits(dn[8 * i + 4], dn[8 * i + 5]), bf16x2_bits(dn[8 * i + 6], dn[8 * i + 7]));
         }
-        float ddh[kHH];
-#pragma unroll
-        for (int hh = 0; hh < kHH; ++hh) {
-            const int h = half * kHH + hh;
-            ddh[hh] = -dda[hh] * inv[hh];
-            if (valid) {
-                dden[row * H + h] = ddh[hh];
-                Dd[row * H + h] = Dda[hh];
-            }
-        }
-        dtx[half * 128 + rt] = dtp;
+        warp_rows_f32_flush(dnum, D, r0, N, c0, stg, lane);
+        xdt[cq * 128 + rt] = dtp;
+        xdd[cq * 128 + rt] = dda[0];
+        xDd[cq * 128 + rt] = Dda[0];
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         mma(sB2, kBroTcAtom, idesc2);
-        if (half == 0 && valid) dZ[row * dz_ld + 3 * D] = g * (1.f - g) * (dtx[rt] + dtx[128 + rt]);
-        if (!wait_mma()) break;
-        // ---- epilogue 2: dq_global = (dphi + z dden) phi'(q) ----
+        // per-row and per-head sums across the column quarters; dden, D_i and dt out
+        float ddh[kHQ];
+        if constexpr (R == 64) {
+            const int q0 = cq & ~1;                // the head's two quarters
+            const float s_dd = xdd[q0 * 128 + rt] + xdd[(q0 + 1) * 128 + rt];
+            const float s_Dd = xDd[q0 * 128 + rt] + xDd[(q0 + 1) * 128 + rt];
+            ddh[0] = -s_dd * inv[0];
+            if (valid && (cq & 1) == 0) {
+                dden[row * H + c0 / R] = ddh[0];
+                Dd[row * H + c0 / R] = s_Dd;
+            }
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c0 = half * 64 + cc * 32;
-            uint32_t av[32];
-            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(c0), av);
-            tmem_ld_wait();
-            if (valid) {
-                uint4 qw[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) qw[i] = *reinterpret_cast<const uint4 *>(Q + row * D + c0 + 8 * i);
-                float out[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const uint32_t qword = (&qw[j / 8].x)[(j % 8) / 2];
-                    const float q = __uint_as_float((j & 1) ? (qword & 0xffff0000u) : (qword << 16));
-                    const int hh = (cc * 32 + j) / R;
-                    out[j] = fmaf(zf[c0 + j], ddh[hh], __uint_as_float(av[j])) * dphi(q);
+            for (int hq = 0; hq < kHQ; ++hq) {
+                ddh[hq] = -dda[hq] * inv[hq];
+                if (valid) {
+                    dden[row * H + c0 / R + hq] = ddh[hq];
+                    Dd[row * H + c0 / R + hq] = Dda[hq];
                 }
-                float4 *o = reinterpret_cast<float4 *>(dZ + row * dz_ld + c0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
             }
         }
+        if (cq == 0 && valid)
+            dZ[row * dz_ld + 3 * D] = g * (1.f - g) * (xdt[rt] + xdt[128 + rt] + xdt[256 + rt] + xdt[384 + rt]);
+        if (!wait_mma()) break;
+        // ---- epilogue 2: dq_global = (dphi + z dden) phi'(q) ----
+        {
+            uint4 qw[4];
+            warp_rows_bf16(Q, D, r0, N, c0, stg, lane, qw);
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                uint32_t av[16];
+                tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), av);
+                tmem_ld_wait();
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    float o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 16 * hb + 4 * p + e, hq = j / R < kHQ ? j / R : 0;
+                        o[e] = fmaf(zf[c0 + j], ddh[hq], __uint_as_float(av[4 * p + e])) * dphi(bf(qw, j));
+                    }
+                    stage_f32_piece(stg, lane, 4 * hb + p, o[0], o[1], o[2], o[3]);
+                }
+            }
+            warp_rows_f32_flush(dZ, dz_ld, r0, N, c0, stg, lane);
+        }
         tc_fence_before();
-        __syncthreads();   // TMEM and the A operand are rewritten by the next tile
+        __syncthreads();   // TMEM, the A operand and the cross-quarter sums are rewritten next tile
     }
     tc_fence_before();
     __syncthreads();
@@ -1561,10 +1625,10 @@ template <int R>
 void launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *dY, float b_g, float eps, int64_t Dz,
                            cudaStream_t s) {
     const int64_t tiles = ceil_div(c->N, 128);
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * c->num_sms));
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, c->num_sms));
     cudaFuncSetAttribute(bwd_readout_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kBroTcSmem));
-    bwd_readout_tc_kernel<R><<<grid, 256, kBroTcSmem, s>>>(
+    bwd_readout_tc_kernel<R><<<grid, kBroTcWarps * 32, kBroTcSmem, s>>>(
         Q, static_cast<const __nv_bfloat16 *>(c->L), c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz,
         dY, c->N, c->H, b_g, eps, c->bw_dL, c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz, c->dev_flag);
 }
