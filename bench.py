@@ -365,9 +365,9 @@ def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
     tg = float(np.mean(gms))
     return {"ms": t, "edge_heads_per_s": w.E * w.H / (t * 1e-3), "steps": steps,
             "graph_ms": tg, "graph_edge_heads_per_s": w.E * w.H / (tg * 1e-3),
-            "kernels": ("CUDA-core (SIMT) kernels, fp32 arithmetic"
-                        + ("; dW and dX as tcgen05 GEMMs (bf16 dW operands, tf32 dX operands)" if w.io == "bf16"
-                           else "; dW and dX as CUDA-core fp32 GEMMs"))}
+            "kernels": ("gathers and reductions on the CUDA cores (fp32 arithmetic)"
+                        + ("; readout backward (H*r = 128), dW and dX on the tcgen05 tensor cores"
+                           if w.io == "bf16" else "; dW and dX as CUDA-core fp32 GEMMs"))}
 
 
 def median_event_ms(fn, steps, warmup, flush):
