@@ -744,13 +744,31 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
 // The global terms of source row j and the store, in the 32-lane layout (every lane of
 // the warp takes part in the shuffles):
 //   dphi(k_j)_f = sum_c dS[f][c] v_c + dz_f,  dv_j,f += sum_c dS[c][f] phi(k_c)
-// (S = sum phi(k) v^T, z = sum phi(k)); dk, dv hold the local terms on entry.
+// (S = sum phi(k) v^T, z = sum phi(k)); dk, dv hold the local terms on entry.  With
+// dST == nullptr the global terms are already in dZ (bwd_kv_global_tc_kernel) and the
+// local terms are added to them.
 template <int EPL>
 __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t j, const float (&k)[EPL],
                                           const float (&v)[EPL], float (&dk)[EPL], float (&dv)[EPL],
                                           const float *dSc, const float *dST, int H, int R, float *dZ,
                                           int64_t dz_ld) {
     const int D = H * R;
+    if (dST == nullptr) {                         // warp-uniform
+        if (lh.act) {
+            float *pk = dZ + j * dz_ld + D + lane * EPL, *pv = pk + D;
+            float gk[EPL], gv[EPL];
+            ld_mrow<EPL, false>(pk, gk);
+            ld_mrow<EPL, false>(pv, gv);
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) {
+                dk[x] += gk[x];
+                dv[x] += gv[x];
+            }
+            st_mrow<EPL>(pk, dk);
+            st_mrow<EPL>(pv, dv);
+        }
+        return;
+    }
     float dphk[EPL], dvg[EPL], pk[EPL];
     ld_mrow<EPL>(dSc + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, dphk);
 #pragma unroll
@@ -1227,6 +1245,10 @@ unsigned warp_grid(int64_t n) {
     return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256)));
 }
 
+// The source side's dST argument: nullptr when bwd_kv_global_tc_kernel wrote the global
+// terms (defined with that kernel).
+const float *kv_dST(const Ctx *c);
+
 // Light source rows: two edges per warp step where a head spans at least two of the
 // 16-lane half's slices (2 EPL <= r, EPL <= 4), else one edge per step.
 template <typename T, int E>
@@ -1235,12 +1257,12 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, kv_dST(c), c->H, c->r, isr, c->bw_dZ, Dz);
             return;
         }
     }
     bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-        nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+        nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, kv_dST(c), c->H, c->r, isr, c->bw_dZ, Dz);
 }
 
 // Light target rows: two edges per warp step under the same condition as the source side.
@@ -1284,7 +1306,7 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
                                      static_cast<int>(kMW * 2 * D * 4));                                     \
             bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(nkh), kMW * 32, kMW * 2 * D * 4, sk>>>( \
                 kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr, c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse,  \
-                c->bw_Dd, c->bw_dSc, c->bw_dST, H, R, isr, c->bw_dZ, Dz);                                 \
+                c->bw_Dd, c->bw_dSc, kv_dST(c), H, R, isr, c->bw_dZ, Dz);                                 \
         }                                                                                                 \
         if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                            \
         if (nqh) {                                                                                        \
@@ -1608,6 +1630,173 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
         tc_fence_after();
         tmem_dealloc(tmem, 256u);
     }
+}
+
+// The source side's global terms on the tensor cores (bf16 layers, H*r = 128, r <= 64):
+// per 128-row tile of source rows j,
+//   G_k = V blockdiag(dS_h)^T       (tcgen05: dphi(k_j)_f = sum_c dS_h[f][c] v_jc)
+//   G_v = phi(K) blockdiag(dS_h)    (tcgen05: dv_jf = sum_c dS_h[c][f] phi(k_jc))
+//   dZ[j, D + f] = (G_k + dz_f) phi'(k_jf),   dZ[j, 2D + f] = G_v
+// written before the source-side gather kernels, which then add their local terms.
+// Layout and row I/O as bwd_readout_tc_kernel (16 warps, 32 rows x 32 columns each).
+constexpr size_t kKvgSmem = 1024 + 4 * 2 * kBroTcAtom + kBroTcWarps * kBroTcStage + kBroTcD * 4;
+
+template <int R>
+__global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
+    const __nv_bfloat16 *__restrict__ KV, const float *__restrict__ dSc, int64_t N, int H, float *__restrict__ dZ,
+    int64_t dz_ld, unsigned *flag) {
+    constexpr int D = kBroTcD;
+    extern __shared__ uint8_t kvg_raw[];
+    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ uint32_t tmem_sh;
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(kvg_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sV = sm;                              // A of the first MMA: V, 2 atoms
+    uint8_t *sP = sV + 2 * kBroTcAtom;             // A of the second: phi(K)
+    uint8_t *sB1 = sP + 2 * kBroTcAtom;            // blockdiag(dS_h)^T as [f][c] = dS_h[f][c]
+    uint8_t *sB2 = sB1 + 2 * kBroTcAtom;           // blockdiag(dS_h) as [f][c] = dS_h[c][f]
+    uint8_t *stg_all = sB2 + 2 * kBroTcAtom;
+    float *dzf = reinterpret_cast<float *>(stg_all + kBroTcWarps * kBroTcStage);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, cq = warp >> 2;
+    const int rt = quad * 32 + lane;
+    const int c0 = cq * 32;
+    uint8_t *stg = stg_all + warp * kBroTcStage;
+    const float *dz = dSc + static_cast<int64_t>(H) * R * R;
+    for (int ch = tid; ch < D * (D / 8); ch += blockDim.x) {
+        const int f = ch / (D / 8), c8 = (ch % (D / 8)) * 8;
+        const int h = f / R, fl = f - h * R;
+        float v1[8], v2[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int c = c8 + e, cl = c - h * R;
+            const bool in = c / R == h;
+            v1[e] = in ? dSc[(static_cast<int64_t>(h) * R + fl) * R + cl] : 0.f;
+            v2[e] = in ? dSc[(static_cast<int64_t>(h) * R + cl) * R + fl] : 0.f;
+        }
+        *reinterpret_cast<uint4 *>(sB1 + swz_off(f, c8, kBroTcAtom)) =
+            make_uint4(bf16x2_bits(v1[0], v1[1]), bf16x2_bits(v1[2], v1[3]), bf16x2_bits(v1[4], v1[5]), bf16x2_bits(v1[6], v1[7]));
+        *reinterpret_cast<uint4 *>(sB2 + swz_off(f, c8, kBroTcAtom)) =
+            make_uint4(bf16x2_bits(v2[0], v2[1]), bf16x2_bits(v2[2], v2[3]), bf16x2_bits(v2[4], v2[5]), bf16x2_bits(v2[6], v2[7]));
+    }
+    for (int f = tid; f < D; f += blockDim.x) dzf[f] = dz[f];
+    if (tid == 0) {
+        mbar_init(&mma_bar, 1);
+        fence_mbar_init();
+    }
+    fence_proxy_async_smem();
+    if (warp == 0) {
+        tmem_alloc(&tmem_sh, 256u);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_sh;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t idesc = instr_desc(128, D, 1u, false, false);
+    const int64_t n_tiles = ceil_div(N, 128);
+    uint32_t phase = 0;
+    auto bf = [](const uint4 (&w)[4], int j) {
+        const uint32_t word = (&w[j / 8].x)[(j % 8) / 2];
+        return __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16));
+    };
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int64_t r0 = tile * 128 + quad * 32;
+        {
+            uint4 kw[4], vw[4];
+            warp_rows_bf16(KV + D, 2 * D, r0, N, c0, stg, lane, vw);
+            warp_rows_bf16(KV, 2 * D, r0, N, c0, stg, lane, kw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                *reinterpret_cast<uint4 *>(sV + swz_off(rt, c0 + 8 * i, kBroTcAtom)) = vw[i];
+                *reinterpret_cast<uint4 *>(sP + swz_off(rt, c0 + 8 * i, kBroTcAtom)) =
+                    make_uint4(phi_bf16x2(kw[i].x), phi_bf16x2(kw[i].y), phi_bf16x2(kw[i].z), phi_bf16x2(kw[i].w));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t v0 = smem_u32(sV), p0 = smem_u32(sP), b10 = smem_u32(sB1), b20 = smem_u32(sB2);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t ko = static_cast<uint32_t>(ks >> 2) * kBroTcAtom, kb = static_cast<uint32_t>(ks & 3) * 32u;
+                umma_bf16(tmem, smem_desc(v0 + ko + kb, 16, 1024, 2), smem_desc(b10 + ko + kb, 16, 1024, 2), idesc, ks != 0);
+                umma_bf16(tmem + D, smem_desc(p0 + ko + kb, 16, 1024, 2), smem_desc(b20 + ko + kb, 16, 1024, 2), idesc,
+                          ks != 0);
+            }
+            umma_commit(&mma_bar);
+        }
+        const bool got = mbar_wait_bounded(&mma_bar, phase);
+        phase ^= 1u;
+        if (__syncthreads_or(!got)) {
+            if (tid == 0) atomicOr(flag, kDevErrTimeout);
+            break;
+        }
+        tc_fence_after();
+        // dk: (G_k + dz) phi'(k); dv: G_v
+        uint4 kw[4];
+        warp_rows_bf16(KV, 2 * D, r0, N, c0, stg, lane, kw);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+            uint32_t a[16];
+            tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), a);
+            tmem_ld_wait();
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                float o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 16 * hb + 4 * p + e;
+                    o[e] = (__uint_as_float(a[4 * p + e]) + dzf[c0 + j]) * dphi(bf(kw, j));
+                }
+                stage_f32_piece(stg, lane, 4 * hb + p, o[0], o[1], o[2], o[3]);
+            }
+        }
+        warp_rows_f32_flush(dZ + D, dz_ld, r0, N, c0, stg, lane);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+            uint32_t a[16];
+            tmem_ld16(tmem + lane_base + static_cast<uint32_t>(D + c0 + 16 * hb), a);
+            tmem_ld_wait();
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                stage_f32_piece(stg, lane, 4 * hb + p, __uint_as_float(a[4 * p]), __uint_as_float(a[4 * p + 1]),
+                                __uint_as_float(a[4 * p + 2]), __uint_as_float(a[4 * p + 3]));
+        }
+        warp_rows_f32_flush(dZ + 2 * D, dz_ld, r0, N, c0, stg, lane);
+        tc_fence_before();
+        __syncthreads();   // TMEM and the A operands are rewritten by the next tile
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256u);
+    }
+}
+
+// bf16 layers with H*r = 128 and r <= 64: the source side's global terms run on the tensor
+// cores before the gather kernels (which then get dST = nullptr and add to them).
+bool kv_global_tc(const Ctx *c) {
+    return c->io == GLGA_BF16 && c->D == kBroTcD && (c->r == 16 || c->r == 32 || c->r == 64);
+}
+const float *kv_dST(const Ctx *c) { return kv_global_tc(c) ? nullptr : c->bw_dST; }
+
+template <int R>
+void launch_kv_global_r(Ctx *c, int64_t Dz, cudaStream_t s) {
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(c->N, 128), c->num_sms));
+    cudaFuncSetAttribute(bwd_kv_global_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kKvgSmem));
+    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(
+        static_cast<const __nv_bfloat16 *>(c->KV), c->bw_dSc, c->N, c->H, c->bw_dZ, Dz, c->dev_flag);
+}
+void launch_kv_global(Ctx *c, int64_t Dz, cudaStream_t s) {
+    if (!kv_global_tc(c) || c->N == 0) return;
+    if (c->r == 32) return launch_kv_global_r<32>(c, Dz, s);
+    if (c->r == 16) return launch_kv_global_r<16>(c, Dz, s);
+    launch_kv_global_r<64>(c, Dz, s);
 }
 
 // Two rows per warp for up to 4 features per lane (one above that); the head loop
@@ -2079,6 +2268,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
                 c->bw_dsz_part, c->bw_parts, total, c->bw_dSz);                                           \
             bwd_heads_prep_kernel<<<tgrid, 256, 0, c->bw_side>>>(c->bw_dSz, R + 1, H, R, c->bw_dST,      \
                                                                 c->bw_dSc);                               \
+            launch_kv_global(c, Dz, c->bw_side);                                                          \
             launch_local_bwd<T>(c, Q, KV, isr, Dz, s, c->bw_side);                                        \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_join, c->bw_side));                                        \
             GLGA_CUDA(cudaStreamWaitEvent(s, c->bw_ev_join, 0));                                          \
