@@ -744,16 +744,16 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
 // The global terms of source row j and the store, in the 32-lane layout (every lane of
 // the warp takes part in the shuffles):
 //   dphi(k_j)_f = sum_c dS[f][c] v_c + dz_f,  dv_j,f += sum_c dS[c][f] phi(k_c)
-// (S = sum phi(k) v^T, z = sum phi(k)); dk, dv hold the local terms on entry.  With
-// dST == nullptr the global terms are already in dZ (bwd_kv_global_tc_kernel) and the
-// local terms are added to them.
-template <int EPL>
+// (S = sum phi(k) v^T, z = sum phi(k)); dk, dv hold the local terms on entry.  With GTC
+// the global terms are already in dZ (bwd_kv_global_tc_kernel) and the local terms are
+// added to them.
+template <int EPL, bool GTC>
 __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t j, const float (&k)[EPL],
                                           const float (&v)[EPL], float (&dk)[EPL], float (&dv)[EPL],
                                           const float *dSc, const float *dST, int H, int R, float *dZ,
                                           int64_t dz_ld) {
     const int D = H * R;
-    if (dST == nullptr) {                         // warp-uniform
+    if constexpr (GTC) {
         if (lh.act) {
             float *pk = dZ + j * dz_ld + D + lane * EPL, *pv = pk + D;
             float gk[EPL], gv[EPL];
@@ -768,7 +768,7 @@ __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t 
             st_mrow<EPL>(pv, dv);
         }
         return;
-    }
+    } else {
     float dphk[EPL], dvg[EPL], pk[EPL];
     ld_mrow<EPL>(dSc + static_cast<int64_t>(H) * R * R + lh.h * R + lh.f0, dphk);
 #pragma unroll
@@ -787,6 +787,7 @@ __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t 
         st_mrow<EPL>(dZ + j * dz_ld + D + lane * EPL, dk);
         st_mrow<EPL>(dZ + j * dz_ld + 2 * D + lane * EPL, dv);
     }
+    }
 }
 
 // Source rows of the transposed CSR (the targets i of j): the local terms of dk_j and
@@ -794,7 +795,7 @@ __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t 
 // Light rows (PARTS false, one warp each) walk their edges; heavy rows (PARTS true, one
 // block of kMW warps each) sum their chunks' shares part[c][0:D] | part[c][D:2D], c in
 // [chunk_ptr[s], chunk_ptr[s + 1]), warp-strided and then in warp order.  dSc holds dS [H][R][R] then dz [H][R]; dST is dS transposed per head.
-template <typename T, int EPL, bool PARTS>
+template <typename T, int EPL, bool PARTS, bool GTC = false>
 __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const int32_t *__restrict__ chunk_ptr, const float *__restrict__ part,
@@ -864,7 +865,7 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
         kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, lh.act, lh.lph, lh.h, inv_sqrt_r, k, v,
                               t_row_ptr[j], t_row_ptr[j + 1], dk, dv);
     }
-    kv_finish<EPL>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
+    kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
 }
 
 // Light source rows with two edges per step: the warp's halves (slots) take alternate
@@ -873,7 +874,7 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
 // edges of a step share one shuffle butterfly and one exponential per lane.  The halves'
 // dk, dv are then added (lower + upper, the same sum in both) and moved to the 32-lane
 // layout for kv_finish.  Needs 2 EPL <= r.
-template <typename T, int EPL>
+template <typename T, int EPL, bool GTC = false>
 __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
@@ -936,6 +937,23 @@ __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
         dk2[x] += __shfl_xor_sync(0xffffffffu, dk2[x], 16);
         dv2[x] += __shfl_xor_sync(0xffffffffu, dv2[x], 16);
     }
+    if constexpr (GTC) {
+        // the global terms are in dZ already: the lower half adds its 8-feature slices
+        if (slot == 0 && act2) {
+            float *pk = dZ + j * dz_ld + D + hl * EPL2, *pv = pk + D;
+            float gk[EPL2], gv[EPL2];
+            ld_mrow<EPL2, false>(pk, gk);
+            ld_mrow<EPL2, false>(pv, gv);
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) {
+                dk2[x] += gk[x];
+                dv2[x] += gv[x];
+            }
+            st_mrow<EPL2>(pk, dk2);
+            st_mrow<EPL2>(pv, dv2);
+        }
+        return;
+    }
     // to the 32-lane layout: lane l's features l*EPL .. are half-lane l/2's, part l % 2
     const LaneHead lh(lane, EPL, D, R);
     const int src = lane >> 1;
@@ -950,7 +968,7 @@ __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
     }
     ld_row<T, EPL>(krow, lane, lh.act, k);
     ld_row<T, EPL>(krow + D, lane, lh.act, v);
-    kv_finish<EPL>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
+    kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
 }
 
 // Chunks of heavy source rows, one warp each (layout as bwd_q_chunk_kernel's, over the
@@ -1245,24 +1263,30 @@ unsigned warp_grid(int64_t n) {
     return static_cast<unsigned>(std::max<int64_t>(1, ceil_div(n * 32, 256)));
 }
 
-// The source side's dST argument: nullptr when bwd_kv_global_tc_kernel wrote the global
-// terms (defined with that kernel).
-const float *kv_dST(const Ctx *c);
+// Whether bwd_kv_global_tc_kernel writes the source side's global terms (defined with it).
+bool kv_global_tc(const Ctx *c);
 
 // Light source rows: two edges per warp step where a head spans at least two of the
 // 16-lane half's slices (2 EPL <= r, EPL <= 4), else one edge per step.
 template <typename T, int E>
 void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cudaStream_t sk) {
     const int64_t nkl = c->bw_nk_light;
+    if constexpr (E == 4 && sizeof(T) == 2) {
+        if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
+            bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
+                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz);
+            return;
+        }
+    }
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, kv_dST(c), c->H, c->r, isr, c->bw_dZ, Dz);
+                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
             return;
         }
     }
     bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-        nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, kv_dST(c), c->H, c->r, isr, c->bw_dZ, Dz);
+        nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
 }
 
 // Light target rows: two edges per warp step under the same condition as the source side.
@@ -1283,6 +1307,25 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
         c->bw_dL, c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
 }
 
+// Heavy source rows: chunk sums, then the global terms (or, with the tensor-core global
+// terms, the local sums added to them).
+template <typename T, int E>
+void launch_kv_heavy(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, const int32_t *kh, int64_t nkh,
+                     cudaStream_t sk) {
+    const size_t sm = static_cast<size_t>(kMW) * 2 * c->D * 4;
+    auto go = [&](auto kern, const float *dSc, const float *dST) {
+        if (sm > 48 * 1024)
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+        kern<<<static_cast<unsigned>(nkh), kMW * 32, sm, sk>>>(kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr,
+                                                               c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd,
+                                                               dSc, dST, c->H, c->r, isr, c->bw_dZ, Dz);
+    };
+    if constexpr (E == 4 && sizeof(T) == 2) {
+        if (kv_global_tc(c)) return go(bwd_local_kv_kernel<T, E, true, true>, nullptr, nullptr);
+    }
+    go(bwd_local_kv_kernel<T, E, true>, c->bw_dSc, c->bw_dST);
+}
+
 // Both local backward kernels with EPL = lane_features(D): light rows one warp each;
 // heavy rows (more than kHeavyDegree entries) as kChunk-edge chunks, one warp each, whose
 // shares the per-row kernels merge in chunk order.  The target-side (dq) kernels go to
@@ -1301,12 +1344,7 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
         if (nkh) {                                                                                        \
             bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, sk>>>(c->bw_k_chunks, nkc, c->t_row_ptr,   \
                 c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
-            if (kMW * 2 * D * 4 > 48 * 1024)                                                             \
-                cudaFuncSetAttribute(bwd_local_kv_kernel<T, E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                     static_cast<int>(kMW * 2 * D * 4));                                     \
-            bwd_local_kv_kernel<T, E, true><<<static_cast<unsigned>(nkh), kMW * 32, kMW * 2 * D * 4, sk>>>( \
-                kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr, c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse,  \
-                c->bw_Dd, c->bw_dSc, kv_dST(c), H, R, isr, c->bw_dZ, Dz);                                 \
+            launch_kv_heavy<T, E>(c, Q, KV, isr, Dz, kh, nkh, sk);                                      \
         }                                                                                                 \
         if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                            \
         if (nqh) {                                                                                        \
@@ -1782,7 +1820,6 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
 bool kv_global_tc(const Ctx *c) {
     return c->io == GLGA_BF16 && c->D == kBroTcD && (c->r == 16 || c->r == 32 || c->r == 64);
 }
-const float *kv_dST(const Ctx *c) { return kv_global_tc(c) ? nullptr : c->bw_dST; }
 
 template <int R>
 void launch_kv_global_r(Ctx *c, int64_t Dz, cudaStream_t s) {
