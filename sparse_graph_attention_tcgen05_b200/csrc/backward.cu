@@ -1605,7 +1605,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
                     make_uint4(bf16x2_bits(dn[8 * i], dn[8 * i + 1]), bf16x2_bits(dn[8 * i + 2], dn[8 * i + 3]),
                                bf16x2_bits(dn[8 * i + 4], dn[8 * i + 5]), bf16x2_bits(dn[8 * i + 6], dn[8 * i + 7]));
         }
-        warp_rows_f32_flush(dnum, D, r0, N, c0, stg, lane);
+        warp_rows_f32_flush(dnum, D + 16, r0, N, c0, stg, lane);   // [dnum | dden] rows
         xdt[cq * 128 + rt] = dtp;
         xdd[cq * 128 + rt] = dda[0];
         xDd[cq * 128 + rt] = Dda[0];
@@ -1621,7 +1621,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             const float s_Dd = xDd[q0 * 128 + rt] + xDd[(q0 + 1) * 128 + rt];
             ddh[0] = -s_dd * inv[0];
             if (valid && (cq & 1) == 0) {
-                dden[row * H + c0 / R] = ddh[0];
+                dnum[row * (D + 16) + D + c0 / R] = ddh[0];
                 Dd[row * H + c0 / R] = s_Dd;
             }
         } else {
@@ -1629,7 +1629,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             for (int hq = 0; hq < kHQ; ++hq) {
                 ddh[hq] = -dda[hq] * inv[hq];
                 if (valid) {
-                    dden[row * H + c0 / R + hq] = ddh[hq];
+                    dnum[row * (D + 16) + D + c0 / R + hq] = ddh[hq];
                     Dd[row * H + c0 / R + hq] = Dda[hq];
                 }
             }
@@ -1847,6 +1847,13 @@ void launch_readout_bwd_e(Ctx *c, const T *Q, const T *dY, float b_g, float eps,
                                                                c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz);
 }
 
+// The readout backward on the tensor cores (and with it dS | dz from [dnum | dden] rows):
+// bf16 layers with H*r = 128, r in {16, 32, 64}, one head group.
+bool readout_bwd_tc(const Ctx *c) {
+    return c->io == GLGA_BF16 && c->D == kBroTcD && c->ro_groups == 1 && c->ro_kp == kBroTcD &&
+           c->ro_bn == kBroTcBN && c->n_seg == 1 && (c->r == 16 || c->r == 32 || c->r == 64);
+}
+
 template <int R>
 void launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *dY, float b_g, float eps, int64_t Dz,
                            cudaStream_t s) {
@@ -1865,10 +1872,10 @@ void launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *
 template <typename T>
 void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
     if constexpr (sizeof(T) == 2) {
-        if (c->D == kBroTcD && c->ro_groups == 1 && c->ro_kp == kBroTcD && c->ro_bn == kBroTcBN && c->n_seg == 1) {
+        if (readout_bwd_tc(c)) {
             if (c->r == 32) return launch_readout_bwd_tc<32>(c, Q, dY, b_g, eps, Dz, s);
             if (c->r == 16) return launch_readout_bwd_tc<16>(c, Q, dY, b_g, eps, Dz, s);
-            if (c->r == 64) return launch_readout_bwd_tc<64>(c, Q, dY, b_g, eps, Dz, s);
+            return launch_readout_bwd_tc<64>(c, Q, dY, b_g, eps, Dz, s);
         }
     }
     const int E = lane_features(c->D), lph = c->r / E;
@@ -1884,22 +1891,6 @@ void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, i
     }
 }
 
-template <typename T>
-void launch_dsz_bwd(Ctx *c, const T *Q, int64_t rpp, cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>(c->bw_parts), static_cast<unsigned>(c->H));
-    const int R = c->r, tiles = (R / 4) * (R / 4), G = tiles >= 256 ? 1 : 256 / tiles;
-    const size_t smem = (2 * 32 * R + 32 + (G > 1 ? static_cast<size_t>(G) * R * (R + 1) : 0)) * sizeof(float);
-#define GLGA_DZ(RR)                                                                                      \
-    case RR:                                                                                             \
-        bwd_dsz_partial_kernel<T, RR><<<grid, 256, smem, s>>>(Q, c->bw_dnum, c->bw_dden, c->N, c->H, rpp, \
-                                                              c->bw_dsz_part);                           \
-        break;
-    switch (c->r) {
-        GLGA_DZ(8) GLGA_DZ(16) GLGA_DZ(32) GLGA_DZ(64) GLGA_DZ(128)
-        default: break;
-    }
-#undef GLGA_DZ
-}
 
 // Work lists over one CSR's offsets: light rows (at most kHeavyDegree entries) sorted by
 // degree, longest first (stable), so a block's warps carry similar loads; then heavy rows
@@ -1960,8 +1951,14 @@ struct DwParams {
     int64_t rows_per_part;
     float *part;              // [P][d][Kc]
     unsigned *flag;
+    int32_t H, R;             // DSZ: heads and head width
 };
 
+// With DSZ the same kernel forms the readout's dS | dz partials: X = Q with phi applied to
+// each landed tile, dZ = [dnum | dden] (float32 rows of D + 16 columns, dden_h in column
+// D + h), and the epilogue keeps the diagonal head blocks and the dden column in the layout
+// [P][H][R][R + 1] (column R = dz) that bwd_sum_parts_kernel adds.
+template <bool DSZ>
 __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                                   const __grid_constant__ CUtensorMap tmZ,
                                                                   DwParams p) {
@@ -2063,6 +2060,14 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
             const uint8_t *z = smem + static_cast<size_t>(s) * kDwStage + kDwXBytes;
             uint8_t *bt = smem + static_cast<size_t>(s) * kDwStage + kDwXBytes + kDwZBytes;
             const int64_t y0 = r0 + static_cast<int64_t>(it) * kDwRows;
+            if constexpr (DSZ) {
+                // phi of the q tile in place (rows past the range meet zero dZ rows)
+                uint4 *xq = reinterpret_cast<uint4 *>(smem + static_cast<size_t>(s) * kDwStage);
+                for (int cidx = threadIdx.x; cidx < static_cast<int>(kDwXBytes / 16); cidx += kDwWorkers) {
+                    const uint4 u = xq[cidx];
+                    xq[cidx] = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
+                }
+            }
             // one 16-byte chunk of the bf16 tile (8 consecutive columns of one row) per step
             for (int cidx = threadIdx.x; cidx < kDwRows * 16; cidx += kDwWorkers) {
                 const int k = cidx >> 4, ch = cidx & 15;
@@ -2097,6 +2102,25 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
         const bool have = ntiles > 0 && done;
         const int a = fa * 128 + warp * 32 + lane;         // TMEM lane = input feature
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        if constexpr (DSZ) {
+            // feature a = h R + al: its head's block row (block fb = 0) or its dz (fb = 1)
+            const int h = a / p.R, al = a - h * p.R;
+            float *dst = p.part + ((static_cast<int64_t>(part) * p.H + h) * p.R + al) * (p.R + 1);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + q * 32, v);
+                tmem_ld_wait();
+                if (a < p.d) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = q * 32 + j;       // column within the 128-column block
+                        if (fb == 0 && col / p.R == h) dst[col - h * p.R] = have ? __uint_as_float(v[j]) : 0.f;
+                        if (fb == 1 && col == h) dst[p.R] = have ? __uint_as_float(v[j]) : 0.f;
+                    }
+                }
+            }
+        } else {
         float *dst = p.part + (static_cast<int64_t>(part) * p.d + a) * p.Kc;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -2109,6 +2133,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
                 for (int j = 0; j < 32; ++j)
                     if (k0 + j < p.Kc) dst[k0 + j] = have ? __uint_as_float(v[j]) : 0.f;
             }
+        }
         }
     }
     tc_fence_before();
@@ -2144,18 +2169,69 @@ glga_status tc_gemms(Ctx *c, const void *X, float *dX, cudaStream_t s) {
     p.rows_per_part = c->bw_dwtc_rpp;
     p.part = c->bw_dwtc_part;
     p.flag = c->dev_flag;
+    p.H = p.R = 0;
     const size_t smem = static_cast<size_t>(kDwStages) * kDwStage + 1024;
-    GLGA_CUDA(cudaFuncSetAttribute(bwd_dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    GLGA_CUDA(cudaFuncSetAttribute(bwd_dw_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(smem)));
     const dim3 grid(static_cast<unsigned>(c->bw_dwtc_parts), static_cast<unsigned>(ceil_div(d, 128)),
                     static_cast<unsigned>(ceil_div(Kc, 128)));
-    bwd_dw_tc_kernel<<<grid, kDwThreads, smem, s>>>(mx, mz, p);
+    bwd_dw_tc_kernel<false><<<grid, kDwThreads, smem, s>>>(mx, mz, p);
     GLGA_CUDA(cudaGetLastError());
     const int64_t total = static_cast<int64_t>(d) * Kc;
     bwd_sum_parts_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 4096)), 256, 0, s>>>(
         c->bw_dwtc_part, c->bw_dwtc_parts, total, c->bw_dW3);
     GLGA_CUDA(cudaGetLastError());
     return gemm_nt_f32out(c, GLGA_F32, c->bw_dZ, N, c->bw_dz_ld, c->bw_Wall, d, c->bw_dz_ld, Kc + 1, dX, d, s);
+}
+
+// dS | dz partials over c->bw_dsz_parts row ranges of c->bw_dsz_rpp rows.
+template <typename T>
+glga_status launch_dsz_bwd(Ctx *c, const T *Q, cudaStream_t s) {
+    const int64_t rpp = c->bw_dsz_rpp;
+    if constexpr (sizeof(T) == 2) {
+        if (readout_bwd_tc(c)) {
+            // tcgen05: X = Q [N][D] (phi applied per tile), dZ = [dnum | dden] [N][D + 16]
+            const int64_t N = c->N, D = c->D;
+            CUtensorMap mx, mz;
+            glga_status st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, static_cast<uint64_t>(D),
+                                            static_cast<uint64_t>(N), static_cast<uint64_t>(D) * 2, 64, kDwRows);
+            if (st == GLGA_OK)
+                st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dnum, static_cast<uint64_t>(D + 16),
+                                    static_cast<uint64_t>(N), static_cast<uint64_t>(D + 16) * 4, 32, kDwRows);
+            if (st != GLGA_OK) return st;
+            DwParams p;
+            p.N = N;
+            p.d = static_cast<int32_t>(D);
+            p.Kc = static_cast<int32_t>(D + 16);
+            p.rows_per_part = rpp;
+            p.part = c->bw_dsz_part;
+            p.flag = c->dev_flag;
+            p.H = c->H;
+            p.R = c->r;
+            const size_t smem = static_cast<size_t>(kDwStages) * kDwStage + 1024;
+            GLGA_CUDA(cudaFuncSetAttribute(bwd_dw_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem)));
+            bwd_dw_tc_kernel<true><<<dim3(static_cast<unsigned>(c->bw_dsz_parts), 1, 2), kDwThreads, smem, s>>>(
+                mx, mz, p);
+            GLGA_CUDA(cudaGetLastError());
+            return GLGA_OK;
+        }
+    }
+    const dim3 grid(static_cast<unsigned>(c->bw_dsz_parts), static_cast<unsigned>(c->H));
+    const int R = c->r, tiles = (R / 4) * (R / 4), G = tiles >= 256 ? 1 : 256 / tiles;
+    const size_t smem = (2 * 32 * R + 32 + (G > 1 ? static_cast<size_t>(G) * R * (R + 1) : 0)) * sizeof(float);
+#define GLGA_DZ(RR)                                                                                      \
+    case RR:                                                                                             \
+        bwd_dsz_partial_kernel<T, RR><<<grid, 256, smem, s>>>(Q, c->bw_dnum, c->bw_dden, c->N, c->H, rpp, \
+                                                              c->bw_dsz_part);                           \
+        break;
+    switch (c->r) {
+        GLGA_DZ(8) GLGA_DZ(16) GLGA_DZ(32) GLGA_DZ(64) GLGA_DZ(128)
+        default: break;
+    }
+#undef GLGA_DZ
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
 }
 
 }  // namespace
@@ -2189,12 +2265,26 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     }
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->t_col), std::max<int64_t>(E, 1) * sizeof(int32_t)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dL), nz * D * f));
-    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dnum), nz * D * f));
+    // [dnum | dden] rows of D + 16 columns (dden_h in column D + h) for the tensor-core dS | dz;
+    // dnum rows of D columns and dden [N, H] on the other paths
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dnum), nz * (D + 16) * f));
+    if (st == GLGA_OK) {
+        const cudaError_t e = cudaMemsetAsync(c->bw_dnum, 0, nz * (D + 16) * f, s);
+        if (e != cudaSuccess) st = cuda_fail(e, "backward buffers");
+    }
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dden), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_lse), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Dd), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dZ), nz * c->bw_dz_ld * f));
-    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dsz_part), static_cast<size_t>(c->bw_parts) * H * R * (R + 1) * f));
+    if (readout_bwd_tc(c)) {
+        // 64-row-aligned ranges, one thread block per SM over the ranges x {dnum, dden} grid
+        c->bw_dsz_rpp = ceil_div(ceil_div(N, std::max<int64_t>(1, c->num_sms / 2)), kDwRows) * kDwRows;
+    } else {
+        c->bw_dsz_rpp = ceil_div(std::max<int64_t>(N, 1), c->bw_parts);
+    }
+    c->bw_dsz_parts = static_cast<int32_t>(std::max<int64_t>(1, ceil_div(std::max<int64_t>(N, 1), c->bw_dsz_rpp)));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dsz_part),
+                   static_cast<size_t>(c->bw_dsz_parts) * H * R * (R + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dSz), static_cast<size_t>(H) * R * (R + 1) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_ST), static_cast<size_t>(H) * R * R * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dST), static_cast<size_t>(H) * R * R * f));
@@ -2285,7 +2375,6 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
     const int Dz = static_cast<int>(c->bw_dz_ld);
     const float isr = 1.f / std::sqrt(static_cast<float>(R));
     const int total = H * R * (R + 1);
-    const int64_t rpp = ceil_div(std::max<int64_t>(N, 1), c->bw_parts);
     const int64_t wrpp = ceil_div(std::max<int64_t>(N, 1), c->bw_wparts);
     const int Dc = 3 * D + 1;                         // columns of dZ in use: dQ | dK | dV | dt
     const int64_t wtotal = static_cast<int64_t>(d) * Dc;
@@ -2300,9 +2389,12 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
             /* fork: the dS | dz chain and the source-side kernels on the side stream */                 \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_fork, s));                                                 \
             GLGA_CUDA(cudaStreamWaitEvent(c->bw_side, c->bw_ev_fork, 0));                                 \
-            launch_dsz_bwd<T>(c, Q, rpp, c->bw_side);                                                     \
+            {                                                                                             \
+                const glga_status ds = launch_dsz_bwd<T>(c, Q, c->bw_side);                               \
+                if (ds != GLGA_OK) return ds;                                                             \
+            }                                                                                             \
             bwd_sum_parts_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, c->bw_side>>>(   \
-                c->bw_dsz_part, c->bw_parts, total, c->bw_dSz);                                           \
+                c->bw_dsz_part, c->bw_dsz_parts, total, c->bw_dSz);                                       \
             bwd_heads_prep_kernel<<<tgrid, 256, 0, c->bw_side>>>(c->bw_dSz, R + 1, H, R, c->bw_dST,      \
                                                                 c->bw_dSc);                               \
             launch_kv_global(c, Dz, c->bw_side);                                                          \

@@ -155,6 +155,8 @@ struct Ctx {
     int64_t bw_nq_light = 0, bw_nq_heavy = 0, bw_nk_light = 0, bw_nk_heavy = 0;
     int64_t bw_dz_ld = 0;
     int32_t bw_parts = 0, bw_wparts = 0;
+    int32_t bw_dsz_parts = 0;                         // dS | dz row ranges and their rows
+    int64_t bw_dsz_rpp = 0;
 
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;
