@@ -2184,6 +2184,372 @@ glga_status tc_gemms(Ctx *c, const void *X, float *dX, cudaStream_t s) {
     return gemm_nt_f32out(c, GLGA_F32, c->bw_dZ, N, c->bw_dz_ld, c->bw_Wall, d, c->bw_dz_ld, Kc + 1, dX, d, s);
 }
 
+// ---------------------------------------------------------------------------------------
+// dX, dW, dw_g and db_g of a bf16 layer with d = 128 in one pass over dZ (tcgen05):
+//   dX[i][a] = sum_k dZ[i][k] W[a][k] + dt_i w_g[a]            (W = [W_Q | W_K | W_V])
+//   dW[a][k] = sum_i X[i][a] dZ[i][k],  dw_g[a] = sum_i X[i][a] dt_i,  db_g = sum_i dt_i
+// A persistent grid: thread block b takes the 128-row tiles b, b + G, ...  Per tile one
+// producer thread loads by TMA the X tile (two [128][64] bf16 boxes) with dt (a [128][4]
+// float box at column 3D), then per 64-column chunk of dZ two [128][32] float boxes and
+// the [128 a][64 k] block of W that the chunk multiplies.  Warps 0-7 round each dZ chunk
+// to a bf16 tile (128-byte swizzle) and, once per tile, add X^T dt and the sum of dt on
+// the CUDA cores.  One thread issues per chunk the dX MMAs (the bf16 chunk K-major as A,
+// the W block K-major as B: M = 128 rows, N = 128 features) into TMEM columns 0-127 and
+// the dW MMAs (X^T MN-major as A, the bf16 chunk MN-major as B: M = 128 features, N = 64)
+// into the chunk's columns of a [128][3D] accumulator that stays in TMEM over all the
+// block's tiles.  Warps 10-13 drain dX per tile (adding dt w_g) through a staging area
+// into coalesced row stores, and after the last tile write the block's dW partial sums;
+// the range-order reductions add the blocks' partials (the result is the same on every
+// call).  Every wait is bounded: on expiry the kernel raises the context's flag, lets its
+// copies land, waits for its MMAs and returns.
+constexpr int kFxRows = 128;
+constexpr int kFxXStages = 2, kFxFStages = 4, kFxBStages = 2;
+constexpr uint32_t kFxBox = kFxRows * 128;                  // a [128][128 B] box: 16 KB
+constexpr uint32_t kFxXStage = 2 * kFxBox + kFxRows * 16;   // X tile, then the dt box
+constexpr uint32_t kFxBStage = 2 * kFxBox;                  // bf16 dZ chunk, then the W block
+constexpr uint32_t kFxEpi = kFxXStages * kFxXStage + kFxFStages * kFxBox + kFxBStages * kFxBStage;
+constexpr uint32_t kFxEpiStage = 4096;                      // per epilogue warp
+constexpr size_t kFxSmem = 1024 + kFxEpi + 4 * kFxEpiStage + (128 + 256 + 2) * sizeof(float);
+constexpr int kFxWorkers = 256, kFxProd = 8, kFxMma = 9, kFxEpi0 = 10, kFxThreads = 448;
+static_assert(kFxXStage % 1024 == 0 && kFxEpi % 1024 == 0, "stages stay 1024-byte aligned");
+
+struct FxParams {
+    int64_t N;
+    int32_t D, Kc, ntiles;          // W blocks of D columns; 3D dZ columns; 128-row tiles
+    const __nv_bfloat16 *wg;        // [128]
+    float *dX;                      // [N][128]
+    float *dw_part;                 // [P][128][3D]
+    float *g_part;                  // [P][128][3D + 1]: column 3D holds dw_g
+    float *b_part;                  // [P]
+    unsigned *flag;
+};
+
+__global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmZ,
+    const __grid_constant__ CUtensorMap tmDt, const __grid_constant__ CUtensorMap tmWq,
+    const __grid_constant__ CUtensorMap tmWk, const __grid_constant__ CUtensorMap tmWv, FxParams p) {
+    extern __shared__ uint8_t dsmem_raw[];
+    __shared__ __align__(8) uint64_t x_full[kFxXStages], x_empty[kFxXStages];
+    __shared__ __align__(8) uint64_t f_full[kFxFStages], f_empty[kFxFStages];
+    __shared__ __align__(8) uint64_t w_full[kFxBStages], b_full[kFxBStages], b_empty[kFxBStages];
+    __shared__ __align__(8) uint64_t dx_full, dx_empty, mma_done;
+    __shared__ uint32_t tmem_base_sh;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sX = smem;                                      // [kFxXStages] X tile + dt
+    uint8_t *sF = sX + kFxXStages * kFxXStage;               // [kFxFStages] float dZ boxes
+    uint8_t *sB = sF + kFxFStages * kFxBox;                  // [kFxBStages] bf16 chunk + W block
+    uint8_t *sE = smem + kFxEpi;                             // epilogue staging
+    float *swg = reinterpret_cast<float *>(sE + 4 * kFxEpiStage);   // w_g as float
+    float *sred = swg + 128;                                 // [256] + [2] worker sums
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, blk = blockIdx.x;
+    const int my = blk < p.ntiles ? (p.ntiles - 1 - blk) / G + 1 : 0;   // this block's tiles
+    const int nc = p.Kc / 64, cpm = p.D / 64;               // chunks per tile, per W matrix
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kFxXStages; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1 + kFxWorkers / 32 + 4);   // MMA commit, workers, epilogue
+        }
+        for (int s = 0; s < kFxFStages; ++s) {
+            mbar_init(&f_full[s], 1);
+            mbar_init(&f_empty[s], kFxWorkers / 32);
+        }
+        for (int s = 0; s < kFxBStages; ++s) {
+            mbar_init(&w_full[s], 1);
+            mbar_init(&b_full[s], kFxWorkers / 32);
+            mbar_init(&b_empty[s], 1);
+        }
+        mbar_init(&dx_full, 1);
+        mbar_init(&dx_empty, 4);
+        mbar_init(&mma_done, 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 128) swg[threadIdx.x] = __bfloat162float(p.wg[threadIdx.x]);
+    if (warp == kFxMma) {
+        tmem_alloc(&tmem_base_sh, 512u);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == kFxProd) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmX);
+            tma_prefetch_desc(&tmZ);
+            bool ok = true;
+            int nx = 0, nf = 0, nb = 0;                          // loads issued per ring
+            for (int j = 0; j < my && ok; ++j) {
+                const int32_t y = (blk + j * G) * kFxRows;
+                const int xs = nx % kFxXStages;
+                if (nx >= kFxXStages && !mbar_wait_bounded(&x_empty[xs], ((nx / kFxXStages) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *xst = sX + xs * kFxXStage;
+                mbar_arrive_expect_tx(&x_full[xs], kFxXStage);
+                tma_load_2d(xst, &tmX, &x_full[xs], 0, y);
+                tma_load_2d(xst + kFxBox, &tmX, &x_full[xs], 64, y);
+                tma_load_2d(xst + 2 * kFxBox, &tmDt, &x_full[xs], p.Kc, y);
+                ++nx;
+                for (int cc = 0; cc < nc && ok; ++cc) {
+                    for (int h = 0; h < 2; ++h) {
+                        const int fs = nf % kFxFStages;
+                        if (nf >= kFxFStages && !mbar_wait_bounded(&f_empty[fs], ((nf / kFxFStages) - 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&f_full[fs], kFxBox);
+                        tma_load_2d(sF + fs * kFxBox, &tmZ, &f_full[fs], cc * 64 + h * 32, y);
+                        ++nf;
+                    }
+                    if (!ok) break;
+                    const int bs = nb % kFxBStages;
+                    if (nb >= kFxBStages && !mbar_wait_bounded(&b_empty[bs], ((nb / kFxBStages) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const CUtensorMap *wm = cc < cpm ? &tmWq : (cc < 2 * cpm ? &tmWk : &tmWv);
+                    mbar_arrive_expect_tx(&w_full[bs], kFxBox);
+                    tma_load_2d(sB + bs * kFxBStage + kFxBox, wm, &w_full[bs], (cc % cpm) * 64, 0);
+                    ++nb;
+                }
+            }
+            if (!ok) atomicOr(p.flag, kDevErrTimeout);
+            // the block leaves only after its copies have landed (already so when all went well)
+            for (int i = std::max(0, nx - kFxXStages); i < nx; ++i)
+                mbar_wait_bounded(&x_full[i % kFxXStages], (i / kFxXStages) & 1);
+            for (int i = std::max(0, nf - kFxFStages); i < nf; ++i)
+                mbar_wait_bounded(&f_full[i % kFxFStages], (i / kFxFStages) & 1);
+            for (int i = std::max(0, nb - kFxBStages); i < nb; ++i)
+                mbar_wait_bounded(&w_full[i % kFxBStages], (i / kFxBStages) & 1);
+        }
+    } else if (warp == kFxMma) {
+        if (lane == 0) {
+            const uint32_t id_dx = instr_desc(128, 128, 1u, false, false);
+            const uint32_t id_dw = instr_desc(128, 64, 1u, true, true);
+            bool ok = true;
+            int nb = 0;
+            for (int j = 0; j < my && ok; ++j) {
+                const int xs = j % kFxXStages;
+                if (!mbar_wait_bounded(&x_full[xs], (j / kFxXStages) & 1) ||
+                    (j > 0 && !mbar_wait_bounded(&dx_empty, (j - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xa = smem_u32(sX + xs * kFxXStage);
+                for (int cc = 0; cc < nc; ++cc, ++nb) {
+                    const int bs = nb % kFxBStages;
+                    const uint32_t par = static_cast<uint32_t>(nb / kFxBStages) & 1u;
+                    if (!mbar_wait_bounded(&w_full[bs], par) || !mbar_wait_bounded(&b_full[bs], par)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t zb = smem_u32(sB + bs * kFxBStage), wb = zb + kFxBox;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)        // dX += dZ chunk (K-major) W block^T
+                        umma_bf16(tmem, smem_desc(zb + ks * 32, 16, 1024, 2), smem_desc(wb + ks * 32, 16, 1024, 2),
+                                  id_dx, (cc | ks) != 0);
+#pragma unroll
+                    for (int ks = 0; ks < kFxRows / 16; ++ks)   // dW chunk += X^T dZ chunk
+                        umma_bf16(tmem + 128 + cc * 64, smem_desc(xa + ks * 2048, kFxBox, 1024, 2),
+                                  smem_desc(zb + ks * 2048, kFxBox, 1024, 2), id_dw, (j | ks) != 0);
+                    umma_commit(&b_empty[bs]);
+                }
+                if (!ok) break;
+                umma_commit(&x_empty[xs]);
+                umma_commit(&dx_full);
+            }
+            if (!ok) atomicOr(p.flag, kDevErrTimeout);
+            umma_commit(&mma_done);
+        }
+    } else if (warp < kFxWorkers / 32) {
+        // ---------------- warps 0-7: dZ chunks to bf16; X^T dt and the sum of dt -------------
+        const int t = threadIdx.x, fa = t & 127, hh = t >> 7;   // feature, half of the tile's rows
+        bool ok = true;
+        int nf = 0, nb = 0;
+        float accg = 0.f, accb = 0.f;
+        for (int j = 0; j < my && ok; ++j) {
+            const int xs = j % kFxXStages;
+            for (int cc = 0; cc < nc; ++cc) {
+                const int fs0 = nf % kFxFStages, fs1 = (nf + 1) % kFxFStages, bs = nb % kFxBStages;
+                const bool got = mbar_wait_bounded(&f_full[fs0], (nf / kFxFStages) & 1) &&
+                                 mbar_wait_bounded(&f_full[fs1], ((nf + 1) / kFxFStages) & 1) &&
+                                 (nb < kFxBStages || mbar_wait_bounded(&b_empty[bs], ((nb / kFxBStages) - 1) & 1));
+                // the warp agrees on the outcome, so it stays converged for its arrivals
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *f0 = sF + fs0 * kFxBox, *f1 = sF + fs1 * kFxBox;
+                uint8_t *bt = sB + bs * kFxBStage;
+                // one 16-byte chunk (8 columns of one row) of the bf16 tile per step
+                for (int it = t; it < kFxRows * 8; it += kFxWorkers) {
+                    const int k = it >> 3, co = it & 7, j0 = (co & 3) * 2;
+                    const uint8_t *zr = (co < 4 ? f0 : f1) + k * 128;
+                    const float4 u = *reinterpret_cast<const float4 *>(zr + ((j0 ^ (k & 7)) << 4));
+                    const float4 v = *reinterpret_cast<const float4 *>(zr + (((j0 + 1) ^ (k & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(bt + k * 128 + ((co ^ (k & 7)) << 4)) =
+                        make_uint4(bf16x2_bits(u.x, u.y), bf16x2_bits(u.z, u.w), bf16x2_bits(v.x, v.y),
+                                   bf16x2_bits(v.z, v.w));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&f_empty[fs0]);
+                    mbar_arrive(&f_empty[fs1]);
+                    mbar_arrive(&b_full[bs]);
+                }
+                nf += 2;
+                ++nb;
+            }
+            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&x_full[xs], (j / kFxXStages) & 1))) {
+                ok = false;
+                break;
+            }
+            const uint8_t *xt = sX + xs * kFxXStage + (fa >> 6) * kFxBox;
+            const float *dt = reinterpret_cast<const float *>(sX + xs * kFxXStage + 2 * kFxBox);
+            const int cb = (fa & 63) >> 3, wi = (fa & 7) * 2;   // 16-byte chunk in the row, byte in it
+            for (int r = hh * 64; r < hh * 64 + 64; ++r) {
+                const float x = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16 *>(xt + r * 128 + ((cb ^ (r & 7)) << 4) + wi));
+                const float dv = dt[r * 4];
+                accg = fmaf(x, dv, accg);
+                accb += dv;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x_empty[xs]);
+        }
+        if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+        // the two row halves of each feature, added in a fixed order
+        sred[t] = accg;
+        if (t == 0 || t == 128) sred[256 + hh] = accb;
+        asm volatile("bar.sync 1, %0;" ::"n"(kFxWorkers) : "memory");
+        if (t < 128)
+            p.g_part[(static_cast<int64_t>(blk) * 128 + t) * (p.Kc + 1) + p.Kc] = sred[t] + sred[t + 128];
+        if (t == 0) p.b_part[blk] = sred[256] + sred[257];
+    } else if (warp >= kFxEpi0) {
+        // ---------------- warps 10-13: dX per tile, then the block's dW ---------------------
+        const int qw = warp & 3;                              // TMEM lane quarter
+        uint8_t *stg = sE + (warp - kFxEpi0) * kFxEpiStage;
+        const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
+        bool ok = true;
+        for (int j = 0; j < my && ok; ++j) {
+            const int xs = j % kFxXStages;
+            const bool got = mbar_wait_bounded(&dx_full, j & 1) && mbar_wait_bounded(&x_full[xs], (j / kFxXStages) & 1);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int64_t r0 = static_cast<int64_t>(blk + j * G) * kFxRows + qw * 32;
+            const float dv = reinterpret_cast<const float *>(sX + xs * kFxXStage + 2 * kFxBox)[(qw * 32 + lane) * 4];
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + q * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int pc = 0; pc < 8; ++pc) {
+                    const float *g = swg + q * 32 + pc * 4;
+                    stage_f32_piece(stg, lane, pc, fmaf(dv, g[0], __uint_as_float(v[4 * pc])),
+                                    fmaf(dv, g[1], __uint_as_float(v[4 * pc + 1])),
+                                    fmaf(dv, g[2], __uint_as_float(v[4 * pc + 2])),
+                                    fmaf(dv, g[3], __uint_as_float(v[4 * pc + 3])));
+                }
+                warp_rows_f32_flush(p.dX, 128, r0, p.N, q * 32, stg, lane);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&dx_empty);
+                mbar_arrive(&x_empty[xs]);
+            }
+        }
+        if (!ok && lane == 0) atomicOr(p.flag, kDevErrTimeout);
+        if (ok && my > 0) {
+            // the last tile's dX commit covers every MMA of the block: dW is complete
+            float *dst = p.dw_part + static_cast<int64_t>(blk) * 128 * p.Kc;
+#pragma unroll 1
+            for (int q = 0; q < p.Kc / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + 128 + q * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int pc = 0; pc < 8; ++pc)
+                    stage_f32_piece(stg, lane, pc, __uint_as_float(v[4 * pc]), __uint_as_float(v[4 * pc + 1]),
+                                    __uint_as_float(v[4 * pc + 2]), __uint_as_float(v[4 * pc + 3]));
+                warp_rows_f32_flush(dst, p.Kc, qw * 32, 128, q * 32, stg, lane);
+            }
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kFxMma) {
+        // every MMA issued has completed before the columns are freed
+        if (lane == 0 && !mbar_wait_bounded(&mma_done, 0)) atomicOr(p.flag, kDevErrTimeout);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512u);
+    }
+}
+
+// Whether dX and the weight gradients of this context take the one-pass kernel: bf16
+// layers with d = 128 and D a multiple of 64 up to 128 (dX and dW fit TMEM together).
+bool bwd_fx(const Ctx *c) {
+    return c->io == GLGA_BF16 && c->d == 128 && c->D % 64 == 0 && c->D <= 128 && c->N > 0;
+}
+
+// dX, and the dW / dw_g / db_g partials that bwd_dw_reduce_kernel and bwd_dbg_kernel add
+// (over c->bw_fx_parts blocks), in one pass over dZ.
+glga_status fx_gemms(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV, const void *wg,
+                     float *dX, cudaStream_t s) {
+    const int64_t N = c->N, D = c->D, Kc = 3 * D;
+    const uint64_t zrow = static_cast<uint64_t>(c->bw_dz_ld) * 4;
+    CUtensorMap mx, mz, mdt, mq, mk, mv;
+    glga_status st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 128, static_cast<uint64_t>(N), 256,
+                                    64, kFxRows);
+    if (st == GLGA_OK)
+        st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dZ, static_cast<uint64_t>(Kc),
+                            static_cast<uint64_t>(N), zrow, 32, kFxRows);
+    if (st == GLGA_OK)
+        st = encode_tmap_2d(&mdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dZ, static_cast<uint64_t>(c->bw_dz_ld),
+                            static_cast<uint64_t>(N), zrow, 4, kFxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    const void *wm[3] = {WQ, WK, WV};
+    CUtensorMap *mw[3] = {&mq, &mk, &mv};
+    for (int m = 0; m < 3 && st == GLGA_OK; ++m)
+        st = encode_tmap_2d(mw[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wm[m], static_cast<uint64_t>(D), 128,
+                            static_cast<uint64_t>(D) * 2, 64, 128);
+    if (st != GLGA_OK) return st;
+    FxParams p;
+    p.N = N;
+    p.D = static_cast<int32_t>(D);
+    p.Kc = static_cast<int32_t>(Kc);
+    p.ntiles = static_cast<int32_t>(ceil_div(N, kFxRows));
+    p.wg = static_cast<const __nv_bfloat16 *>(wg);
+    p.dX = dX;
+    p.dw_part = c->bw_dwtc_part;
+    p.g_part = c->bw_dw_part;
+    p.b_part = c->bw_dbg_part;
+    p.flag = c->dev_flag;
+    GLGA_CUDA(cudaFuncSetAttribute(bwd_dxdw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(kFxSmem)));
+    bwd_dxdw_tc_kernel<<<static_cast<unsigned>(c->bw_fx_parts), kFxThreads, kFxSmem, s>>>(mx, mz, mdt, mq, mk, mv, p);
+    GLGA_CUDA(cudaGetLastError());
+    const int64_t total = 128 * Kc;
+    bwd_sum_parts_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 4096)), 256, 0, s>>>(
+        c->bw_dwtc_part, c->bw_fx_parts, total, c->bw_dW3);
+    GLGA_CUDA(cudaGetLastError());
+    return GLGA_OK;
+}
+
 // dS | dz partials over c->bw_dsz_parts row ranges of c->bw_dsz_rpp rows.
 template <typename T>
 glga_status launch_dsz_bwd(Ctx *c, const T *Q, cudaStream_t s) {
@@ -2289,9 +2655,12 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_ST), static_cast<size_t>(H) * R * R * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dST), static_cast<size_t>(H) * R * R * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dSc), static_cast<size_t>(H) * R * (R + 1) * f));
+    // the one-pass dX / dW kernel: one thread block per SM, each with at least one row tile
+    c->bw_fx_parts = bwd_fx(c) ? static_cast<int32_t>(std::min<int64_t>(c->num_sms, ceil_div(N, kFxRows))) : 0;
+    const int64_t gparts = std::max<int64_t>(c->bw_wparts, c->bw_fx_parts);
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dw_part),
-                   static_cast<size_t>(c->bw_wparts) * c->d * (3 * D + 1) * f));
-    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dbg_part), static_cast<size_t>(c->bw_wparts) * f));
+                   static_cast<size_t>(gparts) * c->d * (3 * D + 1) * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dbg_part), static_cast<size_t>(gparts) * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Wall), static_cast<size_t>(c->d) * c->bw_dz_ld * f));
     if (bwd_tc_gemms(c)) {
         // weight-gradient partials of the tensor-core GEMM: 64-row-aligned ranges, about
@@ -2302,7 +2671,7 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
         c->bw_dwtc_rpp = rpp;
         c->bw_dwtc_parts = static_cast<int32_t>(ceil_div(N, rpp));
         BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dwtc_part),
-                       static_cast<size_t>(c->bw_dwtc_parts) * c->d * 3 * D * f));
+                       static_cast<size_t>(std::max(c->bw_dwtc_parts, c->bw_fx_parts)) * c->d * 3 * D * f));
         BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dW3), static_cast<size_t>(c->d) * 3 * D * f));
     }
 #undef BTRY
@@ -2401,6 +2770,11 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
             launch_local_bwd<T>(c, Q, KV, isr, Dz, s, c->bw_side);                                        \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_join, c->bw_side));                                        \
             GLGA_CUDA(cudaStreamWaitEvent(s, c->bw_ev_join, 0));                                          \
+            if (bwd_fx(c)) {                                                                              \
+                const glga_status gs = fx_gemms(c, X, WQ, WK, WV, wg, dX, s);                             \
+                if (gs != GLGA_OK) return gs;                                                             \
+                break;                                                                                    \
+            }                                                                                             \
             if (bwd_tc_gemms(c)) {                                                                        \
                 bwd_pack_w_kernel<T><<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d * Dz, 256), 1024)), \
                                        256, 0, s>>>(static_cast<const T *>(WQ), static_cast<const T *>(WK), \
@@ -2432,9 +2806,10 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
         BWD_LAUNCHES(__nv_bfloat16);
 #undef BWD_LAUNCHES
     if (N > 0) {
+        const int wp = bwd_fx(c) ? c->bw_fx_parts : c->bw_wparts;   // partials of dw_g (and dW)
         bwd_dw_reduce_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(wtotal, 256), 4096)), 256, 0, s>>>(
-            c->bw_dw_part, c->bw_wparts, bwd_tc_gemms(c) ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
-        bwd_dbg_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, c->bw_wparts, db_g);
+            c->bw_dw_part, wp, bwd_tc_gemms(c) ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
+        bwd_dbg_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, wp, db_g);
     } else {
         GLGA_CUDA(cudaMemsetAsync(dWQ, 0, static_cast<size_t>(d) * D * sizeof(float), s));
         GLGA_CUDA(cudaMemsetAsync(dWK, 0, static_cast<size_t>(d) * D * sizeof(float), s));

@@ -157,6 +157,7 @@ struct Ctx {
     int32_t bw_parts = 0, bw_wparts = 0;
     int32_t bw_dsz_parts = 0;                         // dS | dz row ranges and their rows
     int64_t bw_dsz_rpp = 0;
+    int32_t bw_fx_parts = 0;                          // thread blocks of the one-pass dX / dW kernel (0: off)
 
     unsigned *dev_flag = nullptr;
     int64_t bytes = 0;
@@ -232,7 +233,8 @@ glga_status readout_run(Ctx *c, float b_g, float eps, void *Y, cudaStream_t s);
 // tensor maps (driver entry point resolved at run time; no libcuda link dependency)
 glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
                            uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                           uint32_t box_inner, uint32_t box_outer);
+                           uint32_t box_inner, uint32_t box_outer,
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 // ---------------------------------------------------------------------------------------
 // device helpers

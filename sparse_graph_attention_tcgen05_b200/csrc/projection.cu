@@ -781,7 +781,7 @@ glga_status gemm_nt_f32out(Ctx *c, glga_dtype t, const void *A, int64_t M, int64
 
 glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
                            uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
-                           uint32_t box_outer) {
+                           uint32_t box_outer, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
         set_error("cuTensorMapEncodeTiled unavailable from the driver");
@@ -796,7 +796,7 @@ glga_status encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void 
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         set_error("cuTensorMapEncodeTiled failed (%d) dims=%llu,%llu box=%u,%u", static_cast<int>(r),

@@ -139,3 +139,15 @@ def test_tensor_core_readout_backward(H, r, N):
     dst = np.concatenate([np.repeat(np.arange(N), 4), np.arange(N)]).astype(np.int32)
     w = make_custom(N, 64, H, r, src, dst, io="bf16", seed=N * 3 + H, b_g=0.2)
     _check(w, seed=H, chunked=N > 5000)
+
+
+@pytest.mark.parametrize("H,r,N", [(2, 32, 100), (1, 64, 300), (4, 32, 148 * 128 + 77)])
+def test_one_pass_dx_dw(H, r, N):
+    # bf16 layers with d = 128 form dX, dW, dw_g and db_g in one tensor-core pass over dZ
+    # (dX and the whole dW block in TMEM together): D = 64 and D = 128, a single ragged
+    # 128-row tile, and more tiles than thread blocks with a ragged last one
+    rng = np.random.default_rng(N + H)
+    src = np.concatenate([rng.integers(0, N, 3 * N), np.arange(N)]).astype(np.int32)
+    dst = np.concatenate([np.repeat(np.arange(N), 3), np.arange(N)]).astype(np.int32)
+    w = make_custom(N, 128, H, r, src, dst, io="bf16", seed=N + 7, b_g=-0.1)
+    _check(w, seed=r, chunked=N > 5000)
