@@ -403,14 +403,51 @@ __global__ void bwd_heads_prep_kernel(const float *__restrict__ src, int ld, int
     }
 }
 
-// out[o] = sum over p = 0 .. P-1, in order, of part[p][o].
-__global__ void bwd_sum_parts_kernel(const float *__restrict__ part, int P, int64_t total, float *__restrict__ out) {
-    for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
-         o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float acc = 0.f;
-        for (int p = 0; p < P; ++p) acc += part[static_cast<int64_t>(p) * total + o];
-        out[o] = acc;
+// out[o] = sum over p of part[p][o], in a fixed order: a block takes 32 consecutive
+// outputs o; its warp g adds the partials p = g, g + 8, g + 16, ... in order (coalesced
+// 128-byte rows, four loads in flight), and warp 0 adds the 8 warp sums in warp order.
+constexpr int kSumThreads = 256, kSumOut = 32;
+__global__ void __launch_bounds__(kSumThreads) bwd_sum_parts_kernel(const float *__restrict__ part, int P,
+                                                                    int64_t total, float *__restrict__ out) {
+    __shared__ float red[kSumThreads / 32][kSumOut];
+    const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+    constexpr int kG = kSumThreads / 32;
+    const int64_t o = static_cast<int64_t>(blockIdx.x) * kSumOut + lane;
+    float acc = 0.f;
+    if (o < total) {
+        int p = g;
+        for (; p + 3 * kG < P; p += 4 * kG) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = __ldg(part + static_cast<int64_t>(p + u * kG) * total + o);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc += v[u];
+        }
+        for (; p < P; p += kG) acc += __ldg(part + static_cast<int64_t>(p) * total + o);
     }
+    red[g][lane] = acc;
+    __syncthreads();
+    if (g == 0 && o < total) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kG; ++w) sum += red[w][lane];
+        out[o] = sum;
+    }
+}
+unsigned sum_parts_grid(int64_t total) { return static_cast<unsigned>(ceil_div(total, kSumOut)); }
+
+// out[a] = sum over p of part[p * sp + a * sa] (a < n), one warp per output: lane l adds
+// p = l, l + 32, ... in order, then a fixed butterfly adds the lanes.
+__global__ void __launch_bounds__(256) bwd_strided_sum_kernel(const float *__restrict__ part, int P, int64_t sp,
+                                                              int64_t sa, int n, float *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int a = static_cast<int>((blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5);
+    if (a >= n) return;                                   // warp-uniform
+    float acc = 0.f;
+    for (int p = lane; p < P; p += 32) acc += __ldg(part + static_cast<int64_t>(p) * sp + a * sa);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (lane == 0) out[a] = acc;
 }
 
 constexpr int kEU = 4;            // edges whose rows are loaded before any is used
@@ -1049,15 +1086,6 @@ __global__ void __launch_bounds__(256) bwd_dwg_kernel(const T *__restrict__ X, c
     if (t == 0) dbg_part[blockIdx.x] = red[0];
 }
 
-// db_g = the row-range sums in range order.
-__global__ void bwd_dbg_kernel(const float *__restrict__ dbg_part, int P, float *__restrict__ db_g) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) {
-        float s = 0.f;
-        for (int p = 0; p < P; ++p) s += dbg_part[p];
-        *db_g = s;
-    }
-}
-
 // Register-tiled fp32 GEMM tiles for the weight and input gradients: a 128 x 128 output
 // tile per 256-thread block, 8 reduction steps per shared-memory stage (two stages, the
 // next one loaded into registers while the current one is multiplied), and 8 x 8 outputs
@@ -1151,8 +1179,8 @@ __global__ void __launch_bounds__(256, 2) bwd_dw_kernel(const T *__restrict__ X,
 }
 
 // dW_Q | dW_K | dW_V | dw_g from the row-range parts, summed in range order; when w3 is
-// given (one GEMM wrote the columns k < 3D whole, as w3[a][k] with row stride 3D) those
-// columns are copied from it and only column 3D comes from the parts.
+// given (the tensor cores' sums of the columns k < 3D, as w3[a][k] with row stride 3D)
+// those columns are copied from it and column 3D (dw_g) is left to bwd_strided_sum_kernel.
 __global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, const float *__restrict__ w3, int d,
                                      int D, int Dc, float *__restrict__ dWQ, float *__restrict__ dWK,
                                      float *__restrict__ dWV, float *__restrict__ dwg) {
@@ -1160,8 +1188,9 @@ __global__ void bwd_dw_reduce_kernel(const float *__restrict__ part, int P, cons
     for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < total;
          o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int a = static_cast<int>(o / Dc), k = static_cast<int>(o % Dc);
+        if (w3 && k >= 3 * D) continue;                   // dw_g: bwd_strided_sum_kernel
         float acc = 0.f;
-        if (w3 && k < 3 * D) {
+        if (w3) {
             acc = w3[static_cast<int64_t>(a) * 3 * D + k];
         } else {
             for (int p = 0; p < P; ++p) acc += part[static_cast<int64_t>(p) * total + o];
@@ -1944,6 +1973,13 @@ constexpr uint32_t kDwBox = kDwRows * 128;                 // one 64-row box of 
 constexpr uint32_t kDwXBytes = 2 * kDwBox;                 // X tile (bf16)
 constexpr uint32_t kDwZBytes = 4 * kDwBox;                 // dZ tile (float32)
 constexpr uint32_t kDwStage = kDwXBytes + kDwZBytes + 2 * kDwBox;   // + dZ rounded to bf16
+// the dS | dz form: [dnum | dden] tiles of 144 columns, the dden part a [64][16] float box
+// without swizzle, rounded into a bf16 tile of three 64-column atoms; two stages
+constexpr int kDszStages = 2;
+constexpr uint32_t kDszDBytes = kDwRows * 64;
+constexpr uint32_t kDszZBytes = kDwZBytes + kDszDBytes;
+constexpr uint32_t kDszStage = kDwXBytes + kDszZBytes + 3 * kDwBox;
+static_assert((kDwXBytes + kDszZBytes) % 1024 == 0 && kDszStage % 1024 == 0, "1024-byte aligned tiles");
 
 struct DwParams {
     int64_t N;
@@ -1956,16 +1992,23 @@ struct DwParams {
 
 // With DSZ the same kernel forms the readout's dS | dz partials: X = Q with phi applied to
 // each landed tile, dZ = [dnum | dden] (float32 rows of D + 16 columns, dden_h in column
-// D + h), and the epilogue keeps the diagonal head blocks and the dden column in the layout
+// D + h; tmD loads the 16 dden columns), one M = 128, N = 144 MMA per 16 rows, and the
+// epilogue keeps the diagonal head blocks and the dden column in the layout
 // [P][H][R][R + 1] (column R = dz) that bwd_sum_parts_kernel adds.
 template <bool DSZ>
 __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                                   const __grid_constant__ CUtensorMap tmZ,
+                                                                  const __grid_constant__ CUtensorMap tmD,
                                                                   DwParams p) {
+    constexpr int kStages = DSZ ? kDszStages : kDwStages;
+    constexpr uint32_t kZBytes = DSZ ? kDszZBytes : kDwZBytes;
+    constexpr uint32_t kStageBytes = DSZ ? kDszStage : kDwStage;
+    constexpr int kNCols = DSZ ? 144 : 128;                   // MMA N
+    constexpr uint32_t kTmemCols = DSZ ? 256u : 128u;
     extern __shared__ uint8_t dsmem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[kDwStages];
-    __shared__ __align__(8) uint64_t ready_bar[kDwStages];
-    __shared__ __align__(8) uint64_t empty_bar[kDwStages];
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ __align__(8) uint64_t ready_bar[kStages];
+    __shared__ __align__(8) uint64_t empty_bar[kStages];
     __shared__ __align__(8) uint64_t done_bar;
     __shared__ uint32_t tmem_base_sh;
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -1977,7 +2020,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
     const int ntiles = r1 > r0 ? static_cast<int>(ceil_div(r1 - r0, kDwRows)) : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kDwStages; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&ready_bar[s], kDwWorkers / 32);   // one arrival per worker warp
             mbar_init(&empty_bar[s], 1);
@@ -1986,7 +2029,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
         fence_mbar_init();
     }
     if (warp == kDwMma) {
-        tmem_alloc(&tmem_base_sh, 128u);
+        tmem_alloc(&tmem_base_sh, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -2001,40 +2044,41 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
             int issued = 0;
             RingPos rp;
             bool ok = true;
-            for (int it = 0; it < ntiles; ++it, rp.next(kDwStages)) {
+            for (int it = 0; it < ntiles; ++it, rp.next(kStages)) {
                 const int s = rp.slot;
-                if (it >= kDwStages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
+                if (it >= kStages && !mbar_wait_bounded(&empty_bar[s], rp.phase ^ 1u)) {
                     ok = false;
                     break;
                 }
-                uint8_t *st = smem + static_cast<size_t>(s) * kDwStage;
-                mbar_arrive_expect_tx(&full_bar[s], kDwXBytes + kDwZBytes);
+                uint8_t *st = smem + static_cast<size_t>(s) * kStageBytes;
+                mbar_arrive_expect_tx(&full_bar[s], kDwXBytes + kZBytes);
                 const int32_t y = static_cast<int32_t>(r0 + static_cast<int64_t>(it) * kDwRows);
                 for (int b = 0; b < 2; ++b) tma_load_2d(st + b * kDwBox, &tmX, &full_bar[s], fa * 128 + b * 64, y);
                 for (int b = 0; b < 4; ++b)
                     tma_load_2d(st + kDwXBytes + b * kDwBox, &tmZ, &full_bar[s], fb * 128 + b * 32, y);
+                if constexpr (DSZ) tma_load_2d(st + kDwXBytes + kDwZBytes, &tmD, &full_bar[s], p.d, y);
                 ++issued;
             }
             if (!ok) {
                 atomicOr(p.flag, kDevErrTimeout);
-                for (int it = std::max(0, issued - kDwStages); it < issued; ++it)
-                    mbar_wait_bounded(&full_bar[it % kDwStages], static_cast<uint32_t>(it / kDwStages) & 1u);
+                for (int it = std::max(0, issued - kStages); it < issued; ++it)
+                    mbar_wait_bounded(&full_bar[it % kStages], static_cast<uint32_t>(it / kStages) & 1u);
             }
         }
     } else if (warp == kDwMma) {
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(128, 128, 1u, true, true);
+            const uint32_t idesc = instr_desc(128, kNCols, 1u, true, true);
             bool ok = true;
             RingPos rp;
-            for (int it = 0; it < ntiles; ++it, rp.next(kDwStages)) {
+            for (int it = 0; it < ntiles; ++it, rp.next(kStages)) {
                 const int s = rp.slot;
                 if (!mbar_wait_bounded(&ready_bar[s], rp.phase)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t xb = smem_u32(smem + static_cast<size_t>(s) * kDwStage);
-                const uint32_t bb = xb + kDwXBytes + kDwZBytes;
+                const uint32_t xb = smem_u32(smem + static_cast<size_t>(s) * kStageBytes);
+                const uint32_t bb = xb + kDwXBytes + kZBytes;
 #pragma unroll
                 for (int ks = 0; ks < kDwRows / 16; ++ks) {
                     const uint32_t off = ks * 16 * 128;
@@ -2050,27 +2094,41 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
         // ---------------- warps 0-7: dZ float32 -> bf16 (zero past the range) ----------
         bool ok = true;
         RingPos rp;
-        for (int it = 0; it < ntiles && ok; ++it, rp.next(kDwStages)) {
+        for (int it = 0; it < ntiles && ok; ++it, rp.next(kStages)) {
             const int s = rp.slot;
             // the warp agrees on the outcome, so it stays converged for its arrival
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], rp.phase))) {
                 ok = false;
                 break;
             }
-            const uint8_t *z = smem + static_cast<size_t>(s) * kDwStage + kDwXBytes;
-            uint8_t *bt = smem + static_cast<size_t>(s) * kDwStage + kDwXBytes + kDwZBytes;
+            const uint8_t *z = smem + static_cast<size_t>(s) * kStageBytes + kDwXBytes;
+            uint8_t *bt = smem + static_cast<size_t>(s) * kStageBytes + kDwXBytes + kZBytes;
             const int64_t y0 = r0 + static_cast<int64_t>(it) * kDwRows;
             if constexpr (DSZ) {
                 // phi of the q tile in place (rows past the range meet zero dZ rows)
-                uint4 *xq = reinterpret_cast<uint4 *>(smem + static_cast<size_t>(s) * kDwStage);
+                uint4 *xq = reinterpret_cast<uint4 *>(smem + static_cast<size_t>(s) * kStageBytes);
                 for (int cidx = threadIdx.x; cidx < static_cast<int>(kDwXBytes / 16); cidx += kDwWorkers) {
                     const uint4 u = xq[cidx];
                     xq[cidx] = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
                 }
             }
-            // one 16-byte chunk of the bf16 tile (8 consecutive columns of one row) per step
-            for (int cidx = threadIdx.x; cidx < kDwRows * 16; cidx += kDwWorkers) {
-                const int k = cidx >> 4, ch = cidx & 15;
+            // one 16-byte chunk of the bf16 tile (8 consecutive columns of one row) per step;
+            // with DSZ two more per row carry the dden columns into the third atom
+            constexpr int kChunks = DSZ ? 18 : 16;
+            for (int cidx = threadIdx.x; cidx < kDwRows * kChunks; cidx += kDwWorkers) {
+                const int k = cidx / kChunks, ch = cidx - k * kChunks;
+                if (DSZ && ch >= 16) {
+                    const int co = ch - 16;
+                    uint4 w = make_uint4(0, 0, 0, 0);
+                    if (y0 + k < r1) {
+                        const float4 *dr = reinterpret_cast<const float4 *>(z + kDwZBytes + k * 64 + co * 32);
+                        const float4 a = dr[0], b = dr[1];
+                        w = make_uint4(bf16x2_bits(a.x, a.y), bf16x2_bits(a.z, a.w), bf16x2_bits(b.x, b.y),
+                                       bf16x2_bits(b.z, b.w));
+                    }
+                    *reinterpret_cast<uint4 *>(bt + 2 * kDwBox + k * 128 + ((co ^ (k & 7)) * 16)) = w;
+                    continue;
+                }
                 const int bo = ch >> 3, co = ch & 7;            // bf16 box, chunk in its row
                 const int g0 = bo * 64 + co * 8;                // first column in the tile
                 const int bi = g0 >> 5, j0 = (g0 & 31) >> 2;    // float32 box, its first chunk
@@ -2103,7 +2161,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
         const int a = fa * 128 + warp * 32 + lane;         // TMEM lane = input feature
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         if constexpr (DSZ) {
-            // feature a = h R + al: its head's block row (block fb = 0) or its dz (fb = 1)
+            // feature a = h R + al: its head's block row (columns h R ..) and its dz (column D + h)
             const int h = a / p.R, al = a - h * p.R;
             float *dst = p.part + ((static_cast<int64_t>(part) * p.H + h) * p.R + al) * (p.R + 1);
 #pragma unroll
@@ -2114,12 +2172,19 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
                 if (a < p.d) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int col = q * 32 + j;       // column within the 128-column block
-                        if (fb == 0 && col / p.R == h) dst[col - h * p.R] = have ? __uint_as_float(v[j]) : 0.f;
-                        if (fb == 1 && col == h) dst[p.R] = have ? __uint_as_float(v[j]) : 0.f;
+                        const int col = q * 32 + j;
+                        if (col / p.R == h) dst[col - h * p.R] = have ? __uint_as_float(v[j]) : 0.f;
                     }
                 }
             }
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_base + p.d, v);
+            tmem_ld_wait();
+            float dz = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (j == h) dz = __uint_as_float(v[j]);
+            if (a < p.d) dst[p.R] = have ? dz : 0.f;
         } else {
         float *dst = p.part + (static_cast<int64_t>(part) * p.d + a) * p.Kc;
 #pragma unroll
@@ -2140,7 +2205,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
     __syncthreads();
     if (warp == kDwMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128u);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -2175,10 +2240,10 @@ glga_status tc_gemms(Ctx *c, const void *X, float *dX, cudaStream_t s) {
                                    static_cast<int>(smem)));
     const dim3 grid(static_cast<unsigned>(c->bw_dwtc_parts), static_cast<unsigned>(ceil_div(d, 128)),
                     static_cast<unsigned>(ceil_div(Kc, 128)));
-    bwd_dw_tc_kernel<false><<<grid, kDwThreads, smem, s>>>(mx, mz, p);
+    bwd_dw_tc_kernel<false><<<grid, kDwThreads, smem, s>>>(mx, mz, mz, p);
     GLGA_CUDA(cudaGetLastError());
     const int64_t total = static_cast<int64_t>(d) * Kc;
-    bwd_sum_parts_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 4096)), 256, 0, s>>>(
+    bwd_sum_parts_kernel<<<sum_parts_grid(total), kSumThreads, 0, s>>>(
         c->bw_dwtc_part, c->bw_dwtc_parts, total, c->bw_dW3);
     GLGA_CUDA(cudaGetLastError());
     return gemm_nt_f32out(c, GLGA_F32, c->bw_dZ, N, c->bw_dz_ld, c->bw_Wall, d, c->bw_dz_ld, Kc + 1, dX, d, s);
@@ -2507,7 +2572,7 @@ bool bwd_fx(const Ctx *c) {
     return c->io == GLGA_BF16 && c->d == 128 && c->D % 64 == 0 && c->D <= 128 && c->N > 0;
 }
 
-// dX, and the dW / dw_g / db_g partials that bwd_dw_reduce_kernel and bwd_dbg_kernel add
+// dX, and the dW / dw_g / db_g partials that the reductions after it add
 // (over c->bw_fx_parts blocks), in one pass over dZ.
 glga_status fx_gemms(Ctx *c, const void *X, const void *WQ, const void *WK, const void *WV, const void *wg,
                      float *dX, cudaStream_t s) {
@@ -2544,7 +2609,7 @@ glga_status fx_gemms(Ctx *c, const void *X, const void *WQ, const void *WK, cons
     bwd_dxdw_tc_kernel<<<static_cast<unsigned>(c->bw_fx_parts), kFxThreads, kFxSmem, s>>>(mx, mz, mdt, mq, mk, mv, p);
     GLGA_CUDA(cudaGetLastError());
     const int64_t total = 128 * Kc;
-    bwd_sum_parts_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(total, 256), 4096)), 256, 0, s>>>(
+    bwd_sum_parts_kernel<<<sum_parts_grid(total), kSumThreads, 0, s>>>(
         c->bw_dwtc_part, c->bw_fx_parts, total, c->bw_dW3);
     GLGA_CUDA(cudaGetLastError());
     return GLGA_OK;
@@ -2558,12 +2623,16 @@ glga_status launch_dsz_bwd(Ctx *c, const T *Q, cudaStream_t s) {
         if (readout_bwd_tc(c)) {
             // tcgen05: X = Q [N][D] (phi applied per tile), dZ = [dnum | dden] [N][D + 16]
             const int64_t N = c->N, D = c->D;
-            CUtensorMap mx, mz;
+            CUtensorMap mx, mz, md;
             glga_status st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, static_cast<uint64_t>(D),
                                             static_cast<uint64_t>(N), static_cast<uint64_t>(D) * 2, 64, kDwRows);
             if (st == GLGA_OK)
                 st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dnum, static_cast<uint64_t>(D + 16),
                                     static_cast<uint64_t>(N), static_cast<uint64_t>(D + 16) * 4, 32, kDwRows);
+            if (st == GLGA_OK)   // the 16 dden columns: [64][16] float boxes, no swizzle
+                st = encode_tmap_2d(&md, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dnum, static_cast<uint64_t>(D + 16),
+                                    static_cast<uint64_t>(N), static_cast<uint64_t>(D + 16) * 4, 16, kDwRows,
+                                    CU_TENSOR_MAP_SWIZZLE_NONE);
             if (st != GLGA_OK) return st;
             DwParams p;
             p.N = N;
@@ -2574,11 +2643,10 @@ glga_status launch_dsz_bwd(Ctx *c, const T *Q, cudaStream_t s) {
             p.flag = c->dev_flag;
             p.H = c->H;
             p.R = c->r;
-            const size_t smem = static_cast<size_t>(kDwStages) * kDwStage + 1024;
+            const size_t smem = static_cast<size_t>(kDszStages) * kDszStage + 1024;
             GLGA_CUDA(cudaFuncSetAttribute(bwd_dw_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem)));
-            bwd_dw_tc_kernel<true><<<dim3(static_cast<unsigned>(c->bw_dsz_parts), 1, 2), kDwThreads, smem, s>>>(
-                mx, mz, p);
+            bwd_dw_tc_kernel<true><<<static_cast<unsigned>(c->bw_dsz_parts), kDwThreads, smem, s>>>(mx, mz, md, p);
             GLGA_CUDA(cudaGetLastError());
             return GLGA_OK;
         }
@@ -2643,8 +2711,8 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_Dd), nz * H * f));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dZ), nz * c->bw_dz_ld * f));
     if (readout_bwd_tc(c)) {
-        // 64-row-aligned ranges, one thread block per SM over the ranges x {dnum, dden} grid
-        c->bw_dsz_rpp = ceil_div(ceil_div(N, std::max<int64_t>(1, c->num_sms / 2)), kDwRows) * kDwRows;
+        // 64-row-aligned ranges, one thread block per SM
+        c->bw_dsz_rpp = ceil_div(ceil_div(N, std::max<int64_t>(1, c->num_sms)), kDwRows) * kDwRows;
     } else {
         c->bw_dsz_rpp = ceil_div(std::max<int64_t>(N, 1), c->bw_parts);
     }
@@ -2762,7 +2830,7 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
                 const glga_status ds = launch_dsz_bwd<T>(c, Q, c->bw_side);                               \
                 if (ds != GLGA_OK) return ds;                                                             \
             }                                                                                             \
-            bwd_sum_parts_kernel<<<static_cast<unsigned>(ceil_div(total, 256)), 256, 0, c->bw_side>>>(   \
+            bwd_sum_parts_kernel<<<sum_parts_grid(total), kSumThreads, 0, c->bw_side>>>(                 \
                 c->bw_dsz_part, c->bw_dsz_parts, total, c->bw_dSz);                                       \
             bwd_heads_prep_kernel<<<tgrid, 256, 0, c->bw_side>>>(c->bw_dSz, R + 1, H, R, c->bw_dST,      \
                                                                 c->bw_dSc);                               \
@@ -2807,9 +2875,13 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
 #undef BWD_LAUNCHES
     if (N > 0) {
         const int wp = bwd_fx(c) ? c->bw_fx_parts : c->bw_wparts;   // partials of dw_g (and dW)
+        const bool tcg = bwd_tc_gemms(c);
         bwd_dw_reduce_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(wtotal, 256), 4096)), 256, 0, s>>>(
-            c->bw_dw_part, wp, bwd_tc_gemms(c) ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
-        bwd_dbg_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, wp, db_g);
+            c->bw_dw_part, wp, tcg ? c->bw_dW3 : nullptr, d, D, Dc, dWQ, dWK, dWV, dwg);
+        if (tcg)   // dw_g: column 3D of the partials, one warp per feature
+            bwd_strided_sum_kernel<<<static_cast<unsigned>(ceil_div(d, 8)), 256, 0, s>>>(
+                c->bw_dw_part + 3 * D, wp, static_cast<int64_t>(d) * Dc, Dc, d, dwg);
+        bwd_strided_sum_kernel<<<1, 32, 0, s>>>(c->bw_dbg_part, wp, 1, 0, 1, db_g);
     } else {
         GLGA_CUDA(cudaMemsetAsync(dWQ, 0, static_cast<size_t>(d) * D * sizeof(float), s));
         GLGA_CUDA(cudaMemsetAsync(dWK, 0, static_cast<size_t>(d) * D * sizeof(float), s));
