@@ -134,6 +134,39 @@ __device__ __forceinline__ void st_mrow(float *p, const float (&x)[EPL]) {
     }
 }
 
+// p[0 .. EPL-1] = x rounded to T, for a row slice on an EPL-element boundary.
+template <typename T, int EPL>
+__device__ __forceinline__ void st_row(T *p, const float (&x)[EPL]) {
+    if constexpr (std::is_same<T, float>::value) {
+        st_mrow<EPL>(p, x);
+    } else if constexpr (EPL == 1) {
+        p[0] = __float2bfloat16_rn(x[0]);
+    } else {
+        uint32_t w[EPL / 2];
+#pragma unroll
+        for (int e = 0; e < EPL / 2; ++e) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        if constexpr (EPL % 8 == 0) {
+#pragma unroll
+            for (int v = 0; v < EPL / 8; ++v)
+                reinterpret_cast<uint4 *>(p)[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        } else if constexpr (EPL == 4) {
+            *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
+        } else {
+            *reinterpret_cast<uint32_t *>(p) = w[0];
+        }
+    }
+}
+
+// x as a T row stores it.
+template <typename T>
+__device__ __forceinline__ float round_to(float x) {
+    if constexpr (std::is_same<T, float>::value) return x;
+    else return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ float head_reduce(float x, int lph) {
     for (int o = 1; o < lph; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
@@ -199,7 +232,7 @@ template <typename T, int EPL, int LPH, int RPW>
 __global__ void __launch_bounds__(256, EPL <= 8 ? 2 : 1) bwd_readout_kernel(
     const T *__restrict__ Q, const T *__restrict__ L, const float *__restrict__ t, const float *__restrict__ Sz,
     const float *__restrict__ ST, const T *__restrict__ dY, int64_t N, int H, int R, float b_g, float eps,
-    float *__restrict__ dL, float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden,
+    T *__restrict__ dL, float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden,
     float *__restrict__ dZ, int64_t dz_ld) {
     const int64_t i0 = ((blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5) * RPW;
     const int lane = threadIdx.x & 31;
@@ -244,16 +277,16 @@ __global__ void __launch_bounds__(256, EPL <= 8 ? 2 : 1) bwd_readout_kernel(
 #pragma unroll
         for (int x = 0; x < EPL; ++x) {
             G[k][x] *= inv_den;
-            dLL = fmaf(g * dy[k][x], lv[k][x], dLL);
+            gl[x] = round_to<T>(g * dy[k][x]);            // dL as stored; D_i from the same values
+            dLL = fmaf(gl[x], lv[k][x], dLL);
             dgp[k] = fmaf(dy[k][x], lv[k][x] - G[k][x], dgp[k]);
             const float dG = (1.f - g) * dy[k][x];
             dGG = fmaf(dG, G[k][x], dGG);
-            gl[x] = g * dy[k][x];
             dn[k][x] = dG * inv_den;
         }
         const int64_t o = i * D + lane * EPL;
         if (lh.act && live[k]) {
-            st_mrow<EPL>(dL + o, gl);
+            st_row<T, EPL>(dL + o, gl);
             st_mrow<EPL>(dnum + o, dn[k]);
         }
         const float dd = -head_reduce(dGG, lph) * inv_den;
@@ -492,7 +525,7 @@ template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_local_q_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
-    const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
     const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
     const int lane = threadIdx.x & 31;
     const int64_t slot = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -504,7 +537,7 @@ __global__ void __launch_bounds__(256) bwd_local_q_kernel(
     if (r0 == r1) return;                                 // no local term
     float q[EPL], dl[EPL];
     ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
-    ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
+    ld_row<T, EPL>(dL + i * D, lane, lh.act, dl);
     const float ls = __ldg(lse + i * H + lh.h), dd = __ldg(Dd + i * H + lh.h);
     float dq[EPL];
 #pragma unroll
@@ -536,7 +569,7 @@ template <typename T, int EPL>
 __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
-    const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
     const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
@@ -550,7 +583,7 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     const int lph2 = R / EPL2, h2 = act2 ? hl * EPL2 / R : 0;
     float q2[EPL2], dl2[EPL2], dq2[EPL2];
     ld_row<T, EPL2>(Q + i * D, hl, act2, q2);
-    ld_row<float, EPL2>(dL + i * D, hl, act2, dl2);
+    ld_row<T, EPL2>(dL + i * D, hl, act2, dl2);
     const float ls = __ldg(lse + i * H + h2), dd = __ldg(Dd + i * H + h2);
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dq2[x] = 0.f;
@@ -659,7 +692,7 @@ template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
     const int2 *__restrict__ chunks, int64_t n_chunks, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
-    const float *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
     const float *__restrict__ Dd, float *__restrict__ part) {
     const int lane = threadIdx.x & 31;
     const int64_t c = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -671,7 +704,7 @@ __global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
     const LaneHead lh(lane, EPL, D, R);
     float q[EPL], dl[EPL], dq[EPL];
     ld_row<T, EPL>(Q + i * D, lane, lh.act, q);
-    ld_row<float, EPL>(dL + i * D, lane, lh.act, dl);
+    ld_row<T, EPL>(dL + i * D, lane, lh.act, dl);
 #pragma unroll
     for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
     const float ls = __ldg(lse + i * H + lh.h), dd = __ldg(Dd + i * H + lh.h);
@@ -740,7 +773,7 @@ __global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
 
 // dk, dv += the terms of targets [a, b) of source row j (this warp's lanes).
 template <typename T, int EPL>
-__device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, const float *dL,
+__device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, const T *dL,
                                               const float *lse, const float *Dd, int H, int D, int lane,
                                               bool act, int lph, int h, float inv_sqrt_r, const float (&k)[EPL],
                                               const float (&v)[EPL], int32_t a, int32_t b, float (&dk)[EPL],
@@ -752,7 +785,7 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
             const bool live = e + u < b;
             const int64_t i = live ? t_col[e + u] : 0;
             ld_row<T, EPL>(Q + i * D, lane, act && live, q[u]);
-            ld_row<float, EPL>(dL + i * D, lane, act && live, dl[u]);
+            ld_row<T, EPL>(dL + i * D, lane, act && live, dl[u]);
             ls[u] = live ? __ldg(lse + i * H + h) : 0.f;
             dd[u] = live ? __ldg(Dd + i * H + h) : 0.f;
         }
@@ -836,7 +869,7 @@ template <typename T, int EPL, bool PARTS, bool GTC = false>
 __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const int32_t *__restrict__ chunk_ptr, const float *__restrict__ part,
-    const T *__restrict__ Q, const T *__restrict__ KV, const float *__restrict__ dL,
+    const T *__restrict__ Q, const T *__restrict__ KV, const T *__restrict__ dL,
     const float *__restrict__ lse, const float *__restrict__ Dd, const float *__restrict__ dSc,
     const float *__restrict__ dST, int H, int R, float inv_sqrt_r, float *__restrict__ dZ, int64_t dz_ld) {
     extern __shared__ float msm[];                       // PARTS: [kMW][2D]
@@ -915,7 +948,7 @@ template <typename T, int EPL, bool GTC = false>
 __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
-    const float *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
+    const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
     const float *__restrict__ dSc, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
     float *__restrict__ dZ, int64_t dz_ld) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
@@ -963,7 +996,7 @@ __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
             const bool live = e < b;
             const int64_t i = live ? t_col[e] : 0;
             ld_row<T, EPL2>(Q + i * D, hl, act2 && live, q[u]);
-            ld_row<float, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
+            ld_row<T, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
             ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
             dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
         }
@@ -1014,7 +1047,7 @@ template <typename T, int EPL>
 __global__ void __launch_bounds__(256) bwd_kv_chunk_kernel(
     const int2 *__restrict__ chunks, int64_t n_chunks, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
-    const float *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd, int H, int R,
+    const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd, int H, int R,
     float inv_sqrt_r, float *__restrict__ part) {
     const int lane = threadIdx.x & 31;
     const int64_t c = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -1303,19 +1336,19 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     if constexpr (E == 4 && sizeof(T) == 2) {
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
             bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz);
             return;
         }
     }
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
             return;
         }
     }
     bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-        nullptr, nullptr, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+        nullptr, nullptr, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
 }
 
 // Light target rows: two edges per warp step under the same condition as the source side.
@@ -1328,12 +1361,12 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
                 cudaFuncSetAttribute(bwd_local_q2_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kQRingBytes));
             bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
-                Q, KV, c->bw_dL, c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
             return;
         }
     }
     bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx, Q, KV,
-        c->bw_dL, c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
+        static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
 }
 
 // Heavy source rows: chunk sums, then the global terms (or, with the tensor-core global
@@ -1346,7 +1379,7 @@ void launch_kv_heavy(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, con
         if (sm > 48 * 1024)
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
         kern<<<static_cast<unsigned>(nkh), kMW * 32, sm, sk>>>(kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr,
-                                                               c->bw_kv_part, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd,
+                                                               c->bw_kv_part, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd,
                                                                dSc, dST, c->H, c->r, isr, c->bw_dZ, Dz);
     };
     if constexpr (E == 4 && sizeof(T) == 2) {
@@ -1372,13 +1405,13 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
         if (nkl) launch_kv_light<T, E>(c, Q, KV, isr, Dz, sk);                                           \
         if (nkh) {                                                                                        \
             bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, sk>>>(c->bw_k_chunks, nkc, c->t_row_ptr,   \
-                c->t_col, Q, KV, c->bw_dL, c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
+                c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
             launch_kv_heavy<T, E>(c, Q, KV, isr, Dz, kh, nkh, sk);                                      \
         }                                                                                                 \
         if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                            \
         if (nqh) {                                                                                        \
             bwd_q_chunk_kernel<T, E><<<warp_grid(nqc), 256, 0, sq>>>(c->bw_q_chunks, nqc, c->row_ptr,      \
-                c->col_idx, Q, KV, c->bw_dL, H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);               \
+                c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);               \
             bwd_q_heavy_kernel<E><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, sq>>>(qh, nqh,      \
                 c->bw_q_cptr, c->bw_q_part, H, R, c->bw_dZ, Dz);                                          \
         }                                                                                                 \
@@ -1469,11 +1502,31 @@ __device__ __forceinline__ void warp_rows_f32_flush(float *dst, int64_t ld, int6
     __syncwarp();
 }
 
+// The lane's 32 bf16 values (its row, columns c0 .. c0 + 31) to a row-major bf16 matrix:
+// four 16-byte pieces into the staging area (row r at byte r * 64, piece p at slot
+// p ^ ((r >> 1) & 3)), then four coalesced stores of 8 rows x 64 B.  Rows at or past N are
+// not written.
+__device__ __forceinline__ void stage_bf16_piece(uint8_t *stage, int lane, int p, uint4 v) {
+    *reinterpret_cast<uint4 *>(stage + lane * 64 + ((p ^ ((lane >> 1) & 3)) << 4)) = v;
+}
+__device__ __forceinline__ void warp_rows_bf16_flush(__nv_bfloat16 *dst, int64_t ld, int64_t r0, int64_t N,
+                                                     int c0, uint8_t *stage, int lane) {
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 8 * i + (lane >> 2), p = lane & 3;
+        const int64_t gr = r0 + r;
+        const uint4 x = *reinterpret_cast<const uint4 *>(stage + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
+        if (gr < N) reinterpret_cast<uint4 *>(dst + gr * ld + c0)[p] = x;
+    }
+    __syncwarp();
+}
+
 template <int R>
 __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
     const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ L, const float *__restrict__ t,
     const __nv_bfloat16 *__restrict__ Bg, int ro_kp, const float *__restrict__ Sz,
-    const __nv_bfloat16 *__restrict__ dY, int64_t N, int H, float b_g, float eps, float *__restrict__ dL,
+    const __nv_bfloat16 *__restrict__ dY, int64_t N, int H, float b_g, float eps, __nv_bfloat16 *__restrict__ dL,
     float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ,
     int64_t dz_ld, unsigned *flag) {
     constexpr int D = kBroTcD;
@@ -1596,18 +1649,22 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
         uint4 yw[4], lw[4];
         warp_rows_bf16(dY, D, r0, N, c0, stg, lane, yw);
         warp_rows_bf16(L, D, r0, N, c0, stg, lane, lw);
+        // dL = g dY stored in bf16, and D_i from the stored values
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            float v[4];
+        for (int p = 0; p < 4; ++p) {
+            uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int j = 4 * p + e, hq = j / R < kHQ ? j / R : 0;
-                v[e] = g * bf(yw, j);
-                Dda[hq] = fmaf(v[e], bf(lw, j), Dda[hq]);
+                const int j = 8 * p + 2 * e, hq = j / R < kHQ ? j / R : 0;
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(g * bf(yw, j), g * bf(yw, j + 1));
+                const float2 v = __bfloat1622float2(h2);
+                Dda[hq] = fmaf(v.x, bf(lw, j), Dda[hq]);
+                Dda[hq] = fmaf(v.y, bf(lw, j + 1), Dda[hq]);
+                w[e] = *reinterpret_cast<const uint32_t *>(&h2);
             }
-            stage_f32_piece(stg, lane, p, v[0], v[1], v[2], v[3]);
+            stage_bf16_piece(stg, lane, p, make_uint4(w[0], w[1], w[2], w[3]));
         }
-        warp_rows_f32_flush(dL, D, r0, N, c0, stg, lane);
+        warp_rows_bf16_flush(dL, D, r0, N, c0, stg, lane);
         float dtp = 0.f;
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {           // 16 columns at a time
@@ -1872,7 +1929,7 @@ void launch_readout_bwd_e(Ctx *c, const T *Q, const T *dY, float b_g, float eps,
     constexpr int kRpw = EPL <= 4 ? 2 : 1;
     const unsigned grid = static_cast<unsigned>(ceil_div(ceil_div(c->N, kRpw) * 32, 256));
     bwd_readout_kernel<T, EPL, LPH, kRpw><<<grid, 256, 0, s>>>(Q, static_cast<const T *>(c->L), c->t, c->Sz,
-                                                               c->bw_ST, dY, c->N, c->H, c->r, b_g, eps, c->bw_dL,
+                                                               c->bw_ST, dY, c->N, c->H, c->r, b_g, eps, static_cast<T *>(c->bw_dL),
                                                                c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz);
 }
 
@@ -1892,7 +1949,7 @@ void launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *
                          static_cast<int>(kBroTcSmem));
     bwd_readout_tc_kernel<R><<<grid, kBroTcWarps * 32, kBroTcSmem, s>>>(
         Q, static_cast<const __nv_bfloat16 *>(c->L), c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz,
-        dY, c->N, c->H, b_g, eps, c->bw_dL, c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz, c->dev_flag);
+        dY, c->N, c->H, b_g, eps, static_cast<__nv_bfloat16 *>(c->bw_dL), c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz, c->dev_flag);
 }
 
 // The readout backward runs on the tensor cores for bf16 layers with H*r = 128, r in
@@ -2698,7 +2755,7 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
         if (e != cudaSuccess) st = cuda_fail(e, "backward side stream");
     }
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->t_col), std::max<int64_t>(E, 1) * sizeof(int32_t)));
-    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dL), nz * D * f));
+    BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dL), nz * D * c->elem));
     // [dnum | dden] rows of D + 16 columns (dden_h in column D + h) for the tensor-core dS | dz;
     // dnum rows of D columns and dden [N, H] on the other paths
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dnum), nz * (D + 16) * f));

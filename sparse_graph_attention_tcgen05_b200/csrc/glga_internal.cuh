@@ -132,7 +132,8 @@ struct Ctx {
 
     // backward pass workspaces (opts.backward)
     int32_t *t_row_ptr = nullptr, *t_col = nullptr;   // transposed CSR: rows by source
-    float *bw_dL = nullptr, *bw_dnum = nullptr;       // [N, D]
+    void *bw_dL = nullptr;                            // [N, D] in the io type
+    float *bw_dnum = nullptr;                         // [N, D + 16]
     float *bw_dden = nullptr, *bw_dg = nullptr, *bw_lse = nullptr, *bw_Dd = nullptr;   // [N, H]
     float *bw_dZ = nullptr;                           // [N, 3D + 1]: dQ | dK | dV | dt
     float *bw_dsz_part = nullptr, *bw_dSz = nullptr;  // dS | dz partials and sum
