@@ -1762,29 +1762,33 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
 //   G_v = phi(K) blockdiag(dS_h)    (tcgen05: dv_jf = sum_c dS_h[c][f] phi(k_jc))
 //   dZ[j, D + f] = (G_k + dz_f) phi'(k_jf),   dZ[j, 2D + f] = G_v
 // written before the source-side gather kernels, which then add their local terms.
-// Layout and row I/O as bwd_readout_tc_kernel (16 warps, 32 rows x 32 columns each).
-constexpr size_t kKvgSmem = 1024 + 4 * 2 * kBroTcAtom + kBroTcWarps * kBroTcStage + kBroTcD * 4;
+// 16 warps, each with 32 rows x 32 columns of the epilogue; the block's tiles stream in by
+// TMA (K | V rows, two stages: the next tile lands while this one is multiplied and
+// written), and a landed stage, once read, stages the warps' coalesced row stores.
+constexpr int kKvgStages = 2;
+constexpr uint32_t kKvgStage = 4 * kBroTcAtom;     // the K tile (2 atoms), then the V tile
+constexpr size_t kKvgSmem = 1024 + kKvgStages * kKvgStage + 6 * kBroTcAtom + kBroTcD * 4;
+static_assert(kBroTcWarps * kBroTcStage <= kKvgStage, "a landed stage doubles as the output staging");
 
 template <int R>
 __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
-    const __nv_bfloat16 *__restrict__ KV, const float *__restrict__ dSc, int64_t N, int H, float *__restrict__ dZ,
-    int64_t dz_ld, unsigned *flag) {
+    const __grid_constant__ CUtensorMap tmKV, const float *__restrict__ dSc, int64_t N, int H,
+    float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
     constexpr int D = kBroTcD;
     extern __shared__ uint8_t kvg_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kKvgStages];
     __shared__ __align__(8) uint64_t mma_bar;
     __shared__ uint32_t tmem_sh;
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(kvg_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t *sV = sm;                              // A of the first MMA: V, 2 atoms
-    uint8_t *sP = sV + 2 * kBroTcAtom;             // A of the second: phi(K)
-    uint8_t *sB1 = sP + 2 * kBroTcAtom;            // blockdiag(dS_h)^T as [f][c] = dS_h[f][c]
-    uint8_t *sB2 = sB1 + 2 * kBroTcAtom;           // blockdiag(dS_h) as [f][c] = dS_h[c][f]
-    uint8_t *stg_all = sB2 + 2 * kBroTcAtom;
-    float *dzf = reinterpret_cast<float *>(stg_all + kBroTcWarps * kBroTcStage);
+    uint8_t *sS = sm;                                          // [kKvgStages] K | V tiles (TMA)
+    uint8_t *sP = sS + kKvgStages * kKvgStage;                 // A of the second MMA: phi(K)
+    uint8_t *sB1 = sP + 2 * kBroTcAtom;                        // blockdiag(dS_h)^T as [f][c] = dS_h[f][c]
+    uint8_t *sB2 = sB1 + 2 * kBroTcAtom;                       // blockdiag(dS_h) as [f][c] = dS_h[c][f]
+    float *dzf = reinterpret_cast<float *>(sB2 + 2 * kBroTcAtom);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, cq = warp >> 2;
     const int rt = quad * 32 + lane;
     const int c0 = cq * 32;
-    uint8_t *stg = stg_all + warp * kBroTcStage;
     const float *dz = dSc + static_cast<int64_t>(H) * R * R;
     for (int ch = tid; ch < D * (D / 8); ch += blockDim.x) {
         const int f = ch / (D / 8), c8 = (ch % (D / 8)) * 8;
@@ -1803,9 +1807,23 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
             make_uint4(bf16x2_bits(v2[0], v2[1]), bf16x2_bits(v2[2], v2[3]), bf16x2_bits(v2[4], v2[5]), bf16x2_bits(v2[6], v2[7]));
     }
     for (int f = tid; f < D; f += blockDim.x) dzf[f] = dz[f];
+    const int64_t n_tiles = ceil_div(N, 128);
+    const int my = blockIdx.x < n_tiles ? static_cast<int>((n_tiles - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+    // the K | V rows of this block's k-th tile into stage k % 2
+    auto issue = [&](int k) {
+        const int s = k % kKvgStages;
+        const int32_t y = static_cast<int32_t>((blockIdx.x + static_cast<int64_t>(k) * gridDim.x) * 128);
+        uint8_t *st = sS + s * kKvgStage;
+        mbar_arrive_expect_tx(&full_bar[s], kKvgStage);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(st + b * kBroTcAtom, &tmKV, &full_bar[s], b * 64, y);
+    };
     if (tid == 0) {
+        for (int s = 0; s < kKvgStages; ++s) mbar_init(&full_bar[s], 1);
         mbar_init(&mma_bar, 1);
         fence_mbar_init();
+        tma_prefetch_desc(&tmKV);
+        for (int k = 0; k < my && k < kKvgStages; ++k) issue(k);
     }
     fence_proxy_async_smem();
     if (warp == 0) {
@@ -1818,24 +1836,24 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
     const uint32_t tmem = tmem_sh;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t idesc = instr_desc(128, D, 1u, false, false);
-    const int64_t n_tiles = ceil_div(N, 128);
-    uint32_t phase = 0;
     auto bf = [](const uint4 (&w)[4], int j) {
         const uint32_t word = (&w[j / 8].x)[(j % 8) / 2];
         return __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16));
     };
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t r0 = tile * 128 + quad * 32;
-        {
-            uint4 kw[4], vw[4];
-            warp_rows_bf16(KV + D, 2 * D, r0, N, c0, stg, lane, vw);
-            warp_rows_bf16(KV, 2 * D, r0, N, c0, stg, lane, kw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                *reinterpret_cast<uint4 *>(sV + swz_off(rt, c0 + 8 * i, kBroTcAtom)) = vw[i];
-                *reinterpret_cast<uint4 *>(sP + swz_off(rt, c0 + 8 * i, kBroTcAtom)) =
-                    make_uint4(phi_bf16x2(kw[i].x), phi_bf16x2(kw[i].y), phi_bf16x2(kw[i].z), phi_bf16x2(kw[i].w));
-            }
+    int k = 0;
+    for (; k < my; ++k) {
+        const int s = k % kKvgStages;
+        uint8_t *sK = sS + s * kKvgStage, *sV = sK + 2 * kBroTcAtom;
+        const bool got = mbar_wait_bounded(&full_bar[s], static_cast<uint32_t>(k / kKvgStages) & 1u);
+        if (__syncthreads_or(!got)) {
+            if (tid == 0) atomicOr(flag, kDevErrTimeout);
+            break;
+        }
+        // phi(K) into the second MMA's A operand: elementwise, so at the same byte offsets
+        for (int ch = tid; ch < static_cast<int>(2 * kBroTcAtom / 16); ch += blockDim.x) {
+            const uint32_t off = static_cast<uint32_t>(ch) * 16u;
+            const uint4 u = *reinterpret_cast<const uint4 *>(sK + off);
+            *reinterpret_cast<uint4 *>(sP + off) = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1852,16 +1870,19 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
             }
             umma_commit(&mma_bar);
         }
-        const bool got = mbar_wait_bounded(&mma_bar, phase);
-        phase ^= 1u;
-        if (__syncthreads_or(!got)) {
+        // the warp's k slice (rows rt, columns c0 .. c0 + 31) for phi'(k)
+        uint4 kw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) kw[i] = *reinterpret_cast<const uint4 *>(sK + swz_off(rt, c0 + 8 * i, kBroTcAtom));
+        const bool done = mbar_wait_bounded(&mma_bar, static_cast<uint32_t>(k) & 1u);
+        if (__syncthreads_or(!done)) {   // also: every warp holds its k slice, the stage is free
             if (tid == 0) atomicOr(flag, kDevErrTimeout);
             break;
         }
         tc_fence_after();
+        uint8_t *stg = sK + warp * kBroTcStage;
         // dk: (G_k + dz) phi'(k); dv: G_v
-        uint4 kw[4];
-        warp_rows_bf16(KV, 2 * D, r0, N, c0, stg, lane, kw);
+        const int64_t r0 = (blockIdx.x + static_cast<int64_t>(k) * gridDim.x) * 128 + quad * 32;
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
             uint32_t a[16];
@@ -1890,9 +1911,15 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
                                 __uint_as_float(a[4 * p + 2]), __uint_as_float(a[4 * p + 3]));
         }
         warp_rows_f32_flush(dZ + 2 * D, dz_ld, r0, N, c0, stg, lane);
+        fence_proxy_async_smem();   // the staging writes come before the stage's next TMA load
         tc_fence_before();
-        __syncthreads();   // TMEM and the A operands are rewritten by the next tile
+        __syncthreads();            // TMEM, phi(K) and the stage are free
+        if (tid == 0 && k + kKvgStages < my) issue(k + kKvgStages);
     }
+    // the block leaves only after its copies have landed (already so when all went well)
+    if (tid == 0)
+        for (int kk = k; kk < my && kk < k + kKvgStages; ++kk)
+            mbar_wait_bounded(&full_bar[kk % kKvgStages], static_cast<uint32_t>(kk / kKvgStages) & 1u);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1908,18 +1935,23 @@ bool kv_global_tc(const Ctx *c) {
 }
 
 template <int R>
-void launch_kv_global_r(Ctx *c, int64_t Dz, cudaStream_t s) {
+glga_status launch_kv_global_r(Ctx *c, int64_t Dz, cudaStream_t s) {
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(c->N, 128), c->num_sms));
     cudaFuncSetAttribute(bwd_kv_global_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kKvgSmem));
-    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(
-        static_cast<const __nv_bfloat16 *>(c->KV), c->bw_dSc, c->N, c->H, c->bw_dZ, Dz, c->dev_flag);
+    CUtensorMap m;
+    const glga_status st = encode_tmap_2d(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->KV, 2 * kBroTcD,
+                                          static_cast<uint64_t>(c->N), 4 * kBroTcD, 64, 128);
+    if (st != GLGA_OK) return st;
+    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(m, c->bw_dSc, c->N, c->H, c->bw_dZ, Dz,
+                                                                       c->dev_flag);
+    return GLGA_OK;
 }
-void launch_kv_global(Ctx *c, int64_t Dz, cudaStream_t s) {
-    if (!kv_global_tc(c) || c->N == 0) return;
+glga_status launch_kv_global(Ctx *c, int64_t Dz, cudaStream_t s) {
+    if (!kv_global_tc(c) || c->N == 0) return GLGA_OK;
     if (c->r == 32) return launch_kv_global_r<32>(c, Dz, s);
     if (c->r == 16) return launch_kv_global_r<16>(c, Dz, s);
-    launch_kv_global_r<64>(c, Dz, s);
+    return launch_kv_global_r<64>(c, Dz, s);
 }
 
 // Two rows per warp for up to 4 features per lane (one above that); the head loop
@@ -2891,7 +2923,10 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
                 c->bw_dsz_part, c->bw_dsz_parts, total, c->bw_dSz);                                       \
             bwd_heads_prep_kernel<<<tgrid, 256, 0, c->bw_side>>>(c->bw_dSz, R + 1, H, R, c->bw_dST,      \
                                                                 c->bw_dSc);                               \
-            launch_kv_global(c, Dz, c->bw_side);                                                          \
+            {                                                                                             \
+                const glga_status gs = launch_kv_global(c, Dz, c->bw_side);                               \
+                if (gs != GLGA_OK) return gs;                                                             \
+            }                                                                                             \
             launch_local_bwd<T>(c, Q, KV, isr, Dz, s, c->bw_side);                                        \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_join, c->bw_side));                                        \
             GLGA_CUDA(cudaStreamWaitEvent(s, c->bw_ev_join, 0));                                          \
