@@ -1435,19 +1435,21 @@ int local_bwd_launches(const Ctx *c) {
 //   dphi = dnum blockdiag(S_h)          (tcgen05, A = dnum rounded to bf16)
 //   dq_global = (dphi + z dden) phi'(q)
 // 16 warps, one CTA per SM: warp w reads TMEM lanes 32 (w % 4) (its 32 tile rows) and
-// owns columns 32 (w / 4) .. +31, one thread per row.  Row data moves between global
-// memory and the threads through a 4 KB staging area per warp with coalesced warp-wide
-// copies (bf16 inputs: 8 rows x 64 B per instruction; float32 outputs: 4 rows x 128 B),
-// swizzled so the threads' 16-byte row accesses are free of bank conflicts.  Per-head
-// and per-row sums that span column quarters meet in shared memory.
+// owns columns 32 (w / 4) .. +31, one thread per row.  The Q, dY and L tiles arrive by
+// TMA (128-byte swizzle, the MMA operand layout): Q in two buffers (the next tile's lands
+// while this one runs), dY and L issued as soon as this tile is done with them.  phi(Q)
+// is formed in place as the first A operand and dnum in place of dY as the second; a
+// tile the threads have read doubles as the 2 KB-per-warp staging area of the coalesced
+// row stores (8 rows x 64 B per instruction).  phi'(q) = min(phi(q), 1) from the bf16
+// phi(q).  Per-head and per-row sums that span column quarters meet in shared memory.
 constexpr int kBroTcD = 128;
 constexpr int kBroTcBN = kBroTcD + 16;            // num | den (H <= 8) | zero columns
 constexpr int kBroTcWarps = 16;
 constexpr uint32_t kBroTcAtom = 128 * 128;        // one 64-column atom of a 128-row operand
 constexpr uint32_t kBroTcB1Atom = kBroTcBN * 128; // one 64-column atom of B_g (144 rows)
-constexpr uint32_t kBroTcStage = 4096;            // staging bytes per warp
-constexpr size_t kBroTcSmem = 1024 + 2 * kBroTcAtom + 2 * kBroTcB1Atom + 2 * kBroTcAtom +
-                              kBroTcWarps * kBroTcStage + (kBroTcD + 3 * 4 * 128) * 4;
+constexpr uint32_t kBroTcStage = 4096;            // staging bytes per warp (source side)
+constexpr size_t kBroTcSmem = 1024 + 4 * 2 * kBroTcAtom + 2 * kBroTcB1Atom + 2 * kBroTcAtom +
+                              (kBroTcD + 3 * 4 * 128) * 4;
 
 // byte offset of element (row, k) of a K-major operand with 64-element atoms of `rows` rows
 __device__ __forceinline__ uint32_t swz_off(int row, int k, uint32_t atom_bytes) {
@@ -1502,44 +1504,45 @@ __device__ __forceinline__ void warp_rows_f32_flush(float *dst, int64_t ld, int6
     __syncwarp();
 }
 
-// The lane's 32 bf16 values (its row, columns c0 .. c0 + 31) to a row-major bf16 matrix:
-// four 16-byte pieces into the staging area (row r at byte r * 64, piece p at slot
-// p ^ ((r >> 1) & 3)), then four coalesced stores of 8 rows x 64 B.  Rows at or past N are
-// not written.
-__device__ __forceinline__ void stage_bf16_piece(uint8_t *stage, int lane, int p, uint4 v) {
+// The lane's 64 bytes of a row (lane = row: 32 bf16 or 16 float32 values) to a row-major
+// matrix: four 16-byte pieces into a 2 KB staging area (row r at byte r * 64, piece p at
+// slot p ^ ((r >> 1) & 3)), then four coalesced stores of 8 rows x 64 B to dst + row * ld
+// (bytes).  Rows at or past N are not written.
+__device__ __forceinline__ void stage_row64_piece(uint8_t *stage, int lane, int p, uint4 v) {
     *reinterpret_cast<uint4 *>(stage + lane * 64 + ((p ^ ((lane >> 1) & 3)) << 4)) = v;
 }
-__device__ __forceinline__ void warp_rows_bf16_flush(__nv_bfloat16 *dst, int64_t ld, int64_t r0, int64_t N,
-                                                     int c0, uint8_t *stage, int lane) {
+__device__ __forceinline__ void warp_rows64_flush(uint8_t *dst, int64_t ld, int64_t r0, int64_t N, uint8_t *stage,
+                                                  int lane) {
     __syncwarp();
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = 8 * i + (lane >> 2), p = lane & 3;
         const int64_t gr = r0 + r;
         const uint4 x = *reinterpret_cast<const uint4 *>(stage + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
-        if (gr < N) reinterpret_cast<uint4 *>(dst + gr * ld + c0)[p] = x;
+        if (gr < N) reinterpret_cast<uint4 *>(dst + (r0 + r) * ld)[p] = x;
     }
     __syncwarp();
 }
 
 template <int R>
 __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
-    const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ L, const float *__restrict__ t,
-    const __nv_bfloat16 *__restrict__ Bg, int ro_kp, const float *__restrict__ Sz,
-    const __nv_bfloat16 *__restrict__ dY, int64_t N, int H, float b_g, float eps, __nv_bfloat16 *__restrict__ dL,
-    float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dden, float *__restrict__ dZ,
-    int64_t dz_ld, unsigned *flag) {
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmY,
+    const __grid_constant__ CUtensorMap tmL, const float *__restrict__ t, const __nv_bfloat16 *__restrict__ Bg,
+    int ro_kp, const float *__restrict__ Sz, int64_t N, int H, float b_g, float eps, __nv_bfloat16 *__restrict__ dL,
+    float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
     constexpr int D = kBroTcD;
     constexpr int kHQ = R >= 32 ? 1 : 32 / R;     // heads in a 32-column quarter
+    constexpr uint32_t kTile = 2 * kBroTcAtom;    // a [128][128] bf16 tile
     extern __shared__ uint8_t bro_raw[];
-    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ __align__(8) uint64_t q_full[2], y_full, l_full, mma_bar;
     __shared__ uint32_t tmem_sh;
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(bro_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t *sA = sm;                              // phi(Q), then dnum: 2 atoms
-    uint8_t *sB1 = sA + 2 * kBroTcAtom;            // B_g: 2 atoms of 144 rows
+    uint8_t *sQb = sm;                             // [2] Q tiles: phi(Q) in place is the first A
+    uint8_t *sY = sQb + 2 * kTile;                 // dY tile; dnum in place is the second A
+    uint8_t *sL = sY + kTile;                      // L tile, then the first epilogue's staging
+    uint8_t *sB1 = sL + kTile;                     // B_g: 2 atoms of 144 rows
     uint8_t *sB2 = sB1 + 2 * kBroTcB1Atom;         // blockdiag(S_h): 2 atoms
-    uint8_t *stg_all = sB2 + 2 * kBroTcAtom;       // staging, kBroTcStage per warp
-    float *zf = reinterpret_cast<float *>(stg_all + kBroTcWarps * kBroTcStage);
+    float *zf = reinterpret_cast<float *>(sB2 + 2 * kBroTcAtom);
     float *xdt = zf + D;                           // [4 quarters][128 rows] dt partials
     float *xdd = xdt + 4 * 128;                    // ... (dG . G) partials (r = 64: a head spans 2)
     float *xDd = xdd + 4 * 128;                    // ... (dL . L) partials
@@ -1547,7 +1550,6 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
     const int quad = warp & 3, cq = warp >> 2;     // TMEM lane quarter, column quarter
     const int rt = quad * 32 + lane;               // row in the tile
     const int c0 = cq * 32;                        // first column of this warp
-    uint8_t *stg = stg_all + warp * kBroTcStage;
     const float *z = Sz + static_cast<int64_t>(H) * R * R;
 
     // operands that stay for the whole launch: B_g, blockdiag(S_h), z
@@ -1569,9 +1571,29 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]), bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
     }
     for (int f = tid; f < D; f += blockDim.x) zf[f] = z[f];
+    const int64_t n_tiles = ceil_div(N, 128);
+    const int my = blockIdx.x < n_tiles ? static_cast<int>((n_tiles - 1 - blockIdx.x) / gridDim.x) + 1 : 0;
+    // the rows of this block's k-th tile of one input into a tile buffer (two 64-column boxes)
+    auto issue = [&](const CUtensorMap *m, uint64_t *bar, uint8_t *dst, int k) {
+        const int32_t y = static_cast<int32_t>((blockIdx.x + static_cast<int64_t>(k) * gridDim.x) * 128);
+        mbar_arrive_expect_tx(bar, kTile);
+        tma_load_2d(dst, m, bar, 0, y);
+        tma_load_2d(dst + kBroTcAtom, m, bar, 64, y);
+    };
+    int nq = 0, ny = 0, nl = 0;                    // loads issued (thread 0)
     if (tid == 0) {
+        mbar_init(&q_full[0], 1);
+        mbar_init(&q_full[1], 1);
+        mbar_init(&y_full, 1);
+        mbar_init(&l_full, 1);
         mbar_init(&mma_bar, 1);
         fence_mbar_init();
+        for (; nq < my && nq < 2; ++nq) issue(&tmQ, &q_full[nq], sQb + nq * kTile, nq);
+        if (my > 0) {
+            issue(&tmY, &y_full, sY, 0);
+            issue(&tmL, &l_full, sL, 0);
+            ny = nl = 1;
+        }
     }
     fence_proxy_async_smem();
     if (warp == 0) {
@@ -1585,13 +1607,12 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t idesc1 = instr_desc(128, kBroTcBN, 1u, false, false);
     const uint32_t idesc2 = instr_desc(128, D, 1u, false, false);
-    const int64_t n_tiles = ceil_div(N, 128);
     uint32_t phase = 0;
     // the tile's MMAs: 8 K steps of 16 over the two atoms of A and B, one thread
-    auto mma = [&](const uint8_t *sb, uint32_t b_atom, uint32_t idesc) {
+    auto mma = [&](const uint8_t *sa, const uint8_t *sb, uint32_t b_atom, uint32_t idesc) {
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sb);
+            const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 const uint32_t ko = static_cast<uint32_t>(ks >> 2), kb = static_cast<uint32_t>(ks & 3) * 32u;
@@ -1602,36 +1623,42 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
         }
     };
     // every thread waits; the block leaves together if any wait gave up
-    auto wait_mma = [&]() -> bool {
-        const bool got = mbar_wait_bounded(&mma_bar, phase);
-        phase ^= 1u;
+    auto wait_all = [&](uint64_t *bar, uint32_t par) -> bool {
+        const bool got = mbar_wait_bounded(bar, par);
         const bool bad = __syncthreads_or(!got) != 0;
         if (bad && tid == 0) atomicOr(flag, kDevErrTimeout);
-        tc_fence_after();
         return !bad;
     };
     auto bf = [](const uint4 (&w)[4], int j) {
         const uint32_t word = (&w[j / 8].x)[(j % 8) / 2];
         return __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16));
     };
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t m0 = tile * 128, r0 = m0 + quad * 32;
+    // the warp's 32 rows x 32 columns of a landed tile (lane = row)
+    auto slice = [&](const uint8_t *tile, uint4 (&w)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint4 *>(tile + swz_off(rt, c0 + 8 * i, kBroTcAtom));
+    };
+    int k = 0;
+    for (; k < my; ++k) {
+        const int64_t m0 = (blockIdx.x + static_cast<int64_t>(k) * gridDim.x) * 128, r0 = m0 + quad * 32;
         const int64_t row = m0 + rt;
         const bool valid = row < N;
-        // ---- A = phi(q) for this warp's rows and 32 columns (zero past N) ----
-        {
-            uint4 qw[4];
-            warp_rows_bf16(Q, D, r0, N, c0, stg, lane, qw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<uint4 *>(sA + swz_off(rt, c0 + 8 * i, kBroTcAtom)) =
-                    make_uint4(phi_bf16x2(qw[i].x), phi_bf16x2(qw[i].y), phi_bf16x2(qw[i].z), phi_bf16x2(qw[i].w));
+        uint8_t *sQ = sQb + (k & 1) * kTile;
+        if (!wait_all(&q_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u)) break;
+        // ---- A = phi(q) in place (rows past N hold zeros: phi = 1, never stored) ----
+        for (int ch = tid; ch < static_cast<int>(kTile / 16); ch += blockDim.x) {
+            uint4 *p = reinterpret_cast<uint4 *>(sQ + ch * 16);
+            const uint4 u = *p;
+            *p = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        mma(sB1, kBroTcB1Atom, idesc1);
-        if (!wait_mma()) break;
+        mma(sQ, sB1, kBroTcB1Atom, idesc1);
+        const bool m1 = wait_all(&mma_bar, phase);
+        phase ^= 1u;
+        if (!m1) break;
+        tc_fence_after();
         // ---- epilogue 1 ----
         uint32_t dv[8];
         tmem_ld_n<4>(tmem + lane_base + D, *reinterpret_cast<uint32_t (*)[4]>(&dv[0]));
@@ -1646,9 +1673,13 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             dda[hq] = 0.f;
             Dda[hq] = 0.f;
         }
+        const uint32_t yl_par = static_cast<uint32_t>(k) & 1u;
+        if (!wait_all(&y_full, yl_par) || !wait_all(&l_full, yl_par)) break;
         uint4 yw[4], lw[4];
-        warp_rows_bf16(dY, D, r0, N, c0, stg, lane, yw);
-        warp_rows_bf16(L, D, r0, N, c0, stg, lane, lw);
+        slice(sY, yw);
+        slice(sL, lw);
+        __syncthreads();   // every warp holds its dY and L slices: the L tile is the staging
+        uint8_t *stg = sL + warp * 2048;
         // dL = g dY stored in bf16, and D_i from the stored values
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -1662,9 +1693,9 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
                 Dda[hq] = fmaf(v.y, bf(lw, j + 1), Dda[hq]);
                 w[e] = *reinterpret_cast<const uint32_t *>(&h2);
             }
-            stage_bf16_piece(stg, lane, p, make_uint4(w[0], w[1], w[2], w[3]));
+            stage_row64_piece(stg, lane, p, make_uint4(w[0], w[1], w[2], w[3]));
         }
-        warp_rows_bf16_flush(dL, D, r0, N, c0, stg, lane);
+        warp_rows64_flush(reinterpret_cast<uint8_t *>(dL + c0), static_cast<int64_t>(D) * 2, r0, N, stg, lane);
         float dtp = 0.f;
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {           // 16 columns at a time
@@ -1683,22 +1714,29 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
                 dtp = fmaf(y, bf(lw, j) - G, dtp);
             }
 #pragma unroll
-            for (int p = 0; p < 4; ++p) stage_f32_piece(stg, lane, 4 * hb + p, dn[4 * p], dn[4 * p + 1], dn[4 * p + 2], dn[4 * p + 3]);
-            // A = dnum in bf16 (phi(q) has been read by the first MMA)
+            for (int p = 0; p < 4; ++p)
+                stage_row64_piece(stg, lane, p, make_uint4(__float_as_uint(dn[4 * p]), __float_as_uint(dn[4 * p + 1]),
+                                                           __float_as_uint(dn[4 * p + 2]), __float_as_uint(dn[4 * p + 3])));
+            warp_rows64_flush(reinterpret_cast<uint8_t *>(dnum + c0 + 16 * hb), static_cast<int64_t>(D + 16) * 4, r0, N,
+                              stg, lane);
+            // A = dnum in bf16, in place of the warp's own dY slice
 #pragma unroll
             for (int i = 0; i < 2; ++i)
-                *reinterpret_cast<uint4 *>(sA + swz_off(rt, c0 + 16 * hb + 8 * i, kBroTcAtom)) =
+                *reinterpret_cast<uint4 *>(sY + swz_off(rt, c0 + 16 * hb + 8 * i, kBroTcAtom)) =
                     make_uint4(bf16x2_bits(dn[8 * i], dn[8 * i + 1]), bf16x2_bits(dn[8 * i + 2], dn[8 * i + 3]),
                                bf16x2_bits(dn[8 * i + 4], dn[8 * i + 5]), bf16x2_bits(dn[8 * i + 6], dn[8 * i + 7]));
         }
-        warp_rows_f32_flush(dnum, D + 16, r0, N, c0, stg, lane);   // [dnum | dden] rows
         xdt[cq * 128 + rt] = dtp;
         xdd[cq * 128 + rt] = dda[0];
         xDd[cq * 128 + rt] = Dda[0];
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        mma(sB2, kBroTcAtom, idesc2);
+        mma(sY, sB2, kBroTcAtom, idesc2);
+        if (tid == 0 && nl < my) {                 // the staging is done: the next L tile
+            issue(&tmL, &l_full, sL, nl);
+            ++nl;
+        }
         // per-row and per-head sums across the column quarters; dden, D_i and dt out
         float ddh[kHQ];
         if constexpr (R == 64) {
@@ -1722,31 +1760,50 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
         }
         if (cq == 0 && valid)
             dZ[row * dz_ld + 3 * D] = g * (1.f - g) * (xdt[rt] + xdt[128 + rt] + xdt[256 + rt] + xdt[384 + rt]);
-        if (!wait_mma()) break;
-        // ---- epilogue 2: dq_global = (dphi + z dden) phi'(q) ----
-        {
-            uint4 qw[4];
-            warp_rows_bf16(Q, D, r0, N, c0, stg, lane, qw);
-#pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                uint32_t av[16];
-                tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), av);
-                tmem_ld_wait();
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    float o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 16 * hb + 4 * p + e, hq = j / R < kHQ ? j / R : 0;
-                        o[e] = fmaf(zf[c0 + j], ddh[hq], __uint_as_float(av[4 * p + e])) * dphi(bf(qw, j));
-                    }
-                    stage_f32_piece(stg, lane, 4 * hb + p, o[0], o[1], o[2], o[3]);
-                }
-            }
-            warp_rows_f32_flush(dZ, dz_ld, r0, N, c0, stg, lane);
+        const bool m2 = wait_all(&mma_bar, phase);
+        phase ^= 1u;
+        if (!m2) break;
+        tc_fence_after();
+        if (tid == 0 && ny < my) {                 // the second MMA has read dnum: the next dY tile
+            issue(&tmY, &y_full, sY, ny);
+            ++ny;
         }
+        // ---- epilogue 2: dq_global = (dphi + z dden) phi'(q), phi'(q) = min(phi(q), 1) ----
+        uint4 pw[4];
+        slice(sQ, pw);
+        __syncthreads();   // every warp holds its phi(q) slice: the Q tile is the staging
+        stg = sQ + warp * 2048;
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+            uint32_t av[16];
+            tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), av);
+            tmem_ld_wait();
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                float o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 16 * hb + 4 * p + e, hq = j / R < kHQ ? j / R : 0;
+                    o[e] = fmaf(zf[c0 + j], ddh[hq], __uint_as_float(av[4 * p + e])) * fminf(bf(pw, j), 1.f);
+                }
+                stage_row64_piece(stg, lane, p, make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]),
+                                                           __float_as_uint(o[2]), __float_as_uint(o[3])));
+            }
+            warp_rows64_flush(reinterpret_cast<uint8_t *>(dZ + c0 + 16 * hb), dz_ld * 4, r0, N, stg, lane);
+        }
+        fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();   // TMEM, the A operand and the cross-quarter sums are rewritten next tile
+        __syncthreads();   // TMEM, the cross-quarter sums and the Q tile are free
+        if (tid == 0 && nq < my) {
+            issue(&tmQ, &q_full[nq & 1], sQb + (nq & 1) * kTile, nq);
+            ++nq;
+        }
+    }
+    // the block leaves only after its copies have landed (already so when all went well)
+    if (tid == 0) {
+        for (int i = std::max(0, nq - 2); i < nq; ++i) mbar_wait_bounded(&q_full[i & 1], static_cast<uint32_t>(i >> 1) & 1u);
+        if (ny > 0) mbar_wait_bounded(&y_full, static_cast<uint32_t>(ny - 1) & 1u);
+        if (nl > 0) mbar_wait_bounded(&l_full, static_cast<uint32_t>(nl - 1) & 1u);
     }
     tc_fence_before();
     __syncthreads();
@@ -1973,22 +2030,31 @@ bool readout_bwd_tc(const Ctx *c) {
 }
 
 template <int R>
-void launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *dY, float b_g, float eps, int64_t Dz,
-                           cudaStream_t s) {
+glga_status launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfloat16 *dY, float b_g, float eps,
+                                  int64_t Dz, cudaStream_t s) {
     const int64_t tiles = ceil_div(c->N, 128);
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, c->num_sms));
     cudaFuncSetAttribute(bwd_readout_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kBroTcSmem));
+    CUtensorMap mq, my, ml;
+    const uint64_t n = static_cast<uint64_t>(c->N);
+    glga_status st = encode_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, kBroTcD, n, 2 * kBroTcD, 64, 128);
+    if (st == GLGA_OK)
+        st = encode_tmap_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, kBroTcD, n, 2 * kBroTcD, 64, 128);
+    if (st == GLGA_OK)
+        st = encode_tmap_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->L, kBroTcD, n, 2 * kBroTcD, 64, 128);
+    if (st != GLGA_OK) return st;
     bwd_readout_tc_kernel<R><<<grid, kBroTcWarps * 32, kBroTcSmem, s>>>(
-        Q, static_cast<const __nv_bfloat16 *>(c->L), c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz,
-        dY, c->N, c->H, b_g, eps, static_cast<__nv_bfloat16 *>(c->bw_dL), c->bw_Dd, c->bw_dnum, c->bw_dden, c->bw_dZ, Dz, c->dev_flag);
+        mq, my, ml, c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz, c->N, c->H, b_g, eps,
+        static_cast<__nv_bfloat16 *>(c->bw_dL), c->bw_Dd, c->bw_dnum, c->bw_dZ, Dz, c->dev_flag);
+    return GLGA_OK;
 }
 
 // The readout backward runs on the tensor cores for bf16 layers with H*r = 128, r in
 // {16, 32, 64} and one head group (the forward's readout operand then holds every head);
 // elsewhere on the CUDA cores.
 template <typename T>
-void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
+glga_status launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, int64_t Dz, cudaStream_t s) {
     if constexpr (sizeof(T) == 2) {
         if (readout_bwd_tc(c)) {
             if (c->r == 32) return launch_readout_bwd_tc<32>(c, Q, dY, b_g, eps, Dz, s);
@@ -1997,16 +2063,20 @@ void launch_readout_bwd(Ctx *c, const T *Q, const T *dY, float b_g, float eps, i
         }
     }
     const int E = lane_features(c->D), lph = c->r / E;
-    if (E == 4 && lph == 8) return launch_readout_bwd_e<T, 4, 8>(c, Q, dY, b_g, eps, Dz, s);
+    if (E == 4 && lph == 8) {
+        launch_readout_bwd_e<T, 4, 8>(c, Q, dY, b_g, eps, Dz, s);
+        return GLGA_OK;
+    }
     switch (E) {
-        case 1: return launch_readout_bwd_e<T, 1, 0>(c, Q, dY, b_g, eps, Dz, s);
-        case 2: return launch_readout_bwd_e<T, 2, 0>(c, Q, dY, b_g, eps, Dz, s);
-        case 4: return launch_readout_bwd_e<T, 4, 0>(c, Q, dY, b_g, eps, Dz, s);
-        case 8: return launch_readout_bwd_e<T, 8, 0>(c, Q, dY, b_g, eps, Dz, s);
-        case 16: return launch_readout_bwd_e<T, 16, 0>(c, Q, dY, b_g, eps, Dz, s);
-        case 32: return launch_readout_bwd_e<T, 32, 0>(c, Q, dY, b_g, eps, Dz, s);
+        case 1: launch_readout_bwd_e<T, 1, 0>(c, Q, dY, b_g, eps, Dz, s); break;
+        case 2: launch_readout_bwd_e<T, 2, 0>(c, Q, dY, b_g, eps, Dz, s); break;
+        case 4: launch_readout_bwd_e<T, 4, 0>(c, Q, dY, b_g, eps, Dz, s); break;
+        case 8: launch_readout_bwd_e<T, 8, 0>(c, Q, dY, b_g, eps, Dz, s); break;
+        case 16: launch_readout_bwd_e<T, 16, 0>(c, Q, dY, b_g, eps, Dz, s); break;
+        case 32: launch_readout_bwd_e<T, 32, 0>(c, Q, dY, b_g, eps, Dz, s); break;
         default: break;
     }
+    return GLGA_OK;
 }
 
 
@@ -2911,7 +2981,10 @@ glga_status backward_run(Ctx *c, const void *X, const void *WQ, const void *WK, 
         const unsigned tgrid = static_cast<unsigned>(ceil_div(static_cast<int64_t>(H) * R * R, 256));    \
         if (N > 0) {                                                                                      \
             bwd_heads_prep_kernel<<<tgrid, 256, 0, s>>>(c->Sz, R, H, R, c->bw_ST, nullptr);              \
-            launch_readout_bwd<T>(c, Q, static_cast<const T *>(dY), b_g, eps, Dz, s);                  \
+            {                                                                                             \
+                const glga_status rs = launch_readout_bwd<T>(c, Q, static_cast<const T *>(dY), b_g, eps, Dz, s); \
+                if (rs != GLGA_OK) return rs;                                                             \
+            }                                                                                             \
             /* fork: the dS | dz chain and the source-side kernels on the side stream */                 \
             GLGA_CUDA(cudaEventRecord(c->bw_ev_fork, s));                                                 \
             GLGA_CUDA(cudaStreamWaitEvent(c->bw_side, c->bw_ev_fork, 0));                                 \
