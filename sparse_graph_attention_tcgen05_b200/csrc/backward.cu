@@ -160,6 +160,12 @@ __device__ __forceinline__ void st_row(T *p, const float (&x)[EPL]) {
     }
 }
 
+// Two floats rounded to bf16 (nearest even) in one word, lo in bits 0..15.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
 // x as a T row stores it.
 template <typename T>
 __device__ __forceinline__ float round_to(float x) {
@@ -486,12 +492,66 @@ __global__ void __launch_bounds__(256) bwd_strided_sum_kernel(const float *__res
 constexpr int kEU = 4;            // edges whose rows are loaded before any is used
 constexpr int kChunk = 32;        // edges per chunk of a heavy row (one warp each)
 
-// dq += sum over edges [a, b) of ds_ij k_j (ds already scaled by 1/sqrt(r)).
+// The lane's EPL bf16 values of a row (EPL even) as EPL / 2 packed words (zero if !act).
+template <int EPL>
+__device__ __forceinline__ void ld_words(const __nv_bfloat16 *row, int lane, bool act, uint32_t (&w)[EPL / 2]) {
+#pragma unroll
+    for (int x = 0; x < EPL / 2; ++x) w[x] = 0u;
+    if (!act) return;
+    const __nv_bfloat16 *p = row + lane * EPL;
+    if constexpr (EPL % 8 == 0) {
+#pragma unroll
+        for (int v = 0; v < EPL / 8; ++v) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p) + v);
+            w[4 * v] = u.x; w[4 * v + 1] = u.y; w[4 * v + 2] = u.z; w[4 * v + 3] = u.w;
+        }
+    } else if constexpr (EPL == 4) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        w[0] = u.x; w[1] = u.y;
+    } else {
+        w[0] = __ldg(reinterpret_cast<const unsigned int *>(p));
+    }
+}
+
+// EPL values that are bf16 numbers, packed into EPL / 2 words (exact).
+template <int EPL>
+__device__ __forceinline__ void pack_words(const float (&x)[EPL], uint32_t (&w)[EPL / 2]) {
+#pragma unroll
+    for (int i = 0; i < EPL / 2; ++i) w[i] = bf16x2_bits(x[2 * i], x[2 * i + 1]);
+}
+
+// dq += sum over edges [a, b) of ds_ij k_j (ds already scaled by 1/sqrt(r)).  bf16 rows
+// stay packed (fma.rn.f32.bf16, ds rounded to bf16 for dq).
 template <typename T, int EPL>
 __device__ __forceinline__ void q_grad_range(const int32_t *col_idx, const T *KV, int D, int lane, bool act,
                                              int lph, float inv_sqrt_r, const float (&q)[EPL],
                                              const float (&dl)[EPL], float ls, float dd, int32_t a, int32_t b,
                                              float (&dq)[EPL]) {
+    if constexpr (sizeof(T) == 2 && EPL % 2 == 0) {
+        constexpr int W = EPL / 2;
+        uint32_t qw[W], dw[W];
+        pack_words<EPL>(q, qw);
+        pack_words<EPL>(dl, dw);
+        for (int32_t e = a; e < b; e += kEU) {
+            uint32_t k[kEU][W], v[kEU][W];
+#pragma unroll
+            for (int u = 0; u < kEU; ++u) {
+                const bool live = e + u < b;
+                const T *row = KV + (live ? static_cast<int64_t>(col_idx[e + u]) : 0) * 2 * D;
+                ld_words<EPL>(row, lane, act && live, k[u]);
+                ld_words<EPL>(row + D, lane, act && live, v[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < kEU; ++u) {
+                float s = dot_bf16w<W>(qw, k[u], 0.f), dp = dot_bf16w<W>(dw, v[u], 0.f);
+                s = head_reduce(s, lph);
+                dp = head_reduce(dp, lph);
+                const float ds = e + u < b ? __expf(s * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
+                axpy_bf16w<W>(bf16_splat(ds), k[u], dq);
+            }
+        }
+        return;
+    }
     for (int32_t e = a; e < b; e += kEU) {
         float k[kEU][EPL], v[kEU][EPL];
 #pragma unroll
@@ -629,6 +689,15 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
             }
             cp_async_commit();
         };
+        // q_i, dL_i and the gathered k_j, v_j stay packed: the dot products and dq run on
+        // fma.rn.f32.bf16 (ds rounded to bf16 for dq)
+        uint32_t qw[4] = {0u, 0u, 0u, 0u}, dw[4] = {0u, 0u, 0u, 0u};
+        if (act2) {
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(Q + i * D + hl * EPL2));
+            const uint4 y = __ldg(reinterpret_cast<const uint4 *>(dL + i * D + hl * EPL2));
+            qw[0] = x.x; qw[1] = x.y; qw[2] = x.z; qw[3] = x.w;
+            dw[0] = y.x; dw[1] = y.y; dw[2] = y.z; dw[3] = y.w;
+        }
         const int n_steps = (b - a + 2 * kU - 1) / (2 * kU);
         issue(a, 0);
         for (int it = 0; it < n_steps; ++it) {
@@ -639,15 +708,17 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
             } else {
                 cp_async_wait<0>();
             }
-            float k[kU][EPL2], v[kU][EPL2];
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
-                const uint4 kw = *cell(it & 1, u, 0), vw = *cell(it & 1, u, 1);
-                const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, vv[4] = {vw.x, vw.y, vw.z, vw.w};
-                unpack_bf16<EPL2>(kk, k[u]);
-                unpack_bf16<EPL2>(vv, v[u]);
+                const uint4 kv4 = *cell(it & 1, u, 0), vv4 = *cell(it & 1, u, 1);
+                const uint32_t kk[4] = {kv4.x, kv4.y, kv4.z, kv4.w}, vv[4] = {vv4.x, vv4.y, vv4.z, vv4.w};
+                float sc = dot_bf16w<4>(qw, kk, 0.f), dp = dot_bf16w<4>(dw, vv, 0.f);
+                sc = head_reduce(sc, lph2);
+                dp = head_reduce(dp, lph2);
+                const bool live = e0 + 2 * u + slot < b;
+                const float ds = live ? __expf(sc * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
+                axpy_bf16w<4>(bf16_splat(ds), kk, dq2);
             }
-            use_step(e0, k, v);
         }
     } else {
         for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {      // the same trip count in both halves
@@ -778,6 +849,38 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
                                               bool act, int lph, int h, float inv_sqrt_r, const float (&k)[EPL],
                                               const float (&v)[EPL], int32_t a, int32_t b, float (&dk)[EPL],
                                               float (&dv)[EPL]) {
+    if constexpr (sizeof(T) == 2 && EPL % 2 == 0) {
+        // bf16 rows stay packed (fma.rn.f32.bf16; p and ds rounded to bf16 for dv and dk)
+        constexpr int W = EPL / 2;
+        uint32_t kw[W], vw[W];
+        pack_words<EPL>(k, kw);
+        pack_words<EPL>(v, vw);
+        for (int32_t e = a; e < b; e += kEU) {
+            uint32_t q[kEU][W], dl[kEU][W];
+            float ls[kEU], dd[kEU];
+#pragma unroll
+            for (int u = 0; u < kEU; ++u) {
+                const bool live = e + u < b;
+                const int64_t i = live ? t_col[e + u] : 0;
+                ld_words<EPL>(Q + i * D, lane, act && live, q[u]);
+                ld_words<EPL>(dL + i * D, lane, act && live, dl[u]);
+                ls[u] = live ? __ldg(lse + i * H + h) : 0.f;
+                dd[u] = live ? __ldg(Dd + i * H + h) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kEU; ++u) {
+                float s = dot_bf16w<W>(q[u], kw, 0.f), dp = dot_bf16w<W>(dl[u], vw, 0.f);
+                s = head_reduce(s, lph);
+                dp = head_reduce(dp, lph);
+                const bool live = e + u < b;
+                const float p = live ? __expf(s * inv_sqrt_r - ls[u]) : 0.f;
+                const float ds = p * (dp - dd[u]) * inv_sqrt_r;
+                axpy_bf16w<W>(bf16_splat(p), dl[u], dv);
+                axpy_bf16w<W>(bf16_splat(ds), q[u], dk);
+            }
+        }
+        return;
+    }
     for (int32_t e = a; e < b; e += kEU) {
         float q[kEU][EPL], dl[kEU][EPL], ls[kEU], dd[kEU];
 #pragma unroll
@@ -988,19 +1091,61 @@ __global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
             }
         }
     };
-    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {      // the same trip count in both halves
-        float q[kU][EPL2], dl[kU][EPL2], ls[kU], dd[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int32_t e = e0 + 2 * u + slot;
-            const bool live = e < b;
-            const int64_t i = live ? t_col[e] : 0;
-            ld_row<T, EPL2>(Q + i * D, hl, act2 && live, q[u]);
-            ld_row<T, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
-            ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
-            dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
+    if constexpr (sizeof(T) == 2 && EPL2 == 8) {
+        // k_j, v_j and the gathered q_i, dL_i stay packed: the dot products, dv and dk run on
+        // fma.rn.f32.bf16 (p and ds rounded to bf16 for dv and dk)
+        uint32_t kw[4] = {0u, 0u, 0u, 0u}, vw[4] = {0u, 0u, 0u, 0u};
+        if (act2) {
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(krow + hl * EPL2));
+            const uint4 y = __ldg(reinterpret_cast<const uint4 *>(krow + D + hl * EPL2));
+            kw[0] = x.x; kw[1] = x.y; kw[2] = x.z; kw[3] = x.w;
+            vw[0] = y.x; vw[1] = y.y; vw[2] = y.z; vw[3] = y.w;
         }
-        use_step(e0, q, dl, ls, dd);
+        for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {  // the same trip count in both halves
+            uint4 q4[kU], d4[kU];
+            float ls[kU], dd[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int32_t e = e0 + 2 * u + slot;
+                const bool live = e < b;
+                const int64_t i = live ? t_col[e] : 0;
+                q4[u] = d4[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (act2 && live) {
+                    q4[u] = __ldg(reinterpret_cast<const uint4 *>(Q + i * D + hl * EPL2));
+                    d4[u] = __ldg(reinterpret_cast<const uint4 *>(dL + i * D + hl * EPL2));
+                }
+                ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
+                dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const uint32_t qq[4] = {q4[u].x, q4[u].y, q4[u].z, q4[u].w};
+                const uint32_t ll[4] = {d4[u].x, d4[u].y, d4[u].z, d4[u].w};
+                float sc = dot_bf16w<4>(qq, kw, 0.f), dp = dot_bf16w<4>(ll, vw, 0.f);
+                sc = head_reduce(sc, lph2);
+                dp = head_reduce(dp, lph2);
+                const bool live = e0 + 2 * u + slot < b;
+                const float p = live ? __expf(sc * inv_sqrt_r - ls[u]) : 0.f;
+                const float ds = p * (dp - dd[u]) * inv_sqrt_r;
+                axpy_bf16w<4>(bf16_splat(p), ll, dv2);
+                axpy_bf16w<4>(bf16_splat(ds), qq, dk2);
+            }
+        }
+    } else {
+        for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {  // the same trip count in both halves
+            float q[kU][EPL2], dl[kU][EPL2], ls[kU], dd[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int32_t e = e0 + 2 * u + slot;
+                const bool live = e < b;
+                const int64_t i = live ? t_col[e] : 0;
+                ld_row<T, EPL2>(Q + i * D, hl, act2 && live, q[u]);
+                ld_row<T, EPL2>(dL + i * D, hl, act2 && live, dl[u]);
+                ls[u] = live ? __ldg(lse + i * H + h2) : 0.f;
+                dd[u] = live ? __ldg(Dd + i * H + h2) : 0.f;
+            }
+            use_step(e0, q, dl, ls, dd);
+        }
     }
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) {
@@ -1456,11 +1601,6 @@ __device__ __forceinline__ uint32_t swz_off(int row, int k, uint32_t atom_bytes)
     return static_cast<uint32_t>(k >> 6) * atom_bytes + static_cast<uint32_t>(row) * 128u +
            ((static_cast<uint32_t>((k & 63) >> 3) ^ static_cast<uint32_t>(row & 7)) << 4) +
            static_cast<uint32_t>(k & 7) * 2u;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
 }
 
 // The warp's 32 rows x 32 bf16 columns (64 B per row) of a row-major [N][ld] bf16 matrix,

@@ -536,6 +536,54 @@ __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
     return y;
 }
 
+// d = a * b + c for the bf16 half AH of a and BH of b (1 = the high half): fma.rn.f32.bf16,
+// the product exact, one f32 rounding (the same value as float32 fmaf of the widened halves).
+template <int AH, int BH>
+__device__ __forceinline__ float fma_bf16h(uint32_t a, uint32_t b, float c) {
+    float d;
+    if constexpr (AH == 0 && BH == 0)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a0, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if constexpr (AH == 1 && BH == 1)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a1, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if constexpr (AH == 0 && BH == 1)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a0, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, a1, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+// acc + the dot product of the 2W bf16 values of a and b (W words each), element order.
+template <int W>
+__device__ __forceinline__ float dot_bf16w(const uint32_t *a, const uint32_t *b, float acc) {
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+        acc = fma_bf16h<0, 0>(a[w], b[w], acc);
+        acc = fma_bf16h<1, 1>(a[w], b[w], acc);
+    }
+    return acc;
+}
+
+// acc[2w + e] += s x[w].half(e) for the bf16 s in the low half of s2.
+template <int W>
+__device__ __forceinline__ void axpy_bf16w(uint32_t s2, const uint32_t *x, float *acc) {
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+        acc[2 * w] = fma_bf16h<0, 0>(s2, x[w], acc[2 * w]);
+        acc[2 * w + 1] = fma_bf16h<0, 1>(s2, x[w], acc[2 * w + 1]);
+    }
+}
+
+// x rounded to bf16 (nearest even) in both halves of a word.
+__device__ __forceinline__ uint32_t bf16_splat(float x) {
+    uint32_t w;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(w) : "f"(x));
+    return w;
+}
+
 // 16-byte asynchronous copy global -> shared (L2 only), its group commit and the wait for
 // all but the N most recent groups of this thread.
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
