@@ -1048,7 +1048,7 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
 // dk, dv are then added (lower + upper, the same sum in both) and moved to the 32-lane
 // layout for kv_finish.  Needs 2 EPL <= r.
 template <typename T, int EPL, bool GTC = false>
-__global__ void __launch_bounds__(256, 3) bwd_local_kv2_kernel(
+__global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,

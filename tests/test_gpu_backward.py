@@ -47,11 +47,14 @@ def _check(w, seed=0, chunked=False):
     rp, ci = oracle.csr_from_coo(w.N, w.src, w.dst)
     ref_fn = backward_chunked if chunked else ref_backward
     ref = ref_fn(w.X, w.W_Q, w.W_K, w.W_V, w.w_g, w.b_g, w.eps, rp, ci, w.H, w.r, dY)
+    errs = {}
     for k in NAMES:
         r = np.asarray(ref[k], dtype=np.float64).reshape(got[k].shape)
         scale = max(np.abs(r).max(), 1e-30)
-        err = np.abs(got[k] - r).max() / scale
-        assert np.all(np.isfinite(got[k])) and err <= TOLB[w.io], (k, err)
+        errs[k] = float(np.abs(got[k] - r).max() / scale)
+    print(f"\n{w.name} N={w.N} H={w.H} r={w.r} {w.io}: " + ", ".join(f"{k} {e:.2e}" for k, e in errs.items()))
+    for k in NAMES:
+        assert np.all(np.isfinite(got[k])) and errs[k] <= TOLB[w.io], (k, errs[k])
 
 
 def test_tiny_fp32():
