@@ -1703,9 +1703,11 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
         const int h = f / R;
         float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int c = c8 + e;
-            v[e] = (c / R == h) ? Sz[(static_cast<int64_t>(h) * R + (f - h * R)) * R + (c - h * R)] : 0.f;
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+        if (c8 / R == h) {   // 8 columns of head h: S_h[f - h R][c8 - h R ..]
+            const float4 *sp = reinterpret_cast<const float4 *>(Sz + (static_cast<int64_t>(h) * R + (f - h * R)) * R + (c8 - h * R));
+            const float4 a0 = __ldg(sp), a1 = __ldg(sp + 1);
+            v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
         }
         *reinterpret_cast<uint4 *>(sB2 + swz_off(f, c8, kBroTcAtom)) =
             make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]), bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
@@ -1778,11 +1780,19 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
 #pragma unroll
         for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint4 *>(tile + swz_off(rt, c0 + 8 * i, kBroTcAtom));
     };
+    // the gate pre-activation of this thread's row, one tile ahead
+    auto t_of = [&](int kk) {
+        const int64_t rr = (blockIdx.x + static_cast<int64_t>(kk) * gridDim.x) * 128 + rt;
+        return kk < my && rr < N ? __ldg(t + rr) : 0.f;
+    };
+    float t_next = t_of(0);
     int k = 0;
     for (; k < my; ++k) {
         const int64_t m0 = (blockIdx.x + static_cast<int64_t>(k) * gridDim.x) * 128, r0 = m0 + quad * 32;
         const int64_t row = m0 + rt;
         const bool valid = row < N;
+        const float t_row = t_next;
+        t_next = t_of(k + 1);
         uint8_t *sQ = sQb + (k & 1) * kTile;
         if (!wait_all(&q_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u)) break;
         // ---- A = phi(q) in place (rows past N hold zeros: phi = 1, never stored) ----
@@ -1804,7 +1814,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
         tmem_ld_n<4>(tmem + lane_base + D, *reinterpret_cast<uint32_t (*)[4]>(&dv[0]));
         tmem_ld_n<4>(tmem + lane_base + D + 4, *reinterpret_cast<uint32_t (*)[4]>(&dv[4]));
         tmem_ld_wait();
-        const float g = valid ? 1.f / (1.f + __expf(-(__ldg(t + row) + b_g))) : 0.f;
+        const float g = valid ? 1.f / (1.f + __expf(-(t_row + b_g))) : 0.f;
         float inv[kHQ], dda[kHQ], Dda[kHQ];
 #pragma unroll
         for (int hq = 0; hq < kHQ; ++hq) {
@@ -1969,8 +1979,8 @@ static_assert(kBroTcWarps * kBroTcStage <= kKvgStage, "a landed stage doubles as
 
 template <int R>
 __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
-    const __grid_constant__ CUtensorMap tmKV, const float *__restrict__ dSc, int64_t N, int H,
-    float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
+    const __grid_constant__ CUtensorMap tmKV, const float *__restrict__ dSc, const float *__restrict__ dST,
+    int64_t N, int H, float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
     constexpr int D = kBroTcD;
     extern __shared__ uint8_t kvg_raw[];
     __shared__ __align__(8) uint64_t full_bar[kKvgStages];
@@ -1992,11 +2002,13 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
         const int h = f / R, fl = f - h * R;
         float v1[8], v2[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int c = c8 + e, cl = c - h * R;
-            const bool in = c / R == h;
-            v1[e] = in ? dSc[(static_cast<int64_t>(h) * R + fl) * R + cl] : 0.f;
-            v2[e] = in ? dSc[(static_cast<int64_t>(h) * R + cl) * R + fl] : 0.f;
+        for (int e = 0; e < 8; ++e) v1[e] = v2[e] = 0.f;
+        if (c8 / R == h) {   // 8 columns of head h: dS_h[fl][cl ..] and dS_h^T[fl][cl ..] (= dS_h[cl ..][fl])
+            const int64_t o = (static_cast<int64_t>(h) * R + fl) * R + (c8 - h * R);
+            const float4 a0 = __ldg(reinterpret_cast<const float4 *>(dSc + o)), a1 = __ldg(reinterpret_cast<const float4 *>(dSc + o) + 1);
+            const float4 b0 = __ldg(reinterpret_cast<const float4 *>(dST + o)), b1 = __ldg(reinterpret_cast<const float4 *>(dST + o) + 1);
+            v1[0] = a0.x; v1[1] = a0.y; v1[2] = a0.z; v1[3] = a0.w; v1[4] = a1.x; v1[5] = a1.y; v1[6] = a1.z; v1[7] = a1.w;
+            v2[0] = b0.x; v2[1] = b0.y; v2[2] = b0.z; v2[3] = b0.w; v2[4] = b1.x; v2[5] = b1.y; v2[6] = b1.z; v2[7] = b1.w;
         }
         *reinterpret_cast<uint4 *>(sB1 + swz_off(f, c8, kBroTcAtom)) =
             make_uint4(bf16x2_bits(v1[0], v1[1]), bf16x2_bits(v1[2], v1[3]), bf16x2_bits(v1[4], v1[5]), bf16x2_bits(v1[6], v1[7]));
@@ -2140,7 +2152,7 @@ glga_status launch_kv_global_r(Ctx *c, int64_t Dz, cudaStream_t s) {
     const glga_status st = encode_tmap_2d(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->KV, 2 * kBroTcD,
                                           static_cast<uint64_t>(c->N), 4 * kBroTcD, 64, 128);
     if (st != GLGA_OK) return st;
-    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(m, c->bw_dSc, c->N, c->H, c->bw_dZ, Dz,
+    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(m, c->bw_dSc, c->bw_dST, c->N, c->H, c->bw_dZ, Dz,
                                                                        c->dev_flag);
     return GLGA_OK;
 }
