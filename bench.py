@@ -365,9 +365,11 @@ def time_backward(layer, w, X, WQ, WK, WV, wg, dt, dev, flush, stream, steps):
     tg = float(np.mean(gms))
     return {"ms": t, "edge_heads_per_s": w.E * w.H / (t * 1e-3), "steps": steps,
             "graph_ms": tg, "graph_edge_heads_per_s": w.E * w.H / (tg * 1e-3),
-            "kernels": ("gathers and reductions on the CUDA cores (fp32 arithmetic)"
-                        + ("; readout backward (H*r = 128), dW and dX on the tcgen05 tensor cores"
-                           if w.io == "bf16" else "; dW and dX as CUDA-core fp32 GEMMs"))}
+            "kernels": (("gathers on the CUDA cores with bf16 rows kept packed (fma.rn.f32.bf16, f32 "
+                         "accumulation); readout backward, dS | dz, the source side's global terms and "
+                         "dX | dW in one pass over dZ on the tcgen05 tensor cores (H*r = 128, d = 128)")
+                        if w.io == "bf16" else
+                        "gathers, reductions and the dW / dX GEMMs on the CUDA cores (fp32 arithmetic)")}
 
 
 def median_event_ms(fn, steps, warmup, flush):
