@@ -630,15 +630,25 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
-    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld) {
+    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     if (w >= n_rows) return;                              // warp-uniform
     const int64_t i = rows[w];
     const int32_t a = row_ptr[i], b = row_ptr[i + 1];
-    if (a == b) return;                                   // no local term
     const int D = H * R;
+    if (a == b) {                                         // no local term
+        if (dZb) {                                        // dq_i = its global part, in bf16
+            const LaneHead lh(lane, EPL, D, R);
+            if (lh.act) {
+                float cur[EPL];
+                ld_mrow<EPL, false>(dZ + i * dz_ld + lane * EPL, cur);
+                st_row<__nv_bfloat16, EPL>(dZb + i * 3 * D + lane * EPL, cur);
+            }
+        }
+        return;
+    }
     const bool act2 = hl * EPL2 < D;
     const int lph2 = R / EPL2, h2 = act2 ? hl * EPL2 / R : 0;
     float q2[EPL2], dl2[EPL2], dq2[EPL2];
@@ -752,7 +762,8 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
         ld_mrow<EPL, false>(o, cur);
 #pragma unroll
         for (int x = 0; x < EPL; ++x) cur[x] += dq[x];
-        st_mrow<EPL>(o, cur);
+        if (dZb) st_row<__nv_bfloat16, EPL>(dZb + i * 3 * D + lane * EPL, cur);
+        else st_mrow<EPL>(o, cur);
     }
 }
 
@@ -793,7 +804,8 @@ constexpr int kMW = 8, kMU = 4;
 template <int EPL>
 __global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ chunk_ptr,
-    const float *__restrict__ part, int H, int R, float *__restrict__ dZ, int64_t dz_ld) {
+    const float *__restrict__ part, int H, int R, float *__restrict__ dZ, int64_t dz_ld,
+    __nv_bfloat16 *__restrict__ dZb) {
     extern __shared__ float msm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t slot = blockIdx.x;
@@ -839,7 +851,8 @@ __global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
     }
 #pragma unroll
     for (int x = 0; x < EPL; ++x) acc[x] += dq[x];
-    st_mrow<EPL>(o, acc);
+    if (dZb) st_row<__nv_bfloat16, EPL>(dZb + i * 3 * D + lane * EPL, acc);
+    else st_mrow<EPL>(o, acc);
 }
 
 // dk, dv += the terms of targets [a, b) of source row j (this warp's lanes).
@@ -924,7 +937,7 @@ template <int EPL, bool GTC>
 __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t j, const float (&k)[EPL],
                                           const float (&v)[EPL], float (&dk)[EPL], float (&dv)[EPL],
                                           const float *dSc, const float *dST, int H, int R, float *dZ,
-                                          int64_t dz_ld) {
+                                          int64_t dz_ld, __nv_bfloat16 *dZb) {
     const int D = H * R;
     if constexpr (GTC) {
         if (lh.act) {
@@ -937,8 +950,13 @@ __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t 
                 dk[x] += gk[x];
                 dv[x] += gv[x];
             }
-            st_mrow<EPL>(pk, dk);
-            st_mrow<EPL>(pv, dv);
+            if (dZb) {                                    // the final values in bf16
+                st_row<__nv_bfloat16, EPL>(dZb + j * 3 * D + D + lane * EPL, dk);
+                st_row<__nv_bfloat16, EPL>(dZb + j * 3 * D + 2 * D + lane * EPL, dv);
+            } else {
+                st_mrow<EPL>(pk, dk);
+                st_mrow<EPL>(pv, dv);
+            }
         }
         return;
     } else {
@@ -974,7 +992,8 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
     const int32_t *__restrict__ t_col, const int32_t *__restrict__ chunk_ptr, const float *__restrict__ part,
     const T *__restrict__ Q, const T *__restrict__ KV, const T *__restrict__ dL,
     const float *__restrict__ lse, const float *__restrict__ Dd, const float *__restrict__ dSc,
-    const float *__restrict__ dST, int H, int R, float inv_sqrt_r, float *__restrict__ dZ, int64_t dz_ld) {
+    const float *__restrict__ dST, int H, int R, float inv_sqrt_r, float *__restrict__ dZ, int64_t dz_ld,
+    __nv_bfloat16 *__restrict__ dZb) {
     extern __shared__ float msm[];                       // PARTS: [kMW][2D]
     const int lane = threadIdx.x & 31;
     const int64_t slot = PARTS ? blockIdx.x : (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -1038,7 +1057,7 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
         kv_grad_range<T, EPL>(t_col, Q, dL, lse, Dd, H, D, lane, lh.act, lh.lph, lh.h, inv_sqrt_r, k, v,
                               t_row_ptr[j], t_row_ptr[j + 1], dk, dv);
     }
-    kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
+    kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld, dZb);
 }
 
 // Light source rows with two edges per step: the warp's halves (slots) take alternate
@@ -1053,7 +1072,7 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
     const float *__restrict__ dSc, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
-    float *__restrict__ dZ, int64_t dz_ld) {
+    float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -1164,8 +1183,13 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
                 dk2[x] += gk[x];
                 dv2[x] += gv[x];
             }
-            st_mrow<EPL2>(pk, dk2);
-            st_mrow<EPL2>(pv, dv2);
+            if (dZb) {                                    // the final values in bf16
+                st_row<__nv_bfloat16, EPL2>(dZb + j * 3 * D + D + hl * EPL2, dk2);
+                st_row<__nv_bfloat16, EPL2>(dZb + j * 3 * D + 2 * D + hl * EPL2, dv2);
+            } else {
+                st_mrow<EPL2>(pk, dk2);
+                st_mrow<EPL2>(pv, dv2);
+            }
         }
         return;
     }
@@ -1183,7 +1207,7 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     }
     ld_row<T, EPL>(krow, lane, lh.act, k);
     ld_row<T, EPL>(krow + D, lane, lh.act, v);
-    kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld);
+    kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld, dZb);
 }
 
 // Chunks of heavy source rows, one warp each (layout as bwd_q_chunk_kernel's, over the
@@ -1481,19 +1505,19 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     if constexpr (E == 4 && sizeof(T) == 2) {
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
             bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb);
             return;
         }
     }
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz, nullptr);
             return;
         }
     }
     bwd_local_kv_kernel<T, E, false><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-        nullptr, nullptr, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz);
+        nullptr, nullptr, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz, nullptr);
 }
 
 // Light target rows: two edges per warp step under the same condition as the source side.
@@ -1506,7 +1530,7 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
                 cudaFuncSetAttribute(bwd_local_q2_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kQRingBytes));
             bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
-                Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz, c->bw_dZb);
             return;
         }
     }
@@ -1520,17 +1544,17 @@ template <typename T, int E>
 void launch_kv_heavy(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, const int32_t *kh, int64_t nkh,
                      cudaStream_t sk) {
     const size_t sm = static_cast<size_t>(kMW) * 2 * c->D * 4;
-    auto go = [&](auto kern, const float *dSc, const float *dST) {
+    auto go = [&](auto kern, const float *dSc, const float *dST, __nv_bfloat16 *dZb) {
         if (sm > 48 * 1024)
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
         kern<<<static_cast<unsigned>(nkh), kMW * 32, sm, sk>>>(kh, nkh, c->t_row_ptr, c->t_col, c->bw_k_cptr,
                                                                c->bw_kv_part, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd,
-                                                               dSc, dST, c->H, c->r, isr, c->bw_dZ, Dz);
+                                                               dSc, dST, c->H, c->r, isr, c->bw_dZ, Dz, dZb);
     };
     if constexpr (E == 4 && sizeof(T) == 2) {
-        if (kv_global_tc(c)) return go(bwd_local_kv_kernel<T, E, true, true>, nullptr, nullptr);
+        if (kv_global_tc(c)) return go(bwd_local_kv_kernel<T, E, true, true>, nullptr, nullptr, c->bw_dZb);
     }
-    go(bwd_local_kv_kernel<T, E, true>, c->bw_dSc, c->bw_dST);
+    go(bwd_local_kv_kernel<T, E, true>, c->bw_dSc, c->bw_dST, nullptr);
 }
 
 // Both local backward kernels with EPL = lane_features(D): light rows one warp each;
@@ -1558,7 +1582,7 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
             bwd_q_chunk_kernel<T, E><<<warp_grid(nqc), 256, 0, sq>>>(c->bw_q_chunks, nqc, c->row_ptr,      \
                 c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);               \
             bwd_q_heavy_kernel<E><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, sq>>>(qh, nqh,      \
-                c->bw_q_cptr, c->bw_q_part, H, R, c->bw_dZ, Dz);                                          \
+                c->bw_q_cptr, c->bw_q_part, H, R, c->bw_dZ, Dz, c->bw_dZb);                                          \
         }                                                                                                 \
         break;
     switch (lane_features(c->D)) {
@@ -2564,26 +2588,27 @@ glga_status tc_gemms(Ctx *c, const void *X, float *dX, cudaStream_t s) {
 // dX, dW, dw_g and db_g of a bf16 layer with d = 128 in one pass over dZ (tcgen05):
 //   dX[i][a] = sum_k dZ[i][k] W[a][k] + dt_i w_g[a]            (W = [W_Q | W_K | W_V])
 //   dW[a][k] = sum_i X[i][a] dZ[i][k],  dw_g[a] = sum_i X[i][a] dt_i,  db_g = sum_i dt_i
-// A persistent grid: thread block b takes the 128-row tiles b, b + G, ...  Per tile one
-// producer thread loads by TMA the X tile (two [128][64] bf16 boxes) with dt (a [128][4]
-// float box at column 3D), then per 64-column chunk of dZ two [128][32] float boxes and
-// the [128 a][64 k] block of W that the chunk multiplies.  Warps 0-7 round each dZ chunk
-// to a bf16 tile (128-byte swizzle) and, once per tile, add X^T dt and the sum of dt on
-// the CUDA cores.  One thread issues per chunk the dX MMAs (the bf16 chunk K-major as A,
-// the W block K-major as B: M = 128 rows, N = 128 features) into TMEM columns 0-127 and
-// the dW MMAs (X^T MN-major as A, the bf16 chunk MN-major as B: M = 128 features, N = 64)
-// into the chunk's columns of a [128][3D] accumulator that stays in TMEM over all the
-// block's tiles.  Warps 10-13 drain dX per tile (adding dt w_g) through a staging area
-// into coalesced row stores, and after the last tile write the block's dW partial sums;
-// the range-order reductions add the blocks' partials (the result is the same on every
-// call).  Every wait is bounded: on expiry the kernel raises the context's flag, lets its
-// copies land, waits for its MMAs and returns.
+// dZ's columns 0 .. 3D - 1 come as the bf16 copy the gather kernels write with their
+// final values (dZb [N][3D]); dt stays in the float dZ.  A persistent grid: thread block
+// b takes the 128-row tiles b, b + G, ...  Per tile one producer thread loads by TMA the
+// X tile (two [128][64] bf16 boxes) with dt (a [128][4] float box at column 3D), then per
+// 64-column chunk the [128][64] bf16 dZ box and the [128 a][64 k] block of W it
+// multiplies, into a four-stage ring.  One thread issues per chunk the dX MMAs (the dZ
+// chunk K-major as A, the W block K-major as B: M = 128 rows, N = 128 features) into
+// TMEM columns 0-127 and the dW MMAs (X^T MN-major as A, the dZ chunk MN-major as B:
+// M = 128 features, N = 64) into the chunk's columns of a [128][3D] accumulator that stays
+// in TMEM over all the block's tiles.  Warps 0-7 add X^T dt and the sum of dt on the CUDA
+// cores; warps 10-13 drain dX per tile (adding dt w_g) through a staging area into
+// coalesced row stores, and after the last tile write the block's dW partial sums; the
+// range-order reductions add the blocks' partials (the result is the same on every call).
+// Every wait is bounded: on expiry the kernel raises the context's flag, lets its copies
+// land, waits for its MMAs and returns.
 constexpr int kFxRows = 128;
-constexpr int kFxXStages = 2, kFxFStages = 4, kFxBStages = 2;
+constexpr int kFxXStages = 2, kFxBStages = 4;
 constexpr uint32_t kFxBox = kFxRows * 128;                  // a [128][128 B] box: 16 KB
 constexpr uint32_t kFxXStage = 2 * kFxBox + kFxRows * 16;   // X tile, then the dt box
 constexpr uint32_t kFxBStage = 2 * kFxBox;                  // bf16 dZ chunk, then the W block
-constexpr uint32_t kFxEpi = kFxXStages * kFxXStage + kFxFStages * kFxBox + kFxBStages * kFxBStage;
+constexpr uint32_t kFxEpi = kFxXStages * kFxXStage + kFxBStages * kFxBStage;
 constexpr uint32_t kFxEpiStage = 4096;                      // per epilogue warp
 constexpr size_t kFxSmem = 1024 + kFxEpi + 4 * kFxEpiStage + (128 + 256 + 2) * sizeof(float);
 constexpr int kFxWorkers = 256, kFxProd = 8, kFxMma = 9, kFxEpi0 = 10, kFxThreads = 448;
@@ -2606,15 +2631,13 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
     const __grid_constant__ CUtensorMap tmWk, const __grid_constant__ CUtensorMap tmWv, FxParams p) {
     extern __shared__ uint8_t dsmem_raw[];
     __shared__ __align__(8) uint64_t x_full[kFxXStages], x_empty[kFxXStages];
-    __shared__ __align__(8) uint64_t f_full[kFxFStages], f_empty[kFxFStages];
-    __shared__ __align__(8) uint64_t w_full[kFxBStages], b_full[kFxBStages], b_empty[kFxBStages];
+    __shared__ __align__(8) uint64_t b_full[kFxBStages], b_empty[kFxBStages];
     __shared__ __align__(8) uint64_t dx_full, dx_empty, mma_done;
     __shared__ uint32_t tmem_base_sh;
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *sX = smem;                                      // [kFxXStages] X tile + dt
-    uint8_t *sF = sX + kFxXStages * kFxXStage;               // [kFxFStages] float dZ boxes
-    uint8_t *sB = sF + kFxFStages * kFxBox;                  // [kFxBStages] bf16 chunk + W block
+    uint8_t *sB = sX + kFxXStages * kFxXStage;               // [kFxBStages] dZ chunk + W block
     uint8_t *sE = smem + kFxEpi;                             // epilogue staging
     float *swg = reinterpret_cast<float *>(sE + 4 * kFxEpiStage);   // w_g as float
     float *sred = swg + 128;                                 // [256] + [2] worker sums
@@ -2628,13 +2651,8 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
             mbar_init(&x_full[s], 1);
             mbar_init(&x_empty[s], 1 + kFxWorkers / 32 + 4);   // MMA commit, workers, epilogue
         }
-        for (int s = 0; s < kFxFStages; ++s) {
-            mbar_init(&f_full[s], 1);
-            mbar_init(&f_empty[s], kFxWorkers / 32);
-        }
         for (int s = 0; s < kFxBStages; ++s) {
-            mbar_init(&w_full[s], 1);
-            mbar_init(&b_full[s], kFxWorkers / 32);
+            mbar_init(&b_full[s], 1);
             mbar_init(&b_empty[s], 1);
         }
         mbar_init(&dx_full, 1);
@@ -2657,7 +2675,7 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
             tma_prefetch_desc(&tmX);
             tma_prefetch_desc(&tmZ);
             bool ok = true;
-            int nx = 0, nf = 0, nb = 0;                          // loads issued per ring
+            int nx = 0, nb = 0;                                  // loads issued per ring
             for (int j = 0; j < my && ok; ++j) {
                 const int32_t y = (blk + j * G) * kFxRows;
                 const int xs = nx % kFxXStages;
@@ -2671,26 +2689,17 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
                 tma_load_2d(xst + kFxBox, &tmX, &x_full[xs], 64, y);
                 tma_load_2d(xst + 2 * kFxBox, &tmDt, &x_full[xs], p.Kc, y);
                 ++nx;
-                for (int cc = 0; cc < nc && ok; ++cc) {
-                    for (int h = 0; h < 2; ++h) {
-                        const int fs = nf % kFxFStages;
-                        if (nf >= kFxFStages && !mbar_wait_bounded(&f_empty[fs], ((nf / kFxFStages) - 1) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(&f_full[fs], kFxBox);
-                        tma_load_2d(sF + fs * kFxBox, &tmZ, &f_full[fs], cc * 64 + h * 32, y);
-                        ++nf;
-                    }
-                    if (!ok) break;
+                for (int cc = 0; cc < nc; ++cc) {
                     const int bs = nb % kFxBStages;
                     if (nb >= kFxBStages && !mbar_wait_bounded(&b_empty[bs], ((nb / kFxBStages) - 1) & 1)) {
                         ok = false;
                         break;
                     }
                     const CUtensorMap *wm = cc < cpm ? &tmWq : (cc < 2 * cpm ? &tmWk : &tmWv);
-                    mbar_arrive_expect_tx(&w_full[bs], kFxBox);
-                    tma_load_2d(sB + bs * kFxBStage + kFxBox, wm, &w_full[bs], (cc % cpm) * 64, 0);
+                    uint8_t *bst = sB + bs * kFxBStage;
+                    mbar_arrive_expect_tx(&b_full[bs], kFxBStage);
+                    tma_load_2d(bst, &tmZ, &b_full[bs], cc * 64, y);
+                    tma_load_2d(bst + kFxBox, wm, &b_full[bs], (cc % cpm) * 64, 0);
                     ++nb;
                 }
             }
@@ -2698,10 +2707,8 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
             // the block leaves only after its copies have landed (already so when all went well)
             for (int i = std::max(0, nx - kFxXStages); i < nx; ++i)
                 mbar_wait_bounded(&x_full[i % kFxXStages], (i / kFxXStages) & 1);
-            for (int i = std::max(0, nf - kFxFStages); i < nf; ++i)
-                mbar_wait_bounded(&f_full[i % kFxFStages], (i / kFxFStages) & 1);
             for (int i = std::max(0, nb - kFxBStages); i < nb; ++i)
-                mbar_wait_bounded(&w_full[i % kFxBStages], (i / kFxBStages) & 1);
+                mbar_wait_bounded(&b_full[i % kFxBStages], (i / kFxBStages) & 1);
         }
     } else if (warp == kFxMma) {
         if (lane == 0) {
@@ -2720,8 +2727,7 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
                 const uint32_t xa = smem_u32(sX + xs * kFxXStage);
                 for (int cc = 0; cc < nc; ++cc, ++nb) {
                     const int bs = nb % kFxBStages;
-                    const uint32_t par = static_cast<uint32_t>(nb / kFxBStages) & 1u;
-                    if (!mbar_wait_bounded(&w_full[bs], par) || !mbar_wait_bounded(&b_full[bs], par)) {
+                    if (!mbar_wait_bounded(&b_full[bs], static_cast<uint32_t>(nb / kFxBStages) & 1u)) {
                         ok = false;
                         break;
                     }
@@ -2745,46 +2751,12 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
             umma_commit(&mma_done);
         }
     } else if (warp < kFxWorkers / 32) {
-        // ---------------- warps 0-7: dZ chunks to bf16; X^T dt and the sum of dt -------------
+        // ---------------- warps 0-7: X^T dt and the sum of dt ----------------------------
         const int t = threadIdx.x, fa = t & 127, hh = t >> 7;   // feature, half of the tile's rows
         bool ok = true;
-        int nf = 0, nb = 0;
         float accg = 0.f, accb = 0.f;
         for (int j = 0; j < my && ok; ++j) {
             const int xs = j % kFxXStages;
-            for (int cc = 0; cc < nc; ++cc) {
-                const int fs0 = nf % kFxFStages, fs1 = (nf + 1) % kFxFStages, bs = nb % kFxBStages;
-                const bool got = mbar_wait_bounded(&f_full[fs0], (nf / kFxFStages) & 1) &&
-                                 mbar_wait_bounded(&f_full[fs1], ((nf + 1) / kFxFStages) & 1) &&
-                                 (nb < kFxBStages || mbar_wait_bounded(&b_empty[bs], ((nb / kFxBStages) - 1) & 1));
-                // the warp agrees on the outcome, so it stays converged for its arrivals
-                if (!__all_sync(0xffffffffu, got)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t *f0 = sF + fs0 * kFxBox, *f1 = sF + fs1 * kFxBox;
-                uint8_t *bt = sB + bs * kFxBStage;
-                // one 16-byte chunk (8 columns of one row) of the bf16 tile per step
-                for (int it = t; it < kFxRows * 8; it += kFxWorkers) {
-                    const int k = it >> 3, co = it & 7, j0 = (co & 3) * 2;
-                    const uint8_t *zr = (co < 4 ? f0 : f1) + k * 128;
-                    const float4 u = *reinterpret_cast<const float4 *>(zr + ((j0 ^ (k & 7)) << 4));
-                    const float4 v = *reinterpret_cast<const float4 *>(zr + (((j0 + 1) ^ (k & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(bt + k * 128 + ((co ^ (k & 7)) << 4)) =
-                        make_uint4(bf16x2_bits(u.x, u.y), bf16x2_bits(u.z, u.w), bf16x2_bits(v.x, v.y),
-                                   bf16x2_bits(v.z, v.w));
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&f_empty[fs0]);
-                    mbar_arrive(&f_empty[fs1]);
-                    mbar_arrive(&b_full[bs]);
-                }
-                nf += 2;
-                ++nb;
-            }
-            if (!ok) break;
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&x_full[xs], (j / kFxXStages) & 1))) {
                 ok = false;
                 break;
@@ -2878,10 +2850,11 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
 }
 
 // Whether dX and the weight gradients of this context take the one-pass kernel: bf16
-// layers with d = 128 and D a multiple of 64 up to 128 (dX and dW fit TMEM together).
-bool bwd_fx(const Ctx *c) {
-    return c->io == GLGA_BF16 && c->d == 128 && c->D % 64 == 0 && c->D <= 128 && c->N > 0;
-}
+// layers with d = 128 whose source side's global terms run on the tensor cores (H*r = 128,
+// r in {16, 32, 64}): dX and dW fit TMEM together, and the gather kernels that finish
+// dZ's columns (light rows two edges per step, heavy rows chunk sums) also write its
+// bf16 copy.
+bool bwd_fx(const Ctx *c) { return c->io == GLGA_BF16 && c->d == 128 && kv_global_tc(c) && c->N > 0; }
 
 // dX, and the dW / dw_g / db_g partials that the reductions after it add
 // (over c->bw_fx_parts blocks), in one pass over dZ.
@@ -2893,8 +2866,8 @@ glga_status fx_gemms(Ctx *c, const void *X, const void *WQ, const void *WK, cons
     glga_status st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 128, static_cast<uint64_t>(N), 256,
                                     64, kFxRows);
     if (st == GLGA_OK)
-        st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dZ, static_cast<uint64_t>(Kc),
-                            static_cast<uint64_t>(N), zrow, 32, kFxRows);
+        st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->bw_dZb, static_cast<uint64_t>(Kc),
+                            static_cast<uint64_t>(N), static_cast<uint64_t>(Kc) * 2, 64, kFxRows);
     if (st == GLGA_OK)
         st = encode_tmap_2d(&mdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dZ, static_cast<uint64_t>(c->bw_dz_ld),
                             static_cast<uint64_t>(N), zrow, 4, kFxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -3036,6 +3009,8 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dSc), static_cast<size_t>(H) * R * (R + 1) * f));
     // the one-pass dX / dW kernel: one thread block per SM, each with at least one row tile
     c->bw_fx_parts = bwd_fx(c) ? static_cast<int32_t>(std::min<int64_t>(c->num_sms, ceil_div(N, kFxRows))) : 0;
+    if (bwd_fx(c))   // the bf16 copy of dZ's columns 0 .. 3D - 1 it reads
+        BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dZb), nz * 3 * D * sizeof(__nv_bfloat16)));
     const int64_t gparts = std::max<int64_t>(c->bw_wparts, c->bw_fx_parts);
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dw_part),
                    static_cast<size_t>(gparts) * c->d * (3 * D + 1) * f));

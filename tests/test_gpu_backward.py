@@ -144,11 +144,12 @@ def test_tensor_core_readout_backward(H, r, N):
     _check(w, seed=H, chunked=N > 5000)
 
 
-@pytest.mark.parametrize("H,r,N", [(2, 32, 100), (1, 64, 300), (4, 32, 148 * 128 + 77)])
+@pytest.mark.parametrize("H,r,N", [(8, 16, 100), (2, 64, 300), (4, 32, 148 * 128 + 77)])
 def test_one_pass_dx_dw(H, r, N):
-    # bf16 layers with d = 128 form dX, dW, dw_g and db_g in one tensor-core pass over dZ
-    # (dX and the whole dW block in TMEM together): D = 64 and D = 128, a single ragged
-    # 128-row tile, and more tiles than thread blocks with a ragged last one
+    # bf16 layers with d = 128 and H*r = 128 form dX, dW, dw_g and db_g in one tensor-core
+    # pass over the bf16 copy of dZ that the gather kernels write (dX and the whole dW
+    # block in TMEM together): every head width, a single ragged 128-row tile (rows without
+    # in-edges among them), and more tiles than thread blocks with a ragged last one
     rng = np.random.default_rng(N + H)
     src = np.concatenate([rng.integers(0, N, 3 * N), np.arange(N)]).astype(np.int32)
     dst = np.concatenate([np.repeat(np.arange(N), 3), np.arange(N)]).astype(np.int32)
