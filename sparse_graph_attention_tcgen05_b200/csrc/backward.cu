@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(256) bwd_strided_sum_kernel(const float *__res
 }
 
 constexpr int kEU = 4;            // edges whose rows are loaded before any is used
-constexpr int kChunk = 32;        // edges per chunk of a heavy row (one warp each)
+constexpr int kChunk = 64;        // edges per chunk of a heavy row (one warp each)
 
 // The lane's EPL bf16 values of a row (EPL even) as EPL / 2 packed words (zero if !act).
 template <int EPL>
@@ -625,20 +625,33 @@ constexpr size_t kQRingBytes = 8 * 2 * 2 * 2 * 32 * 16;   // 8 warps x 2 steps x
 // v_j, so a step's two edges share one shuffle butterfly and one exponential per lane.
 // The halves' dq are added (the same sum in both), moved to the 32-lane layout and added
 // into dZ [:, 0:D].  Needs 2 EPL <= r.
-template <typename T, int EPL>
+// With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
+// kChunk entries at most) and write their shares of dq_i to part[w][0:D].
+template <typename T, int EPL, bool CH = false>
 __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
-    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb) {
+    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb,
+    const int2 *__restrict__ chunks, float *__restrict__ part) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     if (w >= n_rows) return;                              // warp-uniform
-    const int64_t i = rows[w];
-    const int32_t a = row_ptr[i], b = row_ptr[i + 1];
+    int64_t i;
+    int32_t a, b;
+    if constexpr (CH) {
+        const int2 ch = chunks[w];
+        i = ch.x;
+        a = ch.y;
+        b = min(row_ptr[i + 1], ch.y + kChunk);
+    } else {
+        i = rows[w];
+        a = row_ptr[i];
+        b = row_ptr[i + 1];
+    }
     const int D = H * R;
-    if (a == b) {                                         // no local term
+    if (!CH && a == b) {                                  // no local term
         if (dZb) {                                        // dq_i = its global part, in bf16
             const LaneHead lh(lane, EPL, D, R);
             if (lh.act) {
@@ -755,6 +768,10 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     for (int x = 0; x < EPL; ++x) {
         const float q0 = __shfl_sync(0xffffffffu, dq2[x], src), q1 = __shfl_sync(0xffffffffu, dq2[EPL + x], src);
         dq[x] = hi ? q1 : q0;
+    }
+    if constexpr (CH) {
+        if (lh.act) st_mrow<EPL>(part + w * D + lane * EPL, dq);
+        return;
     }
     if (lh.act) {
         float *o = dZ + i * dz_ld + lane * EPL;
@@ -1066,18 +1083,21 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
 // edges of a step share one shuffle butterfly and one exponential per lane.  The halves'
 // dk, dv are then added (lower + upper, the same sum in both) and moved to the 32-lane
 // layout for kv_finish.  Needs 2 EPL <= r.
-template <typename T, int EPL, bool GTC = false>
+// With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
+// kChunk entries at most) and write their shares of dk_j | dv_j to part[w][0:2D].
+template <typename T, int EPL, bool GTC = false, bool CH = false>
 __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
     const float *__restrict__ dSc, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
-    float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb) {
+    float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb, const int2 *__restrict__ chunks,
+    float *__restrict__ part) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
     if (w >= n_rows) return;                              // warp-uniform
-    const int64_t j = rows[w];
+    const int64_t j = CH ? static_cast<int64_t>(chunks[w].x) : static_cast<int64_t>(rows[w]);
     const int D = H * R;
     const bool act2 = hl * EPL2 < D;
     const int lph2 = R / EPL2, h2 = act2 ? hl * EPL2 / R : 0;
@@ -1087,7 +1107,8 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     ld_row<T, EPL2>(krow + D, hl, act2, v2);
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dk2[x] = dv2[x] = 0.f;
-    const int32_t a = t_row_ptr[j], b = t_row_ptr[j + 1];
+    const int32_t a = CH ? chunks[w].y : t_row_ptr[j];
+    const int32_t b = CH ? min(t_row_ptr[j + 1], chunks[w].y + kChunk) : t_row_ptr[j + 1];
     auto use_step = [&](int32_t e0, const float (&q)[kU][EPL2], const float (&dl)[kU][EPL2], const float (&ls)[kU],
                         const float (&dd)[kU]) {
 #pragma unroll
@@ -1170,6 +1191,13 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     for (int x = 0; x < EPL2; ++x) {
         dk2[x] += __shfl_xor_sync(0xffffffffu, dk2[x], 16);
         dv2[x] += __shfl_xor_sync(0xffffffffu, dv2[x], 16);
+    }
+    if constexpr (CH) {                                   // the chunk's share, 8-feature slices
+        if (slot == 0 && act2) {
+            st_mrow<EPL2>(part + w * 2 * D + hl * EPL2, dk2);
+            st_mrow<EPL2>(part + w * 2 * D + D + hl * EPL2, dv2);
+        }
+        return;
     }
     if constexpr (GTC) {
         // the global terms are in dZ already: the lower half adds its 8-feature slices
@@ -1505,14 +1533,16 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     if constexpr (E == 4 && sizeof(T) == 2) {
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
             bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb,
+                nullptr, nullptr);
             return;
         }
     }
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
-                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz, nullptr);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz, nullptr,
+                nullptr, nullptr);
             return;
         }
     }
@@ -1530,12 +1560,47 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
                 cudaFuncSetAttribute(bwd_local_q2_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kQRingBytes));
             bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
-                Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz, c->bw_dZb);
+                Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz, c->bw_dZb,
+                nullptr, nullptr);
             return;
         }
     }
     bwd_local_q_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx, Q, KV,
         static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz);
+}
+
+// Chunks of heavy source / target rows: the two-edges-per-step kernels in chunk mode where
+// the light rows use them, else one edge per step across the warp.
+template <typename T, int E>
+void launch_kv_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t sk) {
+    const int64_t nkc = c->bw_nk_chunks;
+    if constexpr (E <= 4) {
+        if (2 * E <= c->r) {
+            bwd_local_kv2_kernel<T, E, false, true><<<warp_grid(nkc), 256, 0, sk>>>(nullptr, nkc, c->t_row_ptr,
+                c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r,
+                isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part);
+            return;
+        }
+    }
+    bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, sk>>>(c->bw_k_chunks, nkc, c->t_row_ptr, c->t_col, Q, KV,
+        static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->H, c->r, isr, c->bw_kv_part);
+}
+template <typename T, int E>
+void launch_q_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t sq) {
+    const int64_t nqc = c->bw_nq_chunks;
+    if constexpr (E <= 4) {
+        if (2 * E <= c->r) {
+            if (kQRing<T, E> && kQRingBytes > 48 * 1024)
+                cudaFuncSetAttribute(bwd_local_q2_kernel<T, E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kQRingBytes));
+            bwd_local_q2_kernel<T, E, true><<<warp_grid(nqc), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(nullptr, nqc,
+                c->row_ptr, c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd,
+                nullptr, 0, nullptr, c->bw_q_chunks, c->bw_q_part);
+            return;
+        }
+    }
+    bwd_q_chunk_kernel<T, E><<<warp_grid(nqc), 256, 0, sq>>>(c->bw_q_chunks, nqc, c->row_ptr, c->col_idx, Q, KV,
+        static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);
 }
 
 // Heavy source rows: chunk sums, then the global terms (or, with the tensor-core global
@@ -1573,14 +1638,12 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
     case E:                                                                                               \
         if (nkl) launch_kv_light<T, E>(c, Q, KV, isr, Dz, sk);                                           \
         if (nkh) {                                                                                        \
-            bwd_kv_chunk_kernel<T, E><<<warp_grid(nkc), 256, 0, sk>>>(c->bw_k_chunks, nkc, c->t_row_ptr,   \
-                c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, H, R, isr, c->bw_kv_part);                \
+            launch_kv_chunks<T, E>(c, Q, KV, isr, sk);                                                   \
             launch_kv_heavy<T, E>(c, Q, KV, isr, Dz, kh, nkh, sk);                                      \
         }                                                                                                 \
         if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                            \
         if (nqh) {                                                                                        \
-            bwd_q_chunk_kernel<T, E><<<warp_grid(nqc), 256, 0, sq>>>(c->bw_q_chunks, nqc, c->row_ptr,      \
-                c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), H, R, isr, c->bw_lse, c->bw_Dd, c->bw_q_part);               \
+            launch_q_chunks<T, E>(c, Q, KV, isr, sq);                                                    \
             bwd_q_heavy_kernel<E><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, sq>>>(qh, nqh,      \
                 c->bw_q_cptr, c->bw_q_part, H, R, c->bw_dZ, Dz, c->bw_dZb);                                          \
         }                                                                                                 \
