@@ -690,8 +690,13 @@ __device__ __forceinline__ void block_edges(const LocalParams &p, const uint4 (&
 constexpr int local_min_blocks(int VPL, int U, bool PIPE) {
     return ((PIPE ? 2 : 1) * U * VPL * 8 <= 32 && VPL <= 2) ? 3 : 2;
 }
+// The gather-ring layout with one vector per lane runs four blocks per SM (64 registers);
+// the log-sum-exp store would otherwise take it to 71 registers and three blocks.
+constexpr int local_min_blocks_opt(int VPL, int U, bool PIPE, bool LSE, int OPT) {
+    return (LSE && (OPT & kOptAsync) != 0 && VPL == 1 && U <= 2 && !PIPE) ? 4 : local_min_blocks(VPL, U, PIPE);
+}
 template <typename T, int NV, int LPH, int VPL, int U, bool DBG, bool J, bool LSE, bool PIPE, bool CB, int OPT>
-__global__ void __launch_bounds__(kLocalThreads, local_min_blocks(VPL, U, PIPE))
+__global__ void __launch_bounds__(kLocalThreads, local_min_blocks_opt(VPL, U, PIPE, LSE, OPT))
     local_kernel(const LocalParams p) {
     using Sh = Shape<T, NV, LPH, VPL, J>;
     using St = State<T, VPL, J>;
