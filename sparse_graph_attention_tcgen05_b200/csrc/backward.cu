@@ -1756,7 +1756,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmY,
     const __grid_constant__ CUtensorMap tmL, const float *__restrict__ t, const __nv_bfloat16 *__restrict__ Bg,
     int ro_kp, const float *__restrict__ Sz, int64_t N, int H, float b_g, float eps, __nv_bfloat16 *__restrict__ dL,
-    float *__restrict__ Dd, float *__restrict__ dnum, float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
+    float *__restrict__ Dd, __nv_bfloat16 *__restrict__ dnum, float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
     constexpr int D = kBroTcD;
     constexpr int kHQ = R >= 32 ? 1 : 32 / R;     // heads in a 32-column quarter
     constexpr uint32_t kTile = 2 * kBroTcAtom;    // a [128][128] bf16 tile
@@ -1950,19 +1950,17 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
                 dda[hq] = fmaf(dG, G, dda[hq]);
                 dtp = fmaf(y, bf(lw, j) - G, dtp);
             }
+            // dnum in bf16: the second MMA's A operand, in place of the warp's own dY slice,
+            // and the rows the dS | dz kernel reads
 #pragma unroll
-            for (int p = 0; p < 4; ++p)
-                stage_row64_piece(stg, lane, p, make_uint4(__float_as_uint(dn[4 * p]), __float_as_uint(dn[4 * p + 1]),
-                                                           __float_as_uint(dn[4 * p + 2]), __float_as_uint(dn[4 * p + 3])));
-            warp_rows64_flush(reinterpret_cast<uint8_t *>(dnum + c0 + 16 * hb), static_cast<int64_t>(D + 16) * 4, r0, N,
-                              stg, lane);
-            // A = dnum in bf16, in place of the warp's own dY slice
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                *reinterpret_cast<uint4 *>(sY + swz_off(rt, c0 + 16 * hb + 8 * i, kBroTcAtom)) =
-                    make_uint4(bf16x2_bits(dn[8 * i], dn[8 * i + 1]), bf16x2_bits(dn[8 * i + 2], dn[8 * i + 3]),
-                               bf16x2_bits(dn[8 * i + 4], dn[8 * i + 5]), bf16x2_bits(dn[8 * i + 6], dn[8 * i + 7]));
+            for (int i = 0; i < 2; ++i) {
+                const uint4 wv = make_uint4(bf16x2_bits(dn[8 * i], dn[8 * i + 1]), bf16x2_bits(dn[8 * i + 2], dn[8 * i + 3]),
+                                            bf16x2_bits(dn[8 * i + 4], dn[8 * i + 5]), bf16x2_bits(dn[8 * i + 6], dn[8 * i + 7]));
+                *reinterpret_cast<uint4 *>(sY + swz_off(rt, c0 + 16 * hb + 8 * i, kBroTcAtom)) = wv;
+                stage_row64_piece(stg, lane, 2 * hb + i, wv);
+            }
         }
+        warp_rows64_flush(reinterpret_cast<uint8_t *>(dnum + c0), static_cast<int64_t>(D + 16) * 2, r0, N, stg, lane);
         xdt[cq * 128 + rt] = dtp;
         xdd[cq * 128 + rt] = dda[0];
         xDd[cq * 128 + rt] = Dda[0];
@@ -1982,7 +1980,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             const float s_Dd = xDd[q0 * 128 + rt] + xDd[(q0 + 1) * 128 + rt];
             ddh[0] = -s_dd * inv[0];
             if (valid && (cq & 1) == 0) {
-                dnum[row * (D + 16) + D + c0 / R] = ddh[0];
+                dnum[row * (D + 16) + D + c0 / R] = __float2bfloat16_rn(ddh[0]);
                 Dd[row * H + c0 / R] = s_Dd;
             }
         } else {
@@ -1990,7 +1988,7 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             for (int hq = 0; hq < kHQ; ++hq) {
                 ddh[hq] = -dda[hq] * inv[hq];
                 if (valid) {
-                    dnum[row * (D + 16) + D + c0 / R + hq] = ddh[hq];
+                    dnum[row * (D + 16) + D + c0 / R + hq] = __float2bfloat16_rn(ddh[hq]);
                     Dd[row * H + c0 / R + hq] = Dda[hq];
                 }
             }
@@ -2285,7 +2283,8 @@ glga_status launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfl
     if (st != GLGA_OK) return st;
     bwd_readout_tc_kernel<R><<<grid, kBroTcWarps * 32, kBroTcSmem, s>>>(
         mq, my, ml, c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz, c->N, c->H, b_g, eps,
-        static_cast<__nv_bfloat16 *>(c->bw_dL), c->bw_Dd, c->bw_dnum, c->bw_dZ, Dz, c->dev_flag);
+        static_cast<__nv_bfloat16 *>(c->bw_dL), c->bw_Dd, reinterpret_cast<__nv_bfloat16 *>(c->bw_dnum), c->bw_dZ, Dz,
+        c->dev_flag);
     return GLGA_OK;
 }
 
@@ -2371,13 +2370,13 @@ constexpr uint32_t kDwBox = kDwRows * 128;                 // one 64-row box of 
 constexpr uint32_t kDwXBytes = 2 * kDwBox;                 // X tile (bf16)
 constexpr uint32_t kDwZBytes = 4 * kDwBox;                 // dZ tile (float32)
 constexpr uint32_t kDwStage = kDwXBytes + kDwZBytes + 2 * kDwBox;   // + dZ rounded to bf16
-// the dS | dz form: [dnum | dden] tiles of 144 columns, the dden part a [64][16] float box
-// without swizzle, rounded into a bf16 tile of three 64-column atoms; two stages
-constexpr int kDszStages = 2;
-constexpr uint32_t kDszDBytes = kDwRows * 64;
-constexpr uint32_t kDszZBytes = kDwZBytes + kDszDBytes;
-constexpr uint32_t kDszStage = kDwXBytes + kDszZBytes + 3 * kDwBox;
-static_assert((kDwXBytes + kDszZBytes) % 1024 == 0 && kDszStage % 1024 == 0, "1024-byte aligned tiles");
+// the dS | dz form: bf16 [dnum | dden] rows of 144 columns loaded by TMA straight into a B
+// tile of three 64-column atoms (columns 144 .. 191 past the rows' end read as zero); four
+// stages
+constexpr int kDszStages = 4;
+constexpr uint32_t kDszZBytes = 0;
+constexpr uint32_t kDszStage = kDwXBytes + 3 * kDwBox;
+static_assert(kDszStage % 1024 == 0, "1024-byte aligned tiles");
 
 struct DwParams {
     int64_t N;
@@ -2389,14 +2388,14 @@ struct DwParams {
 };
 
 // With DSZ the same kernel forms the readout's dS | dz partials: X = Q with phi applied to
-// each landed tile, dZ = [dnum | dden] (float32 rows of D + 16 columns, dden_h in column
-// D + h; tmD loads the 16 dden columns), one M = 128, N = 144 MMA per 16 rows, and the
-// epilogue keeps the diagonal head blocks and the dden column in the layout
-// [P][H][R][R + 1] (column R = dz) that bwd_sum_parts_kernel adds.
+// each landed tile, dZ = [dnum | dden] (bf16 rows of D + 16 columns, dden_h in column
+// D + h, loaded as the B operand itself: the ranges are whole 64-row tiles, so no row
+// needs zeroing), one M = 128, N = 144 MMA per 16 rows, and the epilogue keeps the
+// diagonal head blocks and the dden column in the layout [P][H][R][R + 1] (column R = dz)
+// that bwd_sum_parts_kernel adds.
 template <bool DSZ>
 __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                                   const __grid_constant__ CUtensorMap tmZ,
-                                                                  const __grid_constant__ CUtensorMap tmD,
                                                                   DwParams p) {
     constexpr int kStages = DSZ ? kDszStages : kDwStages;
     constexpr uint32_t kZBytes = DSZ ? kDszZBytes : kDwZBytes;
@@ -2449,12 +2448,18 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
                     break;
                 }
                 uint8_t *st = smem + static_cast<size_t>(s) * kStageBytes;
-                mbar_arrive_expect_tx(&full_bar[s], kDwXBytes + kZBytes);
                 const int32_t y = static_cast<int32_t>(r0 + static_cast<int64_t>(it) * kDwRows);
-                for (int b = 0; b < 2; ++b) tma_load_2d(st + b * kDwBox, &tmX, &full_bar[s], fa * 128 + b * 64, y);
-                for (int b = 0; b < 4; ++b)
-                    tma_load_2d(st + kDwXBytes + b * kDwBox, &tmZ, &full_bar[s], fb * 128 + b * 32, y);
-                if constexpr (DSZ) tma_load_2d(st + kDwXBytes + kDwZBytes, &tmD, &full_bar[s], p.d, y);
+                if constexpr (DSZ) {
+                    mbar_arrive_expect_tx(&full_bar[s], kDszStage);
+                    for (int b = 0; b < 2; ++b) tma_load_2d(st + b * kDwBox, &tmX, &full_bar[s], b * 64, y);
+                    for (int b = 0; b < 3; ++b) tma_load_2d(st + kDwXBytes + b * kDwBox, &tmZ, &full_bar[s], b * 64, y);
+                } else {
+                    mbar_arrive_expect_tx(&full_bar[s], kDwXBytes + kZBytes);
+                    for (int b = 0; b < 2; ++b)
+                        tma_load_2d(st + b * kDwBox, &tmX, &full_bar[s], fa * 128 + b * 64, y);
+                    for (int b = 0; b < 4; ++b)
+                        tma_load_2d(st + kDwXBytes + b * kDwBox, &tmZ, &full_bar[s], fb * 128 + b * 32, y);
+                }
                 ++issued;
             }
             if (!ok) {
@@ -2503,30 +2508,16 @@ __global__ void __launch_bounds__(kDwThreads, 1) bwd_dw_tc_kernel(const __grid_c
             uint8_t *bt = smem + static_cast<size_t>(s) * kStageBytes + kDwXBytes + kZBytes;
             const int64_t y0 = r0 + static_cast<int64_t>(it) * kDwRows;
             if constexpr (DSZ) {
-                // phi of the q tile in place (rows past the range meet zero dZ rows)
+                // phi of the q tile in place (rows past N are zero in both tiles)
                 uint4 *xq = reinterpret_cast<uint4 *>(smem + static_cast<size_t>(s) * kStageBytes);
                 for (int cidx = threadIdx.x; cidx < static_cast<int>(kDwXBytes / 16); cidx += kDwWorkers) {
                     const uint4 u = xq[cidx];
                     xq[cidx] = make_uint4(phi_bf16x2(u.x), phi_bf16x2(u.y), phi_bf16x2(u.z), phi_bf16x2(u.w));
                 }
             }
-            // one 16-byte chunk of the bf16 tile (8 consecutive columns of one row) per step;
-            // with DSZ two more per row carry the dden columns into the third atom
-            constexpr int kChunks = DSZ ? 18 : 16;
-            for (int cidx = threadIdx.x; cidx < kDwRows * kChunks; cidx += kDwWorkers) {
-                const int k = cidx / kChunks, ch = cidx - k * kChunks;
-                if (DSZ && ch >= 16) {
-                    const int co = ch - 16;
-                    uint4 w = make_uint4(0, 0, 0, 0);
-                    if (y0 + k < r1) {
-                        const float4 *dr = reinterpret_cast<const float4 *>(z + kDwZBytes + k * 64 + co * 32);
-                        const float4 a = dr[0], b = dr[1];
-                        w = make_uint4(bf16x2_bits(a.x, a.y), bf16x2_bits(a.z, a.w), bf16x2_bits(b.x, b.y),
-                                       bf16x2_bits(b.z, b.w));
-                    }
-                    *reinterpret_cast<uint4 *>(bt + 2 * kDwBox + k * 128 + ((co ^ (k & 7)) * 16)) = w;
-                    continue;
-                }
+            // one 16-byte chunk of the bf16 tile (8 consecutive columns of one row) per step
+            for (int cidx = threadIdx.x; !DSZ && cidx < kDwRows * 16; cidx += kDwWorkers) {
+                const int k = cidx >> 4, ch = cidx & 15;
                 const int bo = ch >> 3, co = ch & 7;            // bf16 box, chunk in its row
                 const int g0 = bo * 64 + co * 8;                // first column in the tile
                 const int bi = g0 >> 5, j0 = (g0 & 31) >> 2;    // float32 box, its first chunk
@@ -2638,7 +2629,7 @@ glga_status tc_gemms(Ctx *c, const void *X, float *dX, cudaStream_t s) {
                                    static_cast<int>(smem)));
     const dim3 grid(static_cast<unsigned>(c->bw_dwtc_parts), static_cast<unsigned>(ceil_div(d, 128)),
                     static_cast<unsigned>(ceil_div(Kc, 128)));
-    bwd_dw_tc_kernel<false><<<grid, kDwThreads, smem, s>>>(mx, mz, mz, p);
+    bwd_dw_tc_kernel<false><<<grid, kDwThreads, smem, s>>>(mx, mz, p);
     GLGA_CUDA(cudaGetLastError());
     const int64_t total = static_cast<int64_t>(d) * Kc;
     bwd_sum_parts_kernel<<<sum_parts_grid(total), kSumThreads, 0, s>>>(
@@ -2968,18 +2959,14 @@ glga_status launch_dsz_bwd(Ctx *c, const T *Q, cudaStream_t s) {
     const int64_t rpp = c->bw_dsz_rpp;
     if constexpr (sizeof(T) == 2) {
         if (readout_bwd_tc(c)) {
-            // tcgen05: X = Q [N][D] (phi applied per tile), dZ = [dnum | dden] [N][D + 16]
+            // tcgen05: X = Q [N][D] (phi applied per tile), dZ = bf16 [dnum | dden] [N][D + 16]
             const int64_t N = c->N, D = c->D;
-            CUtensorMap mx, mz, md;
+            CUtensorMap mx, mz;
             glga_status st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, static_cast<uint64_t>(D),
                                             static_cast<uint64_t>(N), static_cast<uint64_t>(D) * 2, 64, kDwRows);
             if (st == GLGA_OK)
-                st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dnum, static_cast<uint64_t>(D + 16),
-                                    static_cast<uint64_t>(N), static_cast<uint64_t>(D + 16) * 4, 32, kDwRows);
-            if (st == GLGA_OK)   // the 16 dden columns: [64][16] float boxes, no swizzle
-                st = encode_tmap_2d(&md, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c->bw_dnum, static_cast<uint64_t>(D + 16),
-                                    static_cast<uint64_t>(N), static_cast<uint64_t>(D + 16) * 4, 16, kDwRows,
-                                    CU_TENSOR_MAP_SWIZZLE_NONE);
+                st = encode_tmap_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->bw_dnum, static_cast<uint64_t>(D + 16),
+                                    static_cast<uint64_t>(N), static_cast<uint64_t>(D + 16) * 2, 64, kDwRows);
             if (st != GLGA_OK) return st;
             DwParams p;
             p.N = N;
@@ -2993,7 +2980,7 @@ glga_status launch_dsz_bwd(Ctx *c, const T *Q, cudaStream_t s) {
             const size_t smem = static_cast<size_t>(kDszStages) * kDszStage + 1024;
             GLGA_CUDA(cudaFuncSetAttribute(bwd_dw_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem)));
-            bwd_dw_tc_kernel<true><<<static_cast<unsigned>(c->bw_dsz_parts), kDwThreads, smem, s>>>(mx, mz, md, p);
+            bwd_dw_tc_kernel<true><<<static_cast<unsigned>(c->bw_dsz_parts), kDwThreads, smem, s>>>(mx, mz, p);
             GLGA_CUDA(cudaGetLastError());
             return GLGA_OK;
         }
@@ -3046,8 +3033,8 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     }
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->t_col), std::max<int64_t>(E, 1) * sizeof(int32_t)));
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dL), nz * D * c->elem));
-    // [dnum | dden] rows of D + 16 columns (dden_h in column D + h) for the tensor-core dS | dz;
-    // dnum rows of D columns and dden [N, H] on the other paths
+    // bf16 [dnum | dden] rows of D + 16 columns (dden_h in column D + h) for the tensor-core
+    // dS | dz; float dnum rows of D columns and dden [N, H] on the other paths
     BTRY(dev_alloc(c, reinterpret_cast<void **>(&c->bw_dnum), nz * (D + 16) * f));
     if (st == GLGA_OK) {
         const cudaError_t e = cudaMemsetAsync(c->bw_dnum, 0, nz * (D + 16) * f, s);
