@@ -166,6 +166,34 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// x = the EPL bf16 values at p (p on an EPL-element boundary), by plain loads
+// (the kernel may write the same place afterwards).
+template <int EPL>
+__device__ __forceinline__ void ld_bf16_slice(const __nv_bfloat16 *p, float (&x)[EPL]) {
+    if constexpr (EPL == 1) {
+        x[0] = __bfloat162float(*p);
+        return;
+    }
+    uint32_t w[EPL > 1 ? EPL / 2 : 1];
+    if constexpr (EPL % 8 == 0) {
+#pragma unroll
+        for (int v = 0; v < EPL / 8; ++v) {
+            const uint4 u = reinterpret_cast<const uint4 *>(p)[v];
+            w[4 * v] = u.x; w[4 * v + 1] = u.y; w[4 * v + 2] = u.z; w[4 * v + 3] = u.w;
+        }
+    } else if constexpr (EPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        w[0] = u.x; w[1] = u.y;
+    } else {
+        w[0] = *reinterpret_cast<const uint32_t *>(p);
+    }
+#pragma unroll
+    for (int e = 0; e < EPL / 2; ++e) {
+        x[2 * e] = __uint_as_float(w[e] << 16);
+        x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+
 // x as a T row stores it.
 template <typename T>
 __device__ __forceinline__ float round_to(float x) {
@@ -651,17 +679,7 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
         b = row_ptr[i + 1];
     }
     const int D = H * R;
-    if (!CH && a == b) {                                  // no local term
-        if (dZb) {                                        // dq_i = its global part, in bf16
-            const LaneHead lh(lane, EPL, D, R);
-            if (lh.act) {
-                float cur[EPL];
-                ld_mrow<EPL, false>(dZ + i * dz_ld + lane * EPL, cur);
-                st_row<__nv_bfloat16, EPL>(dZb + i * 3 * D + lane * EPL, cur);
-            }
-        }
-        return;
-    }
+    if (!CH && a == b) return;                            // no local term (dq_i = its global part)
     const bool act2 = hl * EPL2 < D;
     const int lph2 = R / EPL2, h2 = act2 ? hl * EPL2 / R : 0;
     float q2[EPL2], dl2[EPL2], dq2[EPL2];
@@ -773,13 +791,15 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
         if (lh.act) st_mrow<EPL>(part + w * D + lane * EPL, dq);
         return;
     }
-    if (lh.act) {
+    if (lh.act) {                                         // the global part + the local one
         float *o = dZ + i * dz_ld + lane * EPL;
+        __nv_bfloat16 *ob = dZb + i * 3 * D + lane * EPL;
         float cur[EPL];
-        ld_mrow<EPL, false>(o, cur);
+        if (dZb) ld_bf16_slice<EPL>(ob, cur);
+        else ld_mrow<EPL, false>(o, cur);
 #pragma unroll
         for (int x = 0; x < EPL; ++x) cur[x] += dq[x];
-        if (dZb) st_row<__nv_bfloat16, EPL>(dZb + i * 3 * D + lane * EPL, cur);
+        if (dZb) st_row<__nv_bfloat16, EPL>(ob, cur);
         else st_mrow<EPL>(o, cur);
     }
 }
@@ -858,7 +878,8 @@ __global__ void __launch_bounds__(kMW * 32) bwd_q_heavy_kernel(
     if (warp != 0 || !lh.act) return;
     float acc[EPL], pv[EPL];
     float *o = dZ + i * dz_ld + lane * EPL;
-    ld_mrow<EPL, false>(o, acc);                           // the global part of dq_i
+    if (dZb) ld_bf16_slice<EPL>(dZb + i * 3 * D + lane * EPL, acc);   // the global part of dq_i
+    else ld_mrow<EPL, false>(o, acc);
 #pragma unroll
     for (int x = 0; x < EPL; ++x) dq[x] = 0.f;
     for (int w = 0; w < kMW; ++w) {
@@ -960,8 +981,13 @@ __device__ __forceinline__ void kv_finish(const LaneHead &lh, int lane, int64_t 
         if (lh.act) {
             float *pk = dZ + j * dz_ld + D + lane * EPL, *pv = pk + D;
             float gk[EPL], gv[EPL];
-            ld_mrow<EPL, false>(pk, gk);
-            ld_mrow<EPL, false>(pv, gv);
+            if (dZb) {
+                ld_bf16_slice<EPL>(dZb + j * 3 * D + D + lane * EPL, gk);
+                ld_bf16_slice<EPL>(dZb + j * 3 * D + 2 * D + lane * EPL, gv);
+            } else {
+                ld_mrow<EPL, false>(pk, gk);
+                ld_mrow<EPL, false>(pv, gv);
+            }
 #pragma unroll
             for (int x = 0; x < EPL; ++x) {
                 dk[x] += gk[x];
@@ -1204,8 +1230,13 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
         if (slot == 0 && act2) {
             float *pk = dZ + j * dz_ld + D + hl * EPL2, *pv = pk + D;
             float gk[EPL2], gv[EPL2];
-            ld_mrow<EPL2, false>(pk, gk);
-            ld_mrow<EPL2, false>(pv, gv);
+            if (dZb) {
+                ld_bf16_slice<EPL2>(dZb + j * 3 * D + D + hl * EPL2, gk);
+                ld_bf16_slice<EPL2>(dZb + j * 3 * D + 2 * D + hl * EPL2, gv);
+            } else {
+                ld_mrow<EPL2, false>(pk, gk);
+                ld_mrow<EPL2, false>(pv, gv);
+            }
 #pragma unroll
             for (int x = 0; x < EPL2; ++x) {
                 dk2[x] += gk[x];
@@ -1756,7 +1787,8 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmY,
     const __grid_constant__ CUtensorMap tmL, const float *__restrict__ t, const __nv_bfloat16 *__restrict__ Bg,
     int ro_kp, const float *__restrict__ Sz, int64_t N, int H, float b_g, float eps, __nv_bfloat16 *__restrict__ dL,
-    float *__restrict__ Dd, __nv_bfloat16 *__restrict__ dnum, float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
+    float *__restrict__ Dd, __nv_bfloat16 *__restrict__ dnum, float *__restrict__ dZ, int64_t dz_ld,
+    __nv_bfloat16 *__restrict__ dZb, unsigned *flag) {
     constexpr int D = kBroTcD;
     constexpr int kHQ = R >= 32 ? 1 : 32 / R;     // heads in a 32-column quarter
     constexpr uint32_t kTile = 2 * kBroTcAtom;    // a [128][128] bf16 tile
@@ -2013,18 +2045,27 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_readout_tc_kernel(
             uint32_t av[16];
             tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), av);
             tmem_ld_wait();
+            float o[16];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                float o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 16 * hb + 4 * p + e, hq = j / R < kHQ ? j / R : 0;
-                    o[e] = fmaf(zf[c0 + j], ddh[hq], __uint_as_float(av[4 * p + e])) * fminf(bf(pw, j), 1.f);
-                }
-                stage_row64_piece(stg, lane, p, make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]),
-                                                           __float_as_uint(o[2]), __float_as_uint(o[3])));
+            for (int e = 0; e < 16; ++e) {
+                const int j = 16 * hb + e, hq = j / R < kHQ ? j / R : 0;
+                o[e] = fmaf(zf[c0 + j], ddh[hq], __uint_as_float(av[e])) * fminf(bf(pw, j), 1.f);
             }
-            warp_rows64_flush(reinterpret_cast<uint8_t *>(dZ + c0 + 16 * hb), dz_ld * 4, r0, N, stg, lane);
+            if (dZb) {                         // bf16 rows of 3D columns: both halves, one store
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    stage_row64_piece(stg, lane, 2 * hb + i,
+                                      make_uint4(bf16x2_bits(o[8 * i], o[8 * i + 1]), bf16x2_bits(o[8 * i + 2], o[8 * i + 3]),
+                                                 bf16x2_bits(o[8 * i + 4], o[8 * i + 5]), bf16x2_bits(o[8 * i + 6], o[8 * i + 7])));
+                if (hb == 1)
+                    warp_rows64_flush(reinterpret_cast<uint8_t *>(dZb + c0), static_cast<int64_t>(3 * D) * 2, r0, N, stg, lane);
+            } else {
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    stage_row64_piece(stg, lane, p, make_uint4(__float_as_uint(o[4 * p]), __float_as_uint(o[4 * p + 1]),
+                                                               __float_as_uint(o[4 * p + 2]), __float_as_uint(o[4 * p + 3])));
+                warp_rows64_flush(reinterpret_cast<uint8_t *>(dZ + c0 + 16 * hb), dz_ld * 4, r0, N, stg, lane);
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -2065,7 +2106,7 @@ static_assert(kBroTcWarps * kBroTcStage <= kKvgStage, "a landed stage doubles as
 template <int R>
 __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
     const __grid_constant__ CUtensorMap tmKV, const float *__restrict__ dSc, const float *__restrict__ dST,
-    int64_t N, int H, float *__restrict__ dZ, int64_t dz_ld, unsigned *flag) {
+    int64_t N, int H, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb, unsigned *flag) {
     constexpr int D = kBroTcD;
     extern __shared__ uint8_t kvg_raw[];
     __shared__ __align__(8) uint64_t full_bar[kKvgStages];
@@ -2177,34 +2218,44 @@ __global__ void __launch_bounds__(kBroTcWarps * 32, 1) bwd_kv_global_tc_kernel(
         uint8_t *stg = sK + warp * kBroTcStage;
         // dk: (G_k + dz) phi'(k); dv: G_v
         const int64_t r0 = (blockIdx.x + static_cast<int64_t>(k) * gridDim.x) * 128 + quad * 32;
+        // the k or v half's 32 columns of this warp: float rows of dZ, or bf16 rows of dZb
+        auto put = [&](const float (&o)[16], int hb, int col0) {
+            if (dZb) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    stage_row64_piece(stg, lane, 2 * hb + i,
+                                      make_uint4(bf16x2_bits(o[8 * i], o[8 * i + 1]), bf16x2_bits(o[8 * i + 2], o[8 * i + 3]),
+                                                 bf16x2_bits(o[8 * i + 4], o[8 * i + 5]), bf16x2_bits(o[8 * i + 6], o[8 * i + 7])));
+                if (hb == 1)
+                    warp_rows64_flush(reinterpret_cast<uint8_t *>(dZb + col0 + c0), static_cast<int64_t>(3 * D) * 2, r0, N,
+                                      stg, lane);
+            } else {
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    stage_f32_piece(stg, lane, 4 * hb + p, o[4 * p], o[4 * p + 1], o[4 * p + 2], o[4 * p + 3]);
+                if (hb == 1) warp_rows_f32_flush(dZ + col0, dz_ld, r0, N, c0, stg, lane);
+            }
+        };
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
             uint32_t a[16];
             tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c0 + 16 * hb), a);
             tmem_ld_wait();
+            float o[16];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                float o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 16 * hb + 4 * p + e;
-                    o[e] = (__uint_as_float(a[4 * p + e]) + dzf[c0 + j]) * dphi(bf(kw, j));
-                }
-                stage_f32_piece(stg, lane, 4 * hb + p, o[0], o[1], o[2], o[3]);
-            }
+            for (int e = 0; e < 16; ++e) o[e] = (__uint_as_float(a[e]) + dzf[c0 + 16 * hb + e]) * dphi(bf(kw, 16 * hb + e));
+            put(o, hb, D);
         }
-        warp_rows_f32_flush(dZ + D, dz_ld, r0, N, c0, stg, lane);
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
             uint32_t a[16];
             tmem_ld16(tmem + lane_base + static_cast<uint32_t>(D + c0 + 16 * hb), a);
             tmem_ld_wait();
+            float o[16];
 #pragma unroll
-            for (int p = 0; p < 4; ++p)
-                stage_f32_piece(stg, lane, 4 * hb + p, __uint_as_float(a[4 * p]), __uint_as_float(a[4 * p + 1]),
-                                __uint_as_float(a[4 * p + 2]), __uint_as_float(a[4 * p + 3]));
+            for (int e = 0; e < 16; ++e) o[e] = __uint_as_float(a[e]);
+            put(o, hb, 2 * D);
         }
-        warp_rows_f32_flush(dZ + 2 * D, dz_ld, r0, N, c0, stg, lane);
         fence_proxy_async_smem();   // the staging writes come before the stage's next TMA load
         tc_fence_before();
         __syncthreads();            // TMEM, phi(K) and the stage are free
@@ -2237,7 +2288,7 @@ glga_status launch_kv_global_r(Ctx *c, int64_t Dz, cudaStream_t s) {
     const glga_status st = encode_tmap_2d(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->KV, 2 * kBroTcD,
                                           static_cast<uint64_t>(c->N), 4 * kBroTcD, 64, 128);
     if (st != GLGA_OK) return st;
-    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(m, c->bw_dSc, c->bw_dST, c->N, c->H, c->bw_dZ, Dz,
+    bwd_kv_global_tc_kernel<R><<<grid, kBroTcWarps * 32, kKvgSmem, s>>>(m, c->bw_dSc, c->bw_dST, c->N, c->H, c->bw_dZ, Dz, c->bw_dZb,
                                                                        c->dev_flag);
     return GLGA_OK;
 }
@@ -2284,7 +2335,7 @@ glga_status launch_readout_bwd_tc(Ctx *c, const __nv_bfloat16 *Q, const __nv_bfl
     bwd_readout_tc_kernel<R><<<grid, kBroTcWarps * 32, kBroTcSmem, s>>>(
         mq, my, ml, c->t, static_cast<const __nv_bfloat16 *>(c->Bro), c->ro_kp, c->Sz, c->N, c->H, b_g, eps,
         static_cast<__nv_bfloat16 *>(c->bw_dL), c->bw_Dd, reinterpret_cast<__nv_bfloat16 *>(c->bw_dnum), c->bw_dZ, Dz,
-        c->dev_flag);
+        c->bw_dZb, c->dev_flag);
     return GLGA_OK;
 }
 
@@ -2904,11 +2955,14 @@ __global__ void __launch_bounds__(kFxThreads, 1) bwd_dxdw_tc_kernel(
 }
 
 // Whether dX and the weight gradients of this context take the one-pass kernel: bf16
-// layers with d = 128 whose source side's global terms run on the tensor cores (H*r = 128,
-// r in {16, 32, 64}): dX and dW fit TMEM together, and the gather kernels that finish
-// dZ's columns (light rows two edges per step, heavy rows chunk sums) also write its
-// bf16 copy.
-bool bwd_fx(const Ctx *c) { return c->io == GLGA_BF16 && c->d == 128 && kv_global_tc(c) && c->N > 0; }
+// layers with d = 128 whose readout backward and source-side global terms run on the
+// tensor cores (H*r = 128, r in {16, 32, 64}, one head group): dX and dW fit TMEM
+// together, and dZ's columns 0 .. 3D - 1 live in bf16 (dZb) from the start: the two
+// tensor-core kernels write the global parts there and the gather kernels (light rows two
+// edges per step, heavy rows chunk sums) add the local parts in place.
+bool bwd_fx(const Ctx *c) {
+    return c->io == GLGA_BF16 && c->d == 128 && kv_global_tc(c) && readout_bwd_tc(c) && c->N > 0;
+}
 
 // dX, and the dW / dw_g / db_g partials that the reductions after it add
 // (over c->bw_fx_parts blocks), in one pass over dZ.

@@ -149,7 +149,7 @@ struct Ctx {
     int64_t bw_dwtc_rpp = 0;                          // ... rows per range (multiple of 64)
     int32_t bw_dwtc_parts = 0;                        // ... ranges
     float *bw_dW3 = nullptr;                          // [d][3D] their sum
-    __nv_bfloat16 *bw_dZb = nullptr;                  // [N][3D] final dQ | dK | dV for the one-pass dX / dW
+    __nv_bfloat16 *bw_dZb = nullptr;                  // [N][3D] dQ | dK | dV in bf16 (global parts, then the finals)
     cudaEvent_t bw_ev_fork = nullptr, bw_ev_join = nullptr;
     float *bw_dbg_part = nullptr;                     // [wparts] row-range sums of dt
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
