@@ -166,6 +166,23 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// acc[2w + e] += s x[w].half(e) for the bf16 s in the HIGH half of s2.
+template <int W>
+__device__ __forceinline__ void axpy_bf16w_hi(uint32_t s2, const uint32_t *x, float *acc) {
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+        acc[2 * w] = fma_bf16h<1, 0>(s2, x[w], acc[2 * w]);
+        acc[2 * w + 1] = fma_bf16h<1, 1>(s2, x[w], acc[2 * w + 1]);
+    }
+}
+
+// (p, ds) rounded to bf16 in one word: p in the low half, ds in the high half.
+__device__ __forceinline__ uint32_t pack_p_ds(float p, float ds) {
+    uint32_t w;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(ds), "f"(p));
+    return w;
+}
+
 // x = the EPL bf16 values at p (p on an EPL-element boundary), by plain loads
 // (the kernel may write the same place afterwards).
 template <int EPL>
@@ -656,12 +673,13 @@ constexpr size_t kQRingBytes = 8 * 2 * 2 * 2 * 32 * 16;   // 8 warps x 2 steps x
 // With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
 // kChunk entries at most) and write their shares of dq_i to part[w][0:D].
 template <typename T, int EPL, bool CH = false>
-__global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
+__global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
     const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb,
-    const int2 *__restrict__ chunks, float *__restrict__ part) {
+    const int2 *__restrict__ chunks, float *__restrict__ part, const int32_t *__restrict__ perm,
+    uint32_t *__restrict__ pds) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -718,7 +736,9 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
         extern __shared__ uint4 q_ring[];
         uint4 *ring = q_ring + (threadIdx.x >> 5) * (2 * kU * 2 * 32) + lane;
         auto cell = [&](int st, int u, int kv) { return ring + ((st * kU + u) * 2 + kv) * 32; };
-        auto issue = [&](int32_t e0, int st) {
+        // with pds, each edge's (p, ds) also goes to the source side, at the edge's position
+        // in the transposed CSR (perm, prefetched with the gathers)
+        auto issue = [&](int32_t e0, int st, int32_t (&pe)[kU]) {
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int32_t e = e0 + 2 * u + slot;
@@ -727,6 +747,7 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
                     cp_async16(cell(st, u, 0), row);
                     cp_async16(cell(st, u, 1), row + D);
                 }
+                pe[u] = (pds && e < b) ? __ldg(perm + e) : 0;
             }
             cp_async_commit();
         };
@@ -740,11 +761,13 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
             dw[0] = y.x; dw[1] = y.y; dw[2] = y.z; dw[3] = y.w;
         }
         const int n_steps = (b - a + 2 * kU - 1) / (2 * kU);
-        issue(a, 0);
+        int32_t pc[kU], pn[kU];
+        issue(a, 0, pc);
+        const bool head_lead = act2 && (hl & (lph2 - 1)) == 0;   // one lane per head writes (p, ds)
         for (int it = 0; it < n_steps; ++it) {
             const int32_t e0 = a + it * 2 * kU;
             if (it + 1 < n_steps) {
-                issue(e0 + 2 * kU, (it + 1) & 1);
+                issue(e0 + 2 * kU, (it + 1) & 1, pn);
                 cp_async_wait<1>();
             } else {
                 cp_async_wait<0>();
@@ -757,9 +780,13 @@ __global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
                 sc = head_reduce(sc, lph2);
                 dp = head_reduce(dp, lph2);
                 const bool live = e0 + 2 * u + slot < b;
-                const float ds = live ? __expf(sc * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
+                const float p = __expf(sc * inv_sqrt_r - ls);
+                const float ds = live ? p * (dp - dd) * inv_sqrt_r : 0.f;
                 axpy_bf16w<4>(bf16_splat(ds), kk, dq2);
+                if (pds && live && head_lead) pds[static_cast<int64_t>(pc[u]) * H + h2] = pack_p_ds(p, ds);
             }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) pc[u] = pn[u];
         }
     } else {
         for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {      // the same trip count in both halves
@@ -1118,7 +1145,7 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
     const float *__restrict__ dSc, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
     float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb, const int2 *__restrict__ chunks,
-    float *__restrict__ part) {
+    float *__restrict__ part, const uint32_t *__restrict__ pds) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -1167,6 +1194,34 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
             kw[0] = x.x; kw[1] = x.y; kw[2] = x.z; kw[3] = x.w;
             vw[0] = y.x; vw[1] = y.y; vw[2] = y.z; vw[3] = y.w;
         }
+        if (pds) {
+            // the target side stored each edge's (p, ds) in bf16 at its transposed position:
+            // dv += p dL_i, dk += ds q_i, nothing recomputed
+            for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {
+                uint4 q4[kU], d4[kU];
+                uint32_t pw[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int32_t e = e0 + 2 * u + slot;
+                    const bool live = e < b;
+                    const int64_t i = live ? t_col[e] : 0;
+                    q4[u] = d4[u] = make_uint4(0u, 0u, 0u, 0u);
+                    pw[u] = 0u;
+                    if (act2 && live) {
+                        q4[u] = __ldg(reinterpret_cast<const uint4 *>(Q + i * D + hl * EPL2));
+                        d4[u] = __ldg(reinterpret_cast<const uint4 *>(dL + i * D + hl * EPL2));
+                        pw[u] = __ldg(pds + static_cast<int64_t>(e) * H + h2);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const uint32_t qq[4] = {q4[u].x, q4[u].y, q4[u].z, q4[u].w};
+                    const uint32_t ll[4] = {d4[u].x, d4[u].y, d4[u].z, d4[u].w};
+                    axpy_bf16w<4>(pw[u], ll, dv2);
+                    axpy_bf16w_hi<4>(pw[u], qq, dk2);
+                }
+            }
+        } else
         for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {  // the same trip count in both halves
             uint4 q4[kU], d4[kU];
             float ls[kU], dd[kU];
@@ -1565,7 +1620,7 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
             bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb,
-                nullptr, nullptr);
+                nullptr, nullptr, c->bw_pds);
             return;
         }
     }
@@ -1573,7 +1628,7 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz, nullptr,
-                nullptr, nullptr);
+                nullptr, nullptr, nullptr);
             return;
         }
     }
@@ -1592,7 +1647,7 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
                                      static_cast<int>(kQRingBytes));
             bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz, c->bw_dZb,
-                nullptr, nullptr);
+                nullptr, nullptr, c->bw_perm, c->bw_pds);
             return;
         }
     }
@@ -1609,7 +1664,7 @@ void launch_kv_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t s
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E, false, true><<<warp_grid(nkc), 256, 0, sk>>>(nullptr, nkc, c->t_row_ptr,
                 c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r,
-                isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part);
+                isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part, c->bw_pds);
             return;
         }
     }
@@ -1626,7 +1681,7 @@ void launch_q_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t sq
                                      static_cast<int>(kQRingBytes));
             bwd_local_q2_kernel<T, E, true><<<warp_grid(nqc), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(nullptr, nqc,
                 c->row_ptr, c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd,
-                nullptr, 0, nullptr, c->bw_q_chunks, c->bw_q_part);
+                nullptr, 0, nullptr, c->bw_q_chunks, c->bw_q_part, c->bw_perm, c->bw_pds);
             return;
         }
     }
@@ -1665,16 +1720,24 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
     const int64_t nql = c->bw_nq_light, nqh = c->bw_nq_heavy, nkl = c->bw_nk_light, nkh = c->bw_nk_heavy;
     const int64_t nqc = c->bw_nq_chunks, nkc = c->bw_nk_chunks;
     const int32_t *qh = c->bw_q_rows + nql, *kh = c->bw_k_rows + nkl;
+    // with stored (p, ds) the source side reads what the target side wrote: it waits for
+    // the target side's light rows and chunks (ev_q), else the two sides run side by side
 #define GLGA_LB(E)                                                                                        \
     case E:                                                                                               \
+        if (c->bw_pds) {                                                                                  \
+            if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                        \
+            if (nqh) launch_q_chunks<T, E>(c, Q, KV, isr, sq);                                           \
+            cudaEventRecord(c->bw_ev_q, sq);                                                              \
+            cudaStreamWaitEvent(sk, c->bw_ev_q, 0);                                                       \
+        }                                                                                                 \
         if (nkl) launch_kv_light<T, E>(c, Q, KV, isr, Dz, sk);                                           \
         if (nkh) {                                                                                        \
             launch_kv_chunks<T, E>(c, Q, KV, isr, sk);                                                   \
             launch_kv_heavy<T, E>(c, Q, KV, isr, Dz, kh, nkh, sk);                                      \
         }                                                                                                 \
-        if (nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                                            \
+        if (!c->bw_pds && nql) launch_q_light<T, E>(c, Q, KV, isr, Dz, sq);                              \
         if (nqh) {                                                                                        \
-            launch_q_chunks<T, E>(c, Q, KV, isr, sq);                                                    \
+            if (!c->bw_pds) launch_q_chunks<T, E>(c, Q, KV, isr, sq);                                    \
             bwd_q_heavy_kernel<E><<<static_cast<unsigned>(nqh), kMW * 32, kMW * D * 4, sq>>>(qh, nqh,      \
                 c->bw_q_cptr, c->bw_q_part, H, R, c->bw_dZ, Dz, c->bw_dZb);                                          \
         }                                                                                                 \
@@ -3163,6 +3226,36 @@ glga_status backward_setup(Ctx *c, cudaStream_t s) {
     RowPlan qp, kp;
     plan_rows(rp, qp);
     plan_rows(trp, kp);
+    // the hand-over of each edge's (p, ds) from the target side to the source side (bf16
+    // layers on the two-edges-per-step kernels): perm maps a forward CSR entry to its
+    // position in the transposed CSR (a source row's entries in target order, ties in
+    // entry order), checked entry by entry against the transposed CSR; without a match
+    // the source side recomputes p and ds
+    if (kv_global_tc(c) && E > 0) {
+        std::vector<int32_t> ci(static_cast<size_t>(E)), tci(static_cast<size_t>(E)), perm(static_cast<size_t>(E));
+        GLGA_CUDA(cudaMemcpy(ci.data(), c->col_idx, ci.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
+        GLGA_CUDA(cudaMemcpy(tci.data(), c->t_col, tci.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
+        std::vector<int32_t> cur(trp.begin(), trp.end() - 1);
+        bool match = true;
+        for (int64_t i = 0; i < N && match; ++i) {
+            for (int32_t e = rp[i]; e < rp[i + 1]; ++e) {
+                const int32_t j = ci[e];
+                if (j < 0 || j >= N || cur[j] >= trp[j + 1] || tci[cur[j]] != i) {
+                    match = false;
+                    break;
+                }
+                perm[e] = cur[j]++;
+            }
+        }
+        if (match) {
+            st = dev_alloc(c, reinterpret_cast<void **>(&c->bw_perm), perm.size() * sizeof(int32_t));
+            if (st == GLGA_OK)
+                st = dev_alloc(c, reinterpret_cast<void **>(&c->bw_pds), static_cast<size_t>(E) * H * sizeof(uint32_t));
+            if (st != GLGA_OK) return st;
+            GLGA_CUDA(cudaMemcpy(c->bw_perm, perm.data(), perm.size() * sizeof(int32_t), cudaMemcpyHostToDevice));
+            GLGA_CUDA(cudaEventCreateWithFlags(&c->bw_ev_q, cudaEventDisableTiming));
+        }
+    }
     c->bw_nq_light = qp.n_light;
     c->bw_nq_heavy = qp.n_heavy;
     c->bw_nk_light = kp.n_light;

@@ -99,13 +99,15 @@ static void release_ctx(Ctx *c) {
                     c->bw_dg, c->bw_lse, c->bw_Dd, c->bw_dZ, c->bw_dsz_part, c->bw_dSz,
                     c->bw_dw_part, c->bw_q_rows, c->bw_k_rows, c->bw_ST, c->bw_dST, c->bw_Wall, c->bw_dbg_part,
                     c->bw_dSc, c->bw_q_chunks, c->bw_k_chunks, c->bw_q_cptr, c->bw_k_cptr,
-                    c->bw_q_part, c->bw_kv_part, c->bw_dwtc_part, c->bw_dW3, c->bw_dZb, c->part_seg, c->dev_flag};
+                    c->bw_q_part, c->bw_kv_part, c->bw_dwtc_part, c->bw_dW3, c->bw_dZb, c->bw_perm, c->bw_pds,
+                    c->part_seg, c->dev_flag};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     for (auto &e : c->ev)
         if (e) cudaEventDestroy(e);
     if (c->bw_ev_fork) cudaEventDestroy(c->bw_ev_fork);
     if (c->bw_ev_join) cudaEventDestroy(c->bw_ev_join);
+    if (c->bw_ev_q) cudaEventDestroy(c->bw_ev_q);
     if (c->bw_side) cudaStreamDestroy(c->bw_side);
 }
 

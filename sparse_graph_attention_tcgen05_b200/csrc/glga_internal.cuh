@@ -150,6 +150,9 @@ struct Ctx {
     int32_t bw_dwtc_parts = 0;                        // ... ranges
     float *bw_dW3 = nullptr;                          // [d][3D] their sum
     __nv_bfloat16 *bw_dZb = nullptr;                  // [N][3D] dQ | dK | dV in bf16 (global parts, then the finals)
+    int32_t *bw_perm = nullptr;                       // [E] forward CSR entry -> its transposed CSR position
+    uint32_t *bw_pds = nullptr;                       // [E][H] (p_ij, ds_ij) as bf16 pairs, transposed order
+    cudaEvent_t bw_ev_q = nullptr;                    // the target side has written bw_pds
     cudaEvent_t bw_ev_fork = nullptr, bw_ev_join = nullptr;
     float *bw_dbg_part = nullptr;                     // [wparts] row-range sums of dt
     float *bw_dw_part = nullptr;                      // [wparts][d][3D + 1]
