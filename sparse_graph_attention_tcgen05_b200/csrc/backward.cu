@@ -1138,7 +1138,10 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
 // layout for kv_finish.  Needs 2 EPL <= r.
 // With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
 // kChunk entries at most) and write their shares of dk_j | dv_j to part[w][0:2D].
-template <typename T, int EPL, bool GTC = false, bool CH = false>
+// With PDS the target side's stored (p, ds) of every edge replace the recomputation
+// (kPdsEdges edges per half-warp step).
+constexpr int kPdsEdges = 2;
+template <typename T, int EPL, bool GTC = false, bool CH = false, bool PDS = false>
 __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
@@ -1194,14 +1197,15 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
             kw[0] = x.x; kw[1] = x.y; kw[2] = x.z; kw[3] = x.w;
             vw[0] = y.x; vw[1] = y.y; vw[2] = y.z; vw[3] = y.w;
         }
-        if (pds) {
+        if constexpr (PDS) {
             // the target side stored each edge's (p, ds) in bf16 at its transposed position:
             // dv += p dL_i, dk += ds q_i, nothing recomputed
-            for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {
-                uint4 q4[kU], d4[kU];
-                uint32_t pw[kU];
+            constexpr int kP = kPdsEdges;
+            for (int32_t e0 = a; e0 < b; e0 += 2 * kP) {
+                uint4 q4[kP], d4[kP];
+                uint32_t pw[kP];
 #pragma unroll
-                for (int u = 0; u < kU; ++u) {
+                for (int u = 0; u < kP; ++u) {
                     const int32_t e = e0 + 2 * u + slot;
                     const bool live = e < b;
                     const int64_t i = live ? t_col[e] : 0;
@@ -1214,7 +1218,7 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < kU; ++u) {
+                for (int u = 0; u < kP; ++u) {
                     const uint32_t qq[4] = {q4[u].x, q4[u].y, q4[u].z, q4[u].w};
                     const uint32_t ll[4] = {d4[u].x, d4[u].y, d4[u].z, d4[u].w};
                     axpy_bf16w<4>(pw[u], ll, dv2);
@@ -1618,7 +1622,8 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     const int64_t nkl = c->bw_nk_light;
     if constexpr (E == 4 && sizeof(T) == 2) {
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
-            bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
+            auto kern = c->bw_pds ? bwd_local_kv2_kernel<T, E, true, false, true> : bwd_local_kv2_kernel<T, E, true>;
+            kern<<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb,
                 nullptr, nullptr, c->bw_pds);
             return;
@@ -1662,7 +1667,8 @@ void launch_kv_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t s
     const int64_t nkc = c->bw_nk_chunks;
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
-            bwd_local_kv2_kernel<T, E, false, true><<<warp_grid(nkc), 256, 0, sk>>>(nullptr, nkc, c->t_row_ptr,
+            auto kern = c->bw_pds ? bwd_local_kv2_kernel<T, E, false, true, true> : bwd_local_kv2_kernel<T, E, false, true>;
+            kern<<<warp_grid(nkc), 256, 0, sk>>>(nullptr, nkc, c->t_row_ptr,
                 c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r,
                 isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part, c->bw_pds);
             return;
