@@ -668,8 +668,8 @@ constexpr size_t kQRingBytes = 8 * 2 * 2 * 2 * 32 * 16;   // 8 warps x 2 steps x
 // warp's 16-lane halves take alternate edges of the row, lane hl of a half holding the
 // EPL2 = 2 EPL features hl*EPL2 .. hl*EPL2+EPL2-1 of q_i, dL_i and of the gathered k_j,
 // v_j, so a step's two edges share one shuffle butterfly and one exponential per lane.
-// The halves' dq are added (the same sum in both), moved to the 32-lane layout and added
-// into dZ [:, 0:D].  Needs 2 EPL <= r.
+// The halves' dq are added (the same sum in both) and the lower half's lanes add their
+// EPL2-feature slices into dZ [:, 0:D] (or dZb).  Needs 2 EPL <= r.
 // With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
 // kChunk entries at most) and write their shares of dq_i to part[w][0:D].
 template <typename T, int EPL, bool CH = false>
@@ -804,30 +804,22 @@ __global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
     }
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dq2[x] += __shfl_xor_sync(0xffffffffu, dq2[x], 16);
-    // to the 32-lane layout: lane l's features l*EPL .. are half-lane l/2's, part l % 2
-    const LaneHead lh(lane, EPL, D, R);
-    const int src = lane >> 1;
-    const bool hi = lane & 1;
-    float dq[EPL];
-#pragma unroll
-    for (int x = 0; x < EPL; ++x) {
-        const float q0 = __shfl_sync(0xffffffffu, dq2[x], src), q1 = __shfl_sync(0xffffffffu, dq2[EPL + x], src);
-        dq[x] = hi ? q1 : q0;
-    }
+    // the lower half's lanes hold the row's features hl*EPL2 .. hl*EPL2 + EPL2 - 1
+    if (slot != 0 || !act2) return;
     if constexpr (CH) {
-        if (lh.act) st_mrow<EPL>(part + w * D + lane * EPL, dq);
+        st_mrow<EPL2>(part + w * D + hl * EPL2, dq2);
         return;
     }
-    if (lh.act) {                                         // the global part + the local one
-        float *o = dZ + i * dz_ld + lane * EPL;
-        __nv_bfloat16 *ob = dZb + i * 3 * D + lane * EPL;
-        float cur[EPL];
-        if (dZb) ld_bf16_slice<EPL>(ob, cur);
-        else ld_mrow<EPL, false>(o, cur);
+    {                                                     // the global part + the local one
+        float *o = dZ + i * dz_ld + hl * EPL2;
+        __nv_bfloat16 *ob = dZb + i * 3 * D + hl * EPL2;
+        float cur[EPL2];
+        if (dZb) ld_bf16_slice<EPL2>(ob, cur);
+        else ld_mrow<EPL2, false>(o, cur);
 #pragma unroll
-        for (int x = 0; x < EPL; ++x) cur[x] += dq[x];
-        if (dZb) st_row<__nv_bfloat16, EPL>(ob, cur);
-        else st_mrow<EPL>(o, cur);
+        for (int x = 0; x < EPL2; ++x) cur[x] += dq2[x];
+        if (dZb) st_row<__nv_bfloat16, EPL2>(ob, cur);
+        else st_mrow<EPL2>(o, cur);
     }
 }
 
@@ -861,7 +853,7 @@ __global__ void __launch_bounds__(256) bwd_q_chunk_kernel(
 // Heavy rows are merged by one block of kMW warps each: warp w takes the row's chunks
 // c0 + w, c0 + w + kMW, ... (in order, kMU loads in flight), and warp 0 then combines the
 // warps' results in warp order through shared memory, so the order is fixed.
-constexpr int kMW = 8, kMU = 4;
+constexpr int kMW = 8, kMU = 8;
 
 // Heavy target rows over their chunks [chunk_ptr[s], chunk_ptr[s + 1]): dq_i = the
 // chunks' shares summed, added into dZ [:, 0:D].  Dynamic shared memory: kMW * D floats.
