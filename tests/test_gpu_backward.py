@@ -155,3 +155,18 @@ def test_one_pass_dx_dw(H, r, N):
     dst = np.concatenate([np.repeat(np.arange(N), 3), np.arange(N)]).astype(np.int32)
     w = make_custom(N, 128, H, r, src, dst, io="bf16", seed=N + 7, b_g=-0.1)
     _check(w, seed=r, chunked=N > 5000)
+
+
+def test_duplicate_edges_heavy_rows_and_isolated_rows_bf16():
+    # the tensor-core layer shape (H*r = 128, d = 128) on a graph with repeated entries
+    # (the (p, ds) hand-over maps each repeat to its own transposed position), a target and
+    # a source row of 300 entries each (64-edge chunks, the last one ragged), and rows
+    # with no entries at all on either side
+    rng = np.random.default_rng(31)
+    N = 700
+    dst = np.concatenate([np.full(300, 5), rng.integers(0, N, 300), np.repeat(np.arange(0, N, 3), 2)])
+    src = np.concatenate([rng.integers(0, N, 300), np.full(300, 9), np.repeat(np.arange(0, N, 3), 2)[::-1]])
+    keep = (dst % 7 != 3) & (src % 11 != 4)            # rows without in- or out-entries
+    w = make_custom(N, 128, 4, 32, src[keep].astype(np.int32), dst[keep].astype(np.int32), io="bf16",
+                    seed=32, b_g=0.05)
+    _check(w, seed=33)
