@@ -1131,8 +1131,9 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
 // With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
 // kChunk entries at most) and write their shares of dk_j | dv_j to part[w][0:2D].
 // With PDS the target side's stored (p, ds) of every edge replace the recomputation
-// (kPdsEdges edges per half-warp step).
+// (kPdsEdges edges per half-warp step, gathers through a two-step shared-memory ring).
 constexpr int kPdsEdges = 2;
+constexpr size_t kKvRingBytes = 8 * 2 * kPdsEdges * 2 * 32 * 16;   // 8 warps x 2 steps x edges x (q, dL) x 32 lanes
 template <typename T, int EPL, bool GTC = false, bool CH = false, bool PDS = false>
 __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
@@ -1191,31 +1192,50 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
         }
         if constexpr (PDS) {
             // the target side stored each edge's (p, ds) in bf16 at its transposed position:
-            // dv += p dL_i, dk += ds q_i, nothing recomputed
+            // dv += p dL_i, dk += ds q_i, nothing recomputed.  The q_i | dL_i gathers of step
+            // it + 1 wait in this warp's two-step shared-memory ring while step it is used.
             constexpr int kP = kPdsEdges;
-            for (int32_t e0 = a; e0 < b; e0 += 2 * kP) {
-                uint4 q4[kP], d4[kP];
-                uint32_t pw[kP];
+            extern __shared__ uint4 kv_ring[];
+            uint4 *ring = kv_ring + (threadIdx.x >> 5) * (2 * kP * 2 * 32) + lane;
+            auto cell = [&](int st, int u, int which) { return ring + ((st * kP + u) * 2 + which) * 32; };
+            // never-written cells are read with p = ds = 0: keep them finite
+#pragma unroll
+            for (int c = 0; c < 2 * kP * 2; ++c) ring[c * 32] = make_uint4(0u, 0u, 0u, 0u);
+            auto issue = [&](int32_t e0, int st, uint32_t (&pw)[kP]) {
 #pragma unroll
                 for (int u = 0; u < kP; ++u) {
                     const int32_t e = e0 + 2 * u + slot;
-                    const bool live = e < b;
-                    const int64_t i = live ? t_col[e] : 0;
-                    q4[u] = d4[u] = make_uint4(0u, 0u, 0u, 0u);
                     pw[u] = 0u;
-                    if (act2 && live) {
-                        q4[u] = __ldg(reinterpret_cast<const uint4 *>(Q + i * D + hl * EPL2));
-                        d4[u] = __ldg(reinterpret_cast<const uint4 *>(dL + i * D + hl * EPL2));
+                    if (e < b && act2) {
+                        const int64_t i = t_col[e];
+                        cp_async16(cell(st, u, 0), Q + i * D + hl * EPL2);
+                        cp_async16(cell(st, u, 1), dL + i * D + hl * EPL2);
                         pw[u] = __ldg(pds + static_cast<int64_t>(e) * H + h2);
                     }
                 }
+                cp_async_commit();
+            };
+            const int n_steps = (b - a + 2 * kP - 1) / (2 * kP);   // the same in both halves
+            uint32_t pc[kP], pn[kP];
+            if (n_steps > 0) issue(a, 0, pc);
+            for (int it = 0; it < n_steps; ++it) {
+                const int32_t e0 = a + it * 2 * kP;
+                if (it + 1 < n_steps) {
+                    issue(e0 + 2 * kP, (it + 1) & 1, pn);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
+                }
 #pragma unroll
                 for (int u = 0; u < kP; ++u) {
-                    const uint32_t qq[4] = {q4[u].x, q4[u].y, q4[u].z, q4[u].w};
-                    const uint32_t ll[4] = {d4[u].x, d4[u].y, d4[u].z, d4[u].w};
-                    axpy_bf16w<4>(pw[u], ll, dv2);
-                    axpy_bf16w_hi<4>(pw[u], qq, dk2);
+                    const uint4 q4 = *cell(it & 1, u, 0), d4 = *cell(it & 1, u, 1);
+                    const uint32_t qq[4] = {q4.x, q4.y, q4.z, q4.w};
+                    const uint32_t ll[4] = {d4.x, d4.y, d4.z, d4.w};
+                    axpy_bf16w<4>(pc[u], ll, dv2);
+                    axpy_bf16w_hi<4>(pc[u], qq, dk2);
                 }
+#pragma unroll
+                for (int u = 0; u < kP; ++u) pc[u] = pn[u];
             }
         } else
         for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {  // the same trip count in both halves
@@ -1615,7 +1635,7 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     if constexpr (E == 4 && sizeof(T) == 2) {
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
             auto kern = c->bw_pds ? bwd_local_kv2_kernel<T, E, true, false, true> : bwd_local_kv2_kernel<T, E, true>;
-            kern<<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
+            kern<<<warp_grid(nkl), 256, c->bw_pds ? kKvRingBytes : 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb,
                 nullptr, nullptr, c->bw_pds);
             return;
@@ -1660,7 +1680,7 @@ void launch_kv_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t s
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             auto kern = c->bw_pds ? bwd_local_kv2_kernel<T, E, false, true, true> : bwd_local_kv2_kernel<T, E, false, true>;
-            kern<<<warp_grid(nkc), 256, 0, sk>>>(nullptr, nkc, c->t_row_ptr,
+            kern<<<warp_grid(nkc), 256, c->bw_pds ? kKvRingBytes : 0, sk>>>(nullptr, nkc, c->t_row_ptr,
                 c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r,
                 isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part, c->bw_pds);
             return;
