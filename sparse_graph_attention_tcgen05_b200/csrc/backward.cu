@@ -823,6 +823,121 @@ __global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
     }
 }
 
+// Light target rows (or, with CH, chunks of heavy rows: chunk = {row, first entry},
+// kChunk entries at most) of bf16 layers with 8 features per half-lane (EPL = 4), one
+// row per 16-lane half: lane hl of a half holds features hl*8 .. hl*8+7 of its row's q_i
+// and dL_i and of the gathered k_j, v_j (through the same two-step cp.async ring per warp
+// as bwd_local_q2_kernel), kU edges of its own row per step; the warp steps as long as
+// its longer row (rows come sorted by degree, so the two are alike).  No combine across
+// the halves: each writes its row's dq_i (or, with CH, its chunk's share to part) and,
+// with pds, each edge's (p, ds) at its transposed position.
+template <bool CH>
+__global__ void __launch_bounds__(256, 4) bwd_q_pair_kernel(
+    const int32_t *__restrict__ rows, int64_t n_items, const int32_t *__restrict__ row_ptr,
+    const int32_t *__restrict__ col_idx, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ KV,
+    const __nv_bfloat16 *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
+    const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb,
+    const int2 *__restrict__ chunks, float *__restrict__ part, const int32_t *__restrict__ perm,
+    uint32_t *__restrict__ pds) {
+    constexpr int EPL2 = 8, kU = 2;
+    const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
+    const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (2 * w >= n_items) return;                         // warp-uniform
+    const int64_t item = 2 * w + slot;
+    const bool have = item < n_items;
+    int64_t i = 0;
+    int32_t a = 0, b = 0;
+    if (have) {
+        if constexpr (CH) {
+            const int2 ch = chunks[item];
+            i = ch.x;
+            a = ch.y;
+            b = min(row_ptr[i + 1], ch.y + kChunk);
+        } else {
+            i = rows[item];
+            a = row_ptr[i];
+            b = row_ptr[i + 1];
+        }
+    }
+    const int D = H * R;
+    const bool act2 = have && hl * EPL2 < D;
+    const int lph2 = R / EPL2, h2 = hl * EPL2 < D ? hl * EPL2 / R : 0;
+    uint32_t qw[4] = {0u, 0u, 0u, 0u}, dw[4] = {0u, 0u, 0u, 0u};
+    if (act2) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(Q + i * D + hl * EPL2));
+        const uint4 y = __ldg(reinterpret_cast<const uint4 *>(dL + i * D + hl * EPL2));
+        qw[0] = x.x; qw[1] = x.y; qw[2] = x.z; qw[3] = x.w;
+        dw[0] = y.x; dw[1] = y.y; dw[2] = y.z; dw[3] = y.w;
+    }
+    const float ls = have ? __ldg(lse + i * H + h2) : 0.f, dd = have ? __ldg(Dd + i * H + h2) : 0.f;
+    float dq2[EPL2];
+#pragma unroll
+    for (int x = 0; x < EPL2; ++x) dq2[x] = 0.f;
+    // never-written cells (edges past the row's end) are read with ds = 0: keep them finite
+    extern __shared__ uint4 q_ring[];
+    uint4 *ring = q_ring + (threadIdx.x >> 5) * (2 * kU * 2 * 32) + lane;
+    auto cell = [&](int st, int u, int kv) { return ring + ((st * kU + u) * 2 + kv) * 32; };
+#pragma unroll
+    for (int c = 0; c < 2 * kU * 2; ++c) ring[c * 32] = make_uint4(0u, 0u, 0u, 0u);
+    auto issue = [&](int32_t e0, int st, int32_t (&pe)[kU]) {
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int32_t e = e0 + u;
+            if (e < b && act2) {
+                const __nv_bfloat16 *row = KV + static_cast<int64_t>(col_idx[e]) * 2 * D + hl * EPL2;
+                cp_async16(cell(st, u, 0), row);
+                cp_async16(cell(st, u, 1), row + D);
+            }
+            pe[u] = (pds && e < b) ? __ldg(perm + e) : 0;
+        }
+        cp_async_commit();
+    };
+    const int mine = (b - a + kU - 1) / kU;
+    const int n_steps = max(mine, __shfl_xor_sync(0xffffffffu, mine, 16));
+    const bool head_lead = act2 && (hl & (lph2 - 1)) == 0;   // one lane per head writes (p, ds)
+    int32_t pc[kU], pn[kU];
+    issue(a, 0, pc);
+    for (int it = 0; it < n_steps; ++it) {
+        const int32_t e0 = a + it * kU;
+        if (it + 1 < n_steps) {
+            issue(e0 + kU, (it + 1) & 1, pn);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const uint4 kv4 = *cell(it & 1, u, 0), vv4 = *cell(it & 1, u, 1);
+            const uint32_t kk[4] = {kv4.x, kv4.y, kv4.z, kv4.w}, vv[4] = {vv4.x, vv4.y, vv4.z, vv4.w};
+            float sc = dot_bf16w<4>(qw, kk, 0.f), dp = dot_bf16w<4>(dw, vv, 0.f);
+            sc = head_reduce(sc, lph2);
+            dp = head_reduce(dp, lph2);
+            const bool live = e0 + u < b;
+            const float p = __expf(sc * inv_sqrt_r - ls);
+            const float ds = live ? p * (dp - dd) * inv_sqrt_r : 0.f;
+            axpy_bf16w<4>(bf16_splat(ds), kk, dq2);
+            if (pds && live && head_lead) pds[static_cast<int64_t>(pc[u]) * H + h2] = pack_p_ds(p, ds);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) pc[u] = pn[u];
+    }
+    if (!act2) return;
+    if constexpr (CH) {
+        st_mrow<EPL2>(part + item * D + hl * EPL2, dq2);
+    } else {
+        if (a == b) return;                               // no local term (dq_i = its global part)
+        float *o = dZ + i * dz_ld + hl * EPL2;
+        __nv_bfloat16 *ob = dZb + i * 3 * D + hl * EPL2;
+        float cur[EPL2];
+        if (dZb) ld_bf16_slice<EPL2>(ob, cur);
+        else ld_mrow<EPL2, false>(o, cur);
+#pragma unroll
+        for (int x = 0; x < EPL2; ++x) cur[x] += dq2[x];
+        if (dZb) st_row<__nv_bfloat16, EPL2>(ob, cur);
+        else st_mrow<EPL2>(o, cur);
+    }
+}
+
 // Chunks of heavy target rows, one warp each: chunk c covers the edges
 // [chunks[c].y, min(chunks[c].y + kChunk, row end)) of row chunks[c].x, and writes its
 // share of dq_i into part[c][0:D].
@@ -1657,6 +1772,14 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
 template <typename T, int E>
 void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cudaStream_t sq) {
     const int64_t nql = c->bw_nq_light;
+    if constexpr (kQRing<T, E>) {
+        if (2 * E <= c->r) {                      // one row per half-warp
+            bwd_q_pair_kernel<false><<<warp_grid(ceil_div(nql, 2)), 256, kQRingBytes, sq>>>(c->bw_q_rows, nql,
+                c->row_ptr, c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse,
+                c->bw_Dd, c->bw_dZ, Dz, c->bw_dZb, nullptr, nullptr, c->bw_perm, c->bw_pds);
+            return;
+        }
+    }
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             if (kQRing<T, E> && kQRingBytes > 48 * 1024)
@@ -1692,6 +1815,14 @@ void launch_kv_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t s
 template <typename T, int E>
 void launch_q_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t sq) {
     const int64_t nqc = c->bw_nq_chunks;
+    if constexpr (kQRing<T, E>) {
+        if (2 * E <= c->r) {                      // one chunk per half-warp
+            bwd_q_pair_kernel<true><<<warp_grid(ceil_div(nqc, 2)), 256, kQRingBytes, sq>>>(nullptr, nqc, c->row_ptr,
+                c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, nullptr, 0,
+                nullptr, c->bw_q_chunks, c->bw_q_part, c->bw_perm, c->bw_pds);
+            return;
+        }
+    }
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
             if (kQRing<T, E> && kQRingBytes > 48 * 1024)
