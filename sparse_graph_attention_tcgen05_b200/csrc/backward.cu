@@ -658,8 +658,8 @@ __global__ void __launch_bounds__(256) bwd_local_q_kernel(
     }
 }
 
-// bf16 rows with 4 features per lane (8 per half-lane: one 16-byte slice) go through a
-// shared-memory ring of cp.async gathers in bwd_local_q2_kernel.
+// bf16 rows with 4 features per lane (8 per half-lane: one 16-byte slice) take
+// bwd_q_pair_kernel, with a shared-memory ring of cp.async gathers.
 template <typename T, int EPL>
 constexpr bool kQRing = sizeof(T) == 2 && EPL == 4;
 constexpr size_t kQRingBytes = 8 * 2 * 2 * 2 * 32 * 16;   // 8 warps x 2 steps x kU x (k, v) x 32 lanes
@@ -673,13 +673,12 @@ constexpr size_t kQRingBytes = 8 * 2 * 2 * 2 * 32 * 16;   // 8 warps x 2 steps x
 // With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
 // kChunk entries at most) and write their shares of dq_i to part[w][0:D].
 template <typename T, int EPL, bool CH = false>
-__global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
+__global__ void __launch_bounds__(256, 3) bwd_local_q2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col_idx, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, int H, int R, float inv_sqrt_r, const float *__restrict__ lse,
     const float *__restrict__ Dd, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb,
-    const int2 *__restrict__ chunks, float *__restrict__ part, const int32_t *__restrict__ perm,
-    uint32_t *__restrict__ pds) {
+    const int2 *__restrict__ chunks, float *__restrict__ part) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -706,15 +705,7 @@ __global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
     const float ls = __ldg(lse + i * H + h2), dd = __ldg(Dd + i * H + h2);
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dq2[x] = 0.f;
-    if constexpr (kQRing<T, EPL>) {
-        // never-written cells (edges past the row's end) are read with ds = 0: keep them finite
-        extern __shared__ uint4 q_ring[];
-        uint4 *ring = q_ring + (threadIdx.x >> 5) * (2 * kU * 2 * 32) + lane;
-#pragma unroll
-        for (int c = 0; c < 2 * kU * 2; ++c) ring[c * 32] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    // the edges of step it (kU per half); the gathers of step it + 1 wait in this warp's
-    // two-step shared-memory ring (bf16 rows of 8 features per lane) while step it is used
+    // the edges of step it (kU per half)
     auto use_step = [&](int32_t e0, const float (&k)[kU][EPL2], const float (&v)[kU][EPL2]) {
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -732,75 +723,17 @@ __global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
             for (int x = 0; x < EPL2; ++x) dq2[x] = fmaf(ds, k[u][x], dq2[x]);
         }
     };
-    if constexpr (kQRing<T, EPL>) {
-        extern __shared__ uint4 q_ring[];
-        uint4 *ring = q_ring + (threadIdx.x >> 5) * (2 * kU * 2 * 32) + lane;
-        auto cell = [&](int st, int u, int kv) { return ring + ((st * kU + u) * 2 + kv) * 32; };
-        // with pds, each edge's (p, ds) also goes to the source side, at the edge's position
-        // in the transposed CSR (perm, prefetched with the gathers)
-        auto issue = [&](int32_t e0, int st, int32_t (&pe)[kU]) {
+    for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {          // the same trip count in both halves
+        float k[kU][EPL2], v[kU][EPL2];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int32_t e = e0 + 2 * u + slot;
-                if (e < b && act2) {
-                    const T *row = KV + static_cast<int64_t>(col_idx[e]) * 2 * D + hl * EPL2;
-                    cp_async16(cell(st, u, 0), row);
-                    cp_async16(cell(st, u, 1), row + D);
-                }
-                pe[u] = (pds && e < b) ? __ldg(perm + e) : 0;
-            }
-            cp_async_commit();
-        };
-        // q_i, dL_i and the gathered k_j, v_j stay packed: the dot products and dq run on
-        // fma.rn.f32.bf16 (ds rounded to bf16 for dq)
-        uint32_t qw[4] = {0u, 0u, 0u, 0u}, dw[4] = {0u, 0u, 0u, 0u};
-        if (act2) {
-            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(Q + i * D + hl * EPL2));
-            const uint4 y = __ldg(reinterpret_cast<const uint4 *>(dL + i * D + hl * EPL2));
-            qw[0] = x.x; qw[1] = x.y; qw[2] = x.z; qw[3] = x.w;
-            dw[0] = y.x; dw[1] = y.y; dw[2] = y.z; dw[3] = y.w;
+        for (int u = 0; u < kU; ++u) {
+            const int32_t e = e0 + 2 * u + slot;
+            const bool live = e < b;
+            const T *row = KV + (live ? static_cast<int64_t>(col_idx[e]) : 0) * 2 * D;
+            ld_row<T, EPL2>(row, hl, act2 && live, k[u]);
+            ld_row<T, EPL2>(row + D, hl, act2 && live, v[u]);
         }
-        const int n_steps = (b - a + 2 * kU - 1) / (2 * kU);
-        int32_t pc[kU], pn[kU];
-        issue(a, 0, pc);
-        const bool head_lead = act2 && (hl & (lph2 - 1)) == 0;   // one lane per head writes (p, ds)
-        for (int it = 0; it < n_steps; ++it) {
-            const int32_t e0 = a + it * 2 * kU;
-            if (it + 1 < n_steps) {
-                issue(e0 + 2 * kU, (it + 1) & 1, pn);
-                cp_async_wait<1>();
-            } else {
-                cp_async_wait<0>();
-            }
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const uint4 kv4 = *cell(it & 1, u, 0), vv4 = *cell(it & 1, u, 1);
-                const uint32_t kk[4] = {kv4.x, kv4.y, kv4.z, kv4.w}, vv[4] = {vv4.x, vv4.y, vv4.z, vv4.w};
-                float sc = dot_bf16w<4>(qw, kk, 0.f), dp = dot_bf16w<4>(dw, vv, 0.f);
-                sc = head_reduce(sc, lph2);
-                dp = head_reduce(dp, lph2);
-                const bool live = e0 + 2 * u + slot < b;
-                const float p = __expf(sc * inv_sqrt_r - ls);
-                const float ds = live ? p * (dp - dd) * inv_sqrt_r : 0.f;
-                axpy_bf16w<4>(bf16_splat(ds), kk, dq2);
-                if (pds && live && head_lead) pds[static_cast<int64_t>(pc[u]) * H + h2] = pack_p_ds(p, ds);
-            }
-#pragma unroll
-            for (int u = 0; u < kU; ++u) pc[u] = pn[u];
-        }
-    } else {
-        for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {      // the same trip count in both halves
-            float k[kU][EPL2], v[kU][EPL2];
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int32_t e = e0 + 2 * u + slot;
-                const bool live = e < b;
-                const T *row = KV + (live ? static_cast<int64_t>(col_idx[e]) : 0) * 2 * D;
-                ld_row<T, EPL2>(row, hl, act2 && live, k[u]);
-                ld_row<T, EPL2>(row + D, hl, act2 && live, v[u]);
-            }
-            use_step(e0, k, v);
-        }
+        use_step(e0, k, v);
     }
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dq2[x] += __shfl_xor_sync(0xffffffffu, dq2[x], 16);
@@ -826,8 +759,8 @@ __global__ void __launch_bounds__(256, 4) bwd_local_q2_kernel(
 // Light target rows (or, with CH, chunks of heavy rows: chunk = {row, first entry},
 // kChunk entries at most) of bf16 layers with 8 features per half-lane (EPL = 4), one
 // row per 16-lane half: lane hl of a half holds features hl*8 .. hl*8+7 of its row's q_i
-// and dL_i and of the gathered k_j, v_j (through the same two-step cp.async ring per warp
-// as bwd_local_q2_kernel), kU edges of its own row per step; the warp steps as long as
+// and dL_i and of the gathered k_j, v_j (through a two-step cp.async ring per warp), kU
+// edges of its own row per step; the warp steps as long as
 // its longer row (rows come sorted by degree, so the two are alike).  No combine across
 // the halves: each writes its row's dq_i (or, with CH, its chunk's share to part) and,
 // with pds, each edge's (p, ds) at its transposed position.
@@ -1245,18 +1178,18 @@ __global__ void __launch_bounds__(PARTS ? kMW * 32 : 256) bwd_local_kv_kernel(
 // layout for kv_finish.  Needs 2 EPL <= r.
 // With CH the warps take the chunks of heavy rows instead (chunk w = {row, first entry},
 // kChunk entries at most) and write their shares of dk_j | dv_j to part[w][0:2D].
-// With PDS the target side's stored (p, ds) of every edge replace the recomputation
+// With the target side's stored (p, ds), bwd_kv_pair_kernel takes these rows instead
 // (kPdsEdges edges per half-warp step, gathers through a two-step shared-memory ring).
 constexpr int kPdsEdges = 2;
 constexpr size_t kKvRingBytes = 8 * 2 * kPdsEdges * 2 * 32 * 16;   // 8 warps x 2 steps x edges x (q, dL) x 32 lanes
-template <typename T, int EPL, bool GTC = false, bool CH = false, bool PDS = false>
+template <typename T, int EPL, bool GTC = false, bool CH = false>
 __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     const int32_t *__restrict__ rows, int64_t n_rows, const int32_t *__restrict__ t_row_ptr,
     const int32_t *__restrict__ t_col, const T *__restrict__ Q, const T *__restrict__ KV,
     const T *__restrict__ dL, const float *__restrict__ lse, const float *__restrict__ Dd,
     const float *__restrict__ dSc, const float *__restrict__ dST, int H, int R, float inv_sqrt_r,
     float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb, const int2 *__restrict__ chunks,
-    float *__restrict__ part, const uint32_t *__restrict__ pds) {
+    float *__restrict__ part) {
     constexpr int EPL2 = 2 * EPL, kU = 2;             // kU edges per slot per step
     const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
     const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
@@ -1305,54 +1238,6 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
             kw[0] = x.x; kw[1] = x.y; kw[2] = x.z; kw[3] = x.w;
             vw[0] = y.x; vw[1] = y.y; vw[2] = y.z; vw[3] = y.w;
         }
-        if constexpr (PDS) {
-            // the target side stored each edge's (p, ds) in bf16 at its transposed position:
-            // dv += p dL_i, dk += ds q_i, nothing recomputed.  The q_i | dL_i gathers of step
-            // it + 1 wait in this warp's two-step shared-memory ring while step it is used.
-            constexpr int kP = kPdsEdges;
-            extern __shared__ uint4 kv_ring[];
-            uint4 *ring = kv_ring + (threadIdx.x >> 5) * (2 * kP * 2 * 32) + lane;
-            auto cell = [&](int st, int u, int which) { return ring + ((st * kP + u) * 2 + which) * 32; };
-            // never-written cells are read with p = ds = 0: keep them finite
-#pragma unroll
-            for (int c = 0; c < 2 * kP * 2; ++c) ring[c * 32] = make_uint4(0u, 0u, 0u, 0u);
-            auto issue = [&](int32_t e0, int st, uint32_t (&pw)[kP]) {
-#pragma unroll
-                for (int u = 0; u < kP; ++u) {
-                    const int32_t e = e0 + 2 * u + slot;
-                    pw[u] = 0u;
-                    if (e < b && act2) {
-                        const int64_t i = t_col[e];
-                        cp_async16(cell(st, u, 0), Q + i * D + hl * EPL2);
-                        cp_async16(cell(st, u, 1), dL + i * D + hl * EPL2);
-                        pw[u] = __ldg(pds + static_cast<int64_t>(e) * H + h2);
-                    }
-                }
-                cp_async_commit();
-            };
-            const int n_steps = (b - a + 2 * kP - 1) / (2 * kP);   // the same in both halves
-            uint32_t pc[kP], pn[kP];
-            if (n_steps > 0) issue(a, 0, pc);
-            for (int it = 0; it < n_steps; ++it) {
-                const int32_t e0 = a + it * 2 * kP;
-                if (it + 1 < n_steps) {
-                    issue(e0 + 2 * kP, (it + 1) & 1, pn);
-                    cp_async_wait<1>();
-                } else {
-                    cp_async_wait<0>();
-                }
-#pragma unroll
-                for (int u = 0; u < kP; ++u) {
-                    const uint4 q4 = *cell(it & 1, u, 0), d4 = *cell(it & 1, u, 1);
-                    const uint32_t qq[4] = {q4.x, q4.y, q4.z, q4.w};
-                    const uint32_t ll[4] = {d4.x, d4.y, d4.z, d4.w};
-                    axpy_bf16w<4>(pc[u], ll, dv2);
-                    axpy_bf16w_hi<4>(pc[u], qq, dk2);
-                }
-#pragma unroll
-                for (int u = 0; u < kP; ++u) pc[u] = pn[u];
-            }
-        } else
         for (int32_t e0 = a; e0 < b; e0 += 2 * kU) {  // the same trip count in both halves
             uint4 q4[kU], d4[kU];
             float ls[kU], dd[kU];
@@ -1453,6 +1338,120 @@ __global__ void __launch_bounds__(256, 4) bwd_local_kv2_kernel(
     ld_row<T, EPL>(krow, lane, lh.act, k);
     ld_row<T, EPL>(krow + D, lane, lh.act, v);
     kv_finish<EPL, GTC>(lh, lane, j, k, v, dk, dv, dSc, dST, H, R, dZ, dz_ld, dZb);
+}
+
+// The source side with stored (p, ds) (bf16 layers, 8 features per half-lane, global terms
+// already in dZ / dZb), one row (or, with CH, one chunk of a heavy row) per 16-lane half:
+// lane hl of a half gathers features hl*8 .. hl*8+7 of q_i and dL_i through a two-step
+// cp.async ring per warp, kPdsEdges edges of its own row per step, and accumulates
+// dv_j += p dL_i, dk_j += ds q_i; the warp steps as long as its longer row.  Each half then
+// adds its row's local terms to the global ones in place (or, with CH, writes its chunk's
+// share of dk_j | dv_j to part).
+template <bool CH>
+__global__ void __launch_bounds__(256, 4) bwd_kv_pair_kernel(
+    const int32_t *__restrict__ rows, int64_t n_items, const int32_t *__restrict__ t_row_ptr,
+    const int32_t *__restrict__ t_col, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ dL,
+    int H, int R, float *__restrict__ dZ, int64_t dz_ld, __nv_bfloat16 *__restrict__ dZb,
+    const int2 *__restrict__ chunks, float *__restrict__ part, const uint32_t *__restrict__ pds) {
+    constexpr int EPL2 = 8, kP = kPdsEdges;
+    const int lane = threadIdx.x & 31, slot = lane >> 4, hl = lane & 15;
+    const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+    if (2 * w >= n_items) return;                         // warp-uniform
+    const int64_t item = 2 * w + slot;
+    const bool have = item < n_items;
+    int64_t j = 0;
+    int32_t a = 0, b = 0;
+    if (have) {
+        if constexpr (CH) {
+            const int2 ch = chunks[item];
+            j = ch.x;
+            a = ch.y;
+            b = min(t_row_ptr[j + 1], ch.y + kChunk);
+        } else {
+            j = rows[item];
+            a = t_row_ptr[j];
+            b = t_row_ptr[j + 1];
+        }
+    }
+    const int D = H * R;
+    const bool act2 = have && hl * EPL2 < D;
+    const int h2 = hl * EPL2 < D ? hl * EPL2 / R : 0;
+    float dk2[EPL2], dv2[EPL2];
+#pragma unroll
+    for (int x = 0; x < EPL2; ++x) dk2[x] = dv2[x] = 0.f;
+    extern __shared__ uint4 kv_ring[];
+    uint4 *ring = kv_ring + (threadIdx.x >> 5) * (2 * kP * 2 * 32) + lane;
+    auto cell = [&](int st, int u, int which) { return ring + ((st * kP + u) * 2 + which) * 32; };
+    // never-written cells are read with p = ds = 0: keep them finite
+#pragma unroll
+    for (int c = 0; c < 2 * kP * 2; ++c) ring[c * 32] = make_uint4(0u, 0u, 0u, 0u);
+    auto issue = [&](int32_t e0, int st, uint32_t (&pw)[kP]) {
+#pragma unroll
+        for (int u = 0; u < kP; ++u) {
+            const int32_t e = e0 + u;
+            pw[u] = 0u;
+            if (e < b && act2) {
+                const int64_t i = t_col[e];
+                cp_async16(cell(st, u, 0), Q + i * D + hl * EPL2);
+                cp_async16(cell(st, u, 1), dL + i * D + hl * EPL2);
+                pw[u] = __ldg(pds + static_cast<int64_t>(e) * H + h2);
+            }
+        }
+        cp_async_commit();
+    };
+    const int mine = (b - a + kP - 1) / kP;
+    const int n_steps = max(mine, __shfl_xor_sync(0xffffffffu, mine, 16));
+    uint32_t pc[kP], pn[kP];
+    issue(a, 0, pc);
+    for (int it = 0; it < n_steps; ++it) {
+        const int32_t e0 = a + it * kP;
+        if (it + 1 < n_steps) {
+            issue(e0 + kP, (it + 1) & 1, pn);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+#pragma unroll
+        for (int u = 0; u < kP; ++u) {
+            const uint4 q4 = *cell(it & 1, u, 0), d4 = *cell(it & 1, u, 1);
+            const uint32_t qq[4] = {q4.x, q4.y, q4.z, q4.w};
+            const uint32_t ll[4] = {d4.x, d4.y, d4.z, d4.w};
+            axpy_bf16w<4>(pc[u], ll, dv2);
+            axpy_bf16w_hi<4>(pc[u], qq, dk2);
+        }
+#pragma unroll
+        for (int u = 0; u < kP; ++u) pc[u] = pn[u];
+    }
+    if (!act2) return;
+    if constexpr (CH) {
+        st_mrow<EPL2>(part + item * 2 * D + hl * EPL2, dk2);
+        st_mrow<EPL2>(part + item * 2 * D + D + hl * EPL2, dv2);
+    } else {
+        float gk[EPL2], gv[EPL2];
+        if (dZb) {
+            __nv_bfloat16 *pk = dZb + j * 3 * D + D + hl * EPL2, *pv = pk + D;
+            ld_bf16_slice<EPL2>(pk, gk);
+            ld_bf16_slice<EPL2>(pv, gv);
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) {
+                gk[x] += dk2[x];
+                gv[x] += dv2[x];
+            }
+            st_row<__nv_bfloat16, EPL2>(pk, gk);
+            st_row<__nv_bfloat16, EPL2>(pv, gv);
+        } else {
+            float *pk = dZ + j * dz_ld + D + hl * EPL2, *pv = pk + D;
+            ld_mrow<EPL2, false>(pk, gk);
+            ld_mrow<EPL2, false>(pv, gv);
+#pragma unroll
+            for (int x = 0; x < EPL2; ++x) {
+                gk[x] += dk2[x];
+                gv[x] += dv2[x];
+            }
+            st_mrow<EPL2>(pk, gk);
+            st_mrow<EPL2>(pv, gv);
+        }
+    }
 }
 
 // Chunks of heavy source rows, one warp each (layout as bwd_q_chunk_kernel's, over the
@@ -1749,10 +1748,15 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
     const int64_t nkl = c->bw_nk_light;
     if constexpr (E == 4 && sizeof(T) == 2) {
         if (kv_global_tc(c)) {                    // (2 E <= r holds: r >= 16)
-            auto kern = c->bw_pds ? bwd_local_kv2_kernel<T, E, true, false, true> : bwd_local_kv2_kernel<T, E, true>;
-            kern<<<warp_grid(nkl), 256, c->bw_pds ? kKvRingBytes : 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
+            if (c->bw_pds) {                      // stored (p, ds): one row per half-warp
+                bwd_kv_pair_kernel<false><<<warp_grid(ceil_div(nkl, 2)), 256, kKvRingBytes, sk>>>(c->bw_k_rows, nkl,
+                    c->t_row_ptr, c->t_col, Q, static_cast<const T *>(c->bw_dL), c->H, c->r, c->bw_dZ, Dz, c->bw_dZb,
+                    nullptr, nullptr, c->bw_pds);
+                return;
+            }
+            bwd_local_kv2_kernel<T, E, true><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r, isr, c->bw_dZ, Dz, c->bw_dZb,
-                nullptr, nullptr, c->bw_pds);
+                nullptr, nullptr);
             return;
         }
     }
@@ -1760,7 +1764,7 @@ void launch_kv_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cud
         if (2 * E <= c->r) {
             bwd_local_kv2_kernel<T, E><<<warp_grid(nkl), 256, 0, sk>>>(c->bw_k_rows, nkl, c->t_row_ptr, c->t_col,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, c->bw_dSc, c->bw_dST, c->H, c->r, isr, c->bw_dZ, Dz, nullptr,
-                nullptr, nullptr, nullptr);
+                nullptr, nullptr);
             return;
         }
     }
@@ -1780,14 +1784,11 @@ void launch_q_light(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cuda
             return;
         }
     }
-    if constexpr (E <= 4) {
+    if constexpr (E <= 4 && !kQRing<T, E>) {
         if (2 * E <= c->r) {
-            if (kQRing<T, E> && kQRingBytes > 48 * 1024)
-                cudaFuncSetAttribute(bwd_local_q2_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(kQRingBytes));
-            bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
+            bwd_local_q2_kernel<T, E><<<warp_grid(nql), 256, 0, sq>>>(c->bw_q_rows, nql, c->row_ptr, c->col_idx,
                 Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd, c->bw_dZ, Dz, c->bw_dZb,
-                nullptr, nullptr, c->bw_perm, c->bw_pds);
+                nullptr, nullptr);
             return;
         }
     }
@@ -1802,10 +1803,17 @@ void launch_kv_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t s
     const int64_t nkc = c->bw_nk_chunks;
     if constexpr (E <= 4) {
         if (2 * E <= c->r) {
-            auto kern = c->bw_pds ? bwd_local_kv2_kernel<T, E, false, true, true> : bwd_local_kv2_kernel<T, E, false, true>;
-            kern<<<warp_grid(nkc), 256, c->bw_pds ? kKvRingBytes : 0, sk>>>(nullptr, nkc, c->t_row_ptr,
+            if constexpr (sizeof(T) == 2 && E == 4) {
+                if (c->bw_pds) {                  // stored (p, ds): one chunk per half-warp
+                    bwd_kv_pair_kernel<true><<<warp_grid(ceil_div(nkc, 2)), 256, kKvRingBytes, sk>>>(nullptr, nkc,
+                        c->t_row_ptr, c->t_col, Q, static_cast<const T *>(c->bw_dL), c->H, c->r, nullptr, 0, nullptr,
+                        c->bw_k_chunks, c->bw_kv_part, c->bw_pds);
+                    return;
+                }
+            }
+            bwd_local_kv2_kernel<T, E, false, true><<<warp_grid(nkc), 256, 0, sk>>>(nullptr, nkc, c->t_row_ptr,
                 c->t_col, Q, KV, static_cast<const T *>(c->bw_dL), c->bw_lse, c->bw_Dd, nullptr, nullptr, c->H, c->r,
-                isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part, c->bw_pds);
+                isr, nullptr, 0, nullptr, c->bw_k_chunks, c->bw_kv_part);
             return;
         }
     }
@@ -1823,14 +1831,11 @@ void launch_q_chunks(Ctx *c, const T *Q, const T *KV, float isr, cudaStream_t sq
             return;
         }
     }
-    if constexpr (E <= 4) {
+    if constexpr (E <= 4 && !kQRing<T, E>) {
         if (2 * E <= c->r) {
-            if (kQRing<T, E> && kQRingBytes > 48 * 1024)
-                cudaFuncSetAttribute(bwd_local_q2_kernel<T, E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(kQRingBytes));
-            bwd_local_q2_kernel<T, E, true><<<warp_grid(nqc), 256, kQRing<T, E> ? kQRingBytes : 0, sq>>>(nullptr, nqc,
+            bwd_local_q2_kernel<T, E, true><<<warp_grid(nqc), 256, 0, sq>>>(nullptr, nqc,
                 c->row_ptr, c->col_idx, Q, KV, static_cast<const T *>(c->bw_dL), c->H, c->r, isr, c->bw_lse, c->bw_Dd,
-                nullptr, 0, nullptr, c->bw_q_chunks, c->bw_q_part, c->bw_perm, c->bw_pds);
+                nullptr, 0, nullptr, c->bw_q_chunks, c->bw_q_part);
             return;
         }
     }
