@@ -166,6 +166,14 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// 2^x by the PTX ex2.approx.ftz instruction (the arguments are scores minus the row's
+// log-sum-exp, at most a few units above zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // acc[2w + e] += s x[w].half(e) for the bf16 s in the HIGH half of s2.
 template <int W>
 __device__ __forceinline__ void axpy_bf16w_hi(uint32_t s2, const uint32_t *x, float *acc) {
@@ -803,6 +811,8 @@ __global__ void __launch_bounds__(256, 4) bwd_q_pair_kernel(
         dw[0] = y.x; dw[1] = y.y; dw[2] = y.z; dw[3] = y.w;
     }
     const float ls = have ? __ldg(lse + i * H + h2) : 0.f, dd = have ? __ldg(Dd + i * H + h2) : 0.f;
+    // p = 2^(sc log2(e) / sqrt(r) - lse log2(e)), ds = p (dp / sqrt(r) - D_i / sqrt(r))
+    const float sc2 = inv_sqrt_r * 1.4426950408889634f, ls2 = ls * 1.4426950408889634f, dd_s = dd * inv_sqrt_r;
     float dq2[EPL2];
 #pragma unroll
     for (int x = 0; x < EPL2; ++x) dq2[x] = 0.f;
@@ -846,8 +856,8 @@ __global__ void __launch_bounds__(256, 4) bwd_q_pair_kernel(
             sc = head_reduce(sc, lph2);
             dp = head_reduce(dp, lph2);
             const bool live = e0 + u < b;
-            const float p = __expf(sc * inv_sqrt_r - ls);
-            const float ds = live ? p * (dp - dd) * inv_sqrt_r : 0.f;
+            const float p = ex2_approx(fmaf(sc, sc2, -ls2));
+            const float ds = live ? p * fmaf(dp, inv_sqrt_r, -dd_s) : 0.f;
             axpy_bf16w<4>(bf16_splat(ds), kk, dq2);
             if (pds && live && head_lead) pds[static_cast<int64_t>(pc[u]) * H + h2] = pack_p_ds(p, ds);
         }
