@@ -16,12 +16,14 @@
 //       dZ = [dQ | dK | dV | dt].
 // The target-grouped terms (dq) walk the forward CSR; the source-grouped terms (dk, dv)
 // walk a transposed CSR built at create, so every sum has a fixed order and there are no
-// atomics (two runs give identical bits).  CUDA-core kernels with fp32 arithmetic (one
-// warp per row or per 32-edge chunk of a heavy row); the two dense GEMMs dW = X^T dZ and
-// dX = dZ W^T run on the tcgen05 tensor cores for bf16 layers (bwd_dw_tc_kernel with bf16
-// operands, the persistent projection GEMM on kind::tf32) and as register-tiled fp32
-// CUDA-core GEMMs for fp32 layers; gradients are fp32.  The log-sum-exp of each row's
-// scores comes from the forward.
+// atomics (two runs give identical bits).  The gathers run on the CUDA cores (one row, or
+// one 64-edge chunk of a heavy row, per warp or per 16-lane half), bf16 rows kept packed
+// for fma.rn.f32.bf16 with f32 accumulation; for bf16 layers each edge's (p, ds) is formed
+// once, by the target side, and handed to the source side at the edge's transposed
+// position.  Every dense product of bf16 layers with H*r = 128 runs on the tcgen05 tensor
+// cores (the readout backward, dS | dz, the source side's global terms, dX | dW in one
+// pass); fp32 layers and other widths use register-tiled CUDA-core kernels.  Gradients are
+// fp32.  The log-sum-exp of each row's scores comes from the forward.
 #include <algorithm>
 #include <cmath>
 #include <type_traits>
