@@ -605,30 +605,30 @@ __device__ __forceinline__ void q_grad_range(const int32_t *col_idx, const T *KV
                 axpy_bf16w<W>(bf16_splat(ds), k[u], dq);
             }
         }
-        return;
-    }
-    for (int32_t e = a; e < b; e += kEU) {
-        float k[kEU][EPL], v[kEU][EPL];
+    } else {
+        for (int32_t e = a; e < b; e += kEU) {
+            float k[kEU][EPL], v[kEU][EPL];
 #pragma unroll
-        for (int u = 0; u < kEU; ++u) {
-            const bool live = e + u < b;
-            const T *row = KV + (live ? static_cast<int64_t>(col_idx[e + u]) : 0) * 2 * D;
-            ld_row<T, EPL>(row, lane, act && live, k[u]);
-            ld_row<T, EPL>(row + D, lane, act && live, v[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kEU; ++u) {
-            float s = 0.f, dp = 0.f;
-#pragma unroll
-            for (int x = 0; x < EPL; ++x) {
-                s = fmaf(q[x], k[u][x], s);
-                dp = fmaf(dl[x], v[u][x], dp);
+            for (int u = 0; u < kEU; ++u) {
+                const bool live = e + u < b;
+                const T *row = KV + (live ? static_cast<int64_t>(col_idx[e + u]) : 0) * 2 * D;
+                ld_row<T, EPL>(row, lane, act && live, k[u]);
+                ld_row<T, EPL>(row + D, lane, act && live, v[u]);
             }
-            s = head_reduce(s, lph);
-            dp = head_reduce(dp, lph);
-            const float ds = e + u < b ? __expf(s * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
 #pragma unroll
-            for (int x = 0; x < EPL; ++x) dq[x] = fmaf(ds, k[u][x], dq[x]);
+            for (int u = 0; u < kEU; ++u) {
+                float s = 0.f, dp = 0.f;
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) {
+                    s = fmaf(q[x], k[u][x], s);
+                    dp = fmaf(dl[x], v[u][x], dp);
+                }
+                s = head_reduce(s, lph);
+                dp = head_reduce(dp, lph);
+                const float ds = e + u < b ? __expf(s * inv_sqrt_r - ls) * (dp - dd) * inv_sqrt_r : 0.f;
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) dq[x] = fmaf(ds, k[u][x], dq[x]);
+            }
         }
     }
 }
@@ -1009,36 +1009,36 @@ __device__ __forceinline__ void kv_grad_range(const int32_t *t_col, const T *Q, 
                 axpy_bf16w<W>(bf16_splat(ds), q[u], dk);
             }
         }
-        return;
-    }
-    for (int32_t e = a; e < b; e += kEU) {
-        float q[kEU][EPL], dl[kEU][EPL], ls[kEU], dd[kEU];
+    } else {
+        for (int32_t e = a; e < b; e += kEU) {
+            float q[kEU][EPL], dl[kEU][EPL], ls[kEU], dd[kEU];
 #pragma unroll
-        for (int u = 0; u < kEU; ++u) {
-            const bool live = e + u < b;
-            const int64_t i = live ? t_col[e + u] : 0;
-            ld_row<T, EPL>(Q + i * D, lane, act && live, q[u]);
-            ld_row<T, EPL>(dL + i * D, lane, act && live, dl[u]);
-            ls[u] = live ? __ldg(lse + i * H + h) : 0.f;
-            dd[u] = live ? __ldg(Dd + i * H + h) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kEU; ++u) {
-            float s = 0.f, dp = 0.f;
-#pragma unroll
-            for (int x = 0; x < EPL; ++x) {
-                s = fmaf(q[u][x], k[x], s);
-                dp = fmaf(dl[u][x], v[x], dp);
+            for (int u = 0; u < kEU; ++u) {
+                const bool live = e + u < b;
+                const int64_t i = live ? t_col[e + u] : 0;
+                ld_row<T, EPL>(Q + i * D, lane, act && live, q[u]);
+                ld_row<T, EPL>(dL + i * D, lane, act && live, dl[u]);
+                ls[u] = live ? __ldg(lse + i * H + h) : 0.f;
+                dd[u] = live ? __ldg(Dd + i * H + h) : 0.f;
             }
-            s = head_reduce(s, lph);
-            dp = head_reduce(dp, lph);
-            const bool live = e + u < b;
-            const float p = live ? __expf(s * inv_sqrt_r - ls[u]) : 0.f;
-            const float ds = p * (dp - dd[u]) * inv_sqrt_r;
 #pragma unroll
-            for (int x = 0; x < EPL; ++x) {
-                dv[x] = fmaf(p, dl[u][x], dv[x]);
-                dk[x] = fmaf(ds, q[u][x], dk[x]);
+            for (int u = 0; u < kEU; ++u) {
+                float s = 0.f, dp = 0.f;
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) {
+                    s = fmaf(q[u][x], k[x], s);
+                    dp = fmaf(dl[u][x], v[x], dp);
+                }
+                s = head_reduce(s, lph);
+                dp = head_reduce(dp, lph);
+                const bool live = e + u < b;
+                const float p = live ? __expf(s * inv_sqrt_r - ls[u]) : 0.f;
+                const float ds = p * (dp - dd[u]) * inv_sqrt_r;
+#pragma unroll
+                for (int x = 0; x < EPL; ++x) {
+                    dv[x] = fmaf(p, dl[u][x], dv[x]);
+                    dk[x] = fmaf(ds, q[u][x], dk[x]);
+                }
             }
         }
     }
@@ -1884,7 +1884,6 @@ void launch_local_bwd(Ctx *c, const T *Q, const T *KV, float isr, int64_t Dz, cu
     const int H = c->H, R = c->r;
     const size_t D = static_cast<size_t>(c->D);
     const int64_t nql = c->bw_nq_light, nqh = c->bw_nq_heavy, nkl = c->bw_nk_light, nkh = c->bw_nk_heavy;
-    const int64_t nqc = c->bw_nq_chunks, nkc = c->bw_nk_chunks;
     const int32_t *qh = c->bw_q_rows + nql, *kh = c->bw_k_rows + nkl;
     // with stored (p, ds) the source side reads what the target side wrote: it waits for
     // the target side's light rows and chunks (ev_q), else the two sides run side by side
@@ -1948,27 +1947,6 @@ __device__ __forceinline__ uint32_t swz_off(int row, int k, uint32_t atom_bytes)
     return static_cast<uint32_t>(k >> 6) * atom_bytes + static_cast<uint32_t>(row) * 128u +
            ((static_cast<uint32_t>((k & 63) >> 3) ^ static_cast<uint32_t>(row & 7)) << 4) +
            static_cast<uint32_t>(k & 7) * 2u;
-}
-
-// The warp's 32 rows x 32 bf16 columns (64 B per row) of a row-major [N][ld] bf16 matrix,
-// starting at global row r0 and column c0, into the lane's registers (lane = row): four
-// coalesced loads of 8 rows x 64 B through the staging area (row r at byte r * 64, its
-// 16-byte piece p at slot p ^ ((r >> 1) & 3)).  Rows at or past N read as zero.
-__device__ __forceinline__ void warp_rows_bf16(const __nv_bfloat16 *src, int64_t ld, int64_t r0, int64_t N, int c0,
-                                               uint8_t *stage, int lane, uint4 (&out)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = 8 * i + (lane >> 2), p = lane & 3;
-        const int64_t gr = r0 + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (gr < N) v = __ldg(reinterpret_cast<const uint4 *>(src + gr * ld + c0) + p);
-        *reinterpret_cast<uint4 *>(stage + r * 64 + ((p ^ ((r >> 1) & 3)) << 4)) = v;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-        out[p] = *reinterpret_cast<const uint4 *>(stage + lane * 64 + ((p ^ ((lane >> 1) & 3)) << 4));
-    __syncwarp();
 }
 
 // The lane's 32 floats (its row, columns c0 .. c0 + 31) to a row-major float32 matrix:

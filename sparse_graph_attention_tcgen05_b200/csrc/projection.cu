@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) proj_gemm_kernel(
             // (TMEM lanes = its 64 features) and write the rows of their heads' blocks
             const int g = wg;
             const int f = g * 64 + quad * 32 + lane;            // feature
-            const int h = f / p.R, a = f - h * p.R;
+            const int h = f / p.R;
             const int hc0 = h * p.R - g * 64;                   // the head's first V column
             uint32_t s0[32], s1[32], zv[32];
             // the last tile's commit follows every statistics MMA of the CTA
