@@ -494,19 +494,27 @@ def run_sweep():
                       "slope_loglog_N_ge_2^17": loglog_slope(upper)}), flush=True)
 
 
-def e2e_pipelined(layer, w, host, dt, dev, steps, warmup=3):
-    """End-to-end throughput through the public API (Layer.forward): every step copies its
-    inputs (X and the weights) from pinned host memory, runs the forward and copies Y back
-    to pinned host memory.  Copies run on their own streams with two buffer sets, so step
-    i's host->device copy and step i-1's device->host copy overlap step i's forward (PCIe
-    is full duplex); events order every buffer reuse.  Device time from the first copy's
+def e2e_pipelined(layer, w, host, dt, dev, steps, warmup=3, graphs=False):
+    """End-to-end throughput through the public API: every step copies its inputs (X and
+    the weights) from pinned host memory, runs the forward and copies Y back to pinned host
+    memory.  The inputs sit in one glga.HostInputs slab, so they cross PCIe as one copy per
+    step.  Copies run on their own streams with two slots, so step i's host->device copy
+    and step i-1's device->host copy overlap step i's forward (PCIe is full duplex); events
+    order every buffer reuse.  With `graphs` each slot's forward is a Layer.capture graph
+    replayed per step, as in the device-timed value.  Device time from the first copy's
     start to the last copy's end."""
     import torch
-    names = ("X", "W_Q", "W_K", "W_V", "w_g")
-    ins = [[torch.empty_like(host[k], device=dev) for k in names] for _ in range(2)]
+    from sparse_graph_attention_tcgen05_b200 import glga
+    stage = glga.HostInputs(w.N, w.d, w.D, dt, dev, slots=2)
+    for k in stage.NAMES:
+        stage.host[k].copy_(host[k])
     Yd = [torch.empty(w.N, w.D, dtype=dt, device=dev) for _ in range(2)]
     Yh = [torch.empty(w.N, w.D, dtype=dt).pin_memory() for _ in range(2)]
     comp = torch.cuda.current_stream()
+    replays = None
+    if graphs:
+        replays = [layer.capture(*stage.device_inputs[b], w.b_g, w.eps, Y=Yd[b])[0] for b in range(2)]
+        torch.cuda.synchronize()
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_fwd = [torch.cuda.Event() for _ in range(2)]
@@ -515,16 +523,17 @@ def e2e_pipelined(layer, w, host, dt, dev, steps, warmup=3):
 
     def step(i):
         b = i % 2
-        with torch.cuda.stream(s_in):
-            if used[b]:
-                s_in.wait_event(ev_fwd[b])          # the forward that read buffer b is done
-            for t, k in zip(ins[b], names):
-                t.copy_(host[k], non_blocking=True)
-            ev_in[b].record(s_in)
+        if used[b]:
+            s_in.wait_event(ev_fwd[b])              # the forward that read slot b is done
+        ins = stage.upload(b, s_in)
+        ev_in[b].record(s_in)
         comp.wait_event(ev_in[b])
         if used[b]:
             comp.wait_event(ev_out[b])              # Y buffer b has been copied out
-        layer.forward(*ins[b], b_g=w.b_g, eps=w.eps, Y=Yd[b], stream=comp)
+        if replays is not None:
+            replays[b].replay()
+        else:
+            layer.forward(*ins, b_g=w.b_g, eps=w.eps, Y=Yd[b], stream=comp)
         ev_fwd[b].record(comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_fwd[b])
@@ -543,9 +552,8 @@ def e2e_pipelined(layer, w, host, dt, dev, steps, warmup=3):
     t1.synchronize()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
-    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
-    d2h = Yh[0].numel() * Yh[0].element_size()
-    return ms, h2d, d2h
+    del replays
+    return ms, stage.nbytes, Yh[0].numel() * Yh[0].element_size()
 
 
 def run_sharded(args, rank, world, local_rank):
@@ -812,8 +820,9 @@ def run_single(args, rank, world, local_rank, mode):
     e2e_total = max_over_ranks(e2e_ms)
     e2e = {"value": replica_throughput(world, w.E * w.H, e2e_total, args.e2e_steps), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_total / args.e2e_steps,
-           "note": "Layer.forward per step with its inputs copied in and Y copied out (pinned host "
-                   "buffers); copies on their own streams, double-buffered, overlapping the forwards"}
+           "note": "Layer.forward per step with its inputs copied in (one glga.HostInputs slab: X and "
+                   "the weights, pinned) and Y copied out to pinned host memory; copies on their own "
+                   "streams, two slots, overlapping the forwards"}
 
     peaks, peak_kind = load_peaks()
     if local_ms:

@@ -348,3 +348,54 @@ class Layer:
             self.close()
         except Exception:
             pass
+
+
+class HostInputs:
+    """Page-locked host staging of one layer's inputs for host-to-device use.
+
+    X [N, d] and W_Q, W_K, W_V [d, D] and w_g [d] live in ONE pinned slab, each piece at a
+    256-byte aligned offset, so a step's inputs cross PCIe as a single host->device copy
+    instead of five (measured on B200 with arxiv-sized inputs: the four small weight copies
+    issued beside X's lengthened a pipelined copy-in/forward/copy-out step by 7-14 %).
+    `slots` device twins of the slab let copies of one step overlap the forward of another.
+
+    Fill the host views (`host["X"]`, ...) in place; `upload(slot, stream)` enqueues the
+    copy of the whole slab into device slot `slot` on `stream` and returns that slot's
+    device views in forward's argument order (X, W_Q, W_K, W_V, w_g).  Ordering the
+    copy against forwards that still read the slot is the caller's (stream events)."""
+
+    NAMES = ("X", "W_Q", "W_K", "W_V", "w_g")
+
+    def __init__(self, N: int, d: int, D: int, dtype: torch.dtype, device, slots: int = 2):
+        shapes = {"X": (N, d), "W_Q": (d, D), "W_K": (d, D), "W_V": (d, D), "w_g": (d,)}
+        esz = torch.empty((), dtype=dtype).element_size()
+        align = 256 // esz
+        self._offs, total = {}, 0
+        for k in self.NAMES:
+            self._offs[k] = total
+            n = int(np.prod(shapes[k]))
+            total += (n + align - 1) // align * align
+        self._shapes = shapes
+        self.slab = torch.zeros(total, dtype=dtype).pin_memory()
+        self.host = self._views(self.slab)
+        self._dev = [torch.empty(total, dtype=dtype, device=device) for _ in range(int(slots))]
+        self.device_inputs = [tuple(self._views(b)[k] for k in self.NAMES) for b in self._dev]
+
+    def _views(self, buf: torch.Tensor) -> dict:
+        out = {}
+        for k in self.NAMES:
+            n = int(np.prod(self._shapes[k]))
+            out[k] = buf[self._offs[k]:self._offs[k] + n].view(self._shapes[k])
+        return out
+
+    @property
+    def nbytes(self) -> int:
+        """Bytes one upload copies (the slab, alignment padding included)."""
+        return self.slab.numel() * self.slab.element_size()
+
+    def upload(self, slot: int, stream=None):
+        """Enqueue the host->device copy of the slab into `slot`; returns its device views."""
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self._dev[slot].copy_(self.slab, non_blocking=True)
+        return self.device_inputs[slot]

@@ -102,3 +102,25 @@ def test_every_declared_entry_point_has_a_binding_signature():
     L = glga.lib()
     for name in glga.declared_symbols():
         assert getattr(L, name).argtypes is not None, name
+
+
+def test_host_inputs_slab_layout(monkeypatch):
+    """glga.HostInputs lays X and the weights out in one slab, each piece 256-byte aligned,
+    non-overlapping, in forward's argument order (host side only: pinning is stubbed)."""
+    import torch
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    for N, d, D, dt in ((1000, 128, 64, torch.bfloat16), (7, 3, 5, torch.float32)):
+        st = glga.HostInputs(N, d, D, dt, "cpu", slots=2)
+        shapes = {"X": (N, d), "W_Q": (d, D), "W_K": (d, D), "W_V": (d, D), "w_g": (d,)}
+        base, end = st.slab.data_ptr(), -1
+        for k in st.NAMES:
+            v = st.host[k]
+            assert tuple(v.shape) == shapes[k] and v.is_contiguous()
+            off = v.data_ptr() - base
+            assert off % 256 == 0 and off > end
+            end = off + v.numel() * v.element_size() - 1
+        assert end < st.nbytes
+        for slot in range(2):
+            assert [tuple(t.shape) for t in st.device_inputs[slot]] == [shapes[k] for k in st.NAMES]
+        st.host["W_K"].fill_(3)
+        assert float(st.slab.sum()) == 3 * d * D

@@ -68,3 +68,33 @@ def test_backward_graph_replay_matches_eager(name, scale):
     assert layer.last_device_error() == 0
     del graph
     layer.close()
+
+
+@pytest.mark.parametrize("name,scale", [("tiny", 1.0), ("arxiv", 0.05)])
+def test_host_inputs_slab_upload_matches_separate_copies(name, scale):
+    """glga.HostInputs: one pinned slab uploaded per step gives the forward the same inputs
+    (bit for bit) as five separate copies, in every slot, and a refill of the host views
+    reaches the device with the next upload only."""
+    w = make_workload(name, scale=scale)
+    row_ptr, col_idx = glga.csr_from_coo(w.N, to_dev(w.src), to_dev(w.dst))
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+    dt = glga.torch_dtype(w.io)
+    arrays = (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)
+    stage = glga.HostInputs(w.N, w.d, w.D, dt, torch.device("cuda"), slots=2)
+    for k, a in zip(stage.NAMES, arrays):
+        stage.host[k].copy_(torch.from_numpy(np.ascontiguousarray(a)).to(dt))
+    plain = layer.forward(*(to_dev(a, dt) for a in arrays), b_g=w.b_g, eps=w.eps).clone()
+    for slot in (0, 1):
+        ins = stage.upload(slot)
+        for t in ins:
+            assert t.is_cuda and t.is_contiguous() and t.data_ptr() % 256 == 0
+        Y = layer.forward(*ins, b_g=w.b_g, eps=w.eps)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, plain)
+    stage.host["X"].mul_(-1)
+    stale = layer.forward(*stage.device_inputs[0], b_g=w.b_g, eps=w.eps).clone()
+    fresh = layer.forward(*stage.upload(0), b_g=w.b_g, eps=w.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(stale, plain) and not torch.equal(fresh, plain)
+    assert layer.last_device_error() == 0
+    layer.close()
