@@ -208,7 +208,8 @@ class Layer:
     def capture(self, X, W_Q, W_K, W_V, w_g, b_g: float, eps: float, Y=None):
         """Records one glga_forward on these buffers into a CUDA graph and returns
         (graph, Y): graph.replay() reruns the whole forward on the same X, weights and Y
-        (refill them in place between replays; b_g and eps are fixed at capture).  The
+        (refill them in place between replays; b_g and eps are fixed at capture; the graph
+        holds references to all six buffers, so they live as long as it does).  The
         forward enqueues kernels only (no allocation, no host synchronisation, tensor maps
         passed by value), so it records whole; one eager call first settles the lazy
         per-kernel attributes outside the capture.  With stage timing on, the stage events
@@ -224,6 +225,9 @@ class Layer:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             self.forward(X, W_Q, W_K, W_V, w_g, b_g, eps, Y=Y)
+        # the replays read and write these buffers: the graph keeps them alive, so that a
+        # caller dropping its own references cannot hand their memory to another tensor
+        graph.glga_buffers = (X, W_Q, W_K, W_V, w_g, Y)
         return graph, Y
 
     # -- introspection ---------------------------------------------------------------
@@ -294,6 +298,7 @@ class Layer:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             grads = self.backward(X, W_Q, W_K, W_V, w_g, b_g, eps, dY)
+        graph.glga_buffers = (X, W_Q, W_K, W_V, w_g, dY, grads)   # kept alive with the graph
         return graph, grads
 
     def block_output(self, Y, X, Wo, gamma, beta, ln_eps: float = 1e-5, Z=None, stream=None):

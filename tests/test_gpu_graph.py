@@ -98,3 +98,25 @@ def test_host_inputs_slab_upload_matches_separate_copies(name, scale):
     assert torch.equal(stale, plain) and not torch.equal(fresh, plain)
     assert layer.last_device_error() == 0
     layer.close()
+
+
+def test_captured_graph_keeps_its_buffers_alive():
+    """A forward graph holds X, the weights and Y: with every caller reference dropped,
+    their memory is not handed to new tensors that a replay would then overwrite."""
+    w = make_workload("arxiv", scale=0.02)
+    row_ptr, col_idx = glga.csr_from_coo(w.N, to_dev(w.src), to_dev(w.dst))
+    layer = glga.Layer(w.N, w.d, w.H, w.r, w.io, row_ptr, col_idx)
+    dt = glga.torch_dtype(w.io)
+    args = [to_dev(a, dt) for a in (w.X, w.W_Q, w.W_K, w.W_V, w.w_g)]
+    eager = layer.forward(*args, b_g=w.b_g, eps=w.eps).clone()
+    graph, Y = layer.capture(*args, w.b_g, w.eps)
+    del Y, args
+    probes = [torch.full_like(eager, 7.0) for _ in range(4)]
+    graph.replay()
+    torch.cuda.synchronize()
+    for p in probes:
+        assert bool((p == 7.0).all())
+    assert torch.equal(graph.glga_buffers[-1], eager)
+    assert layer.last_device_error() == 0
+    del graph
+    layer.close()
