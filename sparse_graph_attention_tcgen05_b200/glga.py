@@ -366,8 +366,10 @@ class HostInputs:
 
     Fill the host views (`host["X"]`, ...) in place; `upload(slot, stream)` enqueues the
     copy of the whole slab into device slot `slot` on `stream` and returns that slot's
-    device views in forward's argument order (X, W_Q, W_K, W_V, w_g).  Ordering the
-    copy against forwards that still read the slot is the caller's (stream events)."""
+    device views in forward's argument order (X, W_Q, W_K, W_V, w_g).  The copy reads the
+    slab when the stream reaches it: refill the host views only after it has completed
+    (an event recorded after upload).  Ordering the copy against forwards that still read
+    the slot is the caller's as well (stream events)."""
 
     NAMES = ("X", "W_Q", "W_K", "W_V", "w_g")
 
